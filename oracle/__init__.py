@@ -1,0 +1,215 @@
+"""fp64 CPU oracle for the sparse MoE layer forward (ctypes wrapper over moe_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the benchmark's CPU
+baseline leg may import this package; the product package never does.  It
+shares no code with the CUDA library.
+
+Functions (all inputs numpy arrays; x and weights may be float32, float64 or
+bf16 bit patterns stored as uint16, and are widened exactly to double):
+
+  router(x, W_g, K)                     -> idx [T,K] int32, gate [T,K] f64, logits [T,n] f64
+  expert(x_row, w1, w3, w2, e)          -> [d] f64, one SwiGLU expert on one token
+  forward_with_routing(x, idx, gate, w1, w3, w2) -> y [T,d] f64
+  moe_forward(x, W_g, w1, w3, w2, K)    -> y, idx, gate
+  dispatch(idx, n)                      -> counts, offsets, row_token, token_row
+  silu(z)                               -> z * sigmoid(z) in double
+
+Sources: the layer equation of "Mixtral of Experts" section 2.1 (flash-card
+page learn.ifs.name/d/jiang2024) and Part 3, Steps 1-4, of "Mixture of
+Experts: Why Mixtral Only Wakes Up Two Specialists" (neobadger.com).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "libmoe_oracle.so")
+
+_F32, _BF16, _F64 = 0, 1, 2
+
+
+def compile_source(src: str, out: str) -> str:
+    """gcc -O2 (no fast-math: IEEE double semantics), OpenMP over tokens."""
+    tmp = out + ".tmp%d" % os.getpid()
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                           "-Wall", "-Wextra", "-o", tmp, src, "-lm"])
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    """Compile moe_oracle.c in place (libmoe_oracle.so beside it)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        compile_source(_SRC, _LIB)
+    return _LIB
+
+
+def _bind(L):
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    L.oracle_router.argtypes = [i64, i32, i32, i32, vp, i32, vp, i32, vp, vp, vp]
+    L.oracle_expert.argtypes = [i32, i32, i32, i32, vp, i32, vp, vp, vp, i32, vp]
+    L.oracle_forward_with_routing.argtypes = [i64, i32, i32, i32, i32, vp, i32, vp, vp,
+                                              vp, vp, vp, i32, vp]
+    L.oracle_moe_forward.argtypes = [i64, i32, i32, i32, i32, vp, i32, vp, i32,
+                                     vp, vp, vp, i32, vp, vp, vp]
+    L.oracle_dispatch.argtypes = [i64, i32, i32, vp, vp, vp, vp, vp]
+    L.oracle_silu.argtypes = [ctypes.c_double]
+    L.oracle_silu.restype = ctypes.c_double
+    L.oracle_num_threads.restype = ctypes.c_int
+    L.oracle_set_num_threads.argtypes = [ctypes.c_int]
+    for f in ("oracle_router", "oracle_expert", "oracle_forward_with_routing",
+              "oracle_moe_forward", "oracle_dispatch"):
+        getattr(L, f).restype = ctypes.c_int
+    return L
+
+
+def _dt(a: np.ndarray) -> int:
+    if a.dtype == np.float32:
+        return _F32
+    if a.dtype == np.uint16:
+        return _BF16
+    if a.dtype == np.float64:
+        return _F64
+    raise TypeError("oracle inputs must be float32, float64 or bf16 bits (uint16), got %s" % a.dtype)
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a):
+    a = np.asarray(a)
+    if a.dtype not in (np.float32, np.float64, np.uint16):
+        a = a.astype(np.float64)
+    return np.ascontiguousarray(a)
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise ValueError("oracle %s rejected its arguments" % what)
+
+
+class Oracle:
+    """The oracle's entry points bound to one compiled copy of moe_oracle.c."""
+
+    def __init__(self, path: str):
+        self.path = path
+        self.L = _bind(ctypes.CDLL(path))
+
+    def num_threads(self) -> int:
+        return int(self.L.oracle_num_threads())
+
+    def set_num_threads(self, n: int) -> None:
+        self.L.oracle_set_num_threads(int(n))
+
+    def silu(self, z: float) -> float:
+        return float(self.L.oracle_silu(float(z)))
+
+    def router(self, x, W_g, K: int):
+        x, W_g = _c(x), _c(W_g)
+        T, d = x.shape
+        d2, n = W_g.shape
+        assert d == d2
+        idx = np.empty((T, K), np.int32)
+        gate = np.empty((T, K), np.float64)
+        logits = np.empty((T, n), np.float64)
+        _check(self.L.oracle_router(T, d, n, K, _p(x), _dt(x), _p(W_g), _dt(W_g),
+                                    _p(idx), _p(gate), _p(logits)), "router")
+        return idx, gate, logits
+
+    def expert(self, x_row, w1, w3, w2, e: int):
+        x_row, w1, w3, w2 = _c(x_row), _c(w1), _c(w3), _c(w2)
+        n, d, F = w1.shape
+        assert w3.shape == (n, d, F) and w2.shape == (n, F, d) and x_row.shape == (d,)
+        assert w1.dtype == w3.dtype == w2.dtype
+        out = np.empty(d, np.float64)
+        _check(self.L.oracle_expert(d, F, n, e, _p(x_row), _dt(x_row), _p(w1), _p(w3), _p(w2),
+                                    _dt(w1), _p(out)), "expert")
+        return out
+
+    def forward_with_routing(self, x, idx, gate, w1, w3, w2):
+        x, w1, w3, w2 = _c(x), _c(w1), _c(w3), _c(w2)
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+        gate = np.ascontiguousarray(gate, dtype=np.float64)
+        T, d = x.shape
+        n, d2, F = w1.shape
+        K = idx.shape[1]
+        assert d == d2 and idx.shape == (T, K) and gate.shape == (T, K)
+        assert w1.dtype == w3.dtype == w2.dtype
+        y = np.empty((T, d), np.float64)
+        _check(self.L.oracle_forward_with_routing(T, d, F, n, K, _p(x), _dt(x), _p(idx), _p(gate),
+                                                  _p(w1), _p(w3), _p(w2), _dt(w1), _p(y)),
+               "forward_with_routing")
+        return y
+
+    def moe_forward(self, x, W_g, w1, w3, w2, K: int):
+        x, W_g, w1, w3, w2 = _c(x), _c(W_g), _c(w1), _c(w3), _c(w2)
+        T, d = x.shape
+        n, d2, F = w1.shape
+        assert d == d2 and W_g.shape == (d, n)
+        assert w1.dtype == w3.dtype == w2.dtype
+        y = np.empty((T, d), np.float64)
+        idx = np.empty((T, K), np.int32)
+        gate = np.empty((T, K), np.float64)
+        _check(self.L.oracle_moe_forward(T, d, F, n, K, _p(x), _dt(x), _p(W_g), _dt(W_g),
+                                         _p(w1), _p(w3), _p(w2), _dt(w1), _p(y), _p(idx), _p(gate)),
+               "moe_forward")
+        return y, idx, gate
+
+    def dispatch(self, idx, n: int):
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+        T, K = idx.shape
+        counts = np.empty(n, np.int64)
+        offsets = np.empty(n + 1, np.int64)
+        row_token = np.empty(T * K, np.int64)
+        token_row = np.empty(T * K, np.int64)
+        _check(self.L.oracle_dispatch(T, n, K, _p(idx), _p(counts), _p(offsets), _p(row_token),
+                                      _p(token_row)), "dispatch")
+        return counts, offsets, row_token, token_row.reshape(T, K)
+
+
+_default = None
+
+
+def default() -> Oracle:
+    global _default
+    if _default is None:
+        _default = Oracle(build())
+    return _default
+
+
+def num_threads() -> int:
+    return default().num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    default().set_num_threads(n)
+
+
+def silu(z: float) -> float:
+    return default().silu(z)
+
+
+def router(x, W_g, K: int):
+    return default().router(x, W_g, K)
+
+
+def expert(x_row, w1, w3, w2, e: int):
+    return default().expert(x_row, w1, w3, w2, e)
+
+
+def forward_with_routing(x, idx, gate, w1, w3, w2):
+    return default().forward_with_routing(x, idx, gate, w1, w3, w2)
+
+
+def moe_forward(x, W_g, w1, w3, w2, K: int):
+    return default().moe_forward(x, W_g, w1, w3, w2, K)
+
+
+def dispatch(idx, n: int):
+    return default().dispatch(idx, n)

@@ -1,0 +1,292 @@
+/*
+ * moe_oracle.c -- plain, slow, fp64 CPU oracle for the sparse MoE layer forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file; only the tests, the smoke check and the benchmark's CPU
+ * baseline leg use it.  It shares no code, header or table with the CUDA
+ * library.
+ *
+ * What it computes (the layer equation of "Mixtral of Experts", section 2.1
+ * "Sparse Mixture of Experts", as restated on the learn.ifs.name flash-card
+ * page; the three routing lines and Steps 1-4 of Part 3 of "Mixture of
+ * Experts: Why Mixtral Only Wakes Up Two Specialists"):
+ *
+ *   y = sum_{i=0}^{n-1} Softmax(TopK(x . W_g))_i * SwiGLU_i(x)
+ *   SwiGLU_i(x) = (silu(x . w1_i) (*) (x . w3_i)) . w2_i,  silu(z) = z * sigmoid(z)
+ *
+ * Every value is read from its stored type (fp32, bf16 bits, or fp64) and
+ * widened exactly to double; all arithmetic is in double.  Loops follow the
+ * definitions directly: no blocking, no fusion, no reordering beyond the plain
+ * ascending-index sums.
+ *
+ * Readings of points the pages leave open:
+ *   - top-K order: descending logit; equal logits -> lower expert index first
+ *     (torch.topk, which the pages quote, fixes neither);
+ *   - the softmax runs over the K kept logits only (the others are -inf);
+ *   - the three expert matrices: w1, w3 [d][ffn] (gate and up), w2 [ffn][d]
+ *     (down), no biases;
+ *   - dispatch order: rows grouped by expert ascending, tokens ascending within
+ *     an expert (the pages say only that unchosen experts are skipped).
+ *
+ * Error behaviour: functions return 0 on success and -1 on a bad argument
+ * (null pointer, non-positive size, K > n); they never abort.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { OR_F32 = 0, OR_BF16 = 1, OR_F64 = 2 };
+
+/* Element i of a stored array, widened exactly to double. */
+static double elem(const void *base, int dt, size_t i)
+{
+    if (dt == OR_F64)
+        return ((const double *)base)[i];
+    if (dt == OR_F32)
+        return (double)((const float *)base)[i];
+    /* bf16: the 16 stored bits are the upper half of an IEEE binary32 value */
+    uint32_t u = (uint32_t)((const uint16_t *)base)[i] << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static int dt_ok(int dt) { return dt == OR_F32 || dt == OR_BF16 || dt == OR_F64; }
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/* silu(z) = z * sigmoid(z) = z / (1 + e^{-z}) */
+double oracle_silu(double z) { return z / (1.0 + exp(-z)); }
+
+/*
+ * Router for one token: logits L_e = sum_j x_j W_g[j][e] (the bias-free
+ * linear gate, Step 1), keep the K largest (Step 2), softmax over the kept K
+ * (Step 3).  idx gets the K expert indices in selection order; gate the K
+ * weights; logits (n values) is optional.
+ */
+static void route_one(int d, int n, int K, const void *x, int x_dt, size_t xoff,
+                      const void *Wg, int wg_dt, int32_t *idx, double *gate,
+                      double *L, unsigned char *taken)
+{
+    for (int e = 0; e < n; ++e) {
+        double s = 0.0;
+        for (int j = 0; j < d; ++j)
+            s += elem(x, x_dt, xoff + (size_t)j) * elem(Wg, wg_dt, (size_t)j * n + e);
+        L[e] = s;
+        taken[e] = 0;
+    }
+    /* Top-K: K rounds of "largest remaining logit"; scanning e upwards with a
+     * strict '>' keeps the lower index on equal logits. */
+    for (int k = 0; k < K; ++k) {
+        int best = -1;
+        for (int e = 0; e < n; ++e)
+            if (!taken[e] && (best < 0 || L[e] > L[best]))
+                best = e;
+        taken[best] = 1;
+        idx[k] = best;
+    }
+    /* Softmax over the kept logits (the others are -inf and contribute 0). */
+    double m = L[idx[0]];
+    double z = 0.0;
+    for (int k = 0; k < K; ++k)
+        z += exp(L[idx[k]] - m);
+    for (int k = 0; k < K; ++k)
+        gate[k] = exp(L[idx[k]] - m) / z;
+}
+
+int oracle_router(int64_t T, int d, int n, int K, const void *x, int x_dt,
+                  const void *Wg, int wg_dt, int32_t *idx, double *gate, double *logits)
+{
+    if (T < 0 || d <= 0 || n <= 0 || K <= 0 || K > n || !dt_ok(x_dt) || !dt_ok(wg_dt))
+        return -1;
+    if (T == 0)
+        return 0;
+    if (!x || !Wg || !idx || !gate)
+        return -1;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *L = (double *)malloc(sizeof(double) * (size_t)n);
+        unsigned char *taken = (unsigned char *)malloc((size_t)n);
+        if (!L || !taken) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t t = 0; t < T; ++t) {
+                route_one(d, n, K, x, x_dt, (size_t)t * d, Wg, wg_dt, idx + t * K, gate + t * K, L, taken);
+                if (logits)
+                    memcpy(logits + t * n, L, sizeof(double) * (size_t)n);
+            }
+        }
+        free(L);
+        free(taken);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * One expert e on one token: out[d] = (silu(x.w1_e) * (x.w3_e)) . w2_e.
+ * a, b, h are caller scratch of ffn doubles.
+ */
+static void expert_one(int d, int F, const void *x, int x_dt, size_t xoff,
+                       const void *w1, const void *w3, const void *w2, int w_dt, int e,
+                       double *a, double *b, double *out)
+{
+    size_t ebase1 = (size_t)e * (size_t)d * (size_t)F; /* w1[e], w3[e]: [d][F] */
+    size_t ebase2 = (size_t)e * (size_t)F * (size_t)d; /* w2[e]: [F][d] */
+    for (int f = 0; f < F; ++f) {
+        a[f] = 0.0;
+        b[f] = 0.0;
+    }
+    for (int j = 0; j < d; ++j) {
+        double xj = elem(x, x_dt, xoff + (size_t)j);
+        size_t row = ebase1 + (size_t)j * F;
+        for (int f = 0; f < F; ++f) {
+            a[f] += xj * elem(w1, w_dt, row + f);
+            b[f] += xj * elem(w3, w_dt, row + f);
+        }
+    }
+    for (int f = 0; f < F; ++f)
+        a[f] = oracle_silu(a[f]) * b[f]; /* a now holds h */
+    for (int i = 0; i < d; ++i)
+        out[i] = 0.0;
+    for (int f = 0; f < F; ++f) {
+        size_t row = ebase2 + (size_t)f * d;
+        for (int i = 0; i < d; ++i)
+            out[i] += a[f] * elem(w2, w_dt, row + i);
+    }
+}
+
+int oracle_expert(int d, int F, int n, int e, const void *x_row, int x_dt,
+                  const void *w1, const void *w3, const void *w2, int w_dt, double *out)
+{
+    if (d <= 0 || F <= 0 || n <= 0 || e < 0 || e >= n || !x_row || !w1 || !w3 || !w2 || !out ||
+        !dt_ok(x_dt) || !dt_ok(w_dt))
+        return -1;
+    double *a = (double *)malloc(sizeof(double) * (size_t)F);
+    double *b = (double *)malloc(sizeof(double) * (size_t)F);
+    if (!a || !b) {
+        free(a);
+        free(b);
+        return -1;
+    }
+    expert_one(d, F, x_row, x_dt, 0, w1, w3, w2, w_dt, e, a, b, out);
+    free(a);
+    free(b);
+    return 0;
+}
+
+/*
+ * y[t] = sum_k gate[t][k] * SwiGLU_{idx[t][k]}(x[t]) under a routing given
+ * from outside (the gate-weighted additive combine of Step 4).
+ */
+int oracle_forward_with_routing(int64_t T, int d, int F, int n, int K,
+                                const void *x, int x_dt, const int32_t *idx, const double *gate,
+                                const void *w1, const void *w3, const void *w2, int w_dt, double *y)
+{
+    if (T < 0 || d <= 0 || F <= 0 || n <= 0 || K <= 0 || K > n || !dt_ok(x_dt) || !dt_ok(w_dt))
+        return -1;
+    if (T == 0)
+        return 0;
+    if (!x || !idx || !gate || !w1 || !w3 || !w2 || !y)
+        return -1;
+    for (int64_t i = 0; i < T * K; ++i)
+        if (idx[i] < 0 || idx[i] >= n)
+            return -1;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *a = (double *)malloc(sizeof(double) * (size_t)F);
+        double *b = (double *)malloc(sizeof(double) * (size_t)F);
+        double *o = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!a || !b || !o) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t t = 0; t < T; ++t) {
+                double *yt = y + t * d;
+                for (int i = 0; i < d; ++i)
+                    yt[i] = 0.0;
+                for (int k = 0; k < K; ++k) {
+                    expert_one(d, F, x, x_dt, (size_t)t * d, w1, w3, w2, w_dt, idx[t * K + k], a, b, o);
+                    double g = gate[t * K + k];
+                    for (int i = 0; i < d; ++i)
+                        yt[i] += g * o[i];
+                }
+            }
+        }
+        free(a);
+        free(b);
+        free(o);
+    }
+    return bad ? -1 : 0;
+}
+
+/* The whole layer: route, then combine the chosen experts. */
+int oracle_moe_forward(int64_t T, int d, int F, int n, int K,
+                       const void *x, int x_dt, const void *Wg, int wg_dt,
+                       const void *w1, const void *w3, const void *w2, int w_dt,
+                       double *y, int32_t *idx, double *gate)
+{
+    int rc = oracle_router(T, d, n, K, x, x_dt, Wg, wg_dt, idx, gate, NULL);
+    if (rc)
+        return rc;
+    return oracle_forward_with_routing(T, d, F, n, K, x, x_dt, idx, gate, w1, w3, w2, w_dt, y);
+}
+
+/*
+ * Dispatch: the (token, slot) pairs grouped into per-expert segments.  The
+ * method only says that experts with a zero gate are skipped; this lays the
+ * chosen pairs out expert by expert (ascending), tokens ascending inside an
+ * expert.  counts[n], offsets[n+1], row_token[T*K] (token of each row),
+ * token_row[T*K] (row of each (token, slot) pair).
+ */
+int oracle_dispatch(int64_t T, int n, int K, const int32_t *idx, int64_t *counts,
+                    int64_t *offsets, int64_t *row_token, int64_t *token_row)
+{
+    if (T < 0 || n <= 0 || K <= 0 || K > n || !counts || !offsets)
+        return -1;
+    if (T > 0 && (!idx || !row_token || !token_row))
+        return -1;
+    for (int64_t i = 0; i < T * K; ++i)
+        if (idx[i] < 0 || idx[i] >= n)
+            return -1;
+    int64_t row = 0;
+    for (int e = 0; e < n; ++e) {
+        offsets[e] = row;
+        for (int64_t t = 0; t < T; ++t)
+            for (int k = 0; k < K; ++k)
+                if (idx[t * K + k] == e) {
+                    row_token[row] = t;
+                    token_row[t * K + k] = row;
+                    ++row;
+                }
+        counts[e] = row - offsets[e];
+    }
+    offsets[n] = row;
+    return 0;
+}

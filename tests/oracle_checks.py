@@ -1,0 +1,310 @@
+"""Pins for the fp64 oracle: each check compares it with something other than
+itself -- values printed on the pages, closed forms, special cases that reduce
+to a textbook or library routine (torch fp64), brute force on tiny inputs and
+invariants.  Every check takes an `oracle.Oracle` so the mutation tests can run
+the same checks against deliberately broken copies of the oracle.
+
+Pages cited:
+  [P2] "Mixtral of Experts" flash cards (learn.ifs.name/d/jiang2024), section
+       2.1 "Sparse Mixture of Experts": the layer equation, n and K.
+  [P5] "Mixture of Experts: Why Mixtral Only Wakes Up Two Specialists"
+       (neobadger.com), Part 3 Steps 1-4 and Part 4.
+"""
+from __future__ import annotations
+
+import itertools
+import math
+import os
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def read_golden(name: str) -> dict:
+    out = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *vals = line.split()
+            out[key] = [float(v) for v in vals]
+    return out
+
+
+def rand_layer(seed, T, d, F, n, scale_x=1.0):
+    g = np.random.default_rng(seed)
+    x = g.standard_normal((T, d)) * scale_x
+    Wg = g.standard_normal((d, n)) / math.sqrt(d)
+    w1 = g.standard_normal((n, d, F)) / math.sqrt(d)
+    w3 = g.standard_normal((n, d, F)) / math.sqrt(d)
+    w2 = g.standard_normal((n, F, d)) / math.sqrt(F)
+    return x, Wg, w1, w3, w2
+
+
+def torch_swiglu(x, w1e, w3e, w2e):
+    """Textbook SwiGLU FFN with torch's own silu and matmul, fp64."""
+    X = torch.from_numpy(np.asarray(x, np.float64))
+    a = X @ torch.from_numpy(np.asarray(w1e, np.float64))
+    b = X @ torch.from_numpy(np.asarray(w3e, np.float64))
+    h = torch.nn.functional.silu(a) * b
+    return (h @ torch.from_numpy(np.asarray(w2e, np.float64))).numpy()
+
+
+def rel_l2(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+# --------------------------------------------------------------------------
+# Router, top-K, softmax
+# --------------------------------------------------------------------------
+
+def check_worked_example(O):
+    """[P5] Part 3 Steps 1-3: logits (0.1, -0.4, 2.3, 0.0, -1.2, 0.6, 1.5, -0.3)
+    -> experts 3 and 7 (1-based), weights about 0.69 and 0.31."""
+    g = read_golden("worked_routing_example.txt")
+    L = np.array(g["logits"])
+    n = L.size
+    # W_g = I: the logits are x itself.
+    idx, gate, logits = O.router(L[None, :], np.eye(n), 2)
+    assert list(idx[0] + 1) == [int(v) for v in g["top2_one_based"]]
+    dec = int(g["gates_decimals"][0])
+    assert [round(float(v), dec) for v in gate[0]] == g["gates_printed"]
+    # The same logits produced by a non-square W_g (d=3 != n=8) whose first
+    # row holds them: fails if the gate's operand is transposed.
+    rng = np.random.default_rng(7)
+    Wg = np.vstack([L[None, :], rng.standard_normal((2, n))])
+    x = np.array([[1.0, 0.0, 0.0]])
+    idx2, gate2, logits2 = O.router(x, Wg, 2)
+    assert np.array_equal(idx2, idx) and np.allclose(gate2, gate, rtol=0, atol=1e-15)
+    assert np.allclose(logits2[0], L, rtol=0, atol=0)
+
+
+def check_two_way_softmax_closed_form(O):
+    """K=2: the softmax over the two kept logits is the logistic function of
+    their difference, g0 = 1/(1+e^-(L0-L1))."""
+    rng = np.random.default_rng(3)
+    for _ in range(20):
+        L = rng.standard_normal(6) * 3
+        idx, gate, _ = O.router(L[None, :], np.eye(6), 2)
+        a, b = sorted(L)[-1], sorted(L)[-2]
+        g0 = 1.0 / (1.0 + math.exp(-(a - b)))
+        assert abs(gate[0, 0] - g0) < 1e-15 and abs(gate[0, 1] - (1 - g0)) < 1e-15
+
+
+def check_logits_are_x_times_Wg(O):
+    """Step 1: the logits are the bias-free linear map x . W_g (numpy matmul)."""
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((17, 40))
+    Wg = rng.standard_normal((40, 12))
+    _, _, logits = O.router(x, Wg, 3)
+    assert np.allclose(logits, x @ Wg, rtol=1e-13, atol=1e-13)
+
+
+def check_topk_brute_force(O):
+    """For tiny n the kept set maximises the sum of K logits over all K-subsets
+    (brute force), ordered by descending logit."""
+    rng = np.random.default_rng(5)
+    for n, K in ((4, 2), (8, 2), (8, 3), (13, 2), (16, 4), (5, 5), (6, 1)):
+        x = rng.standard_normal((40, 24))
+        Wg = rng.standard_normal((24, n))
+        idx, gate, _ = O.router(x, Wg, K)
+        L = x @ Wg
+        for t in range(x.shape[0]):
+            best = max(itertools.combinations(range(n), K), key=lambda s: sum(L[t, list(s)]))
+            assert sorted(idx[t].tolist()) == sorted(best)
+            vals = L[t, idx[t]]
+            assert all(vals[i] >= vals[i + 1] for i in range(K - 1))
+
+
+def check_ties_go_to_lower_index(O):
+    """Equal logits: the lower expert index is kept first (the reading taken
+    where torch.topk leaves the order open)."""
+    cases = [([1.0, 3.0, 3.0, 0.0], 2, [1, 2]),
+             ([5.0, 5.0, 5.0, 5.0], 2, [0, 1]),
+             ([0.0, 2.0, 1.0, 2.0, 2.0], 3, [1, 3, 4]),
+             ([-1.0, -1.0, -2.0], 1, [0])]
+    for L, K, want in cases:
+        idx, gate, _ = O.router(np.array([L]), np.eye(len(L)), K)
+        assert idx[0].tolist() == want, (L, idx)
+        assert np.allclose(gate[0], np.full(K, 1.0 / K)) or len(set(np.array(L)[want])) > 1
+
+
+def check_gate_invariants(O):
+    """[P5] Step 3: positive weights that add up to 1, larger logit -> larger
+    weight; K=1 gives weight exactly 1."""
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((64, 32))
+    Wg = rng.standard_normal((32, 8)) * 2
+    for K in (1, 2, 3, 8):
+        _, gate, _ = O.router(x, Wg, K)
+        assert np.all(gate > 0)
+        assert np.allclose(gate.sum(1), 1.0, rtol=0, atol=1e-14)
+        assert np.all(np.diff(gate, axis=1) <= 0)
+        if K == 1:
+            assert np.all(gate == 1.0)
+
+
+# --------------------------------------------------------------------------
+# Experts and the combine
+# --------------------------------------------------------------------------
+
+def check_silu(O):
+    """silu(z) = z*sigmoid(z): special values and torch's silu."""
+    assert O.silu(0.0) == 0.0
+    assert abs(O.silu(40.0) - 40.0) < 1e-12
+    assert abs(O.silu(-40.0)) < 1e-15
+    assert abs(O.silu(1.0) - 1.0 / (1.0 + math.exp(-1.0))) < 1e-16
+    z = np.linspace(-12, 12, 97)
+    ref = torch.nn.functional.silu(torch.from_numpy(z)).numpy()
+    got = np.array([O.silu(v) for v in z])
+    assert np.allclose(got, ref, rtol=1e-14, atol=1e-16)
+
+
+def check_n1_is_plain_swiglu(O):
+    """n=1, K=1: the layer is a plain SwiGLU FFN (torch fp64)."""
+    x, Wg, w1, w3, w2 = rand_layer(21, 9, 48, 80, 1)
+    y, idx, gate = O.moe_forward(x, Wg, w1, w3, w2, 1)
+    assert np.all(idx == 0) and np.all(gate == 1.0)
+    ref = torch_swiglu(x, w1[0], w3[0], w2[0])
+    assert rel_l2(y, ref) < 1e-13
+
+
+def check_expert_indexing(O):
+    """One expert e of n on one token matches torch on w1[e], w3[e], w2[e]."""
+    x, Wg, w1, w3, w2 = rand_layer(22, 3, 32, 48, 5)
+    for e in range(5):
+        got = O.expert(x[1], w1, w3, w2, e)
+        ref = torch_swiglu(x[1:2], w1[e], w3[e], w2[e])[0]
+        assert rel_l2(got, ref) < 1e-13
+
+
+def check_K_equals_n_is_dense_mixture(O):
+    """K=n: Top-K keeps everything, so y is the dense softmax-weighted sum of
+    all experts (torch softmax and matmul, fp64)."""
+    T, d, F, n = 11, 40, 56, 6
+    x, Wg, w1, w3, w2 = rand_layer(23, T, d, F, n)
+    y, idx, gate = O.moe_forward(x, Wg, w1, w3, w2, n)
+    p = torch.softmax(torch.from_numpy(x @ Wg), dim=1).numpy()
+    ref = np.zeros((T, d))
+    for e in range(n):
+        ref += p[:, e:e + 1] * torch_swiglu(x, w1[e], w3[e], w2[e])
+    assert rel_l2(y, ref) < 1e-13
+
+
+def check_top2_layer_against_torch(O):
+    """The Top-2 layer on random data against a torch restatement that
+    builds the sparse gate vector (others -inf) and sums all experts."""
+    T, d, F, n = 13, 32, 40, 8
+    x, Wg, w1, w3, w2 = rand_layer(24, T, d, F, n)
+    y, idx, gate = O.moe_forward(x, Wg, w1, w3, w2, 2)
+    L = torch.from_numpy(x @ Wg)
+    top = torch.topk(L, 2, dim=1)
+    masked = torch.full_like(L, float("-inf")).scatter(1, top.indices, top.values)
+    p = torch.softmax(masked, dim=1).numpy()
+    ref = np.zeros((T, d))
+    for e in range(n):
+        ref += p[:, e:e + 1] * torch_swiglu(x, w1[e], w3[e], w2[e])
+    assert rel_l2(y, ref) < 1e-13
+
+
+def check_relabel_invariance(O):
+    """Relabelling experts together with their W_g columns leaves y unchanged
+    and relabels the chosen indices."""
+    T, d, F, n = 20, 24, 32, 7
+    x, Wg, w1, w3, w2 = rand_layer(25, T, d, F, n)
+    y, idx, gate = O.moe_forward(x, Wg, w1, w3, w2, 2)
+    perm = np.random.default_rng(1).permutation(n)  # new expert j is old perm[j]
+    y2, idx2, gate2 = O.moe_forward(x, Wg[:, perm], w1[perm], w3[perm], w2[perm], 2)
+    inv = np.argsort(perm)
+    assert np.array_equal(inv[idx], idx2)
+    assert np.allclose(gate, gate2, rtol=0, atol=1e-15)
+    assert rel_l2(y2, y) < 1e-14
+
+
+def check_unchosen_experts_do_not_matter(O):
+    """[P5] Step 2: the experts not kept are not run: changing them leaves y
+    bit-identical.  Also y is linear in w2 (scaling by 2 is exact)."""
+    T, d, F, n = 3, 16, 24, 8
+    x, Wg, w1, w3, w2 = rand_layer(26, T, d, F, n)
+    y, idx, gate = O.moe_forward(x, Wg, w1, w3, w2, 2)
+    unused = sorted(set(range(n)) - set(idx.ravel().tolist()))
+    assert unused, "seeded case should leave an expert unused"
+    w1b, w3b, w2b = w1.copy(), w3.copy(), w2.copy()
+    for e in unused:
+        w1b[e] = 1e3
+        w3b[e] = -7.0
+        w2b[e] = 5.0
+    yb, _, _ = O.moe_forward(x, Wg, w1b, w3b, w2b, 2)
+    assert np.array_equal(y, yb)
+    y2, _, _ = O.moe_forward(x, Wg, w1, w3, 2.0 * w2, 2)
+    assert np.array_equal(y2, 2.0 * y)
+
+
+def check_forward_with_routing_consistent(O):
+    """Routing supplied from outside reproduces the full forward exactly, and
+    a hand-made routing matches torch per token."""
+    T, d, F, n = 10, 24, 32, 5
+    x, Wg, w1, w3, w2 = rand_layer(27, T, d, F, n)
+    y, idx, gate = O.moe_forward(x, Wg, w1, w3, w2, 2)
+    y2 = O.forward_with_routing(x, idx, gate, w1, w3, w2)
+    assert np.array_equal(y, y2)
+    idx3 = np.array([[t % n, (t + 2) % n] for t in range(T)], np.int32)
+    gate3 = np.array([[0.25, 0.75]] * T)
+    y3 = O.forward_with_routing(x, idx3, gate3, w1, w3, w2)
+    for t in range(T):
+        ref = 0.25 * torch_swiglu(x[t:t + 1], w1[idx3[t, 0]], w3[idx3[t, 0]], w2[idx3[t, 0]]) + \
+            0.75 * torch_swiglu(x[t:t + 1], w1[idx3[t, 1]], w3[idx3[t, 1]], w2[idx3[t, 1]])
+        assert rel_l2(y3[t], ref[0]) < 1e-13
+
+
+def check_bf16_inputs_widen_exactly(O):
+    """bf16 bit patterns are read as the exact values they encode."""
+    from moe_inputs import f32_to_bf16_bits, bf16_bits_to_f32
+    x, Wg, w1, w3, w2 = rand_layer(28, 5, 32, 64, 4)
+    xb, w1b, w3b, w2b = (f32_to_bf16_bits(a.astype(np.float32)) for a in (x, w1, w3, w2))
+    y_b, idx_b, g_b = O.moe_forward(xb, Wg, w1b, w3b, w2b, 2)
+    wide = [bf16_bits_to_f32(a).astype(np.float64) for a in (xb, w1b, w3b, w2b)]
+    y_w, idx_w, g_w = O.moe_forward(wide[0], Wg, wide[1], wide[2], wide[3], 2)
+    assert np.array_equal(idx_b, idx_w) and np.array_equal(g_b, g_w) and np.array_equal(y_b, y_w)
+
+
+# --------------------------------------------------------------------------
+# Dispatch (the per-expert segments)
+# --------------------------------------------------------------------------
+
+def check_dispatch(O):
+    """Segments: counts add to T*K, each (token, slot) lands in exactly one
+    row of its expert's segment, and the order equals a stable library sort
+    of the flattened pairs by expert."""
+    rng = np.random.default_rng(31)
+    for T, n, K in ((1, 1, 1), (7, 4, 2), (50, 8, 2), (33, 16, 3), (64, 5, 5), (0, 3, 2)):
+        idx = np.array([rng.permutation(n)[:K] for _ in range(T)], np.int32).reshape(T, K)
+        counts, offsets, row_token, token_row = O.dispatch(idx, n)
+        assert counts.sum() == T * K and offsets[0] == 0 and offsets[-1] == T * K
+        assert np.array_equal(np.diff(offsets), counts)
+        assert np.array_equal(counts, np.bincount(idx.ravel(), minlength=n))
+        order = np.argsort(idx.ravel(), kind="stable")  # flattened pair ids, by expert
+        assert np.array_equal(row_token, order // K)
+        inv = np.empty(T * K, np.int64)
+        inv[order] = np.arange(T * K)
+        assert np.array_equal(token_row.ravel(), inv)
+        for r in range(T * K):
+            e = np.searchsorted(offsets, r, side="right") - 1
+            t = row_token[r]
+            k = list(idx[t]).index(e)
+            assert token_row[t, k] == r
+
+
+ALL_CHECKS = [
+    check_worked_example, check_two_way_softmax_closed_form, check_logits_are_x_times_Wg,
+    check_topk_brute_force, check_ties_go_to_lower_index, check_gate_invariants, check_silu,
+    check_n1_is_plain_swiglu, check_expert_indexing, check_K_equals_n_is_dense_mixture,
+    check_top2_layer_against_torch, check_relabel_invariance,
+    check_unchosen_experts_do_not_matter, check_forward_with_routing_consistent,
+    check_bf16_inputs_widen_exactly, check_dispatch,
+]

@@ -1,0 +1,48 @@
+"""Plant one mistake at a time in a private copy of the oracle (CPU only) and
+require that at least one pin catches it.  This is how we know the pins are
+sharp enough to trust the oracle."""
+import os
+
+import pytest
+
+import oracle
+from oracle_checks import ALL_CHECKS
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "moe_oracle.c")
+
+MUTANTS = {
+    "silu_sign": [("z / (1.0 + exp(-z))", "z / (1.0 + exp(z))")],
+    "swap_w1_w3": [("a[f] += xj * elem(w1,", "a[f] += xj * elem(@W3@,"),
+                   ("b[f] += xj * elem(w3,", "b[f] += xj * elem(w1,"),
+                   ("@W3@", "w3")],
+    "silu_on_up_proj": [("a[f] = oracle_silu(a[f]) * b[f];", "a[f] = a[f] * oracle_silu(b[f]);")],
+    "tie_break_high_index": [("L[e] > L[best]", "L[e] >= L[best]")],
+    "gate_dropped": [("yt[i] += g * o[i];", "yt[i] += o[i];")],
+    "gate_unnormalised": [("gate[k] = exp(L[idx[k]] - m) / z;", "gate[k] = exp(L[idx[k]] - m);")],
+    "router_transposed": [("(size_t)j * n + e", "(size_t)e * d + j")],
+    "w2_transposed": [("out[i] += a[f] * elem(w2, w_dt, row + i);",
+                       "out[i] += a[f] * elem(w2, w_dt, ebase2 + (size_t)i * F + f);")],
+    "bf16_shift": [("<< 16;", "<< 15;")],
+    "dispatch_slot_major": [("        for (int64_t t = 0; t < T; ++t)\n            for (int k = 0; k < K; ++k)\n                if (idx[t * K + k] == e) {",
+                             "        for (int k = 0; k < K; ++k)\n            for (int64_t t = 0; t < T; ++t)\n                if (idx[t * K + k] == e) {")],
+    "softmax_first_logit_only": [("z += exp(L[idx[k]] - m);", "z += (k == 0) ? 1.0 : 0.0;")],
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    src = open(SRC).read()
+    for old, new in MUTANTS[name]:
+        assert old in src, "mutation anchor not found: %r" % old
+        src = src.replace(old, new)
+    path = tmp_path / "mutant.c"
+    path.write_text(src)
+    so = oracle.compile_source(str(path), str(tmp_path / ("libmutant_%s.so" % name)))
+    O = oracle.Oracle(so)
+    caught = []
+    for check in ALL_CHECKS:
+        try:
+            check(O)
+        except (AssertionError, ValueError):
+            caught.append(check.__name__)
+    assert caught, "no pin caught mutant %s" % name
