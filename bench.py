@@ -1,0 +1,422 @@
+#!/usr/bin/env python
+"""Benchmark of the sparse MoE layer forward (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+A step is one moe_forward over one batch: router, top-K, softmax, dispatch,
+gather, GEMM1 (w1/w3 + SwiGLU), GEMM2 (w2), combine.  The default workload is
+the Mixtral-shape decode layer (T=32, d=4096, ffn=14336, n=8, K=2, bf16);
+--config picks another of the five (tiny_fp32, decode, prefill, skew_prefill,
+many_expert).  Inputs are seeded synthetic data resident in HBM before the
+timed region; the expert weights (>= 1.2 GB) are larger than the 126 MB L2,
+so no flush is needed between steps (tiny_fp32 flushes L2 with a 256 MB write).
+
+`value` is tokens/s over all ranks (replicas: each rank runs the same
+workload on its own GPU; no collective on the data path), timed with CUDA
+events on the launching stream, max over ranks.  `e2e` is the same metric
+through the C ABI with the step's activations copied from pinned host memory
+and y / topk_idx / topk_w copied back inside the timed region.  `roofline`
+reports the dominant kernel (per-stage CUDA events recorded by the library
+over the timed steps).  `cpu_baseline` times the fp64 oracle on a bounded
+sample of the same workload on this host's cores.
+
+--impl reference runs the oracle (the reference arm of this build) on the
+host, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import moe_inputs as mi  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def workload_desc(cfg):
+    return "%s: T=%d, d=%d, ffn=%d, n=%d, K=%d, %s%s" % (
+        cfg.name, cfg.T, cfg.d, cfg.ffn, cfg.n, cfg.K, cfg.dtype, ", skewed router" if cfg.skew else "")
+
+
+# --------------------------------------------------------------------------
+# algorithmic work per launch: what each stage must read, write and compute
+# --------------------------------------------------------------------------
+
+def touched_experts(idx: np.ndarray, n: int) -> np.ndarray:
+    return np.bincount(idx.ravel(), minlength=n)
+
+
+def algorithmic(cfg, counts):
+    """Bytes and FLOPs each stage must move / do, from the routing of the step."""
+    es = 2 if cfg.dtype == "bf16" else 4
+    T, d, F, n, K = cfg.T, cfg.d, cfg.ffn, cfg.n, cfg.K
+    R = T * K
+    used = int((counts > 0).sum())
+    w13 = used * 2 * d * F * es
+    w2 = used * F * d * es
+    gemm1_bytes = w13 + R * d * es + R * F * es           # weights + Xp read + H write
+    gemm2_bytes = w2 + R * F * es + R * d * es             # weights + H read + O write
+    gemm1_flops = 4.0 * R * d * F
+    gemm2_flops = 2.0 * R * F * d
+    return {
+        "gemm1": {"bytes": gemm1_bytes, "flops": gemm1_flops},
+        "gemm2": {"bytes": gemm2_bytes, "flops": gemm2_flops},
+        "layer_bytes": w13 + w2 + T * d * es * 2 + d * n * 4,
+        "active_flops": 6.0 * R * d * F + 2.0 * T * d * n,
+        "experts_touched": used,
+    }
+
+
+def source_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel, config):
+    """dram read+write bytes per launch from a committed ncu summary, if that
+    summary was taken on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    src = os.path.join(ROOT, "sparse_mixture_experts_24_b200", "csrc", "gemm_tc.cu")
+    sha = source_sha(src)
+    with open(p) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 5 and parts[0] == "traffic" and parts[1] == kernel and parts[2] == config:
+                if parts[4] == "src_sha=" + sha:
+                    return float(parts[3])
+    return None
+
+
+# --------------------------------------------------------------------------
+# clocks sampled during the timed region (NVML)
+# --------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = None
+            try:  # the CUDA device's own NVML handle (indices differ under CUDA_VISIBLE_DEVICES)
+                import torch
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self._reasons_fn(self.h)
+                for k, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------
+# CPU baseline: the oracle on a bounded sample of the workload
+# --------------------------------------------------------------------------
+
+def oracle_tokens_per_s(cfg, L, budget_s=15.0, max_tokens=None):
+    import oracle
+    threads = oracle.num_threads()
+    T = cfg.T if max_tokens is None else min(cfg.T, max_tokens)
+    # calibrate on one token, then size the sample to the budget
+    t0 = time.perf_counter()
+    oracle.moe_forward(L["x"][:1], L["W_g"], L["w1"], L["w3"], L["w2"], cfg.K)
+    one = time.perf_counter() - t0
+    par = max(1, threads)
+    s = int(max(1, min(T, budget_s * par / max(one, 1e-6))))
+    s = min(s, T)
+    t0 = time.perf_counter()
+    oracle.moe_forward(L["x"][:s], L["W_g"], L["w1"], L["w3"], L["w2"], cfg.K)
+    el = time.perf_counter() - t0
+    return s / el, s, min(threads, s), el
+
+
+# --------------------------------------------------------------------------
+# reference arm: the oracle on the host
+# --------------------------------------------------------------------------
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    L = mi.make_layer(cfg, seed=0)
+    threads = oracle.num_threads()
+    # per-step sample sized so that warmup + steps finish in about two minutes
+    t0 = time.perf_counter()
+    oracle.moe_forward(L["x"][:1], L["W_g"], L["w1"], L["w3"], L["w2"], cfg.K)
+    one = max(time.perf_counter() - t0, 1e-6)
+    per_step_budget = 120.0 / max(1, args.steps + args.warmup)
+    s = int(max(1, min(cfg.T, per_step_budget * max(1, threads) / one)))
+    for i in range(args.warmup):
+        oracle.moe_forward(L["x"][:s], L["W_g"], L["w1"], L["w3"], L["w2"], cfg.K)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        lo = (i * s) % max(1, cfg.T - s + 1)
+        oracle.moe_forward(L["x"][lo:lo + s], L["W_g"], L["w1"], L["w3"], L["w2"], cfg.K)
+    el = time.perf_counter() - t0
+    v = s * args.steps / el
+    line = {
+        "impl": "reference", "metric": "MoE-layer tokens/s", "value": v, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(cfg), "sample_tokens_per_step": s},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": min(threads, s), "kind": "oracle",
+                         "sample": "%d of %d tokens per step, full layer (router + %d experts each)"
+                                   % (s, cfg.T, cfg.K)},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="decode", choices=sorted(mi.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    cfg = mi.CONFIGS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+
+    import torch
+    import sparse_mixture_experts_24_b200 as m
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local_rank if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    L = mi.make_layer(cfg, seed=rank)     # each replica gets its own seeded batch
+    tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+
+    def to_dev(a):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        if a.dtype == np.uint16:
+            t = t.view(torch.int16).view(torch.bfloat16)
+        return t.to(dev)
+
+    x, Wg, w1, w3, w2 = (to_dev(L[k]) for k in ("x", "W_g", "w1", "w3", "w2"))
+    T = cfg.T
+    layer = m.MoELayer(cfg.n, cfg.K, cfg.d, cfg.ffn, cfg.dtype)
+    layer.reserve(T)
+    y = torch.empty_like(x)
+    idx = torch.empty((T, cfg.K), dtype=torch.int32, device=dev)
+    gw = torch.empty((T, cfg.K), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if cfg.name == "tiny_fp32" else None
+
+    def step():
+        if flush is not None:
+            flush.fill_(1)
+        m.moe_forward(layer.h, T, x, Wg, w1, w3, w2, y, idx, gw, stream)
+
+    for _ in range(args.warmup):
+        step()
+    layer.sync_status(stream)
+    counts = touched_experts(idx.cpu().numpy(), cfg.n)
+
+    # ---- device-timed region ----
+    sampler = ClockSampler(dev.index)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    m.moe_trace_begin(layer.h, args.steps)
+    sampler.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    stage_ms, traced = m.moe_trace_end(layer.h)
+    if dist:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    layer.sync_status(stream)
+    if dist:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    value = T * world / (ms * 1e-3)
+
+    # ---- end to end: pinned host activations in, y / routing out ----
+    xh = x.cpu().pin_memory()
+    yh = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    ih = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+    wh = torch.empty(gw.shape, dtype=gw.dtype).pin_memory()
+    xd = torch.empty_like(x)
+
+    def e2e_step():
+        if flush is not None:
+            flush.fill_(1)
+        xd.copy_(xh, non_blocking=True)
+        m.moe_forward(layer.h, T, xd, Wg, w1, w3, w2, y, idx, gw, stream)
+        yh.copy_(y, non_blocking=True)
+        ih.copy_(idx, non_blocking=True)
+        wh.copy_(gw, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ems = e0.elapsed_time(e1) / args.steps
+    if dist:
+        tt = torch.tensor([ems], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ems = float(tt.item())
+    e2e_value = T * world / (ems * 1e-3)
+    h2d = x.numel() * x.element_size()
+    d2h = y.numel() * y.element_size() + idx.numel() * 4 + gw.numel() * 4
+
+    # ---- roofline of the dominant kernel ----
+    peaks, peak_src = load_peaks()
+    work = algorithmic(cfg, counts)
+    per_launch = {k: v / max(1, traced) for k, v in stage_ms.items()}
+    dom = max(("gemm1", "gemm2"), key=lambda k: per_launch[k])
+    dom_ms = per_launch[dom]
+    if cfg.dtype == "f32":
+        roof = None
+    else:
+        intensity = work[dom]["flops"] / work[dom]["bytes"]
+        ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        if intensity < ridge:
+            ach = work[dom]["bytes"] / (dom_ms * 1e-3) / 1e9
+            roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": ach / peaks["hbm_gbs"]}
+        else:
+            timed_s = ms * args.steps * 1e-3
+            pk = peaks["bf16_tflops_sustained"] if timed_s > 1.0 else peaks["bf16_tflops"]
+            ach = work[dom]["flops"] / (dom_ms * 1e-3) / 1e12
+            roof = {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
+                    "peak_kind": "sustained" if timed_s > 1.0 else "burst"}
+        roof["kernel"] = dom
+        roof["peak_source"] = peak_src
+        roof["algorithmic_per_launch"] = work[dom]["bytes"] if roof["bound"] == "hbm" else work[dom]["flops"]
+        roof["launch_ms"] = dom_ms
+        roof["traffic"] = recorded_traffic(dom, cfg.name)
+
+    # ---- CPU baseline (rank 0, N = 1 only) ----
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, s, cores, el = oracle_tokens_per_s(cfg, L)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": "first %d of %d tokens, full layer in fp64 (%.1f s)" % (s, cfg.T, el)}
+
+    if rank == 0:
+        layer_ms = ms
+        line = {
+            "metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+            "config": {"workload": workload_desc(cfg), "global_batch_tokens": T * world,
+                       "parallelism": "replicas%d" % world if world > 1 else "single",
+                       "l2": "256 MB flush per step" if flush is not None else
+                             "no flush: %.2f GB of expert weights per step > 126 MB L2"
+                             % (work["layer_bytes"] / 1e9)},
+            "active_tflops": work["active_flops"] / (layer_ms * 1e-3) / 1e12,
+            "hbm_gbs_over_bytes_touched": work["layer_bytes"] / (layer_ms * 1e-3) / 1e9,
+            "stage_ms_per_step": {k: round(v, 5) for k, v in per_launch.items()},
+            "experts_touched": work["experts_touched"],
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps * (9 if cfg.n > 32 else 8),
+            "clocks": clocks,
+        }
+        print(json.dumps(line))
+    layer.close()
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

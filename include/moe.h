@@ -1,0 +1,201 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) sparse mixture-of-experts layer.
+ *
+ * The layer (the equation of "Mixtral of Experts", section 2.1 "Sparse
+ * Mixture of Experts", as given on the learn.ifs.name flash-card page):
+ *
+ *   y = sum_{i=0}^{n-1} Softmax(TopK(x . W_g))_i * SwiGLU_i(x)
+ *   SwiGLU_i(x) = (silu(x . w1_i) (*) (x . w3_i)) . w2_i,  silu(z) = z * sigmoid(z)
+ *
+ * A bias-free linear router scores n experts per token, keeps the K largest
+ * logits, normalises those K with a softmax, and sums the chosen experts'
+ * SwiGLU outputs with those weights ("Mixture of Experts: Why Mixtral Only
+ * Wakes Up Two Specialists", Part 3, Steps 1-4).
+ *
+ * Conventions shared by every entry point
+ *   - All tensors are row-major and live in device memory of the current CUDA
+ *     device; every pointer must be 16-byte aligned.
+ *       x[T][d]            activations, dtype of the handle
+ *       W_g[d][n]          router weights, always fp32 (column e scores expert e)
+ *       w1[n][d][ffn]      gate projection of each expert, dtype of the handle
+ *       w3[n][d][ffn]      up projection of each expert, dtype of the handle
+ *       w2[n][ffn][d]      down projection of each expert, dtype of the handle
+ *       y[T][d]            output, dtype of the handle (fp32 accumulation,
+ *                          rounded once to bf16 for bf16 handles)
+ *       topk_idx[T][K]     chosen experts, int32, by descending logit; equal
+ *                          logits keep the lower expert index first
+ *       topk_w[T][K]       their softmax weights, fp32, summing to 1 per token
+ *   - The caller owns every tensor it passes.  The handle owns only its
+ *     workspace (routing maps, permuted activations, the expert hidden layer
+ *     and per-row expert outputs), which it allocates with cudaMalloc on the
+ *     first call that needs more room and frees in moe_destroy.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and runs asynchronously; a returned MOE_OK reports launch-time
+ *     success only.  moe_sync_status reports device-side failures.
+ *   - A handle may be used by one host thread at a time, on the device on
+ *     which its workspace was first allocated.  Calls on one handle must not
+ *     overlap on the GPU (they share the workspace): issue them on one stream
+ *     or order the streams.
+ *   - On any error nothing is launched, the outputs are untouched, and
+ *     moe_last_error() describes the failure.
+ */
+#ifndef MOE_B200_MOE_H
+#define MOE_B200_MOE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported symbols stay visible when the library is built with hidden
+ * default visibility. */
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+/* Same object as cudaStream_t; declared here so that this header needs no
+ * CUDA header. */
+typedef struct CUstream_st *moe_stream_t;
+
+typedef struct moe_handle moe_handle;
+
+typedef enum {
+    MOE_F32 = 0,  /* fp32 x, w1, w3, w2, y: CUDA-core fp32 path */
+    MOE_BF16 = 1  /* bf16 x, w1, w3, w2, y: tcgen05 tensor-core path */
+} moe_dtype;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* bad size, null or misaligned pointer, wrong device */
+    MOE_ERR_UNSUPPORTED = 2, /* not an sm_100 device */
+    MOE_ERR_ALLOC = 3,       /* workspace cudaMalloc failed */
+    MOE_ERR_CUDA = 4,        /* a CUDA runtime call or a launch failed */
+    MOE_ERR_TIMEOUT = 5      /* a kernel gave up a bounded wait (see moe_sync_status) */
+} moe_status;
+
+/*
+ * Create a handle for a layer with n experts, K experts per token, model dim
+ * d and expert hidden dim ffn.  Sources: the roles of n and K in section 2.1
+ * of "Mixtral of Experts" (flash cards); the router nn.Linear(dim, n,
+ * bias=False) quoted in Part 3 Step 1 of the neobadger page.
+ *   Constraints: 1 <= K <= n <= 256; d and ffn multiples of 64 in [64, 65536];
+ *   dtype MOE_F32 or MOE_BF16; out != NULL.
+ *   Touches no GPU state (no allocation happens here).
+ *   Errors: MOE_ERR_INVALID_ARG; *out is set to NULL on error.
+ */
+MOE_API moe_status moe_create(int n, int K, int d, int ffn, moe_dtype dtype, moe_handle **out);
+
+/*
+ * Allocate the workspace for up to T_max tokens on the current device, so
+ * that later moe_forward calls with T <= T_max allocate nothing (needed before
+ * capturing a CUDA graph, and outside timed loops).
+ *   Errors: MOE_ERR_INVALID_ARG (null handle, T_max < 0, T_max * K > 2^31 - 1,
+ *   handle bound to another device), MOE_ERR_UNSUPPORTED (device is not
+ *   sm_100), MOE_ERR_ALLOC.
+ */
+MOE_API moe_status moe_reserve(moe_handle *h, int64_t T_max);
+
+/*
+ * The whole layer forward on T tokens: router logits x . W_g (fp32), top-K,
+ * softmax over the K kept logits, dispatch of (token, slot) pairs into
+ * per-expert segments, SwiGLU experts on those segments, gate-weighted
+ * combine into y.  Sources: the layer equation (flash cards, section 2.1);
+ * the three routing lines and Steps 1-4 of Part 3 of the neobadger page.
+ *   T = 0 is a no-op returning MOE_OK.  Grows the workspace if T exceeds the
+ *   reservation.  topk_idx and topk_w are outputs.
+ *   Errors: MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_ALLOC, MOE_ERR_CUDA.
+ */
+MOE_API moe_status moe_forward(moe_handle *h, int64_t T, const void *x, const float *W_g,
+                       const void *w1, const void *w3, const void *w2, void *y,
+                       int32_t *topk_idx, float *topk_w, moe_stream_t stream);
+
+/*
+ * Router only: logits x . W_g in fp32, the K largest (descending; ties to the
+ * lower index), softmax over those K.  Sources: Steps 1-3 of Part 3 of the
+ * neobadger page and the routing lines quoted there (gate, topk, softmax).
+ *   Errors: as moe_forward.
+ */
+MOE_API moe_status moe_route(moe_handle *h, int64_t T, const void *x, const float *W_g,
+                     int32_t *topk_idx, float *topk_w, moe_stream_t stream);
+
+/*
+ * Dispatch only: group the T*K (token, slot) pairs of topk_idx into
+ * per-expert segments, expert by expert, tokens ascending inside an expert
+ * (the "skip the experts whose gate is zero" of the Mixtral paper as quoted
+ * on the ainotis page, laid out for grouped GEMMs).  Outputs (device, int32):
+ *   counts[n]          rows of each expert
+ *   offsets[n+1]       first row of each expert's segment; offsets[n] = T*K
+ *   row_token[T*K]     token of each row
+ *   token_row[T][K]    row of each (token, slot) pair
+ * Any output pointer may be NULL to skip it.  topk_idx values must lie in
+ * [0, n) and be distinct within a token; out-of-range values are counted into
+ * no segment and make the results unspecified (never an out-of-bounds access).
+ *   Errors: as moe_forward.
+ */
+MOE_API moe_status moe_dispatch(moe_handle *h, int64_t T, const int32_t *topk_idx, int32_t *counts,
+                        int32_t *offsets, int32_t *row_token, int32_t *token_row,
+                        moe_stream_t stream);
+
+/*
+ * Experts and combine under a routing supplied by the caller:
+ * y[t] = sum_k topk_w[t][k] * SwiGLU_{topk_idx[t][k]}(x[t]).  Source: the
+ * gate-weighted additive combine of Step 4 (Part 3, neobadger page) and the
+ * sum over experts in the layer equation.  topk_idx must hold distinct experts
+ * per token in [0, n).
+ *   Errors: as moe_forward.
+ */
+MOE_API moe_status moe_forward_with_routing(moe_handle *h, int64_t T, const void *x,
+                                    const int32_t *topk_idx, const float *topk_w,
+                                    const void *w1, const void *w3, const void *w2, void *y,
+                                    moe_stream_t stream);
+
+/*
+ * Debug view of the workspace written by the last moe_forward /
+ * moe_forward_with_routing: name is "H" (expert hidden layer, [rows][ffn],
+ * handle dtype) or "O" (per-row expert outputs, [rows][d], handle dtype for
+ * bf16 handles, fp32 for fp32 handles).  Returns the device pointer and the
+ * row capacity; rows are in dispatch order.
+ *   Errors: MOE_ERR_INVALID_ARG (unknown name, null argument, no workspace yet).
+ */
+MOE_API moe_status moe_workspace_view(moe_handle *h, const char *name, void **ptr, int64_t *rows);
+
+/*
+ * Wait for `stream`, then report whether any kernel of this handle gave up a
+ * bounded wait since the last call (MOE_ERR_TIMEOUT; the flag is cleared) or a
+ * CUDA error is pending (MOE_ERR_CUDA).
+ */
+MOE_API moe_status moe_sync_status(moe_handle *h, moe_stream_t stream);
+
+/*
+ * Per-stage timing with CUDA events, for profiling.  After moe_trace_begin(h,
+ * max_calls) each of the next max_calls moe_forward / moe_forward_with_routing
+ * calls records events around its stages on its stream:
+ *   stage 0 router, 1 dispatch (rank, scan, scatter), 2 gather, 3 GEMM1 (w1/w3
+ *   + SwiGLU), 4 GEMM2 (w2), 5 combine
+ * (stage 0 is 0 ms for moe_forward_with_routing).  moe_trace_end waits for the
+ * recorded events, writes the summed milliseconds of each stage into
+ * stage_ms[0 .. n_stages-1] (n_stages <= 6), the number of traced calls into
+ * *calls, and stops tracing.  Calls beyond max_calls are not traced.
+ *   Errors: MOE_ERR_INVALID_ARG (null handle or output, max_calls < 1 or
+ *   > 100000, end without begin), MOE_ERR_CUDA.
+ */
+MOE_API moe_status moe_trace_begin(moe_handle *h, int max_calls);
+MOE_API moe_status moe_trace_end(moe_handle *h, double *stage_ms, int n_stages, int *calls);
+
+/* Free the workspace and the handle.  NULL is allowed. */
+MOE_API moe_status moe_destroy(moe_handle *h);
+
+/* Message for the last failing call on this host thread ("" if none). */
+MOE_API const char *moe_last_error(void);
+
+/* Library version string. */
+MOE_API const char *moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_MOE_H */

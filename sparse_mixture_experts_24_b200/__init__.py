@@ -1,0 +1,232 @@
+"""B200 (sm_100a) sparse mixture-of-experts layer forward: thin ctypes binding.
+
+The functions here carry the names of the C ABI in include/moe.h and only
+marshal arguments (torch tensors or raw device pointers) into that library;
+every step of the layer runs in its CUDA kernels.  Importing this package
+fails with ImportError when libmoe_b200.so has not been built
+(`python sparse_mixture_experts_24_b200/build.py`): there is no fallback.
+
+The layer: y = sum_i Softmax(TopK(x . W_g))_i * SwiGLU_i(x) with
+SwiGLU_i(x) = (silu(x . w1_i) * (x . w3_i)) . w2_i ("Mixtral of Experts",
+section 2.1; Part 3, Steps 1-4 of "Mixture of Experts: Why Mixtral Only Wakes
+Up Two Specialists").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_F32 = 0
+MOE_BF16 = 1
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_ALLOC = 3
+MOE_ERR_CUDA = 4
+MOE_ERR_TIMEOUT = 5
+
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
+                3: "MOE_ERR_ALLOC", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT"}
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        super().__init__("%s: %s (%s)" % (where, message, STATUS_NAMES.get(status, status)))
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError("libmoe_b200.so is not built; run `python sparse_mixture_experts_24_b200/build.py`")
+
+_vp, _i64, _int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+lib = ctypes.CDLL(LIB_PATH)
+lib.moe_create.argtypes = [_int, _int, _int, _int, _int, ctypes.POINTER(_vp)]
+lib.moe_reserve.argtypes = [_vp, _i64]
+lib.moe_forward.argtypes = [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.moe_route.argtypes = [_vp, _i64, _vp, _vp, _vp, _vp, _vp]
+lib.moe_dispatch.argtypes = [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.moe_forward_with_routing.argtypes = [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.moe_workspace_view.argtypes = [_vp, ctypes.c_char_p, ctypes.POINTER(_vp), ctypes.POINTER(_i64)]
+lib.moe_sync_status.argtypes = [_vp, _vp]
+lib.moe_destroy.argtypes = [_vp]
+lib.moe_trace_begin.argtypes = [_vp, _int]
+lib.moe_trace_end.argtypes = [_vp, ctypes.POINTER(ctypes.c_double), _int, ctypes.POINTER(_int)]
+lib.moe_last_error.restype = ctypes.c_char_p
+lib.moe_version.restype = ctypes.c_char_p
+for _f in ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
+           "moe_forward_with_routing", "moe_workspace_view", "moe_sync_status", "moe_destroy",
+           "moe_trace_begin", "moe_trace_end"):
+    getattr(lib, _f).restype = _int
+
+EXPORTED = ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
+            "moe_forward_with_routing", "moe_workspace_view", "moe_sync_status", "moe_destroy",
+            "moe_last_error", "moe_version", "moe_trace_begin", "moe_trace_end")
+
+TRACE_STAGES = ("router", "dispatch", "gather", "gemm1", "gemm2", "combine")
+
+
+def _ptr(a):
+    """Device (or host) address of a tensor, an int address, or None -> NULL."""
+    if a is None:
+        return None
+    if isinstance(a, int):
+        return a
+    return a.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        try:
+            import torch
+            if torch.cuda.is_available() and torch.cuda.is_initialized():
+                return torch.cuda.current_stream().cuda_stream
+        except ImportError:
+            pass
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != MOE_OK:
+        raise MoEError(rc, where, moe_last_error())
+
+
+def moe_last_error() -> str:
+    return lib.moe_last_error().decode()
+
+
+def moe_version() -> str:
+    return lib.moe_version().decode()
+
+
+def moe_create(n: int, K: int, d: int, ffn: int, dtype: int) -> int:
+    h = _vp()
+    _check(lib.moe_create(n, K, d, ffn, dtype, ctypes.byref(h)), "moe_create")
+    return h.value
+
+
+def moe_reserve(h: int, T_max: int) -> None:
+    _check(lib.moe_reserve(h, T_max), "moe_reserve")
+
+
+def moe_forward(h, T, x, W_g, w1, w3, w2, y, topk_idx, topk_w, stream=None) -> None:
+    _check(lib.moe_forward(h, T, _ptr(x), _ptr(W_g), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(y),
+                           _ptr(topk_idx), _ptr(topk_w), _stream(stream)), "moe_forward")
+
+
+def moe_route(h, T, x, W_g, topk_idx, topk_w, stream=None) -> None:
+    _check(lib.moe_route(h, T, _ptr(x), _ptr(W_g), _ptr(topk_idx), _ptr(topk_w), _stream(stream)),
+           "moe_route")
+
+
+def moe_dispatch(h, T, topk_idx, counts=None, offsets=None, row_token=None, token_row=None,
+                 stream=None) -> None:
+    _check(lib.moe_dispatch(h, T, _ptr(topk_idx), _ptr(counts), _ptr(offsets), _ptr(row_token),
+                            _ptr(token_row), _stream(stream)), "moe_dispatch")
+
+
+def moe_forward_with_routing(h, T, x, topk_idx, topk_w, w1, w3, w2, y, stream=None) -> None:
+    _check(lib.moe_forward_with_routing(h, T, _ptr(x), _ptr(topk_idx), _ptr(topk_w), _ptr(w1),
+                                        _ptr(w3), _ptr(w2), _ptr(y), _stream(stream)),
+           "moe_forward_with_routing")
+
+
+def moe_workspace_view(h, name: str):
+    p, rows = _vp(), _i64()
+    _check(lib.moe_workspace_view(h, name.encode(), ctypes.byref(p), ctypes.byref(rows)),
+           "moe_workspace_view")
+    return p.value, rows.value
+
+
+def moe_sync_status(h, stream=None) -> None:
+    _check(lib.moe_sync_status(h, _stream(stream)), "moe_sync_status")
+
+
+def moe_trace_begin(h, max_calls: int) -> None:
+    _check(lib.moe_trace_begin(h, max_calls), "moe_trace_begin")
+
+
+def moe_trace_end(h):
+    """-> (dict stage -> summed ms, number of traced calls)"""
+    ms = (ctypes.c_double * len(TRACE_STAGES))()
+    calls = _int()
+    _check(lib.moe_trace_end(h, ms, len(TRACE_STAGES), ctypes.byref(calls)), "moe_trace_end")
+    return dict(zip(TRACE_STAGES, list(ms))), calls.value
+
+
+def moe_destroy(h) -> None:
+    _check(lib.moe_destroy(h), "moe_destroy")
+
+
+class MoELayer:
+    """Owns one handle; allocates outputs with torch and calls the C ABI.
+
+    Tensors are torch CUDA tensors; bf16 layers take torch.bfloat16 x and
+    weights, fp32 layers torch.float32; W_g is always torch.float32 [d][n].
+    """
+
+    def __init__(self, n: int, K: int, d: int, ffn: int, dtype: str = "bf16"):
+        self.n, self.K, self.d, self.ffn = n, K, d, ffn
+        self.dtype = dtype
+        self.h = moe_create(n, K, d, ffn, MOE_BF16 if dtype == "bf16" else MOE_F32)
+
+    def reserve(self, T_max: int) -> None:
+        moe_reserve(self.h, T_max)
+
+    def forward(self, x, W_g, w1, w3, w2, y=None, topk_idx=None, topk_w=None, stream=None):
+        import torch
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty_like(x)
+        if topk_idx is None:
+            topk_idx = torch.empty((T, self.K), dtype=torch.int32, device=x.device)
+        if topk_w is None:
+            topk_w = torch.empty((T, self.K), dtype=torch.float32, device=x.device)
+        moe_forward(self.h, T, x, W_g, w1, w3, w2, y, topk_idx, topk_w, stream)
+        return y, topk_idx, topk_w
+
+    def route(self, x, W_g, stream=None):
+        import torch
+        T = x.shape[0]
+        idx = torch.empty((T, self.K), dtype=torch.int32, device=x.device)
+        w = torch.empty((T, self.K), dtype=torch.float32, device=x.device)
+        moe_route(self.h, T, x, W_g, idx, w, stream)
+        return idx, w
+
+    def forward_with_routing(self, x, topk_idx, topk_w, w1, w3, w2, y=None, stream=None):
+        import torch
+        if y is None:
+            y = torch.empty_like(x)
+        moe_forward_with_routing(self.h, x.shape[0], x, topk_idx, topk_w, w1, w3, w2, y, stream)
+        return y
+
+    def dispatch(self, topk_idx, stream=None):
+        import torch
+        T = topk_idx.shape[0]
+        dev = topk_idx.device
+        counts = torch.empty(self.n, dtype=torch.int32, device=dev)
+        offsets = torch.empty(self.n + 1, dtype=torch.int32, device=dev)
+        row_token = torch.empty(max(1, T * self.K), dtype=torch.int32, device=dev)
+        token_row = torch.empty((max(1, T), self.K), dtype=torch.int32, device=dev)
+        moe_dispatch(self.h, T, topk_idx, counts, offsets, row_token, token_row, stream)
+        return counts, offsets, row_token[:T * self.K], token_row[:T]
+
+    def sync_status(self, stream=None) -> None:
+        moe_sync_status(self.h, stream)
+
+    def close(self) -> None:
+        if self.h:
+            moe_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,178 @@
+// dispatch.cu -- group the T*K (token, slot) pairs into contiguous per-expert
+// segments so that each expert runs as one dense GEMM over only the tokens
+// that chose it.
+//
+// Source: the Mixtral paper as quoted on the ainotis page ("How a
+// mixture-of-experts model activates only part of its parameters"): when the
+// gating vector is sparse, the outputs of experts with a zero gate are not
+// computed; and Part 3, Step 2 of "Mixture of Experts: Why Mixtral Only Wakes
+// Up Two Specialists" (the experts not kept are not run at all).  The layout
+// (experts ascending, tokens ascending inside an expert) is this library's.
+//
+// Kernels:
+//   rank_kernel    per block of 256 pairs: expert histogram and the stable
+//                  rank of every pair among the block's pairs of its expert
+//                  (warp match + per-warp counts, no global atomics);
+//   scan_kernel    one block: per-expert counts, segment offsets, each
+//                  block's base inside each segment, and the M-block prefix
+//                  the grouped GEMMs schedule from;
+//   scatter_kernel row of every pair -> row_token, token_row;
+//   gather_kernel  Xp[r] = x[row_token[r]] with 16-byte vectors, a warp per row.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+constexpr int kMaxExperts = 256;
+constexpr int kWarps = kPairsPerBlock / 32;
+
+__global__ void __launch_bounds__(kPairsPerBlock) rank_kernel(const int32_t* __restrict__ idx,
+                                                              int64_t R, int n,
+                                                              int32_t* __restrict__ blockcounts,
+                                                              int32_t* __restrict__ pair_rank) {
+    __shared__ int32_t whist[kWarps][kMaxExperts];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < kWarps * kMaxExperts; i += kPairsPerBlock) (&whist[0][0])[i] = 0;
+    __syncthreads();
+
+    const int64_t p = static_cast<int64_t>(blockIdx.x) * kPairsPerBlock + tid;
+    int e = (p < R) ? idx[p] : -1;
+    if (e < 0 || e >= n) e = -1;  // not a valid expert: ranked nowhere
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const uint32_t lt = (1u << lane) - 1u;
+    const int wrank = __popc(peers & lt);
+    if (e >= 0 && wrank == 0) whist[warp][e] = __popc(peers);
+    __syncthreads();
+    // exclusive prefix over the warps, per expert; block total
+    for (int ex = tid; ex < n; ex += kPairsPerBlock) {
+        int run = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const int c = whist[w][ex];
+            whist[w][ex] = run;
+            run += c;
+        }
+        blockcounts[static_cast<int64_t>(blockIdx.x) * n + ex] = run;
+    }
+    __syncthreads();
+    if (p < R) pair_rank[p] = (e >= 0) ? whist[warp][e] + wrank : -1;
+}
+
+// Exclusive scan of one value per thread over a 256-thread block.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = (lane < 8) ? s_warp[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += u;
+        }
+        if (lane < 8) s_warp[lane] = wi - w;  // exclusive warp bases
+    }
+    __syncthreads();
+    const int r = s_warp[warp] + incl - v;
+    __syncthreads();
+    return r;
+}
+
+__global__ void __launch_bounds__(256) scan_kernel(int32_t* __restrict__ blockcounts, int nblk,
+                                                   int n, int64_t R, int bm,
+                                                   int32_t* __restrict__ counts,
+                                                   int32_t* __restrict__ offsets,
+                                                   int32_t* __restrict__ mblk_base) {
+    __shared__ int s_warp[8];
+    const int e = threadIdx.x;
+    int total = 0;
+    if (e < n) {
+        for (int b = 0; b < nblk; ++b) {
+            int32_t* c = blockcounts + static_cast<int64_t>(b) * n + e;
+            const int v = *c;
+            *c = total;  // exclusive within the expert
+            total += v;
+        }
+    }
+    const int off = block_exclusive_scan(e < n ? total : 0, s_warp);
+    const int mb = (e < n) ? (total + bm - 1) / bm : 0;
+    const int mbase = block_exclusive_scan(mb, s_warp);
+    if (e < n) {
+        counts[e] = total;
+        offsets[e] = off;
+        mblk_base[e] = mbase;
+        for (int b = 0; b < nblk; ++b) blockcounts[static_cast<int64_t>(b) * n + e] += off;
+    }
+    if (e == n - 1) {
+        offsets[n] = off + total;
+        mblk_base[n] = mbase + mb;
+    }
+    (void)R;
+}
+
+__global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict__ idx, int64_t R,
+                                                      int K, int n,
+                                                      const int32_t* __restrict__ blockbase,
+                                                      const int32_t* __restrict__ pair_rank,
+                                                      int32_t* __restrict__ row_token,
+                                                      int32_t* __restrict__ token_row) {
+    const int64_t p = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (p >= R) return;
+    const int e = idx[p];
+    const int rk = pair_rank[p];
+    if (e < 0 || e >= n || rk < 0) {
+        token_row[p] = -1;
+        return;
+    }
+    const int dest = blockbase[(p / kPairsPerBlock) * n + e] + rk;
+    row_token[dest] = static_cast<int32_t>(p / K);
+    token_row[p] = dest;
+}
+
+cudaError_t launch_dispatch(const int32_t* topk_idx, int64_t T, int K, int n, int bm,
+                            const DispatchBufs& b, cudaStream_t st) {
+    const int64_t R = T * K;
+    const int nblk = static_cast<int>((R + kPairsPerBlock - 1) / kPairsPerBlock);
+    rank_kernel<<<nblk, kPairsPerBlock, 0, st>>>(topk_idx, R, n, b.blockcounts, b.pair_rank);
+    scan_kernel<<<1, 256, 0, st>>>(b.blockcounts, nblk, n, R, bm, b.counts, b.offsets, b.mblk_base);
+    scatter_kernel<<<static_cast<unsigned>((R + 255) / 256), 256, 0, st>>>(
+        topk_idx, R, K, n, b.blockcounts, b.pair_rank, b.row_token, b.token_row);
+    return cudaGetLastError();
+}
+
+__global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ x,
+                                                     const int32_t* __restrict__ row_token,
+                                                     int64_t R, int64_t T, int64_t vec_per_row,
+                                                     uint4* __restrict__ xp) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < R;
+         r += nwarps) {
+        const int64_t t = row_token[r];
+        if (t < 0 || t >= T) continue;  // a row no valid pair reached (bad expert ids)
+        const uint4* src = x + t * vec_per_row;
+        uint4* dst = xp + r * vec_per_row;
+        for (int64_t v = lane; v < vec_per_row; v += 32) dst[v] = __ldg(src + v);
+    }
+}
+
+cudaError_t launch_gather(const void* x, const int32_t* row_token, int64_t R, int64_t T,
+                          int64_t row_bytes, void* xp, int num_sms, cudaStream_t st) {
+    const int64_t warps = R;
+    int64_t blocks = (warps + 7) / 8;
+    const int64_t cap = static_cast<int64_t>(num_sms) * 16;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    gather_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        static_cast<const uint4*>(x), row_token, R, T, row_bytes / 16, static_cast<uint4*>(xp));
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,76 @@
+// kernels.h -- host-side launchers of the MoE kernels (internal to the library).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Rows of one M-block of the tensor-core GEMMs and of the CUDA-core GEMMs.
+constexpr int kTcBM = 128;
+constexpr int kSimtBM = 64;
+// (token, slot) pairs per dispatch block.
+constexpr int kPairsPerBlock = 256;
+
+// Router: logits (fp32), top-K, softmax over the kept K.
+cudaError_t launch_router(const void* x, bool x_bf16, const float* Wg, int64_t T, int d, int n,
+                          int K, int32_t* topk_idx, float* topk_w, float* logits_ws, int num_sms,
+                          cudaStream_t st);
+
+// Dispatch workspace (device, int32 unless noted).
+struct DispatchBufs {
+    int32_t* blockcounts;  // [nblk][n]: per-block counts, then per-block segment bases
+    int32_t* pair_rank;    // [R]: stable rank of each pair inside its block and expert
+    int32_t* counts;       // [n]
+    int32_t* offsets;      // [n+1]
+    int32_t* mblk_base;    // [n+1]: exclusive prefix of M-blocks per expert
+    int32_t* row_token;    // [R]
+    int32_t* token_row;    // [R] = [T][K]
+};
+
+// Histogram + stable in-block ranks, scan, scatter.  bm = rows per M-block of
+// the GEMM that consumes the segments.
+cudaError_t launch_dispatch(const int32_t* topk_idx, int64_t T, int K, int n, int bm,
+                            const DispatchBufs& b, cudaStream_t st);
+
+// Xp[r] = x[row_token[r]] for r < R (row_bytes per row, multiple of 16);
+// rows whose token is outside [0, T) are skipped.
+cudaError_t launch_gather(const void* x, const int32_t* row_token, int64_t R, int64_t T,
+                          int64_t row_bytes, void* xp, int num_sms, cudaStream_t st);
+
+// y[t] = sum_k topk_w[t][k] * O[token_row[t][k]]; O and y bf16 (o_bf16) or fp32.
+cudaError_t launch_combine(const void* O, bool bf16, const int32_t* token_row, const float* topk_w,
+                           int64_t T, int K, int d, void* y, int num_sms, cudaStream_t st);
+
+// CUDA-core fp32 grouped GEMMs (fp32 handles).
+//   H[r] = silu(Xp[r] . w1[e]) * (Xp[r] . w3[e]) for rows r of expert e
+cudaError_t launch_simt_gemm1(const float* xp, const float* w1, const float* w3, float* h,
+                              const int32_t* offsets, const int32_t* mblk_base, int n, int64_t R,
+                              int d, int F, cudaStream_t st);
+//   O[r] = H[r] . w2[e]
+cudaError_t launch_simt_gemm2(const float* h, const float* w2, float* o, const int32_t* offsets,
+                              const int32_t* mblk_base, int n, int64_t R, int d, int F,
+                              cudaStream_t st);
+
+// tcgen05 grouped GEMMs (bf16 handles).  Tensor maps are built by the host
+// (see moe_api.cu) over: Xp [R_cap][d], w1/w3 [n][d][F], H [R_cap][F], w2 [n][F][d].
+struct TcGemmArgs {
+    const int32_t* offsets;
+    const int32_t* mblk_base;
+    int n;
+    int64_t R;         // rows (T*K): bounds the tile count
+    int k_blocks;      // reduction length / 64
+    int n_tiles;       // tiles along the output columns
+    int out_cols;      // F (GEMM1) or d (GEMM2)
+    void* out;         // H (GEMM1) or O (GEMM2), bf16 row-major [R][out_cols]
+    int* status;       // device status word
+};
+
+cudaError_t launch_tc_gemm1(const CUtensorMap& tm_xp, const CUtensorMap& tm_w1,
+                            const CUtensorMap& tm_w3, const TcGemmArgs& a, int num_sms,
+                            cudaStream_t st);
+cudaError_t launch_tc_gemm2(const CUtensorMap& tm_h, const CUtensorMap& tm_w2, const TcGemmArgs& a,
+                            int num_sms, cudaStream_t st);
+
+}  // namespace moe

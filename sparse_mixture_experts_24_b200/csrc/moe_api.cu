@@ -1,0 +1,544 @@
+// moe_api.cu -- the C ABI declared in include/moe.h: argument checking, the
+// workspace, TMA tensor maps, and the launch sequence of the layer forward
+//   router -> dispatch (rank, scan, scatter) -> gather -> GEMM1 -> GEMM2 -> combine
+// all on the caller's stream with no host synchronisation.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+moe_status fail(moe_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+moe_status ok() {
+    g_err[0] = '\0';
+    return MOE_OK;
+}
+
+moe_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// cuTensorMapEncodeTiled, fetched through the runtime so the library does not
+// link libcuda directly.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// bf16 row-major [rows][cols] operand read in 128 (rows) x 64 (cols) boxes.
+bool encode_rows(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t es[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 weights [n][rows][cols] read in 64 (rows) x 64 (cols) boxes of one expert.
+bool encode_weights(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t n) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[3] = {cols, rows, n};
+    cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
+    cuuint32_t box[3] = {64, 64, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+struct moe_handle {
+    int n, K, d, F;
+    moe_dtype dtype;
+    int device = -1;
+    int num_sms = 0;
+    int64_t T_cap = 0;
+    void* ws = nullptr;
+    size_t ws_bytes = 0;
+    moe::DispatchBufs db{};
+    float* logits = nullptr;
+    void* xp = nullptr;
+    void* h = nullptr;
+    void* o = nullptr;
+    int* status = nullptr;
+    CUtensorMap tm_xp, tm_h, tm_w1, tm_w3, tm_w2;
+    const void* c_w1 = nullptr;
+    const void* c_w3 = nullptr;
+    const void* c_w2 = nullptr;
+    // tracing: kTraceEvents events per traced call
+    std::vector<cudaEvent_t> trace_ev;
+    int trace_max = 0;
+    int trace_calls = 0;
+    bool tracing = false;
+
+    size_t esize() const { return dtype == MOE_BF16 ? 2 : 4; }
+    size_t osize() const { return dtype == MOE_BF16 ? 2 : 4; }
+};
+
+namespace {
+
+constexpr int kTraceStages = 6;
+constexpr int kTraceEvents = kTraceStages + 1;
+
+// Event that closes `stage` of the current traced call (stage -1 = the start),
+// or nullptr when this call is not traced.
+cudaEvent_t trace_event(moe_handle* h, int stage) {
+    if (!h->tracing || h->trace_calls >= h->trace_max) return nullptr;
+    return h->trace_ev[static_cast<size_t>(h->trace_calls) * kTraceEvents + (stage + 1)];
+}
+
+void trace_mark(moe_handle* h, int stage, cudaStream_t st) {
+    cudaEvent_t e = trace_event(h, stage);
+    if (e) cudaEventRecord(e, st);
+}
+
+void trace_finish_call(moe_handle* h) {
+    if (h->tracing && h->trace_calls < h->trace_max) ++h->trace_calls;
+}
+
+void trace_free(moe_handle* h) {
+    for (cudaEvent_t e : h->trace_ev) cudaEventDestroy(e);
+    h->trace_ev.clear();
+    h->tracing = false;
+    h->trace_max = h->trace_calls = 0;
+}
+
+moe_status check_device(moe_handle* h) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (h->device < 0) {
+        int major = 0, minor = 0, sms = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        if (major != 10 || minor != 0)
+            return fail(MOE_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
+                        dev, major, minor);
+        h->device = dev;
+        h->num_sms = sms;
+    } else if (dev != h->device) {
+        return fail(MOE_ERR_INVALID_ARG, "handle belongs to device %d, current device is %d",
+                    h->device, dev);
+    }
+    return MOE_OK;
+}
+
+moe_status grow(moe_handle* h, int64_t T) {
+    if (T <= h->T_cap && h->ws) return MOE_OK;
+    const int64_t R = T * h->K;
+    const int64_t nblk = (R + moe::kPairsPerBlock - 1) / moe::kPairsPerBlock;
+    const size_t A = 256;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off = align_up(off + (bytes ? bytes : 1), A);
+        return o;
+    };
+    const size_t o_blockcounts = take(static_cast<size_t>(nblk) * h->n * 4);
+    const size_t o_pair_rank = take(static_cast<size_t>(R) * 4);
+    const size_t o_counts = take(static_cast<size_t>(h->n) * 4);
+    const size_t o_offsets = take(static_cast<size_t>(h->n + 1) * 4);
+    const size_t o_mblk = take(static_cast<size_t>(h->n + 1) * 4);
+    const size_t o_row_token = take(static_cast<size_t>(R) * 4);
+    const size_t o_token_row = take(static_cast<size_t>(R) * 4);
+    const size_t o_logits = take(h->n > 32 ? static_cast<size_t>(T) * h->n * 4 : 0);
+    const size_t o_status = take(64);
+    const size_t o_xp = take(static_cast<size_t>(R) * h->d * h->esize());
+    const size_t o_h = take(static_cast<size_t>(R) * h->F * h->esize());
+    const size_t o_o = take(static_cast<size_t>(R) * h->d * h->osize());
+    const size_t total = off;
+
+    if (h->ws) {
+        cudaFree(h->ws);
+        h->ws = nullptr;
+        h->T_cap = 0;
+    }
+    void* p = nullptr;
+    cudaError_t e = cudaMalloc(&p, total);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(MOE_ERR_ALLOC, "cudaMalloc(%zu bytes) for the workspace failed: %s", total,
+                    cudaGetErrorString(e));
+    }
+    e = cudaMemset(p, 0, total);
+    if (e != cudaSuccess) {
+        cudaFree(p);
+        return cuda_fail(e, "cudaMemset(workspace)");
+    }
+    uint8_t* b = static_cast<uint8_t*>(p);
+    h->ws = p;
+    h->ws_bytes = total;
+    h->T_cap = T;
+    h->db.blockcounts = reinterpret_cast<int32_t*>(b + o_blockcounts);
+    h->db.pair_rank = reinterpret_cast<int32_t*>(b + o_pair_rank);
+    h->db.counts = reinterpret_cast<int32_t*>(b + o_counts);
+    h->db.offsets = reinterpret_cast<int32_t*>(b + o_offsets);
+    h->db.mblk_base = reinterpret_cast<int32_t*>(b + o_mblk);
+    h->db.row_token = reinterpret_cast<int32_t*>(b + o_row_token);
+    h->db.token_row = reinterpret_cast<int32_t*>(b + o_token_row);
+    h->logits = reinterpret_cast<float*>(b + o_logits);
+    h->status = reinterpret_cast<int*>(b + o_status);
+    h->xp = b + o_xp;
+    h->h = b + o_h;
+    h->o = b + o_o;
+    if (h->dtype == MOE_BF16) {
+        if (!encode_rows(&h->tm_xp, h->xp, h->d, static_cast<uint64_t>(R)) ||
+            !encode_rows(&h->tm_h, h->h, h->F, static_cast<uint64_t>(R)))
+            return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the workspace");
+    }
+    return MOE_OK;
+}
+
+moe_status check_common(moe_handle* h, int64_t T) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "null handle");
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T = %lld < 0", static_cast<long long>(T));
+    if (T > 0 && T * h->K > 2147483647LL)
+        return fail(MOE_ERR_INVALID_ARG, "T * K = %lld exceeds 2^31 - 1",
+                    static_cast<long long>(T * h->K));
+    return MOE_OK;
+}
+
+#define REQUIRE_PTR(p)                                                                        \
+    do {                                                                                      \
+        if (!(p)) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", #p);                         \
+        if (!aligned16(p)) return fail(MOE_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p); \
+    } while (0)
+
+moe_status prepare(moe_handle* h, int64_t T) {
+    moe_status s = check_device(h);
+    if (s != MOE_OK) return s;
+    return grow(h, T);
+}
+
+moe_status run_experts(moe_handle* h, int64_t T, const void* x, const int32_t* topk_idx,
+                       const float* topk_w, const void* w1, const void* w3, const void* w2, void* y,
+                       cudaStream_t st) {
+    const bool bf = h->dtype == MOE_BF16;
+    const int64_t R = T * h->K;
+    cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n, bf ? moe::kTcBM : moe::kSimtBM,
+                                         h->db, st);
+    if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
+    trace_mark(h, 1, st);
+    e = moe::launch_gather(x, h->db.row_token, R, T, static_cast<int64_t>(h->d) * h->esize(), h->xp,
+                           h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+    trace_mark(h, 2, st);
+    if (bf) {
+        if (w1 != h->c_w1) {
+            if (!encode_weights(&h->tm_w1, w1, h->F, h->d, h->n))
+                return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for w1");
+            h->c_w1 = w1;
+        }
+        if (w3 != h->c_w3) {
+            if (!encode_weights(&h->tm_w3, w3, h->F, h->d, h->n))
+                return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for w3");
+            h->c_w3 = w3;
+        }
+        if (w2 != h->c_w2) {
+            if (!encode_weights(&h->tm_w2, w2, h->d, h->F, h->n))
+                return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for w2");
+            h->c_w2 = w2;
+        }
+        moe::TcGemmArgs a1{};
+        a1.offsets = h->db.offsets;
+        a1.mblk_base = h->db.mblk_base;
+        a1.n = h->n;
+        a1.R = R;
+        a1.k_blocks = h->d / 64;
+        a1.n_tiles = (h->F + 127) / 128;
+        a1.out_cols = h->F;
+        a1.out = h->h;
+        a1.status = h->status;
+        e = moe::launch_tc_gemm1(h->tm_xp, h->tm_w1, h->tm_w3, a1, h->num_sms, st);
+        if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
+        trace_mark(h, 3, st);
+        moe::TcGemmArgs a2 = a1;
+        a2.k_blocks = h->F / 64;
+        a2.n_tiles = (h->d + 255) / 256;
+        a2.out_cols = h->d;
+        a2.out = h->o;
+        e = moe::launch_tc_gemm2(h->tm_h, h->tm_w2, a2, h->num_sms, st);
+        if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
+        trace_mark(h, 4, st);
+    } else {
+        e = moe::launch_simt_gemm1(static_cast<const float*>(h->xp), static_cast<const float*>(w1),
+                                   static_cast<const float*>(w3), static_cast<float*>(h->h),
+                                   h->db.offsets, h->db.mblk_base, h->n, R, h->d, h->F, st);
+        if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
+        trace_mark(h, 3, st);
+        e = moe::launch_simt_gemm2(static_cast<const float*>(h->h), static_cast<const float*>(w2),
+                                   static_cast<float*>(h->o), h->db.offsets, h->db.mblk_base, h->n,
+                                   R, h->d, h->F, st);
+        if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
+        trace_mark(h, 4, st);
+    }
+    e = moe::launch_combine(h->o, bf, h->db.token_row, topk_w, T, h->K, h->d, y, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+    trace_mark(h, 5, st);
+    trace_finish_call(h);
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_create(int n, int K, int d, int ffn, moe_dtype dtype, moe_handle** out) {
+    if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (n < 1 || n > 256) return fail(MOE_ERR_INVALID_ARG, "n = %d outside [1, 256]", n);
+    if (K < 1 || K > n) return fail(MOE_ERR_INVALID_ARG, "K = %d outside [1, n = %d]", K, n);
+    if (d < 64 || d > 65536 || d % 64 != 0)
+        return fail(MOE_ERR_INVALID_ARG, "d = %d is not a multiple of 64 in [64, 65536]", d);
+    if (ffn < 64 || ffn > 65536 || ffn % 64 != 0)
+        return fail(MOE_ERR_INVALID_ARG, "ffn = %d is not a multiple of 64 in [64, 65536]", ffn);
+    if (dtype != MOE_F32 && dtype != MOE_BF16)
+        return fail(MOE_ERR_INVALID_ARG, "dtype = %d is not MOE_F32 or MOE_BF16", static_cast<int>(dtype));
+    moe_handle* h = new (std::nothrow) moe_handle();
+    if (!h) return fail(MOE_ERR_ALLOC, "out of host memory");
+    h->n = n;
+    h->K = K;
+    h->d = d;
+    h->F = ffn;
+    h->dtype = dtype;
+    *out = h;
+    return ok();
+}
+
+moe_status moe_reserve(moe_handle* h, int64_t T_max) {
+    moe_status s = check_common(h, T_max);
+    if (s != MOE_OK) return s;
+    if (T_max == 0) return ok();
+    s = prepare(h, T_max);
+    return s == MOE_OK ? ok() : s;
+}
+
+moe_status moe_route(moe_handle* h, int64_t T, const void* x, const float* W_g, int32_t* topk_idx,
+                     float* topk_w, moe_stream_t stream) {
+    moe_status s = check_common(h, T);
+    if (s != MOE_OK) return s;
+    if (T == 0) return ok();
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(W_g);
+    REQUIRE_PTR(topk_idx);
+    REQUIRE_PTR(topk_w);
+    s = prepare(h, T);
+    if (s != MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = moe::launch_router(x, h->dtype == MOE_BF16, W_g, T, h->d, h->n, h->K, topk_idx,
+                                       topk_w, h->logits, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "router launch");
+    return ok();
+}
+
+moe_status moe_forward(moe_handle* h, int64_t T, const void* x, const float* W_g, const void* w1,
+                       const void* w3, const void* w2, void* y, int32_t* topk_idx, float* topk_w,
+                       moe_stream_t stream) {
+    moe_status s = check_common(h, T);
+    if (s != MOE_OK) return s;
+    if (T == 0) return ok();
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(W_g);
+    REQUIRE_PTR(w1);
+    REQUIRE_PTR(w3);
+    REQUIRE_PTR(w2);
+    REQUIRE_PTR(y);
+    REQUIRE_PTR(topk_idx);
+    REQUIRE_PTR(topk_w);
+    s = prepare(h, T);
+    if (s != MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    trace_mark(h, -1, st);
+    cudaError_t e = moe::launch_router(x, h->dtype == MOE_BF16, W_g, T, h->d, h->n, h->K, topk_idx,
+                                       topk_w, h->logits, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "router launch");
+    trace_mark(h, 0, st);
+    s = run_experts(h, T, x, topk_idx, topk_w, w1, w3, w2, y, st);
+    return s == MOE_OK ? ok() : s;
+}
+
+moe_status moe_forward_with_routing(moe_handle* h, int64_t T, const void* x,
+                                    const int32_t* topk_idx, const float* topk_w, const void* w1,
+                                    const void* w3, const void* w2, void* y, moe_stream_t stream) {
+    moe_status s = check_common(h, T);
+    if (s != MOE_OK) return s;
+    if (T == 0) return ok();
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(topk_idx);
+    REQUIRE_PTR(topk_w);
+    REQUIRE_PTR(w1);
+    REQUIRE_PTR(w3);
+    REQUIRE_PTR(w2);
+    REQUIRE_PTR(y);
+    s = prepare(h, T);
+    if (s != MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    trace_mark(h, -1, st);
+    trace_mark(h, 0, st);
+    s = run_experts(h, T, x, topk_idx, topk_w, w1, w3, w2, y, st);
+    return s == MOE_OK ? ok() : s;
+}
+
+moe_status moe_dispatch(moe_handle* h, int64_t T, const int32_t* topk_idx, int32_t* counts,
+                        int32_t* offsets, int32_t* row_token, int32_t* token_row,
+                        moe_stream_t stream) {
+    moe_status s = check_common(h, T);
+    if (s != MOE_OK) return s;
+    REQUIRE_PTR(topk_idx);
+    if (T == 0) return ok();
+    if (counts && !aligned16(counts)) return fail(MOE_ERR_INVALID_ARG, "counts is not 16-byte aligned");
+    if (offsets && !aligned16(offsets)) return fail(MOE_ERR_INVALID_ARG, "offsets is not 16-byte aligned");
+    if (row_token && !aligned16(row_token))
+        return fail(MOE_ERR_INVALID_ARG, "row_token is not 16-byte aligned");
+    if (token_row && !aligned16(token_row))
+        return fail(MOE_ERR_INVALID_ARG, "token_row is not 16-byte aligned");
+    s = prepare(h, T);
+    if (s != MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t R = T * h->K;
+    cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n,
+                                         h->dtype == MOE_BF16 ? moe::kTcBM : moe::kSimtBM, h->db, st);
+    if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
+    struct {
+        void* dst;
+        const void* src;
+        size_t bytes;
+    } cp[4] = {{counts, h->db.counts, static_cast<size_t>(h->n) * 4},
+               {offsets, h->db.offsets, static_cast<size_t>(h->n + 1) * 4},
+               {row_token, h->db.row_token, static_cast<size_t>(R) * 4},
+               {token_row, h->db.token_row, static_cast<size_t>(R) * 4}};
+    for (auto& c : cp) {
+        if (!c.dst) continue;
+        e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyDeviceToDevice, st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(dispatch output)");
+    }
+    return ok();
+}
+
+moe_status moe_workspace_view(moe_handle* h, const char* name, void** ptr, int64_t* rows) {
+    if (!h || !name || !ptr || !rows) return fail(MOE_ERR_INVALID_ARG, "null argument");
+    if (!h->ws) return fail(MOE_ERR_INVALID_ARG, "no workspace allocated yet");
+    if (strcmp(name, "H") == 0)
+        *ptr = h->h;
+    else if (strcmp(name, "O") == 0)
+        *ptr = h->o;
+    else
+        return fail(MOE_ERR_INVALID_ARG, "unknown workspace buffer '%s' (use \"H\" or \"O\")", name);
+    *rows = h->T_cap * h->K;
+    return ok();
+}
+
+moe_status moe_sync_status(moe_handle* h, moe_stream_t stream) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "null handle");
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "pending CUDA error");
+    if (!h->status) return ok();
+    int st = 0;
+    e = cudaMemcpy(&st, h->status, sizeof st, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(status)");
+    if (st != 0) {
+        cudaMemset(h->status, 0, sizeof st);
+        return fail(MOE_ERR_TIMEOUT, "a kernel gave up a bounded wait (status bits 0x%x)", st);
+    }
+    return ok();
+}
+
+moe_status moe_trace_begin(moe_handle* h, int max_calls) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "null handle");
+    if (max_calls < 1 || max_calls > 100000)
+        return fail(MOE_ERR_INVALID_ARG, "max_calls = %d outside [1, 100000]", max_calls);
+    trace_free(h);
+    h->trace_ev.resize(static_cast<size_t>(max_calls) * kTraceEvents, nullptr);
+    for (auto& ev : h->trace_ev) {
+        cudaError_t e = cudaEventCreate(&ev);
+        if (e != cudaSuccess) {
+            ev = nullptr;
+            trace_free(h);
+            return cuda_fail(e, "cudaEventCreate");
+        }
+    }
+    h->trace_max = max_calls;
+    h->trace_calls = 0;
+    h->tracing = true;
+    return ok();
+}
+
+moe_status moe_trace_end(moe_handle* h, double* stage_ms, int n_stages, int* calls) {
+    if (!h || !stage_ms || !calls) return fail(MOE_ERR_INVALID_ARG, "null argument");
+    if (!h->tracing) return fail(MOE_ERR_INVALID_ARG, "moe_trace_end without moe_trace_begin");
+    if (n_stages < 1 || n_stages > kTraceStages)
+        return fail(MOE_ERR_INVALID_ARG, "n_stages = %d outside [1, %d]", n_stages, kTraceStages);
+    for (int s = 0; s < n_stages; ++s) stage_ms[s] = 0.0;
+    for (int c = 0; c < h->trace_calls; ++c) {
+        cudaEvent_t* ev = &h->trace_ev[static_cast<size_t>(c) * kTraceEvents];
+        cudaError_t e = cudaEventSynchronize(ev[kTraceEvents - 1]);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+        for (int s = 0; s < n_stages; ++s) {
+            float ms = 0.f;
+            e = cudaEventElapsedTime(&ms, ev[s], ev[s + 1]);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaEventElapsedTime");
+            stage_ms[s] += ms;
+        }
+    }
+    *calls = h->trace_calls;
+    trace_free(h);
+    return ok();
+}
+
+moe_status moe_destroy(moe_handle* h) {
+    if (!h) return ok();
+    trace_free(h);
+    if (h->ws) cudaFree(h->ws);
+    delete h;
+    return ok();
+}
+
+const char* moe_last_error(void) { return g_err; }
+
+const char* moe_version(void) { return "moe-b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

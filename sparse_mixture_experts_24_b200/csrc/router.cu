@@ -1,0 +1,313 @@
+// router.cu -- the MoE gate on CUDA cores in fp32: logits L = x . W_g, the K
+// largest logits per token (descending; equal logits keep the lower expert
+// index), and the softmax over those K.
+//
+// Source: "Mixture of Experts: Why Mixtral Only Wakes Up Two Specialists",
+// Part 3, Step 1 (a bias-free linear layer scores every expert), Step 2 (keep
+// the two highest scores and their positions) and Step 3 (softmax over the two
+// kept scores); the layer equation of "Mixtral of Experts" section 2.1 (the
+// dropped logits are -inf, so the softmax runs over the kept ones only).
+//
+// Two kernels:
+//   router_small_kernel  n <= 32: one warp per group of TPW tokens; the lanes
+//                        split d in 16-byte vectors, every lane keeps all n
+//                        partial logits of its tokens in registers, a shuffle
+//                        butterfly sums them, lane 0 picks the top K.
+//   router_logits_kernel + router_topk_kernel  n > 32: a 64x64 register-tiled
+//                        fp32 GEMM writes the logits to the workspace, then a
+//                        warp per token selects the top K with shuffles.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+template <typename XT>
+struct XVec;  // 16-byte vector of x elements widened to fp32
+
+template <>
+struct XVec<uint16_t> {
+    static constexpr int kElems = 8;
+    __device__ __forceinline__ static void load(const uint16_t* p, float (&v)[8]) {
+        uint4 q = __ldg(reinterpret_cast<const uint4*>(p));
+        unpack_bf16x2(q.x, v[0], v[1]);
+        unpack_bf16x2(q.y, v[2], v[3]);
+        unpack_bf16x2(q.z, v[4], v[5]);
+        unpack_bf16x2(q.w, v[6], v[7]);
+    }
+};
+
+template <>
+struct XVec<float> {
+    static constexpr int kElems = 4;
+    __device__ __forceinline__ static void load(const float* p, float (&v)[4]) {
+        float4 q = __ldg(reinterpret_cast<const float4*>(p));
+        v[0] = q.x;
+        v[1] = q.y;
+        v[2] = q.z;
+        v[3] = q.w;
+    }
+};
+
+// Top-K of one token's logits held in registers (NE slots, n valid), written
+// with the softmax over the kept logits.  Strict '>' while scanning upwards
+// keeps the lower index on ties (NaN logits arrive here as -inf).
+template <int NE>
+__device__ __forceinline__ void topk_softmax_regs(const float (&L)[NE], int n, int K,
+                                                  int32_t* idx_out, float* w_out) {
+    uint32_t taken = 0;
+    float m = 0.f, s = 0.f;
+    for (int k = 0; k < K; ++k) {
+        int best = -1;
+        float bv = 0.f;
+#pragma unroll
+        for (int e = 0; e < NE; ++e) {
+            if (e < n && !((taken >> e) & 1u)) {
+                if (best < 0 || L[e] > bv) {
+                    best = e;
+                    bv = L[e];
+                }
+            }
+        }
+        taken |= 1u << best;
+        if (k == 0) m = bv;
+        const float ex = expf(bv - m);
+        s += ex;
+        idx_out[k] = best;
+        w_out[k] = ex;
+    }
+    const float inv = 1.f / s;
+    for (int k = 0; k < K; ++k) w_out[k] *= inv;
+}
+
+template <typename XT, int NE, int TPW>
+__global__ void __launch_bounds__(256) router_small_kernel(const XT* __restrict__ x,
+                                                           const float* __restrict__ Wg, int64_t T,
+                                                           int d, int n, int K,
+                                                           int32_t* __restrict__ topk_idx,
+                                                           float* __restrict__ topk_w) {
+    constexpr int VE = XVec<XT>::kElems;
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t t0 = warp * TPW;
+    if (t0 >= T) return;
+
+    float acc[TPW][NE];
+#pragma unroll
+    for (int t = 0; t < TPW; ++t)
+#pragma unroll
+        for (int e = 0; e < NE; ++e) acc[t][e] = 0.f;
+
+    const int nvec = d / VE;
+    for (int v = lane; v < nvec; v += 32) {
+        float xv[TPW][VE];
+#pragma unroll
+        for (int t = 0; t < TPW; ++t) {
+            if (t0 + t < T) {
+                XVec<XT>::load(x + (t0 + t) * static_cast<int64_t>(d) + static_cast<int64_t>(v) * VE,
+                               xv[t]);
+            } else {
+#pragma unroll
+                for (int u = 0; u < VE; ++u) xv[t][u] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < VE; ++u) {
+            const float* wrow = Wg + static_cast<int64_t>(v * VE + u) * n;
+#pragma unroll
+            for (int e = 0; e < NE; ++e) {
+                if (e < n) {
+                    const float w = __ldg(wrow + e);
+#pragma unroll
+                    for (int t = 0; t < TPW; ++t) acc[t][e] = fmaf(xv[t][u], w, acc[t][e]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < TPW; ++t)
+#pragma unroll
+        for (int e = 0; e < NE; ++e) {
+            float a = acc[t][e];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+            acc[t][e] = (a != a) ? -INFINITY : a;  // NaN ranks lowest
+        }
+    if (lane == 0) {
+#pragma unroll
+        for (int t = 0; t < TPW; ++t)
+            if (t0 + t < T)
+                topk_softmax_regs<NE>(acc[t], n, K, topk_idx + (t0 + t) * K, topk_w + (t0 + t) * K);
+    }
+}
+
+// ---- n > 32: tiled logits GEMM ---------------------------------------------
+constexpr int kRT = 64;   // tokens per tile
+constexpr int kRE = 64;   // experts per tile
+constexpr int kRK = 32;   // d per smem chunk
+
+template <typename XT>
+__global__ void __launch_bounds__(256) router_logits_kernel(const XT* __restrict__ x,
+                                                            const float* __restrict__ Wg,
+                                                            int64_t T, int d, int n,
+                                                            float* __restrict__ logits) {
+    __shared__ float xs[kRK][kRT + 4];
+    __shared__ float ws[kRK][kRE + 4];
+    const int tid = threadIdx.x;
+    const int tx = tid & 15;   // expert group
+    const int ty = tid >> 4;   // token group
+    const int64_t tok0 = static_cast<int64_t>(blockIdx.x) * kRT;
+    const int e0 = blockIdx.y * kRE;
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+    for (int k0 = 0; k0 < d; k0 += kRK) {
+        // x chunk: 64 tokens x 32 d, stored transposed (d-major).
+        for (int i = tid; i < kRT * kRK; i += 256) {
+            const int t = i / kRK, k = i % kRK;
+            const int64_t tok = tok0 + t;
+            float v = 0.f;
+            if (tok < T) {
+                const int64_t off = tok * d + k0 + k;
+                if constexpr (sizeof(XT) == 2)
+                    v = bf16_bits_to_float(x[off]);
+                else
+                    v = static_cast<float>(x[off]);
+            }
+            xs[k][t] = v;
+        }
+        for (int i = tid; i < kRK * kRE; i += 256) {
+            const int k = i / kRE, e = i % kRE;
+            ws[k][e] = (e0 + e < n) ? __ldg(Wg + static_cast<int64_t>(k0 + k) * n + e0 + e) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int k = 0; k < kRK; ++k) {
+            float a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = xs[k][ty * 4 + i];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) b[j] = ws[k][tx * 4 + j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int64_t tok = tok0 + ty * 4 + i;
+        if (tok >= T) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int e = e0 + tx * 4 + j;
+            if (e < n) logits[tok * n + e] = acc[i][j];
+        }
+    }
+}
+
+// One warp per token: lane l holds logits l, l+32, ... (up to 8 per lane).
+__global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ logits,
+                                                          int64_t T, int n, int K,
+                                                          int32_t* __restrict__ topk_idx,
+                                                          float* __restrict__ topk_w) {
+    const int lane = threadIdx.x & 31;
+    const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    if (t >= T) return;
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = (e < n) ? logits[t * n + e] : 0.f;
+        if (v[i] != v[i]) v[i] = -INFINITY;  // NaN ranks lowest: keeps the order total
+    }
+    uint32_t taken = 0;  // bit i: slot i of this lane already chosen
+    float m = 0.f, s = 0.f;
+    for (int k = 0; k < K; ++k) {
+        // best candidate of this lane (strict '>' scanning upwards: lowest index on ties)
+        int bi = -1;
+        float bv = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane + 32 * i;
+            if (e < n && !((taken >> i) & 1u) && (bi < 0 || v[i] > bv)) {
+                bi = e;
+                bv = v[i];
+            }
+        }
+        // warp argmax: larger value wins, equal values -> lower index; a lane
+        // without candidates (bi < 0) never wins.
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            const bool take = (oi >= 0) && (bi < 0 || ov > bv || (ov == bv && oi < bi));
+            if (take) {
+                bv = ov;
+                bi = oi;
+            }
+        }
+        if ((bi & 31) == lane && bi >= 0) taken |= 1u << (bi >> 5);
+        if (k == 0) m = bv;
+        const float ex = expf(bv - m);
+        s += ex;
+        if (lane == 0) {
+            topk_idx[t * K + k] = bi;
+            topk_w[t * K + k] = ex;
+        }
+    }
+    if (lane == 0) {
+        const float inv = 1.f / s;
+        for (int k = 0; k < K; ++k) topk_w[t * K + k] *= inv;
+    }
+}
+
+template <typename XT>
+static cudaError_t launch_router_t(const XT* x, const float* Wg, int64_t T, int d, int n, int K,
+                                   int32_t* idx, float* w, float* logits_ws, int num_sms,
+                                   cudaStream_t st) {
+    if (n <= 32) {
+        // Few tokens: one token per warp for parallelism; many tokens: share
+        // each W_g row between several tokens.
+        const bool many = T >= static_cast<int64_t>(num_sms) * 8 * 8;
+        const int64_t warps_needed = many ? (T + 3) / 4 : T;
+        const int64_t blocks = (warps_needed + 7) / 8;
+        dim3 grid(static_cast<unsigned>(blocks)), block(256);
+        if (n <= 8) {
+            if (many)
+                router_small_kernel<XT, 8, 4><<<grid, block, 0, st>>>(x, Wg, T, d, n, K, idx, w);
+            else
+                router_small_kernel<XT, 8, 1><<<grid, block, 0, st>>>(x, Wg, T, d, n, K, idx, w);
+        } else if (n <= 16) {
+            if (many)
+                router_small_kernel<XT, 16, 2><<<dim3(static_cast<unsigned>(((T + 1) / 2 + 7) / 8)), block, 0, st>>>(
+                    x, Wg, T, d, n, K, idx, w);
+            else
+                router_small_kernel<XT, 16, 1><<<grid, block, 0, st>>>(x, Wg, T, d, n, K, idx, w);
+        } else {
+            router_small_kernel<XT, 32, 1><<<dim3(static_cast<unsigned>((T + 7) / 8)), block, 0, st>>>(
+                x, Wg, T, d, n, K, idx, w);
+        }
+        return cudaGetLastError();
+    }
+    dim3 g1(static_cast<unsigned>((T + kRT - 1) / kRT), static_cast<unsigned>((n + kRE - 1) / kRE));
+    router_logits_kernel<XT><<<g1, 256, 0, st>>>(x, Wg, T, d, n, logits_ws);
+    router_topk_kernel<<<dim3(static_cast<unsigned>((T + 7) / 8)), 256, 0, st>>>(logits_ws, T, n, K,
+                                                                                 idx, w);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_router(const void* x, bool x_bf16, const float* Wg, int64_t T, int d, int n,
+                          int K, int32_t* topk_idx, float* topk_w, float* logits_ws, int num_sms,
+                          cudaStream_t st) {
+    if (x_bf16)
+        return launch_router_t<uint16_t>(static_cast<const uint16_t*>(x), Wg, T, d, n, K, topk_idx,
+                                         topk_w, logits_ws, num_sms, st);
+    return launch_router_t<float>(static_cast<const float*>(x), Wg, T, d, n, K, topk_idx, topk_w,
+                                  logits_ws, num_sms, st);
+}
+
+}  // namespace moe

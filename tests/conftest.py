@@ -8,3 +8,13 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
+
+
+def build_library():
+    """Build libmoe_b200.so (if stale) without importing the package first."""
+    import importlib.util
+    path = os.path.join(ROOT, "sparse_mixture_experts_24_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_moe_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
