@@ -110,6 +110,29 @@ def recorded_traffic(kernel, config):
 
 
 # --------------------------------------------------------------------------
+# replicas: each rank runs the whole workload on its own GPU and its own batch
+# --------------------------------------------------------------------------
+
+def replica_seed(rank: int) -> int:
+    return rank
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """Max of a per-rank timing over all ranks (identity without a process group)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def tokens_per_s(T: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processed T tokens per step."""
+    return T * world / (ms_per_step * 1e-3)
+
+
+# --------------------------------------------------------------------------
 # clocks sampled during the timed region (NVML)
 # --------------------------------------------------------------------------
 
@@ -264,7 +287,7 @@ def main():
     dev = torch.device("cuda", local_rank if world > 1 else 0)
     torch.cuda.set_device(dev)
 
-    L = mi.make_layer(cfg, seed=rank)     # each replica gets its own seeded batch
+    L = mi.make_layer(cfg, seed=replica_seed(rank))  # each replica gets its own seeded batch
     tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
 
     def to_dev(a):
@@ -312,11 +335,8 @@ def main():
         dist.barrier()
     ms = ev0.elapsed_time(ev1) / args.steps
     layer.sync_status(stream)
-    if dist:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
-    value = T * world / (ms * 1e-3)
+    ms = max_over_ranks(ms, dist, dev)
+    value = tokens_per_s(T, world, ms)
 
     # ---- end to end: pinned host activations in, y / routing out ----
     xh = x.cpu().pin_memory()
@@ -345,12 +365,8 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    ems = e0.elapsed_time(e1) / args.steps
-    if dist:
-        tt = torch.tensor([ems], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ems = float(tt.item())
-    e2e_value = T * world / (ems * 1e-3)
+    ems = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, dev)
+    e2e_value = tokens_per_s(T, world, ems)
     h2d = x.numel() * x.element_size()
     d2h = y.numel() * y.element_size() + idx.numel() * 4 + gw.numel() * 4
 
