@@ -185,6 +185,31 @@ MOE_API moe_status moe_sync_status(moe_handle *h, moe_stream_t stream);
 MOE_API moe_status moe_trace_begin(moe_handle *h, int max_calls);
 MOE_API moe_status moe_trace_end(moe_handle *h, double *stage_ms, int n_stages, int *calls);
 
+/*
+ * Dispatch for callers that cannot allocate device memory.  The pages have no
+ * counterpart: this is an interface convenience of this library.
+ *
+ * Same outputs as moe_dispatch (counts[n], offsets[n+1], row_token[T*K],
+ * token_row[T][K], all caller-owned device int32, all required here), but no
+ * handle and no cudaMalloc / cudaFree: the scratch lives in a fixed device
+ * array inside the library (about 0.5 MB, held on every GPU that loads the
+ * library until the process exits).  Meant for callers whose device memory
+ * comes from a framework allocator or a fixed memory plan, and for callers
+ * that cannot take cudaMalloc's implicit device-wide synchronisation.
+ *   Limit: T * K <= 65,536 pairs, n <= 256; larger sizes return
+ *   MOE_ERR_INVALID_ARG with a message naming the limit.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   Every call shares the array and it keeps the last call's contents (each
+ *   call overwrites what it reads).  Calls that overlap on the GPU race on
+ *   it: order them on one stream.
+ *   Errors: MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA.
+ */
+MOE_API moe_status moe_dispatch_noalloc(int64_t T, int n, int K, const int32_t *topk_idx,
+                                        int32_t *counts, int32_t *offsets, int32_t *row_token,
+                                        int32_t *token_row, moe_stream_t stream);
+
 /* Free the workspace and the handle.  NULL is allowed. */
 MOE_API moe_status moe_destroy(moe_handle *h);
 

@@ -54,17 +54,19 @@ lib.moe_workspace_view.argtypes = [_vp, ctypes.c_char_p, ctypes.POINTER(_vp), ct
 lib.moe_sync_status.argtypes = [_vp, _vp]
 lib.moe_destroy.argtypes = [_vp]
 lib.moe_trace_begin.argtypes = [_vp, _int]
+lib.moe_dispatch_noalloc.argtypes = [_i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.moe_trace_end.argtypes = [_vp, ctypes.POINTER(ctypes.c_double), _int, ctypes.POINTER(_int)]
 lib.moe_last_error.restype = ctypes.c_char_p
 lib.moe_version.restype = ctypes.c_char_p
 for _f in ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
            "moe_forward_with_routing", "moe_workspace_view", "moe_sync_status", "moe_destroy",
-           "moe_trace_begin", "moe_trace_end"):
+           "moe_trace_begin", "moe_trace_end", "moe_dispatch_noalloc"):
     getattr(lib, _f).restype = _int
 
 EXPORTED = ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
             "moe_forward_with_routing", "moe_workspace_view", "moe_sync_status", "moe_destroy",
-            "moe_last_error", "moe_version", "moe_trace_begin", "moe_trace_end")
+            "moe_last_error", "moe_version", "moe_trace_begin", "moe_trace_end",
+            "moe_dispatch_noalloc")
 
 TRACE_STAGES = ("router", "dispatch", "gather", "gemm1", "gemm2", "combine")
 
@@ -146,6 +148,15 @@ def moe_workspace_view(h, name: str):
 
 def moe_sync_status(h, stream=None) -> None:
     _check(lib.moe_sync_status(h, _stream(stream)), "moe_sync_status")
+
+
+def moe_dispatch_noalloc(T, n, K, topk_idx, counts, offsets, row_token, token_row,
+                         stream=None) -> None:
+    """Dispatch without a handle and without allocating device memory (scratch
+    in a fixed array inside the library; T * K <= 65,536)."""
+    _check(lib.moe_dispatch_noalloc(T, n, K, _ptr(topk_idx), _ptr(counts), _ptr(offsets),
+                                    _ptr(row_token), _ptr(token_row), _stream(stream)),
+           "moe_dispatch_noalloc")
 
 
 def moe_trace_begin(h, max_calls: int) -> None:

@@ -31,6 +31,15 @@ moe_status ok() {
     return MOE_OK;
 }
 
+}  // namespace
+
+namespace moe_api_detail {
+// Lets other translation units of the library set the moe_last_error() text.
+void set_last_error(const char* msg) { snprintf(g_err, sizeof g_err, "%s", msg); }
+}  // namespace moe_api_detail
+
+namespace {
+
 moe_status cuda_fail(cudaError_t e, const char* what) {
     return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
