@@ -9,10 +9,12 @@
 // dropped logits are -inf, so the softmax runs over the kept ones only).
 //
 // Two kernels:
-//   router_small_kernel  n <= 32: one warp per group of TPW tokens; the lanes
-//                        split d in 16-byte vectors, every lane keeps all n
-//                        partial logits of its tokens in registers, a shuffle
-//                        butterfly sums them, lane 0 picks the top K.
+//   router_small_kernel  n <= 32: W_g staged through shared memory transposed
+//                        to [expert][row]; one warp per group of TPW tokens,
+//                        the lanes split d four rows at a time, every lane
+//                        keeps all n partial logits of its tokens in
+//                        registers, a shuffle butterfly sums them, lane 0
+//                        picks the top K.
 //   router_logits_kernel + router_topk_kernel  n > 32: a 64x64 register-tiled
 //                        fp32 GEMM writes the logits to the workspace, then a
 //                        warp per token selects the top K with shuffles.
@@ -21,32 +23,25 @@
 
 namespace moe {
 
+// 4 consecutive x elements widened to fp32 (8 bytes of bf16, 16 of fp32).
 template <typename XT>
-struct XVec;  // 16-byte vector of x elements widened to fp32
+__device__ __forceinline__ void load_x4(const XT* p, float (&v)[4]);
 
 template <>
-struct XVec<uint16_t> {
-    static constexpr int kElems = 8;
-    __device__ __forceinline__ static void load(const uint16_t* p, float (&v)[8]) {
-        uint4 q = __ldg(reinterpret_cast<const uint4*>(p));
-        unpack_bf16x2(q.x, v[0], v[1]);
-        unpack_bf16x2(q.y, v[2], v[3]);
-        unpack_bf16x2(q.z, v[4], v[5]);
-        unpack_bf16x2(q.w, v[6], v[7]);
-    }
-};
+__device__ __forceinline__ void load_x4<uint16_t>(const uint16_t* p, float (&v)[4]) {
+    const uint2 q = __ldg(reinterpret_cast<const uint2*>(p));
+    unpack_bf16x2(q.x, v[0], v[1]);
+    unpack_bf16x2(q.y, v[2], v[3]);
+}
 
 template <>
-struct XVec<float> {
-    static constexpr int kElems = 4;
-    __device__ __forceinline__ static void load(const float* p, float (&v)[4]) {
-        float4 q = __ldg(reinterpret_cast<const float4*>(p));
-        v[0] = q.x;
-        v[1] = q.y;
-        v[2] = q.z;
-        v[3] = q.w;
-    }
-};
+__device__ __forceinline__ void load_x4<float>(const float* p, float (&v)[4]) {
+    const float4 q = __ldg(reinterpret_cast<const float4*>(p));
+    v[0] = q.x;
+    v[1] = q.y;
+    v[2] = q.z;
+    v[3] = q.w;
+}
 
 // Top-K of one token's logits held in registers (NE slots, n valid), written
 // with the softmax over the kept logits.  Strict '>' while scanning upwards
@@ -79,17 +74,30 @@ __device__ __forceinline__ void topk_softmax_regs(const float (&L)[NE], int n, i
     for (int k = 0; k < K; ++k) w_out[k] *= inv;
 }
 
+// Rows of W_g staged per pass: NE x (chunk + 4) floats stay under 48 KB.
+template <int NE>
+struct SmallRouterCfg {
+    static constexpr int kChunk = NE <= 8 ? 1024 : (NE <= 16 ? 512 : 256);
+    static constexpr int kPitch = kChunk + 4;  // floats per staged expert row
+};
+
+// n <= 32.  Each warp owns TPW tokens; W_g is staged through shared memory in
+// chunks of kChunk rows, transposed to [expert][row], so that a warp reads 32
+// consecutive float4 (512 contiguous bytes) per expert: lane l covers rows
+// 4l .. 4l+3 of every 128-row slice of the chunk and the matching 4 columns
+// of x (8 or 16 contiguous bytes per token).  Shuffles sum the lanes; lane 0
+// selects the top K.
 template <typename XT, int NE, int TPW>
 __global__ void __launch_bounds__(256) router_small_kernel(const XT* __restrict__ x,
                                                            const float* __restrict__ Wg, int64_t T,
                                                            int d, int n, int K,
                                                            int32_t* __restrict__ topk_idx,
                                                            float* __restrict__ topk_w) {
-    constexpr int VE = XVec<XT>::kElems;
+    using C = SmallRouterCfg<NE>;
+    __shared__ __align__(16) float Ws[NE * C::kPitch];
     const int lane = threadIdx.x & 31;
-    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const int64_t t0 = warp * TPW;
-    if (t0 >= T) return;
+    const int warp = threadIdx.x >> 5;
+    const int64_t t0 = (static_cast<int64_t>(blockIdx.x) * 8 + warp) * TPW;
 
     float acc[TPW][NE];
 #pragma unroll
@@ -97,32 +105,44 @@ __global__ void __launch_bounds__(256) router_small_kernel(const XT* __restrict_
 #pragma unroll
         for (int e = 0; e < NE; ++e) acc[t][e] = 0.f;
 
-    const int nvec = d / VE;
-    for (int v = lane; v < nvec; v += 32) {
-        float xv[TPW][VE];
-#pragma unroll
-        for (int t = 0; t < TPW; ++t) {
-            if (t0 + t < T) {
-                XVec<XT>::load(x + (t0 + t) * static_cast<int64_t>(d) + static_cast<int64_t>(v) * VE,
-                               xv[t]);
-            } else {
-#pragma unroll
-                for (int u = 0; u < VE; ++u) xv[t][u] = 0.f;
-            }
+    for (int c0 = 0; c0 < d; c0 += C::kChunk) {
+        const int rows = min(C::kChunk, d - c0);   // multiple of 64
+        __syncthreads();
+        for (int i = threadIdx.x; i < rows * n; i += 256) {
+            const int j = i / n, e = i - j * n;
+            Ws[e * C::kPitch + j] = __ldg(Wg + static_cast<int64_t>(c0 + j) * n + e);
         }
+        __syncthreads();
+        if (t0 >= T) continue;
+        for (int j = lane * 4; j < rows; j += 128) {
+            float xv[TPW][4];
 #pragma unroll
-        for (int u = 0; u < VE; ++u) {
-            const float* wrow = Wg + static_cast<int64_t>(v * VE + u) * n;
+            for (int t = 0; t < TPW; ++t) {
+                if (t0 + t < T) {
+                    load_x4<XT>(x + (t0 + t) * static_cast<int64_t>(d) + c0 + j, xv[t]);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) xv[t][u] = 0.f;
+                }
+            }
 #pragma unroll
             for (int e = 0; e < NE; ++e) {
                 if (e < n) {
-                    const float w = __ldg(wrow + e);
+                    const float4 w = *reinterpret_cast<const float4*>(&Ws[e * C::kPitch + j]);
 #pragma unroll
-                    for (int t = 0; t < TPW; ++t) acc[t][e] = fmaf(xv[t][u], w, acc[t][e]);
+                    for (int t = 0; t < TPW; ++t) {
+                        float a = acc[t][e];
+                        a = fmaf(xv[t][0], w.x, a);
+                        a = fmaf(xv[t][1], w.y, a);
+                        a = fmaf(xv[t][2], w.z, a);
+                        a = fmaf(xv[t][3], w.w, a);
+                        acc[t][e] = a;
+                    }
                 }
             }
         }
     }
+    if (t0 >= T) return;
 #pragma unroll
     for (int t = 0; t < TPW; ++t)
 #pragma unroll
@@ -265,32 +285,38 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
     }
 }
 
+template <typename XT, int NE>
+static void launch_small(const XT* x, const float* Wg, int64_t T, int d, int n, int K, int32_t* idx,
+                         float* w, int num_sms, cudaStream_t st) {
+    // Several tokens per warp share each staged W_g chunk when there are
+    // enough tokens to fill the GPU; otherwise one token per warp.
+    constexpr int kTpwMany = NE <= 8 ? 4 : (NE <= 16 ? 2 : 1);
+    const bool many = T >= static_cast<int64_t>(num_sms) * 8 * kTpwMany;
+    if (many && kTpwMany > 1) {
+        const int64_t blocks = (T + 8 * kTpwMany - 1) / (8 * kTpwMany);
+        router_small_kernel<XT, NE, kTpwMany><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+            x, Wg, T, d, n, K, idx, w);
+    } else {
+        const int64_t blocks = (T + 7) / 8;
+        router_small_kernel<XT, NE, 1><<<static_cast<unsigned>(blocks), 256, 0, st>>>(x, Wg, T, d, n,
+                                                                                     K, idx, w);
+    }
+}
+
 template <typename XT>
 static cudaError_t launch_router_t(const XT* x, const float* Wg, int64_t T, int d, int n, int K,
                                    int32_t* idx, float* w, float* logits_ws, int num_sms,
                                    cudaStream_t st) {
+    if (n <= 8) {
+        launch_small<XT, 8>(x, Wg, T, d, n, K, idx, w, num_sms, st);
+        return cudaGetLastError();
+    }
+    if (n <= 16) {
+        launch_small<XT, 16>(x, Wg, T, d, n, K, idx, w, num_sms, st);
+        return cudaGetLastError();
+    }
     if (n <= 32) {
-        // Few tokens: one token per warp for parallelism; many tokens: share
-        // each W_g row between several tokens.
-        const bool many = T >= static_cast<int64_t>(num_sms) * 8 * 8;
-        const int64_t warps_needed = many ? (T + 3) / 4 : T;
-        const int64_t blocks = (warps_needed + 7) / 8;
-        dim3 grid(static_cast<unsigned>(blocks)), block(256);
-        if (n <= 8) {
-            if (many)
-                router_small_kernel<XT, 8, 4><<<grid, block, 0, st>>>(x, Wg, T, d, n, K, idx, w);
-            else
-                router_small_kernel<XT, 8, 1><<<grid, block, 0, st>>>(x, Wg, T, d, n, K, idx, w);
-        } else if (n <= 16) {
-            if (many)
-                router_small_kernel<XT, 16, 2><<<dim3(static_cast<unsigned>(((T + 1) / 2 + 7) / 8)), block, 0, st>>>(
-                    x, Wg, T, d, n, K, idx, w);
-            else
-                router_small_kernel<XT, 16, 1><<<grid, block, 0, st>>>(x, Wg, T, d, n, K, idx, w);
-        } else {
-            router_small_kernel<XT, 32, 1><<<dim3(static_cast<unsigned>((T + 7) / 8)), block, 0, st>>>(
-                x, Wg, T, d, n, K, idx, w);
-        }
+        launch_small<XT, 32>(x, Wg, T, d, n, K, idx, w, num_sms, st);
         return cudaGetLastError();
     }
     dim3 g1(static_cast<unsigned>((T + kRT - 1) / kRT), static_cast<unsigned>((n + kRE - 1) / kRE));

@@ -18,3 +18,13 @@ def build_library():
     mod = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(mod)
     return mod.build()
+
+
+import pytest  # noqa: E402
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _library_built():
+    """Every test session starts with an up-to-date libmoe_b200.so."""
+    build_library()
+    yield
