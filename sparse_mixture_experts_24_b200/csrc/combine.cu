@@ -7,8 +7,9 @@
 // the products are added), and the sum over experts in the layer equation of
 // "Mixtral of Experts" section 2.1.
 //
-// One warp per token, 16-byte loads and stores: the kernel reads K rows of O
-// and writes one row of y, so it runs at HBM speed.
+// One thread per 16-byte vector of y (grid-stride): it reads the K matching
+// vectors of O and writes one vector of y, so every load of a small batch is
+// in flight at once and large batches stream at HBM speed.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -19,40 +20,40 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const uint4* __restri
                                                            const float* __restrict__ topk_w,
                                                            int64_t T, int K, int vec_per_row,
                                                            uint4* __restrict__ y) {
-    const int lane = threadIdx.x & 31;
-    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    for (int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; t < T;
-         t += nwarps) {
-        for (int v = lane; v < vec_per_row; v += 32) {
-            float acc[8];
+    const int64_t total = T * vec_per_row;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += stride) {
+        const int64_t t = i / vec_per_row;
+        const int64_t v = i - t * vec_per_row;
+        float acc[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-            for (int k = 0; k < K; ++k) {
-                const int32_t r = token_row[t * K + k];
-                if (r < 0) continue;
-                const float g = topk_w[t * K + k];
-                const uint4 q = __ldg(O + static_cast<int64_t>(r) * vec_per_row + v);
-                float a, b;
-                unpack_bf16x2(q.x, a, b);
-                acc[0] = fmaf(g, a, acc[0]);
-                acc[1] = fmaf(g, b, acc[1]);
-                unpack_bf16x2(q.y, a, b);
-                acc[2] = fmaf(g, a, acc[2]);
-                acc[3] = fmaf(g, b, acc[3]);
-                unpack_bf16x2(q.z, a, b);
-                acc[4] = fmaf(g, a, acc[4]);
-                acc[5] = fmaf(g, b, acc[5]);
-                unpack_bf16x2(q.w, a, b);
-                acc[6] = fmaf(g, a, acc[6]);
-                acc[7] = fmaf(g, b, acc[7]);
-            }
-            uint4 out;
-            out.x = pack_bf16x2(acc[0], acc[1]);
-            out.y = pack_bf16x2(acc[2], acc[3]);
-            out.z = pack_bf16x2(acc[4], acc[5]);
-            out.w = pack_bf16x2(acc[6], acc[7]);
-            y[t * vec_per_row + v] = out;
+        for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+        for (int k = 0; k < K; ++k) {
+            const int32_t r = __ldg(token_row + t * K + k);
+            if (r < 0) continue;
+            const float g = __ldg(topk_w + t * K + k);
+            const uint4 q = __ldg(O + static_cast<int64_t>(r) * vec_per_row + v);
+            float a, b;
+            unpack_bf16x2(q.x, a, b);
+            acc[0] = fmaf(g, a, acc[0]);
+            acc[1] = fmaf(g, b, acc[1]);
+            unpack_bf16x2(q.y, a, b);
+            acc[2] = fmaf(g, a, acc[2]);
+            acc[3] = fmaf(g, b, acc[3]);
+            unpack_bf16x2(q.z, a, b);
+            acc[4] = fmaf(g, a, acc[4]);
+            acc[5] = fmaf(g, b, acc[5]);
+            unpack_bf16x2(q.w, a, b);
+            acc[6] = fmaf(g, a, acc[6]);
+            acc[7] = fmaf(g, b, acc[7]);
         }
+        uint4 out;
+        out.x = pack_bf16x2(acc[0], acc[1]);
+        out.y = pack_bf16x2(acc[2], acc[3]);
+        out.z = pack_bf16x2(acc[4], acc[5]);
+        out.w = pack_bf16x2(acc[6], acc[7]);
+        y[i] = out;
     }
 }
 
@@ -61,30 +62,31 @@ __global__ void __launch_bounds__(256) combine_f32_kernel(const float4* __restri
                                                           const float* __restrict__ topk_w,
                                                           int64_t T, int K, int vec_per_row,
                                                           float4* __restrict__ y) {
-    const int lane = threadIdx.x & 31;
-    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    for (int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; t < T;
-         t += nwarps) {
-        for (int v = lane; v < vec_per_row; v += 32) {
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int k = 0; k < K; ++k) {
-                const int32_t r = token_row[t * K + k];
-                if (r < 0) continue;
-                const float g = topk_w[t * K + k];
-                const float4 q = __ldg(O + static_cast<int64_t>(r) * vec_per_row + v);
-                acc.x = fmaf(g, q.x, acc.x);
-                acc.y = fmaf(g, q.y, acc.y);
-                acc.z = fmaf(g, q.z, acc.z);
-                acc.w = fmaf(g, q.w, acc.w);
-            }
-            y[t * vec_per_row + v] = acc;
+    const int64_t total = T * vec_per_row;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += stride) {
+        const int64_t t = i / vec_per_row;
+        const int64_t v = i - t * vec_per_row;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k = 0; k < K; ++k) {
+            const int32_t r = __ldg(token_row + t * K + k);
+            if (r < 0) continue;
+            const float g = __ldg(topk_w + t * K + k);
+            const float4 q = __ldg(O + static_cast<int64_t>(r) * vec_per_row + v);
+            acc.x = fmaf(g, q.x, acc.x);
+            acc.y = fmaf(g, q.y, acc.y);
+            acc.z = fmaf(g, q.z, acc.z);
+            acc.w = fmaf(g, q.w, acc.w);
         }
+        y[i] = acc;
     }
 }
 
 cudaError_t launch_combine(const void* O, bool bf16, const int32_t* token_row, const float* topk_w,
                            int64_t T, int K, int d, void* y, int num_sms, cudaStream_t st) {
-    int64_t blocks = (T + 7) / 8;
+    const int64_t vecs = T * (bf16 ? d / 8 : d / 4);
+    int64_t blocks = (vecs + 255) / 256;
     const int64_t cap = static_cast<int64_t>(num_sms) * 16;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;

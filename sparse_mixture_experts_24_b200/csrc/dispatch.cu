@@ -17,7 +17,7 @@
 //                  block's base inside each segment, and the M-block prefix
 //                  the grouped GEMMs schedule from;
 //   scatter_kernel row of every pair -> row_token, token_row;
-//   gather_kernel  Xp[r] = x[row_token[r]] with 16-byte vectors, a warp per row.
+//   gather_kernel  Xp[r] = x[row_token[r]], one thread per 16-byte vector.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -151,22 +151,21 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ x
                                                      const int32_t* __restrict__ row_token,
                                                      int64_t R, int64_t T, int64_t vec_per_row,
                                                      uint4* __restrict__ xp) {
-    const int lane = threadIdx.x & 31;
-    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < R;
-         r += nwarps) {
-        const int64_t t = row_token[r];
+    const int64_t total = R * vec_per_row;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += stride) {
+        const int64_t r = i / vec_per_row;
+        const int64_t v = i - r * vec_per_row;
+        const int64_t t = __ldg(row_token + r);
         if (t < 0 || t >= T) continue;  // a row no valid pair reached (bad expert ids)
-        const uint4* src = x + t * vec_per_row;
-        uint4* dst = xp + r * vec_per_row;
-        for (int64_t v = lane; v < vec_per_row; v += 32) dst[v] = __ldg(src + v);
+        xp[i] = __ldg(x + t * vec_per_row + v);
     }
 }
 
 cudaError_t launch_gather(const void* x, const int32_t* row_token, int64_t R, int64_t T,
                           int64_t row_bytes, void* xp, int num_sms, cudaStream_t st) {
-    const int64_t warps = R;
-    int64_t blocks = (warps + 7) / 8;
+    int64_t blocks = (R * (row_bytes / 16) + 255) / 256;
     const int64_t cap = static_cast<int64_t>(num_sms) * 16;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;

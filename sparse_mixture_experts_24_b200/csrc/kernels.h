@@ -18,6 +18,21 @@ cudaError_t launch_router(const void* x, bool x_bf16, const float* Wg, int64_t T
                           int K, int32_t* topk_idx, float* topk_w, float* logits_ws, int num_sms,
                           cudaStream_t st);
 
+// Top-K + softmax of logits [T][n] already in memory (warp per token).
+cudaError_t launch_router_topk(const float* logits, int64_t T, int n, int K, int32_t* topk_idx,
+                               float* topk_w, cudaStream_t st);
+
+// Tensor-core router for bf16 x: splits W_g into three bf16 parts
+// (parts [3][npad][d], npad = n rounded up to 16), computes the logits
+// [T][n] with tcgen05 (tm_x over x [T][d], tm_w over parts [3*npad][d], both
+// with 64 x rows boxes: 128 rows for x, npad rows for the parts), then the
+// top-K and softmax.
+cudaError_t launch_router_tc(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const float* Wg,
+                             uint16_t* parts, int64_t T, int d, int n, int K, float* logits,
+                             int32_t* topk_idx, float* topk_w, int* status, int num_sms,
+                             cudaStream_t st);
+int router_tc_smem_bytes(int n);
+
 // Dispatch workspace (device, int32 unless noted).
 struct DispatchBufs {
     int32_t* blockcounts;  // [nblk][n]: per-block counts, then per-block segment bases

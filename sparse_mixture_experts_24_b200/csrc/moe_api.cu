@@ -68,13 +68,14 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// bf16 row-major [rows][cols] operand read in 128 (rows) x 64 (cols) boxes.
-bool encode_rows(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows) {
+// bf16 row-major [rows][cols] operand read in box_rows x 64 (cols) boxes.
+bool encode_rows(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
+                 uint32_t box_rows = 128) {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64, 128};
+    cuuint32_t box[2] = {64, box_rows};
     cuuint32_t es[2] = {1, 1};
     return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -114,6 +115,11 @@ struct moe_handle {
     const void* c_w1 = nullptr;
     const void* c_w3 = nullptr;
     const void* c_w2 = nullptr;
+    // tensor-core router: W_g split parts and the maps over x and the parts
+    uint16_t* wg_parts = nullptr;
+    CUtensorMap tm_rx, tm_parts;
+    const void* c_rx = nullptr;
+    int64_t c_rx_T = -1;
     // tracing: kTraceEvents events per traced call
     std::vector<cudaEvent_t> trace_ev;
     int trace_max = 0;
@@ -192,7 +198,10 @@ moe_status grow(moe_handle* h, int64_t T) {
     const size_t o_mblk = take(static_cast<size_t>(h->n + 1) * 4);
     const size_t o_row_token = take(static_cast<size_t>(R) * 4);
     const size_t o_token_row = take(static_cast<size_t>(R) * 4);
-    const size_t o_logits = take(h->n > 32 ? static_cast<size_t>(T) * h->n * 4 : 0);
+    const bool bf = h->dtype == MOE_BF16;
+    const int npad = (h->n + 15) / 16 * 16;
+    const size_t o_logits = take((bf || h->n > 32) ? static_cast<size_t>(T) * h->n * 4 : 0);
+    const size_t o_parts = take(bf ? static_cast<size_t>(3) * npad * h->d * 2 : 0);
     const size_t o_status = take(64);
     const size_t o_xp = take(static_cast<size_t>(R) * h->d * h->esize());
     const size_t o_h = take(static_cast<size_t>(R) * h->F * h->esize());
@@ -228,13 +237,17 @@ moe_status grow(moe_handle* h, int64_t T) {
     h->db.row_token = reinterpret_cast<int32_t*>(b + o_row_token);
     h->db.token_row = reinterpret_cast<int32_t*>(b + o_token_row);
     h->logits = reinterpret_cast<float*>(b + o_logits);
+    h->wg_parts = reinterpret_cast<uint16_t*>(b + o_parts);
+    h->c_rx = nullptr;
     h->status = reinterpret_cast<int*>(b + o_status);
     h->xp = b + o_xp;
     h->h = b + o_h;
     h->o = b + o_o;
     if (h->dtype == MOE_BF16) {
         if (!encode_rows(&h->tm_xp, h->xp, h->d, static_cast<uint64_t>(R)) ||
-            !encode_rows(&h->tm_h, h->h, h->F, static_cast<uint64_t>(R)))
+            !encode_rows(&h->tm_h, h->h, h->F, static_cast<uint64_t>(R)) ||
+            !encode_rows(&h->tm_parts, h->wg_parts, h->d, static_cast<uint64_t>(3 * npad),
+                         static_cast<uint32_t>(npad)))
             return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the workspace");
     }
     return MOE_OK;
@@ -259,6 +272,28 @@ moe_status prepare(moe_handle* h, int64_t T) {
     moe_status s = check_device(h);
     if (s != MOE_OK) return s;
     return grow(h, T);
+}
+
+// Router: the tensor-core path (bf16 x, enough tokens or many experts) or the
+// CUDA-core kernels.
+moe_status run_router(moe_handle* h, int64_t T, const void* x, const float* W_g, int32_t* topk_idx,
+                      float* topk_w, cudaStream_t st) {
+    cudaError_t e;
+    if (h->dtype == MOE_BF16 && (T >= 512 || h->n > 32)) {
+        if (x != h->c_rx || T != h->c_rx_T) {
+            if (!encode_rows(&h->tm_rx, x, h->d, static_cast<uint64_t>(T)))
+                return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for x");
+            h->c_rx = x;
+            h->c_rx_T = T;
+        }
+        e = moe::launch_router_tc(h->tm_rx, h->tm_parts, W_g, h->wg_parts, T, h->d, h->n, h->K,
+                                  h->logits, topk_idx, topk_w, h->status, h->num_sms, st);
+    } else {
+        e = moe::launch_router(x, h->dtype == MOE_BF16, W_g, T, h->d, h->n, h->K, topk_idx, topk_w,
+                               h->logits, h->num_sms, st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "router launch");
+    return MOE_OK;
 }
 
 moe_status run_experts(moe_handle* h, int64_t T, const void* x, const int32_t* topk_idx,
@@ -376,10 +411,8 @@ moe_status moe_route(moe_handle* h, int64_t T, const void* x, const float* W_g, 
     s = prepare(h, T);
     if (s != MOE_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = moe::launch_router(x, h->dtype == MOE_BF16, W_g, T, h->d, h->n, h->K, topk_idx,
-                                       topk_w, h->logits, h->num_sms, st);
-    if (e != cudaSuccess) return cuda_fail(e, "router launch");
-    return ok();
+    s = run_router(h, T, x, W_g, topk_idx, topk_w, st);
+    return s == MOE_OK ? ok() : s;
 }
 
 moe_status moe_forward(moe_handle* h, int64_t T, const void* x, const float* W_g, const void* w1,
@@ -400,9 +433,8 @@ moe_status moe_forward(moe_handle* h, int64_t T, const void* x, const float* W_g
     if (s != MOE_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     trace_mark(h, -1, st);
-    cudaError_t e = moe::launch_router(x, h->dtype == MOE_BF16, W_g, T, h->d, h->n, h->K, topk_idx,
-                                       topk_w, h->logits, h->num_sms, st);
-    if (e != cudaSuccess) return cuda_fail(e, "router launch");
+    s = run_router(h, T, x, W_g, topk_idx, topk_w, st);
+    if (s != MOE_OK) return s;
     trace_mark(h, 0, st);
     s = run_experts(h, T, x, topk_idx, topk_w, w1, w3, w2, y, st);
     return s == MOE_OK ? ok() : s;

@@ -8,7 +8,9 @@
 // kept scores); the layer equation of "Mixtral of Experts" section 2.1 (the
 // dropped logits are -inf, so the softmax runs over the kept ones only).
 //
-// Two kernels:
+// Kernels:
+//   router_token_kernel  n <= 32, T < 512: one block per token, W_g rows read
+//                        straight from global memory, block reduction.
 //   router_small_kernel  n <= 32: W_g staged through shared memory transposed
 //                        to [expert][row]; one warp per group of TPW tokens,
 //                        the lanes split d four rows at a time, every lane
@@ -74,6 +76,9 @@ __device__ __forceinline__ void topk_softmax_regs(const float (&L)[NE], int n, i
     for (int k = 0; k < K; ++k) w_out[k] *= inv;
 }
 
+// Below this many tokens the router runs one block per token.
+constexpr int64_t kTokenKernelMaxT = 512;
+
 // Rows of W_g staged per pass: NE x (chunk + 4) floats stay under 48 KB.
 template <int NE>
 struct SmallRouterCfg {
@@ -108,9 +113,25 @@ __global__ void __launch_bounds__(256) router_small_kernel(const XT* __restrict_
     for (int c0 = 0; c0 < d; c0 += C::kChunk) {
         const int rows = min(C::kChunk, d - c0);   // multiple of 64
         __syncthreads();
-        for (int i = threadIdx.x; i < rows * n; i += 256) {
-            const int j = i / n, e = i - j * n;
-            Ws[e * C::kPitch + j] = __ldg(Wg + static_cast<int64_t>(c0 + j) * n + e);
+        if ((n & 3) == 0) {
+            // float4 loads (4 experts of one row); rows * n is a multiple of 256 floats
+            const float4* src = reinterpret_cast<const float4*>(Wg + static_cast<int64_t>(c0) * n);
+            const int nv = rows * n / 4;
+#pragma unroll 4
+            for (int i = threadIdx.x; i < nv; i += 256) {
+                const float4 v = __ldg(src + i);
+                const int j = (i * 4) / n, e = (i * 4) - j * n;
+                float* dst = &Ws[e * C::kPitch + j];
+                dst[0] = v.x;
+                dst[C::kPitch] = v.y;
+                dst[2 * C::kPitch] = v.z;
+                dst[3 * C::kPitch] = v.w;
+            }
+        } else {
+            for (int i = threadIdx.x; i < rows * n; i += 256) {
+                const int j = i / n, e = i - j * n;
+                Ws[e * C::kPitch + j] = __ldg(Wg + static_cast<int64_t>(c0 + j) * n + e);
+            }
         }
         __syncthreads();
         if (t0 >= T) continue;
@@ -157,6 +178,68 @@ __global__ void __launch_bounds__(256) router_small_kernel(const XT* __restrict_
         for (int t = 0; t < TPW; ++t)
             if (t0 + t < T)
                 topk_softmax_regs<NE>(acc[t], n, K, topk_idx + (t0 + t) * K, topk_w + (t0 + t) * K);
+    }
+}
+
+// n <= 32, few tokens: one 256-thread block per token.  Thread i covers rows
+// 4i .. 4i+3 of every 1024-row slice of d, reading those rows of W_g straight
+// from global memory (4n contiguous floats per thread, contiguous across the
+// block); shuffles then shared memory sum the 256 partial logit vectors.
+template <typename XT, int NE>
+__global__ void __launch_bounds__(256) router_token_kernel(const XT* __restrict__ x,
+                                                           const float* __restrict__ Wg, int64_t T,
+                                                           int d, int n, int K,
+                                                           int32_t* __restrict__ topk_idx,
+                                                           float* __restrict__ topk_w) {
+    __shared__ float red[8][NE];
+    const int64_t t = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float acc[NE];
+#pragma unroll
+    for (int e = 0; e < NE; ++e) acc[e] = 0.f;
+    const XT* xr = x + t * static_cast<int64_t>(d);
+    for (int j = threadIdx.x * 4; j < d; j += 1024) {
+        float xv[4];
+        load_x4<XT>(xr + j, xv);
+        const float* w = Wg + static_cast<int64_t>(j) * n;
+        if (n == NE) {
+            // rows j .. j+3 are 4*NE contiguous floats
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int q = 0; q < NE / 4; ++q) {
+                    const float4 v = __ldg(reinterpret_cast<const float4*>(w + r * NE) + q);
+                    acc[4 * q + 0] = fmaf(xv[r], v.x, acc[4 * q + 0]);
+                    acc[4 * q + 1] = fmaf(xv[r], v.y, acc[4 * q + 1]);
+                    acc[4 * q + 2] = fmaf(xv[r], v.z, acc[4 * q + 2]);
+                    acc[4 * q + 3] = fmaf(xv[r], v.w, acc[4 * q + 3]);
+                }
+        } else {
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int e = 0; e < NE; ++e)
+                    if (e < n) acc[e] = fmaf(xv[r], __ldg(w + r * n + e), acc[e]);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < NE; ++e) {
+        float a = acc[e];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (lane == 0) red[warp][e] = a;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float L[NE];
+#pragma unroll
+        for (int e = 0; e < NE; ++e) {
+            float a = 0.f;
+#pragma unroll
+            for (int w8 = 0; w8 < 8; ++w8) a += red[w8][e];
+            L[e] = (a != a) ? -INFINITY : a;  // NaN ranks lowest
+        }
+        topk_softmax_regs<NE>(L, n, K, topk_idx + t * K, topk_w + t * K);
     }
 }
 
@@ -285,22 +368,37 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
     }
 }
 
+cudaError_t launch_router_topk(const float* logits, int64_t T, int n, int K, int32_t* topk_idx,
+                               float* topk_w, cudaStream_t st) {
+    router_topk_kernel<<<dim3(static_cast<unsigned>((T + 7) / 8)), 256, 0, st>>>(logits, T, n, K,
+                                                                                 topk_idx, topk_w);
+    return cudaGetLastError();
+}
+
 template <typename XT, int NE>
 static void launch_small(const XT* x, const float* Wg, int64_t T, int d, int n, int K, int32_t* idx,
                          float* w, int num_sms, cudaStream_t st) {
-    // Several tokens per warp share each staged W_g chunk when there are
-    // enough tokens to fill the GPU; otherwise one token per warp.
-    constexpr int kTpwMany = NE <= 8 ? 4 : (NE <= 16 ? 2 : 1);
-    const bool many = T >= static_cast<int64_t>(num_sms) * 8 * kTpwMany;
-    if (many && kTpwMany > 1) {
-        const int64_t blocks = (T + 8 * kTpwMany - 1) / (8 * kTpwMany);
-        router_small_kernel<XT, NE, kTpwMany><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-            x, Wg, T, d, n, K, idx, w);
-    } else {
-        const int64_t blocks = (T + 7) / 8;
-        router_small_kernel<XT, NE, 1><<<static_cast<unsigned>(blocks), 256, 0, st>>>(x, Wg, T, d, n,
-                                                                                     K, idx, w);
+    if (T < kTokenKernelMaxT) {
+        // few tokens: a whole block per token keeps every SM's loads in flight
+        router_token_kernel<XT, NE><<<static_cast<unsigned>(T), 256, 0, st>>>(x, Wg, T, d, n, K, idx, w);
+        return;
     }
+    // many tokens: share each staged W_g chunk between TPW tokens per warp,
+    // choosing TPW so that about two blocks land on every SM
+    constexpr int kTpwMax = NE <= 8 ? 4 : (NE <= 16 ? 2 : 1);
+    int tpw = 1;
+    if (kTpwMax >= 4 && T >= static_cast<int64_t>(num_sms) * 8 * 4)
+        tpw = 4;
+    else if (kTpwMax >= 2 && T >= static_cast<int64_t>(num_sms) * 8 * 2)
+        tpw = 2;
+    const int64_t blocks = (T + 8 * tpw - 1) / (8 * tpw);
+    const unsigned g = static_cast<unsigned>(blocks);
+    if (tpw == 4)
+        router_small_kernel<XT, NE, (kTpwMax >= 4 ? 4 : 1)><<<g, 256, 0, st>>>(x, Wg, T, d, n, K, idx, w);
+    else if (tpw == 2)
+        router_small_kernel<XT, NE, (kTpwMax >= 2 ? 2 : 1)><<<g, 256, 0, st>>>(x, Wg, T, d, n, K, idx, w);
+    else
+        router_small_kernel<XT, NE, 1><<<g, 256, 0, st>>>(x, Wg, T, d, n, K, idx, w);
 }
 
 template <typename XT>
