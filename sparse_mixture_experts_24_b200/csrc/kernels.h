@@ -88,4 +88,13 @@ cudaError_t launch_tc_gemm1(const CUtensorMap& tm_xp, const CUtensorMap& tm_w1,
 cudaError_t launch_tc_gemm2(const CUtensorMap& tm_h, const CUtensorMap& tm_w2, const TcGemmArgs& a,
                             int num_sms, cudaStream_t st);
 
+// The same GEMMs on CTA pairs (cta_group::2, 256-row tiles): mblk_base must
+// count 256-row blocks.
+constexpr int kTcPairBM = 256;
+cudaError_t launch_tc_gemm1_pair(const CUtensorMap& tm_xp, const CUtensorMap& tm_w1,
+                                 const CUtensorMap& tm_w3, const TcGemmArgs& a, int num_sms,
+                                 cudaStream_t st);
+cudaError_t launch_tc_gemm2_pair(const CUtensorMap& tm_h, const CUtensorMap& tm_w2, const TcGemmArgs& a,
+                                 int num_sms, cudaStream_t st);
+
 }  // namespace moe

@@ -7,6 +7,7 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -296,12 +297,25 @@ moe_status run_router(moe_handle* h, int64_t T, const void* x, const float* W_g,
     return MOE_OK;
 }
 
+// GEMM tiling: single-SM 128-row tiles (default) or CTA-pair 256-row tiles
+// (MOE_GEMM_PATH=pair).  On the Mixtral prefill shapes the pair tiles halve
+// the shared-memory operand traffic but measured no faster (tensor pipe ~80%
+// busy either way), so the single-SM kernel stays the default.
+bool use_pair_gemm(const moe_handle* h, int64_t T) {
+    (void)T;
+    if (h->dtype != MOE_BF16) return false;
+    const char* env = getenv("MOE_GEMM_PATH");
+    return env && strcmp(env, "pair") == 0;
+}
+
 moe_status run_experts(moe_handle* h, int64_t T, const void* x, const int32_t* topk_idx,
                        const float* topk_w, const void* w1, const void* w3, const void* w2, void* y,
                        cudaStream_t st) {
     const bool bf = h->dtype == MOE_BF16;
+    const bool pair = use_pair_gemm(h, T);
     const int64_t R = T * h->K;
-    cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n, bf ? moe::kTcBM : moe::kSimtBM,
+    cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n,
+                                         pair ? moe::kTcPairBM : (bf ? moe::kTcBM : moe::kSimtBM),
                                          h->db, st);
     if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
     trace_mark(h, 1, st);
@@ -335,7 +349,8 @@ moe_status run_experts(moe_handle* h, int64_t T, const void* x, const int32_t* t
         a1.out_cols = h->F;
         a1.out = h->h;
         a1.status = h->status;
-        e = moe::launch_tc_gemm1(h->tm_xp, h->tm_w1, h->tm_w3, a1, h->num_sms, st);
+        e = pair ? moe::launch_tc_gemm1_pair(h->tm_xp, h->tm_w1, h->tm_w3, a1, h->num_sms, st)
+                 : moe::launch_tc_gemm1(h->tm_xp, h->tm_w1, h->tm_w3, a1, h->num_sms, st);
         if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
         trace_mark(h, 3, st);
         moe::TcGemmArgs a2 = a1;
@@ -343,7 +358,8 @@ moe_status run_experts(moe_handle* h, int64_t T, const void* x, const int32_t* t
         a2.n_tiles = (h->d + 255) / 256;
         a2.out_cols = h->d;
         a2.out = h->o;
-        e = moe::launch_tc_gemm2(h->tm_h, h->tm_w2, a2, h->num_sms, st);
+        e = pair ? moe::launch_tc_gemm2_pair(h->tm_h, h->tm_w2, a2, h->num_sms, st)
+                 : moe::launch_tc_gemm2(h->tm_h, h->tm_w2, a2, h->num_sms, st);
         if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
         trace_mark(h, 4, st);
     } else {

@@ -67,6 +67,25 @@ def test_small_layer_matches_oracle(case):
     assert per_tok.max() <= 5 * TOL_Y[dt], per_tok.max()
 
 
+@pytest.mark.parametrize("path", ["single", "pair"])
+@pytest.mark.parametrize("case", [("pair_big_segments", 2048, 256, 512, 4, 2),
+                                  ("pair_ragged", 700, 192, 320, 2, 1),
+                                  ("pair_odd_blocks", 1333, 128, 384, 3, 2)], ids=lambda c: c[0])
+def test_gemm_paths_match_oracle(case, path, monkeypatch):
+    """Both GEMM tilings (single SM, CTA pair) against the oracle on cases with
+    large, ragged and odd-numbered 256-row segments."""
+    monkeypatch.setenv("MOE_GEMM_PATH", path)
+    name, T, d, F, n, K = case
+    cfg = mi.custom_config(name, T=T, d=d, ffn=F, n=n, K=K, dtype="bf16")
+    L = mi.make_layer(cfg, seed=zlib.crc32(name.encode()) % 1000)
+    y, idx, w = run_layer(cfg, L)
+    y_ref = oracle.forward_with_routing(L["x"], idx, w.astype(np.float64), L["w1"], L["w3"], L["w2"])
+    err = rel_l2(y_as_f64(y), y_ref)
+    assert err <= TOL_Y["bf16"], (name, path, err)
+    per_tok = np.linalg.norm(y_as_f64(y) - y_ref, axis=1) / np.maximum(np.linalg.norm(y_ref, axis=1), 1e-30)
+    assert per_tok.max() <= 5 * TOL_Y["bf16"], per_tok.max()
+
+
 def test_route_entry_point_matches_forward_routing():
     import sparse_mixture_experts_24_b200 as m
     cfg = mi.custom_config("route", T=257, d=256, ffn=128, n=8, K=2, dtype="bf16")

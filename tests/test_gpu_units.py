@@ -35,8 +35,12 @@ def read_ws(layer, name, rows, cols, torch_dtype):
     return t.view(torch.bfloat16) if torch_dtype == torch.bfloat16 else t
 
 
-@pytest.mark.parametrize("T,d,F,n,K", [(200, 128, 256, 4, 2), (333, 256, 384, 8, 2), (129, 320, 192, 3, 1)])
-def test_gemm1_and_gemm2_rows(T, d, F, n, K):
+@pytest.mark.parametrize("path", ["single", "pair"])
+@pytest.mark.parametrize("T,d,F,n,K", [(200, 128, 256, 4, 2), (333, 256, 384, 8, 2), (129, 320, 192, 3, 1),
+                                       (700, 192, 320, 2, 1), (1500, 256, 512, 3, 2)])
+def test_gemm1_and_gemm2_rows(T, d, F, n, K, path, monkeypatch):
+    """path: single-SM tiles (128 rows) or CTA-pair tiles (256 rows, cta_group::2)."""
+    monkeypatch.setenv("MOE_GEMM_PATH", path)
     import sparse_mixture_experts_24_b200 as m
     torch = require_cuda()
     cfg = mi.custom_config("units", T=T, d=d, ffn=F, n=n, K=K, dtype="bf16")
