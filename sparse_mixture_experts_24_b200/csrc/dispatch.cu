@@ -85,21 +85,39 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp) {
     return r;
 }
 
+// Per-block counts are walked in chunks staged through shared memory, so
+// the loads of a chunk are all in flight together; each expert's column is
+// then scanned in place.  blockcounts ends up holding, for every block and
+// expert, the block's first rank inside the expert's segment (the segment's
+// offset is added by the scatter).
+constexpr int kScanSmemInts = 8192;
+
 __global__ void __launch_bounds__(256) scan_kernel(int32_t* __restrict__ blockcounts, int nblk,
                                                    int n, int64_t R, int bm,
                                                    int32_t* __restrict__ counts,
                                                    int32_t* __restrict__ offsets,
                                                    int32_t* __restrict__ mblk_base) {
     __shared__ int s_warp[8];
+    __shared__ int32_t s_chunk[kScanSmemInts];
     const int e = threadIdx.x;
+    const int chunk_blocks = kScanSmemInts / n;
     int total = 0;
-    if (e < n) {
-        for (int b = 0; b < nblk; ++b) {
-            int32_t* c = blockcounts + static_cast<int64_t>(b) * n + e;
-            const int v = *c;
-            *c = total;  // exclusive within the expert
-            total += v;
+    for (int b0 = 0; b0 < nblk; b0 += chunk_blocks) {
+        const int nb = min(chunk_blocks, nblk - b0);
+        const int cnt = nb * n;
+        int32_t* g = blockcounts + static_cast<int64_t>(b0) * n;
+        __syncthreads();
+        for (int i = threadIdx.x; i < cnt; i += 256) s_chunk[i] = g[i];
+        __syncthreads();
+        if (e < n) {
+            for (int b = 0; b < nb; ++b) {
+                const int v = s_chunk[b * n + e];
+                s_chunk[b * n + e] = total;  // exclusive within the expert
+                total += v;
+            }
         }
+        __syncthreads();
+        for (int i = threadIdx.x; i < cnt; i += 256) g[i] = s_chunk[i];
     }
     const int off = block_exclusive_scan(e < n ? total : 0, s_warp);
     const int mb = (e < n) ? (total + bm - 1) / bm : 0;
@@ -108,7 +126,6 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* __restrict__ blockco
         counts[e] = total;
         offsets[e] = off;
         mblk_base[e] = mbase;
-        for (int b = 0; b < nblk; ++b) blockcounts[static_cast<int64_t>(b) * n + e] += off;
     }
     if (e == n - 1) {
         offsets[n] = off + total;
@@ -119,6 +136,7 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* __restrict__ blockco
 
 __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict__ idx, int64_t R,
                                                       int K, int n,
+                                                      const int32_t* __restrict__ offsets,
                                                       const int32_t* __restrict__ blockbase,
                                                       const int32_t* __restrict__ pair_rank,
                                                       int32_t* __restrict__ row_token,
@@ -131,7 +149,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
         token_row[p] = -1;
         return;
     }
-    const int dest = blockbase[(p / kPairsPerBlock) * n + e] + rk;
+    const int dest = offsets[e] + blockbase[(p / kPairsPerBlock) * n + e] + rk;
     row_token[dest] = static_cast<int32_t>(p / K);
     token_row[p] = dest;
 }
@@ -143,7 +161,7 @@ cudaError_t launch_dispatch(const int32_t* topk_idx, int64_t T, int K, int n, in
     rank_kernel<<<nblk, kPairsPerBlock, 0, st>>>(topk_idx, R, n, b.blockcounts, b.pair_rank);
     scan_kernel<<<1, 256, 0, st>>>(b.blockcounts, nblk, n, R, bm, b.counts, b.offsets, b.mblk_base);
     scatter_kernel<<<static_cast<unsigned>((R + 255) / 256), 256, 0, st>>>(
-        topk_idx, R, K, n, b.blockcounts, b.pair_rank, b.row_token, b.token_row);
+        topk_idx, R, K, n, b.offsets, b.blockcounts, b.pair_rank, b.row_token, b.token_row);
     return cudaGetLastError();
 }
 

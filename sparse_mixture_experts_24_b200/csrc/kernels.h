@@ -18,9 +18,14 @@ cudaError_t launch_router(const void* x, bool x_bf16, const float* Wg, int64_t T
                           int K, int32_t* topk_idx, float* topk_w, float* logits_ws, int num_sms,
                           cudaStream_t st);
 
-// Top-K + softmax of logits [T][n] already in memory (warp per token).
-cudaError_t launch_router_topk(const float* logits, int64_t T, int n, int K, int32_t* topk_idx,
-                               float* topk_w, cudaStream_t st);
+// Top-K + softmax of logits already in memory (warp per token): the logits
+// are the sum, in order, of `splits` partial arrays [splits][T][n].
+cudaError_t launch_router_topk(const float* logits, int splits, int64_t T, int n, int K,
+                               int32_t* topk_idx, float* topk_w, cudaStream_t st);
+
+// Largest number of K splits of the tensor-core router (workspace: logits
+// [kRouterMaxSplits][T][n]).
+constexpr int kRouterMaxSplits = 4;
 
 // Tensor-core router for bf16 x: splits W_g into three bf16 parts
 // (parts [3][npad][d], npad = n rounded up to 16), computes the logits
@@ -35,7 +40,7 @@ int router_tc_smem_bytes(int n);
 
 // Dispatch workspace (device, int32 unless noted).
 struct DispatchBufs {
-    int32_t* blockcounts;  // [nblk][n]: per-block counts, then per-block segment bases
+    int32_t* blockcounts;  // [nblk][n]: per-block counts, then each block's first rank in a segment
     int32_t* pair_rank;    // [R]: stable rank of each pair inside its block and expert
     int32_t* counts;       // [n]
     int32_t* offsets;      // [n+1]

@@ -201,7 +201,8 @@ moe_status grow(moe_handle* h, int64_t T) {
     const size_t o_token_row = take(static_cast<size_t>(R) * 4);
     const bool bf = h->dtype == MOE_BF16;
     const int npad = (h->n + 15) / 16 * 16;
-    const size_t o_logits = take((bf || h->n > 32) ? static_cast<size_t>(T) * h->n * 4 : 0);
+    const size_t o_logits =
+        take((bf || h->n > 32) ? static_cast<size_t>(moe::kRouterMaxSplits) * T * h->n * 4 : 0);
     const size_t o_parts = take(bf ? static_cast<size_t>(3) * npad * h->d * 2 : 0);
     const size_t o_status = take(64);
     const size_t o_xp = take(static_cast<size_t>(R) * h->d * h->esize());

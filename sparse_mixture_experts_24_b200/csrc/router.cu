@@ -312,9 +312,10 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const XT* __restrict
     }
 }
 
-// One warp per token: lane l holds logits l, l+32, ... (up to 8 per lane).
+// One warp per token: lane l holds logits l, l+32, ... (up to 8 per lane),
+// each the in-order sum of `splits` partial logits [splits][T][n].
 __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ logits,
-                                                          int64_t T, int n, int K,
+                                                          int splits, int64_t T, int n, int K,
                                                           int32_t* __restrict__ topk_idx,
                                                           float* __restrict__ topk_w) {
     const int lane = threadIdx.x & 31;
@@ -324,7 +325,10 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int e = lane + 32 * i;
-        v[i] = (e < n) ? logits[t * n + e] : 0.f;
+        float a = 0.f;
+        if (e < n)
+            for (int sp = 0; sp < splits; ++sp) a += logits[(static_cast<int64_t>(sp) * T + t) * n + e];
+        v[i] = a;
         if (v[i] != v[i]) v[i] = -INFINITY;  // NaN ranks lowest: keeps the order total
     }
     uint32_t taken = 0;  // bit i: slot i of this lane already chosen
@@ -368,10 +372,10 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
     }
 }
 
-cudaError_t launch_router_topk(const float* logits, int64_t T, int n, int K, int32_t* topk_idx,
-                               float* topk_w, cudaStream_t st) {
-    router_topk_kernel<<<dim3(static_cast<unsigned>((T + 7) / 8)), 256, 0, st>>>(logits, T, n, K,
-                                                                                 topk_idx, topk_w);
+cudaError_t launch_router_topk(const float* logits, int splits, int64_t T, int n, int K,
+                               int32_t* topk_idx, float* topk_w, cudaStream_t st) {
+    router_topk_kernel<<<dim3(static_cast<unsigned>((T + 7) / 8)), 256, 0, st>>>(logits, splits, T, n,
+                                                                                 K, topk_idx, topk_w);
     return cudaGetLastError();
 }
 
@@ -419,7 +423,7 @@ static cudaError_t launch_router_t(const XT* x, const float* Wg, int64_t T, int 
     }
     dim3 g1(static_cast<unsigned>((T + kRT - 1) / kRT), static_cast<unsigned>((n + kRE - 1) / kRE));
     router_logits_kernel<XT><<<g1, 256, 0, st>>>(x, Wg, T, d, n, logits_ws);
-    router_topk_kernel<<<dim3(static_cast<unsigned>((T + 7) / 8)), 256, 0, st>>>(logits_ws, T, n, K,
+    router_topk_kernel<<<dim3(static_cast<unsigned>((T + 7) / 8)), 256, 0, st>>>(logits_ws, 1, T, n, K,
                                                                                  idx, w);
     return cudaGetLastError();
 }

@@ -13,10 +13,13 @@
 // exact in fp32, and the three MMAs accumulate into one fp32 TMEM accumulator,
 // so the logits carry fp32-class rounding, not bf16's.
 //
-// router_tc_kernel: one CTA per 128 tokens; warp 0 streams x (128 x 64) and the
-// three W_g parts (Npad x 64 each) by TMA through a multi-stage ring; warp 1
-// issues tcgen05.mma M=128, N=Npad, K=16 three times per K step; warps 2-5 read
-// the 128 x Npad fp32 accumulator from TMEM and store the logits [T][n].
+// router_tc_kernel: one CTA per (128 tokens, slice of d): the d range is split
+// over gridDim.y CTAs so that small token counts still fill the GPU; warp 0
+// streams x (128 x 64) and the three W_g parts (Npad x 64 each) by TMA through
+// a multi-stage ring; warp 1 issues tcgen05.mma M=128, N=Npad, K=16 three
+// times per K step; warps 2-5 read the 128 x Npad fp32 accumulator from TMEM
+// and store the slice's partial logits [split][T][n], which the top-K kernel
+// sums in split order (deterministic).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -80,8 +83,12 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     const int stages = rt_stages(npad);
     RtTail* tail = reinterpret_cast<RtTail*>(smem + stages * stage_bytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int k_blocks = d / kRtBK;
+    const int kb_total = d / kRtBK;
+    const int kb_begin = static_cast<int>(static_cast<int64_t>(kb_total) * blockIdx.y / gridDim.y);
+    const int kb_end = static_cast<int>(static_cast<int64_t>(kb_total) * (blockIdx.y + 1) / gridDim.y);
+    const int k_blocks = kb_end - kb_begin;
     const int m0 = blockIdx.x * kRtBM;
+    logits += static_cast<int64_t>(blockIdx.y) * T * n;
     const int part_bytes = npad * kRtBK * 2;
 
     if (threadIdx.x == 0) {
@@ -120,10 +127,11 @@ __global__ void __launch_bounds__(kRtThreads, 1)
                 mbar_arrive_expect_tx(fb, static_cast<uint32_t>(stage_bytes));
                 armed[stage] = static_cast<int>(phase);
                 const uint32_t dst = smem_u32(smem + stage * stage_bytes);
-                tma_load_2d(dst, &tm_x, fb, kb * kRtBK, m0);
+                const int kx = (kb_begin + kb) * kRtBK;
+                tma_load_2d(dst, &tm_x, fb, kx, m0);
 #pragma unroll
                 for (int p = 0; p < 3; ++p)
-                    tma_load_2d(dst + kRtBM * kRtBK * 2 + p * part_bytes, &tm_w, fb, kb * kRtBK, p * npad);
+                    tma_load_2d(dst + kRtBM * kRtBK * 2 + p * part_bytes, &tm_w, fb, kx, p * npad);
                 if (++stage == stages) {
                     stage = 0;
                     phase ^= 1u;
@@ -213,11 +221,19 @@ cudaError_t launch_router_tc(const CUtensorMap& tm_x, const CUtensorMap& tm_w, c
     const int smem = router_tc_smem_bytes(n);
     cudaError_t e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    router_tc_kernel<<<static_cast<unsigned>((T + kRtBM - 1) / kRtBM), kRtThreads, smem, st>>>(
-        tm_x, tm_w, T, d, n, npad, rt_tmem_cols(npad), logits, status);
+    // split d so that about one CTA per SM runs, at least 8 K blocks each
+    const int64_t mtiles = (T + kRtBM - 1) / kRtBM;
+    int splits = static_cast<int>((num_sms + mtiles - 1) / mtiles);
+    const int kb_total = d / kRtBK;
+    if (splits > kRouterMaxSplits) splits = kRouterMaxSplits;
+    if (splits > kb_total / 8) splits = kb_total / 8;
+    if (splits < 1) splits = 1;
+    dim3 grid(static_cast<unsigned>(mtiles), static_cast<unsigned>(splits));
+    router_tc_kernel<<<grid, kRtThreads, smem, st>>>(tm_x, tm_w, T, d, n, npad, rt_tmem_cols(npad),
+                                                     logits, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    return launch_router_topk(logits, T, n, K, topk_idx, topk_w, st);
+    return launch_router_topk(logits, splits, T, n, K, topk_idx, topk_w, st);
 }
 
 }  // namespace moe
