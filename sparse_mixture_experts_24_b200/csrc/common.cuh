@@ -299,4 +299,36 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster) {
                  : "memory");
 }
 
+// ---------------------------------------------------------------------------
+// Epilogue stores through a per-warp shared-memory staging block
+// ---------------------------------------------------------------------------
+// A warp holds 32 rows (one per lane) x 64 bf16 columns as 32 packed words per
+// lane.  Writing them straight from registers makes every 16-byte store touch
+// 32 different rows; instead the warp transposes the block through shared
+// memory and each store instruction writes 4 whole 128-byte row segments.
+constexpr int kStageRowBytes = 128 + 16;                  // 64 bf16 + pad (no bank conflicts)
+constexpr int kWarpStageBytes = 32 * kStageRowBytes;      // 4,608 bytes per warp
+
+// pk[32]: this lane's row, columns col0 .. col0+63 as bf16 pairs.  Rows with
+// row_valid == false (past the expert's segment) are not written.
+__device__ __forceinline__ void warp_store_rows_64(uint8_t* stage, const uint32_t (&pk)[32], int lane,
+                                                   uint16_t* out, int64_t out_ld, int64_t row_base,
+                                                   int valid_rows, int col0) {
+    uint8_t* mine = stage + lane * kStageRowBytes;
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+        *reinterpret_cast<uint4*>(mine + q * 16) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int i = j * 32 + lane;   // 16-byte chunk i of the 32 x 128-byte block
+        const int r = i >> 3, c = i & 7;
+        if (r < valid_rows) {
+            const uint4 v = *reinterpret_cast<const uint4*>(stage + r * kStageRowBytes + c * 16);
+            *reinterpret_cast<uint4*>(out + (row_base + r) * out_ld + col0 + c * 8) = v;
+        }
+    }
+    __syncwarp();
+}
+
 }  // namespace moe

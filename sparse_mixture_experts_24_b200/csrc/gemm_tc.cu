@@ -59,7 +59,8 @@ struct __align__(8) TcSmemTail {
     int32_t mblk[kMaxN + 1];
 };
 
-constexpr int kSmemBytes = kStages * kStageBytes + static_cast<int>(sizeof(TcSmemTail)) + 1024;
+constexpr int kTailBytes = (static_cast<int>(sizeof(TcSmemTail)) + 127) / 128 * 128;
+constexpr int kSmemBytes = kStages * kStageBytes + kTailBytes + 4 * kWarpStageBytes + 1024;
 
 struct TileInfo {
     int e, n_tile, row0, rows;
@@ -235,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ---------------- epilogue (warps 2..5) ----------------
         const int quad = warp & 3;  // TMEM lanes [32*quad, 32*quad+32)
-        const int r = quad * 32 + lane;
+        uint8_t* stage = smem + kStages * kStageBytes + kTailBytes + (warp - 2) * kWarpStageBytes;
         int local = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++local) {
             const TileInfo ti = tile_info(t, tail->off, tail->mblk, n, args.n_tiles);
@@ -245,10 +246,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const uint32_t tbase =
                 tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf * kBN);
-            const bool row_ok = r < ti.rows;
-            const int64_t out_row = static_cast<int64_t>(ti.row0) + r;
+            // this warp's 32 rows: [row0 + 32*quad, ...), `valid` of them inside the segment
+            const int valid = min(32, ti.rows - quad * 32);
+            const int64_t row_base = static_cast<int64_t>(ti.row0) + quad * 32;
             uint16_t* out = static_cast<uint16_t*>(args.out);
             if (kSwiGLU) {
+                // GEMM1: direct 16-byte stores of each lane's row (measured faster here
+                // than staging through shared memory)
+                const bool row_ok = lane < valid;
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t a[32], b[32];
@@ -265,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 silu_f(__uint_as_float(a[2 * j + 1])) * __uint_as_float(b[2 * j + 1]);
                             pk[j] = pack_bf16x2(h0, h1);
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(out + out_row * args.out_cols + col);
+                        uint4* dst = reinterpret_cast<uint4*>(out + (row_base + lane) * args.out_cols + col);
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
                             dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
@@ -273,21 +278,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             } else {
 #pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t a[32];
-                    tmem_ld_32x32b_x32(tbase + c * 32, a);
-                    tmem_wait_ld();
-                    const int col = ti.n_tile * 256 + c * 32;
-                    if (row_ok && col < args.out_cols) {
-                        uint32_t pk[16];
+                for (int g = 0; g < 4; ++g) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t a[32];
+                        tmem_ld_32x32b_x32(tbase + g * 64 + c * 32, a);
+                        tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
-                            pk[j] = pack_bf16x2(__uint_as_float(a[2 * j]), __uint_as_float(a[2 * j + 1]));
-                        uint4* dst = reinterpret_cast<uint4*>(out + out_row * args.out_cols + col);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                            pk[c * 16 + j] = pack_bf16x2(__uint_as_float(a[2 * j]), __uint_as_float(a[2 * j + 1]));
                     }
+                    const int col = ti.n_tile * 256 + g * 64;
+                    if (col < args.out_cols && valid > 0)
+                        warp_store_rows_64(stage, pk, lane, out, args.out_cols, row_base, valid, col);
                 }
             }
             tc_fence_before();

@@ -58,7 +58,8 @@ struct __align__(8) PairTail {
     int32_t mblk[kPairMaxN + 1];
 };
 
-constexpr int kPairSmemBytes = kPairStages * kPairStageBytes + static_cast<int>(sizeof(PairTail)) + 1024;
+constexpr int kPairTailBytes = (static_cast<int>(sizeof(PairTail)) + 127) / 128 * 128;
+constexpr int kPairSmemBytes = kPairStages * kPairStageBytes + kPairTailBytes + 4 * kWarpStageBytes + 1024;
 
 struct PairTile {
     int e, n_tile, row0, rows;
@@ -238,7 +239,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     } else {
         // ---------------- epilogue (warps 2..5 of both CTAs) ----------------
         const int quad = warp & 3;
-        const int r = quad * 32 + lane;
+        uint8_t* stage = smem + kPairStages * kPairStageBytes + kPairTailBytes + (warp - 2) * kWarpStageBytes;
         const uint32_t accum_empty_leader0 = mapa_shared(smem_u32(&tail->accum_empty[0]), 0);
         const uint32_t accum_empty_leader1 = mapa_shared(smem_u32(&tail->accum_empty[1]), 0);
         int local = 0;
@@ -250,11 +251,15 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             tc_fence_after();
             const uint32_t tbase =
                 tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf * kPairBN);
+            // this warp's 32 rows of this CTA's half of the pair tile
             const int my_rows = pt.rows - 128 * static_cast<int>(rank);
-            const bool row_ok = r < my_rows;
-            const int64_t out_row = static_cast<int64_t>(pt.row0) + 128 * static_cast<int>(rank) + r;
+            const int valid = min(32, my_rows - quad * 32);
+            const int64_t row_base = static_cast<int64_t>(pt.row0) + 128 * static_cast<int>(rank) + quad * 32;
             uint16_t* out = static_cast<uint16_t*>(args.out);
             if (kSwiGLU) {
+                // GEMM1: direct 16-byte stores of each lane's row (measured faster here
+                // than staging through shared memory)
+                const bool row_ok = lane < valid;
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t a[32], b[32];
@@ -271,7 +276,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                                 silu_pair(__uint_as_float(a[2 * j + 1])) * __uint_as_float(b[2 * j + 1]);
                             pk[j] = pack_bf16x2(h0, h1);
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(out + out_row * args.out_cols + col);
+                        uint4* dst = reinterpret_cast<uint4*>(out + (row_base + lane) * args.out_cols + col);
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
                             dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
@@ -279,21 +284,20 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 }
             } else {
 #pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t a[32];
-                    tmem_ld_32x32b_x32(tbase + c * 32, a);
-                    tmem_wait_ld();
-                    const int col = pt.n_tile * kPairBN + c * 32;
-                    if (row_ok && col < args.out_cols) {
-                        uint32_t pk[16];
+                for (int g = 0; g < 4; ++g) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t a[32];
+                        tmem_ld_32x32b_x32(tbase + g * 64 + c * 32, a);
+                        tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
-                            pk[j] = pack_bf16x2(__uint_as_float(a[2 * j]), __uint_as_float(a[2 * j + 1]));
-                        uint4* dst = reinterpret_cast<uint4*>(out + out_row * args.out_cols + col);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                            pk[c * 16 + j] = pack_bf16x2(__uint_as_float(a[2 * j]), __uint_as_float(a[2 * j + 1]));
                     }
+                    const int col = pt.n_tile * kPairBN + g * 64;
+                    if (col < args.out_cols && valid > 0)
+                        warp_store_rows_64(stage, pk, lane, out, args.out_cols, row_base, valid, col);
                 }
             }
             tc_fence_before();

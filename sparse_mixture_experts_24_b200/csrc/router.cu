@@ -325,9 +325,15 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int e = lane + 32 * i;
+        // all partials in flight at once, then summed in split order
+        float part[kRouterMaxSplits];
+#pragma unroll
+        for (int sp = 0; sp < kRouterMaxSplits; ++sp)
+            part[sp] = (e < n && sp < splits) ? logits[(static_cast<int64_t>(sp) * T + t) * n + e] : 0.f;
         float a = 0.f;
-        if (e < n)
-            for (int sp = 0; sp < splits; ++sp) a += logits[(static_cast<int64_t>(sp) * T + t) * n + e];
+#pragma unroll
+        for (int sp = 0; sp < kRouterMaxSplits; ++sp)
+            if (sp < splits) a += part[sp];
         v[i] = a;
         if (v[i] != v[i]) v[i] = -INFINITY;  // NaN ranks lowest: keeps the order total
     }
