@@ -12,6 +12,8 @@ bf16 bit patterns stored as uint16, and are widened exactly to double):
   forward_with_routing(x, idx, gate, w1, w3, w2) -> y [T,d] f64
   moe_forward(x, W_g, w1, w3, w2, K)    -> y, idx, gate
   dispatch(idx, n)                      -> counts, offsets, row_token, token_row
+  dispatch_capacity(idx, n, C)          -> the same with at most C pairs per expert
+  router_stats(x, W_g, idx, alpha)      -> f [n], P [n], aux (load-balancing statistics)
   silu(z)                               -> z * sigmoid(z) in double
 
 Sources: the layer equation of "Mixtral of Experts" section 2.1 (flash-card
@@ -58,12 +60,16 @@ def _bind(L):
     L.oracle_moe_forward.argtypes = [i64, i32, i32, i32, i32, vp, i32, vp, i32,
                                      vp, vp, vp, i32, vp, vp, vp]
     L.oracle_dispatch.argtypes = [i64, i32, i32, vp, vp, vp, vp, vp]
+    L.oracle_router_stats.argtypes = [i64, i32, i32, i32, vp, i32, vp, i32, vp, ctypes.c_double,
+                                      vp, vp, vp]
+    L.oracle_dispatch_capacity.argtypes = [i64, i32, i32, vp, i64, vp, vp, vp, vp]
     L.oracle_silu.argtypes = [ctypes.c_double]
     L.oracle_silu.restype = ctypes.c_double
     L.oracle_num_threads.restype = ctypes.c_int
     L.oracle_set_num_threads.argtypes = [ctypes.c_int]
     for f in ("oracle_router", "oracle_expert", "oracle_forward_with_routing",
-              "oracle_moe_forward", "oracle_dispatch"):
+              "oracle_moe_forward", "oracle_dispatch", "oracle_router_stats",
+              "oracle_dispatch_capacity"):
         getattr(L, f).restype = ctypes.c_int
     return L
 
@@ -173,6 +179,33 @@ class Oracle:
         return counts, offsets, row_token, token_row.reshape(T, K)
 
 
+    def router_stats(self, x, W_g, idx, alpha: float):
+        """-> f [n], P [n], aux (the load-balancing statistics of the routing idx)."""
+        x, W_g = _c(x), _c(W_g)
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+        T, d = x.shape
+        n = W_g.shape[1]
+        K = idx.shape[1]
+        f = np.empty(n, np.float64)
+        P = np.empty(n, np.float64)
+        aux = np.empty(1, np.float64)
+        _check(self.L.oracle_router_stats(T, d, n, K, _p(x), _dt(x), _p(W_g), _dt(W_g), _p(idx),
+                                          float(alpha), _p(f), _p(P), _p(aux)), "router_stats")
+        return f, P, float(aux[0])
+
+    def dispatch_capacity(self, idx, n: int, capacity: int):
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+        T, K = idx.shape
+        counts = np.empty(n, np.int64)
+        offsets = np.empty(n + 1, np.int64)
+        row_token = np.full(max(1, T * K), -1, np.int64)
+        token_row = np.empty(max(1, T * K), np.int64)
+        _check(self.L.oracle_dispatch_capacity(T, n, K, _p(idx), int(capacity), _p(counts),
+                                               _p(offsets), _p(row_token), _p(token_row)),
+               "dispatch_capacity")
+        return counts, offsets, row_token[:T * K], token_row[:T * K].reshape(T, K)
+
+
 _default = None
 
 
@@ -213,3 +246,11 @@ def moe_forward(x, W_g, w1, w3, w2, K: int):
 
 def dispatch(idx, n: int):
     return default().dispatch(idx, n)
+
+
+def router_stats(x, W_g, idx, alpha: float):
+    return default().router_stats(x, W_g, idx, alpha)
+
+
+def dispatch_capacity(idx, n: int, capacity: int):
+    return default().dispatch_capacity(idx, n, capacity)

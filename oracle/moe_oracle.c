@@ -290,3 +290,100 @@ int oracle_dispatch(int64_t T, int n, int K, const int32_t *idx, int64_t *counts
     offsets[n] = row;
     return 0;
 }
+
+/*
+ * Load-balancing statistics of the router ("Mixture of Experts: Why Mixtral
+ * Only Wakes Up Two Specialists", Part 5, "Tool 2: a fine for favouritism",
+ * after the Switch Transformers paper):
+ *   f_i = share of the routed (token, slot) pairs sent to expert i
+ *         (count_i / (T*K); with K = 1 this is the share of tokens);
+ *   P_i = average over the tokens of the router's probability for expert i,
+ *         the softmax over ALL n logits;
+ *   aux = alpha * n * sum_i f_i * P_i.
+ * idx are the routed experts ([T][K], e.g. from oracle_router); the logits
+ * are recomputed here from x and W_g.
+ */
+int oracle_router_stats(int64_t T, int d, int n, int K, const void *x, int x_dt, const void *Wg,
+                        int wg_dt, const int32_t *idx, double alpha, double *f, double *P,
+                        double *aux)
+{
+    if (T <= 0 || d <= 0 || n <= 0 || K <= 0 || K > n || !x || !Wg || !idx || !f || !P || !aux ||
+        !dt_ok(x_dt) || !dt_ok(wg_dt))
+        return -1;
+    for (int64_t i = 0; i < T * K; ++i)
+        if (idx[i] < 0 || idx[i] >= n)
+            return -1;
+    double *L = (double *)malloc(sizeof(double) * (size_t)n);
+    if (!L)
+        return -1;
+    for (int e = 0; e < n; ++e) {
+        f[e] = 0.0;
+        P[e] = 0.0;
+    }
+    for (int64_t t = 0; t < T; ++t) {
+        double m = 0.0;
+        for (int e = 0; e < n; ++e) {
+            double s = 0.0;
+            for (int j = 0; j < d; ++j)
+                s += elem(x, x_dt, (size_t)t * d + j) * elem(Wg, wg_dt, (size_t)j * n + e);
+            L[e] = s;
+            if (e == 0 || s > m)
+                m = s;
+        }
+        double z = 0.0;
+        for (int e = 0; e < n; ++e)
+            z += exp(L[e] - m);
+        for (int e = 0; e < n; ++e)
+            P[e] += exp(L[e] - m) / z;
+        for (int k = 0; k < K; ++k)
+            f[idx[t * K + k]] += 1.0;
+    }
+    double acc = 0.0;
+    for (int e = 0; e < n; ++e) {
+        f[e] /= (double)(T * K);
+        P[e] /= (double)T;
+        acc += f[e] * P[e];
+    }
+    *aux = alpha * (double)n * acc;
+    free(L);
+    return 0;
+}
+
+/*
+ * Dispatch with an expert capacity (the Switch paper's capacity, Part 5 of
+ * the neobadger page: "the tokens in the batch divided by the number of
+ * experts, times a capacity factor"; the pairs that overflow are dropped and
+ * skip the expert).  capacity = the most (token, slot) pairs one expert takes;
+ * the first ones in dispatch order (tokens ascending) are kept.  Dropped pairs
+ * get token_row = -1 and are not counted.  Outputs as oracle_dispatch.
+ */
+int oracle_dispatch_capacity(int64_t T, int n, int K, const int32_t *idx, int64_t capacity,
+                             int64_t *counts, int64_t *offsets, int64_t *row_token,
+                             int64_t *token_row)
+{
+    if (T < 0 || n <= 0 || K <= 0 || K > n || capacity < 0 || !counts || !offsets)
+        return -1;
+    if (T > 0 && (!idx || !row_token || !token_row))
+        return -1;
+    for (int64_t i = 0; i < T * K; ++i)
+        if (idx[i] < 0 || idx[i] >= n)
+            return -1;
+    int64_t row = 0;
+    for (int e = 0; e < n; ++e) {
+        offsets[e] = row;
+        for (int64_t t = 0; t < T; ++t)
+            for (int k = 0; k < K; ++k)
+                if (idx[t * K + k] == e) {
+                    if (row - offsets[e] < capacity) {
+                        row_token[row] = t;
+                        token_row[t * K + k] = row;
+                        ++row;
+                    } else {
+                        token_row[t * K + k] = -1;
+                    }
+                }
+        counts[e] = row - offsets[e];
+    }
+    offsets[n] = row;
+    return 0;
+}

@@ -300,6 +300,71 @@ def check_dispatch(O):
             assert token_row[t, k] == r
 
 
+# --------------------------------------------------------------------------
+# Load-balancing statistics and expert capacity ([P5] Part 5)
+# --------------------------------------------------------------------------
+
+def check_router_stats_closed_forms(O):
+    """[P5] Part 5 Tool 2: f_i = share of the routed pairs sent to expert i,
+    P_i = mean router probability (softmax over all n logits), aux =
+    alpha * N * sum f_i P_i.  All-equal logits give P_i = 1/N exactly; the
+    tie-break then sends every token to experts 0..K-1, so aux = alpha; a
+    uniform routing with uniform probabilities also gives aux = alpha (the
+    minimum of N * sum f_i P_i is 1)."""
+    T, d, n, K = 24, 16, 8, 2
+    x = np.random.default_rng(40).standard_normal((T, d))
+    Wg = np.zeros((d, n))
+    idx, _, _ = O.router(x, Wg, K)
+    f, P, aux = O.router_stats(x, Wg, idx, 0.01)
+    assert np.allclose(P, 1.0 / n, rtol=0, atol=1e-15)
+    assert np.allclose(f, [0.5, 0.5] + [0.0] * 6, rtol=0, atol=0)
+    assert abs(aux - 0.01) < 1e-15
+    uni = np.array([[t % n, (t + 1) % n] for t in range(T)], np.int32)
+    f2, P2, aux2 = O.router_stats(x, Wg, uni, 0.02)
+    assert np.allclose(f2, 1.0 / n, rtol=0, atol=1e-15) and abs(aux2 - 0.02) < 1e-15
+
+
+def check_router_stats_against_torch(O):
+    """Random case against torch's softmax and a bincount."""
+    T, d, n, K = 37, 24, 6, 2
+    g = np.random.default_rng(41)
+    x = g.standard_normal((T, d))
+    Wg = g.standard_normal((d, n)) / math.sqrt(d)
+    idx, _, _ = O.router(x, Wg, K)
+    f, P, aux = O.router_stats(x, Wg, idx, 0.01)
+    Pt = torch.softmax(torch.from_numpy(x @ Wg), dim=1).mean(0).numpy()
+    ft = np.bincount(idx.ravel(), minlength=n) / (T * K)
+    assert np.allclose(P, Pt, rtol=1e-13, atol=1e-15)
+    assert np.allclose(f, ft, rtol=0, atol=1e-15)
+    assert abs(aux - 0.01 * n * float((ft * Pt).sum())) < 1e-14
+    assert abs(P.sum() - 1.0) < 1e-13 and abs(f.sum() - 1.0) < 1e-14
+
+
+def check_dispatch_capacity(O):
+    """[P5] Part 5 'What happens when an expert is full': at most C pairs per
+    expert, the first ones in dispatch order kept, the overflow dropped."""
+    rng = np.random.default_rng(42)
+    for T, n, K, C in ((50, 4, 2, 10), (64, 8, 2, 0), (33, 5, 3, 7), (40, 3, 1, 100), (1, 2, 2, 1)):
+        idx = np.array([rng.permutation(n)[:K] for _ in range(T)], np.int32).reshape(T, K)
+        counts, offsets, row_token, token_row = O.dispatch_capacity(idx, n, C)
+        full = np.bincount(idx.ravel(), minlength=n)
+        assert np.array_equal(counts, np.minimum(full, C))
+        assert np.array_equal(np.diff(offsets), counts) and offsets[0] == 0
+        order = np.argsort(idx.ravel(), kind="stable")
+        kept = []
+        for e in range(n):
+            pe = order[idx.ravel()[order] == e]
+            kept.extend(pe[:C].tolist())
+        kept = np.array(kept, np.int64)
+        tr = token_row.ravel()
+        assert np.array_equal(np.sort(np.nonzero(tr >= 0)[0]), np.sort(kept))
+        assert np.array_equal(tr[kept], np.arange(kept.size))
+        assert np.array_equal(row_token[:kept.size], kept // K)
+        if C >= full.max():
+            c0, o0, rt0, tr0 = O.dispatch(idx, n)
+            assert np.array_equal(c0, counts) and np.array_equal(tr0, token_row)
+
+
 ALL_CHECKS = [
     check_worked_example, check_two_way_softmax_closed_form, check_logits_are_x_times_Wg,
     check_topk_brute_force, check_ties_go_to_lower_index, check_gate_invariants, check_silu,
@@ -307,4 +372,5 @@ ALL_CHECKS = [
     check_top2_layer_against_torch, check_relabel_invariance,
     check_unchosen_experts_do_not_matter, check_forward_with_routing_consistent,
     check_bf16_inputs_widen_exactly, check_dispatch,
+    check_router_stats_closed_forms, check_router_stats_against_torch, check_dispatch_capacity,
 ]

@@ -26,6 +26,9 @@ MUTANTS = {
     "dispatch_slot_major": [("        for (int64_t t = 0; t < T; ++t)\n            for (int k = 0; k < K; ++k)\n                if (idx[t * K + k] == e) {",
                              "        for (int k = 0; k < K; ++k)\n            for (int64_t t = 0; t < T; ++t)\n                if (idx[t * K + k] == e) {")],
     "softmax_first_logit_only": [("z += exp(L[idx[k]] - m);", "z += (k == 0) ? 1.0 : 0.0;")],
+    "stats_f_over_tokens": [("f[e] /= (double)(T * K);", "f[e] /= (double)T;")],
+    "stats_P_unnormalised": [("P[e] += exp(L[e] - m) / z;", "P[e] += exp(L[e] - m);")],
+    "capacity_keeps_one_more": [("if (row - offsets[e] < capacity) {", "if (row - offsets[e] <= capacity) {")],
 }
 
 
