@@ -153,6 +153,38 @@ MOE_API moe_status moe_forward_with_routing(moe_handle *h, int64_t T, const void
                                     moe_stream_t stream);
 
 /*
+ * Expert capacity (Part 5 of the neobadger page, "What happens when an expert
+ * is full", after the Switch paper: capacity = tokens in the batch / experts x
+ * a capacity factor).  With factor > 0, each later forward / dispatch call on
+ * T tokens gives every expert at most C = ceil(factor * T * K / n) (token,
+ * slot) pairs: the first C in dispatch order (tokens ascending) are kept, the
+ * overflow pairs skip their expert and add nothing to y (the caller's residual
+ * carries those tokens on), and moe_dispatch reports them with token_row = -1.
+ * Gates are not renormalised.  factor = 0 (the default) is the dropless layer
+ * of the layer equation.
+ *   Errors: MOE_ERR_INVALID_ARG (null handle, factor < 0 or not finite).
+ */
+MOE_API moe_status moe_set_capacity_factor(moe_handle *h, double factor);
+
+/*
+ * Load-balancing statistics of a routing (Part 5 of the neobadger page, "Tool
+ * 2: a fine for favouritism", the Switch Transformers loss):
+ *   f[i]  = share of the T*K routed (token, slot) pairs of topk_idx sent to
+ *           expert i (the share of tokens when K = 1);
+ *   P[i]  = mean over the T tokens of the router probability of expert i, the
+ *           softmax over all n logits x . W_g (fp32);
+ *   aux[0] = alpha * n * sum_i f[i] * P[i]  (alpha: 0.01 in the Switch paper,
+ *           0.02 in the Hugging Face Mixtral configuration).
+ * x, W_g as for moe_forward; topk_idx [T][K] an input (e.g. from moe_route);
+ * f, P (n floats) and aux (1 float) device outputs.  Sums run in a fixed order
+ * (deterministic).
+ *   Errors: MOE_ERR_INVALID_ARG (also T = 0, alpha not finite), as moe_forward.
+ */
+MOE_API moe_status moe_router_stats(moe_handle *h, int64_t T, const void *x, const float *W_g,
+                                    const int32_t *topk_idx, float alpha, float *f, float *P,
+                                    float *aux, moe_stream_t stream);
+
+/*
  * Debug view of the workspace written by the last moe_forward /
  * moe_forward_with_routing: name is "H" (expert hidden layer, [rows][ffn],
  * handle dtype) or "O" (per-row expert outputs, [rows][d], handle dtype for

@@ -54,19 +54,22 @@ lib.moe_workspace_view.argtypes = [_vp, ctypes.c_char_p, ctypes.POINTER(_vp), ct
 lib.moe_sync_status.argtypes = [_vp, _vp]
 lib.moe_destroy.argtypes = [_vp]
 lib.moe_trace_begin.argtypes = [_vp, _int]
+lib.moe_set_capacity_factor.argtypes = [_vp, ctypes.c_double]
+lib.moe_router_stats.argtypes = [_vp, _i64, _vp, _vp, _vp, ctypes.c_float, _vp, _vp, _vp, _vp]
 lib.moe_dispatch_noalloc.argtypes = [_i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.moe_trace_end.argtypes = [_vp, ctypes.POINTER(ctypes.c_double), _int, ctypes.POINTER(_int)]
 lib.moe_last_error.restype = ctypes.c_char_p
 lib.moe_version.restype = ctypes.c_char_p
 for _f in ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
            "moe_forward_with_routing", "moe_workspace_view", "moe_sync_status", "moe_destroy",
-           "moe_trace_begin", "moe_trace_end", "moe_dispatch_noalloc"):
+           "moe_trace_begin", "moe_trace_end", "moe_dispatch_noalloc", "moe_set_capacity_factor",
+           "moe_router_stats"):
     getattr(lib, _f).restype = _int
 
 EXPORTED = ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
             "moe_forward_with_routing", "moe_workspace_view", "moe_sync_status", "moe_destroy",
             "moe_last_error", "moe_version", "moe_trace_begin", "moe_trace_end",
-            "moe_dispatch_noalloc")
+            "moe_dispatch_noalloc", "moe_set_capacity_factor", "moe_router_stats")
 
 TRACE_STAGES = ("router", "dispatch", "gather", "gemm1", "gemm2", "combine")
 
@@ -159,6 +162,15 @@ def moe_dispatch_noalloc(T, n, K, topk_idx, counts, offsets, row_token, token_ro
            "moe_dispatch_noalloc")
 
 
+def moe_set_capacity_factor(h, factor: float) -> None:
+    _check(lib.moe_set_capacity_factor(h, float(factor)), "moe_set_capacity_factor")
+
+
+def moe_router_stats(h, T, x, W_g, topk_idx, alpha, f, P, aux, stream=None) -> None:
+    _check(lib.moe_router_stats(h, T, _ptr(x), _ptr(W_g), _ptr(topk_idx), float(alpha), _ptr(f),
+                                _ptr(P), _ptr(aux), _stream(stream)), "moe_router_stats")
+
+
 def moe_trace_begin(h, max_calls: int) -> None:
     _check(lib.moe_trace_begin(h, max_calls), "moe_trace_begin")
 
@@ -227,6 +239,18 @@ class MoELayer:
         token_row = torch.empty((max(1, T), self.K), dtype=torch.int32, device=dev)
         moe_dispatch(self.h, T, topk_idx, counts, offsets, row_token, token_row, stream)
         return counts, offsets, row_token[:T * self.K], token_row[:T]
+
+    def set_capacity_factor(self, factor: float) -> None:
+        moe_set_capacity_factor(self.h, factor)
+
+    def router_stats(self, x, W_g, topk_idx, alpha=0.01, stream=None):
+        """-> f [n], P [n], aux [1] (device float32 tensors)."""
+        import torch
+        f = torch.empty(self.n, dtype=torch.float32, device=x.device)
+        P = torch.empty(self.n, dtype=torch.float32, device=x.device)
+        aux = torch.empty(1, dtype=torch.float32, device=x.device)
+        moe_router_stats(self.h, x.shape[0], x, W_g, topk_idx, alpha, f, P, aux, stream)
+        return f, P, aux
 
     def sync_status(self, stream=None) -> None:
         moe_sync_status(self.h, stream)

@@ -8,6 +8,9 @@
 // computed; and Part 3, Step 2 of "Mixture of Experts: Why Mixtral Only Wakes
 // Up Two Specialists" (the experts not kept are not run at all).  The layout
 // (experts ascending, tokens ascending inside an expert) is this library's.
+// An optional expert capacity (the Switch capacity described in Part 5 of the
+// same page) keeps the first `capacity` pairs of each expert in that order and
+// drops the rest (token_row = -1: the pair adds nothing to y).
 //
 // Kernels:
 //   rank_kernel    per block of 256 pairs: expert histogram and the stable
@@ -93,7 +96,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp) {
 constexpr int kScanSmemInts = 8192;
 
 __global__ void __launch_bounds__(256) scan_kernel(int32_t* __restrict__ blockcounts, int nblk,
-                                                   int n, int64_t R, int bm,
+                                                   int n, int capacity, int bm,
                                                    int32_t* __restrict__ counts,
                                                    int32_t* __restrict__ offsets,
                                                    int32_t* __restrict__ mblk_base) {
@@ -119,6 +122,7 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* __restrict__ blockco
         __syncthreads();
         for (int i = threadIdx.x; i < cnt; i += 256) g[i] = s_chunk[i];
     }
+    total = min(total, capacity);  // pairs past the expert's capacity are dropped
     const int off = block_exclusive_scan(e < n ? total : 0, s_warp);
     const int mb = (e < n) ? (total + bm - 1) / bm : 0;
     const int mbase = block_exclusive_scan(mb, s_warp);
@@ -131,11 +135,10 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* __restrict__ blockco
         offsets[n] = off + total;
         mblk_base[n] = mbase + mb;
     }
-    (void)R;
 }
 
 __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict__ idx, int64_t R,
-                                                      int K, int n,
+                                                      int K, int n, int capacity,
                                                       const int32_t* __restrict__ offsets,
                                                       const int32_t* __restrict__ blockbase,
                                                       const int32_t* __restrict__ pair_rank,
@@ -149,19 +152,24 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
         token_row[p] = -1;
         return;
     }
-    const int dest = offsets[e] + blockbase[(p / kPairsPerBlock) * n + e] + rk;
+    const int rank_in_expert = blockbase[(p / kPairsPerBlock) * n + e] + rk;
+    if (rank_in_expert >= capacity) {  // overflow: this pair skips its expert
+        token_row[p] = -1;
+        return;
+    }
+    const int dest = offsets[e] + rank_in_expert;
     row_token[dest] = static_cast<int32_t>(p / K);
     token_row[p] = dest;
 }
 
 cudaError_t launch_dispatch(const int32_t* topk_idx, int64_t T, int K, int n, int bm,
-                            const DispatchBufs& b, cudaStream_t st) {
+                            const DispatchBufs& b, cudaStream_t st, int capacity) {
     const int64_t R = T * K;
     const int nblk = static_cast<int>((R + kPairsPerBlock - 1) / kPairsPerBlock);
     rank_kernel<<<nblk, kPairsPerBlock, 0, st>>>(topk_idx, R, n, b.blockcounts, b.pair_rank);
-    scan_kernel<<<1, 256, 0, st>>>(b.blockcounts, nblk, n, R, bm, b.counts, b.offsets, b.mblk_base);
+    scan_kernel<<<1, 256, 0, st>>>(b.blockcounts, nblk, n, capacity, bm, b.counts, b.offsets, b.mblk_base);
     scatter_kernel<<<static_cast<unsigned>((R + 255) / 256), 256, 0, st>>>(
-        topk_idx, R, K, n, b.offsets, b.blockcounts, b.pair_rank, b.row_token, b.token_row);
+        topk_idx, R, K, n, capacity, b.offsets, b.blockcounts, b.pair_rank, b.row_token, b.token_row);
     return cudaGetLastError();
 }
 

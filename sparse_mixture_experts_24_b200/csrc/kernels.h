@@ -50,9 +50,26 @@ struct DispatchBufs {
 };
 
 // Histogram + stable in-block ranks, scan, scatter.  bm = rows per M-block of
-// the GEMM that consumes the segments.
+// the GEMM that consumes the segments; capacity = most pairs one expert takes
+// (kNoCapacity: all).
+constexpr int kNoCapacity = 2147483647;
 cudaError_t launch_dispatch(const int32_t* topk_idx, int64_t T, int K, int n, int bm,
-                            const DispatchBufs& b, cudaStream_t st);
+                            const DispatchBufs& b, cudaStream_t st, int capacity = kNoCapacity);
+
+// Load-balancing statistics from logits [splits][T][n] (summed in split
+// order) and the routing topk_idx [T][K]: f[n] (share of routed pairs),
+// P[n] (mean softmax probability), aux[0] = alpha * n * sum f P.  partial is
+// scratch of ceil(T/256) * n floats, counts scratch of n ints.
+cudaError_t launch_router_stats(const float* logits, int splits, int64_t T, int n, int K,
+                                const int32_t* topk_idx, float alpha, float* partial,
+                                int32_t* counts, float* f, float* P, float* aux, cudaStream_t st);
+
+// Logits only (no top-K) into logits [splits][T][n]; returns the split count.
+cudaError_t launch_router_logits_tc(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const float* Wg,
+                                    uint16_t* parts, int64_t T, int d, int n, float* logits, int* status,
+                                    int num_sms, cudaStream_t st, int* splits_out);
+cudaError_t launch_router_logits_simt(const void* x, bool x_bf16, const float* Wg, int64_t T, int d,
+                                      int n, float* logits, cudaStream_t st);
 
 // Xp[r] = x[row_token[r]] for r < R (row_bytes per row, multiple of 16);
 // rows whose token is outside [0, T) are skipped.

@@ -7,6 +7,7 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <cmath>
 #include <cstdlib>
 #include <cstring>
 #include <new>
@@ -121,6 +122,10 @@ struct moe_handle {
     CUtensorMap tm_rx, tm_parts;
     const void* c_rx = nullptr;
     int64_t c_rx_T = -1;
+    // expert capacity factor (0: dropless) and load-balancing statistics scratch
+    double capacity_factor = 0.0;
+    float* stats_partial = nullptr;
+    int32_t* stats_counts = nullptr;
     // tracing: kTraceEvents events per traced call
     std::vector<cudaEvent_t> trace_ev;
     int trace_max = 0;
@@ -201,8 +206,9 @@ moe_status grow(moe_handle* h, int64_t T) {
     const size_t o_token_row = take(static_cast<size_t>(R) * 4);
     const bool bf = h->dtype == MOE_BF16;
     const int npad = (h->n + 15) / 16 * 16;
-    const size_t o_logits =
-        take((bf || h->n > 32) ? static_cast<size_t>(moe::kRouterMaxSplits) * T * h->n * 4 : 0);
+    const size_t o_logits = take(static_cast<size_t>(moe::kRouterMaxSplits) * T * h->n * 4);
+    const size_t o_stats_partial = take(static_cast<size_t>((T + 255) / 256) * h->n * 4);
+    const size_t o_stats_counts = take(static_cast<size_t>(h->n) * 4);
     const size_t o_parts = take(bf ? static_cast<size_t>(3) * npad * h->d * 2 : 0);
     const size_t o_status = take(64);
     const size_t o_xp = take(static_cast<size_t>(R) * h->d * h->esize());
@@ -240,6 +246,8 @@ moe_status grow(moe_handle* h, int64_t T) {
     h->db.token_row = reinterpret_cast<int32_t*>(b + o_token_row);
     h->logits = reinterpret_cast<float*>(b + o_logits);
     h->wg_parts = reinterpret_cast<uint16_t*>(b + o_parts);
+    h->stats_partial = reinterpret_cast<float*>(b + o_stats_partial);
+    h->stats_counts = reinterpret_cast<int32_t*>(b + o_stats_counts);
     h->c_rx = nullptr;
     h->status = reinterpret_cast<int*>(b + o_status);
     h->xp = b + o_xp;
@@ -309,6 +317,14 @@ bool use_pair_gemm(const moe_handle* h, int64_t T) {
     return env && strcmp(env, "pair") == 0;
 }
 
+// Most (token, slot) pairs one expert takes in a call of T tokens:
+// ceil(factor * T * K / n), or no limit when the factor is 0.
+int capacity_for(const moe_handle* h, int64_t T) {
+    if (!(h->capacity_factor > 0.0)) return moe::kNoCapacity;
+    const double c = std::ceil(h->capacity_factor * static_cast<double>(T) * h->K / h->n);
+    return c >= static_cast<double>(moe::kNoCapacity) ? moe::kNoCapacity : static_cast<int>(c);
+}
+
 moe_status run_experts(moe_handle* h, int64_t T, const void* x, const int32_t* topk_idx,
                        const float* topk_w, const void* w1, const void* w3, const void* w2, void* y,
                        cudaStream_t st) {
@@ -317,7 +333,7 @@ moe_status run_experts(moe_handle* h, int64_t T, const void* x, const int32_t* t
     const int64_t R = T * h->K;
     cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n,
                                          pair ? moe::kTcPairBM : (bf ? moe::kTcBM : moe::kSimtBM),
-                                         h->db, st);
+                                         h->db, st, capacity_for(h, T));
     if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
     trace_mark(h, 1, st);
     e = moe::launch_gather(x, h->db.row_token, R, T, static_cast<int64_t>(h->d) * h->esize(), h->xp,
@@ -497,7 +513,8 @@ moe_status moe_dispatch(moe_handle* h, int64_t T, const int32_t* topk_idx, int32
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int64_t R = T * h->K;
     cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n,
-                                         h->dtype == MOE_BF16 ? moe::kTcBM : moe::kSimtBM, h->db, st);
+                                         h->dtype == MOE_BF16 ? moe::kTcBM : moe::kSimtBM, h->db, st,
+                                         capacity_for(h, T));
     if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
     struct {
         void* dst;
@@ -512,6 +529,51 @@ moe_status moe_dispatch(moe_handle* h, int64_t T, const int32_t* topk_idx, int32
         e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyDeviceToDevice, st);
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(dispatch output)");
     }
+    return ok();
+}
+
+moe_status moe_set_capacity_factor(moe_handle* h, double factor) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "null handle");
+    if (!(factor >= 0.0) || !std::isfinite(factor))
+        return fail(MOE_ERR_INVALID_ARG, "capacity factor must be finite and >= 0 (0 = no capacity)");
+    h->capacity_factor = factor;
+    return ok();
+}
+
+moe_status moe_router_stats(moe_handle* h, int64_t T, const void* x, const float* W_g,
+                            const int32_t* topk_idx, float alpha, float* f, float* P, float* aux,
+                            moe_stream_t stream) {
+    moe_status s = check_common(h, T);
+    if (s != MOE_OK) return s;
+    if (T == 0) return fail(MOE_ERR_INVALID_ARG, "T = 0: the statistics are averages over tokens");
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(W_g);
+    REQUIRE_PTR(topk_idx);
+    REQUIRE_PTR(f);
+    REQUIRE_PTR(P);
+    REQUIRE_PTR(aux);
+    if (!std::isfinite(alpha)) return fail(MOE_ERR_INVALID_ARG, "alpha is not finite");
+    s = prepare(h, T);
+    if (s != MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int splits = 1;
+    cudaError_t e;
+    if (h->dtype == MOE_BF16) {
+        if (x != h->c_rx || T != h->c_rx_T) {
+            if (!encode_rows(&h->tm_rx, x, h->d, static_cast<uint64_t>(T)))
+                return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for x");
+            h->c_rx = x;
+            h->c_rx_T = T;
+        }
+        e = moe::launch_router_logits_tc(h->tm_rx, h->tm_parts, W_g, h->wg_parts, T, h->d, h->n, h->logits,
+                                         h->status, h->num_sms, st, &splits);
+    } else {
+        e = moe::launch_router_logits_simt(x, false, W_g, T, h->d, h->n, h->logits, st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "router logits launch");
+    e = moe::launch_router_stats(h->logits, splits, T, h->n, h->K, topk_idx, alpha, h->stats_partial,
+                                 h->stats_counts, f, P, aux, st);
+    if (e != cudaSuccess) return cuda_fail(e, "router statistics launch");
     return ok();
 }
 

@@ -434,6 +434,17 @@ static cudaError_t launch_router_t(const XT* x, const float* Wg, int64_t T, int 
     return cudaGetLastError();
 }
 
+cudaError_t launch_router_logits_simt(const void* x, bool x_bf16, const float* Wg, int64_t T, int d,
+                                      int n, float* logits, cudaStream_t st) {
+    dim3 g1(static_cast<unsigned>((T + kRT - 1) / kRT), static_cast<unsigned>((n + kRE - 1) / kRE));
+    if (x_bf16)
+        router_logits_kernel<uint16_t><<<g1, 256, 0, st>>>(static_cast<const uint16_t*>(x), Wg, T, d, n,
+                                                           logits);
+    else
+        router_logits_kernel<float><<<g1, 256, 0, st>>>(static_cast<const float*>(x), Wg, T, d, n, logits);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_router(const void* x, bool x_bf16, const float* Wg, int64_t T, int d, int n,
                           int K, int32_t* topk_idx, float* topk_w, float* logits_ws, int num_sms,
                           cudaStream_t st) {

@@ -209,10 +209,9 @@ int router_tc_smem_bytes(int n) {
     return rt_stages(npad) * rt_stage_bytes(npad) + static_cast<int>(sizeof(RtTail)) + 1024;
 }
 
-cudaError_t launch_router_tc(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const float* Wg,
-                             uint16_t* parts, int64_t T, int d, int n, int K, float* logits,
-                             int32_t* topk_idx, float* topk_w, int* status, int num_sms,
-                             cudaStream_t st) {
+cudaError_t launch_router_logits_tc(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const float* Wg,
+                                    uint16_t* parts, int64_t T, int d, int n, float* logits, int* status,
+                                    int num_sms, cudaStream_t st, int* splits_out) {
     const int npad = (n + 15) / 16 * 16;
     const int64_t total = static_cast<int64_t>(npad) * d;
     int64_t sb = (total + 255) / 256;
@@ -231,7 +230,17 @@ cudaError_t launch_router_tc(const CUtensorMap& tm_x, const CUtensorMap& tm_w, c
     dim3 grid(static_cast<unsigned>(mtiles), static_cast<unsigned>(splits));
     router_tc_kernel<<<grid, kRtThreads, smem, st>>>(tm_x, tm_w, T, d, n, npad, rt_tmem_cols(npad),
                                                      logits, status);
-    e = cudaGetLastError();
+    *splits_out = splits;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_router_tc(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const float* Wg,
+                             uint16_t* parts, int64_t T, int d, int n, int K, float* logits,
+                             int32_t* topk_idx, float* topk_w, int* status, int num_sms,
+                             cudaStream_t st) {
+    int splits = 1;
+    cudaError_t e = launch_router_logits_tc(tm_x, tm_w, Wg, parts, T, d, n, logits, status, num_sms, st,
+                                            &splits);
     if (e != cudaSuccess) return e;
     return launch_router_topk(logits, splits, T, n, K, topk_idx, topk_w, st);
 }

@@ -101,3 +101,23 @@ def test_forward_rejects_bad_arguments_on_the_host(m):
         assert m.moe_last_error() != ""
     finally:
         m.moe_destroy(h)
+
+
+def test_capacity_and_stats_argument_checks_on_the_host(m):
+    h = m.moe_create(8, 2, 128, 256, m.MOE_BF16)
+    try:
+        m.moe_set_capacity_factor(h, 1.25)
+        m.moe_set_capacity_factor(h, 0.0)
+        for bad in (-1.0, float("nan"), float("inf")):
+            with pytest.raises(m.MoEError) as ei:
+                m.moe_set_capacity_factor(h, bad)
+            assert ei.value.status == m.MOE_ERR_INVALID_ARG
+        good = 1 << 20
+        with pytest.raises(m.MoEError) as ei:
+            m.moe_router_stats(h, 0, good, good, good, 0.01, good, good, good, 0)
+        assert "T = 0" in str(ei.value)
+        with pytest.raises(m.MoEError) as ei:
+            m.moe_router_stats(h, 4, good, good, good, 0.01, good, None, good, 0)
+        assert "P is NULL" in str(ei.value)
+    finally:
+        m.moe_destroy(h)
