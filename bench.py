@@ -196,21 +196,26 @@ class ClockSampler:
 # CPU baseline: the oracle on a bounded sample of the workload
 # --------------------------------------------------------------------------
 
-def oracle_tokens_per_s(cfg, L, budget_s=15.0, max_tokens=None):
+def oracle_tokens_per_s(cfg, L, budget_s=12.0):
+    """The oracle on the first tokens of the workload, repeated until about
+    budget_s of host time (a bounded sample of the same layer)."""
     import oracle
     threads = oracle.num_threads()
-    T = cfg.T if max_tokens is None else min(cfg.T, max_tokens)
-    # calibrate on one token, then size the sample to the budget
     t0 = time.perf_counter()
     oracle.moe_forward(L["x"][:1], L["W_g"], L["w1"], L["w3"], L["w2"], cfg.K)
-    one = time.perf_counter() - t0
-    par = max(1, threads)
-    s = int(max(1, min(T, budget_s * par / max(one, 1e-6))))
-    s = min(s, T)
+    one = max(time.perf_counter() - t0, 1e-6)
+    # tokens per repetition: enough to keep every thread busy, within budget
+    s = int(max(1, min(cfg.T, max(threads, budget_s * threads / one / 4))))
+    done, reps = 0, 0
     t0 = time.perf_counter()
-    oracle.moe_forward(L["x"][:s], L["W_g"], L["w1"], L["w3"], L["w2"], cfg.K)
-    el = time.perf_counter() - t0
-    return s / el, s, min(threads, s), el
+    while True:
+        oracle.moe_forward(L["x"][:s], L["W_g"], L["w1"], L["w3"], L["w2"], cfg.K)
+        done += s
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or reps >= 1000:
+            break
+    return done / el, s, reps, min(threads, s), el
 
 
 # --------------------------------------------------------------------------
@@ -322,6 +327,7 @@ def main():
         dist.barrier()
     torch.cuda.synchronize(dev)
     m.moe_trace_begin(layer.h, args.steps)
+    launches0 = m.moe_launch_count(layer.h)
     sampler.start()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
@@ -330,6 +336,7 @@ def main():
     ev1.record(stream)
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
+    launches = m.moe_launch_count(layer.h) - launches0
     stage_ms, traced = m.moe_trace_end(layer.h)
     if dist:
         dist.barrier()
@@ -400,9 +407,10 @@ def main():
     # ---- CPU baseline (rank 0, N = 1 only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, s, cores, el = oracle_tokens_per_s(cfg, L)
+        v, s, reps, cores, el = oracle_tokens_per_s(cfg, L)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": "first %d of %d tokens, full layer in fp64 (%.1f s)" % (s, cfg.T, el)}
+               "sample": "first %d of %d tokens x %d repetitions, full layer in fp64 (%.1f s)"
+                         % (s, cfg.T, reps, el)}
 
     if rank == 0:
         layer_ms = ms
@@ -423,7 +431,7 @@ def main():
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": args.steps * (9 if cfg.n > 32 else 8),
+            "gpu_launches": launches,
             "clocks": clocks,
         }
         print(json.dumps(line))

@@ -242,6 +242,9 @@ MOE_API moe_status moe_dispatch_noalloc(int64_t T, int n, int K, const int32_t *
                                         int32_t *counts, int32_t *offsets, int32_t *row_token,
                                         int32_t *token_row, moe_stream_t stream);
 
+/* Number of CUDA kernels this handle has launched so far (all entry points). */
+MOE_API moe_status moe_launch_count(moe_handle *h, int64_t *count);
+
 /* Free the workspace and the handle.  NULL is allowed. */
 MOE_API moe_status moe_destroy(moe_handle *h);
 

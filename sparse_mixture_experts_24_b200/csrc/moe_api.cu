@@ -124,6 +124,8 @@ struct moe_handle {
     int64_t c_rx_T = -1;
     // expert capacity factor (0: dropless) and load-balancing statistics scratch
     double capacity_factor = 0.0;
+    // kernels this handle has launched (for profiling and launch accounting)
+    int64_t launches = 0;
     float* stats_partial = nullptr;
     int32_t* stats_counts = nullptr;
     // tracing: kTraceEvents events per traced call
@@ -298,9 +300,11 @@ moe_status run_router(moe_handle* h, int64_t T, const void* x, const float* W_g,
         }
         e = moe::launch_router_tc(h->tm_rx, h->tm_parts, W_g, h->wg_parts, T, h->d, h->n, h->K,
                                   h->logits, topk_idx, topk_w, h->status, h->num_sms, st);
+        h->launches += 3;  // W_g split, logits, top-K
     } else {
         e = moe::launch_router(x, h->dtype == MOE_BF16, W_g, T, h->d, h->n, h->K, topk_idx, topk_w,
                                h->logits, h->num_sms, st);
+        h->launches += h->n > 32 ? 2 : 1;
     }
     if (e != cudaSuccess) return cuda_fail(e, "router launch");
     return MOE_OK;
@@ -335,10 +339,12 @@ moe_status run_experts(moe_handle* h, int64_t T, const void* x, const int32_t* t
                                          pair ? moe::kTcPairBM : (bf ? moe::kTcBM : moe::kSimtBM),
                                          h->db, st, capacity_for(h, T));
     if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
+    h->launches += 3;  // rank, scan, scatter
     trace_mark(h, 1, st);
     e = moe::launch_gather(x, h->db.row_token, R, T, static_cast<int64_t>(h->d) * h->esize(), h->xp,
                            h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+    h->launches += 1;
     trace_mark(h, 2, st);
     if (bf) {
         if (w1 != h->c_w1) {
@@ -369,6 +375,7 @@ moe_status run_experts(moe_handle* h, int64_t T, const void* x, const int32_t* t
         e = pair ? moe::launch_tc_gemm1_pair(h->tm_xp, h->tm_w1, h->tm_w3, a1, h->num_sms, st)
                  : moe::launch_tc_gemm1(h->tm_xp, h->tm_w1, h->tm_w3, a1, h->num_sms, st);
         if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
+        h->launches += 1;
         trace_mark(h, 3, st);
         moe::TcGemmArgs a2 = a1;
         a2.k_blocks = h->F / 64;
@@ -378,21 +385,25 @@ moe_status run_experts(moe_handle* h, int64_t T, const void* x, const int32_t* t
         e = pair ? moe::launch_tc_gemm2_pair(h->tm_h, h->tm_w2, a2, h->num_sms, st)
                  : moe::launch_tc_gemm2(h->tm_h, h->tm_w2, a2, h->num_sms, st);
         if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
+        h->launches += 1;
         trace_mark(h, 4, st);
     } else {
         e = moe::launch_simt_gemm1(static_cast<const float*>(h->xp), static_cast<const float*>(w1),
                                    static_cast<const float*>(w3), static_cast<float*>(h->h),
                                    h->db.offsets, h->db.mblk_base, h->n, R, h->d, h->F, st);
         if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
+        h->launches += 1;
         trace_mark(h, 3, st);
         e = moe::launch_simt_gemm2(static_cast<const float*>(h->h), static_cast<const float*>(w2),
                                    static_cast<float*>(h->o), h->db.offsets, h->db.mblk_base, h->n,
                                    R, h->d, h->F, st);
         if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
+        h->launches += 1;
         trace_mark(h, 4, st);
     }
     e = moe::launch_combine(h->o, bf, h->db.token_row, topk_w, T, h->K, h->d, y, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+    h->launches += 1;
     trace_mark(h, 5, st);
     trace_finish_call(h);
     return MOE_OK;
@@ -516,6 +527,7 @@ moe_status moe_dispatch(moe_handle* h, int64_t T, const int32_t* topk_idx, int32
                                          h->dtype == MOE_BF16 ? moe::kTcBM : moe::kSimtBM, h->db, st,
                                          capacity_for(h, T));
     if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
+    h->launches += 3;
     struct {
         void* dst;
         const void* src;
@@ -571,9 +583,11 @@ moe_status moe_router_stats(moe_handle* h, int64_t T, const void* x, const float
         e = moe::launch_router_logits_simt(x, false, W_g, T, h->d, h->n, h->logits, st);
     }
     if (e != cudaSuccess) return cuda_fail(e, "router logits launch");
+    h->launches += h->dtype == MOE_BF16 ? 2 : 1;
     e = moe::launch_router_stats(h->logits, splits, T, h->n, h->K, topk_idx, alpha, h->stats_partial,
                                  h->stats_counts, f, P, aux, st);
     if (e != cudaSuccess) return cuda_fail(e, "router statistics launch");
+    h->launches += 2;
     return ok();
 }
 
@@ -646,6 +660,12 @@ moe_status moe_trace_end(moe_handle* h, double* stage_ms, int n_stages, int* cal
     }
     *calls = h->trace_calls;
     trace_free(h);
+    return ok();
+}
+
+moe_status moe_launch_count(moe_handle* h, int64_t* count) {
+    if (!h || !count) return fail(MOE_ERR_INVALID_ARG, "null argument");
+    *count = h->launches;
     return ok();
 }
 
