@@ -16,8 +16,9 @@ workload on its own GPU; no collective on the data path), timed with CUDA
 events on the launching stream, max over ranks.  `e2e` is the same metric
 through the C ABI with the step's activations copied from pinned host memory
 and y / topk_idx / topk_w copied back inside the timed region.  `roofline`
-reports the dominant kernel (per-stage CUDA events recorded by the library
-over the timed steps).  `cpu_baseline` times the fp64 oracle on a bounded
+reports the dominant kernel, timed by the library's per-stage CUDA events over
+a second run of the same K steps (events between the kernels would serialise
+their programmatic dependent launches in the headline run).  `cpu_baseline` times the fp64 oracle on a bounded
 sample of the same workload on this host's cores.
 
 --impl reference runs the oracle (the reference arm of this build) on the
@@ -321,12 +322,12 @@ def main():
     layer.sync_status(stream)
     counts = touched_experts(idx.cpu().numpy(), cfg.n)
 
-    # ---- device-timed region ----
+    # ---- device-timed region (no per-stage events: they would sit between
+    # the layer's kernels and serialise their programmatic dependent launches)
     sampler = ClockSampler(dev.index)
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    m.moe_trace_begin(layer.h, args.steps)
     launches0 = m.moe_launch_count(layer.h)
     sampler.start()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -337,13 +338,22 @@ def main():
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
     launches = m.moe_launch_count(layer.h) - launches0
-    stage_ms, traced = m.moe_trace_end(layer.h)
     if dist:
         dist.barrier()
     ms = ev0.elapsed_time(ev1) / args.steps
     layer.sync_status(stream)
     ms = max_over_ranks(ms, dist, dev)
     value = tokens_per_s(T, world, ms)
+
+    # ---- the same K steps again with the library's per-stage CUDA events,
+    # which time each kernel (the roofline's launch duration)
+    torch.cuda.synchronize(dev)
+    m.moe_trace_begin(layer.h, args.steps)
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize(dev)
+    stage_ms, traced = m.moe_trace_end(layer.h)
+    layer.sync_status(stream)
 
     # ---- end to end: pinned host activations in, y / routing out ----
     xh = x.cpu().pin_memory()

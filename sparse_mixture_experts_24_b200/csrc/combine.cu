@@ -20,6 +20,7 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const uint4* __restri
                                                            const float* __restrict__ topk_w,
                                                            int64_t T, int K, int vec_per_row,
                                                            uint4* __restrict__ y) {
+    griddep_wait();
     const int64_t total = T * vec_per_row;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
@@ -55,6 +56,7 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const uint4* __restri
         out.w = pack_bf16x2(acc[6], acc[7]);
         y[i] = out;
     }
+    griddep_launch_dependents();
 }
 
 __global__ void __launch_bounds__(256) combine_f32_kernel(const float4* __restrict__ O,
@@ -62,6 +64,7 @@ __global__ void __launch_bounds__(256) combine_f32_kernel(const float4* __restri
                                                           const float* __restrict__ topk_w,
                                                           int64_t T, int K, int vec_per_row,
                                                           float4* __restrict__ y) {
+    griddep_wait();
     const int64_t total = T * vec_per_row;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
@@ -81,6 +84,7 @@ __global__ void __launch_bounds__(256) combine_f32_kernel(const float4* __restri
         }
         y[i] = acc;
     }
+    griddep_launch_dependents();
 }
 
 cudaError_t launch_combine(const void* O, bool bf16, const int32_t* token_row, const float* topk_w,
@@ -91,10 +95,10 @@ cudaError_t launch_combine(const void* O, bool bf16, const int32_t* token_row, c
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     if (bf16)
-        combine_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        launch_k(combine_bf16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, 
             static_cast<const uint4*>(O), token_row, topk_w, T, K, d / 8, static_cast<uint4*>(y));
     else
-        combine_f32_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        launch_k(combine_f32_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, 
             static_cast<const float4*>(O), token_row, topk_w, T, K, d / 4, static_cast<float4*>(y));
     return cudaGetLastError();
 }

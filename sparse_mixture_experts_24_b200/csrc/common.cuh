@@ -207,6 +207,14 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, int a_mn, i
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
+// Programmatic dependent launch: wait until the previous kernel of the stream
+// has finished and its writes are visible (a no-op for a normal launch), and
+// let the next kernel start launching once this block's work is done.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // Clusters of two CTAs (tcgen05 cta_group::2)
 // ---------------------------------------------------------------------------

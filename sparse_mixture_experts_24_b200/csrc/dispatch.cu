@@ -33,6 +33,7 @@ __global__ void __launch_bounds__(kPairsPerBlock) rank_kernel(const int32_t* __r
                                                               int64_t R, int n,
                                                               int32_t* __restrict__ blockcounts,
                                                               int32_t* __restrict__ pair_rank) {
+    griddep_wait();
     __shared__ int32_t whist[kWarps][kMaxExperts];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     for (int i = tid; i < kWarps * kMaxExperts; i += kPairsPerBlock) (&whist[0][0])[i] = 0;
@@ -59,6 +60,7 @@ __global__ void __launch_bounds__(kPairsPerBlock) rank_kernel(const int32_t* __r
     }
     __syncthreads();
     if (p < R) pair_rank[p] = (e >= 0) ? whist[warp][e] + wrank : -1;
+    griddep_launch_dependents();
 }
 
 // Exclusive scan of one value per thread over a 256-thread block.
@@ -100,6 +102,7 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* __restrict__ blockco
                                                    int32_t* __restrict__ counts,
                                                    int32_t* __restrict__ offsets,
                                                    int32_t* __restrict__ mblk_base) {
+    griddep_wait();
     __shared__ int s_warp[8];
     __shared__ int32_t s_chunk[kScanSmemInts];
     const int e = threadIdx.x;
@@ -135,6 +138,7 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* __restrict__ blockco
         offsets[n] = off + total;
         mblk_base[n] = mbase + mb;
     }
+    griddep_launch_dependents();
 }
 
 __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict__ idx, int64_t R,
@@ -144,6 +148,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
                                                       const int32_t* __restrict__ pair_rank,
                                                       int32_t* __restrict__ row_token,
                                                       int32_t* __restrict__ token_row) {
+    griddep_wait();
     const int64_t p = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (p >= R) return;
     const int e = idx[p];
@@ -160,15 +165,127 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
     const int dest = offsets[e] + rank_in_expert;
     row_token[dest] = static_cast<int32_t>(p / K);
     token_row[p] = dest;
+    griddep_launch_dependents();
+}
+
+// Small batches (T*K <= kSmallDispatchPairs): the whole dispatch in one
+// 1024-thread block -- counts, capped offsets, M-block prefix, stable ranks
+// and the scatter -- with no global round trips between the steps.
+constexpr int kSmallWarps = 32;
+
+__global__ void __launch_bounds__(1024) dispatch_small_kernel(const int32_t* __restrict__ idx, int64_t R,
+                                                              int K, int n, int capacity, int bm,
+                                                              int32_t* __restrict__ counts,
+                                                              int32_t* __restrict__ offsets,
+                                                              int32_t* __restrict__ mblk_base,
+                                                              int32_t* __restrict__ row_token,
+                                                              int32_t* __restrict__ token_row) {
+    griddep_wait();
+    __shared__ int32_t whist[kSmallWarps][kMaxExperts];   // per-warp counts, then warp bases
+    __shared__ int32_t run[kMaxExperts];                  // pairs of each expert in earlier chunks
+    __shared__ int32_t s_off[kMaxExperts];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int e = tid; e < kMaxExperts; e += 1024) run[e] = 0;
+    // pass 1: per-expert totals -> capped counts, offsets, M-block prefix
+    for (int i = tid; i < kSmallWarps * kMaxExperts; i += 1024) (&whist[0][0])[i] = 0;
+    __syncthreads();
+    for (int64_t p = tid; p < R; p += 1024) {
+        const int e = idx[p];
+        if (e >= 0 && e < n) atomicAdd(&whist[0][e], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // lane l scans experts 8l .. 8l+7; a shuffle scan joins the lanes
+        int tot[8], mbs[8];
+        int lane_tot = 0, lane_mb = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane * 8 + i;
+            tot[i] = (e < n) ? min(whist[0][e], capacity) : 0;
+            mbs[i] = (tot[i] + bm - 1) / bm;
+            lane_tot += tot[i];
+            lane_mb += mbs[i];
+        }
+        int inc_tot = lane_tot, inc_mb = lane_mb;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int a = __shfl_up_sync(0xffffffffu, inc_tot, o);
+            const int b2 = __shfl_up_sync(0xffffffffu, inc_mb, o);
+            if (lane >= o) {
+                inc_tot += a;
+                inc_mb += b2;
+            }
+        }
+        int off = inc_tot - lane_tot, mbase = inc_mb - lane_mb;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane * 8 + i;
+            if (e < n) {
+                counts[e] = tot[i];
+                offsets[e] = off;
+                mblk_base[e] = mbase;
+                s_off[e] = off;
+            }
+            if (e == n - 1) {
+                offsets[n] = off + tot[i];
+                mblk_base[n] = mbase + mbs[i];
+            }
+            off += tot[i];
+            mbase += mbs[i];
+        }
+    }
+    // pass 2: stable ranks chunk by chunk (1024 pairs per chunk, in pair order)
+    for (int64_t c0 = 0; c0 < R; c0 += 1024) {
+        __syncthreads();
+        for (int i = tid; i < kSmallWarps * kMaxExperts; i += 1024) (&whist[0][0])[i] = 0;
+        __syncthreads();
+        const int64_t p = c0 + tid;
+        int e = (p < R) ? idx[p] : -1;
+        if (e < 0 || e >= n) e = -1;
+        const uint32_t peers = __match_any_sync(0xffffffffu, e);
+        const int wrank = __popc(peers & ((1u << lane) - 1u));
+        if (e >= 0 && wrank == 0) whist[warp][e] = __popc(peers);
+        __syncthreads();
+        for (int ex = tid; ex < n; ex += 1024) {
+            int acc = run[ex];
+            for (int w = 0; w < kSmallWarps; ++w) {
+                const int cnt = whist[w][ex];
+                whist[w][ex] = acc;
+                acc += cnt;
+            }
+            run[ex] = acc;
+        }
+        __syncthreads();
+        if (p < R) {
+            if (e < 0) {
+                token_row[p] = -1;
+            } else {
+                const int rank_in_expert = whist[warp][e] + wrank;
+                if (rank_in_expert >= capacity) {
+                    token_row[p] = -1;
+                } else {
+                    const int dest = s_off[e] + rank_in_expert;
+                    row_token[dest] = static_cast<int32_t>(p / K);
+                    token_row[p] = dest;
+                }
+            }
+        }
+    }
+    griddep_launch_dependents();
 }
 
 cudaError_t launch_dispatch(const int32_t* topk_idx, int64_t T, int K, int n, int bm,
                             const DispatchBufs& b, cudaStream_t st, int capacity) {
     const int64_t R = T * K;
+    if (R <= kSmallDispatchPairs) {
+        launch_k(dispatch_small_kernel, dim3(1), dim3(1024), 0, st, topk_idx, R, K, n, capacity, bm, b.counts, b.offsets,
+                                                  b.mblk_base, b.row_token, b.token_row);
+        return cudaGetLastError();
+    }
     const int nblk = static_cast<int>((R + kPairsPerBlock - 1) / kPairsPerBlock);
-    rank_kernel<<<nblk, kPairsPerBlock, 0, st>>>(topk_idx, R, n, b.blockcounts, b.pair_rank);
-    scan_kernel<<<1, 256, 0, st>>>(b.blockcounts, nblk, n, capacity, bm, b.counts, b.offsets, b.mblk_base);
-    scatter_kernel<<<static_cast<unsigned>((R + 255) / 256), 256, 0, st>>>(
+    launch_k(rank_kernel, dim3(nblk), dim3(kPairsPerBlock), 0, st, topk_idx, R, n, b.blockcounts, b.pair_rank);
+    launch_k(scan_kernel, dim3(1), dim3(256), 0, st, b.blockcounts, nblk, n, capacity, bm, b.counts, b.offsets, b.mblk_base);
+    launch_k(scatter_kernel, dim3(static_cast<unsigned>((R + 255) / 256)), dim3(256), 0, st, 
         topk_idx, R, K, n, capacity, b.offsets, b.blockcounts, b.pair_rank, b.row_token, b.token_row);
     return cudaGetLastError();
 }
@@ -177,6 +294,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ x
                                                      const int32_t* __restrict__ row_token,
                                                      int64_t R, int64_t T, int64_t vec_per_row,
                                                      uint4* __restrict__ xp) {
+    griddep_wait();
     const int64_t total = R * vec_per_row;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
@@ -187,6 +305,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ x
         if (t < 0 || t >= T) continue;  // a row no valid pair reached (bad expert ids)
         xp[i] = __ldg(x + t * vec_per_row + v);
     }
+    griddep_launch_dependents();
 }
 
 cudaError_t launch_gather(const void* x, const int32_t* row_token, int64_t R, int64_t T,
@@ -195,7 +314,7 @@ cudaError_t launch_gather(const void* x, const int32_t* row_token, int64_t R, in
     const int64_t cap = static_cast<int64_t>(num_sms) * 16;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    gather_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+    launch_k(gather_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, 
         static_cast<const uint4*>(x), row_token, R, T, row_bytes / 16, static_cast<uint4*>(xp));
     return cudaGetLastError();
 }

@@ -135,6 +135,7 @@ extern "C" MOE_API moe_status moe_dispatch_noalloc(int64_t T, int n, int K, cons
     b.offsets = offsets;
     b.row_token = row_token;
     b.token_row = token_row;
+    moe::chain_begin();
     cudaError_t e = moe::launch_dispatch(topk_idx, T, K, n, moe::kTcBM, b,
                                          reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {

@@ -42,6 +42,7 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const float* __restrict_
                                                         const int32_t* __restrict__ offsets,
                                                         const int32_t* __restrict__ mblk_base,
                                                         int n, int Kdim, int Ncols) {
+    griddep_wait();
     __shared__ float As[kSK][kSM + 4];
     __shared__ float Bs0[kSK][kSN + 4];
     __shared__ float Bs1[kSK][kSN + 4];
@@ -107,6 +108,7 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const float* __restrict_
             C[static_cast<int64_t>(row0 + r) * Ncols + c] = v;
         }
     }
+    griddep_launch_dependents();
 }
 
 static unsigned mblk_cap(int64_t R, int n) {
@@ -117,7 +119,7 @@ cudaError_t launch_simt_gemm1(const float* xp, const float* w1, const float* w3,
                               const int32_t* offsets, const int32_t* mblk_base, int n, int64_t R,
                               int d, int F, cudaStream_t st) {
     dim3 grid(mblk_cap(R, n), static_cast<unsigned>((F + kSN - 1) / kSN));
-    simt_gemm_kernel<true><<<grid, 256, 0, st>>>(xp, w1, w3, h, offsets, mblk_base, n, d, F);
+    launch_k(simt_gemm_kernel<true>, dim3(grid), dim3(256), 0, st, xp, w1, w3, h, offsets, mblk_base, n, d, F);
     return cudaGetLastError();
 }
 
@@ -125,7 +127,7 @@ cudaError_t launch_simt_gemm2(const float* h, const float* w2, float* o, const i
                               const int32_t* mblk_base, int n, int64_t R, int d, int F,
                               cudaStream_t st) {
     dim3 grid(mblk_cap(R, n), static_cast<unsigned>((d + kSN - 1) / kSN));
-    simt_gemm_kernel<false><<<grid, 256, 0, st>>>(h, w2, nullptr, o, offsets, mblk_base, n, F, d);
+    launch_k(simt_gemm_kernel<false>, dim3(grid), dim3(256), 0, st, h, w2, nullptr, o, offsets, mblk_base, n, F, d);
     return cudaGetLastError();
 }
 

@@ -104,10 +104,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lane = threadIdx.x & 31;
     const int n = args.n;
 
-    for (int i = threadIdx.x; i <= n; i += kThreads) {
-        tail->off[i] = args.offsets[i];
-        tail->mblk[i] = args.mblk_base[i];
-    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(smem_u32(&tail->full[s]), 1);
@@ -129,6 +125,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         tmem_alloc(smem_u32(&tail->tmem_base), kTmemCols);
         tmem_relinquish();
+    }
+    // everything above overlaps the previous kernel; its outputs (segment
+    // offsets, the A operand) are read only after this wait
+    griddep_wait();
+    for (int i = threadIdx.x; i <= n; i += kThreads) {
+        tail->off[i] = args.offsets[i];
+        tail->mblk[i] = args.mblk_base[i];
     }
     tc_fence_before();
     __syncthreads();
@@ -302,6 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     tc_fence_before();
     __syncthreads();
+    griddep_launch_dependents();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, kTmemCols);
@@ -321,7 +325,7 @@ static cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb0, cons
     cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<kSwiGLU>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    tc_gemm_kernel<kSwiGLU><<<grid_for(a, num_sms), kThreads, kSmemBytes, st>>>(ta, tb0, tb1, a);
+    launch_k(tc_gemm_kernel<kSwiGLU>, dim3(grid_for(a, num_sms)), dim3(kThreads), kSmemBytes, st, ta, tb0, tb1, a);
     return cudaGetLastError();
 }
 

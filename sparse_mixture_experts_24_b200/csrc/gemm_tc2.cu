@@ -105,10 +105,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const int cid = static_cast<int>(cluster_id_x());
     const int ncl = static_cast<int>(nclusters_x());
 
-    for (int i = threadIdx.x; i <= n; i += kPairThreads) {
-        tail->off[i] = args.offsets[i];
-        tail->mblk[i] = args.mblk_base[i];
-    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < kPairStages; ++s) {
             mbar_init(smem_u32(&tail->full[s]), 1);
@@ -130,6 +126,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     if (warp == 1) {
         tmem_alloc_pair(smem_u32(&tail->tmem_base), kPairTmemCols);
         tmem_relinquish_pair();
+    }
+    griddep_wait();  // segment offsets and the A operand come from earlier kernels
+    for (int i = threadIdx.x; i <= n; i += kPairThreads) {
+        tail->off[i] = args.offsets[i];
+        tail->mblk[i] = args.mblk_base[i];
     }
     tc_fence_before();
     __syncthreads();
@@ -310,6 +311,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     __syncwarp();
     __syncthreads();
     cluster_sync();  // no remote arrive or commit may target a CTA that has left
+    griddep_launch_dependents();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc_pair(tmem_base, kPairTmemCols);
@@ -331,13 +333,16 @@ static cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb0, co
     cfg.blockDim = dim3(kPairThreads);
     cfg.dynamicSmemBytes = kPairSmemBytes;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = (g_chain_started && pdl_enabled()) ? 2 : 1;
+    g_chain_started = true;
     return cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<kSwiGLU>, ta, tb0, tb1, a);
 }
 

@@ -7,6 +7,31 @@
 
 namespace moe {
 
+// Kernels launched by one API call form a chain on its stream; every launch
+// after the first carries the programmatic-stream-serialization attribute, so
+// it can be scheduled while its predecessor drains (each kernel waits with
+// griddepcontrol.wait before touching memory).  MOE_PDL=0 turns this off.
+bool pdl_enabled();
+extern thread_local bool g_chain_started;
+inline void chain_begin() { g_chain_started = false; }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                            Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = (g_chain_started && pdl_enabled()) ? 1 : 0;
+    g_chain_started = true;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Rows of one M-block of the tensor-core GEMMs and of the CUDA-core GEMMs.
 constexpr int kTcBM = 128;
 constexpr int kSimtBM = 64;
@@ -53,6 +78,9 @@ struct DispatchBufs {
 // the GEMM that consumes the segments; capacity = most pairs one expert takes
 // (kNoCapacity: all).
 constexpr int kNoCapacity = 2147483647;
+// Up to this many pairs the dispatch is one single-block kernel (else three).
+constexpr int kSmallDispatchPairs = 4096;
+inline int dispatch_kernel_count(int64_t pairs) { return pairs <= kSmallDispatchPairs ? 1 : 3; }
 cudaError_t launch_dispatch(const int32_t* topk_idx, int64_t T, int K, int n, int bm,
                             const DispatchBufs& b, cudaStream_t st, int capacity = kNoCapacity);
 

@@ -35,6 +35,17 @@ moe_status ok() {
 
 }  // namespace
 
+namespace moe {
+thread_local bool g_chain_started = false;
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char* e = getenv("MOE_PDL");
+        return !(e && strcmp(e, "0") == 0);
+    }();
+    return on;
+}
+}  // namespace moe
+
 namespace moe_api_detail {
 // Lets other translation units of the library set the moe_last_error() text.
 void set_last_error(const char* msg) { snprintf(g_err, sizeof g_err, "%s", msg); }
@@ -339,7 +350,7 @@ moe_status run_experts(moe_handle* h, int64_t T, const void* x, const int32_t* t
                                          pair ? moe::kTcPairBM : (bf ? moe::kTcBM : moe::kSimtBM),
                                          h->db, st, capacity_for(h, T));
     if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
-    h->launches += 3;  // rank, scan, scatter
+    h->launches += moe::dispatch_kernel_count(R);
     trace_mark(h, 1, st);
     e = moe::launch_gather(x, h->db.row_token, R, T, static_cast<int64_t>(h->d) * h->esize(), h->xp,
                            h->num_sms, st);
@@ -455,6 +466,7 @@ moe_status moe_route(moe_handle* h, int64_t T, const void* x, const float* W_g, 
     s = prepare(h, T);
     if (s != MOE_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    moe::chain_begin();
     s = run_router(h, T, x, W_g, topk_idx, topk_w, st);
     return s == MOE_OK ? ok() : s;
 }
@@ -476,6 +488,7 @@ moe_status moe_forward(moe_handle* h, int64_t T, const void* x, const float* W_g
     s = prepare(h, T);
     if (s != MOE_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    moe::chain_begin();
     trace_mark(h, -1, st);
     s = run_router(h, T, x, W_g, topk_idx, topk_w, st);
     if (s != MOE_OK) return s;
@@ -500,6 +513,7 @@ moe_status moe_forward_with_routing(moe_handle* h, int64_t T, const void* x,
     s = prepare(h, T);
     if (s != MOE_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    moe::chain_begin();
     trace_mark(h, -1, st);
     trace_mark(h, 0, st);
     s = run_experts(h, T, x, topk_idx, topk_w, w1, w3, w2, y, st);
@@ -522,12 +536,13 @@ moe_status moe_dispatch(moe_handle* h, int64_t T, const int32_t* topk_idx, int32
     s = prepare(h, T);
     if (s != MOE_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    moe::chain_begin();
     const int64_t R = T * h->K;
     cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n,
                                          h->dtype == MOE_BF16 ? moe::kTcBM : moe::kSimtBM, h->db, st,
                                          capacity_for(h, T));
     if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
-    h->launches += 3;
+    h->launches += moe::dispatch_kernel_count(R);
     struct {
         void* dst;
         const void* src;
@@ -568,6 +583,7 @@ moe_status moe_router_stats(moe_handle* h, int64_t T, const void* x, const float
     s = prepare(h, T);
     if (s != MOE_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    moe::chain_begin();
     int splits = 1;
     cudaError_t e;
     if (h->dtype == MOE_BF16) {

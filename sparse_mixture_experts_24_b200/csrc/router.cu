@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(256) router_small_kernel(const XT* __restrict_
                                                            int d, int n, int K,
                                                            int32_t* __restrict__ topk_idx,
                                                            float* __restrict__ topk_w) {
+    griddep_wait();
     using C = SmallRouterCfg<NE>;
     __shared__ __align__(16) float Ws[NE * C::kPitch];
     const int lane = threadIdx.x & 31;
@@ -179,6 +180,7 @@ __global__ void __launch_bounds__(256) router_small_kernel(const XT* __restrict_
             if (t0 + t < T)
                 topk_softmax_regs<NE>(acc[t], n, K, topk_idx + (t0 + t) * K, topk_w + (t0 + t) * K);
     }
+    griddep_launch_dependents();
 }
 
 // n <= 32, few tokens: one 256-thread block per token.  Thread i covers rows
@@ -191,6 +193,7 @@ __global__ void __launch_bounds__(256) router_token_kernel(const XT* __restrict_
                                                            int d, int n, int K,
                                                            int32_t* __restrict__ topk_idx,
                                                            float* __restrict__ topk_w) {
+    griddep_wait();
     __shared__ float red[8][NE];
     const int64_t t = blockIdx.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -241,6 +244,7 @@ __global__ void __launch_bounds__(256) router_token_kernel(const XT* __restrict_
         }
         topk_softmax_regs<NE>(L, n, K, topk_idx + t * K, topk_w + t * K);
     }
+    griddep_launch_dependents();
 }
 
 // ---- n > 32: tiled logits GEMM ---------------------------------------------
@@ -253,6 +257,7 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const XT* __restrict
                                                             const float* __restrict__ Wg,
                                                             int64_t T, int d, int n,
                                                             float* __restrict__ logits) {
+    griddep_wait();
     __shared__ float xs[kRK][kRT + 4];
     __shared__ float ws[kRK][kRE + 4];
     const int tid = threadIdx.x;
@@ -310,6 +315,7 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const XT* __restrict
             if (e < n) logits[tok * n + e] = acc[i][j];
         }
     }
+    griddep_launch_dependents();
 }
 
 // One warp per token: lane l holds logits l, l+32, ... (up to 8 per lane),
@@ -318,6 +324,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
                                                           int splits, int64_t T, int n, int K,
                                                           int32_t* __restrict__ topk_idx,
                                                           float* __restrict__ topk_w) {
+    griddep_wait();
     const int lane = threadIdx.x & 31;
     const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     if (t >= T) return;
@@ -376,11 +383,12 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
         const float inv = 1.f / s;
         for (int k = 0; k < K; ++k) topk_w[t * K + k] *= inv;
     }
+    griddep_launch_dependents();
 }
 
 cudaError_t launch_router_topk(const float* logits, int splits, int64_t T, int n, int K,
                                int32_t* topk_idx, float* topk_w, cudaStream_t st) {
-    router_topk_kernel<<<dim3(static_cast<unsigned>((T + 7) / 8)), 256, 0, st>>>(logits, splits, T, n,
+    launch_k(router_topk_kernel, dim3(dim3(static_cast<unsigned>((T + 7) / 8))), dim3(256), 0, st, logits, splits, T, n,
                                                                                  K, topk_idx, topk_w);
     return cudaGetLastError();
 }
@@ -390,7 +398,7 @@ static void launch_small(const XT* x, const float* Wg, int64_t T, int d, int n, 
                          float* w, int num_sms, cudaStream_t st) {
     if (T < kTokenKernelMaxT) {
         // few tokens: a whole block per token keeps every SM's loads in flight
-        router_token_kernel<XT, NE><<<static_cast<unsigned>(T), 256, 0, st>>>(x, Wg, T, d, n, K, idx, w);
+        launch_k(router_token_kernel<XT, NE>, dim3(static_cast<unsigned>(T)), dim3(256), 0, st, x, Wg, T, d, n, K, idx, w);
         return;
     }
     // many tokens: share each staged W_g chunk between TPW tokens per warp,
@@ -404,11 +412,11 @@ static void launch_small(const XT* x, const float* Wg, int64_t T, int d, int n, 
     const int64_t blocks = (T + 8 * tpw - 1) / (8 * tpw);
     const unsigned g = static_cast<unsigned>(blocks);
     if (tpw == 4)
-        router_small_kernel<XT, NE, (kTpwMax >= 4 ? 4 : 1)><<<g, 256, 0, st>>>(x, Wg, T, d, n, K, idx, w);
+        launch_k(router_small_kernel<XT, NE, (kTpwMax >= 4 ? 4 : 1)>, dim3(g), dim3(256), 0, st, x, Wg, T, d, n, K, idx, w);
     else if (tpw == 2)
-        router_small_kernel<XT, NE, (kTpwMax >= 2 ? 2 : 1)><<<g, 256, 0, st>>>(x, Wg, T, d, n, K, idx, w);
+        launch_k(router_small_kernel<XT, NE, (kTpwMax >= 2 ? 2 : 1)>, dim3(g), dim3(256), 0, st, x, Wg, T, d, n, K, idx, w);
     else
-        router_small_kernel<XT, NE, 1><<<g, 256, 0, st>>>(x, Wg, T, d, n, K, idx, w);
+        launch_k(router_small_kernel<XT, NE, 1>, dim3(g), dim3(256), 0, st, x, Wg, T, d, n, K, idx, w);
 }
 
 template <typename XT>
@@ -428,8 +436,8 @@ static cudaError_t launch_router_t(const XT* x, const float* Wg, int64_t T, int 
         return cudaGetLastError();
     }
     dim3 g1(static_cast<unsigned>((T + kRT - 1) / kRT), static_cast<unsigned>((n + kRE - 1) / kRE));
-    router_logits_kernel<XT><<<g1, 256, 0, st>>>(x, Wg, T, d, n, logits_ws);
-    router_topk_kernel<<<dim3(static_cast<unsigned>((T + 7) / 8)), 256, 0, st>>>(logits_ws, 1, T, n, K,
+    launch_k(router_logits_kernel<XT>, dim3(g1), dim3(256), 0, st, x, Wg, T, d, n, logits_ws);
+    launch_k(router_topk_kernel, dim3(dim3(static_cast<unsigned>((T + 7) / 8))), dim3(256), 0, st, logits_ws, 1, T, n, K,
                                                                                  idx, w);
     return cudaGetLastError();
 }
@@ -438,10 +446,10 @@ cudaError_t launch_router_logits_simt(const void* x, bool x_bf16, const float* W
                                       int n, float* logits, cudaStream_t st) {
     dim3 g1(static_cast<unsigned>((T + kRT - 1) / kRT), static_cast<unsigned>((n + kRE - 1) / kRE));
     if (x_bf16)
-        router_logits_kernel<uint16_t><<<g1, 256, 0, st>>>(static_cast<const uint16_t*>(x), Wg, T, d, n,
+        launch_k(router_logits_kernel<uint16_t>, dim3(g1), dim3(256), 0, st, static_cast<const uint16_t*>(x), Wg, T, d, n,
                                                            logits);
     else
-        router_logits_kernel<float><<<g1, 256, 0, st>>>(static_cast<const float*>(x), Wg, T, d, n, logits);
+        launch_k(router_logits_kernel<float>, dim3(g1), dim3(256), 0, st, static_cast<const float*>(x), Wg, T, d, n, logits);
     return cudaGetLastError();
 }
 

@@ -28,6 +28,7 @@ namespace moe {
 // W_g [d][n] fp32 -> parts [3][npad][d] bf16 (rows n..npad-1 are zero).
 __global__ void __launch_bounds__(256) wg_split_kernel(const float* __restrict__ Wg, int d, int n,
                                                        int npad, uint16_t* __restrict__ parts) {
+    griddep_wait();
     const int64_t total = static_cast<int64_t>(npad) * d;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -43,6 +44,7 @@ __global__ void __launch_bounds__(256) wg_split_kernel(const float* __restrict__
         parts[total + i] = __bfloat16_as_ushort(mid);
         parts[2 * total + i] = __bfloat16_as_ushort(lo);
     }
+    griddep_launch_dependents();
 }
 
 constexpr int kRtThreads = 192;
@@ -109,6 +111,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         tmem_alloc(smem_u32(&tail->tmem_base), static_cast<uint32_t>(tmem_cols));
         tmem_relinquish();
     }
+    griddep_wait();  // the W_g parts come from the previous kernel
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -198,6 +201,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         }
     }
     __syncthreads();
+    griddep_launch_dependents();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, static_cast<uint32_t>(tmem_cols));
@@ -216,7 +220,7 @@ cudaError_t launch_router_logits_tc(const CUtensorMap& tm_x, const CUtensorMap& 
     const int64_t total = static_cast<int64_t>(npad) * d;
     int64_t sb = (total + 255) / 256;
     if (sb > static_cast<int64_t>(num_sms) * 8) sb = static_cast<int64_t>(num_sms) * 8;
-    wg_split_kernel<<<static_cast<unsigned>(sb), 256, 0, st>>>(Wg, d, n, npad, parts);
+    launch_k(wg_split_kernel, dim3(static_cast<unsigned>(sb)), dim3(256), 0, st, Wg, d, n, npad, parts);
     const int smem = router_tc_smem_bytes(n);
     cudaError_t e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -228,7 +232,7 @@ cudaError_t launch_router_logits_tc(const CUtensorMap& tm_x, const CUtensorMap& 
     if (splits > kb_total / 8) splits = kb_total / 8;
     if (splits < 1) splits = 1;
     dim3 grid(static_cast<unsigned>(mtiles), static_cast<unsigned>(splits));
-    router_tc_kernel<<<grid, kRtThreads, smem, st>>>(tm_x, tm_w, T, d, n, npad, rt_tmem_cols(npad),
+    launch_k(router_tc_kernel, dim3(grid), dim3(kRtThreads), smem, st, tm_x, tm_w, T, d, n, npad, rt_tmem_cols(npad),
                                                      logits, status);
     *splits_out = splits;
     return cudaGetLastError();

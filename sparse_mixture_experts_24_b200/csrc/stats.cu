@@ -22,6 +22,7 @@ __global__ void __launch_bounds__(256) stats_partial_kernel(const float* __restr
                                                             const int32_t* __restrict__ idx,
                                                             float* __restrict__ partial,
                                                             int32_t* __restrict__ counts) {
+    griddep_wait();
     __shared__ float red[8][256];
     __shared__ int32_t hist[256];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -79,6 +80,7 @@ __global__ void __launch_bounds__(256) stats_partial_kernel(const float* __restr
         partial[static_cast<int64_t>(blockIdx.x) * n + e] = s;
         if (hist[e]) atomicAdd(&counts[e], hist[e]);
     }
+    griddep_launch_dependents();
 }
 
 __global__ void __launch_bounds__(256) stats_final_kernel(const float* __restrict__ partial, int nblk,
@@ -86,6 +88,7 @@ __global__ void __launch_bounds__(256) stats_final_kernel(const float* __restric
                                                           const int32_t* __restrict__ counts,
                                                           float* __restrict__ f, float* __restrict__ P,
                                                           float* __restrict__ aux) {
+    griddep_wait();
     __shared__ float fp[256];
     const int e = threadIdx.x;
     float prod = 0.f;
@@ -105,6 +108,7 @@ __global__ void __launch_bounds__(256) stats_final_kernel(const float* __restric
         for (int i = 0; i < n; ++i) s += fp[i];
         aux[0] = alpha * static_cast<float>(n) * s;
     }
+    griddep_launch_dependents();
 }
 
 cudaError_t launch_router_stats(const float* logits, int splits, int64_t T, int n, int K,
@@ -113,8 +117,8 @@ cudaError_t launch_router_stats(const float* logits, int splits, int64_t T, int 
     const int nblk = static_cast<int>((T + kStatsTokens - 1) / kStatsTokens);
     cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * n, st);
     if (e != cudaSuccess) return e;
-    stats_partial_kernel<<<nblk, 256, 0, st>>>(logits, splits, T, n, K, topk_idx, partial, counts);
-    stats_final_kernel<<<1, 256, 0, st>>>(partial, nblk, T, n, K, alpha, counts, f, P, aux);
+    launch_k(stats_partial_kernel, dim3(nblk), dim3(256), 0, st, logits, splits, T, n, K, topk_idx, partial, counts);
+    launch_k(stats_final_kernel, dim3(1), dim3(256), 0, st, partial, nblk, T, n, K, alpha, counts, f, P, aux);
     return cudaGetLastError();
 }
 
