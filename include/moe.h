@@ -242,6 +242,19 @@ MOE_API moe_status moe_dispatch_noalloc(int64_t T, int n, int K, const int32_t *
                                         int32_t *counts, int32_t *offsets, int32_t *row_token,
                                         int32_t *token_row, moe_stream_t stream);
 
+/*
+ * Self-test of failure detection (the pages have no counterpart).  Launches
+ * one kernel whose bounded wait -- the same helper every pipelined kernel of
+ * this library waits through -- is on a barrier nothing ever completes, with
+ * a budget of budget_us microseconds.  The wait gives up, sets the handle's
+ * status flag and the kernel returns normally; the next moe_sync_status then
+ * returns MOE_ERR_TIMEOUT and clears the flag.  Nothing faults or hangs, and
+ * the context stays usable.
+ *   Errors: MOE_ERR_INVALID_ARG (null handle, budget_us outside [1, 10^6]),
+ *   MOE_ERR_UNSUPPORTED, MOE_ERR_ALLOC, MOE_ERR_CUDA.
+ */
+MOE_API moe_status moe_selftest_timeout(moe_handle *h, int budget_us, moe_stream_t stream);
+
 /* Number of CUDA kernels this handle has launched so far (all entry points). */
 MOE_API moe_status moe_launch_count(moe_handle *h, int64_t *count);
 

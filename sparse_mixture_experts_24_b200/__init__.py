@@ -54,6 +54,7 @@ lib.moe_workspace_view.argtypes = [_vp, ctypes.c_char_p, ctypes.POINTER(_vp), ct
 lib.moe_sync_status.argtypes = [_vp, _vp]
 lib.moe_destroy.argtypes = [_vp]
 lib.moe_trace_begin.argtypes = [_vp, _int]
+lib.moe_selftest_timeout.argtypes = [_vp, _int, _vp]
 lib.moe_launch_count.argtypes = [_vp, ctypes.POINTER(_i64)]
 lib.moe_set_capacity_factor.argtypes = [_vp, ctypes.c_double]
 lib.moe_router_stats.argtypes = [_vp, _i64, _vp, _vp, _vp, ctypes.c_float, _vp, _vp, _vp, _vp]
@@ -64,14 +65,14 @@ lib.moe_version.restype = ctypes.c_char_p
 for _f in ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
            "moe_forward_with_routing", "moe_workspace_view", "moe_sync_status", "moe_destroy",
            "moe_trace_begin", "moe_trace_end", "moe_dispatch_noalloc", "moe_set_capacity_factor",
-           "moe_router_stats", "moe_launch_count"):
+           "moe_router_stats", "moe_launch_count", "moe_selftest_timeout"):
     getattr(lib, _f).restype = _int
 
 EXPORTED = ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
             "moe_forward_with_routing", "moe_workspace_view", "moe_sync_status", "moe_destroy",
             "moe_last_error", "moe_version", "moe_trace_begin", "moe_trace_end",
             "moe_dispatch_noalloc", "moe_set_capacity_factor", "moe_router_stats",
-            "moe_launch_count")
+            "moe_launch_count", "moe_selftest_timeout")
 
 TRACE_STAGES = ("router", "dispatch", "gather", "gemm1", "gemm2", "combine")
 
@@ -183,6 +184,10 @@ def moe_trace_end(h):
     calls = _int()
     _check(lib.moe_trace_end(h, ms, len(TRACE_STAGES), ctypes.byref(calls)), "moe_trace_end")
     return dict(zip(TRACE_STAGES, list(ms))), calls.value
+
+
+def moe_selftest_timeout(h, budget_us: int = 1000, stream=None) -> None:
+    _check(lib.moe_selftest_timeout(h, budget_us, _stream(stream)), "moe_selftest_timeout")
 
 
 def moe_launch_count(h) -> int:

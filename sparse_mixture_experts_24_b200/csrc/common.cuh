@@ -17,6 +17,7 @@ enum : int {
     kStatusTimeoutEmpty = 2,     // waited too long for the MMA to free a stage
     kStatusTimeoutAccum = 4,     // waited too long for an accumulator buffer
     kStatusTimeoutDrain = 8,     // waited too long while draining at exit
+    kStatusSelfTest = 16,        // the self-test's wait ran out (as it should)
 };
 
 // About 2 s at the B200's 1.9 GHz: far beyond any legitimate wait in these
@@ -80,12 +81,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait until the phase of `bar` with parity `parity` has completed, for at
 // most kWaitBudgetCycles.  On timeout set `flag` in *status and return false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* status, int flag) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* status, int flag,
+                                          long long budget = kWaitBudgetCycles) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (clock64() - t0 > kWaitBudgetCycles) {
+        if (clock64() - t0 > budget) {
             if (status) atomicOr(status, flag);
             return false;
         }

@@ -108,6 +108,10 @@ cudaError_t launch_gather(const void* x, const int32_t* row_token, int64_t R, in
 cudaError_t launch_combine(const void* O, bool bf16, const int32_t* token_row, const float* topk_w,
                            int64_t T, int K, int d, void* y, int num_sms, cudaStream_t st);
 
+// One thread waits on an mbarrier nothing arrives at, with the given budget;
+// sets kStatusSelfTest in *status when the wait runs out.
+cudaError_t launch_bounded_wait_probe(int* status, long long budget_cycles, cudaStream_t st);
+
 // CUDA-core fp32 grouped GEMMs (fp32 handles).
 //   H[r] = silu(Xp[r] . w1[e]) * (Xp[r] . w3[e]) for rows r of expert e
 cudaError_t launch_simt_gemm1(const float* xp, const float* w1, const float* w3, float* h,

@@ -679,6 +679,24 @@ moe_status moe_trace_end(moe_handle* h, double* stage_ms, int n_stages, int* cal
     return ok();
 }
 
+moe_status moe_selftest_timeout(moe_handle* h, int budget_us, moe_stream_t stream) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "null handle");
+    if (budget_us < 1 || budget_us > 1000000)
+        return fail(MOE_ERR_INVALID_ARG, "budget_us = %d outside [1, 1000000]", budget_us);
+    moe_status s = prepare(h, 1);
+    if (s != MOE_OK) return s;
+    int clk_khz = 0;
+    cudaDeviceGetAttribute(&clk_khz, cudaDevAttrClockRate, h->device);
+    if (clk_khz <= 0) clk_khz = 2000000;
+    const long long budget = static_cast<long long>(budget_us) * clk_khz / 1000;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    moe::chain_begin();
+    cudaError_t e = moe::launch_bounded_wait_probe(h->status, budget, st);
+    if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+    h->launches += 1;
+    return ok();
+}
+
 moe_status moe_launch_count(moe_handle* h, int64_t* count) {
     if (!h || !count) return fail(MOE_ERR_INVALID_ARG, "null argument");
     *count = h->launches;
