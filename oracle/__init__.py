@@ -14,6 +14,7 @@ bf16 bit patterns stored as uint16, and are widened exactly to double):
   dispatch(idx, n)                      -> counts, offsets, row_token, token_row
   dispatch_capacity(idx, n, C)          -> the same with at most C pairs per expert
   router_stats(x, W_g, idx, alpha)      -> f [n], P [n], aux (load-balancing statistics)
+  expert_choice(x, W_g, w1, w3, w2, C)  -> y, sel_token [n][C], sel_gate [n][C]
   silu(z)                               -> z * sigmoid(z) in double
 
 Sources: the layer equation of "Mixtral of Experts" section 2.1 (flash-card
@@ -63,13 +64,15 @@ def _bind(L):
     L.oracle_router_stats.argtypes = [i64, i32, i32, i32, vp, i32, vp, i32, vp, ctypes.c_double,
                                       vp, vp, vp]
     L.oracle_dispatch_capacity.argtypes = [i64, i32, i32, vp, i64, vp, vp, vp, vp]
+    L.oracle_expert_choice.argtypes = [i64, i32, i32, i32, i64, vp, i32, vp, i32, vp, vp, vp, i32,
+                                       vp, vp, vp]
     L.oracle_silu.argtypes = [ctypes.c_double]
     L.oracle_silu.restype = ctypes.c_double
     L.oracle_num_threads.restype = ctypes.c_int
     L.oracle_set_num_threads.argtypes = [ctypes.c_int]
     for f in ("oracle_router", "oracle_expert", "oracle_forward_with_routing",
               "oracle_moe_forward", "oracle_dispatch", "oracle_router_stats",
-              "oracle_dispatch_capacity"):
+              "oracle_dispatch_capacity", "oracle_expert_choice"):
         getattr(L, f).restype = ctypes.c_int
     return L
 
@@ -206,6 +209,21 @@ class Oracle:
         return counts, offsets, row_token[:T * K], token_row[:T * K].reshape(T, K)
 
 
+    def expert_choice(self, x, W_g, w1, w3, w2, C: int):
+        """-> y [T,d], sel_token [n,C] (ascending tokens), sel_gate [n,C]."""
+        x, W_g, w1, w3, w2 = _c(x), _c(W_g), _c(w1), _c(w3), _c(w2)
+        T, d = x.shape
+        n, d2, F = w1.shape
+        assert d == d2 and W_g.shape == (d, n)
+        y = np.empty((T, d), np.float64)
+        sel = np.empty((n, C), np.int64)
+        gate = np.empty((n, C), np.float64)
+        _check(self.L.oracle_expert_choice(T, d, F, n, int(C), _p(x), _dt(x), _p(W_g), _dt(W_g),
+                                           _p(w1), _p(w3), _p(w2), _dt(w1), _p(y), _p(sel), _p(gate)),
+               "expert_choice")
+        return y, sel, gate
+
+
 _default = None
 
 
@@ -254,3 +272,7 @@ def router_stats(x, W_g, idx, alpha: float):
 
 def dispatch_capacity(idx, n: int, capacity: int):
     return default().dispatch_capacity(idx, n, capacity)
+
+
+def expert_choice(x, W_g, w1, w3, w2, C: int):
+    return default().expert_choice(x, W_g, w1, w3, w2, C)

@@ -387,3 +387,93 @@ int oracle_dispatch_capacity(int64_t T, int n, int K, const int32_t *idx, int64_
     offsets[n] = row;
     return 0;
 }
+
+/*
+ * Expert-choice routing ("Mixtral of Experts? Mixture of Experts? Try to
+ * explain Mixtral 8x7B", section "How Experts Are Chosen", item 2: experts
+ * choose which tokens to process, each with a fixed capacity).  Reading taken:
+ *   S[t][e] = softmax over the n experts of the logits x_t . W_g;
+ *   expert e keeps the C tokens with the largest S[.][e] (equal scores: lower
+ *   token index first), listed in sel_token[e][0..C) by ascending token, with
+ *   sel_gate[e][j] = S[token][e];
+ *   y[t] = sum over the experts e that kept t (ascending e) of S[t][e] * SwiGLU_e(x_t);
+ *   a token no expert kept gets y[t] = 0.
+ * Requires 1 <= C <= T.
+ */
+static const double *g_sort_S; /* qsort context: one expert's column */
+static int g_sort_n, g_sort_e;
+
+static int cmp_score_desc_token_asc(const void *a, const void *b)
+{
+    int64_t ta = *(const int64_t *)a, tb = *(const int64_t *)b;
+    double sa = g_sort_S[ta * g_sort_n + g_sort_e], sb = g_sort_S[tb * g_sort_n + g_sort_e];
+    if (sa > sb) return -1;
+    if (sa < sb) return 1;
+    return (ta < tb) ? -1 : (ta > tb);
+}
+
+static int cmp_i64(const void *a, const void *b)
+{
+    int64_t x = *(const int64_t *)a, y = *(const int64_t *)b;
+    return (x < y) ? -1 : (x > y);
+}
+
+int oracle_expert_choice(int64_t T, int d, int F, int n, int64_t C, const void *x, int x_dt,
+                         const void *Wg, int wg_dt, const void *w1, const void *w3, const void *w2,
+                         int w_dt, double *y, int64_t *sel_token, double *sel_gate)
+{
+    if (T <= 0 || d <= 0 || F <= 0 || n <= 0 || C < 1 || C > T || !x || !Wg || !w1 || !w3 || !w2 ||
+        !y || !sel_token || !sel_gate || !dt_ok(x_dt) || !dt_ok(wg_dt) || !dt_ok(w_dt))
+        return -1;
+    double *S = (double *)malloc(sizeof(double) * (size_t)T * n);
+    int64_t *order = (int64_t *)malloc(sizeof(int64_t) * (size_t)T);
+    double *a = (double *)malloc(sizeof(double) * (size_t)F);
+    double *b = (double *)malloc(sizeof(double) * (size_t)F);
+    double *o = (double *)malloc(sizeof(double) * (size_t)d);
+    if (!S || !order || !a || !b || !o) {
+        free(S); free(order); free(a); free(b); free(o);
+        return -1;
+    }
+    /* router probabilities: softmax over all n logits of each token */
+    for (int64_t t = 0; t < T; ++t) {
+        double m = 0.0;
+        for (int e = 0; e < n; ++e) {
+            double s = 0.0;
+            for (int j = 0; j < d; ++j)
+                s += elem(x, x_dt, (size_t)t * d + j) * elem(Wg, wg_dt, (size_t)j * n + e);
+            S[t * n + e] = s;
+            if (e == 0 || s > m) m = s;
+        }
+        double z = 0.0;
+        for (int e = 0; e < n; ++e)
+            z += exp(S[t * n + e] - m);
+        for (int e = 0; e < n; ++e)
+            S[t * n + e] = exp(S[t * n + e] - m) / z;
+    }
+    /* each expert keeps its C best tokens */
+    for (int e = 0; e < n; ++e) {
+        for (int64_t t = 0; t < T; ++t)
+            order[t] = t;
+        g_sort_S = S;
+        g_sort_n = n;
+        g_sort_e = e;
+        qsort(order, (size_t)T, sizeof(int64_t), cmp_score_desc_token_asc);
+        qsort(order, (size_t)C, sizeof(int64_t), cmp_i64);
+        for (int64_t j = 0; j < C; ++j) {
+            sel_token[e * C + j] = order[j];
+            sel_gate[e * C + j] = S[order[j] * n + e];
+        }
+    }
+    /* y: the chosen experts' outputs, weighted by the router probability */
+    for (int64_t i = 0; i < T * (int64_t)d; ++i)
+        y[i] = 0.0;
+    for (int e = 0; e < n; ++e)
+        for (int64_t j = 0; j < C; ++j) {
+            int64_t t = sel_token[e * C + j];
+            expert_one(d, F, x, x_dt, (size_t)t * d, w1, w3, w2, w_dt, e, a, b, o);
+            for (int i = 0; i < d; ++i)
+                y[t * d + i] += sel_gate[e * C + j] * o[i];
+        }
+    free(S); free(order); free(a); free(b); free(o);
+    return 0;
+}

@@ -365,6 +365,61 @@ def check_dispatch_capacity(O):
             assert np.array_equal(c0, counts) and np.array_equal(tr0, token_row)
 
 
+# --------------------------------------------------------------------------
+# Expert-choice routing ([P1] "How Experts Are Chosen", item 2)
+# --------------------------------------------------------------------------
+
+def check_expert_choice_full_capacity_is_dense(O):
+    """C = T: every expert keeps every token, so y is the dense
+    softmax-weighted sum of all experts -- the token-choice layer with K = n,
+    and torch's dense restatement."""
+    T, d, F, n = 9, 24, 40, 5
+    x, Wg, w1, w3, w2 = rand_layer(43, T, d, F, n)
+    y, sel, gate = O.expert_choice(x, Wg, w1, w3, w2, T)
+    assert np.array_equal(sel, np.tile(np.arange(T), (n, 1)))
+    y_tc, _, _ = O.moe_forward(x, Wg, w1, w3, w2, n)
+    assert rel_l2(y, y_tc) < 1e-13
+    p = torch.softmax(torch.from_numpy(x @ Wg), dim=1).numpy()
+    ref = sum(p[:, e:e + 1] * torch_swiglu(x, w1[e], w3[e], w2[e]) for e in range(n))
+    assert rel_l2(y, ref) < 1e-13
+    assert np.allclose(gate, p.T, rtol=1e-13, atol=0)
+
+
+def check_expert_choice_ties_and_unchosen_tokens(O):
+    """All-equal scores (W_g = 0): every expert keeps tokens 0..C-1 with gate
+    1/n; the other tokens get y = 0 exactly."""
+    T, d, F, n, C = 10, 16, 24, 4, 3
+    x, _, w1, w3, w2 = rand_layer(44, T, d, F, n)
+    y, sel, gate = O.expert_choice(x, np.zeros((d, n)), w1, w3, w2, C)
+    assert np.array_equal(sel, np.tile(np.arange(C), (n, 1)))
+    assert np.all(gate == 0.25)
+    assert np.all(y[C:] == 0.0)
+    ref = sum(torch_swiglu(x[:C], w1[e], w3[e], w2[e]) for e in range(n)) / n
+    assert rel_l2(y[:C], ref) < 1e-13
+
+
+def check_expert_choice_selection_brute_force(O):
+    """Each expert's kept set is its C best tokens by probability (lower index
+    first on ties), cross-checked with a lexsort of torch's softmax."""
+    rng = np.random.default_rng(45)
+    for T, n, C in ((30, 4, 7), (17, 8, 17), (50, 3, 1)):
+        d, F = 12, 16
+        x, Wg, w1, w3, w2 = rand_layer(int(rng.integers(1000)), T, d, F, n)
+        y, sel, gate = O.expert_choice(x, Wg, w1, w3, w2, C)
+        p = torch.softmax(torch.from_numpy(x @ Wg), dim=1).numpy()
+        for e in range(n):
+            order = np.lexsort((np.arange(T), -p[:, e]))
+            assert np.array_equal(sel[e], np.sort(order[:C]))
+            assert np.allclose(gate[e], p[sel[e], e], rtol=1e-13, atol=0)
+        # y restated per token from the selection
+        yr = np.zeros_like(y)
+        for e in range(n):
+            for j in range(C):
+                t = sel[e, j]
+                yr[t] += gate[e, j] * torch_swiglu(x[t:t + 1], w1[e], w3[e], w2[e])[0]
+        assert rel_l2(y, yr) < 1e-13
+
+
 ALL_CHECKS = [
     check_worked_example, check_two_way_softmax_closed_form, check_logits_are_x_times_Wg,
     check_topk_brute_force, check_ties_go_to_lower_index, check_gate_invariants, check_silu,
@@ -373,4 +428,6 @@ ALL_CHECKS = [
     check_unchosen_experts_do_not_matter, check_forward_with_routing_consistent,
     check_bf16_inputs_widen_exactly, check_dispatch,
     check_router_stats_closed_forms, check_router_stats_against_torch, check_dispatch_capacity,
+    check_expert_choice_full_capacity_is_dense, check_expert_choice_ties_and_unchosen_tokens,
+    check_expert_choice_selection_brute_force,
 ]

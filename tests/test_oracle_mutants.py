@@ -28,6 +28,10 @@ MUTANTS = {
     "softmax_first_logit_only": [("z += exp(L[idx[k]] - m);", "z += (k == 0) ? 1.0 : 0.0;")],
     "stats_f_over_tokens": [("f[e] /= (double)(T * K);", "f[e] /= (double)T;")],
     "stats_P_unnormalised": [("P[e] += exp(L[e] - m) / z;", "P[e] += exp(L[e] - m);")],
+    "expert_choice_lowest_scores": [("    if (sa > sb) return -1;\n    if (sa < sb) return 1;",
+                                     "    if (sa < sb) return -1;\n    if (sa > sb) return 1;")],
+    "expert_choice_ties_high_token": [("return (ta < tb) ? -1 : (ta > tb);", "return (ta > tb) ? -1 : (ta < tb);")],
+    "expert_choice_gate_unnormalised": [("S[t * n + e] = exp(S[t * n + e] - m) / z;", "S[t * n + e] = exp(S[t * n + e] - m);")],
     "capacity_keeps_one_more": [("if (row - offsets[e] < capacity) {", "if (row - offsets[e] <= capacity) {")],
 }
 
