@@ -167,6 +167,27 @@ MOE_API moe_status moe_forward_with_routing(moe_handle *h, int64_t T, const void
 MOE_API moe_status moe_set_capacity_factor(moe_handle *h, double factor);
 
 /*
+ * Expert-choice routing: every expert chooses its own tokens, up to a fixed
+ * capacity ("Mixtral of Experts? Mixture of Experts? Try to explain Mixtral
+ * 8x7B", section "How Experts Are Chosen", item 2).  With the router
+ * probabilities S[t][e] = softmax over the n experts of x_t . W_g (fp32):
+ *   - expert e keeps the `capacity` tokens with the largest S[.][e] (equal
+ *     probabilities keep the lower token index); sel_token[e][0..capacity)
+ *     lists them in ascending token order and sel_gate[e][j] = S[token][e];
+ *   - y[t] = sum over the experts that kept t, in expert order, of
+ *     S[t][e] * SwiGLU_e(x_t); a token no expert kept gets y[t] = 0.
+ * The handle's K is not used.  x, W_g, w1, w3, w2, y as for moe_forward;
+ * sel_token [n][capacity] int32 and sel_gate [n][capacity] fp32 are device
+ * outputs.  1 <= capacity <= T.  The workspace grows to n * capacity rows.
+ *   Errors: as moe_forward.
+ */
+MOE_API moe_status moe_forward_expert_choice(moe_handle *h, int64_t T, int64_t capacity,
+                                             const void *x, const float *W_g, const void *w1,
+                                             const void *w3, const void *w2, void *y,
+                                             int32_t *sel_token, float *sel_gate,
+                                             moe_stream_t stream);
+
+/*
  * Load-balancing statistics of a routing (Part 5 of the neobadger page, "Tool
  * 2: a fine for favouritism", the Switch Transformers loss):
  *   f[i]  = share of the T*K routed (token, slot) pairs of topk_idx sent to

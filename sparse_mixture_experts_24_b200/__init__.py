@@ -54,6 +54,8 @@ lib.moe_workspace_view.argtypes = [_vp, ctypes.c_char_p, ctypes.POINTER(_vp), ct
 lib.moe_sync_status.argtypes = [_vp, _vp]
 lib.moe_destroy.argtypes = [_vp]
 lib.moe_trace_begin.argtypes = [_vp, _int]
+lib.moe_forward_expert_choice.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                          _vp]
 lib.moe_selftest_timeout.argtypes = [_vp, _int, _vp]
 lib.moe_launch_count.argtypes = [_vp, ctypes.POINTER(_i64)]
 lib.moe_set_capacity_factor.argtypes = [_vp, ctypes.c_double]
@@ -65,14 +67,15 @@ lib.moe_version.restype = ctypes.c_char_p
 for _f in ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
            "moe_forward_with_routing", "moe_workspace_view", "moe_sync_status", "moe_destroy",
            "moe_trace_begin", "moe_trace_end", "moe_dispatch_noalloc", "moe_set_capacity_factor",
-           "moe_router_stats", "moe_launch_count", "moe_selftest_timeout"):
+           "moe_router_stats", "moe_launch_count", "moe_selftest_timeout",
+           "moe_forward_expert_choice"):
     getattr(lib, _f).restype = _int
 
 EXPORTED = ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
             "moe_forward_with_routing", "moe_workspace_view", "moe_sync_status", "moe_destroy",
             "moe_last_error", "moe_version", "moe_trace_begin", "moe_trace_end",
             "moe_dispatch_noalloc", "moe_set_capacity_factor", "moe_router_stats",
-            "moe_launch_count", "moe_selftest_timeout")
+            "moe_launch_count", "moe_selftest_timeout", "moe_forward_expert_choice")
 
 TRACE_STAGES = ("router", "dispatch", "gather", "gemm1", "gemm2", "combine")
 
@@ -186,6 +189,13 @@ def moe_trace_end(h):
     return dict(zip(TRACE_STAGES, list(ms))), calls.value
 
 
+def moe_forward_expert_choice(h, T, capacity, x, W_g, w1, w3, w2, y, sel_token, sel_gate,
+                              stream=None) -> None:
+    _check(lib.moe_forward_expert_choice(h, T, capacity, _ptr(x), _ptr(W_g), _ptr(w1), _ptr(w3),
+                                         _ptr(w2), _ptr(y), _ptr(sel_token), _ptr(sel_gate),
+                                         _stream(stream)), "moe_forward_expert_choice")
+
+
 def moe_selftest_timeout(h, budget_us: int = 1000, stream=None) -> None:
     _check(lib.moe_selftest_timeout(h, budget_us, _stream(stream)), "moe_selftest_timeout")
 
@@ -252,6 +262,16 @@ class MoELayer:
         token_row = torch.empty((max(1, T), self.K), dtype=torch.int32, device=dev)
         moe_dispatch(self.h, T, topk_idx, counts, offsets, row_token, token_row, stream)
         return counts, offsets, row_token[:T * self.K], token_row[:T]
+
+    def forward_expert_choice(self, x, W_g, w1, w3, w2, capacity: int, stream=None):
+        """-> y, sel_token [n][capacity], sel_gate [n][capacity]"""
+        import torch
+        T = x.shape[0]
+        y = torch.empty_like(x)
+        sel = torch.empty((self.n, capacity), dtype=torch.int32, device=x.device)
+        gate = torch.empty((self.n, capacity), dtype=torch.float32, device=x.device)
+        moe_forward_expert_choice(self.h, T, capacity, x, W_g, w1, w3, w2, y, sel, gate, stream)
+        return y, sel, gate
 
     def set_capacity_factor(self, factor: float) -> None:
         moe_set_capacity_factor(self.h, factor)

@@ -108,6 +108,16 @@ cudaError_t launch_gather(const void* x, const int32_t* row_token, int64_t R, in
 cudaError_t launch_combine(const void* O, bool bf16, const int32_t* token_row, const float* topk_w,
                            int64_t T, int K, int d, void* y, int num_sms, cudaStream_t st);
 
+// Expert-choice routing: probabilities St [n][T], per-expert selection of C
+// tokens (rows e*C .. e*C+C-1, tokens ascending) into sel_token / sel_gate /
+// row_token, rowmap [T][n] (row of (t, e) or -1), and the dispatch arrays.
+cudaError_t launch_ec_route(const float* logits, int splits, int64_t T, int n, int C, int bm, float* St,
+                            int32_t* rowmap, int32_t* sel_token, float* sel_gate, int32_t* row_token,
+                            int32_t* counts, int32_t* offsets, int32_t* mblk_base, cudaStream_t st);
+// y[t] = sum_e gate_of_row[rowmap[t][e]] * O[rowmap[t][e]] (expert order).
+cudaError_t launch_ec_combine(const void* O, bool bf16, const int32_t* rowmap, const float* gate_of_row,
+                              int64_t T, int n, int d, void* y, int num_sms, cudaStream_t st);
+
 // One thread waits on an mbarrier nothing arrives at, with the given budget;
 // sets kStatusSelfTest in *status when the wait runs out.
 cudaError_t launch_bounded_wait_probe(int* status, long long budget_cycles, cudaStream_t st);

@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <algorithm>
 #include <new>
 #include <vector>
 
@@ -115,7 +116,8 @@ struct moe_handle {
     moe_dtype dtype;
     int device = -1;
     int num_sms = 0;
-    int64_t T_cap = 0;
+    int64_t T_cap = 0;  // tokens the workspace holds
+    int64_t R_cap = 0;  // expert rows (Xp, H, O) the workspace holds
     void* ws = nullptr;
     size_t ws_bytes = 0;
     moe::DispatchBufs db{};
@@ -139,6 +141,9 @@ struct moe_handle {
     int64_t launches = 0;
     float* stats_partial = nullptr;
     int32_t* stats_counts = nullptr;
+    // expert-choice routing: probabilities [n][T], row of (token, expert) [T][n]
+    float* ec_probs = nullptr;
+    int32_t* ec_rowmap = nullptr;
     // tracing: kTraceEvents events per traced call
     std::vector<cudaEvent_t> trace_ev;
     int trace_max = 0;
@@ -199,9 +204,13 @@ moe_status check_device(moe_handle* h) {
     return MOE_OK;
 }
 
-moe_status grow(moe_handle* h, int64_t T) {
-    if (T <= h->T_cap && h->ws) return MOE_OK;
-    const int64_t R = T * h->K;
+// Workspace for T tokens and at least rows_min expert rows (T*K for
+// token-choice calls, n*C for expert-choice calls).  Capacities only grow.
+moe_status grow(moe_handle* h, int64_t T, int64_t rows_min = 0) {
+    const int64_t R_need = std::max(T * h->K, rows_min);
+    if (h->ws && T <= h->T_cap && R_need <= h->R_cap) return MOE_OK;
+    T = std::max(T, h->T_cap);
+    const int64_t R = std::max(std::max(R_need, h->R_cap), T * h->K);
     const int64_t nblk = (R + moe::kPairsPerBlock - 1) / moe::kPairsPerBlock;
     const size_t A = 256;
     size_t off = 0;
@@ -224,6 +233,8 @@ moe_status grow(moe_handle* h, int64_t T) {
     const size_t o_stats_counts = take(static_cast<size_t>(h->n) * 4);
     const size_t o_parts = take(bf ? static_cast<size_t>(3) * npad * h->d * 2 : 0);
     const size_t o_status = take(64);
+    const size_t o_ec_probs = take(static_cast<size_t>(T) * h->n * 4);
+    const size_t o_ec_rowmap = take(static_cast<size_t>(T) * h->n * 4);
     const size_t o_xp = take(static_cast<size_t>(R) * h->d * h->esize());
     const size_t o_h = take(static_cast<size_t>(R) * h->F * h->esize());
     const size_t o_o = take(static_cast<size_t>(R) * h->d * h->osize());
@@ -233,6 +244,7 @@ moe_status grow(moe_handle* h, int64_t T) {
         cudaFree(h->ws);
         h->ws = nullptr;
         h->T_cap = 0;
+        h->R_cap = 0;
     }
     void* p = nullptr;
     cudaError_t e = cudaMalloc(&p, total);
@@ -250,6 +262,9 @@ moe_status grow(moe_handle* h, int64_t T) {
     h->ws = p;
     h->ws_bytes = total;
     h->T_cap = T;
+    h->R_cap = R;
+    h->ec_probs = reinterpret_cast<float*>(b + o_ec_probs);
+    h->ec_rowmap = reinterpret_cast<int32_t*>(b + o_ec_rowmap);
     h->db.blockcounts = reinterpret_cast<int32_t*>(b + o_blockcounts);
     h->db.pair_rank = reinterpret_cast<int32_t*>(b + o_pair_rank);
     h->db.counts = reinterpret_cast<int32_t*>(b + o_counts);
@@ -291,10 +306,10 @@ moe_status check_common(moe_handle* h, int64_t T) {
         if (!aligned16(p)) return fail(MOE_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p); \
     } while (0)
 
-moe_status prepare(moe_handle* h, int64_t T) {
+moe_status prepare(moe_handle* h, int64_t T, int64_t rows_min = 0) {
     moe_status s = check_device(h);
     if (s != MOE_OK) return s;
-    return grow(h, T);
+    return grow(h, T, rows_min);
 }
 
 // Router: the tensor-core path (bf16 x, enough tokens or many experts) or the
@@ -340,20 +355,13 @@ int capacity_for(const moe_handle* h, int64_t T) {
     return c >= static_cast<double>(moe::kNoCapacity) ? moe::kNoCapacity : static_cast<int>(c);
 }
 
-moe_status run_experts(moe_handle* h, int64_t T, const void* x, const int32_t* topk_idx,
-                       const float* topk_w, const void* w1, const void* w3, const void* w2, void* y,
-                       cudaStream_t st) {
+// Gather the segment rows of x, then GEMM1 (w1/w3 + SwiGLU) and GEMM2 (w2)
+// over R rows laid out by the dispatch arrays already on the device.
+moe_status run_gemms(moe_handle* h, int64_t T, int64_t R, const void* x, const void* w1, const void* w3,
+                     const void* w2, bool pair, cudaStream_t st) {
     const bool bf = h->dtype == MOE_BF16;
-    const bool pair = use_pair_gemm(h, T);
-    const int64_t R = T * h->K;
-    cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n,
-                                         pair ? moe::kTcPairBM : (bf ? moe::kTcBM : moe::kSimtBM),
-                                         h->db, st, capacity_for(h, T));
-    if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
-    h->launches += moe::dispatch_kernel_count(R);
-    trace_mark(h, 1, st);
-    e = moe::launch_gather(x, h->db.row_token, R, T, static_cast<int64_t>(h->d) * h->esize(), h->xp,
-                           h->num_sms, st);
+    cudaError_t e = moe::launch_gather(x, h->db.row_token, R, T, static_cast<int64_t>(h->d) * h->esize(),
+                                       h->xp, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "gather launch");
     h->launches += 1;
     trace_mark(h, 2, st);
@@ -412,11 +420,52 @@ moe_status run_experts(moe_handle* h, int64_t T, const void* x, const int32_t* t
         h->launches += 1;
         trace_mark(h, 4, st);
     }
+    return MOE_OK;
+}
+
+moe_status run_experts(moe_handle* h, int64_t T, const void* x, const int32_t* topk_idx,
+                       const float* topk_w, const void* w1, const void* w3, const void* w2, void* y,
+                       cudaStream_t st) {
+    const bool bf = h->dtype == MOE_BF16;
+    const bool pair = use_pair_gemm(h, T);
+    const int64_t R = T * h->K;
+    cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n,
+                                         pair ? moe::kTcPairBM : (bf ? moe::kTcBM : moe::kSimtBM),
+                                         h->db, st, capacity_for(h, T));
+    if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
+    h->launches += moe::dispatch_kernel_count(R);
+    trace_mark(h, 1, st);
+    moe_status s = run_gemms(h, T, R, x, w1, w3, w2, pair, st);
+    if (s != MOE_OK) return s;
     e = moe::launch_combine(h->o, bf, h->db.token_row, topk_w, T, h->K, h->d, y, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "combine launch");
     h->launches += 1;
     trace_mark(h, 5, st);
     trace_finish_call(h);
+    return MOE_OK;
+}
+
+// Router logits into h->logits (tensor cores for bf16, CUDA cores for fp32);
+// returns the number of split partials.
+moe_status run_logits(moe_handle* h, int64_t T, const void* x, const float* W_g, cudaStream_t st,
+                      int* splits) {
+    cudaError_t e;
+    *splits = 1;
+    if (h->dtype == MOE_BF16) {
+        if (x != h->c_rx || T != h->c_rx_T) {
+            if (!encode_rows(&h->tm_rx, x, h->d, static_cast<uint64_t>(T)))
+                return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for x");
+            h->c_rx = x;
+            h->c_rx_T = T;
+        }
+        e = moe::launch_router_logits_tc(h->tm_rx, h->tm_parts, W_g, h->wg_parts, T, h->d, h->n, h->logits,
+                                         h->status, h->num_sms, st, splits);
+        h->launches += 2;
+    } else {
+        e = moe::launch_router_logits_simt(x, false, W_g, T, h->d, h->n, h->logits, st);
+        h->launches += 1;
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "router logits launch");
     return MOE_OK;
 }
 
@@ -559,6 +608,55 @@ moe_status moe_dispatch(moe_handle* h, int64_t T, const int32_t* topk_idx, int32
     return ok();
 }
 
+moe_status moe_forward_expert_choice(moe_handle* h, int64_t T, int64_t capacity, const void* x,
+                                     const float* W_g, const void* w1, const void* w3, const void* w2,
+                                     void* y, int32_t* sel_token, float* sel_gate, moe_stream_t stream) {
+    moe_status s = check_common(h, T);
+    if (s != MOE_OK) return s;
+    if (T == 0) return ok();
+    if (capacity < 1 || capacity > T)
+        return fail(MOE_ERR_INVALID_ARG, "capacity = %lld outside [1, T = %lld]",
+                    static_cast<long long>(capacity), static_cast<long long>(T));
+    if (capacity * h->n > 2147483647LL)
+        return fail(MOE_ERR_INVALID_ARG, "capacity * n exceeds 2^31 - 1");
+    if (T > 2147483647LL) return fail(MOE_ERR_INVALID_ARG, "T exceeds 2^31 - 1");
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(W_g);
+    REQUIRE_PTR(w1);
+    REQUIRE_PTR(w3);
+    REQUIRE_PTR(w2);
+    REQUIRE_PTR(y);
+    REQUIRE_PTR(sel_token);
+    REQUIRE_PTR(sel_gate);
+    const int64_t R = capacity * h->n;
+    s = prepare(h, T, R);
+    if (s != MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    moe::chain_begin();
+    trace_mark(h, -1, st);
+    int splits = 1;
+    s = run_logits(h, T, x, W_g, st, &splits);
+    if (s != MOE_OK) return s;
+    const bool pair = use_pair_gemm(h, T);
+    const int bm = pair ? moe::kTcPairBM : (h->dtype == MOE_BF16 ? moe::kTcBM : moe::kSimtBM);
+    cudaError_t e = moe::launch_ec_route(h->logits, splits, T, h->n, static_cast<int>(capacity), bm,
+                                         h->ec_probs, h->ec_rowmap, sel_token, sel_gate, h->db.row_token,
+                                         h->db.counts, h->db.offsets, h->db.mblk_base, st);
+    if (e != cudaSuccess) return cuda_fail(e, "expert-choice routing launch");
+    h->launches += 2;
+    trace_mark(h, 0, st);
+    trace_mark(h, 1, st);
+    s = run_gemms(h, T, R, x, w1, w3, w2, pair, st);
+    if (s != MOE_OK) return s;
+    e = moe::launch_ec_combine(h->o, h->dtype == MOE_BF16, h->ec_rowmap, sel_gate, T, h->n, h->d, y,
+                               h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "expert-choice combine launch");
+    h->launches += 1;
+    trace_mark(h, 5, st);
+    trace_finish_call(h);
+    return ok();
+}
+
 moe_status moe_set_capacity_factor(moe_handle* h, double factor) {
     if (!h) return fail(MOE_ERR_INVALID_ARG, "null handle");
     if (!(factor >= 0.0) || !std::isfinite(factor))
@@ -585,21 +683,9 @@ moe_status moe_router_stats(moe_handle* h, int64_t T, const void* x, const float
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     moe::chain_begin();
     int splits = 1;
+    s = run_logits(h, T, x, W_g, st, &splits);
+    if (s != MOE_OK) return s;
     cudaError_t e;
-    if (h->dtype == MOE_BF16) {
-        if (x != h->c_rx || T != h->c_rx_T) {
-            if (!encode_rows(&h->tm_rx, x, h->d, static_cast<uint64_t>(T)))
-                return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for x");
-            h->c_rx = x;
-            h->c_rx_T = T;
-        }
-        e = moe::launch_router_logits_tc(h->tm_rx, h->tm_parts, W_g, h->wg_parts, T, h->d, h->n, h->logits,
-                                         h->status, h->num_sms, st, &splits);
-    } else {
-        e = moe::launch_router_logits_simt(x, false, W_g, T, h->d, h->n, h->logits, st);
-    }
-    if (e != cudaSuccess) return cuda_fail(e, "router logits launch");
-    h->launches += h->dtype == MOE_BF16 ? 2 : 1;
     e = moe::launch_router_stats(h->logits, splits, T, h->n, h->K, topk_idx, alpha, h->stats_partial,
                                  h->stats_counts, f, P, aux, st);
     if (e != cudaSuccess) return cuda_fail(e, "router statistics launch");
@@ -616,7 +702,7 @@ moe_status moe_workspace_view(moe_handle* h, const char* name, void** ptr, int64
         *ptr = h->o;
     else
         return fail(MOE_ERR_INVALID_ARG, "unknown workspace buffer '%s' (use \"H\" or \"O\")", name);
-    *rows = h->T_cap * h->K;
+    *rows = h->R_cap;
     return ok();
 }
 
