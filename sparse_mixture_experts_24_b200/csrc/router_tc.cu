@@ -224,9 +224,10 @@ cudaError_t launch_router_logits_tc(const CUtensorMap& tm_x, const CUtensorMap& 
     const int smem = router_tc_smem_bytes(n);
     cudaError_t e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    // split d so that about one CTA per SM runs, at least 8 K blocks each
+    // split d so that the CTAs fill at most one wave (one CTA per SM: the ring
+    // takes most of shared memory), at least 8 K blocks each
     const int64_t mtiles = (T + kRtBM - 1) / kRtBM;
-    int splits = static_cast<int>((num_sms + mtiles - 1) / mtiles);
+    int splits = static_cast<int>(num_sms / mtiles);
     const int kb_total = d / kRtBK;
     if (splits > kRouterMaxSplits) splits = kRouterMaxSplits;
     if (splits > kb_total / 8) splits = kb_total / 8;
