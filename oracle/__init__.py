@@ -64,6 +64,13 @@ def _bind(L):
     L.oracle_router_stats.argtypes = [i64, i32, i32, i32, vp, i32, vp, i32, vp, ctypes.c_double,
                                       vp, vp, vp]
     L.oracle_dispatch_capacity.argtypes = [i64, i32, i32, vp, i64, vp, vp, vp, vp]
+    L.oracle_e4m3_decode.argtypes = [ctypes.c_int]
+    L.oracle_e4m3_decode.restype = ctypes.c_double
+    L.oracle_e4m3_encode.argtypes = [ctypes.c_double]
+    L.oracle_e4m3_encode.restype = ctypes.c_int
+    L.oracle_quantize_weights_e4m3.argtypes = [i32, i32, i32, vp, i32, vp, vp]
+    L.oracle_forward_e4m3.argtypes = [i64, i32, i32, i32, i32, vp, i32, vp, vp, vp, vp, vp, vp, vp,
+                                      vp, vp]
     L.oracle_expert_choice.argtypes = [i64, i32, i32, i32, i64, vp, i32, vp, i32, vp, vp, vp, i32,
                                        vp, vp, vp]
     L.oracle_silu.argtypes = [ctypes.c_double]
@@ -72,7 +79,8 @@ def _bind(L):
     L.oracle_set_num_threads.argtypes = [ctypes.c_int]
     for f in ("oracle_router", "oracle_expert", "oracle_forward_with_routing",
               "oracle_moe_forward", "oracle_dispatch", "oracle_router_stats",
-              "oracle_dispatch_capacity", "oracle_expert_choice"):
+              "oracle_dispatch_capacity", "oracle_expert_choice", "oracle_quantize_weights_e4m3",
+              "oracle_forward_e4m3"):
         getattr(L, f).restype = ctypes.c_int
     return L
 
@@ -224,6 +232,37 @@ class Oracle:
         return y, sel, gate
 
 
+    def e4m3_decode(self, code: int) -> float:
+        return float(self.L.oracle_e4m3_decode(int(code)))
+
+    def e4m3_encode(self, v: float) -> int:
+        return int(self.L.oracle_e4m3_encode(float(v)))
+
+    def quantize_weights_e4m3(self, w):
+        """w [n][rows][cols] -> codes uint8 [n][rows][cols], scales fp32 [n][cols]."""
+        w = _c(w)
+        n, rows, cols = w.shape
+        codes = np.empty((n, rows, cols), np.uint8)
+        scales = np.empty((n, cols), np.float32)
+        _check(self.L.oracle_quantize_weights_e4m3(n, rows, cols, _p(w), _dt(w), _p(codes), _p(scales)),
+               "quantize_weights_e4m3")
+        return codes, scales
+
+    def forward_e4m3(self, x, idx, gate, q1, s1, q3, s3, q2, s2):
+        x = _c(x)
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+        gate = np.ascontiguousarray(gate, dtype=np.float64)
+        q1, q3, q2 = (np.ascontiguousarray(a, dtype=np.uint8) for a in (q1, q3, q2))
+        s1, s3, s2 = (np.ascontiguousarray(a, dtype=np.float32) for a in (s1, s3, s2))
+        T, d = x.shape
+        n, d2, F = q1.shape
+        K = idx.shape[1]
+        y = np.empty((T, d), np.float64)
+        _check(self.L.oracle_forward_e4m3(T, d, F, n, K, _p(x), _dt(x), _p(idx), _p(gate), _p(q1), _p(s1),
+                                          _p(q3), _p(s3), _p(q2), _p(s2), _p(y)), "forward_e4m3")
+        return y
+
+
 _default = None
 
 
@@ -276,3 +315,19 @@ def dispatch_capacity(idx, n: int, capacity: int):
 
 def expert_choice(x, W_g, w1, w3, w2, C: int):
     return default().expert_choice(x, W_g, w1, w3, w2, C)
+
+
+def e4m3_decode(code: int) -> float:
+    return default().e4m3_decode(code)
+
+
+def e4m3_encode(v: float) -> int:
+    return default().e4m3_encode(v)
+
+
+def quantize_weights_e4m3(w):
+    return default().quantize_weights_e4m3(w)
+
+
+def forward_e4m3(x, idx, gate, q1, s1, q3, s3, q2, s2):
+    return default().forward_e4m3(x, idx, gate, q1, s1, q3, s3, q2, s2)

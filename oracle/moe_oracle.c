@@ -477,3 +477,194 @@ int oracle_expert_choice(int64_t T, int d, int F, int n, int64_t C, const void *
     free(S); free(order); free(a); free(b); free(o);
     return 0;
 }
+
+/*
+ * FP8 E4M3 expert weights and activations (the "load it in 4-bit" option of
+ * Part 4 of the neobadger page, here at 8 bits).  E4M3 as the OCP 8-bit
+ * floating point specification defines it: 1 sign bit, 4 exponent bits (bias
+ * 7), 3 mantissa bits, subnormals, no infinities, largest finite 448, NaN =
+ * S.1111.111.  Encoding rounds to nearest, ties to even, and saturates finite
+ * values beyond 448 to +-448.
+ */
+double oracle_e4m3_decode(int code)
+{
+    int s = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);           /* subnormal: m/8 * 2^-6 */
+    else
+        v = ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+static double round_half_even(double v)
+{
+    double f = floor(v), r = v - f;
+    if (r > 0.5) return f + 1.0;
+    if (r < 0.5) return f;
+    return (fmod(f, 2.0) == 0.0) ? f : f + 1.0;
+}
+
+int oracle_e4m3_encode(double v)
+{
+    if (isnan(v))
+        return 0x7F;
+    int s = signbit(v) ? 1 : 0;
+    double a = fabs(v), q;
+    if (a >= 448.0) {
+        q = 448.0;
+    } else if (a < ldexp(1.0, -6)) {
+        q = ldexp(round_half_even(ldexp(a, 9)), -9);     /* multiples of 2^-9 */
+    } else {
+        int E;
+        frexp(a, &E);                                     /* a = f * 2^E, 0.5 <= f < 1 */
+        double step = ldexp(1.0, E - 1 - 3);              /* 3 mantissa bits below 2^(E-1) */
+        q = round_half_even(a / step) * step;
+        if (q > 448.0) q = 448.0;
+    }
+    /* q is representable: find its code */
+    int code;
+    if (q < ldexp(1.0, -6)) {
+        code = (int)ldexp(q, 9);                          /* e = 0, m = q / 2^-9 */
+    } else {
+        int E;
+        double f = frexp(q, &E);                          /* q = f * 2^E, f in [0.5, 1) */
+        int e = E - 1 + 7;
+        int m = (int)((f * 2.0 - 1.0) * 8.0 + 0.5);
+        code = (e << 3) | m;
+    }
+    return (s << 7) | code;
+}
+
+/* Scale of a group of values: max |v| / 448 in fp32 (1 when the group is all
+ * zero), the same precision the GPU uses, so both sides pick the same codes. */
+static float e4m3_scale_f32(float amax) { return amax > 0.0f ? amax / 448.0f : 1.0f; }
+
+/* Codes of v / scale, the quotient taken in fp32. */
+static int e4m3_code_f32(float v, float scale) { return oracle_e4m3_encode((double)(v / scale)); }
+
+/*
+ * Per-channel weight quantization: w [n][rows][cols] (bf16 bits or fp32) ->
+ * codes [n][rows][cols] (uint8) and scales [n][cols] (fp32): one scale per
+ * output column over all rows (the reduction dimension).
+ */
+int oracle_quantize_weights_e4m3(int n, int rows, int cols, const void *w, int w_dt, uint8_t *codes,
+                                 float *scales)
+{
+    if (n <= 0 || rows <= 0 || cols <= 0 || !w || !codes || !scales || !dt_ok(w_dt))
+        return -1;
+    for (int e = 0; e < n; ++e)
+        for (int c = 0; c < cols; ++c) {
+            float amax = 0.0f;
+            for (int r = 0; r < rows; ++r) {
+                float v = (float)elem(w, w_dt, ((size_t)e * rows + r) * cols + c);
+                if (fabsf(v) > amax) amax = fabsf(v);
+            }
+            float s = e4m3_scale_f32(amax);
+            scales[(size_t)e * cols + c] = s;
+            for (int r = 0; r < rows; ++r) {
+                size_t i = ((size_t)e * rows + r) * cols + c;
+                codes[i] = (uint8_t)e4m3_code_f32((float)elem(w, w_dt, i), s);
+            }
+        }
+    return 0;
+}
+
+/* bf16 rounding (nearest, ties to even) of a float, as a float */
+static float round_bf16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    u = (u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u;
+    float r;
+    memcpy(&r, &u, 4);
+    return r;
+}
+
+/*
+ * The layer with E4M3 experts under a given routing (idx, gate as for
+ * oracle_forward_with_routing), each step in the order and precision of the
+ * quantized path:
+ *   x row -> per-row scale sx = max|x| / 448 (fp32), codes qx;
+ *   a = sum_j qx_j * q1_jf (exact products, summed in double) * sx * s1_f,
+ *   b likewise with w3; h = silu(a) * b, rounded to fp32 then bf16 (the
+ *   stored hidden layer);
+ *   h row -> sh = max|h| / 448, codes qh;
+ *   o_i = sum_f qh_f * q2_fi * sh * s2_i;  y = sum_k gate_k * o (double).
+ * q1, q3: [n][d][F] codes with scales s1, s3 [n][F]; q2: [n][F][d] with s2 [n][d].
+ */
+int oracle_forward_e4m3(int64_t T, int d, int F, int n, int K, const void *x, int x_dt,
+                        const int32_t *idx, const double *gate, const uint8_t *q1, const float *s1,
+                        const uint8_t *q3, const float *s3, const uint8_t *q2, const float *s2,
+                        double *y)
+{
+    if (T <= 0 || d <= 0 || F <= 0 || n <= 0 || K <= 0 || !x || !idx || !gate || !q1 || !s1 || !q3 ||
+        !s3 || !q2 || !s2 || !y || !dt_ok(x_dt))
+        return -1;
+    for (int64_t i = 0; i < T * K; ++i)
+        if (idx[i] < 0 || idx[i] >= n)
+            return -1;
+    double lut[256];
+    for (int c = 0; c < 256; ++c)
+        lut[c] = oracle_e4m3_decode(c);
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *qx = (double *)malloc(sizeof(double) * (size_t)d);
+        double *a = (double *)malloc(sizeof(double) * (size_t)F);
+        double *b = (double *)malloc(sizeof(double) * (size_t)F);
+        float *hf = (float *)malloc(sizeof(float) * (size_t)F);
+        double *qh = (double *)malloc(sizeof(double) * (size_t)F);
+        if (!qx || !a || !b || !hf || !qh) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t t = 0; t < T; ++t) {
+                float amax = 0.0f;
+                for (int j = 0; j < d; ++j) {
+                    float v = (float)elem(x, x_dt, (size_t)t * d + j);
+                    if (fabsf(v) > amax) amax = fabsf(v);
+                }
+                float sx = e4m3_scale_f32(amax);
+                for (int j = 0; j < d; ++j)
+                    qx[j] = lut[e4m3_code_f32((float)elem(x, x_dt, (size_t)t * d + j), sx)];
+                double *yt = y + t * d;
+                for (int i = 0; i < d; ++i)
+                    yt[i] = 0.0;
+                for (int k = 0; k < K; ++k) {
+                    int e = idx[t * K + k];
+                    size_t base1 = (size_t)e * d * F, base2 = (size_t)e * F * d;
+                    for (int f = 0; f < F; ++f)
+                        a[f] = b[f] = 0.0;
+                    for (int j = 0; j < d; ++j)
+                        for (int f = 0; f < F; ++f) {
+                            a[f] += qx[j] * lut[q1[base1 + (size_t)j * F + f]];
+                            b[f] += qx[j] * lut[q3[base1 + (size_t)j * F + f]];
+                        }
+                    float hmax = 0.0f;
+                    for (int f = 0; f < F; ++f) {
+                        double av = a[f] * sx * s1[(size_t)e * F + f];
+                        double bv = b[f] * sx * s3[(size_t)e * F + f];
+                        hf[f] = round_bf16((float)(oracle_silu(av) * bv));
+                        if (fabsf(hf[f]) > hmax) hmax = fabsf(hf[f]);
+                    }
+                    float sh = e4m3_scale_f32(hmax);
+                    for (int f = 0; f < F; ++f)
+                        qh[f] = lut[e4m3_code_f32(hf[f], sh)];
+                    double g = gate[t * K + k];
+                    for (int i = 0; i < d; ++i) {
+                        double o = 0.0;
+                        for (int f = 0; f < F; ++f)
+                            o += qh[f] * lut[q2[base2 + (size_t)f * d + i]];
+                        yt[i] += g * o * sh * s2[(size_t)e * d + i];
+                    }
+                }
+            }
+        }
+        free(qx); free(a); free(b); free(hf); free(qh);
+    }
+    return bad ? -1 : 0;
+}

@@ -420,6 +420,98 @@ def check_expert_choice_selection_brute_force(O):
         assert rel_l2(y, yr) < 1e-13
 
 
+# --------------------------------------------------------------------------
+# FP8 E4M3 experts
+# --------------------------------------------------------------------------
+
+def check_e4m3_codec(O):
+    """E4M3 as the OCP 8-bit floating point specification defines it: largest
+    finite 448 (S.1111.110), NaN S.1111.111, smallest normal 2^-6 (0x08),
+    smallest subnormal 2^-9 (0x01); encode rounds to nearest, ties to even,
+    saturating beyond 448; every non-NaN code round-trips."""
+    assert O.e4m3_decode(0x7E) == 448.0 and O.e4m3_decode(0xFE) == -448.0
+    assert math.isnan(O.e4m3_decode(0x7F)) and math.isnan(O.e4m3_decode(0xFF))
+    assert O.e4m3_decode(0x08) == 2.0 ** -6 and O.e4m3_decode(0x01) == 2.0 ** -9
+    assert O.e4m3_decode(0x38) == 1.0 and O.e4m3_decode(0x00) == 0.0
+    vals = [O.e4m3_decode(c) for c in range(0x7F)]
+    assert all(vals[i] < vals[i + 1] for i in range(len(vals) - 1))
+    for c in range(256):
+        if c in (0x7F, 0xFF):
+            continue
+        assert O.e4m3_encode(O.e4m3_decode(c)) == c, c
+    # ties to even, saturation, rounding
+    assert O.e4m3_encode(1.0 + 1 / 16) == 0x38       # halfway 1 | 1.125 -> even (1)
+    assert O.e4m3_encode(1.125 + 1 / 16) == 0x3A     # halfway 1.125 | 1.25 -> even (1.25)
+    assert O.e4m3_encode(2.0 ** -10) == 0x00          # halfway 0 | 2^-9 -> even (0)
+    assert O.e4m3_encode(3 * 2.0 ** -10) == 0x02      # halfway 2^-9 | 2^-8 -> even (2^-8)
+    assert O.e4m3_encode(1e9) == 0x7E and O.e4m3_encode(-1e9) == 0xFE
+    assert O.e4m3_encode(460.0) == 0x7E and O.e4m3_encode(-3.0) == 0xC4
+    rng = np.random.default_rng(46)
+    for v in rng.standard_normal(200) * 10:
+        q = O.e4m3_decode(O.e4m3_encode(v))
+        assert abs(q - v) <= max(abs(v) * 2.0 ** -4, 2.0 ** -10)
+
+
+def check_e4m3_weight_quantization(O):
+    """One scale per output column (max |w| / 448 over the reduction rows): the
+    column maximum codes to +-448 and every value comes back within E4M3's
+    relative step."""
+    rng = np.random.default_rng(47)
+    w = rng.standard_normal((3, 40, 24)).astype(np.float32)
+    codes, scales = O.quantize_weights_e4m3(w)
+    assert np.allclose(scales, np.abs(w).max(axis=1) / 448, rtol=1e-7, atol=0)
+    deq = np.vectorize(O.e4m3_decode)(codes) * scales[:, None, :]
+    assert np.all(np.abs(deq - w) <= np.abs(w) * 2.0 ** -4 + scales[:, None, :] * 2.0 ** -9)
+    amax_rows = np.abs(w).argmax(axis=1)
+    for e in range(3):
+        for c in range(24):
+            assert codes[e, amax_rows[e, c], c] in (0x7E, 0xFE)
+
+
+def check_e4m3_forward_exact_case(O):
+    """With every x row and weight column exactly representable after its
+    scale (column and row maxima of 3.5 = 448 * 2^-7 make the scales powers
+    of two), and ffn = 1 (the hidden row's single value codes to +-448), the
+    E4M3 layer equals the exact layer up to the bf16 rounding of h."""
+    T, d, F, n = 7, 16, 1, 3
+    rng = np.random.default_rng(48)
+    vals = [-3.5, -1.75, -0.875, 0.875, 1.75, 3.5]
+    x = rng.choice([-3.5, -1.75, 0.0, 1.75, 3.5], size=(T, d))
+    x[:, 0] = 3.5
+    w1 = rng.choice(vals, size=(n, d, F)) / 8
+    w3 = rng.choice(vals, size=(n, d, F)) / 8
+    w2 = rng.choice(vals, size=(n, F, d)) / 8
+    w1[:, 0, :] = w3[:, 0, :] = 3.5 / 8
+    w2[:, :, 0] = 3.5 / 8
+    idx = np.array([[t % n, (t + 1) % n] for t in range(T)], np.int32)
+    gate = np.tile([[0.75, 0.25]], (T, 1))
+    q1, s1 = O.quantize_weights_e4m3(w1)
+    q3, s3 = O.quantize_weights_e4m3(w3)
+    q2, s2 = O.quantize_weights_e4m3(w2)
+    assert np.all(s1 == 2.0 ** -10) and np.all(s3 == 2.0 ** -10)
+    assert np.all(np.log2(s2) == np.round(np.log2(s2)))   # every |value| is 448 * 2^k
+    assert np.array_equal(np.vectorize(O.e4m3_decode)(q1) * s1[:, None, :], w1)
+    assert np.array_equal(np.vectorize(O.e4m3_decode)(q2) * s2[:, None, :], w2)
+    y8 = O.forward_e4m3(x, idx, gate, q1, s1, q3, s3, q2, s2)
+    y = O.forward_with_routing(x, idx, gate, w1, w3, w2)
+    assert rel_l2(y8, y) < 2.0 ** -8
+
+
+def check_e4m3_forward_error_band(O):
+    """On random data the E4M3 layer stays within the quantisation error band
+    of the exact layer (and is not the exact layer)."""
+    T, d, F, n = 12, 64, 96, 4
+    x, Wg, w1, w3, w2 = rand_layer(49, T, d, F, n)
+    idx, gate, _ = O.router(x, Wg, 2)
+    q1, s1 = O.quantize_weights_e4m3(w1)
+    q3, s3 = O.quantize_weights_e4m3(w3)
+    q2, s2 = O.quantize_weights_e4m3(w2)
+    y8 = O.forward_e4m3(x, idx, gate, q1, s1, q3, s3, q2, s2)
+    y = O.forward_with_routing(x, idx, gate, w1, w3, w2)
+    err = rel_l2(y8, y)
+    assert 1e-3 < err < 0.08, err
+
+
 ALL_CHECKS = [
     check_worked_example, check_two_way_softmax_closed_form, check_logits_are_x_times_Wg,
     check_topk_brute_force, check_ties_go_to_lower_index, check_gate_invariants, check_silu,
@@ -430,4 +522,6 @@ ALL_CHECKS = [
     check_router_stats_closed_forms, check_router_stats_against_torch, check_dispatch_capacity,
     check_expert_choice_full_capacity_is_dense, check_expert_choice_ties_and_unchosen_tokens,
     check_expert_choice_selection_brute_force,
+    check_e4m3_codec, check_e4m3_weight_quantization, check_e4m3_forward_exact_case,
+    check_e4m3_forward_error_band,
 ]
