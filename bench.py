@@ -2,6 +2,7 @@
 """Benchmark of the sparse MoE layer forward (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+                    [--experts bf16|e4m3]
 
 A step is one moe_forward over one batch: router, top-K, softmax, dispatch,
 gather, GEMM1 (w1/w3 + SwiGLU), GEMM2 (w2), combine.  The default workload is
@@ -20,6 +21,10 @@ reports the dominant kernel, timed by the library's per-stage CUDA events over
 a second run of the same K steps (events between the kernels would serialise
 their programmatic dependent launches in the headline run).  `cpu_baseline` times the fp64 oracle on a bounded
 sample of the same workload on this host's cores.
+
+--experts e4m3 times moe_forward_e4m3 instead: the same layer with FP8 (E4M3)
+expert weights (per-column scales, quantised once before the timed region)
+and per-row E4M3 activations (bf16 handle and workloads only).
 
 --impl reference runs the oracle (the reference arm of this build) on the
 host, rank 0 only.
@@ -54,9 +59,10 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
-def workload_desc(cfg):
-    return "%s: T=%d, d=%d, ffn=%d, n=%d, K=%d, %s%s" % (
-        cfg.name, cfg.T, cfg.d, cfg.ffn, cfg.n, cfg.K, cfg.dtype, ", skewed router" if cfg.skew else "")
+def workload_desc(cfg, experts="bf16"):
+    return "%s: T=%d, d=%d, ffn=%d, n=%d, K=%d, %s%s%s" % (
+        cfg.name, cfg.T, cfg.d, cfg.ffn, cfg.n, cfg.K, cfg.dtype, ", skewed router" if cfg.skew else "",
+        ", E4M3 experts" if experts == "e4m3" else "")
 
 
 # --------------------------------------------------------------------------
@@ -67,16 +73,24 @@ def touched_experts(idx: np.ndarray, n: int) -> np.ndarray:
     return np.bincount(idx.ravel(), minlength=n)
 
 
-def algorithmic(cfg, counts):
-    """Bytes and FLOPs each stage must move / do, from the routing of the step."""
+def algorithmic(cfg, counts, experts="bf16"):
+    """Bytes and FLOPs each stage must move / do, from the routing of the step.
+    E4M3 experts: one byte per weight plus its column's fp32 scale; the gemm1
+    stage also holds the hidden-row quantisation (bf16 H read, codes written)."""
     es = 2 if cfg.dtype == "bf16" else 4
     T, d, F, n, K = cfg.T, cfg.d, cfg.ffn, cfg.n, cfg.K
     R = T * K
     used = int((counts > 0).sum())
-    w13 = used * 2 * d * F * es
-    w2 = used * F * d * es
-    gemm1_bytes = w13 + R * d * es + R * F * es           # weights + Xp read + H write
-    gemm2_bytes = w2 + R * F * es + R * d * es             # weights + H read + O write
+    if experts == "e4m3":
+        w13 = used * 2 * (d * F + F * 4)
+        w2 = used * (F * d + d * 4)
+        gemm1_bytes = w13 + R * (d + 4) + R * F * 2 + (R * F * 2 + R * (F + 4))
+        gemm2_bytes = w2 + R * (F + 4) + R * d * es
+    else:
+        w13 = used * 2 * d * F * es
+        w2 = used * F * d * es
+        gemm1_bytes = w13 + R * d * es + R * F * es           # weights + Xp read + H write
+        gemm2_bytes = w2 + R * F * es + R * d * es             # weights + H read + O write
     gemm1_flops = 4.0 * R * d * F
     gemm2_flops = 2.0 * R * F * d
     return {
@@ -197,20 +211,31 @@ class ClockSampler:
 # CPU baseline: the oracle on a bounded sample of the workload
 # --------------------------------------------------------------------------
 
-def oracle_tokens_per_s(cfg, L, budget_s=12.0):
+def oracle_tokens_per_s(cfg, L, budget_s=12.0, experts="bf16"):
     """The oracle on the first tokens of the workload, repeated until about
-    budget_s of host time (a bounded sample of the same layer)."""
+    budget_s of host time (a bounded sample of the same layer).  E4M3 experts:
+    the oracle's router and E4M3 layer, on codes it quantised beforehand
+    (untimed)."""
     import oracle
     threads = oracle.num_threads()
+    if experts == "e4m3":
+        q = [a for w in ("w1", "w3", "w2") for a in oracle.quantize_weights_e4m3(L[w])]
+
+        def layer(xs):
+            i, g, _ = oracle.router(xs, L["W_g"], cfg.K)
+            oracle.forward_e4m3(xs, i, g, *q)
+    else:
+        def layer(xs):
+            oracle.moe_forward(xs, L["W_g"], L["w1"], L["w3"], L["w2"], cfg.K)
     t0 = time.perf_counter()
-    oracle.moe_forward(L["x"][:1], L["W_g"], L["w1"], L["w3"], L["w2"], cfg.K)
+    layer(L["x"][:1])
     one = max(time.perf_counter() - t0, 1e-6)
     # tokens per repetition: enough to keep every thread busy, within budget
     s = int(max(1, min(cfg.T, max(threads, budget_s * threads / one / 4))))
     done, reps = 0, 0
     t0 = time.perf_counter()
     while True:
-        oracle.moe_forward(L["x"][:s], L["W_g"], L["w1"], L["w3"], L["w2"], cfg.K)
+        layer(L["x"][:s])
         done += s
         reps += 1
         el = time.perf_counter() - t0
@@ -271,10 +296,13 @@ def main():
     ap.add_argument("--config", default="decode", choices=sorted(mi.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", default="bf16", choices=["bf16", "e4m3"])
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     cfg = mi.CONFIGS[args.config]
+    if args.experts == "e4m3" and cfg.dtype != "bf16":
+        ap.error("--experts e4m3 needs a bf16 workload")
     if args.impl == "reference":
         return run_reference(args, cfg)
 
@@ -311,11 +339,24 @@ def main():
     gw = torch.empty((T, cfg.K), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if cfg.name == "tiny_fp32" else None
+    e4m3 = args.experts == "e4m3"
+    if e4m3:
+        # quantised once, outside the timed region; the bf16 copies are freed
+        q = [t for w in (w1, w3, w2) for t in m.quantize_weights_e4m3(w)]
+        torch.cuda.synchronize(dev)
+        del w1, w3, w2
+        torch.cuda.empty_cache()
+
+    def forward(xin):
+        if e4m3:
+            m.moe_forward_e4m3(layer.h, T, xin, Wg, *q, y, idx, gw, stream)
+        else:
+            m.moe_forward(layer.h, T, xin, Wg, w1, w3, w2, y, idx, gw, stream)
 
     def step():
         if flush is not None:
             flush.fill_(1)
-        m.moe_forward(layer.h, T, x, Wg, w1, w3, w2, y, idx, gw, stream)
+        forward(x)
 
     for _ in range(args.warmup):
         step()
@@ -366,7 +407,7 @@ def main():
         if flush is not None:
             flush.fill_(1)
         xd.copy_(xh, non_blocking=True)
-        m.moe_forward(layer.h, T, xd, Wg, w1, w3, w2, y, idx, gw, stream)
+        forward(xd)
         yh.copy_(y, non_blocking=True)
         ih.copy_(idx, non_blocking=True)
         wh.copy_(gw, non_blocking=True)
@@ -389,7 +430,7 @@ def main():
 
     # ---- roofline of the dominant kernel ----
     peaks, peak_src = load_peaks()
-    work = algorithmic(cfg, counts)
+    work = algorithmic(cfg, counts, args.experts)
     per_launch = {k: v / max(1, traced) for k, v in stage_ms.items()}
     dom = max(("gemm1", "gemm2"), key=lambda k: per_launch[k])
     dom_ms = per_launch[dom]
@@ -397,7 +438,7 @@ def main():
         roof = None
     else:
         intensity = work[dom]["flops"] / work[dom]["bytes"]
-        ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        ridge = peaks["bf16_tflops"] * (2.0 if e4m3 else 1.0) * 1e12 / (peaks["hbm_gbs"] * 1e9)
         if intensity < ridge:
             ach = work[dom]["bytes"] / (dom_ms * 1e-3) / 1e9
             roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -405,6 +446,8 @@ def main():
         else:
             timed_s = ms * args.steps * 1e-3
             pk = peaks["bf16_tflops_sustained"] if timed_s > 1.0 else peaks["bf16_tflops"]
+            if e4m3:  # fp8 dense rate = 2x bf16 (nominal 4.5 vs 2.25 PFLOP/s)
+                pk *= 2.0
             ach = work[dom]["flops"] / (dom_ms * 1e-3) / 1e12
             roof = {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
                     "peak_kind": "sustained" if timed_s > 1.0 else "burst"}
@@ -412,23 +455,23 @@ def main():
         roof["peak_source"] = peak_src
         roof["algorithmic_per_launch"] = work[dom]["bytes"] if roof["bound"] == "hbm" else work[dom]["flops"]
         roof["launch_ms"] = dom_ms
-        roof["traffic"] = recorded_traffic(dom, cfg.name)
+        roof["traffic"] = recorded_traffic(dom, cfg.name + ("_e4m3" if e4m3 else ""))
 
     # ---- CPU baseline (rank 0, N = 1 only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, s, reps, cores, el = oracle_tokens_per_s(cfg, L)
+        v, s, reps, cores, el = oracle_tokens_per_s(cfg, L, experts=args.experts)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": "first %d of %d tokens x %d repetitions, full layer in fp64 (%.1f s)"
-                         % (s, cfg.T, reps, el)}
+               "sample": "first %d of %d tokens x %d repetitions, full layer in fp64%s (%.1f s)"
+                         % (s, cfg.T, reps, ", E4M3 experts" if e4m3 else "", el)}
 
     if rank == 0:
         layer_ms = ms
         line = {
             "metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
-            "config": {"workload": workload_desc(cfg), "global_batch_tokens": T * world,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if e4m3 else cfg.dtype, "data": "synthetic",
+            "config": {"workload": workload_desc(cfg, args.experts), "global_batch_tokens": T * world,
                        "parallelism": "replicas%d" % world if world > 1 else "single",
                        "l2": "256 MB flush per step" if flush is not None else
                              "no flush: %.2f GB of expert weights per step > 126 MB L2"

@@ -70,7 +70,7 @@ typedef enum {
 typedef enum {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = 1, /* bad size, null or misaligned pointer, wrong device */
-    MOE_ERR_UNSUPPORTED = 2, /* not an sm_100 device */
+    MOE_ERR_UNSUPPORTED = 2, /* not an sm_100 device, or a path the handle's dtype lacks */
     MOE_ERR_ALLOC = 3,       /* workspace cudaMalloc failed */
     MOE_ERR_CUDA = 4,        /* a CUDA runtime call or a launch failed */
     MOE_ERR_TIMEOUT = 5      /* a kernel gave up a bounded wait (see moe_sync_status) */
@@ -206,11 +206,54 @@ MOE_API moe_status moe_router_stats(moe_handle *h, int64_t T, const void *x, con
                                     float *aux, moe_stream_t stream);
 
 /*
- * Debug view of the workspace written by the last moe_forward /
- * moe_forward_with_routing: name is "H" (expert hidden layer, [rows][ffn],
- * handle dtype) or "O" (per-row expert outputs, [rows][d], handle dtype for
- * bf16 handles, fp32 for fp32 handles).  Returns the device pointer and the
- * row capacity; rows are in dispatch order.
+ * FP8 expert weights.  Part 4 of "Mixture of Experts: Why Mixtral Only Wakes
+ * Up Two Specialists" ("Why total and active both matter") sizes the weights at
+ * 16 bits and at lower precision; the pages fix no format.  This library
+ * stores them as E4M3 (OCP 8-bit floating point: exponent bias 7, largest
+ * finite 448, no infinities) with one fp32 scale per output column:
+ *   scale[e][c] = max_r |w[e][r][c]| / 448   (1 for an all-zero column)
+ *   code[e][r][c] = E4M3(fp32(w[e][r][c] / scale[e][c])), round to nearest,
+ *                   ties to even, saturating at +-448
+ * so w ~= decode(code) * scale.
+ *
+ * moe_quantize_weights_e4m3: w [n][rows][cols] (MOE_BF16 or MOE_F32, device)
+ * -> codes [n][rows][cols] (uint8, device) and scales [n][cols] (fp32, device).
+ * For the layer: w1 and w3 are [n][d][ffn] (scales [n][ffn]), w2 is
+ * [n][ffn][d] (scales [n][d]).  Needs no handle; enqueued on `stream`.
+ *   Errors: MOE_ERR_INVALID_ARG (n outside [1, 65535], rows < 1, cols not a
+ *   positive multiple of 16, n*rows*cols > 2^40, null / misaligned pointer),
+ *   MOE_ERR_UNSUPPORTED (not an sm_100 device), MOE_ERR_CUDA.
+ */
+MOE_API moe_status moe_quantize_weights_e4m3(int n, int rows, int cols, const void *w, moe_dtype dtype,
+                                             uint8_t *codes, float *scales, moe_stream_t stream);
+
+/*
+ * The layer of moe_forward with E4M3 experts (MOE_BF16 handles only): the same
+ * fp32 router, top-K, softmax and dispatch (and capacity, if set); then per
+ * dispatched (token, slot) row
+ *   x8  = E4M3 codes of x_t with the row scale sx = max|x_t| / 448;
+ *   h   = bf16( silu(sx * s1 (*) (x8 . q1_e)) (*) (sx * s3 (*) (x8 . q3_e)) );
+ *   h8  = E4M3 codes of h with the row scale sh = max|h| / 448;
+ *   o   = bf16( sh * s2 (*) (h8 . q2_e) ),   y_t = sum_k gate_k * o_k
+ * with fp32 tensor-core accumulation of the 8-bit products.  w*_q / w*_s are
+ * the codes and scales of moe_quantize_weights_e4m3; x, W_g, y, topk_idx,
+ * topk_w as for moe_forward.  The first call grows the workspace by
+ * T*K*(ffn + 8) bytes.
+ *   Errors: as moe_forward; MOE_ERR_UNSUPPORTED for an fp32 handle.
+ */
+MOE_API moe_status moe_forward_e4m3(moe_handle *h, int64_t T, const void *x, const float *W_g,
+                                    const uint8_t *w1_q, const float *w1_s, const uint8_t *w3_q,
+                                    const float *w3_s, const uint8_t *w2_q, const float *w2_s, void *y,
+                                    int32_t *topk_idx, float *topk_w, moe_stream_t stream);
+
+/*
+ * Debug view of the workspace written by the last forward call: name is "H"
+ * (expert hidden layer, [rows][ffn], handle dtype) or "O" (per-row expert
+ * outputs, [rows][d], handle dtype for bf16 handles, fp32 for fp32 handles);
+ * after moe_forward_e4m3 also "X8" (E4M3 codes of the gathered x rows,
+ * [rows][d] uint8), "XS" (their scales, [rows] fp32), "H8" (codes of H,
+ * [rows][ffn] uint8) and "HS" ([rows] fp32).  Returns the device pointer and
+ * the row capacity; rows are in dispatch order.
  *   Errors: MOE_ERR_INVALID_ARG (unknown name, null argument, no workspace yet).
  */
 MOE_API moe_status moe_workspace_view(moe_handle *h, const char *name, void **ptr, int64_t *rows);

@@ -555,6 +555,7 @@ int oracle_quantize_weights_e4m3(int n, int rows, int cols, const void *w, int w
 {
     if (n <= 0 || rows <= 0 || cols <= 0 || !w || !codes || !scales || !dt_ok(w_dt))
         return -1;
+#pragma omp parallel for collapse(2) schedule(static)
     for (int e = 0; e < n; ++e)
         for (int c = 0; c < cols; ++c) {
             float amax = 0.0f;

@@ -62,20 +62,23 @@ lib.moe_set_capacity_factor.argtypes = [_vp, ctypes.c_double]
 lib.moe_router_stats.argtypes = [_vp, _i64, _vp, _vp, _vp, ctypes.c_float, _vp, _vp, _vp, _vp]
 lib.moe_dispatch_noalloc.argtypes = [_i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.moe_trace_end.argtypes = [_vp, ctypes.POINTER(ctypes.c_double), _int, ctypes.POINTER(_int)]
+lib.moe_quantize_weights_e4m3.argtypes = [_int, _int, _int, _vp, _int, _vp, _vp, _vp]
+lib.moe_forward_e4m3.argtypes = [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.moe_last_error.restype = ctypes.c_char_p
 lib.moe_version.restype = ctypes.c_char_p
 for _f in ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
            "moe_forward_with_routing", "moe_workspace_view", "moe_sync_status", "moe_destroy",
            "moe_trace_begin", "moe_trace_end", "moe_dispatch_noalloc", "moe_set_capacity_factor",
            "moe_router_stats", "moe_launch_count", "moe_selftest_timeout",
-           "moe_forward_expert_choice"):
+           "moe_forward_expert_choice", "moe_quantize_weights_e4m3", "moe_forward_e4m3"):
     getattr(lib, _f).restype = _int
 
 EXPORTED = ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
             "moe_forward_with_routing", "moe_workspace_view", "moe_sync_status", "moe_destroy",
             "moe_last_error", "moe_version", "moe_trace_begin", "moe_trace_end",
             "moe_dispatch_noalloc", "moe_set_capacity_factor", "moe_router_stats",
-            "moe_launch_count", "moe_selftest_timeout", "moe_forward_expert_choice")
+            "moe_launch_count", "moe_selftest_timeout", "moe_forward_expert_choice",
+            "moe_quantize_weights_e4m3", "moe_forward_e4m3")
 
 TRACE_STAGES = ("router", "dispatch", "gather", "gemm1", "gemm2", "combine")
 
@@ -206,6 +209,30 @@ def moe_launch_count(h) -> int:
     return c.value
 
 
+def moe_quantize_weights_e4m3(n, rows, cols, w, dtype, codes, scales, stream=None) -> None:
+    _check(lib.moe_quantize_weights_e4m3(n, rows, cols, _ptr(w), dtype, _ptr(codes), _ptr(scales),
+                                         _stream(stream)), "moe_quantize_weights_e4m3")
+
+
+def moe_forward_e4m3(h, T, x, W_g, w1_q, w1_s, w3_q, w3_s, w2_q, w2_s, y, topk_idx, topk_w,
+                     stream=None) -> None:
+    _check(lib.moe_forward_e4m3(h, T, _ptr(x), _ptr(W_g), _ptr(w1_q), _ptr(w1_s), _ptr(w3_q), _ptr(w3_s),
+                                _ptr(w2_q), _ptr(w2_s), _ptr(y), _ptr(topk_idx), _ptr(topk_w),
+                                _stream(stream)), "moe_forward_e4m3")
+
+
+def quantize_weights_e4m3(w, stream=None):
+    """w [n][rows][cols] (torch bf16 or fp32, CUDA) -> (codes uint8 [n][rows][cols],
+    scales fp32 [n][cols]), one scale per output column."""
+    import torch
+    n, rows, cols = w.shape
+    codes = torch.empty((n, rows, cols), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((n, cols), dtype=torch.float32, device=w.device)
+    moe_quantize_weights_e4m3(n, rows, cols, w, MOE_BF16 if w.dtype == torch.bfloat16 else MOE_F32,
+                              codes, scales, stream)
+    return codes, scales
+
+
 def moe_destroy(h) -> None:
     _check(lib.moe_destroy(h), "moe_destroy")
 
@@ -272,6 +299,20 @@ class MoELayer:
         gate = torch.empty((self.n, capacity), dtype=torch.float32, device=x.device)
         moe_forward_expert_choice(self.h, T, capacity, x, W_g, w1, w3, w2, y, sel, gate, stream)
         return y, sel, gate
+
+    def forward_e4m3(self, x, W_g, w1_q, w1_s, w3_q, w3_s, w2_q, w2_s, y=None, topk_idx=None,
+                     topk_w=None, stream=None):
+        """The layer with E4M3 experts (codes and scales of quantize_weights_e4m3)."""
+        import torch
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty_like(x)
+        if topk_idx is None:
+            topk_idx = torch.empty((T, self.K), dtype=torch.int32, device=x.device)
+        if topk_w is None:
+            topk_w = torch.empty((T, self.K), dtype=torch.float32, device=x.device)
+        moe_forward_e4m3(self.h, T, x, W_g, w1_q, w1_s, w3_q, w3_s, w2_q, w2_s, y, topk_idx, topk_w, stream)
+        return y, topk_idx, topk_w
 
     def set_capacity_factor(self, factor: float) -> None:
         moe_set_capacity_factor(self.h, factor)

@@ -29,6 +29,13 @@
 // the per-expert M-block prefix the dispatch wrote, so nothing returns to the
 // host between routing and the experts.
 //
+// E4M3 variant (kFp8): the same pipeline over 8-bit operands (a stage is 128
+// K-elements: A 128 x 128 bytes; B two 128-column boxes of 128 K-rows), four
+// kind::f8f6f4 MMAs (K = 32) per stage, and epilogues that undo the scales:
+// GEMM1 multiplies the accumulators by the row's activation scale and the
+// column's weight scale before the SwiGLU, GEMM2 by the hidden row's scale and
+// the column's w2 scale.
+//
 // Every wait is bounded (common.cuh): a pipeline that stops making progress
 // sets a status bit and the CTA drains and exits instead of hanging.
 #include "common.cuh"
@@ -39,6 +46,8 @@ namespace moe {
 constexpr int kBM = kTcBM;           // 128 rows per tile (MMA M)
 constexpr int kBN = 256;             // MMA N
 constexpr int kBK = 64;              // K per stage (one 128-byte swizzle row of bf16)
+constexpr int kBK8 = 128;            // K per stage of the E4M3 kernels (128 bytes too)
+constexpr int kB8ChunkBytes = kBK8 * 128;         // 16 KB: 128 K-rows x 128 one-byte columns
 constexpr int kStages = 4;
 constexpr int kABytes = kBM * kBK * 2;            // 16 KB
 constexpr int kBChunkBytes = kBK * 64 * 2;        // 8 KB: 64 K-rows x 64 columns
@@ -92,7 +101,8 @@ __device__ __forceinline__ TileInfo tile_info(int t, const int32_t* off, const i
 __device__ __forceinline__ float silu_f(float a) { return a / (1.f + __expf(-a)); }
 
 // kSwiGLU: GEMM1 (two B maps, 128 output columns per tile); else GEMM2.
-template <bool kSwiGLU>
+// kFp8: E4M3 operands with the scales of TcGemmArgs applied in the epilogue.
+template <bool kSwiGLU, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
                    const __grid_constant__ CUtensorMap tm_b1, const TcGemmArgs args) {
@@ -161,9 +171,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     armed[stage] = static_cast<int>(phase);
                     const uint32_t a_dst = smem_u32(smem + stage * kStageBytes);
                     const uint32_t b_dst = a_dst + kABytes;
-                    const int k0 = kb * kBK;
+                    const int k0 = kb * (kFp8 ? kBK8 : kBK);
                     tma_load_2d(a_dst, &tm_a, fb, k0, ti.row0);
-                    if (kSwiGLU) {
+                    if (kFp8) {
+                        if (kSwiGLU) {
+                            const int c0 = ti.n_tile * 128;
+                            tma_load_3d(b_dst, &tm_b0, fb, c0, k0, ti.e);
+                            tma_load_3d(b_dst + kB8ChunkBytes, &tm_b1, fb, c0, k0, ti.e);
+                        } else {
+                            const int c0 = ti.n_tile * 256;
+                            tma_load_3d(b_dst, &tm_b0, fb, c0, k0, ti.e);
+                            tma_load_3d(b_dst + kB8ChunkBytes, &tm_b0, fb, c0 + 128, k0, ti.e);
+                        }
+                    } else if (kSwiGLU) {
                         const int c0 = ti.n_tile * 128;
                         tma_load_3d(b_dst + 0 * kBChunkBytes, &tm_b0, fb, c0, k0, ti.e);
                         tma_load_3d(b_dst + 1 * kBChunkBytes, &tm_b0, fb, c0 + 64, k0, ti.e);
@@ -190,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer ----------------
-            constexpr uint32_t idesc = make_idesc_bf16(kBM, kBN, 0, 1);
+            constexpr uint32_t idesc = kFp8 ? make_idesc_e4m3(kBM, kBN, 0, 1) : make_idesc_bf16(kBM, kBN, 0, 1);
             int stage = 0;
             uint32_t phase = 0;
             int local = 0;
@@ -213,6 +233,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     const uint32_t a_base = smem_u32(smem + stage * kStageBytes);
                     const uint32_t b_base = a_base + kABytes;
+                    if (kFp8) {
+#pragma unroll
+                        for (int kk = 0; kk < kBK8 / 32; ++kk) {
+                            // A: K-major, 128-byte swizzle; K by 32 one-byte elements moves 32
+                            // bytes inside the swizzle row.  B: N-major, 128-byte swizzle, two
+                            // 128-column chunks 16 KB apart (LBO); K by 32 = four 8-row groups.
+                            const uint64_t adesc = make_smem_desc(a_base + kk * 32, 16, 1024, 2);
+                            const uint64_t bdesc =
+                                make_smem_desc(b_base + kk * 4096, kB8ChunkBytes, 1024, 2);
+                            tc_mma_f8(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        }
+                    } else {
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
                         // A: K-major, 128-byte swizzle; advancing K by 16 moves 32 bytes
@@ -223,6 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint64_t bdesc =
                             make_smem_desc(b_base + kk * 2048, kBChunkBytes, 1024, 2);
                         tc_mma_f16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
                     }
                     tc_commit(smem_u32(&tail->empty[stage]));
                     if (++stage == kStages) {
@@ -257,6 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // GEMM1: direct 16-byte stores of each lane's row (measured faster here
                 // than staging through shared memory)
                 const bool row_ok = lane < valid;
+                const float rs = (kFp8 && row_ok) ? args.row_scale[row_base + lane] : 1.f;
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t a[32], b[32];
@@ -265,6 +299,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_wait_ld();
                     const int col = ti.n_tile * 128 + c * 32;
                     if (row_ok && col < args.out_cols) {
+                        if (kFp8) {
+                            // dequantise: accumulator x row scale x column scale
+                            const float4* s0 = reinterpret_cast<const float4*>(
+                                args.col_scale0 + static_cast<int64_t>(ti.e) * args.out_cols + col);
+                            const float4* s1 = reinterpret_cast<const float4*>(
+                                args.col_scale1 + static_cast<int64_t>(ti.e) * args.out_cols + col);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                const float4 u = __ldg(s0 + q), v = __ldg(s1 + q);
+                                a[4 * q + 0] = __float_as_uint(__uint_as_float(a[4 * q + 0]) * rs * u.x);
+                                a[4 * q + 1] = __float_as_uint(__uint_as_float(a[4 * q + 1]) * rs * u.y);
+                                a[4 * q + 2] = __float_as_uint(__uint_as_float(a[4 * q + 2]) * rs * u.z);
+                                a[4 * q + 3] = __float_as_uint(__uint_as_float(a[4 * q + 3]) * rs * u.w);
+                                b[4 * q + 0] = __float_as_uint(__uint_as_float(b[4 * q + 0]) * rs * v.x);
+                                b[4 * q + 1] = __float_as_uint(__uint_as_float(b[4 * q + 1]) * rs * v.y);
+                                b[4 * q + 2] = __float_as_uint(__uint_as_float(b[4 * q + 2]) * rs * v.z);
+                                b[4 * q + 3] = __float_as_uint(__uint_as_float(b[4 * q + 3]) * rs * v.w);
+                            }
+                        }
                         uint32_t pk[16];
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
@@ -280,19 +333,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             } else {
+                const float rs = (kFp8 && lane < valid) ? args.row_scale[row_base + lane] : 1.f;
 #pragma unroll 1
                 for (int g = 0; g < 4; ++g) {
                     uint32_t pk[32];
+                    const int col = ti.n_tile * 256 + g * 64;
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
                         uint32_t a[32];
                         tmem_ld_32x32b_x32(tbase + g * 64 + c * 32, a);
                         tmem_wait_ld();
+                        if (kFp8 && col < args.out_cols) {
+                            const float4* s0 = reinterpret_cast<const float4*>(
+                                args.col_scale0 + static_cast<int64_t>(ti.e) * args.out_cols + col + c * 32);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                const float4 u = __ldg(s0 + q);
+                                a[4 * q + 0] = __float_as_uint(__uint_as_float(a[4 * q + 0]) * rs * u.x);
+                                a[4 * q + 1] = __float_as_uint(__uint_as_float(a[4 * q + 1]) * rs * u.y);
+                                a[4 * q + 2] = __float_as_uint(__uint_as_float(a[4 * q + 2]) * rs * u.z);
+                                a[4 * q + 3] = __float_as_uint(__uint_as_float(a[4 * q + 3]) * rs * u.w);
+                            }
+                        }
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
                             pk[c * 16 + j] = pack_bf16x2(__uint_as_float(a[2 * j]), __uint_as_float(a[2 * j + 1]));
                     }
-                    const int col = ti.n_tile * 256 + g * 64;
                     if (col < args.out_cols && valid > 0)
                         warp_store_rows_64(stage, pk, lane, out, args.out_cols, row_base, valid, col);
                 }
@@ -319,25 +385,37 @@ static int grid_for(const TcGemmArgs& a, int num_sms) {
     return static_cast<int>(g < 1 ? 1 : g);
 }
 
-template <bool kSwiGLU>
+template <bool kSwiGLU, bool kFp8>
 static cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1,
                              const TcGemmArgs& a, int num_sms, cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<kSwiGLU>,
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<kSwiGLU, kFp8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    launch_k(tc_gemm_kernel<kSwiGLU>, dim3(grid_for(a, num_sms)), dim3(kThreads), kSmemBytes, st, ta, tb0, tb1, a);
+    launch_k(tc_gemm_kernel<kSwiGLU, kFp8>, dim3(grid_for(a, num_sms)), dim3(kThreads), kSmemBytes, st, ta, tb0,
+             tb1, a);
     return cudaGetLastError();
 }
 
 cudaError_t launch_tc_gemm1(const CUtensorMap& tm_xp, const CUtensorMap& tm_w1,
                             const CUtensorMap& tm_w3, const TcGemmArgs& a, int num_sms,
                             cudaStream_t st) {
-    return launch_tc<true>(tm_xp, tm_w1, tm_w3, a, num_sms, st);
+    return launch_tc<true, false>(tm_xp, tm_w1, tm_w3, a, num_sms, st);
 }
 
 cudaError_t launch_tc_gemm2(const CUtensorMap& tm_h, const CUtensorMap& tm_w2, const TcGemmArgs& a,
                             int num_sms, cudaStream_t st) {
-    return launch_tc<false>(tm_h, tm_w2, tm_w2, a, num_sms, st);
+    return launch_tc<false, false>(tm_h, tm_w2, tm_w2, a, num_sms, st);
+}
+
+cudaError_t launch_tc_gemm1_e4m3(const CUtensorMap& tm_x8, const CUtensorMap& tm_q1,
+                                 const CUtensorMap& tm_q3, const TcGemmArgs& a, int num_sms,
+                                 cudaStream_t st) {
+    return launch_tc<true, true>(tm_x8, tm_q1, tm_q3, a, num_sms, st);
+}
+
+cudaError_t launch_tc_gemm2_e4m3(const CUtensorMap& tm_h8, const CUtensorMap& tm_q2, const TcGemmArgs& a,
+                                 int num_sms, cudaStream_t st) {
+    return launch_tc<false, true>(tm_h8, tm_q2, tm_q2, a, num_sms, st);
 }
 
 }  // namespace moe

@@ -144,6 +144,11 @@ struct TcGemmArgs {
     int out_cols;      // F (GEMM1) or d (GEMM2)
     void* out;         // H (GEMM1) or O (GEMM2), bf16 row-major [R][out_cols]
     int* status;       // device status word
+    // E4M3 kernels only: row scale [R] and per-expert column scales [n][out_cols]
+    // (GEMM1: w1 and w3; GEMM2: w2 in col_scale0)
+    const float* row_scale;
+    const float* col_scale0;
+    const float* col_scale1;
 };
 
 cudaError_t launch_tc_gemm1(const CUtensorMap& tm_xp, const CUtensorMap& tm_w1,
@@ -151,6 +156,26 @@ cudaError_t launch_tc_gemm1(const CUtensorMap& tm_xp, const CUtensorMap& tm_w1,
                             cudaStream_t st);
 cudaError_t launch_tc_gemm2(const CUtensorMap& tm_h, const CUtensorMap& tm_w2, const TcGemmArgs& a,
                             int num_sms, cudaStream_t st);
+cudaError_t launch_tc_gemm1_e4m3(const CUtensorMap& tm_x8, const CUtensorMap& tm_q1,
+                                 const CUtensorMap& tm_q3, const TcGemmArgs& a, int num_sms,
+                                 cudaStream_t st);
+cudaError_t launch_tc_gemm2_e4m3(const CUtensorMap& tm_h8, const CUtensorMap& tm_q2, const TcGemmArgs& a,
+                                 int num_sms, cudaStream_t st);
+
+// E4M3 quantisation (e4m3.cu).  Codes are those of v / scale with the quotient
+// rounded to fp32, then to E4M3 by round-to-nearest-even with saturation to
+// +-448; scale = max |v| / 448 over the group (1 for an all-zero group).
+//   weights [n][rows][cols] -> codes of the same shape, scales [n][cols] (per
+//   output column over the reduction rows); three launches.
+cudaError_t launch_quantize_weights_e4m3(const void* w, bool bf16, int n, int rows, int cols,
+                                         uint8_t* codes, float* scales, int num_sms, cudaStream_t st);
+//   rows of src (bf16 or fp32, `cols` wide) -> codes [rows][cols] and one scale
+//   per row.  With row_src, row r reads source row row_src[r] (a gather; rows
+//   whose source is outside [0, src_rows) are skipped); with row_limit, rows at
+//   or past *row_limit are skipped.
+cudaError_t launch_quantize_rows_e4m3(const void* src, bool bf16, const int32_t* row_src, int64_t src_rows,
+                                      int64_t rows, const int32_t* row_limit, int cols, uint8_t* codes,
+                                      float* scales, int num_sms, cudaStream_t st);
 
 // The same GEMMs on CTA pairs (cta_group::2, 256-row tiles): mblk_base must
 // count 256-row blocks.

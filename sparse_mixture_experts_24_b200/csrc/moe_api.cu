@@ -109,6 +109,20 @@ bool encode_weights(CUtensorMap* m, const void* base, uint64_t cols, uint64_t ro
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// E4M3 codes, uint8: [rows][cols] (box_rows x 128) or weights [n][rows][cols]
+// (128 x 128 boxes of one expert); out-of-range boxes read zeros.
+bool encode_codes(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t n) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[3] = {cols, rows, n};
+    cuuint64_t strides[2] = {cols, cols * rows};
+    cuuint32_t box[3] = {128, 128, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, n ? 3 : 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 struct moe_handle {
@@ -144,6 +158,18 @@ struct moe_handle {
     // expert-choice routing: probabilities [n][T], row of (token, expert) [T][n]
     float* ec_probs = nullptr;
     int32_t* ec_rowmap = nullptr;
+    // E4M3 experts: the workspace also holds x8 (in the Xp buffer), h8 and the
+    // row scales once a call has asked for them
+    bool want_e4m3 = false;
+    bool has_e4m3 = false;
+    uint8_t* x8 = nullptr;
+    uint8_t* h8 = nullptr;
+    float* xs = nullptr;
+    float* hs = nullptr;
+    CUtensorMap tm_x8, tm_h8, tm_q1, tm_q3, tm_q2;
+    const void* c_q1 = nullptr;
+    const void* c_q3 = nullptr;
+    const void* c_q2 = nullptr;
     // tracing: kTraceEvents events per traced call
     std::vector<cudaEvent_t> trace_ev;
     int trace_max = 0;
@@ -208,7 +234,7 @@ moe_status check_device(moe_handle* h) {
 // token-choice calls, n*C for expert-choice calls).  Capacities only grow.
 moe_status grow(moe_handle* h, int64_t T, int64_t rows_min = 0) {
     const int64_t R_need = std::max(T * h->K, rows_min);
-    if (h->ws && T <= h->T_cap && R_need <= h->R_cap) return MOE_OK;
+    if (h->ws && T <= h->T_cap && R_need <= h->R_cap && (h->has_e4m3 || !h->want_e4m3)) return MOE_OK;
     T = std::max(T, h->T_cap);
     const int64_t R = std::max(std::max(R_need, h->R_cap), T * h->K);
     const int64_t nblk = (R + moe::kPairsPerBlock - 1) / moe::kPairsPerBlock;
@@ -238,6 +264,10 @@ moe_status grow(moe_handle* h, int64_t T, int64_t rows_min = 0) {
     const size_t o_xp = take(static_cast<size_t>(R) * h->d * h->esize());
     const size_t o_h = take(static_cast<size_t>(R) * h->F * h->esize());
     const size_t o_o = take(static_cast<size_t>(R) * h->d * h->osize());
+    const bool e4 = h->want_e4m3;
+    const size_t o_h8 = take(e4 ? static_cast<size_t>(R) * h->F : 0);
+    const size_t o_xs = take(e4 ? static_cast<size_t>(R) * 4 : 0);
+    const size_t o_hs = take(e4 ? static_cast<size_t>(R) * 4 : 0);
     const size_t total = off;
 
     if (h->ws) {
@@ -281,6 +311,14 @@ moe_status grow(moe_handle* h, int64_t T, int64_t rows_min = 0) {
     h->xp = b + o_xp;
     h->h = b + o_h;
     h->o = b + o_o;
+    h->has_e4m3 = e4;
+    h->x8 = e4 ? static_cast<uint8_t*>(h->xp) : nullptr;
+    h->h8 = e4 ? b + o_h8 : nullptr;
+    h->xs = e4 ? reinterpret_cast<float*>(b + o_xs) : nullptr;
+    h->hs = e4 ? reinterpret_cast<float*>(b + o_hs) : nullptr;
+    if (e4 && (!encode_codes(&h->tm_x8, h->x8, h->d, static_cast<uint64_t>(R), 0) ||
+               !encode_codes(&h->tm_h8, h->h8, h->F, static_cast<uint64_t>(R), 0)))
+        return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the E4M3 workspace");
     if (h->dtype == MOE_BF16) {
         if (!encode_rows(&h->tm_xp, h->xp, h->d, static_cast<uint64_t>(R)) ||
             !encode_rows(&h->tm_h, h->h, h->F, static_cast<uint64_t>(R)) ||
@@ -438,6 +476,77 @@ moe_status run_experts(moe_handle* h, int64_t T, const void* x, const int32_t* t
     moe_status s = run_gemms(h, T, R, x, w1, w3, w2, pair, st);
     if (s != MOE_OK) return s;
     e = moe::launch_combine(h->o, bf, h->db.token_row, topk_w, T, h->K, h->d, y, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+    h->launches += 1;
+    trace_mark(h, 5, st);
+    trace_finish_call(h);
+    return MOE_OK;
+}
+
+// The E4M3 expert path: dispatch, quantised gather of x (one scale per row),
+// GEMM1 on E4M3 operands (bf16 H), H rows to E4M3 (one scale per row), GEMM2
+// on E4M3 operands (bf16 O), combine.
+moe_status run_experts_e4m3(moe_handle* h, int64_t T, const void* x, const int32_t* topk_idx,
+                            const float* topk_w, const uint8_t* q1, const float* s1, const uint8_t* q3,
+                            const float* s3, const uint8_t* q2, const float* s2, void* y, cudaStream_t st) {
+    const int64_t R = T * h->K;
+    cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n, moe::kTcBM, h->db, st, capacity_for(h, T));
+    if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
+    h->launches += moe::dispatch_kernel_count(R);
+    trace_mark(h, 1, st);
+    const int32_t* used_rows = h->db.offsets + h->n;  // offsets[n]: rows the segments hold
+    e = moe::launch_quantize_rows_e4m3(x, true, h->db.row_token, T, R, used_rows, h->d, h->x8, h->xs, h->num_sms,
+                                       st);
+    if (e != cudaSuccess) return cuda_fail(e, "activation quantisation launch");
+    h->launches += 1;
+    trace_mark(h, 2, st);
+    if (q1 != h->c_q1) {
+        if (!encode_codes(&h->tm_q1, q1, h->F, h->d, h->n))
+            return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for w1 codes");
+        h->c_q1 = q1;
+    }
+    if (q3 != h->c_q3) {
+        if (!encode_codes(&h->tm_q3, q3, h->F, h->d, h->n))
+            return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for w3 codes");
+        h->c_q3 = q3;
+    }
+    if (q2 != h->c_q2) {
+        if (!encode_codes(&h->tm_q2, q2, h->d, h->F, h->n))
+            return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for w2 codes");
+        h->c_q2 = q2;
+    }
+    moe::TcGemmArgs a1{};
+    a1.offsets = h->db.offsets;
+    a1.mblk_base = h->db.mblk_base;
+    a1.n = h->n;
+    a1.R = R;
+    a1.k_blocks = (h->d + 127) / 128;
+    a1.n_tiles = (h->F + 127) / 128;
+    a1.out_cols = h->F;
+    a1.out = h->h;
+    a1.status = h->status;
+    a1.row_scale = h->xs;
+    a1.col_scale0 = s1;
+    a1.col_scale1 = s3;
+    e = moe::launch_tc_gemm1_e4m3(h->tm_x8, h->tm_q1, h->tm_q3, a1, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
+    e = moe::launch_quantize_rows_e4m3(h->h, true, nullptr, R, R, used_rows, h->F, h->h8, h->hs, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "hidden-row quantisation launch");
+    h->launches += 2;
+    trace_mark(h, 3, st);
+    moe::TcGemmArgs a2 = a1;
+    a2.k_blocks = (h->F + 127) / 128;
+    a2.n_tiles = (h->d + 255) / 256;
+    a2.out_cols = h->d;
+    a2.out = h->o;
+    a2.row_scale = h->hs;
+    a2.col_scale0 = s2;
+    a2.col_scale1 = nullptr;
+    e = moe::launch_tc_gemm2_e4m3(h->tm_h8, h->tm_q2, a2, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
+    h->launches += 1;
+    trace_mark(h, 4, st);
+    e = moe::launch_combine(h->o, true, h->db.token_row, topk_w, T, h->K, h->d, y, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "combine launch");
     h->launches += 1;
     trace_mark(h, 5, st);
@@ -657,6 +766,63 @@ moe_status moe_forward_expert_choice(moe_handle* h, int64_t T, int64_t capacity,
     return ok();
 }
 
+moe_status moe_quantize_weights_e4m3(int n, int rows, int cols, const void* w, moe_dtype dtype, uint8_t* codes,
+                                     float* scales, moe_stream_t stream) {
+    if (n < 1 || n > 65535) return fail(MOE_ERR_INVALID_ARG, "n = %d outside [1, 65535]", n);
+    if (rows < 1) return fail(MOE_ERR_INVALID_ARG, "rows = %d < 1", rows);
+    if (cols < 16 || cols % 16 != 0)
+        return fail(MOE_ERR_INVALID_ARG, "cols = %d is not a positive multiple of 16", cols);
+    if (dtype != MOE_F32 && dtype != MOE_BF16)
+        return fail(MOE_ERR_INVALID_ARG, "dtype = %d is not MOE_F32 or MOE_BF16", static_cast<int>(dtype));
+    if (static_cast<int64_t>(n) * rows * cols > (static_cast<int64_t>(1) << 40))
+        return fail(MOE_ERR_INVALID_ARG, "n * rows * cols exceeds 2^40");
+    REQUIRE_PTR(w);
+    REQUIRE_PTR(codes);
+    REQUIRE_PTR(scales);
+    int dev = 0, sms = 0, major = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (major != 10) return fail(MOE_ERR_UNSUPPORTED, "device %d is not sm_100", dev);
+    e = moe::launch_quantize_weights_e4m3(w, dtype == MOE_BF16, n, rows, cols, codes, scales, sms,
+                                          reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "weight quantisation launch");
+    return ok();
+}
+
+moe_status moe_forward_e4m3(moe_handle* h, int64_t T, const void* x, const float* W_g, const uint8_t* w1_q,
+                            const float* w1_s, const uint8_t* w3_q, const float* w3_s, const uint8_t* w2_q,
+                            const float* w2_s, void* y, int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
+    moe_status s = check_common(h, T);
+    if (s != MOE_OK) return s;
+    if (h->dtype != MOE_BF16)
+        return fail(MOE_ERR_UNSUPPORTED, "the E4M3 expert path needs a MOE_BF16 handle");
+    if (T == 0) return ok();
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(W_g);
+    REQUIRE_PTR(w1_q);
+    REQUIRE_PTR(w1_s);
+    REQUIRE_PTR(w3_q);
+    REQUIRE_PTR(w3_s);
+    REQUIRE_PTR(w2_q);
+    REQUIRE_PTR(w2_s);
+    REQUIRE_PTR(y);
+    REQUIRE_PTR(topk_idx);
+    REQUIRE_PTR(topk_w);
+    h->want_e4m3 = true;
+    s = prepare(h, T);
+    if (s != MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    moe::chain_begin();
+    trace_mark(h, -1, st);
+    s = run_router(h, T, x, W_g, topk_idx, topk_w, st);
+    if (s != MOE_OK) return s;
+    trace_mark(h, 0, st);
+    s = run_experts_e4m3(h, T, x, topk_idx, topk_w, w1_q, w1_s, w3_q, w3_s, w2_q, w2_s, y, st);
+    return s == MOE_OK ? ok() : s;
+}
+
 moe_status moe_set_capacity_factor(moe_handle* h, double factor) {
     if (!h) return fail(MOE_ERR_INVALID_ARG, "null handle");
     if (!(factor >= 0.0) || !std::isfinite(factor))
@@ -700,8 +866,13 @@ moe_status moe_workspace_view(moe_handle* h, const char* name, void** ptr, int64
         *ptr = h->h;
     else if (strcmp(name, "O") == 0)
         *ptr = h->o;
-    else
-        return fail(MOE_ERR_INVALID_ARG, "unknown workspace buffer '%s' (use \"H\" or \"O\")", name);
+    else if (strcmp(name, "X8") == 0 || strcmp(name, "H8") == 0 || strcmp(name, "XS") == 0 ||
+             strcmp(name, "HS") == 0) {
+        if (!h->has_e4m3) return fail(MOE_ERR_INVALID_ARG, "no E4M3 workspace yet (no moe_forward_e4m3 call)");
+        *ptr = name[0] == 'X' ? (name[1] == '8' ? static_cast<void*>(h->x8) : static_cast<void*>(h->xs))
+                              : (name[1] == '8' ? static_cast<void*>(h->h8) : static_cast<void*>(h->hs));
+    } else
+        return fail(MOE_ERR_INVALID_ARG, "unknown workspace buffer '%s' (H, O, X8, XS, H8, HS)", name);
     *rows = h->R_cap;
     return ok();
 }

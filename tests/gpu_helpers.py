@@ -36,6 +36,28 @@ def host(t) -> np.ndarray:
     return t.numpy()
 
 
+class DevArray:
+    """Borrowed view of device memory for torch.as_tensor (CUDA array interface)."""
+
+    def __init__(self, ptr, shape, typestr):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr,
+                                         "data": (int(ptr), False), "version": 3, "strides": None}
+
+
+def read_workspace(layer, name: str, rows: int, cols: int, dtype) -> np.ndarray:
+    """Copy rows x cols of a handle's workspace buffer to a numpy array of
+    `dtype` (uint8, uint16 for bf16 bits, float32)."""
+    import sparse_mixture_experts_24_b200 as m
+    torch = require_cuda()
+    ptr, cap = m.moe_workspace_view(layer.h, name)
+    assert cap >= rows
+    typestr = {np.dtype(np.uint8): "|u1", np.dtype(np.uint16): "<i2", np.dtype(np.float32): "<f4"}[np.dtype(dtype)]
+    torch.cuda.synchronize()
+    t = torch.as_tensor(DevArray(ptr, (rows, cols), typestr), device="cuda").clone()
+    torch.cuda.synchronize()
+    return t.cpu().numpy().view(dtype)
+
+
 def y_as_f64(y: np.ndarray) -> np.ndarray:
     return mi.as_f32(y).astype(np.float64)
 
