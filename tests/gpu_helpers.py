@@ -96,6 +96,14 @@ def compare_routing(gpu_idx, gpu_w, o_idx, o_gate, o_logits, x, Wg, K):
             "order_differs": int((~same_order & same_set).sum()), "max_gate_err": float(err.max()) if err.size else 0.0}
 
 
+def agreeing_tokens(gpu_idx, o_idx) -> np.ndarray:
+    """Tokens whose GPU routing equals the oracle's (order included); the
+    others are near-ties that compare_routing has already accounted for."""
+    agree = (gpu_idx == o_idx).all(axis=1)
+    assert agree.mean() >= 0.99, "routing agrees on only %.3f of the tokens" % agree.mean()
+    return agree
+
+
 def stratified_sample(idx: np.ndarray, n: int, count: int, seed: int = 0) -> np.ndarray:
     """Token sample that includes at least one token of every used expert."""
     rng = np.random.default_rng(seed)

@@ -39,15 +39,19 @@ def test_capacity_forward_and_dispatch(case):
         y, idx, w = host(y), host(idx_d), host(w_d)
     finally:
         layer.close()
-    c, o, rt, tr = oracle.dispatch_capacity(idx, n, C)
+    o_idx, o_gate, _ = oracle.router(L["x"], L["W_g"], K)
+    # capacity makes every later pair depend on the routing of all earlier
+    # tokens, so these cases are chosen to route exactly as the oracle does
+    assert np.array_equal(idx, o_idx), "routing differs from the oracle's"
+    c, o, rt, tr = oracle.dispatch_capacity(o_idx, n, C)
     assert np.array_equal(counts, c) and np.array_equal(offsets, o)
     assert np.array_equal(token_row, tr)
     assert np.array_equal(row_token[:o[-1]], rt[:o[-1]])
     dropped = tr < 0
     if factor <= 1.0:
         assert dropped.any(), "the case should overflow an expert"
-    gate = np.where(dropped, 0.0, w.astype(np.float64))
-    y_ref = oracle.forward_with_routing(L["x"], idx, gate, L["w1"], L["w3"], L["w2"])
+    gate = np.where(dropped, 0.0, o_gate)
+    y_ref = oracle.forward_with_routing(L["x"], o_idx, gate, L["w1"], L["w3"], L["w2"])
     err = rel_l2(y_as_f64(y), y_ref)
     assert err <= TOL_Y[dt], (name, err)
     fully = dropped.all(axis=1)
@@ -73,15 +77,15 @@ def test_router_stats_match_oracle(case):
     L = mi.make_layer(cfg, seed=zlib.crc32(name.encode()) % 1000, only=("x", "W_g"))
     layer = m.MoELayer(n, K, d, 64, dt)
     try:
-        x, Wg = dev(L["x"]), dev(L["W_g"])
-        idx_d, _ = layer.route(x, Wg)
+        # the statistics take the routing as an input: both sides get the oracle's
+        o_idx, _, _ = oracle.router(L["x"], L["W_g"], K)
+        x, Wg, idx_d = dev(L["x"]), dev(L["W_g"]), dev(o_idx)
         f, P, aux = (host(t) for t in layer.router_stats(x, Wg, idx_d, alpha=0.02))
         f2, P2, aux2 = (host(t) for t in layer.router_stats(x, Wg, idx_d, alpha=0.02))
         layer.sync_status()
-        idx = host(idx_d)
     finally:
         layer.close()
-    of, oP, oaux = oracle.router_stats(L["x"], L["W_g"], idx, 0.02)
+    of, oP, oaux = oracle.router_stats(L["x"], L["W_g"], o_idx, 0.02)
     # integer counts: f is exact up to the one fp32 division
     assert np.allclose(f, of, rtol=1e-6, atol=0)
     # P: fp32 logits and softmax, fp32 sum over T tokens

@@ -5,7 +5,7 @@ import pytest
 
 import moe_inputs as mi
 import oracle
-from gpu_helpers import TOL_Y, compare_routing, dev, host, rel_l2, require_cuda, y_as_f64
+from gpu_helpers import TOL_Y, agreeing_tokens, compare_routing, dev, host, rel_l2, require_cuda, y_as_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -13,8 +13,9 @@ pytestmark = pytest.mark.gpu
 def _check_layer(cfg, L, y, idx, w):
     o_idx, o_gate, o_logits = oracle.router(L["x"], L["W_g"], cfg.K)
     compare_routing(idx, w, o_idx, o_gate, o_logits, L["x"], L["W_g"], cfg.K)
-    y_ref = oracle.forward_with_routing(L["x"], idx, w.astype(np.float64), L["w1"], L["w3"], L["w2"])
-    assert rel_l2(y_as_f64(y), y_ref) <= TOL_Y[cfg.dtype]
+    y_ref, _, _ = oracle.moe_forward(L["x"], L["W_g"], L["w1"], L["w3"], L["w2"], cfg.K)
+    agree = agreeing_tokens(idx, o_idx)
+    assert rel_l2(y_as_f64(y)[agree], y_ref[agree]) <= TOL_Y[cfg.dtype]
 
 
 def test_bounded_wait_runs_out_and_the_context_stays_usable():
@@ -146,8 +147,10 @@ def test_extreme_sizes(case):
         layer.close()
     o_idx, o_gate, o_logits = oracle.router(L["x"], L["W_g"], K)
     compare_routing(idx, w, o_idx, o_gate, o_logits, L["x"], L["W_g"], K)
+    agree = agreeing_tokens(idx, o_idx)
     sample = np.arange(T) if T <= 300 else np.random.default_rng(0).choice(T, 300, replace=False)
-    y_ref = oracle.forward_with_routing(L["x"][sample], idx[sample], w[sample].astype(np.float64),
+    sample = sample[agree[sample]]
+    y_ref = oracle.forward_with_routing(L["x"][sample], o_idx[sample], o_gate[sample],
                                         L["w1"], L["w3"], L["w2"])
     assert rel_l2(y_as_f64(y[sample]), y_ref) <= TOL_Y[dt]
 
