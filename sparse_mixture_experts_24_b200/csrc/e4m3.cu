@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(256) wq_scale_kernel(float* __restrict__ scale
     if (i < count) scales[i] = e4m3_scale(scales[i]);
 }
 
-constexpr int kQrThreads = 256;
+constexpr int kQrThreads = 512;
 
 // One block per row: max |v| over the row (block reduction), then its codes.
 template <bool kBf16>
@@ -139,12 +139,22 @@ __global__ void __launch_bounds__(kQrThreads) qrows_kernel(const uint4* __restri
             if (s < 0 || s >= src_rows) continue;  // block-uniform
         }
         const uint4* row = src + s * vpr;
+        // four vectors per thread in flight at once (zeros past the row end)
         float m = 0.f;
-        for (int v = tid; v < vpr; v += kQrThreads) {
-            float f[kPer];
-            unpack16<kBf16>(__ldg(row + v), f);
+        for (int v0 = tid; v0 < vpr; v0 += 4 * kQrThreads) {
+            uint4 q[4];
 #pragma unroll
-            for (int i = 0; i < kPer; ++i) m = fmaxf(m, fabsf(f[i]));
+            for (int u = 0; u < 4; ++u) {
+                const int v = v0 + u * kQrThreads;
+                q[u] = v < vpr ? __ldg(row + v) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                float f[kPer];
+                unpack16<kBf16>(q[u], f);
+#pragma unroll
+                for (int i = 0; i < kPer; ++i) m = fmaxf(m, fabsf(f[i]));
+            }
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -158,10 +168,22 @@ __global__ void __launch_bounds__(kQrThreads) qrows_kernel(const uint4* __restri
 #pragma unroll
         for (int i = 0; i < kPer; ++i) sc[i] = scale;
         uint8_t* out = codes + r * cols;
-        for (int v = tid; v < vpr; v += kQrThreads) {
-            float f[kPer];
-            unpack16<kBf16>(__ldg(row + v), f);
-            store_codes<kBf16>(out + static_cast<int64_t>(v) * kPer, f, sc);
+        for (int v0 = tid; v0 < vpr; v0 += 4 * kQrThreads) {
+            uint4 q[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int v = v0 + u * kQrThreads;
+                q[u] = v < vpr ? __ldg(row + v) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int v = v0 + u * kQrThreads;
+                if (v < vpr) {
+                    float f[kPer];
+                    unpack16<kBf16>(q[u], f);
+                    store_codes<kBf16>(out + static_cast<int64_t>(v) * kPer, f, sc);
+                }
+            }
         }
         if (tid == 0) scales[r] = scale;
         __syncthreads();  // s_max is reused by the next row
@@ -202,7 +224,7 @@ cudaError_t launch_quantize_rows_e4m3(const void* src, bool bf16, const int32_t*
                                       float* scales, int num_sms, cudaStream_t st) {
     const int vpr = cols / (bf16 ? 8 : 4);
     int64_t blocks = rows;
-    if (blocks > static_cast<int64_t>(num_sms) * 16) blocks = static_cast<int64_t>(num_sms) * 16;
+    if (blocks > static_cast<int64_t>(num_sms) * 8) blocks = static_cast<int64_t>(num_sms) * 8;
     if (blocks < 1) blocks = 1;
     if (bf16)
         launch_k(qrows_kernel<true>, dim3(static_cast<unsigned>(blocks)), dim3(kQrThreads), 0, st,

@@ -56,7 +56,12 @@ constexpr int kRouterMaxSplits = 4;
 // (parts [3][npad][d], npad = n rounded up to 16), computes the logits
 // [T][n] with tcgen05 (tm_x over x [T][d], tm_w over parts [3*npad][d], both
 // with 64 x rows boxes: 128 rows for x, npad rows for the parts), then the
-// top-K and softmax.
+// top-K and softmax: in the router's own epilogue (the d-splits of a token
+// block are one cluster), or, with MOE_ROUTER_TOPK=separate, by
+// router_topk_kernel over logits in the workspace.
+// Kernels launch_router_tc issues for a top-K of K: W_g split + fused router
+// (K <= 8), or W_g split + logits + top-K.
+int router_tc_launches(int K);
 cudaError_t launch_router_tc(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const float* Wg,
                              uint16_t* parts, int64_t T, int d, int n, int K, float* logits,
                              int32_t* topk_idx, float* topk_w, int* status, int num_sms,

@@ -364,7 +364,7 @@ moe_status run_router(moe_handle* h, int64_t T, const void* x, const float* W_g,
         }
         e = moe::launch_router_tc(h->tm_rx, h->tm_parts, W_g, h->wg_parts, T, h->d, h->n, h->K,
                                   h->logits, topk_idx, topk_w, h->status, h->num_sms, st);
-        h->launches += 3;  // W_g split, logits, top-K
+        h->launches += moe::router_tc_launches(h->K);
     } else {
         e = moe::launch_router(x, h->dtype == MOE_BF16, W_g, T, h->d, h->n, h->K, topk_idx, topk_w,
                                h->logits, h->num_sms, st);

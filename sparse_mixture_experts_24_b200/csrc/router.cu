@@ -9,8 +9,9 @@
 // dropped logits are -inf, so the softmax runs over the kept ones only).
 //
 // Kernels:
-//   router_token_kernel  n <= 32, T < 512: one block per token, W_g rows read
-//                        straight from global memory, block reduction.
+//   router_token_kernel  n <= 32, T < 512: one block per token (up to 1,024
+//                        threads), W_g rows read straight from global memory,
+//                        block reduction.
 //   router_small_kernel  n <= 32: W_g staged through shared memory transposed
 //                        to [expert][row]; one warp per group of TPW tokens,
 //                        the lanes split d four rows at a time, every lane
@@ -22,6 +23,7 @@
 //                        warp per token selects the top K with shuffles.
 #include "common.cuh"
 #include "kernels.h"
+#include "topk.cuh"
 
 namespace moe {
 
@@ -183,25 +185,34 @@ __global__ void __launch_bounds__(256) router_small_kernel(const XT* __restrict_
     griddep_launch_dependents();
 }
 
-// n <= 32, few tokens: one 256-thread block per token.  Thread i covers rows
-// 4i .. 4i+3 of every 1024-row slice of d, reading those rows of W_g straight
-// from global memory (4n contiguous floats per thread, contiguous across the
-// block); shuffles then shared memory sum the 256 partial logit vectors.
+// n <= 32, few tokens: one block per token (1,024 threads for n <= 8, 512 for
+// n <= 16, else 256, so that d = 4,096 takes one or two passes and every
+// thread's loads are in flight together).  Thread i covers rows 4i .. 4i+3 of
+// every (4 x threads)-row slice of d, reading those rows of W_g straight from
+// global memory (4n contiguous floats per thread, contiguous across the
+// block); shuffles, then one lane per expert over the warps' partials in warp
+// order, sum the partial logit vectors.
+template <int NE>
+struct TokenRouterCfg {
+    static constexpr int kThreads = NE <= 8 ? 1024 : (NE <= 16 ? 512 : 256);
+};
+
 template <typename XT, int NE>
-__global__ void __launch_bounds__(256) router_token_kernel(const XT* __restrict__ x,
-                                                           const float* __restrict__ Wg, int64_t T,
-                                                           int d, int n, int K,
-                                                           int32_t* __restrict__ topk_idx,
-                                                           float* __restrict__ topk_w) {
+__global__ void __launch_bounds__(TokenRouterCfg<NE>::kThreads)
+    router_token_kernel(const XT* __restrict__ x, const float* __restrict__ Wg, int64_t T, int d, int n, int K,
+                        int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
     griddep_wait();
-    __shared__ float red[8][NE];
+    constexpr int kThreads = TokenRouterCfg<NE>::kThreads;
+    constexpr int kWarps = kThreads / 32;
+    __shared__ float red[kWarps][NE];
+    __shared__ float logit[NE];
     const int64_t t = blockIdx.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float acc[NE];
 #pragma unroll
     for (int e = 0; e < NE; ++e) acc[e] = 0.f;
     const XT* xr = x + t * static_cast<int64_t>(d);
-    for (int j = threadIdx.x * 4; j < d; j += 1024) {
+    for (int j = threadIdx.x * 4; j < d; j += kThreads * 4) {
         float xv[4];
         load_x4<XT>(xr + j, xv);
         const float* w = Wg + static_cast<int64_t>(j) * n;
@@ -233,16 +244,20 @@ __global__ void __launch_bounds__(256) router_token_kernel(const XT* __restrict_
         if (lane == 0) red[warp][e] = a;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        float L[NE];
-#pragma unroll
-        for (int e = 0; e < NE; ++e) {
+    if (warp == 0) {
+        if (lane < NE) {
             float a = 0.f;
 #pragma unroll
-            for (int w8 = 0; w8 < 8; ++w8) a += red[w8][e];
-            L[e] = (a != a) ? -INFINITY : a;  // NaN ranks lowest
+            for (int w8 = 0; w8 < kWarps; ++w8) a += red[w8][lane];
+            logit[lane] = (a != a) ? -INFINITY : a;  // NaN ranks lowest
         }
-        topk_softmax_regs<NE>(L, n, K, topk_idx + t * K, topk_w + t * K);
+        __syncwarp();
+        if (lane == 0) {
+            float L[NE];
+#pragma unroll
+            for (int e = 0; e < NE; ++e) L[e] = logit[e];
+            topk_softmax_regs<NE>(L, n, K, topk_idx + t * K, topk_w + t * K);
+        }
     }
     griddep_launch_dependents();
 }
@@ -318,8 +333,9 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const XT* __restrict
     griddep_launch_dependents();
 }
 
-// One warp per token: lane l holds logits l, l+32, ... (up to 8 per lane),
-// each the in-order sum of `splits` partial logits [splits][T][n].
+// One warp per token: lane l holds logits l, l+32, ... (NS per lane), each
+// the in-order sum of `splits` partial logits [splits][T][n].
+template <int NS>
 __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ logits,
                                                           int splits, int64_t T, int n, int K,
                                                           int32_t* __restrict__ topk_idx,
@@ -328,68 +344,38 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
     const int lane = threadIdx.x & 31;
     const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     if (t >= T) return;
-    float v[8];
+    const float* row = logits + t * n;
+    const int64_t split_stride = T * n;
+    float v[NS];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < NS; ++i) {
         const int e = lane + 32 * i;
         // all partials in flight at once, then summed in split order
         float part[kRouterMaxSplits];
 #pragma unroll
         for (int sp = 0; sp < kRouterMaxSplits; ++sp)
-            part[sp] = (e < n && sp < splits) ? logits[(static_cast<int64_t>(sp) * T + t) * n + e] : 0.f;
+            part[sp] = (e < n && sp < splits) ? __ldg(row + sp * split_stride + e) : 0.f;
         float a = 0.f;
 #pragma unroll
         for (int sp = 0; sp < kRouterMaxSplits; ++sp)
             if (sp < splits) a += part[sp];
-        v[i] = a;
-        if (v[i] != v[i]) v[i] = -INFINITY;  // NaN ranks lowest: keeps the order total
+        v[i] = (a != a) ? -INFINITY : a;  // NaN ranks lowest: keeps the order total
     }
-    uint32_t taken = 0;  // bit i: slot i of this lane already chosen
-    float m = 0.f, s = 0.f;
-    for (int k = 0; k < K; ++k) {
-        // best candidate of this lane (strict '>' scanning upwards: lowest index on ties)
-        int bi = -1;
-        float bv = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int e = lane + 32 * i;
-            if (e < n && !((taken >> i) & 1u) && (bi < 0 || v[i] > bv)) {
-                bi = e;
-                bv = v[i];
-            }
-        }
-        // warp argmax: larger value wins, equal values -> lower index; a lane
-        // without candidates (bi < 0) never wins.
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            const bool take = (oi >= 0) && (bi < 0 || ov > bv || (ov == bv && oi < bi));
-            if (take) {
-                bv = ov;
-                bi = oi;
-            }
-        }
-        if ((bi & 31) == lane && bi >= 0) taken |= 1u << (bi >> 5);
-        if (k == 0) m = bv;
-        const float ex = expf(bv - m);
-        s += ex;
-        if (lane == 0) {
-            topk_idx[t * K + k] = bi;
-            topk_w[t * K + k] = ex;
-        }
-    }
-    if (lane == 0) {
-        const float inv = 1.f / s;
-        for (int k = 0; k < K; ++k) topk_w[t * K + k] *= inv;
-    }
+    warp_topk_softmax<NS>(v, n, K, lane, topk_idx + t * K, topk_w + t * K);
     griddep_launch_dependents();
 }
 
 cudaError_t launch_router_topk(const float* logits, int splits, int64_t T, int n, int K,
                                int32_t* topk_idx, float* topk_w, cudaStream_t st) {
-    launch_k(router_topk_kernel, dim3(dim3(static_cast<unsigned>((T + 7) / 8))), dim3(256), 0, st, logits, splits, T, n,
-                                                                                 K, topk_idx, topk_w);
+    const dim3 grid(static_cast<unsigned>((T + 7) / 8));
+    if (n <= 32)
+        launch_k(router_topk_kernel<1>, grid, dim3(256), 0, st, logits, splits, T, n, K, topk_idx, topk_w);
+    else if (n <= 64)
+        launch_k(router_topk_kernel<2>, grid, dim3(256), 0, st, logits, splits, T, n, K, topk_idx, topk_w);
+    else if (n <= 128)
+        launch_k(router_topk_kernel<4>, grid, dim3(256), 0, st, logits, splits, T, n, K, topk_idx, topk_w);
+    else
+        launch_k(router_topk_kernel<8>, grid, dim3(256), 0, st, logits, splits, T, n, K, topk_idx, topk_w);
     return cudaGetLastError();
 }
 
@@ -398,7 +384,8 @@ static void launch_small(const XT* x, const float* Wg, int64_t T, int d, int n, 
                          float* w, int num_sms, cudaStream_t st) {
     if (T < kTokenKernelMaxT) {
         // few tokens: a whole block per token keeps every SM's loads in flight
-        launch_k(router_token_kernel<XT, NE>, dim3(static_cast<unsigned>(T)), dim3(256), 0, st, x, Wg, T, d, n, K, idx, w);
+        launch_k(router_token_kernel<XT, NE>, dim3(static_cast<unsigned>(T)), dim3(TokenRouterCfg<NE>::kThreads), 0,
+                 st, x, Wg, T, d, n, K, idx, w);
         return;
     }
     // many tokens: share each staged W_g chunk between TPW tokens per warp,
@@ -437,9 +424,7 @@ static cudaError_t launch_router_t(const XT* x, const float* Wg, int64_t T, int 
     }
     dim3 g1(static_cast<unsigned>((T + kRT - 1) / kRT), static_cast<unsigned>((n + kRE - 1) / kRE));
     launch_k(router_logits_kernel<XT>, dim3(g1), dim3(256), 0, st, x, Wg, T, d, n, logits_ws);
-    launch_k(router_topk_kernel, dim3(dim3(static_cast<unsigned>((T + 7) / 8))), dim3(256), 0, st, logits_ws, 1, T, n, K,
-                                                                                 idx, w);
-    return cudaGetLastError();
+    return launch_router_topk(logits_ws, 1, T, n, K, idx, w, st);
 }
 
 cudaError_t launch_router_logits_simt(const void* x, bool x_bf16, const float* Wg, int64_t T, int d,

@@ -17,11 +17,23 @@
 // over gridDim.y CTAs so that small token counts still fill the GPU; warp 0
 // streams x (128 x 64) and the three W_g parts (Npad x 64 each) by TMA through
 // a multi-stage ring; warp 1 issues tcgen05.mma M=128, N=Npad, K=16 three
-// times per K step; warps 2-5 read the 128 x Npad fp32 accumulator from TMEM
-// and store the slice's partial logits [split][T][n], which the top-K kernel
-// sums in split order (deterministic).
+// times per K step; warps 2-5 read the 128 x Npad fp32 accumulator from TMEM.
+//   Logits variant: each CTA stages its partial logits in shared memory and
+//   writes them as whole rows to [split][T][n]; router_topk_kernel (router.cu)
+//   sums the splits in order and selects.
+//   Fused variant: the splits of one token block form a cluster (1 x splits);
+//   every CTA stages its partial in its own shared memory, and after a cluster
+//   barrier the cluster's CTAs share out the 128 tokens: for each of its
+//   tokens a warp sums the splits' partials in split order (read over
+//   distributed shared memory, lane = expert) and selects the top K with the
+//   same warp selection as router_topk_kernel (topk.cuh).  The logits never
+//   reach global memory and no second kernel runs.
+#include <cstdlib>
+#include <cstring>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "topk.cuh"
 
 namespace moe {
 
@@ -68,22 +80,40 @@ __host__ __device__ inline int rt_stages(int npad) {
     return s > kRtMaxStages ? kRtMaxStages : s;
 }
 
+// Partial logits staged per CTA: 128 rows of npad rounded up to 32 (the
+// accumulator is read 32 columns at a time) plus one float (the odd pitch keeps
+// a warp's 32 rows in 32 different banks).
+__host__ __device__ inline int rt_stage_pitch(int npad) { return (npad + 31) / 32 * 32 + 1; }
+__host__ __device__ inline int rt_ring_bytes(int npad) {
+    const int ring = rt_stages(npad) * rt_stage_bytes(npad);
+    const int staged = kRtBM * rt_stage_pitch(npad) * 4;
+    return ring > staged ? ring : staged;
+}
+
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+
 __host__ inline int rt_tmem_cols(int npad) {
     int c = 32;
     while (c < npad) c <<= 1;
     return c;
 }
 
+// kNS: 32-expert slots per lane in the fused selection (npad <= 32 * kNS).
+template <bool kFused, int kNS>
 __global__ void __launch_bounds__(kRtThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                      int64_t T, int d, int n, int npad, int tmem_cols, float* __restrict__ logits,
-                     int* status) {
+                     int K, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, int* status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     const int stage_bytes = rt_stage_bytes(npad);
     const int stages = rt_stages(npad);
-    RtTail* tail = reinterpret_cast<RtTail*>(smem + stages * stage_bytes);
+    RtTail* tail = reinterpret_cast<RtTail*>(smem + rt_ring_bytes(npad));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int kb_total = d / kRtBK;
     const int kb_begin = static_cast<int>(static_cast<int64_t>(kb_total) * blockIdx.y / gridDim.y);
@@ -180,25 +210,72 @@ __global__ void __launch_bounds__(kRtThreads, 1)
             tc_commit(smem_u32(&tail->done));
             mbar_wait(smem_u32(&tail->done), 0, status, kStatusTimeoutDrain);
         }
-    } else {
+    }
+    // ---- epilogue: warps 2-5, thread = accumulator row (TMEM lane) ----
+    // After accum_full every MMA of this CTA has completed, so the ring's
+    // shared memory is free for staging.
+    const int pitch = rt_stage_pitch(npad);
+    float* stage_rows = reinterpret_cast<float*>(smem);
+    const uint32_t rank = kFused ? blockIdx.y : 0;  // cluster (1 x splits): rank = split
+    bool have_acc = false;
+    if (warp >= 2) {
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
-        const int64_t t = static_cast<int64_t>(m0) + r;
-        if (mbar_wait(smem_u32(&tail->accum_full), 0, status, kStatusTimeoutAccum)) {
+        have_acc = mbar_wait(smem_u32(&tail->accum_full), 0, status, kStatusTimeoutAccum);
+        if (have_acc) {
             tc_fence_after();
             for (int c = 0; c < npad; c += 32) {
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + c, v);
                 tmem_wait_ld();
-                if (t < T) {
-                    float* out = logits + t * n;
 #pragma unroll
-                    for (int q = 0; q < 32; ++q)
-                        if (c + q < n) out[c + q] = __uint_as_float(v[q]);
-                }
+                for (int q = 0; q < 32; ++q) stage_rows[r * pitch + c + q] = __uint_as_float(v[q]);
             }
             tc_fence_before();
         }
+        if (!kFused && have_acc) {
+            // whole rows: lane l writes columns l, l+32, ... of each of the warp's 32 rows
+            __syncwarp();
+            for (int rr = 0; rr < 32; ++rr) {
+                const int64_t t = static_cast<int64_t>(m0) + quad * 32 + rr;
+                if (t >= T) break;
+                const float* src = stage_rows + (quad * 32 + rr) * pitch;
+                float* out = logits + t * n;
+                for (int c = lane; c < n; c += 32) out[c] = src[c];
+            }
+        }
+    }
+    if (kFused) {
+        cluster_sync();  // every split's partial is staged
+        const int splits = static_cast<int>(gridDim.y);
+        const int rows_per = (kRtBM + splits - 1) / splits;
+        const int r_end = min(kRtBM, static_cast<int>(rank) * rows_per + rows_per);
+        uint32_t part_base[kRouterMaxSplits];
+#pragma unroll
+        for (int sp = 0; sp < kRouterMaxSplits; ++sp)
+            part_base[sp] = mapa_shared(smem_u32(stage_rows), static_cast<uint32_t>(sp < splits ? sp : 0));
+        for (int r = static_cast<int>(rank) * rows_per + warp; r < r_end; r += kRtThreads / 32) {
+            const int64_t t = static_cast<int64_t>(m0) + r;
+            if (t >= T) break;  // rows ascend: the rest of this warp's rows are past T too
+            float v[kNS];
+#pragma unroll
+            for (int i = 0; i < kNS; ++i) {
+                const int e = lane + 32 * i;
+                float part[kRouterMaxSplits];
+#pragma unroll
+                for (int sp = 0; sp < kRouterMaxSplits; ++sp)
+                    part[sp] = (e < n && sp < splits)
+                                   ? ld_shared_cluster_f32(part_base[sp] + static_cast<uint32_t>(r * pitch + e) * 4u)
+                                   : 0.f;
+                float a = 0.f;
+#pragma unroll
+                for (int sp = 0; sp < kRouterMaxSplits; ++sp)
+                    if (sp < splits) a += part[sp];
+                v[i] = (a != a) ? -INFINITY : a;  // NaN ranks lowest
+            }
+            warp_topk_softmax<kNS>(v, n, K, lane, topk_idx + t * K, topk_w + t * K);
+        }
+        cluster_sync();  // no CTA leaves while another reads its staged partial
     }
     __syncthreads();
     griddep_launch_dependents();
@@ -210,32 +287,88 @@ __global__ void __launch_bounds__(kRtThreads, 1)
 
 int router_tc_smem_bytes(int n) {
     const int npad = (n + 15) / 16 * 16;
-    return rt_stages(npad) * rt_stage_bytes(npad) + static_cast<int>(sizeof(RtTail)) + 1024;
+    return rt_ring_bytes(npad) + static_cast<int>(sizeof(RtTail)) + 1024;
 }
 
-cudaError_t launch_router_logits_tc(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const float* Wg,
-                                    uint16_t* parts, int64_t T, int d, int n, float* logits, int* status,
-                                    int num_sms, cudaStream_t st, int* splits_out) {
-    const int npad = (n + 15) / 16 * 16;
-    const int64_t total = static_cast<int64_t>(npad) * d;
-    int64_t sb = (total + 255) / 256;
-    if (sb > static_cast<int64_t>(num_sms) * 8) sb = static_cast<int64_t>(num_sms) * 8;
-    launch_k(wg_split_kernel, dim3(static_cast<unsigned>(sb)), dim3(256), 0, st, Wg, d, n, npad, parts);
-    const int smem = router_tc_smem_bytes(n);
-    cudaError_t e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    // split d so that the CTAs fill at most one wave (one CTA per SM: the ring
-    // takes most of shared memory), at least 8 K blocks each
+// split d so that the CTAs fill at most one wave (one CTA per SM: the ring
+// takes most of shared memory), at least 8 K blocks each
+static int router_splits(int64_t T, int d, int num_sms) {
     const int64_t mtiles = (T + kRtBM - 1) / kRtBM;
     int splits = static_cast<int>(num_sms / mtiles);
     const int kb_total = d / kRtBK;
     if (splits > kRouterMaxSplits) splits = kRouterMaxSplits;
     if (splits > kb_total / 8) splits = kb_total / 8;
     if (splits < 1) splits = 1;
+    return splits;
+}
+
+static void launch_wg_split(const float* Wg, uint16_t* parts, int d, int n, int num_sms, cudaStream_t st) {
+    const int npad = (n + 15) / 16 * 16;
+    const int64_t total = static_cast<int64_t>(npad) * d;
+    int64_t sb = (total + 255) / 256;
+    if (sb > static_cast<int64_t>(num_sms) * 8) sb = static_cast<int64_t>(num_sms) * 8;
+    launch_k(wg_split_kernel, dim3(static_cast<unsigned>(sb)), dim3(256), 0, st, Wg, d, n, npad, parts);
+}
+
+cudaError_t launch_router_logits_tc(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const float* Wg,
+                                    uint16_t* parts, int64_t T, int d, int n, float* logits, int* status,
+                                    int num_sms, cudaStream_t st, int* splits_out) {
+    const int npad = (n + 15) / 16 * 16;
+    launch_wg_split(Wg, parts, d, n, num_sms, st);
+    const int smem = router_tc_smem_bytes(n);
+    cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int splits = router_splits(T, d, num_sms);
+    const int64_t mtiles = (T + kRtBM - 1) / kRtBM;
     dim3 grid(static_cast<unsigned>(mtiles), static_cast<unsigned>(splits));
-    launch_k(router_tc_kernel, dim3(grid), dim3(kRtThreads), smem, st, tm_x, tm_w, T, d, n, npad, rt_tmem_cols(npad),
-                                                     logits, status);
+    launch_k(router_tc_kernel<false, 1>, dim3(grid), dim3(kRtThreads), smem, st, tm_x, tm_w, T, d, n, npad,
+             rt_tmem_cols(npad), logits, 0, static_cast<int32_t*>(nullptr), static_cast<float*>(nullptr), status);
     *splits_out = splits;
+    return cudaGetLastError();
+}
+
+// The top-K runs in the router's epilogue unless MOE_ROUTER_TOPK=separate asks
+// for the logits-then-top-K kernels.
+static bool fuse_topk(int K) {
+    (void)K;
+    static const bool separate = [] {
+        const char* e = getenv("MOE_ROUTER_TOPK");
+        return e && strcmp(e, "separate") == 0;
+    }();
+    return !separate;
+}
+
+int router_tc_launches(int K) { return fuse_topk(K) ? 2 : 3; }
+
+// The fused router as clusters of the d-splits of each 128-token block.
+template <int kNS>
+static cudaError_t launch_fused(const CUtensorMap& tm_x, const CUtensorMap& tm_w, int64_t T, int d, int n, int npad,
+                                float* logits, int K, int32_t* topk_idx, float* topk_w, int* status, int num_sms,
+                                cudaStream_t st) {
+    const int smem = router_tc_smem_bytes(n);
+    cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<true, kNS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem);
+    if (e != cudaSuccess) return e;
+    const int splits = router_splits(T, d, num_sms);
+    const int64_t mtiles = (T + kRtBM - 1) / kRtBM;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(mtiles), static_cast<unsigned>(splits));
+    cfg.blockDim = dim3(kRtThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = static_cast<unsigned>(splits);
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = (g_chain_started && pdl_enabled()) ? 2 : 1;
+    g_chain_started = true;
+    e = cudaLaunchKernelEx(&cfg, router_tc_kernel<true, kNS>, tm_x, tm_w, T, d, n, npad, rt_tmem_cols(npad), logits,
+                           K, topk_idx, topk_w, status);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -243,11 +376,22 @@ cudaError_t launch_router_tc(const CUtensorMap& tm_x, const CUtensorMap& tm_w, c
                              uint16_t* parts, int64_t T, int d, int n, int K, float* logits,
                              int32_t* topk_idx, float* topk_w, int* status, int num_sms,
                              cudaStream_t st) {
-    int splits = 1;
-    cudaError_t e = launch_router_logits_tc(tm_x, tm_w, Wg, parts, T, d, n, logits, status, num_sms, st,
-                                            &splits);
-    if (e != cudaSuccess) return e;
-    return launch_router_topk(logits, splits, T, n, K, topk_idx, topk_w, st);
+    if (!fuse_topk(K)) {
+        int splits = 1;
+        cudaError_t e = launch_router_logits_tc(tm_x, tm_w, Wg, parts, T, d, n, logits, status, num_sms, st,
+                                                &splits);
+        if (e != cudaSuccess) return e;
+        return launch_router_topk(logits, splits, T, n, K, topk_idx, topk_w, st);
+    }
+    const int npad = (n + 15) / 16 * 16;
+    launch_wg_split(Wg, parts, d, n, num_sms, st);
+    if (npad <= 32)
+        return launch_fused<1>(tm_x, tm_w, T, d, n, npad, logits, K, topk_idx, topk_w, status, num_sms, st);
+    if (npad <= 64)
+        return launch_fused<2>(tm_x, tm_w, T, d, n, npad, logits, K, topk_idx, topk_w, status, num_sms, st);
+    if (npad <= 128)
+        return launch_fused<4>(tm_x, tm_w, T, d, n, npad, logits, K, topk_idx, topk_w, status, num_sms, st);
+    return launch_fused<8>(tm_x, tm_w, T, d, n, npad, logits, K, topk_idx, topk_w, status, num_sms, st);
 }
 
 }  // namespace moe

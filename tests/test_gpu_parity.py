@@ -26,6 +26,11 @@ SMALL = [
     ("bf16_T1", 1, 256, 256, 8, 2, "bf16"),
     ("bf16_many_experts", 500, 128, 128, 64, 2, "bf16"),
     ("bf16_n256", 700, 64, 64, 256, 8, "bf16"),
+    # tensor-core router: top-K fused over a cluster of 2 and 4 d-splits, and
+    # K > 8 (logits to memory, then the top-K kernel)
+    ("bf16_router_split2", 600, 1024, 128, 40, 3, "bf16"),
+    ("bf16_router_split4", 1000, 2048, 128, 8, 2, "bf16"),
+    ("bf16_router_K10", 600, 1024, 64, 32, 10, "bf16"),
     ("f32_tiny", 64, 128, 256, 8, 2, "f32"),
     ("f32_n40_k4", 200, 64, 128, 40, 4, "f32"),
     ("f32_n1", 33, 64, 64, 1, 1, "f32"),
