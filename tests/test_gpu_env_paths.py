@@ -1,0 +1,34 @@
+"""The alternative launch paths that an environment variable selects, each run
+through a slice of the parity suite in a fresh process (the library reads
+these variables once per process):
+
+  MOE_PDL=0                  kernels launched without programmatic dependent
+                             launch (plain stream order);
+  MOE_ROUTER_TOPK=separate   tensor-core router writes logits, then the
+                             standalone top-K kernel selects;
+  MOE_GEMM_PATH=pair         CTA-pair (cta_group::2) expert GEMMs.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+SLICE = "small and (bf16_ragged or bf16_k3_n16 or router_split2 or router_split4 or router_K10 or f32_tiny)"
+
+
+@pytest.mark.parametrize("env", [{"MOE_PDL": "0"}, {"MOE_ROUTER_TOPK": "separate"}, {"MOE_GEMM_PATH": "pair"}],
+                         ids=lambda e: ",".join("%s=%s" % kv for kv in e.items()))
+def test_parity_slice_under_env(env):
+    full_env = dict(os.environ)
+    full_env.update(env)
+    cmd = [sys.executable, "-m", "pytest", os.path.join(ROOT, "tests", "test_gpu_parity.py"), "-m", "gpu", "-q",
+           "-x", "-p", "no:cacheprovider", "-k", SLICE]
+    r = subprocess.run(cmd, cwd=ROOT, env=full_env, capture_output=True, text=True, timeout=600)
+    tail = "\n".join((r.stdout + r.stderr).strip().splitlines()[-15:])
+    assert r.returncode == 0, tail
+    assert " passed" in r.stdout and "6 passed" in r.stdout, tail
