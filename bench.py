@@ -15,8 +15,10 @@ so no flush is needed between steps (tiny_fp32 flushes L2 with a 256 MB write).
 `value` is tokens/s over all ranks (replicas: each rank runs the same
 workload on its own GPU; no collective on the data path), timed with CUDA
 events on the launching stream, max over ranks.  `e2e` is the same metric
-through the C ABI with the step's activations copied from pinned host memory
-and y / topk_idx / topk_w copied back inside the timed region.  `roofline`
+through the C ABI with every step's activations copied from pinned host memory
+and its y / topk_idx / topk_w copied back inside the timed region; the copies
+run on two copy streams with double buffers, overlapping the neighbouring
+steps' layers.  `roofline`
 reports the dominant kernel, timed by the library's per-stage CUDA events over
 a second run of the same K steps (events between the kernels would serialise
 their programmatic dependent launches in the headline run).  `cpu_baseline` times the fp64 oracle on a bounded
@@ -347,11 +349,14 @@ def main():
         del w1, w3, w2
         torch.cuda.empty_cache()
 
-    def forward(xin):
+    def forward(xin, yout=None, iout=None, wout=None):
+        yout = y if yout is None else yout
+        iout = idx if iout is None else iout
+        wout = gw if wout is None else wout
         if e4m3:
-            m.moe_forward_e4m3(layer.h, T, xin, Wg, *q, y, idx, gw, stream)
+            m.moe_forward_e4m3(layer.h, T, xin, Wg, *q, yout, iout, wout, stream)
         else:
-            m.moe_forward(layer.h, T, xin, Wg, w1, w3, w2, y, idx, gw, stream)
+            m.moe_forward(layer.h, T, xin, Wg, w1, w3, w2, yout, iout, wout, stream)
 
     def step():
         if flush is not None:
@@ -397,20 +402,44 @@ def main():
     layer.sync_status(stream)
 
     # ---- end to end: pinned host activations in, y / routing out ----
+    # Every step copies its x from pinned host memory and its y, topk_idx and
+    # topk_w back.  The copies run on their own streams with two buffer sets,
+    # so step i+1's upload and step i's download overlap step i's layer (a
+    # copy engine per direction); events keep each buffer's uses in order.
     xh = x.cpu().pin_memory()
-    yh = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-    ih = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
-    wh = torch.empty(gw.shape, dtype=gw.dtype).pin_memory()
-    xd = torch.empty_like(x)
+    NB = 2
+    xd = [torch.empty_like(x) for _ in range(NB)]
+    yd = [torch.empty_like(y) for _ in range(NB)]
+    idd = [torch.empty_like(idx) for _ in range(NB)]
+    gwd = [torch.empty_like(gw) for _ in range(NB)]
+    yh = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for _ in range(NB)]
+    ih = [torch.empty(idx.shape, dtype=idx.dtype).pin_memory() for _ in range(NB)]
+    wh = [torch.empty(gw.shape, dtype=gw.dtype).pin_memory() for _ in range(NB)]
+    s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_up = [torch.cuda.Event() for _ in range(NB)]
+    ev_layer = [torch.cuda.Event() for _ in range(NB)]
+    ev_down = [torch.cuda.Event() for _ in range(NB)]
+    step_no = [0]
 
     def e2e_step():
+        b = step_no[0] % NB
+        step_no[0] += 1
+        s_up.wait_event(ev_layer[b])          # the layer two steps back has read xd[b]
+        with torch.cuda.stream(s_up):
+            xd[b].copy_(xh, non_blocking=True)
+        ev_up[b].record(s_up)
+        stream.wait_event(ev_up[b])
+        stream.wait_event(ev_down[b])         # yd[b] etc. were read back two steps ago
         if flush is not None:
             flush.fill_(1)
-        xd.copy_(xh, non_blocking=True)
-        forward(xd)
-        yh.copy_(y, non_blocking=True)
-        ih.copy_(idx, non_blocking=True)
-        wh.copy_(gw, non_blocking=True)
+        forward(xd[b], yd[b], idd[b], gwd[b])
+        ev_layer[b].record(stream)
+        s_down.wait_event(ev_layer[b])
+        with torch.cuda.stream(s_down):
+            yh[b].copy_(yd[b], non_blocking=True)
+            ih[b].copy_(idd[b], non_blocking=True)
+            wh[b].copy_(gwd[b], non_blocking=True)
+        ev_down[b].record(s_down)
 
     for _ in range(args.warmup):
         e2e_step()
@@ -419,12 +448,20 @@ def main():
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    s_up.wait_event(e0)
+    s_down.wait_event(e0)
     for _ in range(args.steps):
         e2e_step()
+    for b in range(NB):
+        stream.wait_event(ev_down[b])
     e1.record(stream)
     torch.cuda.synchronize(dev)
     ems = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, dev)
     e2e_value = tokens_per_s(T, world, ems)
+    # the copied-back outputs of the last step equal the device-timed run's
+    # (same input, deterministic kernels)
+    last = (step_no[0] - 1) % NB
+    e2e_same = bool(torch.equal(yh[last], y.cpu()) and torch.equal(ih[last], idx.cpu()))
     h2d = x.numel() * x.element_size()
     d2h = y.numel() * y.element_size() + idx.numel() * 4 + gw.numel() * 4
 
@@ -483,7 +520,7 @@ def main():
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
+                    "d2h_bytes_per_step": d2h, "outputs_match_device_run": e2e_same},
             "gpu_launches": launches,
             "clocks": clocks,
         }
