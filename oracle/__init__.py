@@ -73,6 +73,12 @@ def _bind(L):
                                       vp, vp]
     L.oracle_expert_choice.argtypes = [i64, i32, i32, i32, i64, vp, i32, vp, i32, vp, vp, vp, i32,
                                        vp, vp, vp]
+    L.oracle_e2m1_decode.argtypes = [ctypes.c_int]
+    L.oracle_e2m1_decode.restype = ctypes.c_double
+    L.oracle_e2m1_encode.argtypes = [ctypes.c_double]
+    L.oracle_e2m1_encode.restype = ctypes.c_int
+    L.oracle_quantize_weights_fp4.argtypes = [i32, i32, i32, vp, i32, vp, vp, vp]
+    L.oracle_dequantize_fp4.argtypes = [i32, i32, i32, vp, vp, vp, vp]
     L.oracle_silu.argtypes = [ctypes.c_double]
     L.oracle_silu.restype = ctypes.c_double
     L.oracle_num_threads.restype = ctypes.c_int
@@ -80,7 +86,7 @@ def _bind(L):
     for f in ("oracle_router", "oracle_expert", "oracle_forward_with_routing",
               "oracle_moe_forward", "oracle_dispatch", "oracle_router_stats",
               "oracle_dispatch_capacity", "oracle_expert_choice", "oracle_quantize_weights_e4m3",
-              "oracle_forward_e4m3"):
+              "oracle_forward_e4m3", "oracle_quantize_weights_fp4", "oracle_dequantize_fp4"):
         getattr(L, f).restype = ctypes.c_int
     return L
 
@@ -248,6 +254,35 @@ class Oracle:
                "quantize_weights_e4m3")
         return codes, scales
 
+    def e2m1_decode(self, code: int) -> float:
+        return float(self.L.oracle_e2m1_decode(int(code)))
+
+    def e2m1_encode(self, v: float) -> int:
+        return int(self.L.oracle_e2m1_encode(float(v)))
+
+    def quantize_weights_fp4(self, w):
+        """w [n][rows][cols] -> codes uint8 [n][rows][cols/2] (column 2j in the low
+        nibble of byte j), block scales uint8 E4M3 codes [n][rows/16][cols],
+        tensor scales fp32 [n]."""
+        w = _c(w)
+        n, rows, cols = w.shape
+        codes = np.empty((n, rows, cols // 2), np.uint8)
+        bscale = np.empty((n, rows // 16, cols), np.uint8)
+        tscale = np.empty(n, np.float32)
+        _check(self.L.oracle_quantize_weights_fp4(n, rows, cols, _p(w), _dt(w), _p(codes), _p(bscale),
+                                                  _p(tscale)), "quantize_weights_fp4")
+        return codes, bscale, tscale
+
+    def dequantize_fp4(self, codes, bscale, tscale):
+        codes = np.ascontiguousarray(codes, dtype=np.uint8)
+        bscale = np.ascontiguousarray(bscale, dtype=np.uint8)
+        tscale = np.ascontiguousarray(tscale, dtype=np.float32)
+        n, rows, half = codes.shape
+        w = np.empty((n, rows, 2 * half), np.float64)
+        _check(self.L.oracle_dequantize_fp4(n, rows, 2 * half, _p(codes), _p(bscale), _p(tscale), _p(w)),
+               "dequantize_fp4")
+        return w
+
     def forward_e4m3(self, x, idx, gate, q1, s1, q3, s3, q2, s2):
         x = _c(x)
         idx = np.ascontiguousarray(idx, dtype=np.int32)
@@ -331,3 +366,19 @@ def quantize_weights_e4m3(w):
 
 def forward_e4m3(x, idx, gate, q1, s1, q3, s3, q2, s2):
     return default().forward_e4m3(x, idx, gate, q1, s1, q3, s3, q2, s2)
+
+
+def e2m1_decode(code: int) -> float:
+    return default().e2m1_decode(code)
+
+
+def e2m1_encode(v: float) -> int:
+    return default().e2m1_encode(v)
+
+
+def quantize_weights_fp4(w):
+    return default().quantize_weights_fp4(w)
+
+
+def dequantize_fp4(codes, bscale, tscale):
+    return default().dequantize_fp4(codes, bscale, tscale)

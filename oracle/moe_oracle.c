@@ -669,3 +669,118 @@ int oracle_forward_e4m3(int64_t T, int d, int F, int n, int K, const void *x, in
     }
     return bad ? -1 : 0;
 }
+
+/*
+ * 4-bit expert weights.  "Mixture of Experts: Why Mixtral Only Wakes Up Two
+ * Specialists", Part 4 ("Why total and active both matter"), sizes the
+ * weights at 16 bits and at 4 bits and names no format; this oracle fixes one:
+ * E2M1 values (1 sign, 2 exponent bits with bias 1, 1 mantissa bit: 0, 0.5,
+ * 1, 1.5, 2, 3, 4, 6; no infinities or NaN) with an E4M3 scale per block of
+ * 16 consecutive reduction rows of one output column and one fp32 scale per
+ * expert matrix:
+ *   st = amax(matrix) / (6 * 448)                 (1 for an all-zero matrix)
+ *   sb = E4M3( fp32(fp32(amax(block) / 6) / st) )  (round to nearest even)
+ *   code = E2M1( fp32(v / fp32(sb * st)) )        (round to nearest even,
+ *          saturating at +-6; 0 when sb is 0)
+ *   w ~= E2M1(code) * sb * st
+ * E2M1(code) * sb has at most 6 significant bits, so it is exact in bf16.
+ */
+double oracle_e2m1_decode(int code)
+{
+    int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    double v = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -v : v;
+}
+
+int oracle_e2m1_encode(double v)
+{
+    static const double grid[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    if (isnan(v))
+        return 0x7; /* not produced by finite inputs; maps to +6 */
+    int s = signbit(v) ? 1 : 0;
+    double a = fabs(v), q;
+    /* the grid is uniform inside [0, 2), [2, 4) and [4, 6]: count steps of
+     * 0.5, 1 and 2 and round half to even (an even step count = an even
+     * mantissa bit) */
+    if (a >= 6.0)
+        q = 6.0;
+    else if (a < 2.0)
+        q = 0.5 * round_half_even(a / 0.5);
+    else if (a < 4.0)
+        q = round_half_even(a);
+    else
+        q = 2.0 * round_half_even(a / 2.0);
+    int mag = 0;
+    for (int c = 0; c < 8; ++c)
+        if (grid[c] == q)
+            mag = c;
+    return (s << 3) | mag;
+}
+
+/*
+ * w [n][rows][cols] (bf16 bits or fp32), rows % 16 == 0, cols even ->
+ *   codes [n][rows][cols / 2]: column 2j in the low nibble of byte j, 2j + 1
+ *   in the high nibble; bscale [n][rows / 16][cols]: E4M3 codes; tscale [n].
+ */
+int oracle_quantize_weights_fp4(int n, int rows, int cols, const void *w, int w_dt, uint8_t *codes,
+                                uint8_t *bscale, float *tscale)
+{
+    if (n <= 0 || rows <= 0 || cols <= 0 || rows % 16 != 0 || cols % 2 != 0 || !w || !codes ||
+        !bscale || !tscale || !dt_ok(w_dt))
+        return -1;
+    for (int e = 0; e < n; ++e) {
+        float amax = 0.0f;
+        for (size_t i = 0; i < (size_t)rows * cols; ++i) {
+            float v = (float)elem(w, w_dt, (size_t)e * rows * cols + i);
+            if (fabsf(v) > amax)
+                amax = fabsf(v);
+        }
+        float st = amax > 0.0f ? amax / 2688.0f : 1.0f;
+        tscale[e] = st;
+        uint8_t *ce = codes + (size_t)e * rows * (cols / 2);
+        memset(ce, 0, (size_t)rows * (cols / 2));
+        /* a thread owns the column pair (2j, 2j + 1) and so whole code bytes */
+#pragma omp parallel for schedule(static)
+        for (int j = 0; j < cols / 2; ++j)
+            for (int h = 0; h < 2; ++h) {
+                const int c = 2 * j + h;
+                for (int b = 0; b < rows / 16; ++b) {
+                    float amax_b = 0.0f;
+                    for (int r = 16 * b; r < 16 * b + 16; ++r) {
+                        float v = (float)elem(w, w_dt, ((size_t)e * rows + r) * cols + c);
+                        if (fabsf(v) > amax_b)
+                            amax_b = fabsf(v);
+                    }
+                    float qb = (amax_b / 6.0f) / st;
+                    int sb_code = oracle_e4m3_encode((double)qb);
+                    bscale[((size_t)e * (rows / 16) + b) * cols + c] = (uint8_t)sb_code;
+                    float sb = (float)oracle_e4m3_decode(sb_code);
+                    float denom = sb * st;
+                    for (int r = 16 * b; r < 16 * b + 16; ++r) {
+                        float v = (float)elem(w, w_dt, ((size_t)e * rows + r) * cols + c);
+                        int code = (sb == 0.0f) ? 0 : oracle_e2m1_encode((double)(v / denom));
+                        ce[(size_t)r * (cols / 2) + j] |= (uint8_t)(code << (4 * h));
+                    }
+                }
+            }
+    }
+    return 0;
+}
+
+/* codes, bscale, tscale as produced above -> w [n][rows][cols] (fp64). */
+int oracle_dequantize_fp4(int n, int rows, int cols, const uint8_t *codes, const uint8_t *bscale,
+                          const float *tscale, double *w)
+{
+    if (n <= 0 || rows <= 0 || cols <= 0 || rows % 16 != 0 || cols % 2 != 0 || !codes || !bscale ||
+        !tscale || !w)
+        return -1;
+    for (int e = 0; e < n; ++e)
+        for (int r = 0; r < rows; ++r)
+            for (int c = 0; c < cols; ++c) {
+                int byte = codes[((size_t)e * rows + r) * (cols / 2) + c / 2];
+                int code = (byte >> (4 * (c & 1))) & 0xF;
+                double sb = oracle_e4m3_decode(bscale[((size_t)e * (rows / 16) + r / 16) * cols + c]);
+                w[((size_t)e * rows + r) * cols + c] = oracle_e2m1_decode(code) * sb * (double)tscale[e];
+            }
+    return 0;
+}

@@ -512,6 +512,114 @@ def check_e4m3_forward_error_band(O):
     assert 1e-3 < err < 0.08, err
 
 
+# --------------------------------------------------------------------------
+# 4-bit (E2M1, block-scaled) experts
+# --------------------------------------------------------------------------
+
+E2M1_VALUES = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def check_e2m1_codec(O):
+    """E2M1: sign, 2 exponent bits (bias 1), 1 mantissa bit -- magnitudes
+    0, 0.5, 1, 1.5, 2, 3, 4, 6; encode rounds to nearest with ties to the even
+    mantissa, saturates at 6 and keeps the sign of zero."""
+    for c in range(16):
+        want = E2M1_VALUES[c & 7] * (-1.0 if c & 8 else 1.0)
+        got = O.e2m1_decode(c)
+        assert got == want and math.copysign(1.0, got) == (-1.0 if c & 8 else 1.0), c
+        assert O.e2m1_encode(got) == c, c
+    ties = {0.25: 0, 0.75: 2, 1.25: 2, 1.75: 4, 2.5: 4, 3.5: 6, 5.0: 6}
+    for v, c in ties.items():
+        assert O.e2m1_encode(v) == c and O.e2m1_encode(-v) == c | 8, v
+    assert O.e2m1_encode(0.26) == 1 and O.e2m1_encode(0.74) == 1 and O.e2m1_encode(5.01) == 7
+    assert O.e2m1_encode(6.5) == 7 and O.e2m1_encode(-1e30) == 15 and O.e2m1_encode(1e-30) == 0
+    rng = np.random.default_rng(51)
+    for v in rng.uniform(-8, 8, 500):
+        q = O.e2m1_decode(O.e2m1_encode(v))
+        nearest = min(E2M1_VALUES, key=lambda g: abs(abs(v) - g)) if abs(v) <= 6 else 6.0
+        assert abs(q) == nearest or abs(abs(q) - abs(v)) == abs(nearest - abs(v))
+
+
+def _fp4_exact_matrix(rng):
+    """One expert matrix [32][6] whose blocks are E2M1 values x a power-of-two
+    block scale (one block at 448) x the tensor scale 2^-8, each block
+    reaching +-6 x its scale: quantisation must recover it exactly."""
+    rows, cols = 32, 6
+    st = 2.0 ** -8
+    w = np.zeros((rows, cols))
+    q_ref = np.zeros((rows, cols), int)
+    sb_ref = np.zeros((rows // 16, cols))
+    for b in range(rows // 16):
+        for c in range(cols):
+            sb = 448.0 if (b, c) == (0, 0) else 2.0 ** int(rng.integers(-3, 9))
+            q = rng.integers(0, 16, 16)
+            q[int(rng.integers(0, 16))] = 7 if rng.random() < 0.5 else 15     # the block maximum, +-6
+            for r in range(16):
+                w[16 * b + r, c] = E2M1_VALUES[q[r] & 7] * (-1 if q[r] & 8 else 1) * sb * st
+            q_ref[16 * b:16 * b + 16, c] = q
+            sb_ref[b, c] = sb
+    return w, q_ref, sb_ref, st
+
+
+def check_fp4_exact_case(O):
+    """Exactly representable weights come back bit-exact: tensor scale =
+    amax / 2688, block scales, codes, nibble order (column 2j low), and the
+    dequantised matrix; negative zeros keep their sign code."""
+    rng = np.random.default_rng(52)
+    w, q_ref, sb_ref, st = _fp4_exact_matrix(rng)
+    codes, bscale, tscale = O.quantize_weights_fp4(w[None].astype(np.float32))
+    assert tscale[0] == np.float32(st)
+    assert np.array_equal(np.vectorize(O.e4m3_decode)(bscale[0]), sb_ref)
+    lo, hi = codes[0] & 0xF, codes[0] >> 4
+    got = np.empty_like(q_ref)
+    got[:, 0::2], got[:, 1::2] = lo, hi
+    assert np.array_equal(got, q_ref)
+    assert np.array_equal(O.dequantize_fp4(codes, bscale, tscale)[0], w)
+
+
+def check_fp4_error_band(O):
+    """Gaussian weights: every element within its block's E2M1 rounding bound
+    (a quarter of the largest grid step, 2 x sb x st, plus the E4M3 rounding
+    of sb), the whole matrix within the 4-bit error band, zero blocks exact."""
+    rng = np.random.default_rng(53)
+    w = rng.standard_normal((3, 64, 40)).astype(np.float32)
+    w[1, 16:32, 5] = 0.0
+    codes, bscale, tscale = O.quantize_weights_fp4(w)
+    d = O.dequantize_fp4(codes, bscale, tscale)
+    for e in range(3):
+        assert tscale[e] == np.float32(np.abs(w[e]).max() / np.float32(2688.0))
+        sb = np.vectorize(O.e4m3_decode)(bscale[e]).repeat(16, axis=0)
+        bound = 1.0 * sb * tscale[e] + 1e-30
+        assert np.all(np.abs(d[e] - w[e]) <= bound)
+    assert np.all(d[1, 16:32, 5] == 0.0)
+    err = np.linalg.norm(d - w) / np.linalg.norm(w)
+    assert 0.03 < err < 0.15, err
+
+
+def check_fp4_layer_uses_dequantised_weights(O):
+    """The 4-bit layer is the layer of the dequantised weights: with exactly
+    representable weights it equals the exact layer."""
+    rng = np.random.default_rng(54)
+    T, d, F, n, K = 9, 32, 32, 2, 2
+    ws = []
+    for _ in range(3):
+        m = np.stack([_fp4_exact_matrix(rng)[0] for _ in range(n)])      # [n][32][6] each
+        ws.append(m)
+    # fit the exact matrices to the layer shapes: w1, w3 [n][d][F], w2 [n][F][d]
+    w1 = np.concatenate([ws[0]] * 6, axis=2)[:, :, :F][:, :d]
+    w3 = np.concatenate([ws[1]] * 6, axis=2)[:, :, :F][:, :d]
+    w2 = np.concatenate([ws[2]] * 6, axis=2)[:, :, :d][:, :F]
+    x = rng.standard_normal((T, d))
+    idx = np.array([[0, 1]] * T, np.int32)
+    gate = np.tile([[0.6, 0.4]], (T, 1))
+    deq = [O.dequantize_fp4(*O.quantize_weights_fp4(w.astype(np.float32))) for w in (w1, w3, w2)]
+    for a, b in zip(deq, (w1, w3, w2)):
+        assert np.array_equal(a, b)
+    y = O.forward_with_routing(x, idx, gate, *deq)
+    y0 = O.forward_with_routing(x, idx, gate, w1, w3, w2)
+    assert np.array_equal(y, y0)
+
+
 ALL_CHECKS = [
     check_worked_example, check_two_way_softmax_closed_form, check_logits_are_x_times_Wg,
     check_topk_brute_force, check_ties_go_to_lower_index, check_gate_invariants, check_silu,
@@ -524,4 +632,5 @@ ALL_CHECKS = [
     check_expert_choice_selection_brute_force,
     check_e4m3_codec, check_e4m3_weight_quantization, check_e4m3_forward_exact_case,
     check_e4m3_forward_error_band,
+    check_e2m1_codec, check_fp4_exact_case, check_fp4_error_band, check_fp4_layer_uses_dequantised_weights,
 ]

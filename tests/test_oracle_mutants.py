@@ -35,6 +35,11 @@ MUTANTS = {
     "e4m3_ties_up": [("return (fmod(f, 2.0) == 0.0) ? f : f + 1.0;", "return f + 1.0;")],
     "e4m3_no_act_scale": [("double av = a[f] * sx * s1[(size_t)e * F + f];", "double av = a[f] * s1[(size_t)e * F + f];")],
     "e4m3_no_down_scale": [("yt[i] += g * o * sh * s2[(size_t)e * d + i];", "yt[i] += g * o * s2[(size_t)e * d + i];")],
+    "e2m1_ties_up": [("q = 0.5 * round_half_even(a / 0.5);", "q = 0.5 * floor(a / 0.5 + 0.5);")],
+    "e2m1_bias_0": [("ldexp(1.0 + 0.5 * m, e - 1)", "ldexp(1.0 + 0.5 * m, e)")],
+    "fp4_tensor_scale_448": [("amax / 2688.0f", "amax / 448.0f")],
+    "fp4_nibbles_swapped": [("(uint8_t)(code << (4 * h))", "(uint8_t)(code << (4 * (1 - h)))")],
+    "fp4_block_scale_no_div6": [("float qb = (amax_b / 6.0f) / st;", "float qb = amax_b / st;")],
     "e4m3_scale_over_256": [("amax / 448.0f", "amax / 256.0f")],
     "e4m3_bias_8": [("v = ldexp(1.0 + m / 8.0, e - 7);", "v = ldexp(1.0 + m / 8.0, e - 8);")],
     "capacity_keeps_one_more": [("if (row - offsets[e] < capacity) {", "if (row - offsets[e] <= capacity) {")],
