@@ -2,7 +2,7 @@
 """Benchmark of the sparse MoE layer forward (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
-                    [--experts bf16|e4m3]
+                    [--experts bf16|e4m3|fp4]
 
 A step is one moe_forward over one batch: router, top-K, softmax, dispatch,
 gather, GEMM1 (w1/w3 + SwiGLU), GEMM2 (w2), combine.  The default workload is
@@ -26,7 +26,9 @@ sample of the same workload on this host's cores.
 
 --experts e4m3 times moe_forward_e4m3 instead: the same layer with FP8 (E4M3)
 expert weights (per-column scales, quantised once before the timed region)
-and per-row E4M3 activations (bf16 handle and workloads only).
+and per-row E4M3 activations; --experts fp4 times moe_forward_fp4: 4-bit
+(E2M1) expert weights with E4M3 scales per 16 rows and bf16 activations (bf16
+handle and workloads only).
 
 --impl reference runs the oracle (the reference arm of this build) on the
 host, rank 0 only.
@@ -64,7 +66,7 @@ def load_peaks():
 def workload_desc(cfg, experts="bf16"):
     return "%s: T=%d, d=%d, ffn=%d, n=%d, K=%d, %s%s%s" % (
         cfg.name, cfg.T, cfg.d, cfg.ffn, cfg.n, cfg.K, cfg.dtype, ", skewed router" if cfg.skew else "",
-        ", E4M3 experts" if experts == "e4m3" else "")
+        {"e4m3": ", E4M3 experts", "fp4": ", 4-bit (E2M1) experts"}.get(experts, ""))
 
 
 # --------------------------------------------------------------------------
@@ -83,7 +85,13 @@ def algorithmic(cfg, counts, experts="bf16"):
     T, d, F, n, K = cfg.T, cfg.d, cfg.ffn, cfg.n, cfg.K
     R = T * K
     used = int((counts > 0).sum())
-    if experts == "e4m3":
+    if experts == "fp4":
+        # codes 0.5 B + block scale 1/16 B per weight; gather, H and O in bf16
+        w13 = used * 2 * (d * F // 2 + d * F // 16 + 4)
+        w2 = used * (F * d // 2 + F * d // 16 + 4)
+        gemm1_bytes = w13 + R * d * es + R * F * es
+        gemm2_bytes = w2 + R * F * es + R * d * es
+    elif experts == "e4m3":
         w13 = used * 2 * (d * F + F * 4)
         w2 = used * (F * d + d * 4)
         gemm1_bytes = w13 + R * (d + 4) + R * F * 2 + (R * F * 2 + R * (F + 4))
@@ -226,6 +234,12 @@ def oracle_tokens_per_s(cfg, L, budget_s=12.0, experts="bf16"):
         def layer(xs):
             i, g, _ = oracle.router(xs, L["W_g"], cfg.K)
             oracle.forward_e4m3(xs, i, g, *q)
+    elif experts == "fp4":
+        q4 = [oracle.quantize_weights_fp4(L[w]) for w in ("w1", "w3", "w2")]
+
+        def layer(xs):
+            i, g, _ = oracle.router(xs, L["W_g"], cfg.K)
+            oracle.forward_fp4(xs, i, g, *q4)
     else:
         def layer(xs):
             oracle.moe_forward(xs, L["W_g"], L["w1"], L["w3"], L["w2"], cfg.K)
@@ -298,13 +312,13 @@ def main():
     ap.add_argument("--config", default="decode", choices=sorted(mi.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--experts", default="bf16", choices=["bf16", "e4m3"])
+    ap.add_argument("--experts", default="bf16", choices=["bf16", "e4m3", "fp4"])
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     cfg = mi.CONFIGS[args.config]
-    if args.experts == "e4m3" and cfg.dtype != "bf16":
-        ap.error("--experts e4m3 needs a bf16 workload")
+    if args.experts != "bf16" and cfg.dtype != "bf16":
+        ap.error("--experts %s needs a bf16 workload" % args.experts)
     if args.impl == "reference":
         return run_reference(args, cfg)
 
@@ -342,9 +356,11 @@ def main():
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if cfg.name == "tiny_fp32" else None
     e4m3 = args.experts == "e4m3"
-    if e4m3:
+    fp4 = args.experts == "fp4"
+    if e4m3 or fp4:
         # quantised once, outside the timed region; the bf16 copies are freed
-        q = [t for w in (w1, w3, w2) for t in m.quantize_weights_e4m3(w)]
+        quant = m.quantize_weights_e4m3 if e4m3 else m.quantize_weights_fp4
+        q = [t for w in (w1, w3, w2) for t in quant(w)]
         torch.cuda.synchronize(dev)
         del w1, w3, w2
         torch.cuda.empty_cache()
@@ -355,6 +371,8 @@ def main():
         wout = gw if wout is None else wout
         if e4m3:
             m.moe_forward_e4m3(layer.h, T, xin, Wg, *q, yout, iout, wout, stream)
+        elif fp4:
+            m.moe_forward_fp4(layer.h, T, xin, Wg, *q, yout, iout, wout, stream)
         else:
             m.moe_forward(layer.h, T, xin, Wg, w1, w3, w2, yout, iout, wout, stream)
 
@@ -492,7 +510,7 @@ def main():
         roof["peak_source"] = peak_src
         roof["algorithmic_per_launch"] = work[dom]["bytes"] if roof["bound"] == "hbm" else work[dom]["flops"]
         roof["launch_ms"] = dom_ms
-        roof["traffic"] = recorded_traffic(dom, cfg.name + ("_e4m3" if e4m3 else ""))
+        roof["traffic"] = recorded_traffic(dom, cfg.name + {"e4m3": "_e4m3", "fp4": "_fp4"}.get(args.experts, ""))
 
     # ---- CPU baseline (rank 0, N = 1 only) ----
     cpu = None
@@ -500,14 +518,16 @@ def main():
         v, s, reps, cores, el = oracle_tokens_per_s(cfg, L, experts=args.experts)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": "first %d of %d tokens x %d repetitions, full layer in fp64%s (%.1f s)"
-                         % (s, cfg.T, reps, ", E4M3 experts" if e4m3 else "", el)}
+                         % (s, cfg.T, reps, {"e4m3": ", E4M3 experts", "fp4": ", 4-bit experts"}.get(args.experts, ""),
+                            el)}
 
     if rank == 0:
         layer_ms = ms
         line = {
             "metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if e4m3 else cfg.dtype, "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3" if e4m3 else ("e2m1 weights, bf16" if fp4 else cfg.dtype), "data": "synthetic",
             "config": {"workload": workload_desc(cfg, args.experts), "global_batch_tokens": T * world,
                        "parallelism": "replicas%d" % world if world > 1 else "single",
                        "l2": "256 MB flush per step" if flush is not None else

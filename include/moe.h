@@ -247,6 +247,50 @@ MOE_API moe_status moe_forward_e4m3(moe_handle *h, int64_t T, const void *x, con
                                     int32_t *topk_idx, float *topk_w, moe_stream_t stream);
 
 /*
+ * 4-bit expert weights (Part 4 of "Mixture of Experts: Why Mixtral Only Wakes
+ * Up Two Specialists" sizes the weights at 4 bits; the format is this
+ * library's): E2M1 values (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6) with an E4M3
+ * scale per 16 consecutive reduction rows of one output column and an fp32
+ * scale per expert matrix:
+ *   st[e]     = max|w[e]| / (6 * 448)                (1 for an all-zero matrix)
+ *   sb[e][b][c] = E4M3( fp32(max|w[e][16b..16b+15][c]| / 6) / st[e] )
+ *   code      = E2M1( fp32(w / fp32(sb * st)) ), round to nearest even,
+ *               saturating at +-6 (0 where sb is 0)
+ *   w ~= E2M1(code) * sb * st
+ *
+ * moe_quantize_weights_fp4: w [n][rows][cols] (MOE_BF16 or MOE_F32, device)
+ * -> codes [n][rows][cols/2] uint8 (column 2j in the low nibble of byte j,
+ * 2j+1 in the high nibble), block_scales [n][rows/16][cols] uint8 (E4M3
+ * codes), matrix_scales [n] fp32, all device memory.  For the layer: w1, w3
+ * [n][d][ffn] and w2 [n][ffn][d].  Needs no handle; enqueued on `stream`.
+ *   Errors: MOE_ERR_INVALID_ARG (n outside [1, 65535], rows not a positive
+ *   multiple of 16, cols not a positive multiple of 32, null / misaligned
+ *   pointer), MOE_ERR_UNSUPPORTED (not an sm_100 device), MOE_ERR_CUDA.
+ */
+MOE_API moe_status moe_quantize_weights_fp4(int n, int rows, int cols, const void *w, moe_dtype dtype,
+                                            uint8_t *codes, uint8_t *block_scales, float *matrix_scales,
+                                            moe_stream_t stream);
+
+/*
+ * The layer of moe_forward with 4-bit experts (MOE_BF16 handles only): the same
+ * router, dispatch (and capacity) and gather; each expert GEMM runs on bf16
+ * activations and the weights E2M1(code) * sb, which are exact in bf16, and
+ * multiplies the fp32 accumulators by the matrix scale st:
+ *   h = bf16( silu(st1 * x . W1) (*) (st3 * x . W3) ),  o = bf16( st2 * h . W2 )
+ * so the result is the bf16 layer of the dequantised weights.  Codes and
+ * scales as moe_quantize_weights_fp4 writes them; x, W_g, y, topk_idx, topk_w
+ * as for moe_forward.
+ *   Errors: as moe_forward; MOE_ERR_UNSUPPORTED for an fp32 handle.
+ */
+MOE_API moe_status moe_forward_fp4(moe_handle *h, int64_t T, const void *x, const float *W_g,
+                                   const uint8_t *w1_codes, const uint8_t *w1_block_scales,
+                                   const float *w1_matrix_scales, const uint8_t *w3_codes,
+                                   const uint8_t *w3_block_scales, const float *w3_matrix_scales,
+                                   const uint8_t *w2_codes, const uint8_t *w2_block_scales,
+                                   const float *w2_matrix_scales, void *y, int32_t *topk_idx, float *topk_w,
+                                   moe_stream_t stream);
+
+/*
  * Debug view of the workspace written by the last forward call: name is "H"
  * (expert hidden layer, [rows][ffn], handle dtype) or "O" (per-row expert
  * outputs, [rows][d], handle dtype for bf16 handles, fp32 for fp32 handles);

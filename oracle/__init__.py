@@ -79,6 +79,7 @@ def _bind(L):
     L.oracle_e2m1_encode.restype = ctypes.c_int
     L.oracle_quantize_weights_fp4.argtypes = [i32, i32, i32, vp, i32, vp, vp, vp]
     L.oracle_dequantize_fp4.argtypes = [i32, i32, i32, vp, vp, vp, vp]
+    L.oracle_forward_fp4.argtypes = [i64, i32, i32, i32, i32, vp, i32, vp, vp] + [vp] * 9 + [vp]
     L.oracle_silu.argtypes = [ctypes.c_double]
     L.oracle_silu.restype = ctypes.c_double
     L.oracle_num_threads.restype = ctypes.c_int
@@ -86,7 +87,8 @@ def _bind(L):
     for f in ("oracle_router", "oracle_expert", "oracle_forward_with_routing",
               "oracle_moe_forward", "oracle_dispatch", "oracle_router_stats",
               "oracle_dispatch_capacity", "oracle_expert_choice", "oracle_quantize_weights_e4m3",
-              "oracle_forward_e4m3", "oracle_quantize_weights_fp4", "oracle_dequantize_fp4"):
+              "oracle_forward_e4m3", "oracle_quantize_weights_fp4", "oracle_dequantize_fp4",
+              "oracle_forward_fp4"):
         getattr(L, f).restype = ctypes.c_int
     return L
 
@@ -283,6 +285,25 @@ class Oracle:
                "dequantize_fp4")
         return w
 
+    def forward_fp4(self, x, idx, gate, w1, w3, w2):
+        """The layer of the dequantised 4-bit weights; w1, w3, w2 are (codes,
+        block scales, matrix scales) triples of quantize_weights_fp4."""
+        x = _c(x)
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+        gate = np.ascontiguousarray(gate, dtype=np.float64)
+        T, d = x.shape
+        n, d2, half = w1[0].shape
+        F = 2 * half
+        K = idx.shape[1]
+        parts = []
+        for c, b, t in (w1, w3, w2):
+            parts += [np.ascontiguousarray(c, dtype=np.uint8), np.ascontiguousarray(b, dtype=np.uint8),
+                      np.ascontiguousarray(t, dtype=np.float32)]
+        y = np.empty((T, d), np.float64)
+        _check(self.L.oracle_forward_fp4(T, d, F, n, K, _p(x), _dt(x), _p(idx), _p(gate), *[_p(a) for a in parts],
+                                         _p(y)), "forward_fp4")
+        return y
+
     def forward_e4m3(self, x, idx, gate, q1, s1, q3, s3, q2, s2):
         x = _c(x)
         idx = np.ascontiguousarray(idx, dtype=np.int32)
@@ -382,3 +403,7 @@ def quantize_weights_fp4(w):
 
 def dequantize_fp4(codes, bscale, tscale):
     return default().dequantize_fp4(codes, bscale, tscale)
+
+
+def forward_fp4(x, idx, gate, w1, w3, w2):
+    return default().forward_fp4(x, idx, gate, w1, w3, w2)

@@ -784,3 +784,84 @@ int oracle_dequantize_fp4(int n, int rows, int cols, const uint8_t *codes, const
             }
     return 0;
 }
+
+/* Decoded E2M1 and E4M3 codes (filled before any parallel region reads them). */
+static double fp4_lut[16], e4m3_lut[256];
+
+static void fp4_luts(void)
+{
+    for (int c = 0; c < 16; ++c)
+        fp4_lut[c] = oracle_e2m1_decode(c);
+    for (int c = 0; c < 256; ++c)
+        e4m3_lut[c] = oracle_e4m3_decode(c);
+}
+
+/* One dequantised 4-bit weight: matrix e of [n][rows][cols]. */
+static double fp4_weight(const uint8_t *codes, const uint8_t *bscale, const float *tscale, int rows, int cols,
+                         int e, int r, int c)
+{
+    int byte = codes[((size_t)e * rows + r) * (cols / 2) + c / 2];
+    int code = (byte >> (4 * (c & 1))) & 0xF;
+    double sb = e4m3_lut[bscale[((size_t)e * (rows / 16) + r / 16) * cols + c]];
+    return fp4_lut[code] * sb * (double)tscale[e];
+}
+
+/*
+ * The layer of the dequantised 4-bit weights (the same loops as
+ * oracle_forward_with_routing, each weight dequantised where it is read):
+ * c1/b1/t1, c3/b3/t3 for w1, w3 [n][d][F]; c2/b2/t2 for w2 [n][F][d].
+ */
+int oracle_forward_fp4(int64_t T, int d, int F, int n, int K, const void *x, int x_dt, const int32_t *idx,
+                       const double *gate, const uint8_t *c1, const uint8_t *b1, const float *t1,
+                       const uint8_t *c3, const uint8_t *b3, const float *t3, const uint8_t *c2,
+                       const uint8_t *b2, const float *t2, double *y)
+{
+    if (T <= 0 || d <= 0 || F <= 0 || n <= 0 || K <= 0 || d % 16 != 0 || F % 16 != 0 || !x || !idx || !gate ||
+        !c1 || !b1 || !t1 || !c3 || !b3 || !t3 || !c2 || !b2 || !t2 || !y || !dt_ok(x_dt))
+        return -1;
+    for (int64_t i = 0; i < T * K; ++i)
+        if (idx[i] < 0 || idx[i] >= n)
+            return -1;
+    fp4_luts();
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *a = (double *)malloc(sizeof(double) * (size_t)F);
+        double *b = (double *)malloc(sizeof(double) * (size_t)F);
+        if (!a || !b) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t t = 0; t < T; ++t) {
+                double *yt = y + t * d;
+                for (int i = 0; i < d; ++i)
+                    yt[i] = 0.0;
+                for (int k = 0; k < K; ++k) {
+                    int e = idx[t * K + k];
+                    for (int f = 0; f < F; ++f)
+                        a[f] = b[f] = 0.0;
+                    for (int j = 0; j < d; ++j) {
+                        double xj = elem(x, x_dt, (size_t)t * d + j);
+                        for (int f = 0; f < F; ++f) {
+                            a[f] += xj * fp4_weight(c1, b1, t1, d, F, e, j, f);
+                            b[f] += xj * fp4_weight(c3, b3, t3, d, F, e, j, f);
+                        }
+                    }
+                    for (int f = 0; f < F; ++f)
+                        a[f] = oracle_silu(a[f]) * b[f];
+                    double g = gate[t * K + k];
+                    for (int i = 0; i < d; ++i) {
+                        double o = 0.0;
+                        for (int f = 0; f < F; ++f)
+                            o += a[f] * fp4_weight(c2, b2, t2, F, d, e, f, i);
+                        yt[i] += g * o;
+                    }
+                }
+            }
+        }
+        free(a);
+        free(b);
+    }
+    return bad ? -1 : 0;
+}

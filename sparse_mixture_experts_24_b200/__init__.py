@@ -64,13 +64,16 @@ lib.moe_dispatch_noalloc.argtypes = [_i64, _int, _int, _vp, _vp, _vp, _vp, _vp, 
 lib.moe_trace_end.argtypes = [_vp, ctypes.POINTER(ctypes.c_double), _int, ctypes.POINTER(_int)]
 lib.moe_quantize_weights_e4m3.argtypes = [_int, _int, _int, _vp, _int, _vp, _vp, _vp]
 lib.moe_forward_e4m3.argtypes = [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.moe_quantize_weights_fp4.argtypes = [_int, _int, _int, _vp, _int, _vp, _vp, _vp, _vp]
+lib.moe_forward_fp4.argtypes = [_vp, _i64, _vp, _vp] + [_vp] * 9 + [_vp, _vp, _vp, _vp]
 lib.moe_last_error.restype = ctypes.c_char_p
 lib.moe_version.restype = ctypes.c_char_p
 for _f in ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
            "moe_forward_with_routing", "moe_workspace_view", "moe_sync_status", "moe_destroy",
            "moe_trace_begin", "moe_trace_end", "moe_dispatch_noalloc", "moe_set_capacity_factor",
            "moe_router_stats", "moe_launch_count", "moe_selftest_timeout",
-           "moe_forward_expert_choice", "moe_quantize_weights_e4m3", "moe_forward_e4m3"):
+           "moe_forward_expert_choice", "moe_quantize_weights_e4m3", "moe_forward_e4m3",
+           "moe_quantize_weights_fp4", "moe_forward_fp4"):
     getattr(lib, _f).restype = _int
 
 EXPORTED = ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
@@ -78,7 +81,7 @@ EXPORTED = ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispat
             "moe_last_error", "moe_version", "moe_trace_begin", "moe_trace_end",
             "moe_dispatch_noalloc", "moe_set_capacity_factor", "moe_router_stats",
             "moe_launch_count", "moe_selftest_timeout", "moe_forward_expert_choice",
-            "moe_quantize_weights_e4m3", "moe_forward_e4m3")
+            "moe_quantize_weights_e4m3", "moe_forward_e4m3", "moe_quantize_weights_fp4", "moe_forward_fp4")
 
 TRACE_STAGES = ("router", "dispatch", "gather", "gemm1", "gemm2", "combine")
 
@@ -233,6 +236,31 @@ def quantize_weights_e4m3(w, stream=None):
     return codes, scales
 
 
+def moe_quantize_weights_fp4(n, rows, cols, w, dtype, codes, block_scales, matrix_scales, stream=None) -> None:
+    _check(lib.moe_quantize_weights_fp4(n, rows, cols, _ptr(w), dtype, _ptr(codes), _ptr(block_scales),
+                                        _ptr(matrix_scales), _stream(stream)), "moe_quantize_weights_fp4")
+
+
+def moe_forward_fp4(h, T, x, W_g, w1_c, w1_b, w1_t, w3_c, w3_b, w3_t, w2_c, w2_b, w2_t, y, topk_idx, topk_w,
+                    stream=None) -> None:
+    _check(lib.moe_forward_fp4(h, T, _ptr(x), _ptr(W_g), _ptr(w1_c), _ptr(w1_b), _ptr(w1_t), _ptr(w3_c),
+                               _ptr(w3_b), _ptr(w3_t), _ptr(w2_c), _ptr(w2_b), _ptr(w2_t), _ptr(y), _ptr(topk_idx),
+                               _ptr(topk_w), _stream(stream)), "moe_forward_fp4")
+
+
+def quantize_weights_fp4(w, stream=None):
+    """w [n][rows][cols] (torch bf16 or fp32, CUDA) -> (codes uint8 [n][rows][cols/2],
+    block scales uint8 [n][rows/16][cols] (E4M3 codes), matrix scales fp32 [n])."""
+    import torch
+    n, rows, cols = w.shape
+    codes = torch.empty((n, rows, cols // 2), dtype=torch.uint8, device=w.device)
+    bscale = torch.empty((n, rows // 16, cols), dtype=torch.uint8, device=w.device)
+    tscale = torch.empty(n, dtype=torch.float32, device=w.device)
+    moe_quantize_weights_fp4(n, rows, cols, w, MOE_BF16 if w.dtype == torch.bfloat16 else MOE_F32, codes, bscale,
+                             tscale, stream)
+    return codes, bscale, tscale
+
+
 def moe_destroy(h) -> None:
     _check(lib.moe_destroy(h), "moe_destroy")
 
@@ -312,6 +340,20 @@ class MoELayer:
         if topk_w is None:
             topk_w = torch.empty((T, self.K), dtype=torch.float32, device=x.device)
         moe_forward_e4m3(self.h, T, x, W_g, w1_q, w1_s, w3_q, w3_s, w2_q, w2_s, y, topk_idx, topk_w, stream)
+        return y, topk_idx, topk_w
+
+    def forward_fp4(self, x, W_g, w1, w3, w2, y=None, topk_idx=None, topk_w=None, stream=None):
+        """The layer with 4-bit experts; w1, w3, w2 are (codes, block scales,
+        matrix scales) triples from quantize_weights_fp4."""
+        import torch
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty_like(x)
+        if topk_idx is None:
+            topk_idx = torch.empty((T, self.K), dtype=torch.int32, device=x.device)
+        if topk_w is None:
+            topk_w = torch.empty((T, self.K), dtype=torch.float32, device=x.device)
+        moe_forward_fp4(self.h, T, x, W_g, *w1, *w3, *w2, y, topk_idx, topk_w, stream)
         return y, topk_idx, topk_w
 
     def set_capacity_factor(self, factor: float) -> None:

@@ -167,6 +167,35 @@ cudaError_t launch_tc_gemm1_e4m3(const CUtensorMap& tm_x8, const CUtensorMap& tm
 cudaError_t launch_tc_gemm2_e4m3(const CUtensorMap& tm_h8, const CUtensorMap& tm_q2, const TcGemmArgs& a,
                                  int num_sms, cudaStream_t st);
 
+// 4-bit weights (fp4.cu, gemm_fp4.cu): codes [n][rows][cols/2] (column 2j in
+// the low nibble of byte j), E4M3 block scales [n][rows/16][cols], fp32
+// matrix scales [n].  Four launches (a memset, max, codes, matrix scale).
+cudaError_t launch_quantize_weights_fp4(const void* w, bool bf16, int n, int rows, int cols, uint8_t* codes,
+                                        uint8_t* bscale, float* tscale, int num_sms, cudaStream_t st);
+
+struct Fp4GemmArgs {
+    const int32_t* offsets;
+    const int32_t* mblk_base;
+    int n;
+    int64_t R;
+    int k_blocks;      // reduction length / 64
+    int n_tiles;
+    int out_cols;
+    void* out;         // bf16 [R][out_cols]
+    int* status;
+    const float* tscale0;  // [n] matrix scales: w1 (GEMM1) or w2 (GEMM2)
+    const float* tscale1;  // [n] w3 (GEMM1)
+};
+
+// tm_xp / tm_h: bf16 rows (64 x 128 boxes, 128-byte swizzle); tm_c*: codes
+// [n][K][N/2] uint8 (64 x 64 boxes, no swizzle); tm_s*: block scales
+// [n][K/16][N] uint8 (128 x 4 boxes, no swizzle).
+cudaError_t launch_fp4_gemm1(const CUtensorMap& tm_xp, const CUtensorMap& tm_c1, const CUtensorMap& tm_s1,
+                             const CUtensorMap& tm_c3, const CUtensorMap& tm_s3, const Fp4GemmArgs& a, int num_sms,
+                             cudaStream_t st);
+cudaError_t launch_fp4_gemm2(const CUtensorMap& tm_h, const CUtensorMap& tm_c2, const CUtensorMap& tm_s2,
+                             const Fp4GemmArgs& a, int num_sms, cudaStream_t st);
+
 // E4M3 quantisation (e4m3.cu).  Codes are those of v / scale with the quotient
 // rounded to fp32, then to E4M3 by round-to-nearest-even with saturation to
 // +-448; scale = max |v| / 448 over the group (1 for an all-zero group).

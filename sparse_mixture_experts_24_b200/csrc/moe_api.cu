@@ -123,6 +123,33 @@ bool encode_codes(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-bit weight codes [n][rows][cols/2] read in 64-byte x 64-row boxes, and
+// their block scales [n][rows/16][cols] in 128 x 4 boxes; no swizzle (the
+// kernel's converter warps read them).
+bool encode_fp4_codes(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t n) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[3] = {cols / 2, rows, n};
+    cuuint64_t strides[2] = {cols / 2, cols / 2 * rows};
+    cuuint32_t box[3] = {64, 64, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_fp4_scales(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t n) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[3] = {cols, rows / 16, n};
+    cuuint64_t strides[2] = {cols, cols * (rows / 16)};
+    cuuint32_t box[3] = {128, 4, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 struct moe_handle {
@@ -170,6 +197,9 @@ struct moe_handle {
     const void* c_q1 = nullptr;
     const void* c_q3 = nullptr;
     const void* c_q2 = nullptr;
+    // 4-bit experts: maps over the caller's codes and block scales
+    CUtensorMap tm_f4[6];  // codes w1, scales w1, codes w3, scales w3, codes w2, scales w2
+    const void* c_f4[6] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
     // tracing: kTraceEvents events per traced call
     std::vector<cudaEvent_t> trace_ev;
     int trace_max = 0;
@@ -554,6 +584,69 @@ moe_status run_experts_e4m3(moe_handle* h, int64_t T, const void* x, const int32
     return MOE_OK;
 }
 
+// The 4-bit expert path: dispatch and gather as for bf16, then both GEMMs on
+// the 4-bit weights (converted to bf16 tiles in shared memory), combine.
+moe_status run_experts_fp4(moe_handle* h, int64_t T, const void* x, const float* topk_w, const uint8_t* const* cw,
+                           const uint8_t* const* bs, const float* const* ts, void* y, const int32_t* topk_idx,
+                           cudaStream_t st) {
+    const int64_t R = T * h->K;
+    cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n, moe::kTcBM, h->db, st, capacity_for(h, T));
+    if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
+    h->launches += moe::dispatch_kernel_count(R);
+    trace_mark(h, 1, st);
+    e = moe::launch_gather(x, h->db.row_token, R, T, static_cast<int64_t>(h->d) * 2, h->xp, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+    h->launches += 1;
+    trace_mark(h, 2, st);
+    // matrices: 0 = w1 [n][d][F], 1 = w3 [n][d][F], 2 = w2 [n][F][d]
+    for (int m = 0; m < 3; ++m) {
+        const uint64_t rows = m < 2 ? h->d : h->F, cols = m < 2 ? h->F : h->d;
+        if (cw[m] != h->c_f4[2 * m]) {
+            if (!encode_fp4_codes(&h->tm_f4[2 * m], cw[m], cols, rows, h->n))
+                return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for 4-bit codes");
+            h->c_f4[2 * m] = cw[m];
+        }
+        if (bs[m] != h->c_f4[2 * m + 1]) {
+            if (!encode_fp4_scales(&h->tm_f4[2 * m + 1], bs[m], cols, rows, h->n))
+                return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for 4-bit block scales");
+            h->c_f4[2 * m + 1] = bs[m];
+        }
+    }
+    moe::Fp4GemmArgs a1{};
+    a1.offsets = h->db.offsets;
+    a1.mblk_base = h->db.mblk_base;
+    a1.n = h->n;
+    a1.R = R;
+    a1.k_blocks = h->d / 64;
+    a1.n_tiles = (h->F + 127) / 128;
+    a1.out_cols = h->F;
+    a1.out = h->h;
+    a1.status = h->status;
+    a1.tscale0 = ts[0];
+    a1.tscale1 = ts[1];
+    e = moe::launch_fp4_gemm1(h->tm_xp, h->tm_f4[0], h->tm_f4[1], h->tm_f4[2], h->tm_f4[3], a1, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
+    h->launches += 1;
+    trace_mark(h, 3, st);
+    moe::Fp4GemmArgs a2 = a1;
+    a2.k_blocks = h->F / 64;
+    a2.n_tiles = (h->d + 255) / 256;
+    a2.out_cols = h->d;
+    a2.out = h->o;
+    a2.tscale0 = ts[2];
+    a2.tscale1 = nullptr;
+    e = moe::launch_fp4_gemm2(h->tm_h, h->tm_f4[4], h->tm_f4[5], a2, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
+    h->launches += 1;
+    trace_mark(h, 4, st);
+    e = moe::launch_combine(h->o, true, h->db.token_row, topk_w, T, h->K, h->d, y, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+    h->launches += 1;
+    trace_mark(h, 5, st);
+    trace_finish_call(h);
+    return MOE_OK;
+}
+
 // Router logits into h->logits (tensor cores for bf16, CUDA cores for fp32);
 // returns the number of split partials.
 moe_status run_logits(moe_handle* h, int64_t T, const void* x, const float* W_g, cudaStream_t st,
@@ -820,6 +913,71 @@ moe_status moe_forward_e4m3(moe_handle* h, int64_t T, const void* x, const float
     if (s != MOE_OK) return s;
     trace_mark(h, 0, st);
     s = run_experts_e4m3(h, T, x, topk_idx, topk_w, w1_q, w1_s, w3_q, w3_s, w2_q, w2_s, y, st);
+    return s == MOE_OK ? ok() : s;
+}
+
+moe_status moe_quantize_weights_fp4(int n, int rows, int cols, const void* w, moe_dtype dtype, uint8_t* codes,
+                                    uint8_t* block_scales, float* matrix_scales, moe_stream_t stream) {
+    if (n < 1 || n > 65535) return fail(MOE_ERR_INVALID_ARG, "n = %d outside [1, 65535]", n);
+    if (rows < 16 || rows % 16 != 0)
+        return fail(MOE_ERR_INVALID_ARG, "rows = %d is not a positive multiple of 16", rows);
+    if (cols < 32 || cols % 32 != 0)
+        return fail(MOE_ERR_INVALID_ARG, "cols = %d is not a positive multiple of 32", cols);
+    if (dtype != MOE_F32 && dtype != MOE_BF16)
+        return fail(MOE_ERR_INVALID_ARG, "dtype = %d is not MOE_F32 or MOE_BF16", static_cast<int>(dtype));
+    if (static_cast<int64_t>(rows) / 16 * (cols / 2) > 2147483647LL / 256)
+        return fail(MOE_ERR_INVALID_ARG, "rows * cols too large");
+    REQUIRE_PTR(w);
+    REQUIRE_PTR(codes);
+    REQUIRE_PTR(block_scales);
+    REQUIRE_PTR(matrix_scales);
+    int dev = 0, sms = 0, major = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (major != 10) return fail(MOE_ERR_UNSUPPORTED, "device %d is not sm_100", dev);
+    e = moe::launch_quantize_weights_fp4(w, dtype == MOE_BF16, n, rows, cols, codes, block_scales, matrix_scales,
+                                         sms, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "4-bit weight quantisation launch");
+    return ok();
+}
+
+moe_status moe_forward_fp4(moe_handle* h, int64_t T, const void* x, const float* W_g, const uint8_t* w1_codes,
+                           const uint8_t* w1_bscale, const float* w1_tscale, const uint8_t* w3_codes,
+                           const uint8_t* w3_bscale, const float* w3_tscale, const uint8_t* w2_codes,
+                           const uint8_t* w2_bscale, const float* w2_tscale, void* y, int32_t* topk_idx,
+                           float* topk_w, moe_stream_t stream) {
+    moe_status s = check_common(h, T);
+    if (s != MOE_OK) return s;
+    if (h->dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "the 4-bit expert path needs a MOE_BF16 handle");
+    if (T == 0) return ok();
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(W_g);
+    REQUIRE_PTR(w1_codes);
+    REQUIRE_PTR(w1_bscale);
+    REQUIRE_PTR(w1_tscale);
+    REQUIRE_PTR(w3_codes);
+    REQUIRE_PTR(w3_bscale);
+    REQUIRE_PTR(w3_tscale);
+    REQUIRE_PTR(w2_codes);
+    REQUIRE_PTR(w2_bscale);
+    REQUIRE_PTR(w2_tscale);
+    REQUIRE_PTR(y);
+    REQUIRE_PTR(topk_idx);
+    REQUIRE_PTR(topk_w);
+    s = prepare(h, T);
+    if (s != MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    moe::chain_begin();
+    trace_mark(h, -1, st);
+    s = run_router(h, T, x, W_g, topk_idx, topk_w, st);
+    if (s != MOE_OK) return s;
+    trace_mark(h, 0, st);
+    const uint8_t* cw[3] = {w1_codes, w3_codes, w2_codes};
+    const uint8_t* bs[3] = {w1_bscale, w3_bscale, w2_bscale};
+    const float* ts[3] = {w1_tscale, w3_tscale, w2_tscale};
+    s = run_experts_fp4(h, T, x, topk_w, cw, bs, ts, y, topk_idx, st);
     return s == MOE_OK ? ok() : s;
 }
 

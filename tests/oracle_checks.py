@@ -620,6 +620,20 @@ def check_fp4_layer_uses_dequantised_weights(O):
     assert np.array_equal(y, y0)
 
 
+def check_fp4_forward_is_layer_of_dequantised(O):
+    """The 4-bit layer (weights dequantised where read) equals the layer of the
+    dequantised matrices, up to summation order."""
+    T, d, F, n = 7, 32, 48, 3
+    x, Wg, w1, w3, w2 = rand_layer(55, T, d, F, n)
+    idx, gate, _ = O.router(x, Wg, 2)
+    q = [O.quantize_weights_fp4(w.astype(np.float32)) for w in (w1, w3, w2)]
+    deq = [O.dequantize_fp4(*t) for t in q]
+    y4 = O.forward_fp4(x, idx, gate, *q)
+    y = O.forward_with_routing(x, idx, gate, *deq)
+    assert rel_l2(y4, y) < 1e-12
+    assert rel_l2(y, O.forward_with_routing(x, idx, gate, w1, w3, w2)) > 1e-3
+
+
 ALL_CHECKS = [
     check_worked_example, check_two_way_softmax_closed_form, check_logits_are_x_times_Wg,
     check_topk_brute_force, check_ties_go_to_lower_index, check_gate_invariants, check_silu,
@@ -633,4 +647,5 @@ ALL_CHECKS = [
     check_e4m3_codec, check_e4m3_weight_quantization, check_e4m3_forward_exact_case,
     check_e4m3_forward_error_band,
     check_e2m1_codec, check_fp4_exact_case, check_fp4_error_band, check_fp4_layer_uses_dequantised_weights,
+    check_fp4_forward_is_layer_of_dequantised,
 ]
