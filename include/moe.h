@@ -38,6 +38,12 @@
  *     or order the streams.
  *   - On any error nothing is launched, the outputs are untouched, and
  *     moe_last_error() describes the failure.
+ *   - After moe_reserve(T_max) (and, for moe_forward_e4m3, one earlier call of
+ *     it, which sizes its part of the workspace), a forward call with T <=
+ *     T_max only enqueues kernels: it allocates nothing and does not
+ *     synchronise with the host, so it can be captured into a CUDA graph and
+ *     replayed (the kernels keep their programmatic dependent launches).  The
+ *     captured call reads x and the weights from the addresses it was given.
  */
 #ifndef MOE_B200_MOE_H
 #define MOE_B200_MOE_H

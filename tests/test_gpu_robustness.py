@@ -165,3 +165,50 @@ def test_zero_tokens_launch_nothing():
         assert m.moe_launch_count(layer.h) == c0
     finally:
         layer.close()
+
+
+NONFINITE_CASES = [
+    # name, T, d, ffn, n, K, dtype: the token router, the tensor-core router (T >= 512
+    # and n > 32), and the fp32 routers
+    ("nf_token_router", 64, 256, 128, 8, 2, "bf16"),
+    ("nf_tc_router", 600, 256, 128, 8, 2, "bf16"),
+    ("nf_tc_router_n64", 300, 128, 128, 64, 4, "bf16"),
+    ("nf_f32", 100, 128, 128, 8, 2, "f32"),
+    ("nf_f32_n40", 100, 64, 64, 40, 3, "f32"),
+]
+
+
+@pytest.mark.parametrize("case", NONFINITE_CASES, ids=[c[0] for c in NONFINITE_CASES])
+def test_nonfinite_tokens_stay_contained(case):
+    """Rows of x holding NaN, +-inf or huge values: their results are
+    unspecified, but every routing index stays a valid, distinct expert, the
+    call reports no error, and every other token's routing and output equal
+    the oracle's (tokens never mix)."""
+    import sparse_mixture_experts_24_b200 as m
+    require_cuda()
+    name, T, d, F, n, K, dt = case
+    cfg = mi.custom_config(name, T=T, d=d, ffn=F, n=n, K=K, dtype=dt)
+    L = mi.make_layer(cfg, seed=9)
+    xf = mi.as_f32(L["x"]).copy()
+    bad = np.array([3, 7, 11, T - 1])
+    xf[3, :] = np.nan
+    xf[7, 0] = np.inf
+    xf[11, 5] = -np.inf
+    xf[T - 1, :] = 1e30
+    x = mi.f32_to_bf16_bits(xf) if dt == "bf16" else xf
+    layer = m.MoELayer(n, K, d, F, dt)
+    try:
+        y, idx, w = layer.forward(dev(x), *[dev(L[k]) for k in ("W_g", "w1", "w3", "w2")])
+        layer.sync_status()
+        y, idx, w = host(y), host(idx), host(w)
+    finally:
+        layer.close()
+    assert ((idx >= 0) & (idx < n)).all()
+    assert all(len(set(row)) == K for row in idx.tolist())
+    good = np.setdiff1d(np.arange(T), bad)
+    xg = x[good]
+    o_idx, o_gate, o_logits = oracle.router(xg, L["W_g"], K)
+    compare_routing(idx[good], w[good], o_idx, o_gate, o_logits, xg, L["W_g"], K)
+    y_ref, _, _ = oracle.moe_forward(xg, L["W_g"], L["w1"], L["w3"], L["w2"], K)
+    agree = agreeing_tokens(idx[good], o_idx)
+    assert rel_l2(y_as_f64(y[good])[agree], y_ref[agree]) <= TOL_Y[dt]
