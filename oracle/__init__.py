@@ -80,6 +80,8 @@ def _bind(L):
     L.oracle_quantize_weights_fp4.argtypes = [i32, i32, i32, vp, i32, vp, vp, vp]
     L.oracle_dequantize_fp4.argtypes = [i32, i32, i32, vp, vp, vp, vp]
     L.oracle_forward_fp4.argtypes = [i64, i32, i32, i32, i32, vp, i32, vp, vp] + [vp] * 9 + [vp]
+    L.oracle_quantize_rows_fp4.argtypes = [i64, i32, vp, i32, vp, vp, vp]
+    L.oracle_forward_w4a4.argtypes = [i64, i32, i32, i32, i32, vp, i32, vp, vp] + [vp] * 9 + [vp]
     L.oracle_silu.argtypes = [ctypes.c_double]
     L.oracle_silu.restype = ctypes.c_double
     L.oracle_num_threads.restype = ctypes.c_int
@@ -88,7 +90,7 @@ def _bind(L):
               "oracle_moe_forward", "oracle_dispatch", "oracle_router_stats",
               "oracle_dispatch_capacity", "oracle_expert_choice", "oracle_quantize_weights_e4m3",
               "oracle_forward_e4m3", "oracle_quantize_weights_fp4", "oracle_dequantize_fp4",
-              "oracle_forward_fp4"):
+              "oracle_forward_fp4", "oracle_quantize_rows_fp4", "oracle_forward_w4a4"):
         getattr(L, f).restype = ctypes.c_int
     return L
 
@@ -304,6 +306,37 @@ class Oracle:
                                          _p(y)), "forward_fp4")
         return y
 
+    def quantize_rows_fp4(self, x):
+        """x [T][d] -> codes uint8 [T][d/2] (element 2j in the low nibble of
+        byte j), block scales uint8 E4M3 codes [T][d/16], row scales fp32 [T]."""
+        x = _c(x)
+        T, d = x.shape
+        codes = np.empty((T, d // 2), np.uint8)
+        bscale = np.empty((T, d // 16), np.uint8)
+        rscale = np.empty(T, np.float32)
+        _check(self.L.oracle_quantize_rows_fp4(T, d, _p(x), _dt(x), _p(codes), _p(bscale), _p(rscale)),
+               "quantize_rows_fp4")
+        return codes, bscale, rscale
+
+    def forward_w4a4(self, x, idx, gate, w1, w3, w2):
+        """The layer with 4-bit weights (triples of quantize_weights_fp4) and
+        4-bit activations (x rows and hidden rows quantised per row)."""
+        x = _c(x)
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+        gate = np.ascontiguousarray(gate, dtype=np.float64)
+        T, d = x.shape
+        n, d2, half = w1[0].shape
+        F = 2 * half
+        K = idx.shape[1]
+        parts = []
+        for c, b, t in (w1, w3, w2):
+            parts += [np.ascontiguousarray(c, dtype=np.uint8), np.ascontiguousarray(b, dtype=np.uint8),
+                      np.ascontiguousarray(t, dtype=np.float32)]
+        y = np.empty((T, d), np.float64)
+        _check(self.L.oracle_forward_w4a4(T, d, F, n, K, _p(x), _dt(x), _p(idx), _p(gate), *[_p(a) for a in parts],
+                                          _p(y)), "forward_w4a4")
+        return y
+
     def forward_e4m3(self, x, idx, gate, q1, s1, q3, s3, q2, s2):
         x = _c(x)
         idx = np.ascontiguousarray(idx, dtype=np.int32)
@@ -407,3 +440,11 @@ def dequantize_fp4(codes, bscale, tscale):
 
 def forward_fp4(x, idx, gate, w1, w3, w2):
     return default().forward_fp4(x, idx, gate, w1, w3, w2)
+
+
+def quantize_rows_fp4(x):
+    return default().quantize_rows_fp4(x)
+
+
+def forward_w4a4(x, idx, gate, w1, w3, w2):
+    return default().forward_w4a4(x, idx, gate, w1, w3, w2)

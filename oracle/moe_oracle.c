@@ -865,3 +865,131 @@ int oracle_forward_fp4(int64_t T, int d, int F, int n, int K, const void *x, int
     }
     return bad ? -1 : 0;
 }
+
+/*
+ * 4-bit activations, the other operand of the 4-bit tensor-core path: each row
+ * of x [T][d] is quantised like one 4-bit weight matrix whose blocks run
+ * along the row -- rs = max|row| / (6 * 448) (1 for a zero row), an E4M3
+ * scale per 16 consecutive elements, E2M1 codes; codes [T][d/2] (element 2j
+ * in the low nibble of byte j), bscale [T][d/16], rscale [T].
+ */
+int oracle_quantize_rows_fp4(int64_t T, int d, const void *x, int x_dt, uint8_t *codes, uint8_t *bscale,
+                             float *rscale)
+{
+    if (T <= 0 || d <= 0 || d % 16 != 0 || !x || !codes || !bscale || !rscale || !dt_ok(x_dt))
+        return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        float amax = 0.0f;
+        for (int j = 0; j < d; ++j) {
+            float v = (float)elem(x, x_dt, (size_t)t * d + j);
+            if (fabsf(v) > amax)
+                amax = fabsf(v);
+        }
+        float rs = amax > 0.0f ? amax / 2688.0f : 1.0f;
+        rscale[t] = rs;
+        uint8_t *ct = codes + (size_t)t * (d / 2);
+        memset(ct, 0, (size_t)d / 2);
+        for (int b = 0; b < d / 16; ++b) {
+            float amax_b = 0.0f;
+            for (int j = 16 * b; j < 16 * b + 16; ++j) {
+                float v = (float)elem(x, x_dt, (size_t)t * d + j);
+                if (fabsf(v) > amax_b)
+                    amax_b = fabsf(v);
+            }
+            int sb_code = oracle_e4m3_encode((double)((amax_b / 6.0f) / rs));
+            bscale[(size_t)t * (d / 16) + b] = (uint8_t)sb_code;
+            float denom = (float)oracle_e4m3_decode(sb_code) * rs;
+            for (int j = 16 * b; j < 16 * b + 16; ++j) {
+                float v = (float)elem(x, x_dt, (size_t)t * d + j);
+                int code = (denom == 0.0f) ? 0 : oracle_e2m1_encode((double)(v / denom));
+                ct[j / 2] |= (uint8_t)(code << (4 * (j & 1)));
+            }
+        }
+    }
+    return 0;
+}
+
+static double fp4_act(const uint8_t *codes, const uint8_t *bscale, float rs, int j)
+{
+    int code = (codes[j / 2] >> (4 * (j & 1))) & 0xF;
+    return fp4_lut[code] * e4m3_lut[bscale[j / 16]] * (double)rs;
+}
+
+/*
+ * The layer with 4-bit weights AND 4-bit activations: per token, x is
+ * quantised per row as above; a, b = the dot products of the dequantised
+ * x row with the dequantised w1, w3 columns; h = bf16(silu(a) * b); h is
+ * quantised per row the same way; o = the dequantised h row times the
+ * dequantised w2; y = sum_k gate_k * o_k.  Weights as oracle_quantize_weights_fp4
+ * writes them (c*, b*, t*).
+ */
+int oracle_forward_w4a4(int64_t T, int d, int F, int n, int K, const void *x, int x_dt, const int32_t *idx,
+                        const double *gate, const uint8_t *c1, const uint8_t *b1, const float *t1,
+                        const uint8_t *c3, const uint8_t *b3, const float *t3, const uint8_t *c2,
+                        const uint8_t *b2, const float *t2, double *y)
+{
+    if (T <= 0 || d <= 0 || F <= 0 || n <= 0 || K <= 0 || d % 16 != 0 || F % 16 != 0 || !x || !idx || !gate ||
+        !c1 || !b1 || !t1 || !c3 || !b3 || !t3 || !c2 || !b2 || !t2 || !y || !dt_ok(x_dt))
+        return -1;
+    for (int64_t i = 0; i < T * K; ++i)
+        if (idx[i] < 0 || idx[i] >= n)
+            return -1;
+    fp4_luts();
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *a = (double *)malloc(sizeof(double) * (size_t)F);
+        double *b = (double *)malloc(sizeof(double) * (size_t)F);
+        float *hf = (float *)malloc(sizeof(float) * (size_t)F);
+        uint8_t *qx = (uint8_t *)malloc((size_t)d / 2), *sx = (uint8_t *)malloc((size_t)d / 16);
+        uint8_t *qh = (uint8_t *)malloc((size_t)F / 2), *sh = (uint8_t *)malloc((size_t)F / 16);
+        if (!a || !b || !hf || !qx || !sx || !qh || !sh) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t t = 0; t < T; ++t) {
+                float rx = 0.0f, rh = 0.0f;
+                double *yt = y + t * d;
+                /* quantise this token's row (bf16 bits or fp32, read as stored) */
+                const size_t es = x_dt == OR_BF16 ? 2 : (x_dt == OR_F32 ? 4 : 8);
+                if (oracle_quantize_rows_fp4(1, d, (const uint8_t *)x + (size_t)t * d * es, x_dt, qx, sx, &rx) != 0) {
+#pragma omp atomic write
+                    bad = 1;
+                    continue;
+                }
+                for (int i = 0; i < d; ++i)
+                    yt[i] = 0.0;
+                for (int k = 0; k < K; ++k) {
+                    int e = idx[t * K + k];
+                    for (int f = 0; f < F; ++f)
+                        a[f] = b[f] = 0.0;
+                    for (int j = 0; j < d; ++j) {
+                        double xj = fp4_act(qx, sx, rx, j);
+                        for (int f = 0; f < F; ++f) {
+                            a[f] += xj * fp4_weight(c1, b1, t1, d, F, e, j, f);
+                            b[f] += xj * fp4_weight(c3, b3, t3, d, F, e, j, f);
+                        }
+                    }
+                    for (int f = 0; f < F; ++f)
+                        hf[f] = round_bf16((float)(oracle_silu(a[f]) * b[f]));
+                    if (oracle_quantize_rows_fp4(1, F, hf, OR_F32, qh, sh, &rh) != 0) {
+#pragma omp atomic write
+                        bad = 1;
+                        break;
+                    }
+                    double g = gate[t * K + k];
+                    for (int i = 0; i < d; ++i) {
+                        double o = 0.0;
+                        for (int f = 0; f < F; ++f)
+                            o += fp4_act(qh, sh, rh, f) * fp4_weight(c2, b2, t2, F, d, e, f, i);
+                        yt[i] += g * o;
+                    }
+                }
+            }
+        }
+        free(a); free(b); free(hf); free(qx); free(sx); free(qh); free(sh);
+    }
+    return bad ? -1 : 0;
+}

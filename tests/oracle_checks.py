@@ -634,6 +634,74 @@ def check_fp4_forward_is_layer_of_dequantised(O):
     assert rel_l2(y, O.forward_with_routing(x, idx, gate, w1, w3, w2)) > 1e-3
 
 
+def check_fp4_rows_match_the_weight_quantiser(O):
+    """Per-row 4-bit quantisation of x equals the 4-bit weight quantiser run on
+    each row as a one-column matrix (blocks of 16 along the row, the row's own
+    tensor scale): two independent code paths of the same definition."""
+    rng = np.random.default_rng(56)
+    x = (rng.standard_normal((5, 64)) * rng.choice([1e-3, 1.0, 50.0], size=(5, 1))).astype(np.float32)
+    x[2, 16:32] = 0.0
+    x[4, :] = 0.0
+    codes, bscale, rscale = O.quantize_rows_fp4(x)
+    for t in range(5):
+        m = np.stack([x[t], np.zeros_like(x[t])], axis=1)[None]          # [1][64][2]
+        wc, wb, wt = O.quantize_weights_fp4(m)
+        assert rscale[t] == wt[0]
+        assert np.array_equal(bscale[t], wb[0, :, 0])
+        assert np.array_equal(codes[t] & 0xF, wc[0, 0::2, 0] & 0xF)
+        assert np.array_equal(codes[t] >> 4, wc[0, 1::2, 0] & 0xF)
+
+
+def check_fp4_rows_exact_case(O):
+    """A row made of E2M1 values x power-of-two block scales x 2^-8, every
+    block reaching 6 x its scale and one block at scale 448, is recovered
+    exactly (codes, block scales, row scale)."""
+    rng = np.random.default_rng(57)
+    w, q_ref, sb_ref, st = _fp4_exact_matrix(rng)        # [32][6]: 2 blocks per column
+    x = w.T.astype(np.float32)                            # 6 rows of 32
+    codes, bscale, rscale = O.quantize_rows_fp4(x)
+    for t in range(6):
+        # each row of the exact matrix is a column of it: its tensor scale is that column's
+        col_amax = np.abs(w[:, t]).max()
+        assert rscale[t] == np.float32(col_amax / np.float32(2688.0))
+        got = np.empty(32, int)
+        got[0::2], got[1::2] = codes[t] & 0xF, codes[t] >> 4
+        if col_amax == 6 * 448 * st:                      # the row holding the 448 block
+            assert np.array_equal(got, q_ref[:, t])
+            assert np.array_equal(np.vectorize(O.e4m3_decode)(bscale[t]), sb_ref[:, t])
+
+
+def check_w4a4_layer_band(O):
+    """The layer with 4-bit weights and activations stays within the 4-bit
+    band of the exact layer and moves further from it than weights-only
+    quantisation does (the activations are really quantised)."""
+    T, d, F, n = 10, 64, 64, 4
+    x, Wg, w1, w3, w2 = rand_layer(58, T, d, F, n)
+    idx, gate, _ = O.router(x, Wg, 2)
+    q = [O.quantize_weights_fp4(w.astype(np.float32)) for w in (w1, w3, w2)]
+    y_exact = O.forward_with_routing(x, idx, gate, w1, w3, w2)
+    e_w4 = rel_l2(O.forward_fp4(x, idx, gate, *q), y_exact)
+    e_w4a4 = rel_l2(O.forward_w4a4(x, idx, gate, *q), y_exact)
+    assert e_w4 < e_w4a4 < 0.35, (e_w4, e_w4a4)
+
+
+def check_w4a4_zero_rows_and_scaling(O):
+    """Zero tokens give exact zeros; scaling a token by a power of two scales
+    its output by the same power (every scale is a ratio of the row's own
+    maximum, so the codes do not change)."""
+    T, d, F, n = 6, 32, 32, 3
+    x, Wg, w1, w3, w2 = rand_layer(59, T, d, F, n)
+    x[1] = 0.0
+    x[3] = 4.0 * x[2]
+    idx = np.array([[0, 1], [1, 2], [2, 0], [2, 0], [0, 2], [1, 0]], np.int32)
+    gate = np.tile([[0.5, 0.5]], (T, 1))
+    q = [O.quantize_weights_fp4(w.astype(np.float32)) for w in (w1, w3, w2)]
+    y = O.forward_w4a4(x.astype(np.float32), idx, gate, *q)
+    assert np.all(y[1] == 0.0)
+    xc, xb, xs = O.quantize_rows_fp4(x.astype(np.float32))
+    assert np.array_equal(xc[3], xc[2]) and np.array_equal(xb[3], xb[2]) and xs[3] == 4 * xs[2]
+
+
 ALL_CHECKS = [
     check_worked_example, check_two_way_softmax_closed_form, check_logits_are_x_times_Wg,
     check_topk_brute_force, check_ties_go_to_lower_index, check_gate_invariants, check_silu,
@@ -648,4 +716,6 @@ ALL_CHECKS = [
     check_e4m3_forward_error_band,
     check_e2m1_codec, check_fp4_exact_case, check_fp4_error_band, check_fp4_layer_uses_dequantised_weights,
     check_fp4_forward_is_layer_of_dequantised,
+    check_fp4_rows_match_the_weight_quantiser, check_fp4_rows_exact_case, check_w4a4_layer_band,
+    check_w4a4_zero_rows_and_scaling,
 ]

@@ -40,6 +40,12 @@ MUTANTS = {
     "fp4_tensor_scale_448": [("amax / 2688.0f", "amax / 448.0f")],
     "fp4_nibbles_swapped": [("(uint8_t)(code << (4 * h))", "(uint8_t)(code << (4 * (1 - h)))")],
     "fp4_block_scale_no_div6": [("float qb = (amax_b / 6.0f) / st;", "float qb = amax_b / st;")],
+    "w4a4_no_row_scale": [("return fp4_lut[code] * e4m3_lut[bscale[j / 16]] * (double)rs;",
+                           "return fp4_lut[code] * e4m3_lut[bscale[j / 16]];")],
+    "w4a4_silu_on_up_proj": [("hf[f] = round_bf16((float)(oracle_silu(a[f]) * b[f]));",
+                              "hf[f] = round_bf16((float)(a[f] * oracle_silu(b[f])));")],
+    "fp4_rows_block_scale_no_div6": [("int sb_code = oracle_e4m3_encode((double)((amax_b / 6.0f) / rs));",
+                                      "int sb_code = oracle_e4m3_encode((double)(amax_b / rs));")],
     "e4m3_scale_over_256": [("amax / 448.0f", "amax / 256.0f")],
     "e4m3_bias_8": [("v = ldexp(1.0 + m / 8.0, e - 7);", "v = ldexp(1.0 + m / 8.0, e - 8);")],
     "capacity_keeps_one_more": [("if (row - offsets[e] < capacity) {", "if (row - offsets[e] <= capacity) {")],
