@@ -2,7 +2,7 @@
 """Benchmark of the sparse MoE layer forward (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
-                    [--experts bf16|e4m3|fp4]
+                    [--experts bf16|e4m3|fp4|w4a4]
 
 A step is one moe_forward over one batch: router, top-K, softmax, dispatch,
 gather, GEMM1 (w1/w3 + SwiGLU), GEMM2 (w2), combine.  The default workload is
@@ -28,7 +28,9 @@ sample of the same workload on this host's cores.
 expert weights (per-column scales, quantised once before the timed region)
 and per-row E4M3 activations; --experts fp4 times moe_forward_fp4: 4-bit
 (E2M1) expert weights with E4M3 scales per 16 rows and bf16 activations (bf16
-handle and workloads only).
+handle and workloads only); --experts w4a4 times moe_forward_w4a4: the same
+4-bit weights with 4-bit activations on the block-scaled tensor cores (d and
+ffn multiples of 256).
 
 --impl reference runs the oracle (the reference arm of this build) on the
 host, rank 0 only.
@@ -66,7 +68,8 @@ def load_peaks():
 def workload_desc(cfg, experts="bf16"):
     return "%s: T=%d, d=%d, ffn=%d, n=%d, K=%d, %s%s%s" % (
         cfg.name, cfg.T, cfg.d, cfg.ffn, cfg.n, cfg.K, cfg.dtype, ", skewed router" if cfg.skew else "",
-        {"e4m3": ", E4M3 experts", "fp4": ", 4-bit (E2M1) experts"}.get(experts, ""))
+        {"e4m3": ", E4M3 experts", "fp4": ", 4-bit (E2M1) experts",
+         "w4a4": ", 4-bit (E2M1) experts and activations"}.get(experts, ""))
 
 
 # --------------------------------------------------------------------------
@@ -91,6 +94,13 @@ def algorithmic(cfg, counts, experts="bf16"):
         w2 = used * (F * d // 2 + F * d // 16 + 4)
         gemm1_bytes = w13 + R * d * es + R * F * es
         gemm2_bytes = w2 + R * F * es + R * d * es
+    elif experts == "w4a4":
+        # weights as fp4; A operands as 4-bit codes + scales; the gemm1 stage
+        # also holds the hidden-row quantisation (bf16 H read, codes written)
+        w13 = used * 2 * (d * F // 2 + d * F // 16 + 4)
+        w2 = used * (F * d // 2 + F * d // 16 + 4)
+        gemm1_bytes = w13 + R * (d // 2 + d // 16 + 4) + R * F * es + (R * F * es + R * (F // 2 + F // 16 + 4))
+        gemm2_bytes = w2 + R * (F // 2 + F // 16 + 4) + R * d * es
     elif experts == "e4m3":
         w13 = used * 2 * (d * F + F * 4)
         w2 = used * (F * d + d * 4)
@@ -234,12 +244,13 @@ def oracle_tokens_per_s(cfg, L, budget_s=12.0, experts="bf16"):
         def layer(xs):
             i, g, _ = oracle.router(xs, L["W_g"], cfg.K)
             oracle.forward_e4m3(xs, i, g, *q)
-    elif experts == "fp4":
+    elif experts in ("fp4", "w4a4"):
         q4 = [oracle.quantize_weights_fp4(L[w]) for w in ("w1", "w3", "w2")]
+        fwd = oracle.forward_fp4 if experts == "fp4" else oracle.forward_w4a4
 
         def layer(xs):
             i, g, _ = oracle.router(xs, L["W_g"], cfg.K)
-            oracle.forward_fp4(xs, i, g, *q4)
+            fwd(xs, i, g, *q4)
     else:
         def layer(xs):
             oracle.moe_forward(xs, L["W_g"], L["w1"], L["w3"], L["w2"], cfg.K)
@@ -312,7 +323,7 @@ def main():
     ap.add_argument("--config", default="decode", choices=sorted(mi.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--experts", default="bf16", choices=["bf16", "e4m3", "fp4"])
+    ap.add_argument("--experts", default="bf16", choices=["bf16", "e4m3", "fp4", "w4a4"])
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -357,10 +368,14 @@ def main():
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if cfg.name == "tiny_fp32" else None
     e4m3 = args.experts == "e4m3"
     fp4 = args.experts == "fp4"
-    if e4m3 or fp4:
+    w4a4 = args.experts == "w4a4"
+    if e4m3 or fp4 or w4a4:
         # quantised once, outside the timed region; the bf16 copies are freed
         quant = m.quantize_weights_e4m3 if e4m3 else m.quantize_weights_fp4
-        q = [t for w in (w1, w3, w2) for t in quant(w)]
+        if w4a4:
+            q = [t for w in (w1, w3, w2) for t in m.pack_weights_w4a4(*m.quantize_weights_fp4(w))]
+        else:
+            q = [t for w in (w1, w3, w2) for t in quant(w)]
         torch.cuda.synchronize(dev)
         del w1, w3, w2
         torch.cuda.empty_cache()
@@ -373,6 +388,8 @@ def main():
             m.moe_forward_e4m3(layer.h, T, xin, Wg, *q, yout, iout, wout, stream)
         elif fp4:
             m.moe_forward_fp4(layer.h, T, xin, Wg, *q, yout, iout, wout, stream)
+        elif w4a4:
+            m.moe_forward_w4a4(layer.h, T, xin, Wg, *q, yout, iout, wout, stream)
         else:
             m.moe_forward(layer.h, T, xin, Wg, w1, w3, w2, yout, iout, wout, stream)
 
@@ -493,7 +510,8 @@ def main():
         roof = None
     else:
         intensity = work[dom]["flops"] / work[dom]["bytes"]
-        ridge = peaks["bf16_tflops"] * (2.0 if e4m3 else 1.0) * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        ratio = 2.0 if e4m3 else (4.0 if w4a4 else 1.0)   # dense fp8 / fp4 rate over bf16 (4.5, 9 vs 2.25 PF)
+        ridge = peaks["bf16_tflops"] * ratio * 1e12 / (peaks["hbm_gbs"] * 1e9)
         if intensity < ridge:
             ach = work[dom]["bytes"] / (dom_ms * 1e-3) / 1e9
             roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -501,8 +519,7 @@ def main():
         else:
             timed_s = ms * args.steps * 1e-3
             pk = peaks["bf16_tflops_sustained"] if timed_s > 1.0 else peaks["bf16_tflops"]
-            if e4m3:  # fp8 dense rate = 2x bf16 (nominal 4.5 vs 2.25 PFLOP/s)
-                pk *= 2.0
+            pk *= ratio
             ach = work[dom]["flops"] / (dom_ms * 1e-3) / 1e12
             roof = {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
                     "peak_kind": "sustained" if timed_s > 1.0 else "burst"}
@@ -510,7 +527,8 @@ def main():
         roof["peak_source"] = peak_src
         roof["algorithmic_per_launch"] = work[dom]["bytes"] if roof["bound"] == "hbm" else work[dom]["flops"]
         roof["launch_ms"] = dom_ms
-        roof["traffic"] = recorded_traffic(dom, cfg.name + {"e4m3": "_e4m3", "fp4": "_fp4"}.get(args.experts, ""))
+        roof["traffic"] = recorded_traffic(dom, cfg.name + {"e4m3": "_e4m3", "fp4": "_fp4", "w4a4": "_w4a4"}.get(
+            args.experts, ""))
 
     # ---- CPU baseline (rank 0, N = 1 only) ----
     cpu = None
@@ -518,7 +536,8 @@ def main():
         v, s, reps, cores, el = oracle_tokens_per_s(cfg, L, experts=args.experts)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": "first %d of %d tokens x %d repetitions, full layer in fp64%s (%.1f s)"
-                         % (s, cfg.T, reps, {"e4m3": ", E4M3 experts", "fp4": ", 4-bit experts"}.get(args.experts, ""),
+                         % (s, cfg.T, reps, {"e4m3": ", E4M3 experts", "fp4": ", 4-bit experts",
+                                             "w4a4": ", 4-bit experts and activations"}.get(args.experts, ""),
                             el)}
 
     if rank == 0:
@@ -527,7 +546,8 @@ def main():
             "metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "e4m3" if e4m3 else ("e2m1 weights, bf16" if fp4 else cfg.dtype), "data": "synthetic",
+            "dtype": "e4m3" if e4m3 else ("e2m1 weights, bf16" if fp4 else ("e2m1" if w4a4 else cfg.dtype)),
+            "data": "synthetic",
             "config": {"workload": workload_desc(cfg, args.experts), "global_batch_tokens": T * world,
                        "parallelism": "replicas%d" % world if world > 1 else "single",
                        "l2": "256 MB flush per step" if flush is not None else

@@ -297,6 +297,50 @@ MOE_API moe_status moe_forward_fp4(moe_handle *h, int64_t T, const void *x, cons
                                    moe_stream_t stream);
 
 /*
+ * 4-bit weights AND 4-bit activations on the block-scaled tensor cores
+ * (tcgen05.mma kind::mxf4nvf4, block 16).  The weights are those of
+ * moe_quantize_weights_fp4, repacked once by moe_pack_weights_w4a4 into the
+ * layout the tensor core reads:
+ *   packed_codes [n][cols][rows/2]: row-contiguous (K-major) codes, rows 2j
+ *                and 2j+1 of a column in the low / high nibble of byte j;
+ *   scale_chunks [n][cols/128][rows/64][512] (bytes): for 128 columns and one
+ *                64-row step, the 4 block scales of column c at byte
+ *                16 * (c % 32) + 4 * ((c % 128) / 32) + s (s = 16-row block).
+ * moe_pack_weights_w4a4: codes / block_scales as moe_quantize_weights_fp4
+ * writes them for a matrix [n][rows][cols]; rows a multiple of 64, cols a
+ * multiple of 128.  Needs no handle; enqueued on `stream`.
+ *   Errors: MOE_ERR_INVALID_ARG (sizes, null / misaligned pointer),
+ *   MOE_ERR_UNSUPPORTED (not an sm_100 device), MOE_ERR_CUDA.
+ */
+MOE_API moe_status moe_pack_weights_w4a4(int n, int rows, int cols, const uint8_t *codes,
+                                         const uint8_t *block_scales, uint8_t *packed_codes,
+                                         uint8_t *scale_chunks, moe_stream_t stream);
+
+/*
+ * The layer with 4-bit weights and 4-bit activations (MOE_BF16 handles with d
+ * and ffn multiples of 256): the router, dispatch and capacity of moe_forward;
+ * every gathered x row and every hidden row is quantised like a weight matrix
+ * whose blocks run along the row (an fp32 scale max|row| / (6 * 448), E4M3
+ * scales per 16 elements, E2M1 codes); the tensor core multiplies the codes
+ * with their block scales and accumulates in fp32; the row and matrix scales
+ * are applied to the accumulators:
+ *   h = bf16( silu(rx st1 (Xq . W1q)) (*) (rx st3 (Xq . W3q)) ),
+ *   o = bf16( rh st2 (Hq . W2q) ),   y_t = sum_k gate_k * o_k
+ * w*_packed / w*_chunks from moe_pack_weights_w4a4, w*_matrix_scales from
+ * moe_quantize_weights_fp4; x, W_g, y, topk_idx, topk_w as for moe_forward.
+ * The first call grows the workspace by about T*K*(d + ffn)*0.6 bytes.
+ *   Errors: as moe_forward; MOE_ERR_UNSUPPORTED for an fp32 handle or d, ffn
+ *   not multiples of 256.
+ */
+MOE_API moe_status moe_forward_w4a4(moe_handle *h, int64_t T, const void *x, const float *W_g,
+                                    const uint8_t *w1_packed, const uint8_t *w1_chunks,
+                                    const float *w1_matrix_scales, const uint8_t *w3_packed,
+                                    const uint8_t *w3_chunks, const float *w3_matrix_scales,
+                                    const uint8_t *w2_packed, const uint8_t *w2_chunks,
+                                    const float *w2_matrix_scales, void *y, int32_t *topk_idx, float *topk_w,
+                                    moe_stream_t stream);
+
+/*
  * Debug view of the workspace written by the last forward call: name is "H"
  * (expert hidden layer, [rows][ffn], handle dtype) or "O" (per-row expert
  * outputs, [rows][d], handle dtype for bf16 handles, fp32 for fp32 handles);

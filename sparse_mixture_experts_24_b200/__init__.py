@@ -66,6 +66,8 @@ lib.moe_quantize_weights_e4m3.argtypes = [_int, _int, _int, _vp, _int, _vp, _vp,
 lib.moe_forward_e4m3.argtypes = [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.moe_quantize_weights_fp4.argtypes = [_int, _int, _int, _vp, _int, _vp, _vp, _vp, _vp]
 lib.moe_forward_fp4.argtypes = [_vp, _i64, _vp, _vp] + [_vp] * 9 + [_vp, _vp, _vp, _vp]
+lib.moe_pack_weights_w4a4.argtypes = [_int, _int, _int, _vp, _vp, _vp, _vp, _vp]
+lib.moe_forward_w4a4.argtypes = [_vp, _i64, _vp, _vp] + [_vp] * 9 + [_vp, _vp, _vp, _vp]
 lib.moe_last_error.restype = ctypes.c_char_p
 lib.moe_version.restype = ctypes.c_char_p
 for _f in ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
@@ -73,7 +75,7 @@ for _f in ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatc
            "moe_trace_begin", "moe_trace_end", "moe_dispatch_noalloc", "moe_set_capacity_factor",
            "moe_router_stats", "moe_launch_count", "moe_selftest_timeout",
            "moe_forward_expert_choice", "moe_quantize_weights_e4m3", "moe_forward_e4m3",
-           "moe_quantize_weights_fp4", "moe_forward_fp4"):
+           "moe_quantize_weights_fp4", "moe_forward_fp4", "moe_pack_weights_w4a4", "moe_forward_w4a4"):
     getattr(lib, _f).restype = _int
 
 EXPORTED = ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
@@ -81,7 +83,8 @@ EXPORTED = ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispat
             "moe_last_error", "moe_version", "moe_trace_begin", "moe_trace_end",
             "moe_dispatch_noalloc", "moe_set_capacity_factor", "moe_router_stats",
             "moe_launch_count", "moe_selftest_timeout", "moe_forward_expert_choice",
-            "moe_quantize_weights_e4m3", "moe_forward_e4m3", "moe_quantize_weights_fp4", "moe_forward_fp4")
+            "moe_quantize_weights_e4m3", "moe_forward_e4m3", "moe_quantize_weights_fp4", "moe_forward_fp4",
+            "moe_pack_weights_w4a4", "moe_forward_w4a4")
 
 TRACE_STAGES = ("router", "dispatch", "gather", "gemm1", "gemm2", "combine")
 
@@ -261,6 +264,31 @@ def quantize_weights_fp4(w, stream=None):
     return codes, bscale, tscale
 
 
+def moe_pack_weights_w4a4(n, rows, cols, codes, block_scales, packed, chunks, stream=None) -> None:
+    _check(lib.moe_pack_weights_w4a4(n, rows, cols, _ptr(codes), _ptr(block_scales), _ptr(packed), _ptr(chunks),
+                                     _stream(stream)), "moe_pack_weights_w4a4")
+
+
+def moe_forward_w4a4(h, T, x, W_g, w1_p, w1_c, w1_t, w3_p, w3_c, w3_t, w2_p, w2_c, w2_t, y, topk_idx, topk_w,
+                     stream=None) -> None:
+    _check(lib.moe_forward_w4a4(h, T, _ptr(x), _ptr(W_g), _ptr(w1_p), _ptr(w1_c), _ptr(w1_t), _ptr(w3_p),
+                                _ptr(w3_c), _ptr(w3_t), _ptr(w2_p), _ptr(w2_c), _ptr(w2_t), _ptr(y), _ptr(topk_idx),
+                                _ptr(topk_w), _stream(stream)), "moe_forward_w4a4")
+
+
+def pack_weights_w4a4(codes, block_scales, matrix_scales, stream=None):
+    """(codes [n][rows][cols/2], block scales [n][rows/16][cols], matrix scales [n])
+    of quantize_weights_fp4 (torch CUDA tensors) -> (packed codes [n][cols][rows/2],
+    scale chunks [n][cols/128][rows/64][512], matrix scales)."""
+    import torch
+    n, rows, half = codes.shape
+    cols = 2 * half
+    packed = torch.empty((n, cols, rows // 2), dtype=torch.uint8, device=codes.device)
+    chunks = torch.empty((n, cols // 128, rows // 64, 512), dtype=torch.uint8, device=codes.device)
+    moe_pack_weights_w4a4(n, rows, cols, codes, block_scales, packed, chunks, stream)
+    return packed, chunks, matrix_scales
+
+
 def moe_destroy(h) -> None:
     _check(lib.moe_destroy(h), "moe_destroy")
 
@@ -354,6 +382,20 @@ class MoELayer:
         if topk_w is None:
             topk_w = torch.empty((T, self.K), dtype=torch.float32, device=x.device)
         moe_forward_fp4(self.h, T, x, W_g, *w1, *w3, *w2, y, topk_idx, topk_w, stream)
+        return y, topk_idx, topk_w
+
+    def forward_w4a4(self, x, W_g, w1, w3, w2, y=None, topk_idx=None, topk_w=None, stream=None):
+        """The layer with 4-bit weights and activations; w1, w3, w2 are (packed
+        codes, scale chunks, matrix scales) triples from pack_weights_w4a4."""
+        import torch
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty_like(x)
+        if topk_idx is None:
+            topk_idx = torch.empty((T, self.K), dtype=torch.int32, device=x.device)
+        if topk_w is None:
+            topk_w = torch.empty((T, self.K), dtype=torch.float32, device=x.device)
+        moe_forward_w4a4(self.h, T, x, W_g, *w1, *w3, *w2, y, topk_idx, topk_w, stream)
         return y, topk_idx, topk_w
 
     def set_capacity_factor(self, factor: float) -> None:

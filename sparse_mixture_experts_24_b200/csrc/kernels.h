@@ -196,6 +196,47 @@ cudaError_t launch_fp4_gemm1(const CUtensorMap& tm_xp, const CUtensorMap& tm_c1,
 cudaError_t launch_fp4_gemm2(const CUtensorMap& tm_h, const CUtensorMap& tm_c2, const CUtensorMap& tm_s2,
                              const Fp4GemmArgs& a, int num_sms, cudaStream_t st);
 
+// 4-bit weights and 4-bit activations on the block-scaled tensor cores
+// (w4a4.cu, gemm_w4a4.cu).  Scale chunks: 512 bytes holding the 4 E4M3 scales
+// (one per 16 K) of 128 rows for one 64-wide K step.
+//   pack: codes [n][K][N/2] + scales [n][K/16][N] (moe_quantize_weights_fp4) ->
+//   K-major codes [n][N][K/2] + chunks [n][N/128][K/64][512].  N % 128 == 0.
+cudaError_t launch_w4a4_pack(const uint8_t* codes, const uint8_t* bscale, int n, int K, int N, uint8_t* packed,
+                             uint8_t* chunks, cudaStream_t st);
+//   rows: bf16 rows (row r reads src row row_src[r], or r without row_src) ->
+//   codes [R][K/2], row scales [R], and the chunks of the 128-row GEMM tiles
+//   [tiles][K/64][512] (tile of row r: mblk_base[e] + (r - offsets[e]) / 128).
+//   Rows past offsets[n] are skipped.
+cudaError_t launch_w4a4_rows(const uint16_t* src, const int32_t* row_src, int64_t src_rows, int64_t rows_max, int K,
+                             const int32_t* offsets, const int32_t* mblk_base, int n, uint8_t* codes,
+                             uint8_t* chunks, float* rscale, int num_sms, cudaStream_t st);
+
+struct W4a4GemmArgs {
+    const int32_t* offsets;
+    const int32_t* mblk_base;
+    int n;
+    int64_t R;
+    int k_steps;           // reduction length / 256
+    int n_tiles;
+    int out_cols;          // F (GEMM1) or d (GEMM2)
+    int n_cols;            // columns of the weight matrix (F for w1/w3, d for w2)
+    void* out;             // bf16 [R][out_cols]
+    int* status;
+    const float* row_scale;    // [R] activation row scales
+    const float* mscale0;      // [n] matrix scales: w1 (GEMM1) / w2 (GEMM2)
+    const float* mscale1;      // [n] w3 (GEMM1)
+    const uint8_t* a_chunks;   // activation scale chunks [tiles][K/64][512]
+    const uint8_t* b_chunks0;  // weight scale chunks [n][N/128][K/64][512]: w1 / w2
+    const uint8_t* b_chunks1;  // w3 (GEMM1) / w2 (GEMM2)
+};
+
+// tm_a: activation codes [R][K/2] uint8 (128 x 128 boxes, 128-byte swizzle);
+// tm_b*: packed weight codes [n][N][K/2] uint8 (128 x 128 x 1 boxes, same).
+cudaError_t launch_w4a4_gemm1(const CUtensorMap& tm_xq, const CUtensorMap& tm_w1, const CUtensorMap& tm_w3,
+                              const W4a4GemmArgs& a, int num_sms, cudaStream_t st);
+cudaError_t launch_w4a4_gemm2(const CUtensorMap& tm_hq, const CUtensorMap& tm_w2, const W4a4GemmArgs& a, int num_sms,
+                              cudaStream_t st);
+
 // E4M3 quantisation (e4m3.cu).  Codes are those of v / scale with the quotient
 // rounded to fp32, then to E4M3 by round-to-nearest-even with saturation to
 // +-448; scale = max |v| / 448 over the group (1 for an all-zero group).

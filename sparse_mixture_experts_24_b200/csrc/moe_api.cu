@@ -197,6 +197,18 @@ struct moe_handle {
     const void* c_q1 = nullptr;
     const void* c_q3 = nullptr;
     const void* c_q2 = nullptr;
+    // 4-bit weights and activations: codes of the gathered x rows and of H,
+    // their row scales and scale chunks (allocated once a call asks for them)
+    bool want_w4a4 = false;
+    bool has_w4a4 = false;
+    uint8_t* xq4 = nullptr;
+    uint8_t* hq4 = nullptr;
+    uint8_t* xc4 = nullptr;
+    uint8_t* hc4 = nullptr;
+    float* xr4 = nullptr;
+    float* hr4 = nullptr;
+    CUtensorMap tm_xq4, tm_hq4, tm_wp4[3];
+    const void* c_wp4[3] = {nullptr, nullptr, nullptr};
     // 4-bit experts: maps over the caller's codes and block scales
     CUtensorMap tm_f4[6];  // codes w1, scales w1, codes w3, scales w3, codes w2, scales w2
     const void* c_f4[6] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
@@ -264,7 +276,9 @@ moe_status check_device(moe_handle* h) {
 // token-choice calls, n*C for expert-choice calls).  Capacities only grow.
 moe_status grow(moe_handle* h, int64_t T, int64_t rows_min = 0) {
     const int64_t R_need = std::max(T * h->K, rows_min);
-    if (h->ws && T <= h->T_cap && R_need <= h->R_cap && (h->has_e4m3 || !h->want_e4m3)) return MOE_OK;
+    if (h->ws && T <= h->T_cap && R_need <= h->R_cap && (h->has_e4m3 || !h->want_e4m3) &&
+        (h->has_w4a4 || !h->want_w4a4))
+        return MOE_OK;
     T = std::max(T, h->T_cap);
     const int64_t R = std::max(std::max(R_need, h->R_cap), T * h->K);
     const int64_t nblk = (R + moe::kPairsPerBlock - 1) / moe::kPairsPerBlock;
@@ -298,6 +312,14 @@ moe_status grow(moe_handle* h, int64_t T, int64_t rows_min = 0) {
     const size_t o_h8 = take(e4 ? static_cast<size_t>(R) * h->F : 0);
     const size_t o_xs = take(e4 ? static_cast<size_t>(R) * 4 : 0);
     const size_t o_hs = take(e4 ? static_cast<size_t>(R) * 4 : 0);
+    const bool w4 = h->want_w4a4;
+    const size_t tiles4 = static_cast<size_t>((R + 127) / 128 + h->n);
+    const size_t o_xq4 = take(w4 ? static_cast<size_t>(R) * (h->d / 2) : 0);
+    const size_t o_hq4 = take(w4 ? static_cast<size_t>(R) * (h->F / 2) : 0);
+    const size_t o_xc4 = take(w4 ? tiles4 * (h->d / 64) * 512 : 0);
+    const size_t o_hc4 = take(w4 ? tiles4 * (h->F / 64) * 512 : 0);
+    const size_t o_xr4 = take(w4 ? static_cast<size_t>(R) * 4 : 0);
+    const size_t o_hr4 = take(w4 ? static_cast<size_t>(R) * 4 : 0);
     const size_t total = off;
 
     if (h->ws) {
@@ -346,6 +368,17 @@ moe_status grow(moe_handle* h, int64_t T, int64_t rows_min = 0) {
     h->h8 = e4 ? b + o_h8 : nullptr;
     h->xs = e4 ? reinterpret_cast<float*>(b + o_xs) : nullptr;
     h->hs = e4 ? reinterpret_cast<float*>(b + o_hs) : nullptr;
+    h->has_w4a4 = w4;
+    h->xq4 = w4 ? b + o_xq4 : nullptr;
+    h->hq4 = w4 ? b + o_hq4 : nullptr;
+    h->xc4 = w4 ? b + o_xc4 : nullptr;
+    h->hc4 = w4 ? b + o_hc4 : nullptr;
+    h->xr4 = w4 ? reinterpret_cast<float*>(b + o_xr4) : nullptr;
+    h->hr4 = w4 ? reinterpret_cast<float*>(b + o_hr4) : nullptr;
+    // 4-bit codes: two per byte, so a row of d codes is d / 2 bytes wide
+    if (w4 && (!encode_codes(&h->tm_xq4, h->xq4, h->d / 2, static_cast<uint64_t>(R), 0) ||
+               !encode_codes(&h->tm_hq4, h->hq4, h->F / 2, static_cast<uint64_t>(R), 0)))
+        return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the 4-bit workspace");
     if (e4 && (!encode_codes(&h->tm_x8, h->x8, h->d, static_cast<uint64_t>(R), 0) ||
                !encode_codes(&h->tm_h8, h->h8, h->F, static_cast<uint64_t>(R), 0)))
         return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the E4M3 workspace");
@@ -636,6 +669,78 @@ moe_status run_experts_fp4(moe_handle* h, int64_t T, const void* x, const float*
     a2.tscale0 = ts[2];
     a2.tscale1 = nullptr;
     e = moe::launch_fp4_gemm2(h->tm_h, h->tm_f4[4], h->tm_f4[5], a2, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
+    h->launches += 1;
+    trace_mark(h, 4, st);
+    e = moe::launch_combine(h->o, true, h->db.token_row, topk_w, T, h->K, h->d, y, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+    h->launches += 1;
+    trace_mark(h, 5, st);
+    trace_finish_call(h);
+    return MOE_OK;
+}
+
+// The 4-bit weight-and-activation path: dispatch, x rows to 4 bits (with the
+// tiles' scale chunks), GEMM1 on the block-scaled tensor cores (bf16 H), H rows
+// to 4 bits, GEMM2, combine.
+moe_status run_experts_w4a4(moe_handle* h, int64_t T, const void* x, const float* topk_w, const uint8_t* const* wp,
+                            const uint8_t* const* wc, const float* const* ws, void* y, const int32_t* topk_idx,
+                            cudaStream_t st) {
+    const int64_t R = T * h->K;
+    cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n, moe::kTcBM, h->db, st, capacity_for(h, T));
+    if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
+    h->launches += moe::dispatch_kernel_count(R);
+    trace_mark(h, 1, st);
+    e = moe::launch_w4a4_rows(static_cast<const uint16_t*>(x), h->db.row_token, T, R, h->d, h->db.offsets,
+                              h->db.mblk_base, h->n, h->xq4, h->xc4, h->xr4, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "activation quantisation launch");
+    h->launches += 1;
+    trace_mark(h, 2, st);
+    for (int m = 0; m < 3; ++m) {
+        const uint64_t K = m < 2 ? h->d : h->F, N = m < 2 ? h->F : h->d;
+        if (wp[m] != h->c_wp4[m]) {
+            if (!encode_codes(&h->tm_wp4[m], wp[m], K / 2, N, h->n))
+                return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for packed 4-bit weights");
+            h->c_wp4[m] = wp[m];
+        }
+    }
+    moe::W4a4GemmArgs a1{};
+    a1.offsets = h->db.offsets;
+    a1.mblk_base = h->db.mblk_base;
+    a1.n = h->n;
+    a1.R = R;
+    a1.k_steps = h->d / 256;
+    a1.n_tiles = h->F / 128;
+    a1.out_cols = h->F;
+    a1.n_cols = h->F;
+    a1.out = h->h;
+    a1.status = h->status;
+    a1.row_scale = h->xr4;
+    a1.mscale0 = ws[0];
+    a1.mscale1 = ws[1];
+    a1.a_chunks = h->xc4;
+    a1.b_chunks0 = wc[0];
+    a1.b_chunks1 = wc[1];
+    e = moe::launch_w4a4_gemm1(h->tm_xq4, h->tm_wp4[0], h->tm_wp4[1], a1, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
+    e = moe::launch_w4a4_rows(static_cast<const uint16_t*>(h->h), nullptr, R, R, h->F, h->db.offsets,
+                              h->db.mblk_base, h->n, h->hq4, h->hc4, h->hr4, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "hidden-row quantisation launch");
+    h->launches += 2;
+    trace_mark(h, 3, st);
+    moe::W4a4GemmArgs a2 = a1;
+    a2.k_steps = h->F / 256;
+    a2.n_tiles = h->d / 256;
+    a2.out_cols = h->d;
+    a2.n_cols = h->d;
+    a2.out = h->o;
+    a2.row_scale = h->hr4;
+    a2.mscale0 = ws[2];
+    a2.mscale1 = ws[2];
+    a2.a_chunks = h->hc4;
+    a2.b_chunks0 = wc[2];
+    a2.b_chunks1 = wc[2];
+    e = moe::launch_w4a4_gemm2(h->tm_hq4, h->tm_wp4[2], a2, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
     h->launches += 1;
     trace_mark(h, 4, st);
@@ -978,6 +1083,70 @@ moe_status moe_forward_fp4(moe_handle* h, int64_t T, const void* x, const float*
     const uint8_t* bs[3] = {w1_bscale, w3_bscale, w2_bscale};
     const float* ts[3] = {w1_tscale, w3_tscale, w2_tscale};
     s = run_experts_fp4(h, T, x, topk_w, cw, bs, ts, y, topk_idx, st);
+    return s == MOE_OK ? ok() : s;
+}
+
+moe_status moe_pack_weights_w4a4(int n, int rows, int cols, const uint8_t* codes, const uint8_t* block_scales,
+                                  uint8_t* packed_codes, uint8_t* scale_chunks, moe_stream_t stream) {
+    if (n < 1 || n > 65535) return fail(MOE_ERR_INVALID_ARG, "n = %d outside [1, 65535]", n);
+    if (rows < 64 || rows % 64 != 0 || rows > 1048576)
+        return fail(MOE_ERR_INVALID_ARG, "rows = %d is not a multiple of 64 in [64, 1048576]", rows);
+    if (cols < 128 || cols % 128 != 0)
+        return fail(MOE_ERR_INVALID_ARG, "cols = %d is not a positive multiple of 128", cols);
+    REQUIRE_PTR(codes);
+    REQUIRE_PTR(block_scales);
+    REQUIRE_PTR(packed_codes);
+    REQUIRE_PTR(scale_chunks);
+    int dev = 0, major = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (major != 10) return fail(MOE_ERR_UNSUPPORTED, "device %d is not sm_100", dev);
+    e = moe::launch_w4a4_pack(codes, block_scales, n, rows, cols, packed_codes, scale_chunks,
+                              reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "4-bit weight packing launch");
+    return ok();
+}
+
+moe_status moe_forward_w4a4(moe_handle* h, int64_t T, const void* x, const float* W_g, const uint8_t* w1_packed,
+                            const uint8_t* w1_chunks, const float* w1_matrix_scales, const uint8_t* w3_packed,
+                            const uint8_t* w3_chunks, const float* w3_matrix_scales, const uint8_t* w2_packed,
+                            const uint8_t* w2_chunks, const float* w2_matrix_scales, void* y, int32_t* topk_idx,
+                            float* topk_w, moe_stream_t stream) {
+    moe_status s = check_common(h, T);
+    if (s != MOE_OK) return s;
+    if (h->dtype != MOE_BF16)
+        return fail(MOE_ERR_UNSUPPORTED, "the 4-bit weight-and-activation path needs a MOE_BF16 handle");
+    if (h->d % 256 != 0 || h->F % 256 != 0)
+        return fail(MOE_ERR_UNSUPPORTED, "the 4-bit weight-and-activation path needs d and ffn multiples of 256");
+    if (T == 0) return ok();
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(W_g);
+    REQUIRE_PTR(w1_packed);
+    REQUIRE_PTR(w1_chunks);
+    REQUIRE_PTR(w1_matrix_scales);
+    REQUIRE_PTR(w3_packed);
+    REQUIRE_PTR(w3_chunks);
+    REQUIRE_PTR(w3_matrix_scales);
+    REQUIRE_PTR(w2_packed);
+    REQUIRE_PTR(w2_chunks);
+    REQUIRE_PTR(w2_matrix_scales);
+    REQUIRE_PTR(y);
+    REQUIRE_PTR(topk_idx);
+    REQUIRE_PTR(topk_w);
+    h->want_w4a4 = true;
+    s = prepare(h, T);
+    if (s != MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    moe::chain_begin();
+    trace_mark(h, -1, st);
+    s = run_router(h, T, x, W_g, topk_idx, topk_w, st);
+    if (s != MOE_OK) return s;
+    trace_mark(h, 0, st);
+    const uint8_t* wp[3] = {w1_packed, w3_packed, w2_packed};
+    const uint8_t* wc[3] = {w1_chunks, w3_chunks, w2_chunks};
+    const float* ws[3] = {w1_matrix_scales, w3_matrix_scales, w2_matrix_scales};
+    s = run_experts_w4a4(h, T, x, topk_w, wp, wc, ws, y, topk_idx, st);
     return s == MOE_OK ? ok() : s;
 }
 

@@ -1,0 +1,175 @@
+// w4a4.cu -- operand preparation for the 4-bit tensor-core expert path
+// (4-bit weights and 4-bit activations, "Mixture of Experts: Why Mixtral Only
+// Wakes Up Two Specialists", Part 4: the weights held at 4 bits).
+//
+// The tcgen05 block-scaled MMA (kind::mxf4nvf4, block 16) reads both operands
+// K-major (two E2M1 codes per byte, the lower K index in the low nibble) and
+// takes the E4M3 block scales from tensor memory, copied there from shared
+// memory in 512-byte chunks: a chunk holds the 4 scales (one per 16 K) of 128
+// rows for one 64-wide K step, row r's 4 bytes at 16 * (r % 32) + 4 * (r / 32).
+//
+//   w4a4_pack_kernel   4-bit weights in the layout of moe_quantize_weights_fp4
+//                      (codes [n][K][N/2], scales [n][K/16][N]) -> K-major codes
+//                      [n][N][K/2] and scale chunks [n][N/128][K/64][512].
+//   w4a4_rows_kernel   rows (gathered x rows or hidden rows, bf16) -> E2M1 codes
+//                      [R][K/2], a fp32 scale per row, and the scale chunks of
+//                      the GEMM's 128-row tiles: row r of expert e's segment
+//                      lands in tile mblk_base[e] + (r - offsets[e]) / 128.
+//   Row quantisation: rs = max|row| / (6 * 448) (1 for a zero row), block scale
+//   sb = E4M3((max|block| / 6) / rs), code = E2M1(v / (sb * rs)) (0 when the
+//   product is 0), every quotient and product rounded to fp32.
+#include <cuda_fp4.h>
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+__device__ __forceinline__ int w4_chunk_byte(int r, int s) { return 16 * (r & 31) + 4 * ((r & 127) >> 5) + s; }
+
+// Thread = (matrix e, column c, 16 K-rows kb16): 8 packed bytes and 1 scale.
+__global__ void __launch_bounds__(256) w4a4_pack_kernel(const uint8_t* __restrict__ codes,
+                                                        const uint8_t* __restrict__ bscale, int K, int N,
+                                                        uint8_t* __restrict__ packed, uint8_t* __restrict__ chunks) {
+    const int e = blockIdx.z;
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    const int kb16 = blockIdx.y;
+    if (c >= N) return;
+    const int64_t in_base = (static_cast<int64_t>(e) * K + kb16 * 16) * (N / 2) + c / 2;
+    const int sh = 4 * (c & 1);
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint32_t nib = (__ldg(codes + in_base + static_cast<int64_t>(i) * (N / 2)) >> sh) & 0xFu;
+        if (i < 8)
+            lo |= nib << (4 * i);
+        else
+            hi |= nib << (4 * (i - 8));
+    }
+    uint2* dst = reinterpret_cast<uint2*>(packed + (static_cast<int64_t>(e) * N + c) * (K / 2) + kb16 * 8);
+    *dst = make_uint2(lo, hi);
+    const int KB = K / 64;
+    const int64_t chunk = (static_cast<int64_t>(e) * (N / 128) + c / 128) * KB + kb16 / 4;
+    chunks[chunk * 512 + w4_chunk_byte(c, kb16 & 3)] = __ldg(bscale + (static_cast<int64_t>(e) * (K / 16) + kb16) * N + c);
+}
+
+cudaError_t launch_w4a4_pack(const uint8_t* codes, const uint8_t* bscale, int n, int K, int N, uint8_t* packed,
+                             uint8_t* chunks, cudaStream_t st) {
+    const dim3 grid(static_cast<unsigned>((N + 255) / 256), static_cast<unsigned>(K / 16), static_cast<unsigned>(n));
+    w4a4_pack_kernel<<<grid, 256, 0, st>>>(codes, bscale, K, N, packed, chunks);
+    return cudaGetLastError();
+}
+
+constexpr int kW4RowThreads = 256;
+
+__device__ __forceinline__ float w4_tensor_scale(float amax) { return amax > 0.f ? __fdiv_rn(amax, 2688.f) : 1.f; }
+
+__device__ __forceinline__ float w4_e4m3_value(uint32_t code) {
+    const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code), __NV_E4M3);
+    return __half2float(__half(h));
+}
+
+// One block per row; thread = blocks of 16 elements (bf16 source).
+__global__ void __launch_bounds__(kW4RowThreads) w4a4_rows_kernel(const uint16_t* __restrict__ src,
+                                                                  const int32_t* __restrict__ row_src,
+                                                                  int64_t src_rows, int K,
+                                                                  const int32_t* __restrict__ offsets,
+                                                                  const int32_t* __restrict__ mblk_base, int n,
+                                                                  uint8_t* __restrict__ codes,
+                                                                  uint8_t* __restrict__ chunks,
+                                                                  float* __restrict__ rscale) {
+    griddep_wait();
+    __shared__ float s_max[kW4RowThreads / 32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t rows = offsets[n];
+    const int nblk = K / 16;
+    const int KB = K / 64;
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+        int64_t s = r;
+        if (row_src) {
+            s = __ldg(row_src + r);
+            if (s < 0 || s >= src_rows) continue;  // block-uniform
+        }
+        const uint4* row = reinterpret_cast<const uint4*>(src + s * K);
+        float m = 0.f;
+        for (int b = tid; b < nblk; b += kW4RowThreads) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint4 q = __ldg(row + 2 * b + h);
+                const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    m = fmaxf(m, fabsf(__uint_as_float(w[i] << 16)));
+                    m = fmaxf(m, fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) s_max[warp] = m;
+        __syncthreads();
+        m = s_max[0];
+#pragma unroll
+        for (int w = 1; w < kW4RowThreads / 32; ++w) m = fmaxf(m, s_max[w]);
+        const float rs = w4_tensor_scale(m);
+        // the row's tile and its row inside the tile
+        int lo = 0, hi = n - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (offsets[mid] <= r)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        const int64_t local = r - offsets[lo];
+        const int64_t tile = mblk_base[lo] + local / 128;
+        const int tr = static_cast<int>(local & 127);
+        for (int b = tid; b < nblk; b += kW4RowThreads) {
+            float v[16];
+            float amax_b = 0.f;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint4 q = __ldg(row + 2 * b + h);
+                const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    v[8 * h + 2 * i] = __uint_as_float(w[i] << 16);
+                    v[8 * h + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) amax_b = fmaxf(amax_b, fabsf(v[i]));
+            const uint32_t sb = static_cast<uint32_t>(
+                __nv_cvt_float_to_fp8(__fdiv_rn(__fdiv_rn(amax_b, 6.f), rs), __NV_SATFINITE, __NV_E4M3));
+            const float denom = __fmul_rn(w4_e4m3_value(sb), rs);
+            uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t c =
+                    denom == 0.f ? 0u
+                                 : static_cast<uint32_t>(__nv_cvt_float_to_fp4(__fdiv_rn(v[i], denom), __NV_E2M1,
+                                                                               cudaRoundNearest)) & 0xFu;
+                packed[i >> 3] |= c << (4 * (i & 7));
+            }
+            *reinterpret_cast<uint2*>(codes + r * (K / 2) + 8 * b) = make_uint2(packed[0], packed[1]);
+            chunks[(tile * KB + b / 4) * 512 + w4_chunk_byte(tr, b & 3)] = static_cast<uint8_t>(sb);
+        }
+        if (tid == 0) rscale[r] = rs;
+        __syncthreads();  // s_max is reused by the next row
+    }
+    griddep_launch_dependents();
+}
+
+cudaError_t launch_w4a4_rows(const uint16_t* src, const int32_t* row_src, int64_t src_rows, int64_t rows_max, int K,
+                             const int32_t* offsets, const int32_t* mblk_base, int n, uint8_t* codes,
+                             uint8_t* chunks, float* rscale, int num_sms, cudaStream_t st) {
+    int64_t blocks = rows_max;
+    if (blocks > static_cast<int64_t>(num_sms) * 8) blocks = static_cast<int64_t>(num_sms) * 8;
+    if (blocks < 1) blocks = 1;
+    launch_k(w4a4_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kW4RowThreads), 0, st, src, row_src,
+             src_rows, K, offsets, mblk_base, n, codes, chunks, rscale);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

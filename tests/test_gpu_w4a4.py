@@ -1,0 +1,164 @@
+"""4-bit weights and 4-bit activations on the block-scaled tensor cores vs the
+fp64 oracle, through the C ABI (needs a B200).
+
+The weight repacking is a pure permutation, checked byte for byte against a
+numpy permutation of the same codes; the layer runs on the oracle's 4-bit
+weights and is compared with the oracle's 4-bit weight-and-activation layer
+under the oracle's routing (tokens whose GPU routing agrees)."""
+import zlib
+
+import numpy as np
+import pytest
+
+import moe_inputs as mi
+import oracle
+from gpu_helpers import (TOL_Y, agreeing_tokens, compare_routing, dev, host, rel_l2, require_cuda,
+                         stratified_sample, y_as_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+def seed_of(name: str) -> int:
+    return zlib.crc32(name.encode()) % 1000
+
+
+def numpy_pack(codes, bscale):
+    """The documented layout of moe_pack_weights_w4a4, written with numpy."""
+    n, K, half = codes.shape
+    N = 2 * half
+    nib = np.empty((n, K, N), np.uint8)
+    nib[:, :, 0::2], nib[:, :, 1::2] = codes & 0xF, codes >> 4
+    kmaj = nib.transpose(0, 2, 1)                                   # [n][N][K]
+    packed = (kmaj[:, :, 0::2] | (kmaj[:, :, 1::2] << 4)).astype(np.uint8)
+    chunks = np.zeros((n, N // 128, K // 64, 512), np.uint8)
+    c = np.arange(N)
+    pos = 16 * (c % 32) + 4 * ((c % 128) // 32)
+    for kb16 in range(K // 16):
+        chunks[:, c // 128, kb16 // 4, pos + kb16 % 4] = bscale[:, kb16, :]
+    return packed, chunks
+
+
+@pytest.mark.parametrize("shape", [(2, 64, 128), (3, 256, 384), (1, 512, 256)])
+def test_pack_is_the_documented_permutation(shape):
+    import sparse_mixture_experts_24_b200 as m
+    torch = require_cuda()
+    n, K, N = shape
+    rng = np.random.default_rng(K + N)
+    codes = rng.integers(0, 256, (n, K, N // 2), dtype=np.uint8)
+    bscale = rng.integers(0, 0x7F, (n, K // 16, N), dtype=np.uint8)
+    packed, chunks, _ = m.pack_weights_w4a4(dev(codes), dev(bscale), None)
+    torch.cuda.synchronize()
+    p_ref, c_ref = numpy_pack(codes, bscale)
+    assert np.array_equal(host(packed), p_ref)
+    assert np.array_equal(host(chunks), c_ref)
+
+
+def prepared_weights(L):
+    """Oracle 4-bit weights (logical layout) and their packed device form."""
+    import sparse_mixture_experts_24_b200 as m
+    q = [oracle.quantize_weights_fp4(L[w]) for w in ("w1", "w3", "w2")]
+    packed = [m.pack_weights_w4a4(dev(c), dev(b), dev(t)) for c, b, t in q]
+    return q, packed
+
+
+FWD_CASES = [
+    # name, T, d, ffn, n, K
+    ("w4a4_small", 300, 256, 512, 8, 2),
+    ("w4a4_tails", 77, 512, 256, 4, 1),
+    ("w4a4_T1", 1, 256, 256, 8, 2),
+    ("w4a4_n64", 700, 256, 256, 64, 4),
+    ("w4a4_big_segments", 1500, 512, 768, 4, 2),
+]
+
+
+@pytest.mark.parametrize("case", FWD_CASES, ids=[c[0] for c in FWD_CASES])
+def test_w4a4_layer_matches_oracle(case):
+    import sparse_mixture_experts_24_b200 as m
+    torch = require_cuda()
+    name, T, d, F, n, K = case
+    cfg = mi.custom_config(name, T=T, d=d, ffn=F, n=n, K=K, dtype="bf16")
+    L = mi.make_layer(cfg, seed=seed_of(name))
+    q, packed = prepared_weights(L)
+    layer = m.MoELayer(n, K, d, F, "bf16")
+    try:
+        y, idx, w = layer.forward_w4a4(dev(L["x"]), dev(L["W_g"]), *packed)
+        layer.sync_status()
+        torch.cuda.synchronize()
+        y, idx, w = host(y), host(idx), host(w)
+    finally:
+        layer.close()
+    o_idx, o_gate, o_logits = oracle.router(L["x"], L["W_g"], K)
+    compare_routing(idx, w, o_idx, o_gate, o_logits, L["x"], L["W_g"], K)
+    agree = agreeing_tokens(idx, o_idx)
+    y_ref = oracle.forward_w4a4(L["x"], o_idx, o_gate, *q)
+    yg = y_as_f64(y)
+    err = rel_l2(yg[agree], y_ref[agree])
+    assert err <= TOL_Y["bf16"], err
+    per_tok = np.linalg.norm(yg - y_ref, axis=1)[agree] / np.maximum(np.linalg.norm(y_ref, axis=1)[agree], 1e-30)
+    assert per_tok.max() <= 5 * TOL_Y["bf16"], per_tok.max()
+    # really 4-bit: away from the exact layer, inside the 4-bit band
+    y_exact = oracle.forward_with_routing(L["x"], o_idx, o_gate, L["w1"], L["w3"], L["w2"])
+    band = rel_l2(yg[agree], y_exact[agree])
+    assert 0.03 < band < 0.4, band
+
+
+def test_w4a4_capacity_and_rejections():
+    import sparse_mixture_experts_24_b200 as m
+    torch = require_cuda()
+    name, T, d, F, n, K = "w4a4_capacity", 600, 256, 256, 8, 2
+    cfg = mi.custom_config(name, T=T, d=d, ffn=F, n=n, K=K, dtype="bf16", skew=True)
+    L = mi.make_layer(cfg, seed=seed_of(name))
+    q, packed = prepared_weights(L)
+    C = int(np.ceil(T * K / n))
+    layer = m.MoELayer(n, K, d, F, "bf16")
+    try:
+        layer.set_capacity_factor(1.0)
+        y, idx, w = layer.forward_w4a4(dev(L["x"]), dev(L["W_g"]), *packed)
+        _, offsets, _, token_row = (host(a) for a in layer.dispatch(idx))
+        layer.sync_status()
+        y, idx = host(y), host(idx)
+    finally:
+        layer.close()
+    o_idx, o_gate, _ = oracle.router(L["x"], L["W_g"], K)
+    assert (idx == o_idx).all()
+    _, o_off, _, o_tr = oracle.dispatch_capacity(o_idx, n, C)
+    assert np.array_equal(offsets, o_off) and np.array_equal(token_row, o_tr)
+    dropped = o_tr < 0
+    assert dropped.any()
+    y_ref = oracle.forward_w4a4(L["x"], o_idx, np.where(dropped, 0.0, o_gate), *q)
+    assert rel_l2(y_as_f64(y), y_ref) <= TOL_Y["bf16"]
+    # d or ffn not a multiple of 256, an fp32 handle
+    for args in ((8, 2, 128, 256, "bf16"), (8, 2, 256, 256, "f32")):
+        layer = m.MoELayer(*args)
+        try:
+            x = torch.zeros((4, args[2]), dtype=torch.bfloat16 if args[4] == "bf16" else torch.float32,
+                            device="cuda")
+            with pytest.raises(m.MoEError) as ei:
+                layer.forward_w4a4(x, x, (x, x, x), (x, x, x), (x, x, x))
+            assert ei.value.status == m.MOE_ERR_UNSUPPORTED
+        finally:
+            layer.close()
+
+
+def test_w4a4_full_size_decode():
+    """The decode workload (Mixtral layer shapes) with 4-bit weights and
+    activations on an expert-stratified token sample."""
+    import sparse_mixture_experts_24_b200 as m
+    torch = require_cuda()
+    cfg = mi.CONFIGS["decode"]
+    L = mi.make_layer(cfg, seed=0)
+    q, packed = prepared_weights(L)
+    layer = m.MoELayer(cfg.n, cfg.K, cfg.d, cfg.ffn, "bf16")
+    try:
+        y, idx, w = layer.forward_w4a4(dev(L["x"]), dev(L["W_g"]), *packed)
+        layer.sync_status()
+        torch.cuda.synchronize()
+        y, idx, w = host(y), host(idx), host(w)
+    finally:
+        layer.close()
+    o_idx, o_gate, o_logits = oracle.router(L["x"], L["W_g"], cfg.K)
+    compare_routing(idx, w, o_idx, o_gate, o_logits, L["x"], L["W_g"], cfg.K)
+    pick = stratified_sample(o_idx, cfg.n, 12)
+    pick = pick[(idx[pick] == o_idx[pick]).all(axis=1)]
+    y_ref = oracle.forward_w4a4(L["x"][pick], o_idx[pick], o_gate[pick], *q)
+    assert rel_l2(y_as_f64(y)[pick], y_ref) <= TOL_Y["bf16"]
