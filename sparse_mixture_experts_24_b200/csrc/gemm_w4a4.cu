@@ -10,7 +10,7 @@
 // 4-bit weights ("Mixture of Experts: Why Mixtral Only Wakes Up Two
 // Specialists", Part 4).
 //
-// One persistent CTA per SM, 192 threads:
+// One persistent CTA per SM, 320 threads:
 //   warp 0     TMA producer, 4-stage ring of 54 KB: per stage a K step of 256
 //              (128 bytes of codes per row): A 128 rows (128-byte swizzle), B
 //              256 rows of K-major weight codes (GEMM1: 128 columns of w1 and
@@ -20,8 +20,10 @@
 //              stages x 48 columns of scale factors); per 64-wide K step it
 //              copies the scale chunks into TMEM (tcgen05.cp 32x128b.warpx4)
 //              and issues tcgen05.mma kind::mxf4nvf4 block16 M=128 N=256.
-//   warps 2-5  epilogue: accumulator x row scale x matrix scale, SwiGLU
-//              (GEMM1) or a copy (GEMM2), bf16 rows.
+//   warps 2-9  epilogue, two warps per TMEM lane quadrant splitting the
+//              columns: accumulator x row scale x matrix scale, SwiGLU (GEMM1)
+//              or a copy (GEMM2), bf16 rows.  With one accumulator the MMAs of
+//              the next tile wait for the epilogue, so it is kept short.
 // Every wait is bounded (common.cuh).
 #include "common.cuh"
 #include "kernels.h"
@@ -32,7 +34,6 @@ namespace w4gemm {
 
 constexpr int kBM = kTcBM;   // 128
 constexpr int kBN = 256;
-constexpr int kKStep = 256;  // K elements per stage
 constexpr int kABytes = kBM * 128;      // 16 KB
 constexpr int kBHalfBytes = 128 * 128;  // 16 KB: 128 rows of 128 bytes
 constexpr int kBBytes = 2 * kBHalfBytes;
@@ -40,7 +41,8 @@ constexpr int kSfaBytes = 4 * 512;
 constexpr int kSfbBytes = 8 * 512;
 constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 54 KB
 constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, each taking half the columns
+constexpr int kThreads = (2 + kEpiWarps) * 32;
 constexpr int kMaxN = 256;
 constexpr int kTmemCols = 512;
 constexpr int kSfCols = 48;  // per stage: 4 K steps x (4 SFA + 8 SFB columns)
@@ -85,7 +87,7 @@ __device__ __forceinline__ Tile tile_at(int t, const int32_t* off, const int32_t
     return ti;
 }
 
-__device__ __forceinline__ float silu(float a) { return a / (1.f + __expf(-a)); }
+__device__ __forceinline__ float silu(float a) { return __fdividef(a, 1.f + __expf(-a)); }
 
 }  // namespace w4gemm
 
@@ -109,7 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&tail->empty[s]), 1);
         }
         mbar_init(smem_u32(&tail->accum_full), 1);
-        mbar_init(smem_u32(&tail->accum_empty), 4);
+        mbar_init(smem_u32(&tail->accum_empty), kEpiWarps);
         mbar_init(smem_u32(&tail->done), 1);
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -231,26 +233,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(smem_u32(&tail->done), 0, status, kStatusTimeoutDrain);
         }
     } else {
-        // ---------------- epilogue (warps 2..5) ----------------
+        // ---------------- epilogue (warps 2..9) ----------------
+        // warp w reads TMEM lanes 32 (w % 4) .. +31 and the column half (w - 2) / 4
         const int quad = warp & 3;
+        const int half = (warp - 2) >> 2;
         int local = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++local) {
             const Tile ti = tile_at(t, tail->off, tail->mblk, n, args.n_tiles);
+            const int valid = min(32, ti.rows - quad * 32);
+            const bool row_ok = lane < valid;
+            const int64_t row_base = static_cast<int64_t>(ti.row0) + quad * 32;
+            // scales first: their loads overlap the wait for the accumulator
+            const float rs = row_ok ? args.row_scale[row_base + lane] : 0.f;
+            const float m0 = __ldg(args.mscale0 + ti.e);
+            const float m1 = kSwiGLU ? __ldg(args.mscale1 + ti.e) : 0.f;
             if (!mbar_wait(smem_u32(&tail->accum_full), static_cast<uint32_t>(local) & 1u, status,
                            kStatusTimeoutAccum))
                 break;
             tc_fence_after();
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
-            const int valid = min(32, ti.rows - quad * 32);
-            const bool row_ok = lane < valid;
-            const int64_t row_base = static_cast<int64_t>(ti.row0) + quad * 32;
-            const float rs = row_ok ? args.row_scale[row_base + lane] : 0.f;
             uint16_t* out = static_cast<uint16_t*>(args.out);
-            const float g0 = __ldg(args.mscale0 + ti.e) * rs;
+            const float g0 = m0 * rs;
             if (kSwiGLU) {
-                const float g1 = __ldg(args.mscale1 + ti.e) * rs;
+                const float g1 = m1 * rs;
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 2 * half; c < 2 * half + 2; ++c) {
                     uint32_t a[32], b[32];
                     tmem_ld_32x32b_x32(tbase + c * 32, a);
                     tmem_ld_32x32b_x32(tbase + 128 + c * 32, b);
@@ -273,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             } else {
 #pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 4 * half; c < 4 * half + 4; ++c) {
                     uint32_t a[32];
                     tmem_ld_32x32b_x32(tbase + c * 32, a);
                     tmem_wait_ld();
