@@ -373,7 +373,9 @@ def main():
         # quantised once, outside the timed region; the bf16 copies are freed
         quant = m.quantize_weights_e4m3 if e4m3 else m.quantize_weights_fp4
         if w4a4:
-            q = [t for w in (w1, w3, w2) for t in m.pack_weights_w4a4(*m.quantize_weights_fp4(w))]
+            # the gate/up pair pack of w1 and w3, then w2
+            q = list(m.pack_weights_w4a4(*m.quantize_weights_fp4(w1), pair=m.quantize_weights_fp4(w3)))
+            q += list(m.pack_weights_w4a4(*m.quantize_weights_fp4(w2)))
         else:
             q = [t for w in (w1, w3, w2) for t in quant(w)]
         torch.cuda.synchronize(dev)

@@ -300,20 +300,29 @@ MOE_API moe_status moe_forward_fp4(moe_handle *h, int64_t T, const void *x, cons
  * 4-bit weights AND 4-bit activations on the block-scaled tensor cores
  * (tcgen05.mma kind::mxf4nvf4, block 16).  The weights are those of
  * moe_quantize_weights_fp4, repacked once by moe_pack_weights_w4a4 into the
- * layout the tensor core reads:
+ * layout the tensor core reads.  A single matrix [n][rows][cols] becomes
  *   packed_codes [n][cols][rows/2]: row-contiguous (K-major) codes, rows 2j
  *                and 2j+1 of a column in the low / high nibble of byte j;
  *   scale_chunks [n][cols/128][rows/64][512] (bytes): for 128 columns and one
  *                64-row step, the 4 block scales of column c at byte
  *                16 * (c % 32) + 4 * ((c % 128) / 32) + s (s = 16-row block).
- * moe_pack_weights_w4a4: codes / block_scales as moe_quantize_weights_fp4
- * writes them for a matrix [n][rows][cols]; rows a multiple of 64, cols a
- * multiple of 128.  Needs no handle; enqueued on `stream`.
- *   Errors: MOE_ERR_INVALID_ARG (sizes, null / misaligned pointer),
- *   MOE_ERR_UNSUPPORTED (not an sm_100 device), MOE_ERR_CUDA.
+ * A gate/up pair (w1 and w3, pair_codes / pair_block_scales = w3's) becomes
+ * one matrix of 2*cols packed columns: packed column p holds column
+ * 64 * (p / 128) + p % 64 of w1 when p % 128 < 64, else the same column of w3,
+ * so each 128-column block carries both projections of 64 hidden columns;
+ * packed_codes is then [n][2*cols][rows/2] and scale_chunks
+ * [n][2*cols/128][rows/64][512], laid out as above for packed columns.
+ * Arguments: codes / block_scales (and the pair's) as moe_quantize_weights_fp4
+ * writes them; rows a multiple of 64; cols a multiple of 128 (64 for a
+ * pair); pair_codes and pair_block_scales both null for a single matrix.
+ * Needs no handle; enqueued on `stream`; the caller owns every buffer.
+ *   Errors: MOE_ERR_INVALID_ARG (sizes, null / misaligned pointer, one of the
+ *   pair pointers null), MOE_ERR_UNSUPPORTED (not an sm_100 device),
+ *   MOE_ERR_CUDA.
  */
 MOE_API moe_status moe_pack_weights_w4a4(int n, int rows, int cols, const uint8_t *codes,
-                                         const uint8_t *block_scales, uint8_t *packed_codes,
+                                         const uint8_t *block_scales, const uint8_t *pair_codes,
+                                         const uint8_t *pair_block_scales, uint8_t *packed_codes,
                                          uint8_t *scale_chunks, moe_stream_t stream);
 
 /*
@@ -326,16 +335,19 @@ MOE_API moe_status moe_pack_weights_w4a4(int n, int rows, int cols, const uint8_
  * are applied to the accumulators:
  *   h = bf16( silu(rx st1 (Xq . W1q)) (*) (rx st3 (Xq . W3q)) ),
  *   o = bf16( rh st2 (Hq . W2q) ),   y_t = sum_k gate_k * o_k
- * w*_packed / w*_chunks from moe_pack_weights_w4a4, w*_matrix_scales from
- * moe_quantize_weights_fp4; x, W_g, y, topk_idx, topk_w as for moe_forward.
+ * w13_packed / w13_chunks: the gate/up pair pack of moe_pack_weights_w4a4
+ * (w1 and w3, rows = d, cols = ffn); w2_packed / w2_chunks: w2 packed alone
+ * (rows = ffn, cols = d); w*_matrix_scales from moe_quantize_weights_fp4;
+ * x, W_g, y, topk_idx, topk_w as for moe_forward.  The GEMMs use tiles of
+ * 256 packed columns; MOE_W4A4_TILE=128 selects 128-column tiles with two
+ * accumulators (same results, measured slower on the Mixtral shapes).
  * The first call grows the workspace by about T*K*(d + ffn)*0.6 bytes.
  *   Errors: as moe_forward; MOE_ERR_UNSUPPORTED for an fp32 handle or d, ffn
  *   not multiples of 256.
  */
 MOE_API moe_status moe_forward_w4a4(moe_handle *h, int64_t T, const void *x, const float *W_g,
-                                    const uint8_t *w1_packed, const uint8_t *w1_chunks,
-                                    const float *w1_matrix_scales, const uint8_t *w3_packed,
-                                    const uint8_t *w3_chunks, const float *w3_matrix_scales,
+                                    const uint8_t *w13_packed, const uint8_t *w13_chunks,
+                                    const float *w1_matrix_scales, const float *w3_matrix_scales,
                                     const uint8_t *w2_packed, const uint8_t *w2_chunks,
                                     const float *w2_matrix_scales, void *y, int32_t *topk_idx, float *topk_w,
                                     moe_stream_t stream);

@@ -66,8 +66,8 @@ lib.moe_quantize_weights_e4m3.argtypes = [_int, _int, _int, _vp, _int, _vp, _vp,
 lib.moe_forward_e4m3.argtypes = [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.moe_quantize_weights_fp4.argtypes = [_int, _int, _int, _vp, _int, _vp, _vp, _vp, _vp]
 lib.moe_forward_fp4.argtypes = [_vp, _i64, _vp, _vp] + [_vp] * 9 + [_vp, _vp, _vp, _vp]
-lib.moe_pack_weights_w4a4.argtypes = [_int, _int, _int, _vp, _vp, _vp, _vp, _vp]
-lib.moe_forward_w4a4.argtypes = [_vp, _i64, _vp, _vp] + [_vp] * 9 + [_vp, _vp, _vp, _vp]
+lib.moe_pack_weights_w4a4.argtypes = [_int, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.moe_forward_w4a4.argtypes = [_vp, _i64, _vp, _vp] + [_vp] * 7 + [_vp, _vp, _vp, _vp]
 lib.moe_last_error.restype = ctypes.c_char_p
 lib.moe_version.restype = ctypes.c_char_p
 for _f in ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
@@ -264,28 +264,36 @@ def quantize_weights_fp4(w, stream=None):
     return codes, bscale, tscale
 
 
-def moe_pack_weights_w4a4(n, rows, cols, codes, block_scales, packed, chunks, stream=None) -> None:
-    _check(lib.moe_pack_weights_w4a4(n, rows, cols, _ptr(codes), _ptr(block_scales), _ptr(packed), _ptr(chunks),
-                                     _stream(stream)), "moe_pack_weights_w4a4")
+def moe_pack_weights_w4a4(n, rows, cols, codes, block_scales, pair_codes, pair_block_scales, packed, chunks,
+                          stream=None) -> None:
+    _check(lib.moe_pack_weights_w4a4(n, rows, cols, _ptr(codes), _ptr(block_scales), _ptr(pair_codes),
+                                     _ptr(pair_block_scales), _ptr(packed), _ptr(chunks), _stream(stream)),
+           "moe_pack_weights_w4a4")
 
 
-def moe_forward_w4a4(h, T, x, W_g, w1_p, w1_c, w1_t, w3_p, w3_c, w3_t, w2_p, w2_c, w2_t, y, topk_idx, topk_w,
+def moe_forward_w4a4(h, T, x, W_g, w13_p, w13_c, w1_t, w3_t, w2_p, w2_c, w2_t, y, topk_idx, topk_w,
                      stream=None) -> None:
-    _check(lib.moe_forward_w4a4(h, T, _ptr(x), _ptr(W_g), _ptr(w1_p), _ptr(w1_c), _ptr(w1_t), _ptr(w3_p),
-                                _ptr(w3_c), _ptr(w3_t), _ptr(w2_p), _ptr(w2_c), _ptr(w2_t), _ptr(y), _ptr(topk_idx),
-                                _ptr(topk_w), _stream(stream)), "moe_forward_w4a4")
+    _check(lib.moe_forward_w4a4(h, T, _ptr(x), _ptr(W_g), _ptr(w13_p), _ptr(w13_c), _ptr(w1_t), _ptr(w3_t),
+                                _ptr(w2_p), _ptr(w2_c), _ptr(w2_t), _ptr(y), _ptr(topk_idx), _ptr(topk_w),
+                                _stream(stream)), "moe_forward_w4a4")
 
 
-def pack_weights_w4a4(codes, block_scales, matrix_scales, stream=None):
+def pack_weights_w4a4(codes, block_scales, matrix_scales, pair=None, stream=None):
     """(codes [n][rows][cols/2], block scales [n][rows/16][cols], matrix scales [n])
     of quantize_weights_fp4 (torch CUDA tensors) -> (packed codes [n][cols][rows/2],
-    scale chunks [n][cols/128][rows/64][512], matrix scales)."""
+    scale chunks [n][cols/128][rows/64][512], matrix scales).  With pair = w3's
+    triple (codes being w1's): the gate/up pair pack of 2*cols packed columns,
+    returned as (packed, chunks, w1 matrix scales, w3 matrix scales)."""
     import torch
     n, rows, half = codes.shape
     cols = 2 * half
-    packed = torch.empty((n, cols, rows // 2), dtype=torch.uint8, device=codes.device)
-    chunks = torch.empty((n, cols // 128, rows // 64, 512), dtype=torch.uint8, device=codes.device)
-    moe_pack_weights_w4a4(n, rows, cols, codes, block_scales, packed, chunks, stream)
+    out_cols = 2 * cols if pair is not None else cols
+    packed = torch.empty((n, out_cols, rows // 2), dtype=torch.uint8, device=codes.device)
+    chunks = torch.empty((n, out_cols // 128, rows // 64, 512), dtype=torch.uint8, device=codes.device)
+    pc, pb = (pair[0], pair[1]) if pair is not None else (None, None)
+    moe_pack_weights_w4a4(n, rows, cols, codes, block_scales, pc, pb, packed, chunks, stream)
+    if pair is not None:
+        return packed, chunks, matrix_scales, pair[2]
     return packed, chunks, matrix_scales
 
 
@@ -384,9 +392,10 @@ class MoELayer:
         moe_forward_fp4(self.h, T, x, W_g, *w1, *w3, *w2, y, topk_idx, topk_w, stream)
         return y, topk_idx, topk_w
 
-    def forward_w4a4(self, x, W_g, w1, w3, w2, y=None, topk_idx=None, topk_w=None, stream=None):
-        """The layer with 4-bit weights and activations; w1, w3, w2 are (packed
-        codes, scale chunks, matrix scales) triples from pack_weights_w4a4."""
+    def forward_w4a4(self, x, W_g, w13, w2, y=None, topk_idx=None, topk_w=None, stream=None):
+        """The layer with 4-bit weights and activations; w13 is the gate/up pair
+        pack (packed, chunks, w1 scales, w3 scales) and w2 the (packed, chunks,
+        matrix scales) triple, both from pack_weights_w4a4."""
         import torch
         T = x.shape[0]
         if y is None:
@@ -395,7 +404,7 @@ class MoELayer:
             topk_idx = torch.empty((T, self.K), dtype=torch.int32, device=x.device)
         if topk_w is None:
             topk_w = torch.empty((T, self.K), dtype=torch.float32, device=x.device)
-        moe_forward_w4a4(self.h, T, x, W_g, *w1, *w3, *w2, y, topk_idx, topk_w, stream)
+        moe_forward_w4a4(self.h, T, x, W_g, *w13, *w2, y, topk_idx, topk_w, stream)
         return y, topk_idx, topk_w
 
     def set_capacity_factor(self, factor: float) -> None:

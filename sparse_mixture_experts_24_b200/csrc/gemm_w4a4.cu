@@ -10,20 +10,20 @@
 // 4-bit weights ("Mixture of Experts: Why Mixtral Only Wakes Up Two
 // Specialists", Part 4).
 //
-// One persistent CTA per SM, 320 threads:
-//   warp 0     TMA producer, 4-stage ring of 54 KB: per stage a K step of 256
-//              (128 bytes of codes per row): A 128 rows (128-byte swizzle), B
-//              256 rows of K-major weight codes (GEMM1: 128 columns of w1 and
-//              the same of w3; GEMM2: 256 columns of w2), and by plain bulk
-//              copies the matching 512-byte scale chunks (4 for A, 8 for B).
-//   warp 1     allocates 512 TMEM columns (one 256-column accumulator, four
-//              stages x 48 columns of scale factors); per 64-wide K step it
-//              copies the scale chunks into TMEM (tcgen05.cp 32x128b.warpx4)
-//              and issues tcgen05.mma kind::mxf4nvf4 block16 M=128 N=256.
+// One persistent CTA per SM, 320 threads, tiles of 128 rows x kBN columns of
+// the packed B (kBN = 128: two accumulators, 6 stages of 36 KB; kBN = 256: one
+// accumulator, 4 stages of 54 KB -- the block scales take the rest of TMEM):
+//   warp 0     TMA producer: per stage a K step of 256 (128 bytes of codes per
+//              row): A 128 rows (128-byte swizzle), kBN / 128 blocks of 128
+//              K-major weight rows (GEMM1: the w1|w3 pair pack, 64 hidden
+//              columns per block; GEMM2: w2), and by plain bulk copies the
+//              matching 512-byte scale chunks (4 for A, 4 per B block).
+//   warp 1     allocates 512 TMEM columns; per 64-wide K step it copies the
+//              scale chunks into TMEM (tcgen05.cp 32x128b.warpx4) and issues
+//              tcgen05.mma kind::mxf4nvf4 block16 M=128 N=kBN.
 //   warps 2-9  epilogue, two warps per TMEM lane quadrant splitting the
 //              columns: accumulator x row scale x matrix scale, SwiGLU (GEMM1)
-//              or a copy (GEMM2), bf16 rows.  With one accumulator the MMAs of
-//              the next tile wait for the epilogue, so it is kept short.
+//              or a copy (GEMM2), bf16 rows.
 // Every wait is bounded (common.cuh).
 #include "common.cuh"
 #include "kernels.h"
@@ -33,27 +33,36 @@ namespace moe {
 namespace w4gemm {
 
 constexpr int kBM = kTcBM;   // 128
-constexpr int kBN = 256;
-constexpr int kABytes = kBM * 128;      // 16 KB
-constexpr int kBHalfBytes = 128 * 128;  // 16 KB: 128 rows of 128 bytes
-constexpr int kBBytes = 2 * kBHalfBytes;
-constexpr int kSfaBytes = 4 * 512;
-constexpr int kSfbBytes = 8 * 512;
-constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 54 KB
-constexpr int kStages = 4;
-constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, each taking half the columns
-constexpr int kThreads = (2 + kEpiWarps) * 32;
+constexpr int kABytes = kBM * 128;      // 16 KB: 128 rows of 128 bytes (K step of 256)
+constexpr int kBBlockBytes = 128 * 128; // 16 KB: one 128-row block of B
+constexpr int kSfaBytes = 4 * 512;      // 4 chunks (64-wide K steps) of A scales
+constexpr int kSfbBlockBytes = 4 * 512; // the same for one 128-row block of B
 constexpr int kMaxN = 256;
 constexpr int kTmemCols = 512;
-constexpr int kSfCols = 48;  // per stage: 4 K steps x (4 SFA + 8 SFB columns)
+constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, each taking half the columns
+constexpr int kThreads = (2 + kEpiWarps) * 32;
 
-static_assert(kStageBytes % 1024 == 0, "stages keep the 1 KB alignment of the swizzled tiles");
+// Tile width kBN (128 or 256 output columns of the packed B, i.e. 64 or 128
+// hidden columns of GEMM1's w1|w3 pairs): B blocks per stage, stages, and
+// TMEM: accumulators from column 0 (two of 128 columns, or one of 256), the
+// scale factors of every stage after them.
+template <int kBN>
+struct Cfg {
+    static constexpr int kBlocks = kBN / 128;
+    static constexpr int kStageBytes = kABytes + kBlocks * kBBlockBytes + kSfaBytes + kBlocks * kSfbBlockBytes;
+    static constexpr int kStages = kBN == 128 ? 6 : 4;
+    static constexpr int kAccBufs = kBN == 128 ? 2 : 1;
+    static constexpr int kSfCols = 4 * (4 + 4 * kBlocks);  // per stage: 4 K steps x (A + B chunks)
+    static constexpr int kSfBase = kAccBufs * kBN;
+    static_assert(kStageBytes % 1024 == 0, "stages keep the 1 KB alignment of the swizzled tiles");
+    static_assert(kSfBase + kStages * kSfCols <= kTmemCols, "TMEM budget");
+};
 
 struct __align__(8) SmemTail {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
-    uint64_t accum_full;
-    uint64_t accum_empty;
+    uint64_t full[6];
+    uint64_t empty[6];
+    uint64_t accum_full[2];
+    uint64_t accum_empty[2];
     uint64_t done;
     uint32_t tmem_base;
     int32_t off[kMaxN + 1];
@@ -61,7 +70,11 @@ struct __align__(8) SmemTail {
 };
 
 constexpr int kTailBytes = (static_cast<int>(sizeof(SmemTail)) + 127) / 128 * 128;
-constexpr int kSmemBytes = kStages * kStageBytes + kTailBytes + 1024;
+
+template <int kBN>
+constexpr int smem_bytes() {
+    return Cfg<kBN>::kStages * Cfg<kBN>::kStageBytes + kTailBytes + 1024;
+}
 
 struct Tile {
     int e, n_tile, m_blk, row0, rows;
@@ -93,33 +106,38 @@ __device__ __forceinline__ float silu(float a) { return __fdividef(a, 1.f + __ex
 
 using namespace w4gemm;
 
-template <bool kSwiGLU>
+// kSwiGLU: GEMM1 over the w1|w3 pair pack (accumulator column j of block
+// j / 128 is w1 for j % 128 < 64, w3 otherwise; hidden column = 64 x block +
+// j % 64); else GEMM2 over w2.
+template <bool kSwiGLU, int kBN>
 __global__ void __launch_bounds__(kThreads, 1)
-    w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
-                     const __grid_constant__ CUtensorMap tm_b1, const W4a4GemmArgs args) {
+    w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                     const W4a4GemmArgs args) {
+    using C = Cfg<kBN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    SmemTail* tail = reinterpret_cast<SmemTail*>(smem + kStages * kStageBytes);
+    SmemTail* tail = reinterpret_cast<SmemTail*>(smem + C::kStages * C::kStageBytes);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int n = args.n;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < C::kStages; ++s) {
             mbar_init(smem_u32(&tail->full[s]), 1);
             mbar_init(smem_u32(&tail->empty[s]), 1);
         }
-        mbar_init(smem_u32(&tail->accum_full), 1);
-        mbar_init(smem_u32(&tail->accum_empty), kEpiWarps);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&tail->accum_full[b]), 1);
+            mbar_init(smem_u32(&tail->accum_empty[b]), kEpiWarps);
+        }
         mbar_init(smem_u32(&tail->done), 1);
         fence_barrier_init();
         fence_proxy_async_smem();
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tm_a);
-        tma_prefetch_desc(&tm_b0);
-        tma_prefetch_desc(&tm_b1);
+        tma_prefetch_desc(&tm_b);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(&tail->tmem_base), kTmemCols);
@@ -143,19 +161,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             // ---------------- TMA producer ----------------
             int stage = 0;
             uint32_t phase = 0;
-            int armed[kStages];
-            for (int s = 0; s < kStages; ++s) armed[s] = -1;
+            int armed[6];
+            for (int s = 0; s < 6; ++s) armed[s] = -1;
             bool ok = true;
+            const int blocks_per_e = args.n_rows_b / 128;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
                 const Tile ti = tile_at(t, tail->off, tail->mblk, n, args.n_tiles);
-                // B rows (output columns) of the two halves and their scale-chunk blocks
-                const int c0 = kSwiGLU ? ti.n_tile * 128 : ti.n_tile * 256;
-                const int c1 = kSwiGLU ? c0 : c0 + 128;
-                const int nb_per_e = args.n_cols / 128;
-                const uint8_t* sfb0 = args.b_chunks0 + (static_cast<int64_t>(ti.e) * nb_per_e + c0 / 128) *
-                                                           kb64_total * 512;
-                const uint8_t* sfb1 = args.b_chunks1 + (static_cast<int64_t>(ti.e) * nb_per_e + c1 / 128) *
-                                                           kb64_total * 512;
+                const int r0 = ti.n_tile * kBN;  // first packed B row of the tile
+                const uint8_t* sfb = args.b_chunks +
+                                     (static_cast<int64_t>(ti.e) * blocks_per_e + r0 / 128) * kb64_total * 512;
                 const uint8_t* sfa =
                     args.a_chunks + (static_cast<int64_t>(tail->mblk[ti.e]) + ti.m_blk) * kb64_total * 512;
                 for (int ks = 0; ks < args.k_steps; ++ks) {
@@ -164,24 +178,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     const uint32_t fb = smem_u32(&tail->full[stage]);
-                    mbar_arrive_expect_tx(fb, kStageBytes);
+                    mbar_arrive_expect_tx(fb, C::kStageBytes);
                     armed[stage] = static_cast<int>(phase);
-                    const uint32_t base = smem_u32(smem + stage * kStageBytes);
+                    const uint32_t base = smem_u32(smem + stage * C::kStageBytes);
+                    const uint32_t sf_smem = base + kABytes + C::kBlocks * kBBlockBytes;
                     const int kx = ks * 128;  // byte column of the codes
-                    tma_load_2d(base, &tm_a, fb, kx, ti.row0);
-                    tma_load_3d(base + kABytes, &tm_b0, fb, kx, c0, ti.e);
-                    tma_load_3d(base + kABytes + kBHalfBytes, &tm_b1, fb, kx, c1, ti.e);
                     const int64_t ck = static_cast<int64_t>(ks) * 4 * 512;
-                    bulk_load(base + kABytes + kBBytes, sfa + ck, kSfaBytes, fb);
-                    bulk_load(base + kABytes + kBBytes + kSfaBytes, sfb0 + ck, kSfbBytes / 2, fb);
-                    bulk_load(base + kABytes + kBBytes + kSfaBytes + kSfbBytes / 2, sfb1 + ck, kSfbBytes / 2, fb);
-                    if (++stage == kStages) {
+                    tma_load_2d(base, &tm_a, fb, kx, ti.row0);
+                    bulk_load(sf_smem, sfa + ck, kSfaBytes, fb);
+#pragma unroll
+                    for (int b = 0; b < C::kBlocks; ++b) {
+                        tma_load_3d(base + kABytes + b * kBBlockBytes, &tm_b, fb, kx, r0 + 128 * b, ti.e);
+                        bulk_load(sf_smem + kSfaBytes + b * kSfbBlockBytes,
+                                  sfb + static_cast<int64_t>(b) * kb64_total * 512 + ck, kSfbBlockBytes, fb);
+                    }
+                    if (++stage == C::kStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
-            for (int s = 0; s < kStages; ++s)
+            for (int s = 0; s < C::kStages; ++s)
                 if (armed[s] >= 0)
                     mbar_wait(smem_u32(&tail->full[s]), static_cast<uint32_t>(armed[s]), status, kStatusTimeoutDrain);
         }
@@ -194,40 +211,44 @@ __global__ void __launch_bounds__(kThreads, 1)
             int local = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++local) {
-                if (!mbar_wait(smem_u32(&tail->accum_empty), (static_cast<uint32_t>(local) & 1u) ^ 1u, status,
-                               kStatusTimeoutAccum)) {
+                const int buf = C::kAccBufs == 2 ? (local & 1) : 0;
+                const uint32_t use = C::kAccBufs == 2 ? static_cast<uint32_t>(local >> 1) : static_cast<uint32_t>(local);
+                if (!mbar_wait(smem_u32(&tail->accum_empty[buf]), (use & 1u) ^ 1u, status, kStatusTimeoutAccum)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
                 for (int ks = 0; ks < args.k_steps; ++ks) {
                     if (!mbar_wait(smem_u32(&tail->full[stage]), phase, status, kStatusTimeoutFull)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t base = smem_u32(smem + stage * kStageBytes);
-                    const uint32_t sfa_smem = base + kABytes + kBBytes;
+                    const uint32_t base = smem_u32(smem + stage * C::kStageBytes);
+                    const uint32_t sfa_smem = base + kABytes + C::kBlocks * kBBlockBytes;
                     const uint32_t sfb_smem = sfa_smem + kSfaBytes;
-                    const uint32_t sf_col = tmem_base + 256 + static_cast<uint32_t>(stage * kSfCols);
+                    const uint32_t sf_col = tmem_base + static_cast<uint32_t>(C::kSfBase + stage * C::kSfCols);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint32_t sfa_t = sf_col + 4 * kk;
-                        const uint32_t sfb_t = sf_col + 16 + 8 * kk;
+                        const uint32_t sfb_t = sf_col + 16 + 4 * C::kBlocks * kk;
                         tc_cp_32x128b_warpx4(sfa_t, make_smem_desc(sfa_smem + kk * 512, 0, 128, 0));
-                        tc_cp_32x128b_warpx4(sfb_t, make_smem_desc(sfb_smem + kk * 512, 0, 128, 0));
-                        tc_cp_32x128b_warpx4(sfb_t + 4, make_smem_desc(sfb_smem + kSfbBytes / 2 + kk * 512, 0, 128, 0));
+#pragma unroll
+                        for (int b = 0; b < C::kBlocks; ++b)
+                            tc_cp_32x128b_warpx4(sfb_t + 4 * b,
+                                                 make_smem_desc(sfb_smem + b * kSfbBlockBytes + kk * 512, 0, 128, 0));
                         const uint64_t adesc = make_smem_desc(base + kk * 32, 16, 1024, 2);
                         const uint64_t bdesc = make_smem_desc(base + kABytes + kk * 32, 16, 1024, 2);
-                        tc_mma_fp4_block16(tmem_base, adesc, bdesc, idesc, sfa_t, sfb_t, (ks | kk) != 0 ? 1u : 0u);
+                        tc_mma_fp4_block16(d_tmem, adesc, bdesc, idesc, sfa_t, sfb_t, (ks | kk) != 0 ? 1u : 0u);
                     }
                     tc_commit(smem_u32(&tail->empty[stage]));
-                    if (++stage == kStages) {
+                    if (++stage == C::kStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
-                if (ok) tc_commit(smem_u32(&tail->accum_full));
+                if (ok) tc_commit(smem_u32(&tail->accum_full[buf]));
             }
             tc_commit(smem_u32(&tail->done));
             mbar_wait(smem_u32(&tail->done), 0, status, kStatusTimeoutDrain);
@@ -240,6 +261,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         int local = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++local) {
             const Tile ti = tile_at(t, tail->off, tail->mblk, n, args.n_tiles);
+            const int buf = C::kAccBufs == 2 ? (local & 1) : 0;
+            const uint32_t use = C::kAccBufs == 2 ? static_cast<uint32_t>(local >> 1) : static_cast<uint32_t>(local);
             const int valid = min(32, ti.rows - quad * 32);
             const bool row_ok = lane < valid;
             const int64_t row_base = static_cast<int64_t>(ti.row0) + quad * 32;
@@ -247,22 +270,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float rs = row_ok ? args.row_scale[row_base + lane] : 0.f;
             const float m0 = __ldg(args.mscale0 + ti.e);
             const float m1 = kSwiGLU ? __ldg(args.mscale1 + ti.e) : 0.f;
-            if (!mbar_wait(smem_u32(&tail->accum_full), static_cast<uint32_t>(local) & 1u, status,
-                           kStatusTimeoutAccum))
-                break;
+            if (!mbar_wait(smem_u32(&tail->accum_full[buf]), use & 1u, status, kStatusTimeoutAccum)) break;
             tc_fence_after();
-            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+            const uint32_t tbase =
+                tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf * kBN);
             uint16_t* out = static_cast<uint16_t*>(args.out);
             const float g0 = m0 * rs;
             if (kSwiGLU) {
                 const float g1 = m1 * rs;
+                // 32-column chunks of hidden columns: chunk q covers block q / 2,
+                // w1 columns 128 (q / 2) + 32 (q % 2) + 0..31 and the w3 ones 64 later
+                constexpr int kChunks = kBN / 64;
 #pragma unroll 1
-                for (int c = 2 * half; c < 2 * half + 2; ++c) {
+                for (int q = half * (kChunks / 2); q < (half + 1) * (kChunks / 2); ++q) {
+                    const int acol = 128 * (q >> 1) + 32 * (q & 1);
                     uint32_t a[32], b[32];
-                    tmem_ld_32x32b_x32(tbase + c * 32, a);
-                    tmem_ld_32x32b_x32(tbase + 128 + c * 32, b);
+                    tmem_ld_32x32b_x32(tbase + acol, a);
+                    tmem_ld_32x32b_x32(tbase + acol + 64, b);
                     tmem_wait_ld();
-                    const int col = ti.n_tile * 128 + c * 32;
+                    const int col = ti.n_tile * (kBN / 2) + 32 * q;
                     if (row_ok && col < args.out_cols) {
                         uint32_t pk[16];
 #pragma unroll
@@ -274,17 +300,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         uint4* dst = reinterpret_cast<uint4*>(out + (row_base + lane) * args.out_cols + col);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                        for (int p = 0; p < 4; ++p)
+                            dst[p] = make_uint4(pk[4 * p], pk[4 * p + 1], pk[4 * p + 2], pk[4 * p + 3]);
                     }
                 }
             } else {
+                constexpr int kChunks = kBN / 32;
 #pragma unroll 1
-                for (int c = 4 * half; c < 4 * half + 4; ++c) {
+                for (int c = half * (kChunks / 2); c < (half + 1) * (kChunks / 2); ++c) {
                     uint32_t a[32];
                     tmem_ld_32x32b_x32(tbase + c * 32, a);
                     tmem_wait_ld();
-                    const int col = ti.n_tile * 256 + c * 32;
+                    const int col = ti.n_tile * kBN + c * 32;
                     if (row_ok && col < args.out_cols) {
                         uint32_t pk[16];
 #pragma unroll
@@ -292,14 +319,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             pk[j] = pack_bf16x2(__uint_as_float(a[2 * j]) * g0, __uint_as_float(a[2 * j + 1]) * g0);
                         uint4* dst = reinterpret_cast<uint4*>(out + (row_base + lane) * args.out_cols + col);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                        for (int p = 0; p < 4; ++p)
+                            dst[p] = make_uint4(pk[4 * p], pk[4 * p + 1], pk[4 * p + 2], pk[4 * p + 3]);
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&tail->accum_empty));
+            if (lane == 0) mbar_arrive(smem_u32(&tail->accum_empty[buf]));
         }
     }
 
@@ -312,29 +339,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <bool kSwiGLU>
-static cudaError_t launch_w4(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1,
-                             const W4a4GemmArgs& a, int num_sms, cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(w4a4_gemm_kernel<kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
+int w4a4_tile_cols(bool wide) { return wide ? 256 : 128; }
+
+template <bool kSwiGLU, int kBN>
+static cudaError_t launch_w4(const CUtensorMap& ta, const CUtensorMap& tb, const W4a4GemmArgs& a, int num_sms,
+                             cudaStream_t st) {
+    constexpr int smem = smem_bytes<kBN>();
+    cudaError_t e = cudaFuncSetAttribute(w4a4_gemm_kernel<kSwiGLU, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem);
     if (e != cudaSuccess) return e;
     const int64_t max_tiles = ((a.R + kBM - 1) / kBM + a.n) * static_cast<int64_t>(a.n_tiles);
     int64_t g = num_sms;
     if (max_tiles < g) g = max_tiles;
     if (g < 1) g = 1;
-    launch_k(w4a4_gemm_kernel<kSwiGLU>, dim3(static_cast<unsigned>(g)), dim3(kThreads), kSmemBytes, st, ta, tb0, tb1,
-             a);
+    launch_k(w4a4_gemm_kernel<kSwiGLU, kBN>, dim3(static_cast<unsigned>(g)), dim3(kThreads), smem, st, ta, tb, a);
     return cudaGetLastError();
 }
 
-cudaError_t launch_w4a4_gemm1(const CUtensorMap& tm_xq, const CUtensorMap& tm_w1, const CUtensorMap& tm_w3,
-                              const W4a4GemmArgs& a, int num_sms, cudaStream_t st) {
-    return launch_w4<true>(tm_xq, tm_w1, tm_w3, a, num_sms, st);
+cudaError_t launch_w4a4_gemm1(const CUtensorMap& tm_xq, const CUtensorMap& tm_w13, const W4a4GemmArgs& a, bool wide,
+                              int num_sms, cudaStream_t st) {
+    return wide ? launch_w4<true, 256>(tm_xq, tm_w13, a, num_sms, st)
+                : launch_w4<true, 128>(tm_xq, tm_w13, a, num_sms, st);
 }
 
-cudaError_t launch_w4a4_gemm2(const CUtensorMap& tm_hq, const CUtensorMap& tm_w2, const W4a4GemmArgs& a, int num_sms,
-                              cudaStream_t st) {
-    return launch_w4<false>(tm_hq, tm_w2, tm_w2, a, num_sms, st);
+cudaError_t launch_w4a4_gemm2(const CUtensorMap& tm_hq, const CUtensorMap& tm_w2, const W4a4GemmArgs& a, bool wide,
+                              int num_sms, cudaStream_t st) {
+    return wide ? launch_w4<false, 256>(tm_hq, tm_w2, a, num_sms, st)
+                : launch_w4<false, 128>(tm_hq, tm_w2, a, num_sms, st);
 }
 
 }  // namespace moe

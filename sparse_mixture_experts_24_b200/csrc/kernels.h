@@ -201,8 +201,11 @@ cudaError_t launch_fp4_gemm2(const CUtensorMap& tm_h, const CUtensorMap& tm_c2, 
 // (one per 16 K) of 128 rows for one 64-wide K step.
 //   pack: codes [n][K][N/2] + scales [n][K/16][N] (moe_quantize_weights_fp4) ->
 //   K-major codes [n][N][K/2] + chunks [n][N/128][K/64][512].  N % 128 == 0.
-cudaError_t launch_w4a4_pack(const uint8_t* codes, const uint8_t* bscale, int n, int K, int N, uint8_t* packed,
-                             uint8_t* chunks, cudaStream_t st);
+//   With codes_pair (w3 next to w1): [n][2N][K/2], 128-row blocks of 64 w1
+//   columns then the same 64 w3 columns; chunks [n][2N/128][K/64][512].
+cudaError_t launch_w4a4_pack(const uint8_t* codes, const uint8_t* bscale, const uint8_t* codes_pair,
+                             const uint8_t* bscale_pair, int n, int K, int N, uint8_t* packed, uint8_t* chunks,
+                             cudaStream_t st);
 //   rows: bf16 rows (row r reads src row row_src[r], or r without row_src) ->
 //   codes [R][K/2], row scales [R], and the chunks of the 128-row GEMM tiles
 //   [tiles][K/64][512] (tile of row r: mblk_base[e] + (r - offsets[e]) / 128).
@@ -219,23 +222,25 @@ struct W4a4GemmArgs {
     int k_steps;           // reduction length / 256
     int n_tiles;
     int out_cols;          // F (GEMM1) or d (GEMM2)
-    int n_cols;            // columns of the weight matrix (F for w1/w3, d for w2)
+    int n_rows_b;          // rows of the packed weight matrix (2F for w1|w3, d for w2)
     void* out;             // bf16 [R][out_cols]
     int* status;
     const float* row_scale;    // [R] activation row scales
     const float* mscale0;      // [n] matrix scales: w1 (GEMM1) / w2 (GEMM2)
     const float* mscale1;      // [n] w3 (GEMM1)
     const uint8_t* a_chunks;   // activation scale chunks [tiles][K/64][512]
-    const uint8_t* b_chunks0;  // weight scale chunks [n][N/128][K/64][512]: w1 / w2
-    const uint8_t* b_chunks1;  // w3 (GEMM1) / w2 (GEMM2)
+    const uint8_t* b_chunks;   // weight scale chunks [n][rows/128][K/64][512] (w1|w3 pairs, or w2)
 };
 
 // tm_a: activation codes [R][K/2] uint8 (128 x 128 boxes, 128-byte swizzle);
-// tm_b*: packed weight codes [n][N][K/2] uint8 (128 x 128 x 1 boxes, same).
-cudaError_t launch_w4a4_gemm1(const CUtensorMap& tm_xq, const CUtensorMap& tm_w1, const CUtensorMap& tm_w3,
-                              const W4a4GemmArgs& a, int num_sms, cudaStream_t st);
-cudaError_t launch_w4a4_gemm2(const CUtensorMap& tm_hq, const CUtensorMap& tm_w2, const W4a4GemmArgs& a, int num_sms,
-                              cudaStream_t st);
+// tm_b: packed weight codes [n][rows][K/2] uint8 (128 x 128 x 1 boxes, same):
+// the w1|w3 pair pack for GEMM1, w2 for GEMM2.  wide: 256-column tiles (one
+// accumulator) instead of 128-column tiles (two accumulators).
+int w4a4_tile_cols(bool wide);
+cudaError_t launch_w4a4_gemm1(const CUtensorMap& tm_xq, const CUtensorMap& tm_w13, const W4a4GemmArgs& a, bool wide,
+                              int num_sms, cudaStream_t st);
+cudaError_t launch_w4a4_gemm2(const CUtensorMap& tm_hq, const CUtensorMap& tm_w2, const W4a4GemmArgs& a, bool wide,
+                              int num_sms, cudaStream_t st);
 
 // E4M3 quantisation (e4m3.cu).  Codes are those of v / scale with the quotient
 // rounded to fp32, then to E4M3 by round-to-nearest-even with saturation to

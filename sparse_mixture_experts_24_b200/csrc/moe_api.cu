@@ -207,8 +207,8 @@ struct moe_handle {
     uint8_t* hc4 = nullptr;
     float* xr4 = nullptr;
     float* hr4 = nullptr;
-    CUtensorMap tm_xq4, tm_hq4, tm_wp4[3];
-    const void* c_wp4[3] = {nullptr, nullptr, nullptr};
+    CUtensorMap tm_xq4, tm_hq4, tm_wp4[2];
+    const void* c_wp4[2] = {nullptr, nullptr};
     // 4-bit experts: maps over the caller's codes and block scales
     CUtensorMap tm_f4[6];  // codes w1, scales w1, codes w3, scales w3, codes w2, scales w2
     const void* c_f4[6] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
@@ -696,32 +696,42 @@ moe_status run_experts_w4a4(moe_handle* h, int64_t T, const void* x, const float
     if (e != cudaSuccess) return cuda_fail(e, "activation quantisation launch");
     h->launches += 1;
     trace_mark(h, 2, st);
-    for (int m = 0; m < 3; ++m) {
-        const uint64_t K = m < 2 ? h->d : h->F, N = m < 2 ? h->F : h->d;
+    // wp[0]: the gate/up pair pack (2 ffn rows of d codes), wp[1]: w2 (d rows of ffn)
+    for (int m = 0; m < 2; ++m) {
+        const uint64_t K = m == 0 ? h->d : h->F, N = m == 0 ? 2 * static_cast<uint64_t>(h->F) : h->d;
         if (wp[m] != h->c_wp4[m]) {
             if (!encode_codes(&h->tm_wp4[m], wp[m], K / 2, N, h->n))
                 return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for packed 4-bit weights");
             h->c_wp4[m] = wp[m];
         }
     }
+    // 256-column tiles (one accumulator) by default: on the Mixtral decode
+    // and prefill shapes and 128 experts of 2048 x 768 they measured faster
+    // than 128-column tiles with two accumulators, which reload A for every
+    // 64 hidden columns.
+    bool wide = true;
+    if (const char* v = getenv("MOE_W4A4_TILE")) {  // 128 or 256 forces a width
+        if (atoi(v) == 128) wide = false;
+        if (atoi(v) == 256) wide = true;
+    }
+    const int bn = moe::w4a4_tile_cols(wide);
     moe::W4a4GemmArgs a1{};
     a1.offsets = h->db.offsets;
     a1.mblk_base = h->db.mblk_base;
     a1.n = h->n;
     a1.R = R;
     a1.k_steps = h->d / 256;
-    a1.n_tiles = h->F / 128;
+    a1.n_tiles = 2 * h->F / bn;
     a1.out_cols = h->F;
-    a1.n_cols = h->F;
+    a1.n_rows_b = 2 * h->F;
     a1.out = h->h;
     a1.status = h->status;
     a1.row_scale = h->xr4;
     a1.mscale0 = ws[0];
     a1.mscale1 = ws[1];
     a1.a_chunks = h->xc4;
-    a1.b_chunks0 = wc[0];
-    a1.b_chunks1 = wc[1];
-    e = moe::launch_w4a4_gemm1(h->tm_xq4, h->tm_wp4[0], h->tm_wp4[1], a1, h->num_sms, st);
+    a1.b_chunks = wc[0];
+    e = moe::launch_w4a4_gemm1(h->tm_xq4, h->tm_wp4[0], a1, wide, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
     e = moe::launch_w4a4_rows(static_cast<const uint16_t*>(h->h), nullptr, R, R, h->F, h->db.offsets,
                               h->db.mblk_base, h->n, h->hq4, h->hc4, h->hr4, h->num_sms, st);
@@ -730,17 +740,16 @@ moe_status run_experts_w4a4(moe_handle* h, int64_t T, const void* x, const float
     trace_mark(h, 3, st);
     moe::W4a4GemmArgs a2 = a1;
     a2.k_steps = h->F / 256;
-    a2.n_tiles = h->d / 256;
+    a2.n_tiles = h->d / bn;
     a2.out_cols = h->d;
-    a2.n_cols = h->d;
+    a2.n_rows_b = h->d;
     a2.out = h->o;
     a2.row_scale = h->hr4;
     a2.mscale0 = ws[2];
     a2.mscale1 = ws[2];
     a2.a_chunks = h->hc4;
-    a2.b_chunks0 = wc[2];
-    a2.b_chunks1 = wc[2];
-    e = moe::launch_w4a4_gemm2(h->tm_hq4, h->tm_wp4[2], a2, h->num_sms, st);
+    a2.b_chunks = wc[1];
+    e = moe::launch_w4a4_gemm2(h->tm_hq4, h->tm_wp4[1], a2, wide, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
     h->launches += 1;
     trace_mark(h, 4, st);
@@ -1087,12 +1096,19 @@ moe_status moe_forward_fp4(moe_handle* h, int64_t T, const void* x, const float*
 }
 
 moe_status moe_pack_weights_w4a4(int n, int rows, int cols, const uint8_t* codes, const uint8_t* block_scales,
-                                  uint8_t* packed_codes, uint8_t* scale_chunks, moe_stream_t stream) {
+                                  const uint8_t* pair_codes, const uint8_t* pair_block_scales, uint8_t* packed_codes,
+                                  uint8_t* scale_chunks, moe_stream_t stream) {
     if (n < 1 || n > 65535) return fail(MOE_ERR_INVALID_ARG, "n = %d outside [1, 65535]", n);
     if (rows < 64 || rows % 64 != 0 || rows > 1048576)
         return fail(MOE_ERR_INVALID_ARG, "rows = %d is not a multiple of 64 in [64, 1048576]", rows);
-    if (cols < 128 || cols % 128 != 0)
-        return fail(MOE_ERR_INVALID_ARG, "cols = %d is not a positive multiple of 128", cols);
+    if (pair_codes) {
+        if (cols < 64 || cols % 64 != 0 || cols > 1048576)
+            return fail(MOE_ERR_INVALID_ARG, "cols = %d is not a multiple of 64 in [64, 1048576]", cols);
+    } else if (cols < 128 || cols % 128 != 0 || cols > 1048576) {
+        return fail(MOE_ERR_INVALID_ARG, "cols = %d is not a multiple of 128 in [128, 1048576]", cols);
+    }
+    if ((pair_codes == nullptr) != (pair_block_scales == nullptr))
+        return fail(MOE_ERR_INVALID_ARG, "pair_codes and pair_block_scales must both be given or both be null");
     REQUIRE_PTR(codes);
     REQUIRE_PTR(block_scales);
     REQUIRE_PTR(packed_codes);
@@ -1102,17 +1118,17 @@ moe_status moe_pack_weights_w4a4(int n, int rows, int cols, const uint8_t* codes
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
     if (major != 10) return fail(MOE_ERR_UNSUPPORTED, "device %d is not sm_100", dev);
-    e = moe::launch_w4a4_pack(codes, block_scales, n, rows, cols, packed_codes, scale_chunks,
-                              reinterpret_cast<cudaStream_t>(stream));
+    e = moe::launch_w4a4_pack(codes, block_scales, pair_codes, pair_block_scales, n, rows, cols, packed_codes,
+                              scale_chunks, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "4-bit weight packing launch");
     return ok();
 }
 
-moe_status moe_forward_w4a4(moe_handle* h, int64_t T, const void* x, const float* W_g, const uint8_t* w1_packed,
-                            const uint8_t* w1_chunks, const float* w1_matrix_scales, const uint8_t* w3_packed,
-                            const uint8_t* w3_chunks, const float* w3_matrix_scales, const uint8_t* w2_packed,
-                            const uint8_t* w2_chunks, const float* w2_matrix_scales, void* y, int32_t* topk_idx,
-                            float* topk_w, moe_stream_t stream) {
+moe_status moe_forward_w4a4(moe_handle* h, int64_t T, const void* x, const float* W_g, const uint8_t* w13_packed,
+                            const uint8_t* w13_chunks, const float* w1_matrix_scales,
+                            const float* w3_matrix_scales, const uint8_t* w2_packed, const uint8_t* w2_chunks,
+                            const float* w2_matrix_scales, void* y, int32_t* topk_idx, float* topk_w,
+                            moe_stream_t stream) {
     moe_status s = check_common(h, T);
     if (s != MOE_OK) return s;
     if (h->dtype != MOE_BF16)
@@ -1122,11 +1138,9 @@ moe_status moe_forward_w4a4(moe_handle* h, int64_t T, const void* x, const float
     if (T == 0) return ok();
     REQUIRE_PTR(x);
     REQUIRE_PTR(W_g);
-    REQUIRE_PTR(w1_packed);
-    REQUIRE_PTR(w1_chunks);
+    REQUIRE_PTR(w13_packed);
+    REQUIRE_PTR(w13_chunks);
     REQUIRE_PTR(w1_matrix_scales);
-    REQUIRE_PTR(w3_packed);
-    REQUIRE_PTR(w3_chunks);
     REQUIRE_PTR(w3_matrix_scales);
     REQUIRE_PTR(w2_packed);
     REQUIRE_PTR(w2_chunks);
@@ -1143,8 +1157,8 @@ moe_status moe_forward_w4a4(moe_handle* h, int64_t T, const void* x, const float
     s = run_router(h, T, x, W_g, topk_idx, topk_w, st);
     if (s != MOE_OK) return s;
     trace_mark(h, 0, st);
-    const uint8_t* wp[3] = {w1_packed, w3_packed, w2_packed};
-    const uint8_t* wc[3] = {w1_chunks, w3_chunks, w2_chunks};
+    const uint8_t* wp[2] = {w13_packed, w2_packed};
+    const uint8_t* wc[2] = {w13_chunks, w2_chunks};
     const float* ws[3] = {w1_matrix_scales, w3_matrix_scales, w2_matrix_scales};
     s = run_experts_w4a4(h, T, x, topk_w, wp, wc, ws, y, topk_idx, st);
     return s == MOE_OK ? ok() : s;

@@ -11,6 +11,10 @@
 //   w4a4_pack_kernel   4-bit weights in the layout of moe_quantize_weights_fp4
 //                      (codes [n][K][N/2], scales [n][K/16][N]) -> K-major codes
 //                      [n][N][K/2] and scale chunks [n][N/128][K/64][512].
+//                      Pair mode (w1 and w3): the packed matrix has 2N rows,
+//                      each 128-row block holding 64 columns of w1 followed by
+//                      the same 64 columns of w3, so one 128-row tile of it
+//                      yields both projections of 64 hidden columns.
 //   w4a4_rows_kernel   rows (gathered x rows or hidden rows, bf16) -> E2M1 codes
 //                      [R][K/2], a fp32 scale per row, and the scale chunks of
 //                      the GEMM's 128-row tiles: row r of expert e's segment
@@ -28,16 +32,31 @@ namespace moe {
 
 __device__ __forceinline__ int w4_chunk_byte(int r, int s) { return 16 * (r & 31) + 4 * ((r & 127) >> 5) + s; }
 
-// Thread = (matrix e, column c, 16 K-rows kb16): 8 packed bytes and 1 scale.
-__global__ void __launch_bounds__(256) w4a4_pack_kernel(const uint8_t* __restrict__ codes,
-                                                        const uint8_t* __restrict__ bscale, int K, int N,
-                                                        uint8_t* __restrict__ packed, uint8_t* __restrict__ chunks) {
+// Thread = (matrix e, packed row c, 16 K-rows kb16): 8 packed bytes and 1
+// scale.  Packed row c reads column c of matrix 0, or in pair mode column
+// 64 (c / 128) + c % 64 of matrix (c % 128) / 64.
+__global__ void __launch_bounds__(256) w4a4_pack_kernel(const uint8_t* __restrict__ codes0,
+                                                        const uint8_t* __restrict__ bscale0,
+                                                        const uint8_t* __restrict__ codes1,
+                                                        const uint8_t* __restrict__ bscale1, int K, int N,
+                                                        int rows_out, uint8_t* __restrict__ packed,
+                                                        uint8_t* __restrict__ chunks) {
     const int e = blockIdx.z;
     const int c = blockIdx.x * blockDim.x + threadIdx.x;
     const int kb16 = blockIdx.y;
-    if (c >= N) return;
-    const int64_t in_base = (static_cast<int64_t>(e) * K + kb16 * 16) * (N / 2) + c / 2;
-    const int sh = 4 * (c & 1);
+    if (c >= rows_out) return;
+    int col = c;
+    const uint8_t* codes = codes0;
+    const uint8_t* bscale = bscale0;
+    if (codes1) {
+        col = 64 * (c >> 7) + (c & 63);
+        if (c & 64) {
+            codes = codes1;
+            bscale = bscale1;
+        }
+    }
+    const int64_t in_base = (static_cast<int64_t>(e) * K + kb16 * 16) * (N / 2) + col / 2;
+    const int sh = 4 * (col & 1);
     uint32_t lo = 0, hi = 0;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -47,17 +66,21 @@ __global__ void __launch_bounds__(256) w4a4_pack_kernel(const uint8_t* __restric
         else
             hi |= nib << (4 * (i - 8));
     }
-    uint2* dst = reinterpret_cast<uint2*>(packed + (static_cast<int64_t>(e) * N + c) * (K / 2) + kb16 * 8);
+    uint2* dst = reinterpret_cast<uint2*>(packed + (static_cast<int64_t>(e) * rows_out + c) * (K / 2) + kb16 * 8);
     *dst = make_uint2(lo, hi);
     const int KB = K / 64;
-    const int64_t chunk = (static_cast<int64_t>(e) * (N / 128) + c / 128) * KB + kb16 / 4;
-    chunks[chunk * 512 + w4_chunk_byte(c, kb16 & 3)] = __ldg(bscale + (static_cast<int64_t>(e) * (K / 16) + kb16) * N + c);
+    const int64_t chunk = (static_cast<int64_t>(e) * (rows_out / 128) + c / 128) * KB + kb16 / 4;
+    chunks[chunk * 512 + w4_chunk_byte(c, kb16 & 3)] =
+        __ldg(bscale + (static_cast<int64_t>(e) * (K / 16) + kb16) * N + col);
 }
 
-cudaError_t launch_w4a4_pack(const uint8_t* codes, const uint8_t* bscale, int n, int K, int N, uint8_t* packed,
-                             uint8_t* chunks, cudaStream_t st) {
-    const dim3 grid(static_cast<unsigned>((N + 255) / 256), static_cast<unsigned>(K / 16), static_cast<unsigned>(n));
-    w4a4_pack_kernel<<<grid, 256, 0, st>>>(codes, bscale, K, N, packed, chunks);
+cudaError_t launch_w4a4_pack(const uint8_t* codes, const uint8_t* bscale, const uint8_t* codes_pair,
+                             const uint8_t* bscale_pair, int n, int K, int N, uint8_t* packed, uint8_t* chunks,
+                             cudaStream_t st) {
+    const int rows_out = codes_pair ? 2 * N : N;
+    const dim3 grid(static_cast<unsigned>((rows_out + 255) / 256), static_cast<unsigned>(K / 16),
+                    static_cast<unsigned>(n));
+    w4a4_pack_kernel<<<grid, 256, 0, st>>>(codes, bscale, codes_pair, bscale_pair, K, N, rows_out, packed, chunks);
     return cudaGetLastError();
 }
 

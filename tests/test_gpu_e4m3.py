@@ -245,3 +245,27 @@ def test_e4m3_full_size_decode():
     y_ref = oracle.forward_e4m3(L["x"][pick], o_idx[pick], o_gate[pick], *q)
     err = rel_l2(y_as_f64(y)[pick], y_ref)
     assert err <= TOL_Y["bf16"], err
+
+
+def test_e4m3_many_rows_sampled():
+    """20,000 tokens over 16 experts, compared on a token sample."""
+    import sparse_mixture_experts_24_b200 as m
+    torch = require_cuda()
+    name, T, d, F, n, K = "e4m3_many_rows", 20000, 256, 320, 16, 2
+    cfg = mi.custom_config(name, T=T, d=d, ffn=F, n=n, K=K, dtype="bf16")
+    L = mi.make_layer(cfg, seed=seed_of(name))
+    q = oracle_codes(L)
+    layer = m.MoELayer(n, K, d, F, "bf16")
+    try:
+        y, idx, w = layer.forward_e4m3(dev(L["x"]), dev(L["W_g"]), *[dev(a) for a in q])
+        layer.sync_status()
+        torch.cuda.synchronize()
+        y, idx, w = host(y), host(idx), host(w)
+    finally:
+        layer.close()
+    o_idx, o_gate, o_logits = oracle.router(L["x"], L["W_g"], K)
+    compare_routing(idx, w, o_idx, o_gate, o_logits, L["x"], L["W_g"], K)
+    pick = stratified_sample(o_idx, n, 300)
+    pick = pick[(idx[pick] == o_idx[pick]).all(axis=1)]
+    y_ref = oracle.forward_e4m3(L["x"][pick], o_idx[pick], o_gate[pick], *q)
+    assert rel_l2(y_as_f64(y)[pick], y_ref) <= TOL_Y["bf16"]

@@ -22,19 +22,34 @@ def seed_of(name: str) -> int:
     return zlib.crc32(name.encode()) % 1000
 
 
-def numpy_pack(codes, bscale):
-    """The documented layout of moe_pack_weights_w4a4, written with numpy."""
+def numpy_pack(codes, bscale, pair=None):
+    """The documented layout of moe_pack_weights_w4a4, written with numpy:
+    the single matrix, or with pair = (codes, bscale) of w3 the gate/up pair
+    whose packed column p is column 64 (p // 128) + p % 64 of w1 (p % 128 < 64)
+    or of w3."""
     n, K, half = codes.shape
     N = 2 * half
-    nib = np.empty((n, K, N), np.uint8)
-    nib[:, :, 0::2], nib[:, :, 1::2] = codes & 0xF, codes >> 4
+
+    def nibbles(c):
+        nib = np.empty((n, K, N), np.uint8)
+        nib[:, :, 0::2], nib[:, :, 1::2] = c & 0xF, c >> 4
+        return nib
+
+    nib, bs = nibbles(codes), bscale
+    if pair is not None:
+        p = np.arange(2 * N)
+        col = 64 * (p // 128) + p % 64
+        from_w3 = (p % 128) >= 64
+        nib = np.where(from_w3[None, None, :], nibbles(pair[0])[:, :, col], nib[:, :, col])
+        bs = np.where(from_w3[None, None, :], pair[1][:, :, col], bscale[:, :, col])
+        N = 2 * N
     kmaj = nib.transpose(0, 2, 1)                                   # [n][N][K]
     packed = (kmaj[:, :, 0::2] | (kmaj[:, :, 1::2] << 4)).astype(np.uint8)
     chunks = np.zeros((n, N // 128, K // 64, 512), np.uint8)
     c = np.arange(N)
     pos = 16 * (c % 32) + 4 * ((c % 128) // 32)
     for kb16 in range(K // 16):
-        chunks[:, c // 128, kb16 // 4, pos + kb16 % 4] = bscale[:, kb16, :]
+        chunks[:, c // 128, kb16 // 4, pos + kb16 % 4] = bs[:, kb16, :]
     return packed, chunks
 
 
@@ -53,12 +68,42 @@ def test_pack_is_the_documented_permutation(shape):
     assert np.array_equal(host(chunks), c_ref)
 
 
+@pytest.mark.parametrize("shape", [(2, 64, 64), (3, 256, 192), (1, 128, 512)])
+def test_pair_pack_is_the_documented_permutation(shape):
+    import sparse_mixture_experts_24_b200 as m
+    torch = require_cuda()
+    n, K, N = shape
+    rng = np.random.default_rng(7 * K + N)
+    c1, c3 = (rng.integers(0, 256, (n, K, N // 2), dtype=np.uint8) for _ in range(2))
+    b1, b3 = (rng.integers(0, 0x7F, (n, K // 16, N), dtype=np.uint8) for _ in range(2))
+    packed, chunks, _, _ = m.pack_weights_w4a4(dev(c1), dev(b1), None, pair=(dev(c3), dev(b3), None))
+    torch.cuda.synchronize()
+    p_ref, c_ref = numpy_pack(c1, b1, pair=(c3, b3))
+    assert np.array_equal(host(packed), p_ref)
+    assert np.array_equal(host(chunks), c_ref)
+
+
+def test_pack_rejects_bad_sizes():
+    import sparse_mixture_experts_24_b200 as m
+    torch = require_cuda()
+    z = torch.zeros(1 << 16, dtype=torch.uint8, device="cuda")
+    for rows, cols, pair in ((64, 64, False), (32, 128, False), (64, 96, True)):
+        with pytest.raises(m.MoEError) as ei:
+            m.moe_pack_weights_w4a4(1, rows, cols, z, z, z if pair else None, z if pair else None, z, z)
+        assert ei.value.status == m.MOE_ERR_INVALID_ARG
+    with pytest.raises(m.MoEError) as ei:                  # one pair pointer alone
+        m.moe_pack_weights_w4a4(1, 64, 128, z, z, z, None, z, z)
+    assert ei.value.status == m.MOE_ERR_INVALID_ARG
+
+
 def prepared_weights(L):
-    """Oracle 4-bit weights (logical layout) and their packed device form."""
+    """Oracle 4-bit weights (logical layout) and their packed device form:
+    the gate/up pair pack and w2."""
     import sparse_mixture_experts_24_b200 as m
     q = [oracle.quantize_weights_fp4(L[w]) for w in ("w1", "w3", "w2")]
-    packed = [m.pack_weights_w4a4(dev(c), dev(b), dev(t)) for c, b, t in q]
-    return q, packed
+    w13 = m.pack_weights_w4a4(*(dev(a) for a in q[0]), pair=tuple(dev(a) for a in q[1]))
+    w2 = m.pack_weights_w4a4(*(dev(a) for a in q[2]))
+    return q, (w13, w2)
 
 
 FWD_CASES = [
@@ -71,10 +116,14 @@ FWD_CASES = [
 ]
 
 
+@pytest.mark.parametrize("tile", ["128", "256"])
 @pytest.mark.parametrize("case", FWD_CASES, ids=[c[0] for c in FWD_CASES])
-def test_w4a4_layer_matches_oracle(case):
+def test_w4a4_layer_matches_oracle(case, tile, monkeypatch):
+    """Both tile widths (128 packed columns with two accumulators, 256 with
+    one) on every case."""
     import sparse_mixture_experts_24_b200 as m
     torch = require_cuda()
+    monkeypatch.setenv("MOE_W4A4_TILE", tile)
     name, T, d, F, n, K = case
     cfg = mi.custom_config(name, T=T, d=d, ffn=F, n=n, K=K, dtype="bf16")
     L = mi.make_layer(cfg, seed=seed_of(name))
@@ -134,7 +183,7 @@ def test_w4a4_capacity_and_rejections():
             x = torch.zeros((4, args[2]), dtype=torch.bfloat16 if args[4] == "bf16" else torch.float32,
                             device="cuda")
             with pytest.raises(m.MoEError) as ei:
-                layer.forward_w4a4(x, x, (x, x, x), (x, x, x), (x, x, x))
+                layer.forward_w4a4(x, x, (x, x, x, x), (x, x, x))
             assert ei.value.status == m.MOE_ERR_UNSUPPORTED
         finally:
             layer.close()
@@ -159,6 +208,31 @@ def test_w4a4_full_size_decode():
     o_idx, o_gate, o_logits = oracle.router(L["x"], L["W_g"], cfg.K)
     compare_routing(idx, w, o_idx, o_gate, o_logits, L["x"], L["W_g"], cfg.K)
     pick = stratified_sample(o_idx, cfg.n, 12)
+    pick = pick[(idx[pick] == o_idx[pick]).all(axis=1)]
+    y_ref = oracle.forward_w4a4(L["x"][pick], o_idx[pick], o_gate[pick], *q)
+    assert rel_l2(y_as_f64(y)[pick], y_ref) <= TOL_Y["bf16"]
+
+
+def test_w4a4_many_rows_sampled():
+    """20,000 tokens over 16 experts (hundreds of 128-row tiles, scale chunks
+    far into the workspace), compared on a token sample."""
+    import sparse_mixture_experts_24_b200 as m
+    torch = require_cuda()
+    name, T, d, F, n, K = "w4a4_many_rows", 20000, 256, 512, 16, 2
+    cfg = mi.custom_config(name, T=T, d=d, ffn=F, n=n, K=K, dtype="bf16")
+    L = mi.make_layer(cfg, seed=seed_of(name))
+    q, packed = prepared_weights(L)
+    layer = m.MoELayer(n, K, d, F, "bf16")
+    try:
+        y, idx, w = layer.forward_w4a4(dev(L["x"]), dev(L["W_g"]), *packed)
+        layer.sync_status()
+        torch.cuda.synchronize()
+        y, idx, w = host(y), host(idx), host(w)
+    finally:
+        layer.close()
+    o_idx, o_gate, o_logits = oracle.router(L["x"], L["W_g"], K)
+    compare_routing(idx, w, o_idx, o_gate, o_logits, L["x"], L["W_g"], K)
+    pick = stratified_sample(o_idx, n, 300)
     pick = pick[(idx[pick] == o_idx[pick]).all(axis=1)]
     y_ref = oracle.forward_w4a4(L["x"][pick], o_idx[pick], o_gate[pick], *q)
     assert rel_l2(y_as_f64(y)[pick], y_ref) <= TOL_Y["bf16"]
