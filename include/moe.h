@@ -353,6 +353,86 @@ MOE_API moe_status moe_forward_w4a4(moe_handle *h, int64_t T, const void *x, con
                                     moe_stream_t stream);
 
 /*
+ * Expert parallelism over `world` ranks (1 <= world <= 16, world divides n):
+ * rank q holds the weights of experts [q*n/world, (q+1)*n/world) and routes
+ * its own tokens.  The flash-card page on "Mixtral of Experts" names this
+ * placement (section 2.1: experts on different GPUs, uneven routing
+ * overloading some of them; section 5: temporal locality); the pages give
+ * no mechanics, so the exchange below is this library's design.  The two
+ * all-to-all exchanges are fused into the kernels around them: the dispatch
+ * STORES each routed x row into its expert owner's receive buffer, and the
+ * combine LOADS each expert output row from its owner's output buffer.  Peer
+ * buffers are device pointers the calling process can dereference (another
+ * GPU's memory mapped through CUDA IPC with peer access, or, for ranks
+ * emulated on one GPU, plain device memory).  Expert parallelism is dropless
+ * (MOE_ERR_UNSUPPORTED while a capacity factor is set) and needs a MOE_BF16
+ * handle created with the GLOBAL n.  One layer step on every rank:
+ *   1. moe_route, then moe_dispatch(..., counts, ...) for this rank's counts[n];
+ *   2. counts_all[world][n] = every rank's counts (row q = rank q's), on the
+ *      device of every rank (e.g. an all-gather);
+ *   3. moe_ep_dispatch;  4. a barrier across ranks;
+ *   5. moe_ep_experts;   6. a barrier across ranks;   7. moe_ep_combine.
+ * Receive layout on an owner: its experts in order; inside an expert the rows
+ * of rank 0, then rank 1, ...; inside a rank its (token, slot) pairs of that
+ * expert in token order.  An owner receives sum over ranks and over its
+ * experts of counts_all rows; recv_rows (the rows every receive buffer holds,
+ * the same on all ranks) must cover that, else moe_sync_status reports
+ * MOE_ERR_INVALID_ARG and nothing is stored.  The y of a token is computed as
+ * moe_forward_with_routing computes it (same kernels, same order), so with the
+ * same routing the two agree bit for bit.
+ *
+ * moe_ep_dispatch: x [T][d], topk_idx [T][K] of this rank (device);
+ * counts_all [world][n] int32 (device); recv_buffers: host array of `world`
+ * device pointers, entry q = rank q's receive buffer [recv_rows][d] bf16;
+ * row_pos [T][K] int32 (device, written): the row of each (token, slot) pair
+ * inside its owner's buffer.  Also checks counts_all's row `rank` against
+ * this rank's routing.
+ */
+MOE_API moe_status moe_ep_dispatch(moe_handle *h, int world, int rank, int64_t T, const void *x,
+                                   const int32_t *topk_idx, const int32_t *counts_all,
+                                   void *const *recv_buffers, int64_t recv_rows, int32_t *row_pos,
+                                   moe_stream_t stream);
+
+/*
+ * moe_ep_experts: the grouped SwiGLU experts of rank `rank` over its receive
+ * buffer recv [recv_rows][d] (filled by every rank's moe_ep_dispatch), with
+ * its local weights w1, w3 [n/world][d][ffn] and w2 [n/world][ffn][d] (bf16);
+ * out [recv_rows][d] bf16 receives the expert output of every received row,
+ * in the receive layout.  The workspace grows to recv_rows rows.
+ */
+MOE_API moe_status moe_ep_experts(moe_handle *h, int world, int rank, const int32_t *counts_all,
+                                  const void *recv, int64_t recv_rows, const void *w1, const void *w3,
+                                  const void *w2, void *out, moe_stream_t stream);
+
+/*
+ * moe_ep_combine: y[t] = sum_k topk_w[t][k] * out_{owner}[row_pos[t][k]],
+ * fp32 in slot order, rounded to bf16; out_buffers: host array of `world`
+ * device pointers, entry q = rank q's `out` of moe_ep_experts.  Pairs with
+ * row_pos < 0 add nothing.
+ *   Errors (all three): MOE_ERR_INVALID_ARG (world, rank, n not divisible,
+ *   null / misaligned pointer, recv_rows outside [1, 2^31 - 1]);
+ *   MOE_ERR_UNSUPPORTED (fp32 handle, capacity factor set); MOE_ERR_CUDA.
+ */
+MOE_API moe_status moe_ep_combine(moe_handle *h, int world, int64_t T, const int32_t *topk_idx,
+                                  const float *topk_w, const int32_t *row_pos, const void *const *out_buffers,
+                                  void *y, moe_stream_t stream);
+
+/*
+ * Buffers that other ranks' kernels read or write (the receive and output
+ * buffers of expert parallelism): moe_ep_buffer_alloc allocates `bytes` of
+ * device memory on the current device (cudaMalloc: the base of its own
+ * allocation) and, when ipc_handle is not NULL, writes its 64-byte CUDA IPC
+ * handle there for the other processes; moe_ep_buffer_open maps another
+ * process's buffer from its handle (peer access enabled); moe_ep_buffer_close
+ * releases one (opened = 1 for a mapped peer buffer, 0 for an own buffer).
+ *   Errors: MOE_ERR_INVALID_ARG (null pointers, bytes < 1), MOE_ERR_ALLOC,
+ *   MOE_ERR_CUDA.
+ */
+MOE_API moe_status moe_ep_buffer_alloc(int64_t bytes, void **ptr, uint8_t *ipc_handle);
+MOE_API moe_status moe_ep_buffer_open(const uint8_t *ipc_handle, void **ptr);
+MOE_API moe_status moe_ep_buffer_close(void *ptr, int opened);
+
+/*
  * Debug view of the workspace written by the last forward call: name is "H"
  * (expert hidden layer, [rows][ffn], handle dtype) or "O" (per-row expert
  * outputs, [rows][d], handle dtype for bf16 handles, fp32 for fp32 handles);

@@ -68,6 +68,12 @@ lib.moe_quantize_weights_fp4.argtypes = [_int, _int, _int, _vp, _int, _vp, _vp, 
 lib.moe_forward_fp4.argtypes = [_vp, _i64, _vp, _vp] + [_vp] * 9 + [_vp, _vp, _vp, _vp]
 lib.moe_pack_weights_w4a4.argtypes = [_int, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.moe_forward_w4a4.argtypes = [_vp, _i64, _vp, _vp] + [_vp] * 7 + [_vp, _vp, _vp, _vp]
+lib.moe_ep_dispatch.argtypes = [_vp, _int, _int, _i64, _vp, _vp, _vp, _vp, _i64, _vp, _vp]
+lib.moe_ep_experts.argtypes = [_vp, _int, _int, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp]
+lib.moe_ep_combine.argtypes = [_vp, _int, _i64, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.moe_ep_buffer_alloc.argtypes = [_i64, ctypes.POINTER(_vp), _vp]
+lib.moe_ep_buffer_open.argtypes = [_vp, ctypes.POINTER(_vp)]
+lib.moe_ep_buffer_close.argtypes = [_vp, _int]
 lib.moe_last_error.restype = ctypes.c_char_p
 lib.moe_version.restype = ctypes.c_char_p
 for _f in ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
@@ -75,7 +81,9 @@ for _f in ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatc
            "moe_trace_begin", "moe_trace_end", "moe_dispatch_noalloc", "moe_set_capacity_factor",
            "moe_router_stats", "moe_launch_count", "moe_selftest_timeout",
            "moe_forward_expert_choice", "moe_quantize_weights_e4m3", "moe_forward_e4m3",
-           "moe_quantize_weights_fp4", "moe_forward_fp4", "moe_pack_weights_w4a4", "moe_forward_w4a4"):
+           "moe_quantize_weights_fp4", "moe_forward_fp4", "moe_pack_weights_w4a4", "moe_forward_w4a4",
+           "moe_ep_dispatch", "moe_ep_experts", "moe_ep_combine", "moe_ep_buffer_alloc", "moe_ep_buffer_open",
+           "moe_ep_buffer_close"):
     getattr(lib, _f).restype = _int
 
 EXPORTED = ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
@@ -84,7 +92,8 @@ EXPORTED = ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispat
             "moe_dispatch_noalloc", "moe_set_capacity_factor", "moe_router_stats",
             "moe_launch_count", "moe_selftest_timeout", "moe_forward_expert_choice",
             "moe_quantize_weights_e4m3", "moe_forward_e4m3", "moe_quantize_weights_fp4", "moe_forward_fp4",
-            "moe_pack_weights_w4a4", "moe_forward_w4a4")
+            "moe_pack_weights_w4a4", "moe_forward_w4a4", "moe_ep_dispatch", "moe_ep_experts", "moe_ep_combine",
+            "moe_ep_buffer_alloc", "moe_ep_buffer_open", "moe_ep_buffer_close")
 
 TRACE_STAGES = ("router", "dispatch", "gather", "gemm1", "gemm2", "combine")
 
@@ -295,6 +304,47 @@ def pack_weights_w4a4(codes, block_scales, matrix_scales, pair=None, stream=None
     if pair is not None:
         return packed, chunks, matrix_scales, pair[2]
     return packed, chunks, matrix_scales
+
+
+def _ptr_table(ptrs):
+    """Host array of device addresses (tensors, ints) for the peer tables."""
+    return (ctypes.c_void_p * len(ptrs))(*[_ptr(p) for p in ptrs])
+
+
+def moe_ep_dispatch(h, world, rank, T, x, topk_idx, counts_all, recv_buffers, recv_rows, row_pos,
+                    stream=None) -> None:
+    _check(lib.moe_ep_dispatch(h, world, rank, T, _ptr(x), _ptr(topk_idx), _ptr(counts_all),
+                               _ptr_table(recv_buffers), recv_rows, _ptr(row_pos), _stream(stream)),
+           "moe_ep_dispatch")
+
+
+def moe_ep_experts(h, world, rank, counts_all, recv, recv_rows, w1, w3, w2, out, stream=None) -> None:
+    _check(lib.moe_ep_experts(h, world, rank, _ptr(counts_all), _ptr(recv), recv_rows, _ptr(w1), _ptr(w3),
+                              _ptr(w2), _ptr(out), _stream(stream)), "moe_ep_experts")
+
+
+def moe_ep_combine(h, world, T, topk_idx, topk_w, row_pos, out_buffers, y, stream=None) -> None:
+    _check(lib.moe_ep_combine(h, world, T, _ptr(topk_idx), _ptr(topk_w), _ptr(row_pos),
+                              _ptr_table(out_buffers), _ptr(y), _stream(stream)), "moe_ep_combine")
+
+
+def moe_ep_buffer_alloc(nbytes: int, with_ipc_handle: bool = True):
+    """-> (device address, 64-byte IPC handle or None)."""
+    p = ctypes.c_void_p()
+    hd = ctypes.create_string_buffer(64) if with_ipc_handle else None
+    _check(lib.moe_ep_buffer_alloc(nbytes, ctypes.byref(p), hd), "moe_ep_buffer_alloc")
+    return p.value, (hd.raw if hd is not None else None)
+
+
+def moe_ep_buffer_open(handle: bytes) -> int:
+    p = ctypes.c_void_p()
+    buf = ctypes.create_string_buffer(bytes(handle), 64)
+    _check(lib.moe_ep_buffer_open(buf, ctypes.byref(p)), "moe_ep_buffer_open")
+    return p.value
+
+
+def moe_ep_buffer_close(ptr: int, opened: bool) -> None:
+    _check(lib.moe_ep_buffer_close(ptr, 1 if opened else 0), "moe_ep_buffer_close")
 
 
 def moe_destroy(h) -> None:

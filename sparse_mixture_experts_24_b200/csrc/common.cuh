@@ -8,17 +8,10 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "kernels.h"
+
 namespace moe {
 
-// Bits of the device status word (workspace): set by a kernel that gave up a
-// bounded wait, read and cleared by moe_sync_status.
-enum : int {
-    kStatusTimeoutFull = 1,      // waited too long for a TMA stage to land
-    kStatusTimeoutEmpty = 2,     // waited too long for the MMA to free a stage
-    kStatusTimeoutAccum = 4,     // waited too long for an accumulator buffer
-    kStatusTimeoutDrain = 8,     // waited too long while draining at exit
-    kStatusSelfTest = 16,        // the self-test's wait ran out (as it should)
-};
 
 // About 2 s at the B200's 1.9 GHz: far beyond any legitimate wait in these
 // kernels, short enough that a broken pipeline returns instead of hanging.
@@ -117,6 +110,33 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
         : "memory");
+}
+
+// Exclusive scan of one value per thread over a 256-thread block.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = (lane < 8) ? s_warp[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += u;
+        }
+        if (lane < 8) s_warp[lane] = wi - w;  // exclusive warp bases
+    }
+    __syncthreads();
+    const int r = s_warp[warp] + incl - v;
+    __syncthreads();
+    return r;
 }
 
 // ---------------------------------------------------------------------------

@@ -63,33 +63,6 @@ __global__ void __launch_bounds__(kPairsPerBlock) rank_kernel(const int32_t* __r
     griddep_launch_dependents();
 }
 
-// Exclusive scan of one value per thread over a 256-thread block.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += u;
-    }
-    if (lane == 31) s_warp[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        int w = (lane < 8) ? s_warp[lane] : 0;
-        int wi = w;
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) {
-            const int u = __shfl_up_sync(0xffffffffu, wi, o);
-            if (lane >= o) wi += u;
-        }
-        if (lane < 8) s_warp[lane] = wi - w;  // exclusive warp bases
-    }
-    __syncthreads();
-    const int r = s_warp[warp] + incl - v;
-    __syncthreads();
-    return r;
-}
-
 // Per-block counts are walked in chunks staged through shared memory, so
 // the loads of a chunk are all in flight together; each expert's column is
 // then scanned in place.  blockcounts ends up holding, for every block and

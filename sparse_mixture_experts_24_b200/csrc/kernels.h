@@ -33,6 +33,17 @@ inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
 }
 
 // Rows of one M-block of the tensor-core GEMMs and of the CUDA-core GEMMs.
+// Bits of the device status word (workspace): set by a kernel that gave up a
+// bounded wait, read and cleared by moe_sync_status.
+enum : int {
+    kStatusTimeoutFull = 1,      // waited too long for a TMA stage to land
+    kStatusTimeoutEmpty = 2,     // waited too long for the MMA to free a stage
+    kStatusTimeoutAccum = 4,     // waited too long for an accumulator buffer
+    kStatusTimeoutDrain = 8,     // waited too long while draining at exit
+    kStatusSelfTest = 16,        // the self-test's wait ran out (as it should)
+    kStatusEpPlan = 32,          // expert-parallel counts disagree, or a receive buffer is too small
+};
+
 constexpr int kTcBM = 128;
 constexpr int kSimtBM = 64;
 // (token, slot) pairs per dispatch block.
@@ -139,6 +150,21 @@ cudaError_t launch_simt_gemm2(const float* h, const float* w2, float* o, const i
 
 // tcgen05 grouped GEMMs (bf16 handles).  Tensor maps are built by the host
 // (see moe_api.cu) over: Xp [R_cap][d], w1/w3 [n][d][F], H [R_cap][F], w2 [n][F][d].
+// Expert parallelism (ep.cu): one device pointer per rank, by value.
+constexpr int kMaxEpRanks = 16;
+struct EpPeers {
+    void* ptr[kMaxEpRanks];
+};
+cudaError_t launch_ep_plan(const int32_t* counts_all, int W, int n, int rank, const int32_t* own_counts,
+                           int64_t recv_rows, int32_t* dst_base, int32_t* loff, int32_t* lmblk, int* status,
+                           cudaStream_t st);
+cudaError_t launch_ep_scatter(const void* x, const int32_t* idx, const int32_t* token_row, const int32_t* offsets,
+                              const int32_t* dst_base, int64_t T, int K, int n, int nl, const EpPeers& recv,
+                              int64_t recv_rows, int d, int32_t* row_pos, const int* status, int num_sms,
+                              cudaStream_t st);
+cudaError_t launch_ep_combine(const int32_t* idx, const float* topk_w, const int32_t* row_pos, int64_t T, int K,
+                              int n, int nl, const EpPeers& out, int d, void* y, int num_sms, cudaStream_t st);
+
 struct TcGemmArgs {
     const int32_t* offsets;
     const int32_t* mblk_base;

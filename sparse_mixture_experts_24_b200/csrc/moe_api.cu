@@ -176,6 +176,16 @@ struct moe_handle {
     CUtensorMap tm_rx, tm_parts;
     const void* c_rx = nullptr;
     int64_t c_rx_T = -1;
+    // expert parallelism: plan arrays (workspace), and tensor maps of the
+    // receive buffer and the local experts' weights
+    int32_t* ep_dst = nullptr;    // [n]
+    int32_t* ep_loff = nullptr;   // [n+1]
+    int32_t* ep_lmblk = nullptr;  // [n+1]
+    CUtensorMap tm_erecv, tm_ew1, tm_ew3, tm_ew2;
+    const void* c_erecv = nullptr;
+    int64_t c_erecv_rows = -1;
+    const void* c_ew[3] = {nullptr, nullptr, nullptr};
+    int c_ew_nl = 0;
     // expert capacity factor (0: dropless) and load-balancing statistics scratch
     double capacity_factor = 0.0;
     // kernels this handle has launched (for profiling and launch accounting)
@@ -303,6 +313,7 @@ moe_status grow(moe_handle* h, int64_t T, int64_t rows_min = 0) {
     const size_t o_stats_counts = take(static_cast<size_t>(h->n) * 4);
     const size_t o_parts = take(bf ? static_cast<size_t>(3) * npad * h->d * 2 : 0);
     const size_t o_status = take(64);
+    const size_t o_ep = take(static_cast<size_t>(3 * h->n + 2) * 4);
     const size_t o_ec_probs = take(static_cast<size_t>(T) * h->n * 4);
     const size_t o_ec_rowmap = take(static_cast<size_t>(T) * h->n * 4);
     const size_t o_xp = take(static_cast<size_t>(R) * h->d * h->esize());
@@ -360,6 +371,10 @@ moe_status grow(moe_handle* h, int64_t T, int64_t rows_min = 0) {
     h->stats_counts = reinterpret_cast<int32_t*>(b + o_stats_counts);
     h->c_rx = nullptr;
     h->status = reinterpret_cast<int*>(b + o_status);
+    h->ep_dst = reinterpret_cast<int32_t*>(b + o_ep);
+    h->ep_loff = h->ep_dst + h->n;
+    h->ep_lmblk = h->ep_loff + h->n + 1;
+    h->c_erecv = nullptr;
     h->xp = b + o_xp;
     h->h = b + o_h;
     h->o = b + o_o;
@@ -785,6 +800,32 @@ moe_status run_logits(moe_handle* h, int64_t T, const void* x, const float* W_g,
     return MOE_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Expert parallelism
+moe_status ep_check(moe_handle* h, int world, int rank) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "null handle");
+    if (world < 1 || world > moe::kMaxEpRanks)
+        return fail(MOE_ERR_INVALID_ARG, "world = %d outside [1, %d]", world, moe::kMaxEpRanks);
+    if (rank < 0 || rank >= world) return fail(MOE_ERR_INVALID_ARG, "rank = %d outside [0, %d)", rank, world);
+    if (h->n % world != 0)
+        return fail(MOE_ERR_INVALID_ARG, "n = %d experts do not split evenly over %d ranks", h->n, world);
+    if (h->dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "expert parallelism needs a MOE_BF16 handle");
+    if (h->capacity_factor > 0.0)
+        return fail(MOE_ERR_UNSUPPORTED, "expert parallelism is dropless: the capacity factor must be 0");
+    return MOE_OK;
+}
+
+moe_status ep_peers(int world, void* const* ptrs, const char* name, moe::EpPeers* out) {
+    if (!ptrs) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", name);
+    *out = moe::EpPeers{};
+    for (int q = 0; q < world; ++q) {
+        if (!ptrs[q]) return fail(MOE_ERR_INVALID_ARG, "%s[%d] is NULL", name, q);
+        if (!aligned16(ptrs[q])) return fail(MOE_ERR_INVALID_ARG, "%s[%d] is not 16-byte aligned", name, q);
+        out->ptr[q] = ptrs[q];
+    }
+    return MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -1164,6 +1205,170 @@ moe_status moe_forward_w4a4(moe_handle* h, int64_t T, const void* x, const float
     return s == MOE_OK ? ok() : s;
 }
 
+moe_status moe_ep_dispatch(moe_handle* h, int world, int rank, int64_t T, const void* x, const int32_t* topk_idx,
+                           const int32_t* counts_all, void* const* recv_buffers, int64_t recv_rows,
+                           int32_t* row_pos, moe_stream_t stream) {
+    moe_status s = ep_check(h, world, rank);
+    if (s != MOE_OK) return s;
+    s = check_common(h, T);
+    if (s != MOE_OK) return s;
+    if (recv_rows < 1 || recv_rows > 2147483647LL)
+        return fail(MOE_ERR_INVALID_ARG, "recv_rows = %lld outside [1, 2^31 - 1]", static_cast<long long>(recv_rows));
+    moe::EpPeers peers;
+    s = ep_peers(world, recv_buffers, "recv_buffers", &peers);
+    if (s != MOE_OK) return s;
+    REQUIRE_PTR(counts_all);
+    if (T == 0) return ok();
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(topk_idx);
+    REQUIRE_PTR(row_pos);
+    s = prepare(h, T);
+    if (s != MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    moe::chain_begin();
+    const int64_t R = T * h->K;
+    cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n, moe::kTcBM, h->db, st, moe::kNoCapacity);
+    if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
+    h->launches += moe::dispatch_kernel_count(R);
+    e = moe::launch_ep_plan(counts_all, world, h->n, rank, h->db.counts, recv_rows, h->ep_dst, h->ep_loff,
+                            h->ep_lmblk, h->status, st);
+    if (e != cudaSuccess) return cuda_fail(e, "expert-parallel plan launch");
+    e = moe::launch_ep_scatter(x, topk_idx, h->db.token_row, h->db.offsets, h->ep_dst, T, h->K, h->n,
+                               h->n / world, peers, recv_rows, h->d, row_pos, h->status, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "expert-parallel scatter launch");
+    h->launches += 2;
+    return ok();
+}
+
+moe_status moe_ep_experts(moe_handle* h, int world, int rank, const int32_t* counts_all, const void* recv,
+                          int64_t recv_rows, const void* w1, const void* w3, const void* w2, void* out,
+                          moe_stream_t stream) {
+    moe_status s = ep_check(h, world, rank);
+    if (s != MOE_OK) return s;
+    if (recv_rows < 1 || recv_rows > 2147483647LL)
+        return fail(MOE_ERR_INVALID_ARG, "recv_rows = %lld outside [1, 2^31 - 1]", static_cast<long long>(recv_rows));
+    REQUIRE_PTR(counts_all);
+    REQUIRE_PTR(recv);
+    REQUIRE_PTR(w1);
+    REQUIRE_PTR(w3);
+    REQUIRE_PTR(w2);
+    REQUIRE_PTR(out);
+    s = prepare(h, 0, recv_rows);
+    if (s != MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    moe::chain_begin();
+    const int nl = h->n / world;
+    if (recv != h->c_erecv || recv_rows != h->c_erecv_rows) {
+        if (!encode_rows(&h->tm_erecv, recv, h->d, static_cast<uint64_t>(recv_rows)))
+            return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the receive buffer");
+        h->c_erecv = recv;
+        h->c_erecv_rows = recv_rows;
+    }
+    const void* w[3] = {w1, w3, w2};
+    CUtensorMap* tm[3] = {&h->tm_ew1, &h->tm_ew3, &h->tm_ew2};
+    for (int m = 0; m < 3; ++m) {
+        if (w[m] == h->c_ew[m] && nl == h->c_ew_nl) continue;
+        const bool down = m == 2;
+        if (!encode_weights(tm[m], w[m], down ? h->d : h->F, down ? h->F : h->d, static_cast<uint64_t>(nl)))
+            return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the local expert weights");
+        h->c_ew[m] = w[m];
+    }
+    h->c_ew_nl = nl;
+    cudaError_t e = moe::launch_ep_plan(counts_all, world, h->n, rank, nullptr, recv_rows, h->ep_dst, h->ep_loff,
+                                        h->ep_lmblk, h->status, st);
+    if (e != cudaSuccess) return cuda_fail(e, "expert-parallel plan launch");
+    moe::TcGemmArgs a1{};
+    a1.offsets = h->ep_loff;
+    a1.mblk_base = h->ep_lmblk;
+    a1.n = nl;
+    a1.R = recv_rows;
+    a1.k_blocks = h->d / 64;
+    a1.n_tiles = (h->F + 127) / 128;
+    a1.out_cols = h->F;
+    a1.out = h->h;
+    a1.status = h->status;
+    e = moe::launch_tc_gemm1(h->tm_erecv, h->tm_ew1, h->tm_ew3, a1, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
+    moe::TcGemmArgs a2 = a1;
+    a2.k_blocks = h->F / 64;
+    a2.n_tiles = (h->d + 255) / 256;
+    a2.out_cols = h->d;
+    a2.out = out;
+    e = moe::launch_tc_gemm2(h->tm_h, h->tm_ew2, a2, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
+    h->launches += 3;
+    return ok();
+}
+
+moe_status moe_ep_combine(moe_handle* h, int world, int64_t T, const int32_t* topk_idx, const float* topk_w,
+                          const int32_t* row_pos, const void* const* out_buffers, void* y, moe_stream_t stream) {
+    moe_status s = ep_check(h, world, 0);
+    if (s != MOE_OK) return s;
+    s = check_common(h, T);
+    if (s != MOE_OK) return s;
+    moe::EpPeers peers;
+    s = ep_peers(world, const_cast<void* const*>(out_buffers), "out_buffers", &peers);
+    if (s != MOE_OK) return s;
+    if (T == 0) return ok();
+    REQUIRE_PTR(topk_idx);
+    REQUIRE_PTR(topk_w);
+    REQUIRE_PTR(row_pos);
+    REQUIRE_PTR(y);
+    s = check_device(h);
+    if (s != MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    moe::chain_begin();
+    cudaError_t e = moe::launch_ep_combine(topk_idx, topk_w, row_pos, T, h->K, h->n, h->n / world, peers, h->d, y,
+                                           h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "expert-parallel combine launch");
+    h->launches += 1;
+    return ok();
+}
+
+moe_status moe_ep_buffer_alloc(int64_t bytes, void** ptr, uint8_t* ipc_handle) {
+    if (!ptr) return fail(MOE_ERR_INVALID_ARG, "ptr is NULL");
+    *ptr = nullptr;
+    if (bytes < 1) return fail(MOE_ERR_INVALID_ARG, "bytes = %lld < 1", static_cast<long long>(bytes));
+    void* p = nullptr;
+    cudaError_t e = cudaMalloc(&p, static_cast<size_t>(bytes));
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(MOE_ERR_ALLOC, "cudaMalloc(%lld bytes) failed: %s", static_cast<long long>(bytes),
+                    cudaGetErrorString(e));
+    }
+    if (ipc_handle) {
+        cudaIpcMemHandle_t hd;
+        e = cudaIpcGetMemHandle(&hd, p);
+        if (e != cudaSuccess) {
+            cudaFree(p);
+            return cuda_fail(e, "cudaIpcGetMemHandle");
+        }
+        static_assert(sizeof hd == 64, "CUDA IPC handles are 64 bytes");
+        memcpy(ipc_handle, &hd, sizeof hd);
+    }
+    *ptr = p;
+    return ok();
+}
+
+moe_status moe_ep_buffer_open(const uint8_t* ipc_handle, void** ptr) {
+    if (!ipc_handle || !ptr) return fail(MOE_ERR_INVALID_ARG, "ipc_handle or ptr is NULL");
+    *ptr = nullptr;
+    cudaIpcMemHandle_t hd;
+    memcpy(&hd, ipc_handle, sizeof hd);
+    void* p = nullptr;
+    cudaError_t e = cudaIpcOpenMemHandle(&p, hd, cudaIpcMemLazyEnablePeerAccess);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaIpcOpenMemHandle");
+    *ptr = p;
+    return ok();
+}
+
+moe_status moe_ep_buffer_close(void* ptr, int opened) {
+    if (!ptr) return ok();
+    cudaError_t e = opened ? cudaIpcCloseMemHandle(ptr) : cudaFree(ptr);
+    if (e != cudaSuccess) return cuda_fail(e, opened ? "cudaIpcCloseMemHandle" : "cudaFree");
+    return ok();
+}
+
 moe_status moe_set_capacity_factor(moe_handle* h, double factor) {
     if (!h) return fail(MOE_ERR_INVALID_ARG, "null handle");
     if (!(factor >= 0.0) || !std::isfinite(factor))
@@ -1230,6 +1435,11 @@ moe_status moe_sync_status(moe_handle* h, moe_stream_t stream) {
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(status)");
     if (st != 0) {
         cudaMemset(h->status, 0, sizeof st);
+        if (st == moe::kStatusEpPlan)
+            return fail(MOE_ERR_INVALID_ARG,
+                        "expert-parallel plan rejected: counts_all disagrees with this rank's routing or holds a "
+                        "negative count, or a receive buffer has too few rows (status bits 0x%x)",
+                        st);
         return fail(MOE_ERR_TIMEOUT, "a kernel gave up a bounded wait (status bits 0x%x)", st);
     }
     return ok();
