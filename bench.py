@@ -315,6 +315,135 @@ def run_reference(args, cfg):
 # our arm
 # --------------------------------------------------------------------------
 
+def run_ep(args, cfg):
+    """--ep W: one expert-parallel layer step of W ranks emulated on this GPU
+    (the workload's T tokens split over the ranks, n/W experts each; every
+    phase runs for all ranks before the next, as the barriers order them
+    across GPUs).  The exchange is the kernels' peer stores and loads, here
+    into this GPU's memory, so the number measures the kernels, not NVLink."""
+    import torch
+    import sparse_mixture_experts_24_b200 as m
+    from sparse_mixture_experts_24_b200.ep import EmulatedExpertParallel
+    W = args.ep
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1 or args.gpus != 1:
+        raise SystemExit("--ep emulates its ranks on one GPU: run it with --gpus 1")
+    if cfg.dtype != "bf16" or args.experts != "bf16" or W < 1 or cfg.n % W:
+        raise SystemExit("--ep needs a bf16 workload with bf16 experts and W dividing n")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    L = mi.make_layer(cfg, seed=replica_seed(0))
+
+    def to_dev(a):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        if a.dtype == np.uint16:
+            t = t.view(torch.int16).view(torch.bfloat16)
+        return t.to(dev)
+
+    x, Wg, w1, w3, w2 = (to_dev(L[k]) for k in ("x", "W_g", "w1", "w3", "w2"))
+    T, n, K = cfg.T, cfg.n, cfg.K
+    bounds = [T * r // W for r in range(W + 1)]
+    xs = [x[bounds[r]:bounds[r + 1]] for r in range(W)]
+    nl = n // W
+    weights = [tuple(t[q * nl:(q + 1) * nl] for t in (w1, w3, w2)) for q in range(W)]
+    ep = EmulatedExpertParallel(n, K, cfg.d, cfg.ffn, W, T * K)
+    ys = [torch.empty_like(xr) for xr in xs]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(mark=None):
+        return ep.forward(xs, Wg, weights, ys, mark=mark)
+
+    for _ in range(args.warmup):
+        _, idxs, _ = step()
+    ep.sync_status()
+    counts = touched_experts(torch.cat(idxs).cpu().numpy(), n)
+
+    sampler = ClockSampler(dev.index)
+    torch.cuda.synchronize(dev)
+    launches0 = ep.launch_count()
+    sampler.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    launches = ep.launch_count() - launches0
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ep.sync_status()
+
+    # the same steps with an event after each phase
+    names = ("route", "dispatch", "experts", "combine")
+    acc = [0.0] * 4
+    for _ in range(args.steps):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        evs[0].record(stream)
+        step(mark=lambda i: evs[i + 1].record(stream))
+        torch.cuda.synchronize(dev)
+        for i in range(4):
+            acc[i] += evs[i].elapsed_time(evs[i + 1])
+    phase_ms = {k: a / args.steps for k, a in zip(names, acc)}
+
+    # end to end: x from pinned host memory in, y back, every step
+    xh = x.cpu().pin_memory()
+    yh = torch.empty(x.shape, dtype=x.dtype).pin_memory()
+    xd = torch.empty_like(x)
+    xds = [xd[bounds[r]:bounds[r + 1]] for r in range(W)]
+    yd = torch.empty_like(x)
+    yds = [yd[bounds[r]:bounds[r + 1]] for r in range(W)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        xd.copy_(xh, non_blocking=True)
+        ep.forward(xds, Wg, weights, yds)
+        yh.copy_(yd, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ems = e0.elapsed_time(e1) / args.steps
+    same = bool(torch.equal(yh, torch.cat(ys).cpu()))
+
+    peaks, peak_src = load_peaks()
+    work = algorithmic(cfg, counts, "bf16")
+    flops = work["gemm1"]["flops"] + work["gemm2"]["flops"]
+    nbytes = work["gemm1"]["bytes"] + work["gemm2"]["bytes"]
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    t_exp = phase_ms["experts"] * 1e-3
+    if flops / nbytes < ridge:
+        ach = nbytes / t_exp / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "algorithmic_per_launch": nbytes}
+    else:
+        pk = peaks["bf16_tflops_sustained"] if ms * args.steps > 1000 else peaks["bf16_tflops"]
+        ach = flops / t_exp / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
+                "algorithmic_per_launch": flops}
+    roof.update({"kernel": "experts phase of all ranks (plan + GEMM1 + GEMM2 per rank)",
+                 "peak_source": peak_src, "launch_ms": phase_ms["experts"], "traffic": None})
+    cpu = None
+    if not args.no_cpu_baseline:
+        v, smp, reps, cores, el = oracle_tokens_per_s(cfg, L)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": "first %d of %d tokens x %d repetitions, full layer in fp64 (%.1f s)" % (smp, T, reps, el)}
+    line = {
+        "metric": "MoE-layer tokens/s", "value": T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_desc(cfg) + "; expert-parallel, %d ranks emulated on one GPU" % W,
+                   "global_batch_tokens": T, "parallelism": "ep%d emulated on 1 GPU" % W,
+                   "l2": "no flush: %.2f GB of expert weights per step > 126 MB L2" % (work["layer_bytes"] / 1e9)},
+        "phase_ms_per_step": {k: round(v, 5) for k, v in phase_ms.items()},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": T / (ems * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": x.numel() * 2,
+                "d2h_bytes_per_step": x.numel() * 2, "outputs_match_device_run": same},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    print(json.dumps(line))
+    ep.close()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -324,10 +453,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--experts", default="bf16", choices=["bf16", "e4m3", "fp4", "w4a4"])
+    ap.add_argument("--ep", type=int, default=0,
+                    help="expert parallelism with this many ranks, emulated on one GPU")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     cfg = mi.CONFIGS[args.config]
+    if args.ep:
+        return run_ep(args, cfg)
     if args.experts != "bf16" and cfg.dtype != "bf16":
         ap.error("--experts %s needs a bf16 workload" % args.experts)
     if args.impl == "reference":

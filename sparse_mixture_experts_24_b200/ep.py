@@ -56,37 +56,72 @@ class _Rank:
         self.layer.close()
 
 
+class EmulatedExpertParallel:
+    """W ranks on the current GPU with persistent handles and buffers: every
+    phase runs for all ranks before the next phase starts (the order the
+    barriers impose across GPUs), each rank's buffers in this GPU's memory.
+    recv_rows: rows of each receive buffer (W * T_max * K always suffices)."""
+
+    def __init__(self, n, K, d, ffn, world, recv_rows):
+        import torch
+        self.n, self.K, self.d, self.world, self.recv_rows = n, K, d, world, recv_rows
+        self.ranks = [_Rank(n, K, d, ffn) for _ in range(world)]
+        dev = torch.device("cuda", torch.cuda.current_device())
+        self.recv = [torch.empty((recv_rows, d), dtype=torch.bfloat16, device=dev) for _ in range(world)]
+        self.out = [torch.empty((recv_rows, d), dtype=torch.bfloat16, device=dev) for _ in range(world)]
+
+    def forward(self, xs, W_g, weights, ys=None, stream=None, mark=None):
+        """xs: W bf16 token blocks [T_r][d]; weights: W (w1, w3, w2) triples of
+        each rank's local experts.  -> (ys, idxs, gates), one entry per rank.
+        mark(i), if given, is called after phase i (0 routing and counts,
+        1 dispatch, 2 experts, 3 combine) -- e.g. to record CUDA events."""
+        import torch
+        W = self.world
+        mark = mark or (lambda i: None)
+        counts_all = torch.stack([rk.route(x, W_g, stream) for rk, x in zip(self.ranks, xs)])
+        mark(0)
+        for r, (rk, x) in enumerate(zip(self.ranks, xs)):
+            rk.dispatch(W, r, x, counts_all, self.recv, self.recv_rows, stream)
+        mark(1)
+        for q, rk in enumerate(self.ranks):
+            rk.experts(W, q, counts_all, self.recv[q], self.recv_rows, *weights[q], self.out[q], stream)
+        mark(2)
+        if ys is None:
+            ys = [torch.empty_like(x) for x in xs]
+        for rk, y in zip(self.ranks, ys):
+            rk.combine(W, self.out, y, stream)
+        mark(3)
+        return ys, [rk.idx for rk in self.ranks], [rk.gate for rk in self.ranks]
+
+    def launch_count(self):
+        from . import moe_launch_count
+        return sum(moe_launch_count(rk.layer.h) for rk in self.ranks)
+
+    def sync_status(self, stream=None):
+        for rk in self.ranks:
+            rk.layer.sync_status(stream)
+
+    def close(self):
+        for rk in self.ranks:
+            rk.close()
+        self.ranks = []
+
+
 def emulate_ranks(xs, W_g, weights, n, K, recv_rows=None, stream=None):
-    """W ranks on the current GPU.  xs: W bf16 token blocks [T_r][d];
-    weights: W (w1, w3, w2) triples of each rank's local experts.
-    -> (ys, idxs, gates): per rank y [T_r][d], topk_idx, topk_w."""
-    import torch
+    """One expert-parallel step of W = len(xs) ranks on the current GPU (see
+    EmulatedExpertParallel).  -> (ys, idxs, gates)."""
     world = len(xs)
     d = xs[0].shape[1]
     ffn = weights[0][0].shape[2]
-    dev = xs[0].device
     if recv_rows is None:
         recv_rows = max(1, sum(int(x.shape[0]) for x in xs) * K)
-    ranks = [_Rank(n, K, d, ffn) for _ in range(world)]
+    ep = EmulatedExpertParallel(n, K, d, ffn, world, recv_rows)
     try:
-        recv = [torch.empty((recv_rows, d), dtype=torch.bfloat16, device=dev) for _ in range(world)]
-        out = [torch.empty((recv_rows, d), dtype=torch.bfloat16, device=dev) for _ in range(world)]
-        counts_all = torch.stack([rk.route(x, W_g, stream) for rk, x in zip(ranks, xs)])
-        for r, (rk, x) in enumerate(zip(ranks, xs)):
-            rk.dispatch(world, r, x, counts_all, recv, recv_rows, stream)
-        for q, rk in enumerate(ranks):
-            rk.experts(world, q, counts_all, recv[q], recv_rows, *weights[q], out[q], stream)
-        ys = []
-        for rk, x in zip(ranks, xs):
-            y = torch.empty_like(x)
-            rk.combine(world, out, y, stream)
-            ys.append(y)
-        for rk in ranks:
-            rk.layer.sync_status(stream)
-        return ys, [rk.idx for rk in ranks], [rk.gate for rk in ranks]
+        out = ep.forward(xs, W_g, weights, stream=stream)
+        ep.sync_status(stream)
+        return out
     finally:
-        for rk in ranks:
-            rk.close()
+        ep.close()
 
 
 class _CudaOps:
