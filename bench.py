@@ -2,7 +2,7 @@
 """Benchmark of the sparse MoE layer forward (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
-                    [--experts bf16|e4m3|fp4|w4a4]
+                    [--experts bf16|e4m3|fp4|w4a4] [--ep W]
 
 A step is one moe_forward over one batch: router, top-K, softmax, dispatch,
 gather, GEMM1 (w1/w3 + SwiGLU), GEMM2 (w2), combine.  The default workload is
@@ -32,7 +32,11 @@ handle and workloads only); --experts w4a4 times moe_forward_w4a4: the same
 4-bit weights with 4-bit activations on the block-scaled tensor cores (d and
 ffn multiples of 256).
 
---impl reference runs the oracle (the reference arm of this build) on the
+--ep W times one expert-parallel step with W ranks emulated on this GPU (n/W
+experts per rank, the tokens split over the ranks; the exchange is the
+kernels' own stores and loads, here into this GPU's memory).
+
+--impl reference runs the oracle (the reference arm: a plain fp64 CPU layer) on the
 host, rank 0 only.
 """
 from __future__ import annotations
