@@ -276,19 +276,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf * kBN);
             uint16_t* out = static_cast<uint16_t*>(args.out);
             const float g0 = m0 * rs;
+            // This warp's accumulator columns go to registers first and the
+            // accumulator is handed back to the MMA warp before any math or
+            // store: with one accumulator the next tile's MMAs wait only for
+            // these TMEM reads.
+            constexpr int kRegChunks = kBN / 64;  // 32-column chunks per warp
+            uint32_t acc[kRegChunks][32];
+#pragma unroll
+            for (int i = 0; i < kRegChunks; ++i) {
+                int col;
+                if (kSwiGLU) {
+                    // chunk pair q (q = half * kRegChunks / 2 + i / 2): w1 columns
+                    // 128 (q / 2) + 32 (q % 2) + 0..31, the w3 ones 64 later
+                    const int q = half * (kRegChunks / 2) + (i >> 1);
+                    col = 128 * (q >> 1) + 32 * (q & 1) + ((i & 1) ? 64 : 0);
+                } else {
+                    col = (half * kRegChunks + i) * 32;
+                }
+                tmem_ld_32x32b_x32(tbase + col, acc[i]);
+            }
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&tail->accum_empty[buf]));
             if (kSwiGLU) {
                 const float g1 = m1 * rs;
-                // 32-column chunks of hidden columns: chunk q covers block q / 2,
-                // w1 columns 128 (q / 2) + 32 (q % 2) + 0..31 and the w3 ones 64 later
-                constexpr int kChunks = kBN / 64;
-#pragma unroll 1
-                for (int q = half * (kChunks / 2); q < (half + 1) * (kChunks / 2); ++q) {
-                    const int acol = 128 * (q >> 1) + 32 * (q & 1);
-                    uint32_t a[32], b[32];
-                    tmem_ld_32x32b_x32(tbase + acol, a);
-                    tmem_ld_32x32b_x32(tbase + acol + 64, b);
-                    tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < kRegChunks / 2; ++i) {
+                    const int q = half * (kRegChunks / 2) + i;
                     const int col = ti.n_tile * (kBN / 2) + 32 * q;
+                    const uint32_t* a = acc[2 * i];
+                    const uint32_t* b = acc[2 * i + 1];
                     if (row_ok && col < args.out_cols) {
                         uint32_t pk[16];
 #pragma unroll
@@ -305,13 +323,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             } else {
-                constexpr int kChunks = kBN / 32;
-#pragma unroll 1
-                for (int c = half * (kChunks / 2); c < (half + 1) * (kChunks / 2); ++c) {
-                    uint32_t a[32];
-                    tmem_ld_32x32b_x32(tbase + c * 32, a);
-                    tmem_wait_ld();
-                    const int col = ti.n_tile * kBN + c * 32;
+#pragma unroll
+                for (int i = 0; i < kRegChunks; ++i) {
+                    const int col = ti.n_tile * kBN + (half * kRegChunks + i) * 32;
+                    const uint32_t* a = acc[i];
                     if (row_ok && col < args.out_cols) {
                         uint32_t pk[16];
 #pragma unroll
@@ -324,9 +339,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&tail->accum_empty[buf]));
         }
     }
 
