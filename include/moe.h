@@ -339,8 +339,10 @@ MOE_API moe_status moe_pack_weights_w4a4(int n, int rows, int cols, const uint8_
  * (w1 and w3, rows = d, cols = ffn); w2_packed / w2_chunks: w2 packed alone
  * (rows = ffn, cols = d); w*_matrix_scales from moe_quantize_weights_fp4;
  * x, W_g, y, topk_idx, topk_w as for moe_forward.  The GEMMs use tiles of
- * 256 packed columns; MOE_W4A4_TILE=128 selects 128-column tiles with two
- * accumulators (same results, measured slower on the Mixtral shapes).
+ * 256 packed columns, over 32 rows when the experts average at most 32 rows
+ * per call (T*K <= 32*n) and over 128 rows otherwise; MOE_W4A4_TILE=128
+ * selects 128-column tiles with two accumulators (128 rows), MOE_W4A4_ROWS=32
+ * or 128 forces the row tiles (same results either way).
  * The first call grows the workspace by about T*K*(d + ffn)*0.6 bytes.
  *   Errors: as moe_forward; MOE_ERR_UNSUPPORTED for an fp32 handle or d, ffn
  *   not multiples of 256.

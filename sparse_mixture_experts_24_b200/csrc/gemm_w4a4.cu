@@ -32,8 +32,7 @@ namespace moe {
 
 namespace w4gemm {
 
-constexpr int kBM = kTcBM;   // 128
-constexpr int kABytes = kBM * 128;      // 16 KB: 128 rows of 128 bytes (K step of 256)
+constexpr int kBM = kTcBM;   // 128: MMA M
 constexpr int kBBlockBytes = 128 * 128; // 16 KB: one 128-row block of B
 constexpr int kSfaBytes = 4 * 512;      // 4 chunks (64-wide K steps) of A scales
 constexpr int kSfbBlockBytes = 4 * 512; // the same for one 128-row block of B
@@ -43,14 +42,18 @@ constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, each taking half th
 constexpr int kThreads = (2 + kEpiWarps) * 32;
 
 // Tile width kBN (128 or 256 output columns of the packed B, i.e. 64 or 128
-// hidden columns of GEMM1's w1|w3 pairs): B blocks per stage, stages, and
-// TMEM: accumulators from column 0 (two of 128 columns, or one of 256), the
-// scale factors of every stage after them.
-template <int kBN>
+// hidden columns of GEMM1's w1|w3 pairs) and tile height kTM (rows of A per
+// tile: 128, or 32 for batches of a few rows per expert): B blocks per stage,
+// stages, and TMEM: accumulators from column 0 (two of 128 columns, or one of
+// 256), the scale factors of every stage after them.  The MMA is always
+// M = 128; with kTM = 32 the A rows past 32 are whatever follows in shared
+// memory (finite codes), and their accumulator rows are never stored.
+template <int kBN, int kTM>
 struct Cfg {
     static constexpr int kBlocks = kBN / 128;
+    static constexpr int kABytes = kTM * 128;  // kTM rows of 128 bytes (a K step of 256)
     static constexpr int kStageBytes = kABytes + kBlocks * kBBlockBytes + kSfaBytes + kBlocks * kSfbBlockBytes;
-    static constexpr int kStages = kBN == 128 ? 6 : 4;
+    static constexpr int kStages = kBN == 128 ? 6 : (kTM == 32 ? 5 : 4);
     static constexpr int kAccBufs = kBN == 128 ? 2 : 1;
     static constexpr int kSfCols = 4 * (4 + 4 * kBlocks);  // per stage: 4 K steps x (A + B chunks)
     static constexpr int kSfBase = kAccBufs * kBN;
@@ -71,15 +74,16 @@ struct __align__(8) SmemTail {
 
 constexpr int kTailBytes = (static_cast<int>(sizeof(SmemTail)) + 127) / 128 * 128;
 
-template <int kBN>
+template <int kBN, int kTM>
 constexpr int smem_bytes() {
-    return Cfg<kBN>::kStages * Cfg<kBN>::kStageBytes + kTailBytes + 1024;
+    return Cfg<kBN, kTM>::kStages * Cfg<kBN, kTM>::kStageBytes + kTailBytes + 1024;
 }
 
 struct Tile {
     int e, n_tile, m_blk, row0, rows;
 };
 
+template <int kTM>
 __device__ __forceinline__ Tile tile_at(int t, const int32_t* off, const int32_t* mblk, int n, int n_tiles) {
     int lo = 0, hi = n - 1;
     while (lo < hi) {
@@ -95,8 +99,8 @@ __device__ __forceinline__ Tile tile_at(int t, const int32_t* off, const int32_t
     const int mb_count = mblk[lo + 1] - mblk[lo];
     ti.n_tile = local / mb_count;
     ti.m_blk = local - ti.n_tile * mb_count;
-    ti.row0 = off[lo] + ti.m_blk * kBM;
-    ti.rows = min(kBM, off[lo + 1] - ti.row0);
+    ti.row0 = off[lo] + ti.m_blk * kTM;
+    ti.rows = min(kTM, off[lo + 1] - ti.row0);
     return ti;
 }
 
@@ -109,11 +113,11 @@ using namespace w4gemm;
 // kSwiGLU: GEMM1 over the w1|w3 pair pack (accumulator column j of block
 // j / 128 is w1 for j % 128 < 64, w3 otherwise; hidden column = 64 x block +
 // j % 64); else GEMM2 over w2.
-template <bool kSwiGLU, int kBN>
+template <bool kSwiGLU, int kBN, int kTM>
 __global__ void __launch_bounds__(kThreads, 1)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                      const W4a4GemmArgs args) {
-    using C = Cfg<kBN>;
+    using C = Cfg<kBN, kTM>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -166,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             const int blocks_per_e = args.n_rows_b / 128;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-                const Tile ti = tile_at(t, tail->off, tail->mblk, n, args.n_tiles);
+                const Tile ti = tile_at<kTM>(t, tail->off, tail->mblk, n, args.n_tiles);
                 const int r0 = ti.n_tile * kBN;  // first packed B row of the tile
                 const uint8_t* sfb = args.b_chunks +
                                      (static_cast<int64_t>(ti.e) * blocks_per_e + r0 / 128) * kb64_total * 512;
@@ -181,14 +185,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(fb, C::kStageBytes);
                     armed[stage] = static_cast<int>(phase);
                     const uint32_t base = smem_u32(smem + stage * C::kStageBytes);
-                    const uint32_t sf_smem = base + kABytes + C::kBlocks * kBBlockBytes;
+                    const uint32_t sf_smem = base + C::kABytes + C::kBlocks * kBBlockBytes;
                     const int kx = ks * 128;  // byte column of the codes
                     const int64_t ck = static_cast<int64_t>(ks) * 4 * 512;
                     tma_load_2d(base, &tm_a, fb, kx, ti.row0);
                     bulk_load(sf_smem, sfa + ck, kSfaBytes, fb);
 #pragma unroll
                     for (int b = 0; b < C::kBlocks; ++b) {
-                        tma_load_3d(base + kABytes + b * kBBlockBytes, &tm_b, fb, kx, r0 + 128 * b, ti.e);
+                        tma_load_3d(base + C::kABytes + b * kBBlockBytes, &tm_b, fb, kx, r0 + 128 * b, ti.e);
                         bulk_load(sf_smem + kSfaBytes + b * kSfbBlockBytes,
                                   sfb + static_cast<int64_t>(b) * kb64_total * 512 + ck, kSfbBlockBytes, fb);
                     }
@@ -226,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after();
                     const uint32_t base = smem_u32(smem + stage * C::kStageBytes);
-                    const uint32_t sfa_smem = base + kABytes + C::kBlocks * kBBlockBytes;
+                    const uint32_t sfa_smem = base + C::kABytes + C::kBlocks * kBBlockBytes;
                     const uint32_t sfb_smem = sfa_smem + kSfaBytes;
                     const uint32_t sf_col = tmem_base + static_cast<uint32_t>(C::kSfBase + stage * C::kSfCols);
 #pragma unroll
@@ -239,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc_cp_32x128b_warpx4(sfb_t + 4 * b,
                                                  make_smem_desc(sfb_smem + b * kSfbBlockBytes + kk * 512, 0, 128, 0));
                         const uint64_t adesc = make_smem_desc(base + kk * 32, 16, 1024, 2);
-                        const uint64_t bdesc = make_smem_desc(base + kABytes + kk * 32, 16, 1024, 2);
+                        const uint64_t bdesc = make_smem_desc(base + C::kABytes + kk * 32, 16, 1024, 2);
                         tc_mma_fp4_block16(d_tmem, adesc, bdesc, idesc, sfa_t, sfb_t, (ks | kk) != 0 ? 1u : 0u);
                     }
                     tc_commit(smem_u32(&tail->empty[stage]));
@@ -260,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int half = (warp - 2) >> 2;
         int local = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++local) {
-            const Tile ti = tile_at(t, tail->off, tail->mblk, n, args.n_tiles);
+            const Tile ti = tile_at<kTM>(t, tail->off, tail->mblk, n, args.n_tiles);
             const int buf = C::kAccBufs == 2 ? (local & 1) : 0;
             const uint32_t use = C::kAccBufs == 2 ? static_cast<uint32_t>(local >> 1) : static_cast<uint32_t>(local);
             const int valid = min(32, ti.rows - quad * 32);
@@ -282,8 +286,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             // these TMEM reads.
             constexpr int kRegChunks = kBN / 64;  // 32-column chunks per warp
             uint32_t acc[kRegChunks][32];
+            // warp-uniform: a quadrant past the tile's rows only hands back
+            const bool any_row = valid > 0;
 #pragma unroll
             for (int i = 0; i < kRegChunks; ++i) {
+                if (!any_row) break;
                 int col;
                 if (kSwiGLU) {
                     // chunk pair q (q = half * kRegChunks / 2 + i / 2): w1 columns
@@ -295,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tmem_ld_32x32b_x32(tbase + col, acc[i]);
             }
-            tmem_wait_ld();
+            if (any_row) tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&tail->accum_empty[buf]));
@@ -353,31 +360,42 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 int w4a4_tile_cols(bool wide) { return wide ? 256 : 128; }
 
-template <bool kSwiGLU, int kBN>
+template <bool kSwiGLU, int kBN, int kTM>
 static cudaError_t launch_w4(const CUtensorMap& ta, const CUtensorMap& tb, const W4a4GemmArgs& a, int num_sms,
                              cudaStream_t st) {
-    constexpr int smem = smem_bytes<kBN>();
-    cudaError_t e = cudaFuncSetAttribute(w4a4_gemm_kernel<kSwiGLU, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem);
+    constexpr int smem = smem_bytes<kBN, kTM>();
+    cudaError_t e = cudaFuncSetAttribute(w4a4_gemm_kernel<kSwiGLU, kBN, kTM>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const int64_t max_tiles = ((a.R + kBM - 1) / kBM + a.n) * static_cast<int64_t>(a.n_tiles);
+    const int64_t max_tiles = ((a.R + kTM - 1) / kTM + a.n) * static_cast<int64_t>(a.n_tiles);
     int64_t g = num_sms;
     if (max_tiles < g) g = max_tiles;
     if (g < 1) g = 1;
-    launch_k(w4a4_gemm_kernel<kSwiGLU, kBN>, dim3(static_cast<unsigned>(g)), dim3(kThreads), smem, st, ta, tb, a);
+    launch_k(w4a4_gemm_kernel<kSwiGLU, kBN, kTM>, dim3(static_cast<unsigned>(g)), dim3(kThreads), smem, st, ta, tb,
+             a);
     return cudaGetLastError();
 }
 
+template <bool kSwiGLU>
+static cudaError_t launch_w4_any(const CUtensorMap& ta, const CUtensorMap& tb, const W4a4GemmArgs& a, bool wide,
+                                 int tile_rows, int num_sms, cudaStream_t st) {
+    if (!wide) {
+        if (tile_rows != 128) return cudaErrorInvalidValue;
+        return launch_w4<kSwiGLU, 128, 128>(ta, tb, a, num_sms, st);
+    }
+    if (tile_rows == 32) return launch_w4<kSwiGLU, 256, 32>(ta, tb, a, num_sms, st);
+    if (tile_rows == 128) return launch_w4<kSwiGLU, 256, 128>(ta, tb, a, num_sms, st);
+    return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_w4a4_gemm1(const CUtensorMap& tm_xq, const CUtensorMap& tm_w13, const W4a4GemmArgs& a, bool wide,
-                              int num_sms, cudaStream_t st) {
-    return wide ? launch_w4<true, 256>(tm_xq, tm_w13, a, num_sms, st)
-                : launch_w4<true, 128>(tm_xq, tm_w13, a, num_sms, st);
+                              int tile_rows, int num_sms, cudaStream_t st) {
+    return launch_w4_any<true>(tm_xq, tm_w13, a, wide, tile_rows, num_sms, st);
 }
 
 cudaError_t launch_w4a4_gemm2(const CUtensorMap& tm_hq, const CUtensorMap& tm_w2, const W4a4GemmArgs& a, bool wide,
-                              int num_sms, cudaStream_t st) {
-    return wide ? launch_w4<false, 256>(tm_hq, tm_w2, a, num_sms, st)
-                : launch_w4<false, 128>(tm_hq, tm_w2, a, num_sms, st);
+                              int tile_rows, int num_sms, cudaStream_t st) {
+    return launch_w4_any<false>(tm_hq, tm_w2, a, wide, tile_rows, num_sms, st);
 }
 
 }  // namespace moe

@@ -233,11 +233,11 @@ cudaError_t launch_w4a4_pack(const uint8_t* codes, const uint8_t* bscale, const 
                              const uint8_t* bscale_pair, int n, int K, int N, uint8_t* packed, uint8_t* chunks,
                              cudaStream_t st);
 //   rows: bf16 rows (row r reads src row row_src[r], or r without row_src) ->
-//   codes [R][K/2], row scales [R], and the chunks of the 128-row GEMM tiles
-//   [tiles][K/64][512] (tile of row r: mblk_base[e] + (r - offsets[e]) / 128).
-//   Rows past offsets[n] are skipped.
+//   codes [R][K/2], row scales [R], and the chunks of the GEMM's tiles of
+//   tile_rows rows (128 or 32) [tiles][K/64][512] (tile of row r: mblk_base[e]
+//   + (r - offsets[e]) / tile_rows).  Rows past offsets[n] are skipped.
 cudaError_t launch_w4a4_rows(const uint16_t* src, const int32_t* row_src, int64_t src_rows, int64_t rows_max, int K,
-                             const int32_t* offsets, const int32_t* mblk_base, int n, uint8_t* codes,
+                             const int32_t* offsets, const int32_t* mblk_base, int n, int tile_rows, uint8_t* codes,
                              uint8_t* chunks, float* rscale, int num_sms, cudaStream_t st);
 
 struct W4a4GemmArgs {
@@ -258,15 +258,17 @@ struct W4a4GemmArgs {
     const uint8_t* b_chunks;   // weight scale chunks [n][rows/128][K/64][512] (w1|w3 pairs, or w2)
 };
 
-// tm_a: activation codes [R][K/2] uint8 (128 x 128 boxes, 128-byte swizzle);
-// tm_b: packed weight codes [n][rows][K/2] uint8 (128 x 128 x 1 boxes, same):
-// the w1|w3 pair pack for GEMM1, w2 for GEMM2.  wide: 256-column tiles (one
-// accumulator) instead of 128-column tiles (two accumulators).
+// tm_a: activation codes [R][K/2] uint8 (boxes of tile_rows rows x 128 bytes,
+// 128-byte swizzle); tm_b: packed weight codes [n][rows][K/2] uint8 (128 x 128
+// x 1 boxes, same): the w1|w3 pair pack for GEMM1, w2 for GEMM2.  wide:
+// 256-column tiles (one accumulator) instead of 128-column tiles (two
+// accumulators); tile_rows: 128, or 32 (wide only) with the segments laid out
+// in 32-row M-blocks.
 int w4a4_tile_cols(bool wide);
 cudaError_t launch_w4a4_gemm1(const CUtensorMap& tm_xq, const CUtensorMap& tm_w13, const W4a4GemmArgs& a, bool wide,
-                              int num_sms, cudaStream_t st);
+                              int tile_rows, int num_sms, cudaStream_t st);
 cudaError_t launch_w4a4_gemm2(const CUtensorMap& tm_hq, const CUtensorMap& tm_w2, const W4a4GemmArgs& a, bool wide,
-                              int num_sms, cudaStream_t st);
+                              int tile_rows, int num_sms, cudaStream_t st);
 
 // E4M3 quantisation (e4m3.cu).  Codes are those of v / scale with the quotient
 // rounded to fp32, then to E4M3 by round-to-nearest-even with saturation to

@@ -111,12 +111,13 @@ bool encode_weights(CUtensorMap* m, const void* base, uint64_t cols, uint64_t ro
 
 // E4M3 codes, uint8: [rows][cols] (box_rows x 128) or weights [n][rows][cols]
 // (128 x 128 boxes of one expert); out-of-range boxes read zeros.
-bool encode_codes(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t n) {
+bool encode_codes(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t n,
+                  uint32_t box_rows = 128) {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
     cuuint64_t dims[3] = {cols, rows, n};
     cuuint64_t strides[2] = {cols, cols * rows};
-    cuuint32_t box[3] = {128, 128, 1};
+    cuuint32_t box[3] = {128, box_rows, 1};
     cuuint32_t es[3] = {1, 1, 1};
     return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, n ? 3 : 2, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -218,6 +219,7 @@ struct moe_handle {
     float* xr4 = nullptr;
     float* hr4 = nullptr;
     CUtensorMap tm_xq4, tm_hq4, tm_wp4[2];
+    CUtensorMap tm_xq4s, tm_hq4s;  // the same codes in 32-row boxes
     const void* c_wp4[2] = {nullptr, nullptr};
     // 4-bit experts: maps over the caller's codes and block scales
     CUtensorMap tm_f4[6];  // codes w1, scales w1, codes w3, scales w3, codes w2, scales w2
@@ -324,7 +326,7 @@ moe_status grow(moe_handle* h, int64_t T, int64_t rows_min = 0) {
     const size_t o_xs = take(e4 ? static_cast<size_t>(R) * 4 : 0);
     const size_t o_hs = take(e4 ? static_cast<size_t>(R) * 4 : 0);
     const bool w4 = h->want_w4a4;
-    const size_t tiles4 = static_cast<size_t>((R + 127) / 128 + h->n);
+    const size_t tiles4 = static_cast<size_t>((R + 31) / 32 + h->n);  // 32-row tiles at most
     const size_t o_xq4 = take(w4 ? static_cast<size_t>(R) * (h->d / 2) : 0);
     const size_t o_hq4 = take(w4 ? static_cast<size_t>(R) * (h->F / 2) : 0);
     const size_t o_xc4 = take(w4 ? tiles4 * (h->d / 64) * 512 : 0);
@@ -392,7 +394,9 @@ moe_status grow(moe_handle* h, int64_t T, int64_t rows_min = 0) {
     h->hr4 = w4 ? reinterpret_cast<float*>(b + o_hr4) : nullptr;
     // 4-bit codes: two per byte, so a row of d codes is d / 2 bytes wide
     if (w4 && (!encode_codes(&h->tm_xq4, h->xq4, h->d / 2, static_cast<uint64_t>(R), 0) ||
-               !encode_codes(&h->tm_hq4, h->hq4, h->F / 2, static_cast<uint64_t>(R), 0)))
+               !encode_codes(&h->tm_hq4, h->hq4, h->F / 2, static_cast<uint64_t>(R), 0) ||
+               !encode_codes(&h->tm_xq4s, h->xq4, h->d / 2, static_cast<uint64_t>(R), 0, 32) ||
+               !encode_codes(&h->tm_hq4s, h->hq4, h->F / 2, static_cast<uint64_t>(R), 0, 32)))
         return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the 4-bit workspace");
     if (e4 && (!encode_codes(&h->tm_x8, h->x8, h->d, static_cast<uint64_t>(R), 0) ||
                !encode_codes(&h->tm_h8, h->h8, h->F, static_cast<uint64_t>(R), 0)))
@@ -702,12 +706,27 @@ moe_status run_experts_w4a4(moe_handle* h, int64_t T, const void* x, const float
                             const uint8_t* const* wc, const float* const* ws, void* y, const int32_t* topk_idx,
                             cudaStream_t st) {
     const int64_t R = T * h->K;
-    cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n, moe::kTcBM, h->db, st, capacity_for(h, T));
+    // 256-column tiles (one accumulator) by default: on the Mixtral decode
+    // and prefill shapes and 128 experts of 2048 x 768 they measured faster
+    // than 128-column tiles with two accumulators, which reload A for every
+    // 64 hidden columns.  Row tiles of 32 when the experts average at most 32
+    // rows: a quarter of the A bytes per stage, and a fifth stage in flight.
+    bool wide = true;
+    if (const char* v = getenv("MOE_W4A4_TILE")) {  // 128 or 256 forces a width
+        if (atoi(v) == 128) wide = false;
+        if (atoi(v) == 256) wide = true;
+    }
+    int tile_rows = (wide && R <= 32 * static_cast<int64_t>(h->n)) ? 32 : 128;
+    if (const char* v = getenv("MOE_W4A4_ROWS")) {  // 32 or 128 forces a height (32: 256-column tiles only)
+        if (atoi(v) == 128) tile_rows = 128;
+        if (atoi(v) == 32 && wide) tile_rows = 32;
+    }
+    cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n, tile_rows, h->db, st, capacity_for(h, T));
     if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
     h->launches += moe::dispatch_kernel_count(R);
     trace_mark(h, 1, st);
     e = moe::launch_w4a4_rows(static_cast<const uint16_t*>(x), h->db.row_token, T, R, h->d, h->db.offsets,
-                              h->db.mblk_base, h->n, h->xq4, h->xc4, h->xr4, h->num_sms, st);
+                              h->db.mblk_base, h->n, tile_rows, h->xq4, h->xc4, h->xr4, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "activation quantisation launch");
     h->launches += 1;
     trace_mark(h, 2, st);
@@ -719,15 +738,6 @@ moe_status run_experts_w4a4(moe_handle* h, int64_t T, const void* x, const float
                 return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for packed 4-bit weights");
             h->c_wp4[m] = wp[m];
         }
-    }
-    // 256-column tiles (one accumulator) by default: on the Mixtral decode
-    // and prefill shapes and 128 experts of 2048 x 768 they measured faster
-    // than 128-column tiles with two accumulators, which reload A for every
-    // 64 hidden columns.
-    bool wide = true;
-    if (const char* v = getenv("MOE_W4A4_TILE")) {  // 128 or 256 forces a width
-        if (atoi(v) == 128) wide = false;
-        if (atoi(v) == 256) wide = true;
     }
     const int bn = moe::w4a4_tile_cols(wide);
     moe::W4a4GemmArgs a1{};
@@ -746,10 +756,11 @@ moe_status run_experts_w4a4(moe_handle* h, int64_t T, const void* x, const float
     a1.mscale1 = ws[1];
     a1.a_chunks = h->xc4;
     a1.b_chunks = wc[0];
-    e = moe::launch_w4a4_gemm1(h->tm_xq4, h->tm_wp4[0], a1, wide, h->num_sms, st);
+    e = moe::launch_w4a4_gemm1(tile_rows == 32 ? h->tm_xq4s : h->tm_xq4, h->tm_wp4[0], a1, wide, tile_rows,
+                               h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
     e = moe::launch_w4a4_rows(static_cast<const uint16_t*>(h->h), nullptr, R, R, h->F, h->db.offsets,
-                              h->db.mblk_base, h->n, h->hq4, h->hc4, h->hr4, h->num_sms, st);
+                              h->db.mblk_base, h->n, tile_rows, h->hq4, h->hc4, h->hr4, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "hidden-row quantisation launch");
     h->launches += 2;
     trace_mark(h, 3, st);
@@ -764,7 +775,8 @@ moe_status run_experts_w4a4(moe_handle* h, int64_t T, const void* x, const float
     a2.mscale1 = ws[2];
     a2.a_chunks = h->hc4;
     a2.b_chunks = wc[1];
-    e = moe::launch_w4a4_gemm2(h->tm_hq4, h->tm_wp4[1], a2, wide, h->num_sms, st);
+    e = moe::launch_w4a4_gemm2(tile_rows == 32 ? h->tm_hq4s : h->tm_hq4, h->tm_wp4[1], a2, wide, tile_rows,
+                               h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
     h->launches += 1;
     trace_mark(h, 4, st);

@@ -17,8 +17,9 @@
 //                      yields both projections of 64 hidden columns.
 //   w4a4_rows_kernel   rows (gathered x rows or hidden rows, bf16) -> E2M1 codes
 //                      [R][K/2], a fp32 scale per row, and the scale chunks of
-//                      the GEMM's 128-row tiles: row r of expert e's segment
-//                      lands in tile mblk_base[e] + (r - offsets[e]) / 128.
+//                      the GEMM's tiles of 128 (or 32) rows: row r of expert
+//                      e's segment lands in tile mblk_base[e] + (r -
+//                      offsets[e]) / tile_rows.
 //   Row quantisation: rs = max|row| / (6 * 448) (1 for a zero row), block scale
 //   sb = E4M3((max|block| / 6) / rs), code = E2M1(v / (sb * rs)) (0 when the
 //   product is 0), every quotient and product rounded to fp32.
@@ -99,7 +100,7 @@ __global__ void __launch_bounds__(kW4RowThreads) w4a4_rows_kernel(const uint16_t
                                                                   int64_t src_rows, int K,
                                                                   const int32_t* __restrict__ offsets,
                                                                   const int32_t* __restrict__ mblk_base, int n,
-                                                                  uint8_t* __restrict__ codes,
+                                                                  int tile_rows, uint8_t* __restrict__ codes,
                                                                   uint8_t* __restrict__ chunks,
                                                                   float* __restrict__ rscale) {
     griddep_wait();
@@ -146,8 +147,8 @@ __global__ void __launch_bounds__(kW4RowThreads) w4a4_rows_kernel(const uint16_t
                 hi = mid - 1;
         }
         const int64_t local = r - offsets[lo];
-        const int64_t tile = mblk_base[lo] + local / 128;
-        const int tr = static_cast<int>(local & 127);
+        const int64_t tile = mblk_base[lo] + local / tile_rows;
+        const int tr = static_cast<int>(local % tile_rows);
         for (int b = tid; b < nblk; b += kW4RowThreads) {
             float v[16];
             float amax_b = 0.f;
@@ -185,13 +186,14 @@ __global__ void __launch_bounds__(kW4RowThreads) w4a4_rows_kernel(const uint16_t
 }
 
 cudaError_t launch_w4a4_rows(const uint16_t* src, const int32_t* row_src, int64_t src_rows, int64_t rows_max, int K,
-                             const int32_t* offsets, const int32_t* mblk_base, int n, uint8_t* codes,
+                             const int32_t* offsets, const int32_t* mblk_base, int n, int tile_rows, uint8_t* codes,
                              uint8_t* chunks, float* rscale, int num_sms, cudaStream_t st) {
+    if (tile_rows != 128 && tile_rows != 32) return cudaErrorInvalidValue;
     int64_t blocks = rows_max;
     if (blocks > static_cast<int64_t>(num_sms) * 8) blocks = static_cast<int64_t>(num_sms) * 8;
     if (blocks < 1) blocks = 1;
     launch_k(w4a4_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kW4RowThreads), 0, st, src, row_src,
-             src_rows, K, offsets, mblk_base, n, codes, chunks, rscale);
+             src_rows, K, offsets, mblk_base, n, tile_rows, codes, chunks, rscale);
     return cudaGetLastError();
 }
 

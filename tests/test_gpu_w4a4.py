@@ -116,14 +116,16 @@ FWD_CASES = [
 ]
 
 
-@pytest.mark.parametrize("tile", ["128", "256"])
+@pytest.mark.parametrize("tile", ["128x128", "256x128", "256x32"])
 @pytest.mark.parametrize("case", FWD_CASES, ids=[c[0] for c in FWD_CASES])
 def test_w4a4_layer_matches_oracle(case, tile, monkeypatch):
-    """Both tile widths (128 packed columns with two accumulators, 256 with
-    one) on every case."""
+    """Every tile shape on every case: 128 packed columns with two
+    accumulators, 256 with one, and 256 columns over 32-row tiles."""
     import sparse_mixture_experts_24_b200 as m
     torch = require_cuda()
-    monkeypatch.setenv("MOE_W4A4_TILE", tile)
+    cols, rows = tile.split("x")
+    monkeypatch.setenv("MOE_W4A4_TILE", cols)
+    monkeypatch.setenv("MOE_W4A4_ROWS", rows)
     name, T, d, F, n, K = case
     cfg = mi.custom_config(name, T=T, d=d, ffn=F, n=n, K=K, dtype="bf16")
     L = mi.make_layer(cfg, seed=seed_of(name))
