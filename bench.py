@@ -137,8 +137,8 @@ def recorded_traffic(kernel, config):
     p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(p):
         return None
-    src = os.path.join(ROOT, "sparse_mixture_experts_24_b200", "csrc", "gemm_tc.cu")
-    sha = source_sha(src)
+    src_file = "gemm_w4a4.cu" if config.endswith("_w4a4") else "gemm_tc.cu"
+    sha = source_sha(os.path.join(ROOT, "sparse_mixture_experts_24_b200", "csrc", src_file))
     with open(p) as f:
         for line in f:
             parts = line.split()
