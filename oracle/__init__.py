@@ -8,6 +8,8 @@ Functions (all inputs numpy arrays; x and weights may be float32, float64 or
 bf16 bit patterns stored as uint16, and are widened exactly to double):
 
   router(x, W_g, K)                     -> idx [T,K] int32, gate [T,K] f64, logits [T,n] f64
+  gates_to_bf16(gate)                   -> the gates cast to bf16 as the quoted routing code
+                                           does (fp64 -> fp32 -> bf16, nearest even), as f64
   expert(x_row, w1, w3, w2, e)          -> [d] f64, one SwiGLU expert on one token
   forward_with_routing(x, idx, gate, w1, w3, w2) -> y [T,d] f64
   moe_forward(x, W_g, w1, w3, w2, K)    -> y, idx, gate
@@ -55,6 +57,7 @@ def build(force: bool = False) -> str:
 def _bind(L):
     vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
     L.oracle_router.argtypes = [i64, i32, i32, i32, vp, i32, vp, i32, vp, vp, vp]
+    L.oracle_gates_to_bf16.argtypes = [i64, vp, vp]
     L.oracle_expert.argtypes = [i32, i32, i32, i32, vp, i32, vp, vp, vp, i32, vp]
     L.oracle_forward_with_routing.argtypes = [i64, i32, i32, i32, i32, vp, i32, vp, vp,
                                               vp, vp, vp, i32, vp]
@@ -148,6 +151,12 @@ class Oracle:
         _check(self.L.oracle_router(T, d, n, K, _p(x), _dt(x), _p(W_g), _dt(W_g),
                                     _p(idx), _p(gate), _p(logits)), "router")
         return idx, gate, logits
+
+    def gates_to_bf16(self, gate):
+        gate = np.ascontiguousarray(gate, dtype=np.float64)
+        out = np.empty_like(gate)
+        _check(self.L.oracle_gates_to_bf16(gate.size, _p(gate), _p(out)), "gates_to_bf16")
+        return out
 
     def expert(self, x_row, w1, w3, w2, e: int):
         x_row, w1, w3, w2 = _c(x_row), _c(w1), _c(w3), _c(w2)
@@ -376,6 +385,10 @@ def silu(z: float) -> float:
 
 def router(x, W_g, K: int):
     return default().router(x, W_g, K)
+
+
+def gates_to_bf16(gate):
+    return default().gates_to_bf16(gate)
 
 
 def expert(x_row, w1, w3, w2, e: int):

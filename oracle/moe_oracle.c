@@ -180,6 +180,35 @@ static void expert_one(int d, int F, const void *x, int x_dt, size_t xoff,
     }
 }
 
+/* Gates in the activations' dtype: the routing code quoted in Part 3 of the
+ * neobadger page computes the softmax in fp32 and then casts the weights to
+ * the inputs' dtype.  For bf16 inputs each gate becomes: the fp64 gate rounded
+ * to fp32 (round to nearest even), then that float rounded to bf16 (its upper
+ * 16 bits, round to nearest even on the 16 dropped bits). */
+int oracle_gates_to_bf16(int64_t count, const double *gate, double *out)
+{
+    if (count < 0 || (count > 0 && (!gate || !out)))
+        return -1;
+    for (int64_t i = 0; i < count; ++i) {
+        float f = (float)gate[i];
+        uint32_t u;
+        memcpy(&u, &f, sizeof u);
+        if ((u & 0x7f800000u) == 0x7f800000u) { /* inf or nan: keep (not reached by gates) */
+            out[i] = (double)f;
+            continue;
+        }
+        uint32_t low = u & 0xffffu;
+        uint32_t hi = u >> 16;
+        if (low > 0x8000u || (low == 0x8000u && (hi & 1u)))
+            hi += 1u; /* carries into the exponent when the mantissa overflows */
+        uint32_t r = hi << 16;
+        float g;
+        memcpy(&g, &r, sizeof g);
+        out[i] = (double)g;
+    }
+    return 0;
+}
+
 int oracle_expert(int d, int F, int n, int e, const void *x_row, int x_dt,
                   const void *w1, const void *w3, const void *w2, int w_dt, double *out)
 {

@@ -149,6 +149,31 @@ def check_gate_invariants(O):
             assert np.all(gate == 1.0)
 
 
+def check_gates_to_bf16(O):
+    """The routing code quoted in [P5] Part 3 computes the softmax in fp32 and
+    casts the weights to the inputs' dtype.  Pins of that cast: the worked
+    example's gates 0.689974 / 0.310026 (printed 0.69 / 0.31) become
+    177/256 and 159/512 (nearest bf16); halfway cases go to the even mantissa;
+    a double just above a bf16 halfway point that rounds onto it in fp32 then
+    goes to the even neighbour (fp32 first, then bf16); values already in bf16
+    are unchanged, and torch's fp32 -> bf16 cast agrees on random gates."""
+    import torch
+    g = O.gates_to_bf16(np.array([0.689974, 0.310026]))
+    assert g[0] == 177 / 256 and g[1] == 159 / 512, g
+    # ulp of bf16 is 2^-7 on [1, 2) and 2^-8 on [0.5, 1): these sit halfway
+    ties = O.gates_to_bf16(np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, 0.5 + 2.0 ** -9, 0.5 + 3 * 2.0 ** -9]))
+    assert list(ties) == [1.0, 1 + 2.0 ** -6, 0.5, 0.5 + 2.0 ** -7], ties
+    # fp32 first: 1 + 2^-8 + 2^-30 is 1 + 2^-8 in fp32 (a tie in bf16 -> 1.0),
+    # while rounding the double straight to bf16 would give 1 + 2^-7
+    assert O.gates_to_bf16(np.array([1 + 2.0 ** -8 + 2.0 ** -30]))[0] == 1.0
+    exact = np.array([1.0, 0.5, 0.75, 2.0 ** -20, 0.0])
+    assert np.array_equal(O.gates_to_bf16(exact), exact)
+    rng = np.random.default_rng(21)
+    r = rng.random(4096)
+    ref = torch.from_numpy(r).float().to(torch.bfloat16).double().numpy()
+    assert np.array_equal(O.gates_to_bf16(r), ref)
+
+
 # --------------------------------------------------------------------------
 # Experts and the combine
 # --------------------------------------------------------------------------
@@ -704,7 +729,7 @@ def check_w4a4_zero_rows_and_scaling(O):
 
 ALL_CHECKS = [
     check_worked_example, check_two_way_softmax_closed_form, check_logits_are_x_times_Wg,
-    check_topk_brute_force, check_ties_go_to_lower_index, check_gate_invariants, check_silu,
+    check_topk_brute_force, check_ties_go_to_lower_index, check_gate_invariants, check_gates_to_bf16, check_silu,
     check_n1_is_plain_swiglu, check_expert_indexing, check_K_equals_n_is_dense_mixture,
     check_top2_layer_against_torch, check_relabel_invariance,
     check_unchosen_experts_do_not_matter, check_forward_with_routing_consistent,

@@ -48,6 +48,11 @@ MUTANTS = {
                                       "int sb_code = oracle_e4m3_encode((double)(amax_b / rs));")],
     "e4m3_scale_over_256": [("amax / 448.0f", "amax / 256.0f")],
     "e4m3_bias_8": [("v = ldexp(1.0 + m / 8.0, e - 7);", "v = ldexp(1.0 + m / 8.0, e - 8);")],
+    "gates_bf16_truncate": [("if (low > 0x8000u || (low == 0x8000u && (hi & 1u)))", "if (0)")],
+    "gates_bf16_ties_up": [("if (low > 0x8000u || (low == 0x8000u && (hi & 1u)))", "if (low >= 0x8000u)")],
+    # straight from double to bf16: the bits lost in the fp32 step break a bf16 tie
+    "gates_bf16_no_fp32_step": [("if (low > 0x8000u || (low == 0x8000u && (hi & 1u)))",
+                                 "if (low > 0x8000u || (low == 0x8000u && ((hi & 1u) || (double)f < gate[i])))")],
     "capacity_keeps_one_more": [("if (row - offsets[e] < capacity) {", "if (row - offsets[e] <= capacity) {")],
 }
 
