@@ -159,6 +159,17 @@ MOE_API moe_status moe_forward_with_routing(moe_handle *h, int64_t T, const void
                                     moe_stream_t stream);
 
 /*
+ * Gate precision.  bf16 = 1: after the fp32 softmax, every topk_w is rounded to
+ * bf16 (nearest even) and kept as an fp32 value, as the routing code quoted in
+ * Part 3 of the neobadger page casts the weights to the inputs' dtype; the
+ * combine then uses those gates.  bf16 = 0 (the default): fp32 gates.  Applies
+ * to every later call that routes (moe_forward, moe_route and the
+ * low-precision forwards).
+ *   Errors: MOE_ERR_INVALID_ARG (null handle, bf16 not 0 or 1).
+ */
+MOE_API moe_status moe_set_gate_rounding(moe_handle *h, int bf16);
+
+/*
  * Expert capacity (Part 5 of the neobadger page, "What happens when an expert
  * is full", after the Switch paper: capacity = tokens in the batch / experts x
  * a capacity factor).  With factor > 0, each later forward / dispatch call on

@@ -59,6 +59,7 @@ lib.moe_forward_expert_choice.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _
 lib.moe_selftest_timeout.argtypes = [_vp, _int, _vp]
 lib.moe_launch_count.argtypes = [_vp, ctypes.POINTER(_i64)]
 lib.moe_set_capacity_factor.argtypes = [_vp, ctypes.c_double]
+lib.moe_set_gate_rounding.argtypes = [_vp, _int]
 lib.moe_router_stats.argtypes = [_vp, _i64, _vp, _vp, _vp, ctypes.c_float, _vp, _vp, _vp, _vp]
 lib.moe_dispatch_noalloc.argtypes = [_i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.moe_trace_end.argtypes = [_vp, ctypes.POINTER(ctypes.c_double), _int, ctypes.POINTER(_int)]
@@ -83,7 +84,7 @@ for _f in ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatc
            "moe_forward_expert_choice", "moe_quantize_weights_e4m3", "moe_forward_e4m3",
            "moe_quantize_weights_fp4", "moe_forward_fp4", "moe_pack_weights_w4a4", "moe_forward_w4a4",
            "moe_ep_dispatch", "moe_ep_experts", "moe_ep_combine", "moe_ep_buffer_alloc", "moe_ep_buffer_open",
-           "moe_ep_buffer_close"):
+           "moe_ep_buffer_close", "moe_set_gate_rounding"):
     getattr(lib, _f).restype = _int
 
 EXPORTED = ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatch",
@@ -93,7 +94,7 @@ EXPORTED = ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispat
             "moe_launch_count", "moe_selftest_timeout", "moe_forward_expert_choice",
             "moe_quantize_weights_e4m3", "moe_forward_e4m3", "moe_quantize_weights_fp4", "moe_forward_fp4",
             "moe_pack_weights_w4a4", "moe_forward_w4a4", "moe_ep_dispatch", "moe_ep_experts", "moe_ep_combine",
-            "moe_ep_buffer_alloc", "moe_ep_buffer_open", "moe_ep_buffer_close")
+            "moe_ep_buffer_alloc", "moe_ep_buffer_open", "moe_ep_buffer_close", "moe_set_gate_rounding")
 
 TRACE_STAGES = ("router", "dispatch", "gather", "gemm1", "gemm2", "combine")
 
@@ -347,6 +348,10 @@ def moe_ep_buffer_close(ptr: int, opened: bool) -> None:
     _check(lib.moe_ep_buffer_close(ptr, 1 if opened else 0), "moe_ep_buffer_close")
 
 
+def moe_set_gate_rounding(h, bf16: int) -> None:
+    _check(lib.moe_set_gate_rounding(h, bf16), "moe_set_gate_rounding")
+
+
 def moe_destroy(h) -> None:
     _check(lib.moe_destroy(h), "moe_destroy")
 
@@ -459,6 +464,9 @@ class MoELayer:
 
     def set_capacity_factor(self, factor: float) -> None:
         moe_set_capacity_factor(self.h, factor)
+
+    def set_gate_rounding(self, bf16: bool) -> None:
+        moe_set_gate_rounding(self.h, 1 if bf16 else 0)
 
     def router_stats(self, x, W_g, topk_idx, alpha=0.01, stream=None):
         """-> f [n], P [n], aux [1] (device float32 tensors)."""

@@ -150,6 +150,9 @@ cudaError_t launch_simt_gemm2(const float* h, const float* w2, float* o, const i
 
 // tcgen05 grouped GEMMs (bf16 handles).  Tensor maps are built by the host
 // (see moe_api.cu) over: Xp [R_cap][d], w1/w3 [n][d][F], H [R_cap][F], w2 [n][F][d].
+// Gates rounded to bf16 in place (router.cu).
+cudaError_t launch_gates_to_bf16(float* topk_w, int64_t count, int num_sms, cudaStream_t st);
+
 // Expert parallelism (ep.cu): one device pointer per rank, by value.
 constexpr int kMaxEpRanks = 16;
 struct EpPeers {

@@ -189,6 +189,7 @@ struct moe_handle {
     int c_ew_nl = 0;
     // expert capacity factor (0: dropless) and load-balancing statistics scratch
     double capacity_factor = 0.0;
+    bool gates_bf16 = false;  // moe_set_gate_rounding
     // kernels this handle has launched (for profiling and launch accounting)
     int64_t launches = 0;
     float* stats_partial = nullptr;
@@ -453,6 +454,11 @@ moe_status run_router(moe_handle* h, int64_t T, const void* x, const float* W_g,
         h->launches += h->n > 32 ? 2 : 1;
     }
     if (e != cudaSuccess) return cuda_fail(e, "router launch");
+    if (h->gates_bf16) {
+        e = moe::launch_gates_to_bf16(topk_w, T * h->K, h->num_sms, st);
+        if (e != cudaSuccess) return cuda_fail(e, "gate rounding launch");
+        h->launches += 1;
+    }
     return MOE_OK;
 }
 
@@ -1378,6 +1384,13 @@ moe_status moe_ep_buffer_close(void* ptr, int opened) {
     if (!ptr) return ok();
     cudaError_t e = opened ? cudaIpcCloseMemHandle(ptr) : cudaFree(ptr);
     if (e != cudaSuccess) return cuda_fail(e, opened ? "cudaIpcCloseMemHandle" : "cudaFree");
+    return ok();
+}
+
+moe_status moe_set_gate_rounding(moe_handle* h, int bf16) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "null handle");
+    if (bf16 != 0 && bf16 != 1) return fail(MOE_ERR_INVALID_ARG, "bf16 = %d is neither 0 nor 1", bf16);
+    h->gates_bf16 = bf16 == 1;
     return ok();
 }
 

@@ -438,6 +438,26 @@ cudaError_t launch_router_logits_simt(const void* x, bool x_bf16, const float* W
     return cudaGetLastError();
 }
 
+// Gates cast to bf16 (round to nearest even) and kept as fp32 values: the
+// routing code quoted in Part 3 of "Mixture of Experts: Why Mixtral Only Wakes
+// Up Two Specialists" computes the softmax in fp32 and casts the weights to
+// the inputs' dtype.
+__global__ void __launch_bounds__(256) gates_to_bf16_kernel(float* __restrict__ w, int64_t count) {
+    griddep_wait();
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count; i += stride)
+        w[i] = __bfloat162float(__float2bfloat16_rn(w[i]));
+    griddep_launch_dependents();
+}
+
+cudaError_t launch_gates_to_bf16(float* topk_w, int64_t count, int num_sms, cudaStream_t st) {
+    int64_t blocks = (count + 255) / 256;
+    if (blocks > static_cast<int64_t>(num_sms) * 4) blocks = static_cast<int64_t>(num_sms) * 4;
+    if (blocks < 1) blocks = 1;
+    launch_k(gates_to_bf16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, topk_w, count);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_router(const void* x, bool x_bf16, const float* Wg, int64_t T, int d, int n,
                           int K, int32_t* topk_idx, float* topk_w, float* logits_ws, int num_sms,
                           cudaStream_t st) {
