@@ -185,10 +185,127 @@ __global__ void __launch_bounds__(kW4RowThreads) w4a4_rows_kernel(const uint16_t
     griddep_launch_dependents();
 }
 
+// Rows of up to 32 * 16 * kBPL elements: one warp per row, lane = blocks of 16
+// (b = lane + 32 i), the whole row held in registers, so there is one read of
+// the row, a warp-shuffle maximum and no block barrier.  Same arithmetic as
+// w4a4_rows_kernel.
+template <int kBPL>
+__global__ void __launch_bounds__(256) w4a4_rows_warp_kernel(const uint16_t* __restrict__ src,
+                                                             const int32_t* __restrict__ row_src,
+                                                             int64_t src_rows, int K,
+                                                             const int32_t* __restrict__ offsets,
+                                                             const int32_t* __restrict__ mblk_base, int n,
+                                                             int tile_rows, uint8_t* __restrict__ codes,
+                                                             uint8_t* __restrict__ chunks,
+                                                             float* __restrict__ rscale) {
+    griddep_wait();
+    const int lane = threadIdx.x & 31;
+    const int64_t rows = offsets[n];
+    const int nblk = K / 16;
+    const int KB = K / 64;
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+         r += warps) {
+        int64_t s = r;
+        if (row_src) {
+            s = __ldg(row_src + r);
+            if (s < 0 || s >= src_rows) continue;  // warp-uniform
+        }
+        const uint4* row = reinterpret_cast<const uint4*>(src + s * K);
+        uint4 q[kBPL][2];
+        float m = 0.f;
+#pragma unroll
+        for (int i = 0; i < kBPL; ++i) {
+            const int b = lane + 32 * i;
+            if (b < nblk) {
+                q[i][0] = __ldg(row + 2 * b);
+                q[i][1] = __ldg(row + 2 * b + 1);
+            } else {
+                q[i][0] = q[i][1] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+        float amax_b[kBPL];
+#pragma unroll
+        for (int i = 0; i < kBPL; ++i) {
+            float a = 0.f;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t w[4] = {q[i][h].x, q[i][h].y, q[i][h].z, q[i][h].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    a = fmaxf(a, fabsf(__uint_as_float(w[j] << 16)));
+                    a = fmaxf(a, fabsf(__uint_as_float(w[j] & 0xFFFF0000u)));
+                }
+            }
+            amax_b[i] = a;
+            m = fmaxf(m, a);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const float rs = w4_tensor_scale(m);
+        int lo = 0, hi = n - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (offsets[mid] <= r)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        const int64_t local = r - offsets[lo];
+        const int64_t tile = mblk_base[lo] + local / tile_rows;
+        const int tr = static_cast<int>(local % tile_rows);
+#pragma unroll
+        for (int i = 0; i < kBPL; ++i) {
+            const int b = lane + 32 * i;
+            if (b >= nblk) continue;
+            const uint32_t sb = static_cast<uint32_t>(
+                __nv_cvt_float_to_fp8(__fdiv_rn(__fdiv_rn(amax_b[i], 6.f), rs), __NV_SATFINITE, __NV_E4M3));
+            const float denom = __fmul_rn(w4_e4m3_value(sb), rs);
+            uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t w[4] = {q[i][h].x, q[i][h].y, q[i][h].z, q[i][h].w};
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float v = (j & 1) ? __uint_as_float(w[j >> 1] & 0xFFFF0000u) : __uint_as_float(w[j >> 1] << 16);
+                    const uint32_t c =
+                        denom == 0.f ? 0u
+                                     : static_cast<uint32_t>(__nv_cvt_float_to_fp4(__fdiv_rn(v, denom), __NV_E2M1,
+                                                                                   cudaRoundNearest)) & 0xFu;
+                    packed[h] |= c << (4 * j);
+                }
+            }
+            *reinterpret_cast<uint2*>(codes + r * (K / 2) + 8 * b) = make_uint2(packed[0], packed[1]);
+            chunks[(tile * KB + b / 4) * 512 + w4_chunk_byte(tr, b & 3)] = static_cast<uint8_t>(sb);
+        }
+        if (lane == 0) rscale[r] = rs;
+    }
+    griddep_launch_dependents();
+}
+
 cudaError_t launch_w4a4_rows(const uint16_t* src, const int32_t* row_src, int64_t src_rows, int64_t rows_max, int K,
                              const int32_t* offsets, const int32_t* mblk_base, int n, int tile_rows, uint8_t* codes,
                              uint8_t* chunks, float* rscale, int num_sms, cudaStream_t st) {
     if (tile_rows != 128 && tile_rows != 32) return cudaErrorInvalidValue;
+    // Many rows of at most 2,048 elements: a warp per row, the row in
+    // registers (measured: many_expert x rows 82 -> 51 us, its H rows and
+    // GEMM1 139 -> 85 us).  Longer rows, or few of them, keep a block per row:
+    // a warp per 4,096-element row ran the decode x rows at half the speed
+    // (64 rows: too few warps in flight) and the prefill ones 1.5x slower.
+    const int bpl = (K / 16 + 31) / 32;
+    if (bpl <= 4 && rows_max >= 4LL * num_sms) {
+        int64_t wblocks = (rows_max + 7) / 8;
+        if (wblocks > static_cast<int64_t>(num_sms) * 8) wblocks = static_cast<int64_t>(num_sms) * 8;
+        if (wblocks < 1) wblocks = 1;
+        const dim3 g(static_cast<unsigned>(wblocks));
+        if (bpl <= 2)
+            launch_k(w4a4_rows_warp_kernel<2>, g, dim3(256), 0, st, src, row_src, src_rows, K, offsets, mblk_base, n,
+                     tile_rows, codes, chunks, rscale);
+        else
+            launch_k(w4a4_rows_warp_kernel<4>, g, dim3(256), 0, st, src, row_src, src_rows, K, offsets, mblk_base, n,
+                     tile_rows, codes, chunks, rscale);
+        return cudaGetLastError();
+    }
     int64_t blocks = rows_max;
     if (blocks > static_cast<int64_t>(num_sms) * 8) blocks = static_cast<int64_t>(num_sms) * 8;
     if (blocks < 1) blocks = 1;

@@ -113,6 +113,7 @@ FWD_CASES = [
     ("w4a4_T1", 1, 256, 256, 8, 2),
     ("w4a4_n64", 700, 256, 256, 64, 4),
     ("w4a4_big_segments", 1500, 512, 768, 4, 2),
+    ("w4a4_d2048_rows", 400, 2048, 256, 8, 2),   # 800 rows of 2,048: the warp-per-row quantiser
 ]
 
 
