@@ -30,6 +30,14 @@
 //            arrives on the leader's accumulator-empty barrier (8 arrivals).
 // Every wait is bounded; both CTAs pass a cluster barrier before exit so that
 // no remote arrive can target a CTA that has already left.
+//
+// E4M3 variant (kFp8): a stage is 128 K-elements of one-byte codes (A: this
+// CTA's 128 rows x 128 bytes; B: this CTA's 128 columns x 128 K-rows, N-major,
+// one box), four tcgen05.mma.cta_group::2.kind::f8f6f4 (K = 32) per stage, and
+// the epilogue of gemm_tc.cu's E4M3 kernels (accumulator x row scale x column
+// scale).  At the fp8 rate the single-SM 128 x 256 tile has to stream its
+// operands through shared memory twice as fast per FLOP as bf16; the pair tile
+// halves the B bytes each SM streams.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -38,6 +46,7 @@ namespace moe {
 constexpr int kPairBM = 256;                       // rows per pair tile
 constexpr int kPairBN = 256;                       // pair MMA N
 constexpr int kPairBK = 64;
+constexpr int kPairBK8 = 128;                      // K per stage of the E4M3 pair kernels (128 bytes)
 constexpr int kPairStages = 6;
 constexpr int kPairABytes = 128 * kPairBK * 2;     // 16 KB: this CTA's 128 rows
 constexpr int kPairBChunk = kPairBK * 64 * 2;      // 8 KB: 64 K-rows x 64 columns
@@ -90,7 +99,7 @@ __device__ __forceinline__ PairTile pair_tile(int t, const int32_t* off, const i
 
 __device__ __forceinline__ float silu_pair(float a) { return a / (1.f + __expf(-a)); }
 
-template <bool kSwiGLU>
+template <bool kSwiGLU, bool kFp8>
 __global__ void __launch_bounds__(kPairThreads, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
                         const __grid_constant__ CUtensorMap tm_b1, const TcGemmArgs args) {
@@ -163,9 +172,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     const uint32_t full_leader = mapa_shared(full_local, 0);
                     const uint32_t a_dst = smem_u32(smem + stage * kPairStageBytes);
                     const uint32_t b_dst = a_dst + kPairABytes;
-                    const int k0 = kb * kPairBK;
+                    const int k0 = kb * (kFp8 ? kPairBK8 : kPairBK);
                     tma_load_2d_pair(a_dst, &tm_a, full_leader, k0, pt.row0 + 128 * static_cast<int>(rank));
-                    if (kSwiGLU) {
+                    if (kFp8) {
+                        // one 128 x 128 box: 128 K-rows of this CTA's 128 columns
+                        const CUtensorMap* src = (kSwiGLU && rank != 0) ? &tm_b1 : &tm_b0;
+                        const int c0 = kSwiGLU ? pt.n_tile * 128 : pt.n_tile * kPairBN + 128 * static_cast<int>(rank);
+                        tma_load_3d_pair(b_dst, src, full_leader, c0, k0, pt.e);
+                    } else if (kSwiGLU) {
                         const CUtensorMap* src = rank == 0 ? &tm_b0 : &tm_b1;
                         const int c0 = pt.n_tile * 128;
                         tma_load_3d_pair(b_dst, src, full_leader, c0, k0, pt.e);
@@ -192,7 +206,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
             // ---------------- pair MMA issuer (leader only) ----------------
-            constexpr uint32_t idesc = make_idesc_bf16(kPairBM, kPairBN, 0, 1);
+            constexpr uint32_t idesc =
+                kFp8 ? make_idesc_e4m3(kPairBM, kPairBN, 0, 1) : make_idesc_bf16(kPairBM, kPairBN, 0, 1);
             int stage = 0;
             uint32_t phase = 0;
             int local = 0;
@@ -214,11 +229,22 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     tc_fence_after();
                     const uint32_t a_base = smem_u32(smem + stage * kPairStageBytes);
                     const uint32_t b_base = a_base + kPairABytes;
+                    if (kFp8) {
 #pragma unroll
-                    for (int kk = 0; kk < kPairBK / 16; ++kk) {
-                        const uint64_t adesc = make_smem_desc(a_base + kk * 32, 16, 1024, 2);
-                        const uint64_t bdesc = make_smem_desc(b_base + kk * 2048, kPairBChunk, 1024, 2);
-                        tc_mma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        for (int kk = 0; kk < kPairBK8 / 32; ++kk) {
+                            // A: K-major, K by 32 one-byte codes = 32 bytes inside the swizzle
+                            // row; B: N-major, one 128-column chunk, K by 32 = four 8-row groups
+                            const uint64_t adesc = make_smem_desc(a_base + kk * 32, 16, 1024, 2);
+                            const uint64_t bdesc = make_smem_desc(b_base + kk * 4096, kPairBBytes, 1024, 2);
+                            tc_mma_f8_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        }
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < kPairBK / 16; ++kk) {
+                            const uint64_t adesc = make_smem_desc(a_base + kk * 32, 16, 1024, 2);
+                            const uint64_t bdesc = make_smem_desc(b_base + kk * 2048, kPairBChunk, 1024, 2);
+                            tc_mma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        }
                     }
                     const uint32_t eb = smem_u32(&tail->empty[stage]);
                     tc_commit_pair(mapa_shared(eb, 0));
@@ -261,6 +287,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 // GEMM1: direct 16-byte stores of each lane's row (measured faster here
                 // than staging through shared memory)
                 const bool row_ok = lane < valid;
+                const float rs = (kFp8 && row_ok) ? args.row_scale[row_base + lane] : 1.f;
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t a[32], b[32];
@@ -269,6 +296,25 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     tmem_wait_ld();
                     const int col = pt.n_tile * 128 + c * 32;
                     if (row_ok && col < args.out_cols) {
+                        if (kFp8) {
+                            // dequantise: accumulator x row scale x column scale
+                            const float4* s0 = reinterpret_cast<const float4*>(
+                                args.col_scale0 + static_cast<int64_t>(pt.e) * args.out_cols + col);
+                            const float4* s1 = reinterpret_cast<const float4*>(
+                                args.col_scale1 + static_cast<int64_t>(pt.e) * args.out_cols + col);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                const float4 u = __ldg(s0 + q), v = __ldg(s1 + q);
+                                a[4 * q + 0] = __float_as_uint(__uint_as_float(a[4 * q + 0]) * rs * u.x);
+                                a[4 * q + 1] = __float_as_uint(__uint_as_float(a[4 * q + 1]) * rs * u.y);
+                                a[4 * q + 2] = __float_as_uint(__uint_as_float(a[4 * q + 2]) * rs * u.z);
+                                a[4 * q + 3] = __float_as_uint(__uint_as_float(a[4 * q + 3]) * rs * u.w);
+                                b[4 * q + 0] = __float_as_uint(__uint_as_float(b[4 * q + 0]) * rs * v.x);
+                                b[4 * q + 1] = __float_as_uint(__uint_as_float(b[4 * q + 1]) * rs * v.y);
+                                b[4 * q + 2] = __float_as_uint(__uint_as_float(b[4 * q + 2]) * rs * v.z);
+                                b[4 * q + 3] = __float_as_uint(__uint_as_float(b[4 * q + 3]) * rs * v.w);
+                            }
+                        }
                         uint32_t pk[16];
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
@@ -284,19 +330,32 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     }
                 }
             } else {
+                const float rs = (kFp8 && lane < valid) ? args.row_scale[row_base + lane] : 1.f;
 #pragma unroll 1
                 for (int g = 0; g < 4; ++g) {
                     uint32_t pk[32];
+                    const int col = pt.n_tile * kPairBN + g * 64;
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
                         uint32_t a[32];
                         tmem_ld_32x32b_x32(tbase + g * 64 + c * 32, a);
                         tmem_wait_ld();
+                        if (kFp8 && col < args.out_cols) {
+                            const float4* s0 = reinterpret_cast<const float4*>(
+                                args.col_scale0 + static_cast<int64_t>(pt.e) * args.out_cols + col + c * 32);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                const float4 u = __ldg(s0 + q);
+                                a[4 * q + 0] = __float_as_uint(__uint_as_float(a[4 * q + 0]) * rs * u.x);
+                                a[4 * q + 1] = __float_as_uint(__uint_as_float(a[4 * q + 1]) * rs * u.y);
+                                a[4 * q + 2] = __float_as_uint(__uint_as_float(a[4 * q + 2]) * rs * u.z);
+                                a[4 * q + 3] = __float_as_uint(__uint_as_float(a[4 * q + 3]) * rs * u.w);
+                            }
+                        }
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
                             pk[c * 16 + j] = pack_bf16x2(__uint_as_float(a[2 * j]), __uint_as_float(a[2 * j + 1]));
                     }
-                    const int col = pt.n_tile * kPairBN + g * 64;
                     if (col < args.out_cols && valid > 0)
                         warp_store_rows_64(stage, pk, lane, out, args.out_cols, row_base, valid, col);
                 }
@@ -318,10 +377,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     }
 }
 
-template <bool kSwiGLU>
+template <bool kSwiGLU, bool kFp8>
 static cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1,
                                const TcGemmArgs& a, int num_sms, cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(tc_gemm_pair_kernel<kSwiGLU>,
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_pair_kernel<kSwiGLU, kFp8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes);
     if (e != cudaSuccess) return e;
     const int64_t max_tiles = ((a.R + kPairBM - 1) / kPairBM + a.n) * static_cast<int64_t>(a.n_tiles);
@@ -343,18 +402,29 @@ static cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb0, co
     cfg.attrs = attr;
     cfg.numAttrs = (g_chain_started && pdl_enabled()) ? 2 : 1;
     g_chain_started = true;
-    return cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<kSwiGLU>, ta, tb0, tb1, a);
+    return cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<kSwiGLU, kFp8>, ta, tb0, tb1, a);
 }
 
 cudaError_t launch_tc_gemm1_pair(const CUtensorMap& tm_xp, const CUtensorMap& tm_w1,
                                  const CUtensorMap& tm_w3, const TcGemmArgs& a, int num_sms,
                                  cudaStream_t st) {
-    return launch_pair<true>(tm_xp, tm_w1, tm_w3, a, num_sms, st);
+    return launch_pair<true, false>(tm_xp, tm_w1, tm_w3, a, num_sms, st);
 }
 
 cudaError_t launch_tc_gemm2_pair(const CUtensorMap& tm_h, const CUtensorMap& tm_w2, const TcGemmArgs& a,
                                  int num_sms, cudaStream_t st) {
-    return launch_pair<false>(tm_h, tm_w2, tm_w2, a, num_sms, st);
+    return launch_pair<false, false>(tm_h, tm_w2, tm_w2, a, num_sms, st);
+}
+
+cudaError_t launch_tc_gemm1_pair_e4m3(const CUtensorMap& tm_x8, const CUtensorMap& tm_q1,
+                                      const CUtensorMap& tm_q3, const TcGemmArgs& a, int num_sms,
+                                      cudaStream_t st) {
+    return launch_pair<true, true>(tm_x8, tm_q1, tm_q3, a, num_sms, st);
+}
+
+cudaError_t launch_tc_gemm2_pair_e4m3(const CUtensorMap& tm_h8, const CUtensorMap& tm_q2, const TcGemmArgs& a,
+                                      int num_sms, cudaStream_t st) {
+    return launch_pair<false, true>(tm_h8, tm_q2, tm_q2, a, num_sms, st);
 }
 
 }  // namespace moe

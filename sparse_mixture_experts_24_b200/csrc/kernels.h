@@ -296,5 +296,11 @@ cudaError_t launch_tc_gemm1_pair(const CUtensorMap& tm_xp, const CUtensorMap& tm
                                  cudaStream_t st);
 cudaError_t launch_tc_gemm2_pair(const CUtensorMap& tm_h, const CUtensorMap& tm_w2, const TcGemmArgs& a,
                                  int num_sms, cudaStream_t st);
+// The same on E4M3 operands (maps as launch_tc_gemm1_e4m3 / launch_tc_gemm2_e4m3).
+cudaError_t launch_tc_gemm1_pair_e4m3(const CUtensorMap& tm_x8, const CUtensorMap& tm_q1,
+                                      const CUtensorMap& tm_q3, const TcGemmArgs& a, int num_sms,
+                                      cudaStream_t st);
+cudaError_t launch_tc_gemm2_pair_e4m3(const CUtensorMap& tm_h8, const CUtensorMap& tm_q2, const TcGemmArgs& a,
+                                      int num_sms, cudaStream_t st);
 
 }  // namespace moe

@@ -473,6 +473,16 @@ bool use_pair_gemm(const moe_handle* h, int64_t T) {
     return env && strcmp(env, "pair") == 0;
 }
 
+// E4M3 GEMM tiling: the same switch (MOE_GEMM_PATH=pair selects CTA pairs).
+bool use_pair_gemm_e4m3(const moe_handle* h, int64_t T) {
+    const char* env = getenv("MOE_GEMM_PATH");
+    if (env && strcmp(env, "single") == 0) return false;
+    if (env && strcmp(env, "pair") == 0) return true;
+    (void)h;
+    (void)T;
+    return false;
+}
+
 // Most (token, slot) pairs one expert takes in a call of T tokens:
 // ceil(factor * T * K / n), or no limit when the factor is 0.
 int capacity_for(const moe_handle* h, int64_t T) {
@@ -578,7 +588,9 @@ moe_status run_experts_e4m3(moe_handle* h, int64_t T, const void* x, const int32
                             const float* topk_w, const uint8_t* q1, const float* s1, const uint8_t* q3,
                             const float* s3, const uint8_t* q2, const float* s2, void* y, cudaStream_t st) {
     const int64_t R = T * h->K;
-    cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n, moe::kTcBM, h->db, st, capacity_for(h, T));
+    const bool pair = use_pair_gemm_e4m3(h, T);
+    cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n, pair ? moe::kTcPairBM : moe::kTcBM, h->db, st,
+                                         capacity_for(h, T));
     if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
     h->launches += moe::dispatch_kernel_count(R);
     trace_mark(h, 1, st);
@@ -616,7 +628,8 @@ moe_status run_experts_e4m3(moe_handle* h, int64_t T, const void* x, const int32
     a1.row_scale = h->xs;
     a1.col_scale0 = s1;
     a1.col_scale1 = s3;
-    e = moe::launch_tc_gemm1_e4m3(h->tm_x8, h->tm_q1, h->tm_q3, a1, h->num_sms, st);
+    e = pair ? moe::launch_tc_gemm1_pair_e4m3(h->tm_x8, h->tm_q1, h->tm_q3, a1, h->num_sms, st)
+             : moe::launch_tc_gemm1_e4m3(h->tm_x8, h->tm_q1, h->tm_q3, a1, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
     e = moe::launch_quantize_rows_e4m3(h->h, true, nullptr, R, R, used_rows, h->F, h->h8, h->hs, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "hidden-row quantisation launch");
@@ -630,7 +643,8 @@ moe_status run_experts_e4m3(moe_handle* h, int64_t T, const void* x, const int32
     a2.row_scale = h->hs;
     a2.col_scale0 = s2;
     a2.col_scale1 = nullptr;
-    e = moe::launch_tc_gemm2_e4m3(h->tm_h8, h->tm_q2, a2, h->num_sms, st);
+    e = pair ? moe::launch_tc_gemm2_pair_e4m3(h->tm_h8, h->tm_q2, a2, h->num_sms, st)
+             : moe::launch_tc_gemm2_e4m3(h->tm_h8, h->tm_q2, a2, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
     h->launches += 1;
     trace_mark(h, 4, st);

@@ -6,7 +6,7 @@ these variables once per process):
                              launch (plain stream order);
   MOE_ROUTER_TOPK=separate   tensor-core router writes logits, then the
                              standalone top-K kernel selects;
-  MOE_GEMM_PATH=pair         CTA-pair (cta_group::2) expert GEMMs.
+  MOE_GEMM_PATH=pair         CTA-pair (cta_group::2) expert GEMMs (bf16 and E4M3).
 """
 import os
 import subprocess
@@ -51,3 +51,15 @@ def test_low_precision_paths_without_pdl(test_file, selection, count):
     assert r.returncode == 0, tail
     assert "%d passed" % count in r.stdout, tail
 
+
+def test_e4m3_layer_on_cta_pairs():
+    """The E4M3 layer with the CTA-pair (cta_group::2, kind::f8f6f4) GEMMs:
+    every layer case, the capacity case and the 20,000-token sampled case."""
+    full_env = dict(os.environ)
+    full_env["MOE_GEMM_PATH"] = "pair"
+    cmd = [sys.executable, "-m", "pytest", os.path.join(ROOT, "tests", "test_gpu_e4m3.py"), "-m", "gpu", "-q", "-x",
+           "-p", "no:cacheprovider", "-k", "layer_matches_oracle or capacity or many_rows or full_size"]
+    r = subprocess.run(cmd, cwd=ROOT, env=full_env, capture_output=True, text=True, timeout=900)
+    tail = "\n".join((r.stdout + r.stderr).strip().splitlines()[-15:])
+    assert r.returncode == 0, tail
+    assert "8 passed" in r.stdout, tail
