@@ -11,8 +11,8 @@ One layer step on rank r, every arithmetic step in the library's kernels:
     barrier
     moe_ep_combine                   expert outputs loaded from the owners' buffers
 
-ExpertParallelMoE runs one rank per process and GPU (torch.distributed with
-NCCL for the counts and the barriers; peer buffers mapped by CUDA IPC).
+ExpertParallelMoE runs one rank per process (torch.distributed for the counts
+and the barriers -- NCCL with a GPU per rank; peer buffers mapped by CUDA IPC).
 emulate_ranks runs W ranks in one process on one GPU, phase by phase, with
 every rank's buffers in that GPU's memory -- the same kernels and layouts.
 """
@@ -197,9 +197,9 @@ class ExpertParallelMoE:
         import torch
         rk = self._rank
         counts = rk.route(x, W_g, stream)
-        flat = torch.empty(self.world * self.n, dtype=torch.int32, device=counts.device)
-        self.dist.all_gather_into_tensor(flat, counts, group=self.group)
-        counts_all = flat.view(self.world, self.n)
+        rows = [torch.empty_like(counts) for _ in range(self.world)]
+        self.dist.all_gather(rows, counts, group=self.group)
+        counts_all = torch.stack(rows)
         rk.dispatch(self.world, self.rank, x, counts_all, self.recv_ptrs, self.recv_rows, stream)
         self._barrier()
         rk.experts(self.world, self.rank, counts_all, self.recv_ptrs[self.rank], self.recv_rows, w1, w3, w2,
