@@ -18,7 +18,8 @@
 //   wq_encode_kernel   codes of every weight, one thread per 16-byte vector;
 //   wq_scale_kernel    max |w| -> scale, in place;
 //   qrows_kernel       one block per row: max |v| over the row, then its codes
-//                      (the second read of the row hits L1/L2).
+//                      (rows of up to 4 vectors per thread stay in registers;
+//                      longer ones are read again, from L1/L2).
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -115,23 +116,26 @@ __global__ void __launch_bounds__(256) wq_scale_kernel(float* __restrict__ scale
     if (i < count) scales[i] = e4m3_scale(scales[i]);
 }
 
-constexpr int kQrThreads = 512;
 
 // One block per row: max |v| over the row (block reduction), then its codes.
-template <bool kBf16>
-__global__ void __launch_bounds__(kQrThreads) qrows_kernel(const uint4* __restrict__ src,
-                                                           const int32_t* __restrict__ row_src,
-                                                           int64_t src_rows, int64_t rows,
-                                                           const int32_t* __restrict__ row_limit, int vpr,
-                                                           uint8_t* __restrict__ codes,
-                                                           float* __restrict__ scales) {
+// kThreads = 512 for few rows (a row's vectors spread over more threads),
+// 128 for many (four times the rows in flight per SM).  A row of at most
+// 4 * kThreads vectors is read once and kept in registers for its codes.
+template <bool kBf16, int kThreads>
+__global__ void __launch_bounds__(kThreads) qrows_kernel(const uint4* __restrict__ src,
+                                                         const int32_t* __restrict__ row_src,
+                                                         int64_t src_rows, int64_t rows,
+                                                         const int32_t* __restrict__ row_limit, int vpr,
+                                                         uint8_t* __restrict__ codes,
+                                                         float* __restrict__ scales) {
     griddep_wait();
     constexpr int kPer = kBf16 ? 8 : 4;
-    __shared__ float s_max[kQrThreads / 32];
+    __shared__ float s_max[kThreads / 32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int64_t limit = rows;
     if (row_limit) limit = min(limit, static_cast<int64_t>(*row_limit));
     const int64_t cols = static_cast<int64_t>(vpr) * kPer;
+    const bool one_pass = vpr <= 4 * kThreads;
     for (int64_t r = blockIdx.x; r < limit; r += gridDim.x) {
         int64_t s = r;
         if (row_src) {
@@ -141,11 +145,11 @@ __global__ void __launch_bounds__(kQrThreads) qrows_kernel(const uint4* __restri
         const uint4* row = src + s * vpr;
         // four vectors per thread in flight at once (zeros past the row end)
         float m = 0.f;
-        for (int v0 = tid; v0 < vpr; v0 += 4 * kQrThreads) {
-            uint4 q[4];
+        uint4 q[4];
+        for (int v0 = tid; v0 < vpr; v0 += 4 * kThreads) {
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int v = v0 + u * kQrThreads;
+                const int v = v0 + u * kThreads;
                 q[u] = v < vpr ? __ldg(row + v) : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
@@ -162,22 +166,23 @@ __global__ void __launch_bounds__(kQrThreads) qrows_kernel(const uint4* __restri
         __syncthreads();
         m = s_max[0];
 #pragma unroll
-        for (int w = 1; w < kQrThreads / 32; ++w) m = fmaxf(m, s_max[w]);
+        for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, s_max[w]);
         const float scale = e4m3_scale(m);
         float sc[kPer];
 #pragma unroll
         for (int i = 0; i < kPer; ++i) sc[i] = scale;
         uint8_t* out = codes + r * cols;
-        for (int v0 = tid; v0 < vpr; v0 += 4 * kQrThreads) {
-            uint4 q[4];
+        for (int v0 = tid; v0 < vpr; v0 += 4 * kThreads) {
+            if (!one_pass) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int v = v0 + u * kQrThreads;
-                q[u] = v < vpr ? __ldg(row + v) : make_uint4(0u, 0u, 0u, 0u);
+                for (int u = 0; u < 4; ++u) {
+                    const int v = v0 + u * kThreads;
+                    q[u] = v < vpr ? __ldg(row + v) : make_uint4(0u, 0u, 0u, 0u);
+                }
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int v = v0 + u * kQrThreads;
+                const int v = v0 + u * kThreads;
                 if (v < vpr) {
                     float f[kPer];
                     unpack16<kBf16>(q[u], f);
@@ -223,15 +228,27 @@ cudaError_t launch_quantize_rows_e4m3(const void* src, bool bf16, const int32_t*
                                       int64_t rows, const int32_t* row_limit, int cols, uint8_t* codes,
                                       float* scales, int num_sms, cudaStream_t st) {
     const int vpr = cols / (bf16 ? 8 : 4);
+    // 16 rows per SM in flight once there are enough rows (measured on the
+    // prefill rows); a few long rows keep 512 threads each
+    const bool many = rows >= 16LL * num_sms;
     int64_t blocks = rows;
-    if (blocks > static_cast<int64_t>(num_sms) * 8) blocks = static_cast<int64_t>(num_sms) * 8;
+    const int64_t cap = static_cast<int64_t>(num_sms) * (many ? 16 : 8);
+    if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    if (bf16)
-        launch_k(qrows_kernel<true>, dim3(static_cast<unsigned>(blocks)), dim3(kQrThreads), 0, st,
-                 static_cast<const uint4*>(src), row_src, src_rows, rows, row_limit, vpr, codes, scales);
+    const dim3 g(static_cast<unsigned>(blocks));
+    const uint4* s = static_cast<const uint4*>(src);
+    if (bf16 && many)
+        launch_k(qrows_kernel<true, 128>, g, dim3(128), 0, st, s, row_src, src_rows, rows, row_limit, vpr, codes,
+                 scales);
+    else if (bf16)
+        launch_k(qrows_kernel<true, 512>, g, dim3(512), 0, st, s, row_src, src_rows, rows, row_limit, vpr, codes,
+                 scales);
+    else if (many)
+        launch_k(qrows_kernel<false, 128>, g, dim3(128), 0, st, s, row_src, src_rows, rows, row_limit, vpr, codes,
+                 scales);
     else
-        launch_k(qrows_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(kQrThreads), 0, st,
-                 static_cast<const uint4*>(src), row_src, src_rows, rows, row_limit, vpr, codes, scales);
+        launch_k(qrows_kernel<false, 512>, g, dim3(512), 0, st, s, row_src, src_rows, rows, row_limit, vpr, codes,
+                 scales);
     return cudaGetLastError();
 }
 

@@ -85,8 +85,6 @@ cudaError_t launch_w4a4_pack(const uint8_t* codes, const uint8_t* bscale, const 
     return cudaGetLastError();
 }
 
-constexpr int kW4RowThreads = 256;
-
 __device__ __forceinline__ float w4_tensor_scale(float amax) { return amax > 0.f ? __fdiv_rn(amax, 2688.f) : 1.f; }
 
 __device__ __forceinline__ float w4_e4m3_value(uint32_t code) {
@@ -94,8 +92,10 @@ __device__ __forceinline__ float w4_e4m3_value(uint32_t code) {
     return __half2float(__half(h));
 }
 
-// One block per row; thread = blocks of 16 elements (bf16 source).
-__global__ void __launch_bounds__(kW4RowThreads) w4a4_rows_kernel(const uint16_t* __restrict__ src,
+// One block per row; thread = blocks of 16 elements (bf16 source).  kThreads
+// = 256 for few rows, 128 for many (twice the rows in flight per SM).
+template <int kThreads>
+__global__ void __launch_bounds__(kThreads) w4a4_rows_kernel(const uint16_t* __restrict__ src,
                                                                   const int32_t* __restrict__ row_src,
                                                                   int64_t src_rows, int K,
                                                                   const int32_t* __restrict__ offsets,
@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(kW4RowThreads) w4a4_rows_kernel(const uint16_t
                                                                   uint8_t* __restrict__ chunks,
                                                                   float* __restrict__ rscale) {
     griddep_wait();
-    __shared__ float s_max[kW4RowThreads / 32];
+    __shared__ float s_max[kThreads / 32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t rows = offsets[n];
     const int nblk = K / 16;
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(kW4RowThreads) w4a4_rows_kernel(const uint16_t
         }
         const uint4* row = reinterpret_cast<const uint4*>(src + s * K);
         float m = 0.f;
-        for (int b = tid; b < nblk; b += kW4RowThreads) {
+        for (int b = tid; b < nblk; b += kThreads) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const uint4 q = __ldg(row + 2 * b + h);
@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kW4RowThreads) w4a4_rows_kernel(const uint16_t
         __syncthreads();
         m = s_max[0];
 #pragma unroll
-        for (int w = 1; w < kW4RowThreads / 32; ++w) m = fmaxf(m, s_max[w]);
+        for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, s_max[w]);
         const float rs = w4_tensor_scale(m);
         // the row's tile and its row inside the tile
         int lo = 0, hi = n - 1;
@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(kW4RowThreads) w4a4_rows_kernel(const uint16_t
         const int64_t local = r - offsets[lo];
         const int64_t tile = mblk_base[lo] + local / tile_rows;
         const int tr = static_cast<int>(local % tile_rows);
-        for (int b = tid; b < nblk; b += kW4RowThreads) {
+        for (int b = tid; b < nblk; b += kThreads) {
             float v[16];
             float amax_b = 0.f;
 #pragma unroll
@@ -306,11 +306,17 @@ cudaError_t launch_w4a4_rows(const uint16_t* src, const int32_t* row_src, int64_
                      tile_rows, codes, chunks, rscale);
         return cudaGetLastError();
     }
+    const bool many = rows_max >= 16LL * num_sms;
     int64_t blocks = rows_max;
-    if (blocks > static_cast<int64_t>(num_sms) * 8) blocks = static_cast<int64_t>(num_sms) * 8;
+    const int64_t cap = static_cast<int64_t>(num_sms) * (many ? 16 : 8);
+    if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    launch_k(w4a4_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kW4RowThreads), 0, st, src, row_src,
-             src_rows, K, offsets, mblk_base, n, tile_rows, codes, chunks, rscale);
+    if (many)
+        launch_k(w4a4_rows_kernel<128>, dim3(static_cast<unsigned>(blocks)), dim3(128), 0, st, src, row_src,
+                 src_rows, K, offsets, mblk_base, n, tile_rows, codes, chunks, rscale);
+    else
+        launch_k(w4a4_rows_kernel<256>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, src, row_src,
+                 src_rows, K, offsets, mblk_base, n, tile_rows, codes, chunks, rscale);
     return cudaGetLastError();
 }
 

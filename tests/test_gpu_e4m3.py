@@ -137,6 +137,7 @@ FWD_CASES = [
     ("e4m3_T1", 1, 256, 256, 8, 2),
     ("e4m3_d64_n64", 700, 64, 64, 64, 4),
     ("e4m3_big_segments", 1500, 384, 512, 4, 2),
+    ("e4m3_many_long_rows", 1200, 256, 4608, 8, 2),   # 2,400 H rows of 4,608: 128-thread blocks, two passes
 ]
 
 

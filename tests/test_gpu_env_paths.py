@@ -62,4 +62,4 @@ def test_e4m3_layer_on_cta_pairs():
     r = subprocess.run(cmd, cwd=ROOT, env=full_env, capture_output=True, text=True, timeout=900)
     tail = "\n".join((r.stdout + r.stderr).strip().splitlines()[-15:])
     assert r.returncode == 0, tail
-    assert "8 passed" in r.stdout, tail
+    assert "9 passed" in r.stdout, tail

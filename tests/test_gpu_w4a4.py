@@ -114,6 +114,7 @@ FWD_CASES = [
     ("w4a4_n64", 700, 256, 256, 64, 4),
     ("w4a4_big_segments", 1500, 512, 768, 4, 2),
     ("w4a4_d2048_rows", 400, 2048, 256, 8, 2),   # 800 rows of 2,048: the warp-per-row quantiser
+    ("w4a4_long_rows", 1300, 2560, 256, 8, 2),   # 2,600 rows of 2,560: 128-thread blocks per row
 ]
 
 
