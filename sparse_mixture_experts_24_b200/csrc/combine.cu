@@ -34,27 +34,9 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const uint4* __restri
             const int32_t r = __ldg(token_row + t * K + k);
             if (r < 0) continue;
             const float g = __ldg(topk_w + t * K + k);
-            const uint4 q = __ldg(O + static_cast<int64_t>(r) * vec_per_row + v);
-            float a, b;
-            unpack_bf16x2(q.x, a, b);
-            acc[0] = fmaf(g, a, acc[0]);
-            acc[1] = fmaf(g, b, acc[1]);
-            unpack_bf16x2(q.y, a, b);
-            acc[2] = fmaf(g, a, acc[2]);
-            acc[3] = fmaf(g, b, acc[3]);
-            unpack_bf16x2(q.z, a, b);
-            acc[4] = fmaf(g, a, acc[4]);
-            acc[5] = fmaf(g, b, acc[5]);
-            unpack_bf16x2(q.w, a, b);
-            acc[6] = fmaf(g, a, acc[6]);
-            acc[7] = fmaf(g, b, acc[7]);
+            fma_bf16x8(acc, g, __ldg(O + static_cast<int64_t>(r) * vec_per_row + v));
         }
-        uint4 out;
-        out.x = pack_bf16x2(acc[0], acc[1]);
-        out.y = pack_bf16x2(acc[2], acc[3]);
-        out.z = pack_bf16x2(acc[4], acc[5]);
-        out.w = pack_bf16x2(acc[6], acc[7]);
-        y[i] = out;
+        y[i] = pack_bf16x8(acc);
     }
     griddep_launch_dependents();
 }

@@ -112,6 +112,34 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+// acc[0..7] += g * (the 8 bf16 values of q), one fmaf each in element order:
+// the combine's accumulation, shared by the single-GPU and expert-parallel
+// combines so that both round identically.
+__device__ __forceinline__ void fma_bf16x8(float (&acc)[8], float g, const uint4& q) {
+    float a, b;
+    unpack_bf16x2(q.x, a, b);
+    acc[0] = fmaf(g, a, acc[0]);
+    acc[1] = fmaf(g, b, acc[1]);
+    unpack_bf16x2(q.y, a, b);
+    acc[2] = fmaf(g, a, acc[2]);
+    acc[3] = fmaf(g, b, acc[3]);
+    unpack_bf16x2(q.z, a, b);
+    acc[4] = fmaf(g, a, acc[4]);
+    acc[5] = fmaf(g, b, acc[5]);
+    unpack_bf16x2(q.w, a, b);
+    acc[6] = fmaf(g, a, acc[6]);
+    acc[7] = fmaf(g, b, acc[7]);
+}
+
+__device__ __forceinline__ uint4 pack_bf16x8(const float (&acc)[8]) {
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    return o;
+}
+
 // Exclusive scan of one value per thread over a 256-thread block.
 __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;

@@ -114,7 +114,8 @@ __global__ void __launch_bounds__(256) ep_scatter_kernel(const uint4* __restrict
     const bool bad = (*status & kStatusEpPlan) != 0;
     const int lane = threadIdx.x & 31;
     const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-    for (int64_t p = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); p < R; p += warps) {
+    const int64_t first = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    for (int64_t p = first; p < R; p += warps) {
         const int e = __ldg(idx + p);
         const int j = __ldg(token_row + p);
         int64_t pos = -1;
@@ -138,8 +139,8 @@ __global__ void __launch_bounds__(256) ep_scatter_kernel(const uint4* __restrict
 __global__ void __launch_bounds__(256) ep_combine_kernel(const int32_t* __restrict__ idx,
                                                          const float* __restrict__ topk_w,
                                                          const int32_t* __restrict__ row_pos, int64_t T, int K,
-                                                         int n, int nl, const __grid_constant__ EpPeers out, int vec_per_row,
-                                                         uint4* __restrict__ y) {
+                                                         int n, int nl, const __grid_constant__ EpPeers out,
+                                                         int vec_per_row, uint4* __restrict__ y) {
     griddep_wait();
     const int64_t total = T * vec_per_row;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -154,27 +155,10 @@ __global__ void __launch_bounds__(256) ep_combine_kernel(const int32_t* __restri
             const int e = __ldg(idx + t * K + k);
             if (pos < 0 || e < 0 || e >= n) continue;
             const float g = __ldg(topk_w + t * K + k);
-            const uint4 q = *(static_cast<const uint4*>(out.ptr[e / nl]) + static_cast<int64_t>(pos) * vec_per_row + v);
-            float a, b;
-            unpack_bf16x2(q.x, a, b);
-            acc[0] = fmaf(g, a, acc[0]);
-            acc[1] = fmaf(g, b, acc[1]);
-            unpack_bf16x2(q.y, a, b);
-            acc[2] = fmaf(g, a, acc[2]);
-            acc[3] = fmaf(g, b, acc[3]);
-            unpack_bf16x2(q.z, a, b);
-            acc[4] = fmaf(g, a, acc[4]);
-            acc[5] = fmaf(g, b, acc[5]);
-            unpack_bf16x2(q.w, a, b);
-            acc[6] = fmaf(g, a, acc[6]);
-            acc[7] = fmaf(g, b, acc[7]);
+            const uint4* o_row = static_cast<const uint4*>(out.ptr[e / nl]) + static_cast<int64_t>(pos) * vec_per_row;
+            fma_bf16x8(acc, g, o_row[v]);
         }
-        uint4 o;
-        o.x = pack_bf16x2(acc[0], acc[1]);
-        o.y = pack_bf16x2(acc[2], acc[3]);
-        o.z = pack_bf16x2(acc[4], acc[5]);
-        o.w = pack_bf16x2(acc[6], acc[7]);
-        y[i] = o;
+        y[i] = pack_bf16x8(acc);
     }
     griddep_launch_dependents();
 }
