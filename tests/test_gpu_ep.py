@@ -30,6 +30,7 @@ CASES = [
     ("ep_w1", (400,), 256, 256, 8, 2),
     ("ep_w2_k1", (129, 255), 192, 320, 4, 1),
     ("ep_w4_many_experts", (700, 300, 512, 1000), 128, 256, 64, 4),
+    ("ep_w16_most_ranks", (40, 0, 17, 90, 33, 1, 64, 8, 120, 5, 77, 2, 50, 30, 11, 60), 128, 128, 32, 2),
 ]
 
 

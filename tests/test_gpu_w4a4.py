@@ -155,9 +155,12 @@ def test_w4a4_layer_matches_oracle(case, tile, monkeypatch):
     assert 0.03 < band < 0.4, band
 
 
-def test_w4a4_capacity_and_rejections():
+@pytest.mark.parametrize("rows", ["128", "32"])
+def test_w4a4_capacity_and_rejections(rows, monkeypatch):
+    """Capacity dropping on both row-tile heights, and the argument checks."""
     import sparse_mixture_experts_24_b200 as m
     torch = require_cuda()
+    monkeypatch.setenv("MOE_W4A4_ROWS", rows)
     name, T, d, F, n, K = "w4a4_capacity", 600, 256, 256, 8, 2
     cfg = mi.custom_config(name, T=T, d=d, ffn=F, n=n, K=K, dtype="bf16", skew=True)
     L = mi.make_layer(cfg, seed=seed_of(name))
