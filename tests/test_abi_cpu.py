@@ -121,3 +121,16 @@ def test_capacity_and_stats_argument_checks_on_the_host(m):
         assert "P is NULL" in str(ei.value)
     finally:
         m.moe_destroy(h)
+
+
+def test_header_is_plain_c():
+    """include/moe.h is a C header (C99, no C++ or CUDA types): a C compiler
+    accepts it on its own."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler on this host")
+    r = subprocess.run([cc, "-fsyntax-only", "-std=c99", "-Wall", "-Werror", "-x", "c", HEADER],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
