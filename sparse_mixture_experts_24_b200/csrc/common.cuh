@@ -112,6 +112,16 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+// Persistent CTAs over `total` tiles: the fewest CTAs that need no more
+// rounds than the whole grid, so every working CTA does the same number of
+// tiles and no CTA runs a last, partial round alone (896 tiles on 148 SMs:
+// 128 CTAs of 7 tiles instead of 8 CTAs running a seventh round by themselves).
+__device__ __forceinline__ int balanced_ctas(int total, int grid) {
+    if (total <= grid) return grid;
+    const int rounds = (total + grid - 1) / grid;
+    return (total + rounds - 1) / rounds;
+}
+
 // acc[0..7] += g * (the 8 bf16 values of q), one fmaf each in element order:
 // the combine's accumulation, shared by the single-GPU and expert-parallel
 // combines so that both round identically.

@@ -148,6 +148,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = tail->tmem_base;
     const int total_tiles = tail->mblk[n] * args.n_tiles;
+    const int stride = args.balanced ? balanced_ctas(total_tiles, static_cast<int>(gridDim.x))
+                                     : static_cast<int>(gridDim.x);
+    const int first = static_cast<int>(blockIdx.x) < stride ? static_cast<int>(blockIdx.x) : total_tiles;
     int* status = args.status;
 
     if (warp == 0) {
@@ -158,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int armed[kStages];
             for (int s = 0; s < kStages; ++s) armed[s] = -1;
             bool ok = true;
-            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+            for (int t = first; t < total_tiles && ok; t += stride) {
                 const TileInfo ti = tile_info(t, tail->off, tail->mblk, n, args.n_tiles);
                 for (int kb = 0; kb < args.k_blocks; ++kb) {
                     if (!mbar_wait(smem_u32(&tail->empty[stage]), phase ^ 1u, status,
@@ -215,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0;
             int local = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++local) {
+            for (int t = first; t < total_tiles && ok; t += stride, ++local) {
                 const int buf = local & 1;
                 const uint32_t bph = static_cast<uint32_t>(local >> 1) & 1u;
                 if (!mbar_wait(smem_u32(&tail->accum_empty[buf]), bph ^ 1u, status,
@@ -274,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quad = warp & 3;  // TMEM lanes [32*quad, 32*quad+32)
         uint8_t* stage = smem + kStages * kStageBytes + kTailBytes + (warp - 2) * kWarpStageBytes;
         int local = 0;
-        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++local) {
+        for (int t = first; t < total_tiles; t += stride, ++local) {
             const TileInfo ti = tile_info(t, tail->off, tail->mblk, n, args.n_tiles);
             const int buf = local & 1;
             const uint32_t bph = static_cast<uint32_t>(local >> 1) & 1u;

@@ -157,6 +157,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = tail->tmem_base;
     const int total_tiles = tail->mblk[n] * args.n_tiles;
+    const int stride = args.balanced ? balanced_ctas(total_tiles, static_cast<int>(gridDim.x))
+                                     : static_cast<int>(gridDim.x);
+    const int first = static_cast<int>(blockIdx.x) < stride ? static_cast<int>(blockIdx.x) : total_tiles;
     const int kb64_total = args.k_steps * 4;  // 64-wide K steps of the whole reduction
     int* status = args.status;
 
@@ -169,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int s = 0; s < 6; ++s) armed[s] = -1;
             bool ok = true;
             const int blocks_per_e = args.n_rows_b / 128;
-            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+            for (int t = first; t < total_tiles && ok; t += stride) {
                 const Tile ti = tile_at<kTM>(t, tail->off, tail->mblk, n, args.n_tiles);
                 const int r0 = ti.n_tile * kBN;  // first packed B row of the tile
                 const uint8_t* sfb = args.b_chunks +
@@ -214,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0;
             int local = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++local) {
+            for (int t = first; t < total_tiles && ok; t += stride, ++local) {
                 const int buf = C::kAccBufs == 2 ? (local & 1) : 0;
                 const uint32_t use = C::kAccBufs == 2 ? static_cast<uint32_t>(local >> 1) : static_cast<uint32_t>(local);
                 if (!mbar_wait(smem_u32(&tail->accum_empty[buf]), (use & 1u) ^ 1u, status, kStatusTimeoutAccum)) {
@@ -263,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quad = warp & 3;
         const int half = (warp - 2) >> 2;
         int local = 0;
-        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++local) {
+        for (int t = first; t < total_tiles; t += stride, ++local) {
             const Tile ti = tile_at<kTM>(t, tail->off, tail->mblk, n, args.n_tiles);
             const int buf = C::kAccBufs == 2 ? (local & 1) : 0;
             const uint32_t use = C::kAccBufs == 2 ? static_cast<uint32_t>(local >> 1) : static_cast<uint32_t>(local);

@@ -183,6 +183,7 @@ struct TcGemmArgs {
     const float* row_scale;
     const float* col_scale0;
     const float* col_scale1;
+    int balanced;      // 1: spread the tiles evenly over the fewest CTAs (balanced_ctas)
 };
 
 cudaError_t launch_tc_gemm1(const CUtensorMap& tm_xp, const CUtensorMap& tm_w1,
@@ -259,6 +260,7 @@ struct W4a4GemmArgs {
     const float* mscale1;      // [n] w3 (GEMM1)
     const uint8_t* a_chunks;   // activation scale chunks [tiles][K/64][512]
     const uint8_t* b_chunks;   // weight scale chunks [n][rows/128][K/64][512] (w1|w3 pairs, or w2)
+    int balanced;              // as TcGemmArgs::balanced
 };
 
 // tm_a: activation codes [R][K/2] uint8 (boxes of tile_rows rows x 128 bytes,

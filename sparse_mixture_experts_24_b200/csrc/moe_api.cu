@@ -483,6 +483,14 @@ bool use_pair_gemm_e4m3(const moe_handle* h, int64_t T) {
     return false;
 }
 
+// Persistent GEMMs spread their tiles over the fewest CTAs that need no more
+// rounds than the whole grid (every working CTA the same number of tiles)
+// unless MOE_GRID_BALANCE=0.
+int grid_balance() {
+    const char* env = getenv("MOE_GRID_BALANCE");
+    return (env && strcmp(env, "0") == 0) ? 0 : 1;
+}
+
 // Most (token, slot) pairs one expert takes in a call of T tokens:
 // ceil(factor * T * K / n), or no limit when the factor is 0.
 int capacity_for(const moe_handle* h, int64_t T) {
@@ -527,6 +535,7 @@ moe_status run_gemms(moe_handle* h, int64_t T, int64_t R, const void* x, const v
         a1.out_cols = h->F;
         a1.out = h->h;
         a1.status = h->status;
+    a1.balanced = grid_balance();
         e = pair ? moe::launch_tc_gemm1_pair(h->tm_xp, h->tm_w1, h->tm_w3, a1, h->num_sms, st)
                  : moe::launch_tc_gemm1(h->tm_xp, h->tm_w1, h->tm_w3, a1, h->num_sms, st);
         if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
@@ -625,6 +634,7 @@ moe_status run_experts_e4m3(moe_handle* h, int64_t T, const void* x, const int32
     a1.out_cols = h->F;
     a1.out = h->h;
     a1.status = h->status;
+    a1.balanced = grid_balance();
     a1.row_scale = h->xs;
     a1.col_scale0 = s1;
     a1.col_scale1 = s3;
@@ -771,6 +781,7 @@ moe_status run_experts_w4a4(moe_handle* h, int64_t T, const void* x, const float
     a1.n_rows_b = 2 * h->F;
     a1.out = h->h;
     a1.status = h->status;
+    a1.balanced = grid_balance();
     a1.row_scale = h->xr4;
     a1.mscale0 = ws[0];
     a1.mscale1 = ws[1];
@@ -1319,6 +1330,7 @@ moe_status moe_ep_experts(moe_handle* h, int world, int rank, const int32_t* cou
     a1.out_cols = h->F;
     a1.out = h->h;
     a1.status = h->status;
+    a1.balanced = grid_balance();
     e = moe::launch_tc_gemm1(h->tm_erecv, h->tm_ew1, h->tm_ew3, a1, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
     moe::TcGemmArgs a2 = a1;
