@@ -217,6 +217,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = tail->tmem_base;
     const int total_tiles = tail->mblk[n] * args.n_tiles;
+    const int stride = args.balanced ? balanced_ctas(total_tiles, static_cast<int>(gridDim.x))
+                                     : static_cast<int>(gridDim.x);
+    const int first = static_cast<int>(blockIdx.x) < stride ? static_cast<int>(blockIdx.x) : total_tiles;
     int* status = args.status;
 
     if (warp == 0 || warp == kAWarp) {
@@ -230,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int armed[kRawStages];
             for (int s = 0; s < kRawStages; ++s) armed[s] = -1;
             bool ok = true;
-            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+            for (int t = first; t < total_tiles && ok; t += stride) {
                 const Tile ti = tile_at(t, tail->off, tail->mblk, n, args.n_tiles);
                 const int c0 = kSwiGLU ? ti.n_tile * 128 : ti.n_tile * 256;
                 const int c1 = kSwiGLU ? c0 : c0 + 128;
@@ -267,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             Ring ra, rb;
             int local = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++local) {
+            for (int t = first; t < total_tiles && ok; t += stride, ++local) {
                 const int buf = local & 1;
                 const uint32_t bph = static_cast<uint32_t>(local >> 1) & 1u;
                 if (!mbar_wait(smem_u32(&tail->accum_empty[buf]), bph ^ 1u, status, kStatusTimeoutAccum)) {
@@ -319,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int u = (col & 63) >> 3;         // 16-byte unit inside a 128-byte row
         Ring rr, rb;
         bool ok = true;
-        for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        for (int t = first; t < total_tiles && ok; t += stride) {
             for (int kb = 0; kb < args.k_blocks; ++kb) {
                 if (!mbar_wait(smem_u32(&tail->raw_full[rr.slot]), rr.phase, status, kStatusTimeoutFull) ||
                     !mbar_wait(smem_u32(&tail->b_empty[rb.slot]), rb.phase ^ 1u, status, kStatusTimeoutEmpty)) {
@@ -369,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------- epilogue (warps 2..5) ----------------
         const int quad = warp & 3;
         int local = 0;
-        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++local) {
+        for (int t = first; t < total_tiles; t += stride, ++local) {
             const Tile ti = tile_at(t, tail->off, tail->mblk, n, args.n_tiles);
             const int buf = local & 1;
             const uint32_t bph = static_cast<uint32_t>(local >> 1) & 1u;

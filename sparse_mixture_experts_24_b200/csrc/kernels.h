@@ -215,6 +215,7 @@ struct Fp4GemmArgs {
     int* status;
     const float* tscale0;  // [n] matrix scales: w1 (GEMM1) or w2 (GEMM2)
     const float* tscale1;  // [n] w3 (GEMM1)
+    int balanced;              // as TcGemmArgs::balanced
 };
 
 // tm_xp / tm_h: bf16 rows (64 x 128 boxes, 128-byte swizzle); tm_c*: codes

@@ -695,6 +695,7 @@ moe_status run_experts_fp4(moe_handle* h, int64_t T, const void* x, const float*
         }
     }
     moe::Fp4GemmArgs a1{};
+    a1.balanced = 0;  // bound by its converter warps: every SM keeps working (measured 0.680 vs 0.688 ms)
     a1.offsets = h->db.offsets;
     a1.mblk_base = h->db.mblk_base;
     a1.n = h->n;
