@@ -1,7 +1,7 @@
 """The layer forward under CUDA graph capture (needs a B200).
 
-After moe_reserve (and, for the E4M3 path, a first call that sizes its
-workspace) a forward call enqueues kernels only -- no allocation, no host
+After moe_reserve (and, for the E4M3 and 4-bit weight-and-activation paths,
+a first call that sizes their workspace) a forward call enqueues kernels only -- no allocation, no host
 synchronisation -- so it can be captured into a CUDA graph with its
 programmatic dependent launches.  Replays must equal the eager call bit for
 bit, also after the input buffer is refilled in place."""
@@ -20,10 +20,12 @@ def _layer_call(m, layer, path, xd, rest, q):
         return layer.forward(xd, *rest)
     if path == "e4m3":
         return layer.forward_e4m3(xd, rest[0], *q)
+    if path == "w4a4":
+        return layer.forward_w4a4(xd, rest[0], *q)
     return layer.forward_fp4(xd, rest[0], *q)
 
 
-@pytest.mark.parametrize("path", ["bf16", "e4m3", "fp4"])
+@pytest.mark.parametrize("path", ["bf16", "e4m3", "fp4", "w4a4"])
 def test_forward_replays_from_a_cuda_graph(path):
     import sparse_mixture_experts_24_b200 as m
     torch = require_cuda()
@@ -41,6 +43,10 @@ def test_forward_replays_from_a_cuda_graph(path):
             q = [dev(a) for a in q]
         elif path == "fp4":
             q = [tuple(dev(a) for a in oracle.quantize_weights_fp4(L[w])) for w in ("w1", "w3", "w2")]
+        elif path == "w4a4":
+            q4 = [oracle.quantize_weights_fp4(L[w]) for w in ("w1", "w3", "w2")]
+            q = [m.pack_weights_w4a4(*(dev(a) for a in q4[0]), pair=tuple(dev(a) for a in q4[1])),
+                 m.pack_weights_w4a4(*(dev(a) for a in q4[2]))]
         y0, i0, w0 = (t.clone() for t in _layer_call(m, layer, path, xd, rest, q))
         torch.cuda.synchronize()
         # outputs of the captured call live in these buffers
@@ -56,6 +62,8 @@ def test_forward_replays_from_a_cuda_graph(path):
                     layer.forward(xd, *rest, y=y, topk_idx=idx, topk_w=gw)
                 elif path == "e4m3":
                     layer.forward_e4m3(xd, rest[0], *q, y=y, topk_idx=idx, topk_w=gw)
+                elif path == "w4a4":
+                    layer.forward_w4a4(xd, rest[0], *q, y=y, topk_idx=idx, topk_w=gw)
                 else:
                     layer.forward_fp4(xd, rest[0], *q, y=y, topk_idx=idx, topk_w=gw)
         torch.cuda.synchronize()
