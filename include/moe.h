@@ -130,8 +130,9 @@ MOE_API moe_status moe_route(moe_handle *h, int64_t T, const void *x, const floa
 /*
  * Dispatch only: group the T*K (token, slot) pairs of topk_idx into
  * per-expert segments, expert by expert, tokens ascending inside an expert
- * (the "skip the experts whose gate is zero" of the Mixtral paper as quoted
- * on the ainotis page, laid out for grouped GEMMs).  Outputs (device, int32):
+ * (experts whose gate is zero compute nothing, as the ainotis page reports of
+ * the Mixtral paper; this is that rule laid out for grouped GEMMs).  Outputs
+ * (device, int32):
  *   counts[n]          rows of each expert
  *   offsets[n+1]       first row of each expert's segment; offsets[n] = T*K
  *   row_token[T*K]     token of each row
