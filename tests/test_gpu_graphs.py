@@ -29,7 +29,9 @@ def _layer_call(m, layer, path, xd, rest, q):
 def test_forward_replays_from_a_cuda_graph(path):
     import sparse_mixture_experts_24_b200 as m
     torch = require_cuda()
-    cfg = mi.custom_config("graph_" + path, T=200, d=256, ffn=384, n=8, K=2, dtype="bf16")
+    # the 4-bit weight-and-activation path needs ffn a multiple of 256
+    cfg = mi.custom_config("graph_" + path, T=200, d=256, ffn=512 if path == "w4a4" else 384, n=8, K=2,
+                           dtype="bf16")
     L = mi.make_layer(cfg, seed=21)
     L2 = mi.make_layer(cfg, seed=22, only=("x",))
     layer = m.MoELayer(cfg.n, cfg.K, cfg.d, cfg.ffn, "bf16")
