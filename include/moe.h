@@ -38,12 +38,18 @@
  *     or order the streams.
  *   - On any error nothing is launched, the outputs are untouched, and
  *     moe_last_error() describes the failure.
- *   - After moe_reserve(T_max) (and, for moe_forward_e4m3, one earlier call of
- *     it, which sizes its part of the workspace), a forward call with T <=
- *     T_max only enqueues kernels: it allocates nothing and does not
- *     synchronise with the host, so it can be captured into a CUDA graph and
- *     replayed (the kernels keep their programmatic dependent launches).  The
- *     captured call reads x and the weights from the addresses it was given.
+ *   - After moe_reserve(T_max) (and, for moe_forward_e4m3 and
+ *     moe_forward_w4a4, one earlier call of it, which sizes its part of the
+ *     workspace), a forward call with T <= T_max only enqueues kernels: it
+ *     allocates nothing and does not synchronise with the host, so it can be
+ *     captured into a CUDA graph and replayed (the kernels keep their
+ *     programmatic dependent launches).  The captured call reads x and the
+ *     weights from the addresses it was given.
+ *   - Environment switches, for measurement and tests (the results do not
+ *     depend on them): MOE_PDL=0 (plain stream order) and
+ *     MOE_ROUTER_TOPK=separate, read once per process; MOE_GEMM_PATH=pair
+ *     (CTA-pair GEMMs), MOE_GRID_BALANCE=0, MOE_W4A4_TILE=128|256 and
+ *     MOE_W4A4_ROWS=32|128, read per call.
  */
 #ifndef MOE_B200_MOE_H
 #define MOE_B200_MOE_H
