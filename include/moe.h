@@ -45,8 +45,8 @@
  *     captured into a CUDA graph and replayed (the kernels keep their
  *     programmatic dependent launches).  The captured call reads x and the
  *     weights from the addresses it was given.
- *   - Environment switches, for measurement and tests (the results do not
- *     depend on them): MOE_PDL=0 (plain stream order) and
+ *   - Environment switches, for measurement and tests (every setting is
+ *     parity-tested against the same oracle and tolerances): MOE_PDL=0 (plain stream order) and
  *     MOE_ROUTER_TOPK=separate, read once per process; MOE_GEMM_PATH=pair
  *     (CTA-pair GEMMs), MOE_GRID_BALANCE=0, MOE_W4A4_TILE=128|256 and
  *     MOE_W4A4_ROWS=32|128, read per call.
