@@ -6,7 +6,8 @@ these variables once per process):
                              launch (plain stream order);
   MOE_ROUTER_TOPK=separate   tensor-core router writes logits, then the
                              standalone top-K kernel selects;
-  MOE_GEMM_PATH=pair         CTA-pair (cta_group::2) expert GEMMs (bf16 and E4M3).
+  MOE_GEMM_PATH=pair         CTA-pair (cta_group::2) expert GEMMs (bf16 and E4M3);
+  MOE_GRID_BALANCE=0         persistent GEMM tiles strided over the whole grid.
 """
 import os
 import subprocess
@@ -21,7 +22,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SLICE = "small and (bf16_ragged or bf16_k3_n16 or router_split2 or router_split4 or router_K10 or f32_tiny)"
 
 
-@pytest.mark.parametrize("env", [{"MOE_PDL": "0"}, {"MOE_ROUTER_TOPK": "separate"}, {"MOE_GEMM_PATH": "pair"}],
+@pytest.mark.parametrize("env", [{"MOE_PDL": "0"}, {"MOE_ROUTER_TOPK": "separate"}, {"MOE_GEMM_PATH": "pair"},
+                                 {"MOE_GRID_BALANCE": "0"}],
                          ids=lambda e: ",".join("%s=%s" % kv for kv in e.items()))
 def test_parity_slice_under_env(env):
     full_env = dict(os.environ)
