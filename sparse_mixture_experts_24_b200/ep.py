@@ -211,11 +211,14 @@ class ExpertParallelMoE:
         return y, rk.idx, rk.gate
 
     def close(self):
-        # no rank may still read this rank's buffers
+        # no rank may still read this rank's buffers, and no rank may still
+        # hold a mapping of them when they are freed
         self._barrier()
         self.ops.synchronize()
         for p in self._opened:
             self.ops.close(p, True)
+        self._barrier()
+        self.ops.synchronize()
         for p in self._own:
             self.ops.close(p, False)
         self._opened, self._own = [], []
