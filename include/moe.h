@@ -500,9 +500,10 @@ MOE_API moe_status moe_trace_end(moe_handle *h, double *stage_ms, int n_stages, 
  * that cannot take cudaMalloc's implicit device-wide synchronisation.
  *   Limit: T * K <= 65,536 pairs, n <= 256; larger sizes return
  *   MOE_ERR_INVALID_ARG with a message naming the limit.
- *   The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   Every call looks up the array's device address (cudaGetSymbolAddress)
+ *   on the current device.  The first lookup on a device may load the
+ *   library's module there, so make the first call on each device before any
+ *   stream capture.
  *   Every call shares the array and it keeps the last call's contents (each
  *   call overwrites what it reads).  Calls that overlap on the GPU race on
  *   it: order them on one stream.

@@ -10,6 +10,9 @@ bf16 bit patterns stored as uint16, and are widened exactly to double):
   router(x, W_g, K)                     -> idx [T,K] int32, gate [T,K] f64, logits [T,n] f64
   gates_to_bf16(gate)                   -> the gates cast to bf16 as the quoted routing code
                                            does (fp64 -> fp32 -> bf16, nearest even), as f64
+  routing_alternatives(logits_row, K, gap) -> the top-K routings (and their softmax gates)
+                                           a ranking that can misorder logits closer
+                                           than gap may produce, the oracle's own first
   expert(x_row, w1, w3, w2, e)          -> [d] f64, one SwiGLU expert on one token
   forward_with_routing(x, idx, gate, w1, w3, w2) -> y [T,d] f64
   moe_forward(x, W_g, w1, w3, w2, K)    -> y, idx, gate
@@ -389,6 +392,48 @@ def router(x, W_g, K: int):
 
 def gates_to_bf16(gate):
     return default().gates_to_bf16(gate)
+
+
+def routing_alternatives(logits_row, K: int, gap: float, limit: int = 720):
+    """Every top-K routing of one token that moving each logit by less than
+    about `gap` can produce, the oracle's own routing first.
+
+    Experts are ranked by (logit descending, index ascending), as the router
+    ranks them.  Neighbours in that ranking whose logits differ by less than
+    `gap` form a run; the experts of a run can come out of a lower-precision
+    ranking in any order.  The alternatives are all routings in which the
+    positions [0, K) that a run covers are filled by an ordered choice of
+    that run's experts.  The gates of each are the softmax over its K chosen
+    logits, listed with their experts: the gate rule of the layer equation
+    ("Mixtral of Experts" section 2.1, softmax over the Top-K logits; Part 3,
+    Step 3 of "Mixture of Experts: Why Mixtral Only Wakes Up Two
+    Specialists").  -> list of (idx [K] int32, gate [K] float64)."""
+    import itertools
+    L = np.asarray(logits_row, np.float64)
+    n = L.size
+    order = sorted(range(n), key=lambda e: (-L[e], e))
+    runs = []                      # (first position, last position) of each run
+    a = 0
+    for p in range(1, n + 1):
+        if p == n or L[order[p - 1]] - L[order[p]] >= gap:
+            runs.append((a, p - 1))
+            a = p
+    choices = []                   # per run meeting [0, K): its possible fillings
+    for a, b in runs:
+        if a >= K:
+            break
+        members = order[a:b + 1]
+        m = min(b, K - 1) - a + 1
+        choices.append(list(itertools.permutations(members, m)))
+    out = []
+    for combo in itertools.product(*choices):
+        sel = [e for part in combo for e in part]
+        z = L[sel]
+        g = np.exp(z - z.max())
+        out.append((np.array(sel, np.int32), g / g.sum()))
+        if len(out) >= limit:
+            break
+    return out
 
 
 def expert(x_row, w1, w3, w2, e: int):

@@ -42,7 +42,7 @@ static __device__ __align__(256) int32_t g_noalloc_scratch[kScratchWords];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-int32_t* g_scratch_addr[kMaxDevices] = {};
+bool g_device_checked[kMaxDevices] = {};
 
 thread_local char g_msg[256];
 
@@ -62,9 +62,11 @@ moe_status set_error(moe_status s, const char* msg) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Device address of the scratch array on the current device.  The first call
-// on a device looks it up with cudaGetSymbolAddress (with that device
-// current); later calls reuse the cached address.
+// Device address of the scratch array on the current device, looked up with
+// cudaGetSymbolAddress on every call (with that device current).  The lookup
+// allocates nothing once the library's module is loaded on the device, and
+// doing it each time keeps the address right after a device reset reloads
+// the module.  Only the device check is cached.
 moe_status scratch_for_current_device(int32_t** out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
@@ -73,25 +75,27 @@ moe_status scratch_for_current_device(int32_t** out) {
         return set_error(MOE_ERR_CUDA, g_msg);
     }
     if (dev < 0 || dev >= kMaxDevices) return set_error(MOE_ERR_UNSUPPORTED, "device index out of range");
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_addr[dev]) {
-        int major = 0, minor = 0;
-        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-        if (major != 10 || minor != 0) {
-            snprintf(g_msg, sizeof g_msg, "device %d is sm_%d%d; this library is built for sm_100a",
-                     dev, major, minor);
-            return set_error(MOE_ERR_UNSUPPORTED, g_msg);
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!g_device_checked[dev]) {
+            int major = 0, minor = 0;
+            cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+            if (major != 10 || minor != 0) {
+                snprintf(g_msg, sizeof g_msg, "device %d is sm_%d%d; this library is built for sm_100a",
+                         dev, major, minor);
+                return set_error(MOE_ERR_UNSUPPORTED, g_msg);
+            }
+            g_device_checked[dev] = true;
         }
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess || !p) {
-            snprintf(g_msg, sizeof g_msg, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
-            return set_error(MOE_ERR_CUDA, g_msg);
-        }
-        g_scratch_addr[dev] = static_cast<int32_t*>(p);
     }
-    *out = g_scratch_addr[dev];
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) {
+        snprintf(g_msg, sizeof g_msg, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+        return set_error(MOE_ERR_CUDA, g_msg);
+    }
+    *out = static_cast<int32_t*>(p);
     return MOE_OK;
 }
 
@@ -104,11 +108,12 @@ extern "C" MOE_API moe_status moe_dispatch_noalloc(int64_t T, int n, int K, cons
     if (n < 1 || n > kNoAllocMaxExperts) return set_error(MOE_ERR_INVALID_ARG, "n outside [1, 256]");
     if (K < 1 || K > n) return set_error(MOE_ERR_INVALID_ARG, "K outside [1, n]");
     if (T < 0) return set_error(MOE_ERR_INVALID_ARG, "T < 0");
-    if (T * K > kNoAllocMaxPairs) {
+    // T > max / K, not T * K > max: the product of a huge T would overflow
+    if (T > kNoAllocMaxPairs / K) {
         snprintf(g_msg, sizeof g_msg,
-                 "T * K = %lld exceeds the %lld (token, slot) pairs moe_dispatch_noalloc's fixed "
-                 "scratch holds; use moe_dispatch",
-                 static_cast<long long>(T * K), static_cast<long long>(kNoAllocMaxPairs));
+                 "T = %lld with K = %d exceeds the %lld (token, slot) pairs moe_dispatch_noalloc's "
+                 "fixed scratch holds; use moe_dispatch",
+                 static_cast<long long>(T), K, static_cast<long long>(kNoAllocMaxPairs));
         return set_error(MOE_ERR_INVALID_ARG, g_msg);
     }
     if (T == 0) return set_error(MOE_OK, "");

@@ -124,6 +124,17 @@ def emulate_ranks(xs, W_g, weights, n, K, recv_rows=None, stream=None):
         ep.close()
 
 
+def _current_stream(stream):
+    """Context that makes `stream` torch's current stream (no-op for None)."""
+    import contextlib
+    if stream is None:
+        return contextlib.nullcontext()
+    import torch
+    if isinstance(stream, int):
+        stream = torch.cuda.ExternalStream(stream)
+    return torch.cuda.stream(stream)
+
+
 class _CudaOps:
     """The library's side of ExpertParallelMoE: handles and IPC buffers."""
 
@@ -193,7 +204,17 @@ class ExpertParallelMoE:
 
     def forward(self, x, W_g, w1, w3, w2, y=None, stream=None):
         """x [T][d] bf16 of this rank; w1, w3 [n/W][d][ffn], w2 [n/W][ffn][d]:
-        this rank's experts.  -> (y, topk_idx, topk_w)."""
+        this rank's experts.  -> (y, topk_idx, topk_w).
+
+        stream (a torch.cuda.Stream or a raw cudaStream_t as an int): the
+        whole step, its all-gather and barriers included, is ordered on it.
+        The barriers are collectives on torch's current stream, so the step
+        makes `stream` current while it runs; otherwise a barrier could pass
+        before this rank's peer stores on `stream` are done."""
+        with _current_stream(stream):
+            return self._forward(x, W_g, w1, w3, w2, y, stream)
+
+    def _forward(self, x, W_g, w1, w3, w2, y, stream):
         import torch
         rk = self._rank
         counts = rk.route(x, W_g, stream)

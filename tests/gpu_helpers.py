@@ -9,6 +9,8 @@ import oracle
 
 NEAR_TIE = 1e-4          # gap below which two logits count as a near-tie
 TOL_Y = {"f32": 1e-5, "bf16": 2e-2}   # relative L2 bars on y
+PER_TOKEN_FACTOR = 5                   # per-token relative L2 bar = 5 x the aggregate one
+GEMM_ROW_BLOCK = 128                   # rows per M-block of the bf16 grouped GEMMs (MMA M)
 
 
 def require_cuda():
@@ -119,3 +121,82 @@ def stratified_sample(idx: np.ndarray, n: int, count: int, seed: int = 0) -> np.
             break
         pick.append(int(t))
     return np.array(sorted(set(pick)), np.int64)
+
+
+def near_tie_mask(o_logits, K):
+    """Tokens with an adjacent gap below NEAR_TIE among the oracle's top K+1
+    logits (the definition compare_routing counts)."""
+    T, n = o_logits.shape
+    srt = -np.sort(-o_logits, axis=1)
+    m = min(K + 1, n)
+    if m < 2:
+        return np.zeros(T, bool)
+    return (np.diff(-srt[:, :m], axis=1) < NEAR_TIE).any(axis=1)
+
+
+def block_covering_sample(o_idx, n, count=512, block=GEMM_ROW_BLOCK, seed=0):
+    """Tokens such that every (expert, M-block) of the grouped GEMMs holds at
+    least one sampled row.  The GEMMs cut each expert's segment of the
+    dispatch (oracle.dispatch of the oracle's routing: experts ascending,
+    tokens ascending) into `block`-row M-blocks from the segment start; one
+    random row of every block is taken, and the segment's last row (the
+    ragged end of its last block), then random tokens up to `count`.
+    -> (tokens sorted, number of M-blocks)."""
+    counts, offsets, row_token, _ = oracle.dispatch(o_idx, n)
+    rng = np.random.default_rng(seed)
+    pick = set()
+    blocks = 0
+    for e in range(n):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        for b0 in range(lo, hi, block):
+            pick.add(int(row_token[rng.integers(b0, min(b0 + block, hi))]))
+            blocks += 1
+        if hi > lo:
+            pick.add(int(row_token[hi - 1]))
+    T = o_idx.shape[0]
+    for t in rng.permutation(T):
+        if len(pick) >= min(count, T):
+            break
+        pick.add(int(t))
+    return np.array(sorted(pick), np.int64), blocks
+
+
+def blocks_covered(tokens, o_idx, n, block=GEMM_ROW_BLOCK):
+    """Number of distinct (expert, M-block) pairs the rows of `tokens` fall in."""
+    counts, offsets, _, token_row = oracle.dispatch(o_idx, n)
+    seg = np.repeat(np.arange(n), counts)             # expert of each row
+    rows = token_row[tokens].ravel()
+    e = seg[rows]
+    return len(set(zip(e.tolist(), ((rows - offsets[e]) // block).tolist())))
+
+
+def y_check_with_alternatives(y_gpu, gpu_idx, o_logits, o_idx, o_gate, tokens, L, K, tol):
+    """y of the sampled tokens against the oracle's layer.  A token whose
+    routing agrees with the oracle's is compared with the oracle's y; a
+    near-tie token with the closest of the oracle's own alternative routings
+    (oracle.routing_alternatives: every ordering of its top logits closer
+    than NEAR_TIE, with the oracle's gates for each), and its GPU routing
+    must be one of those alternatives.  No GPU value is an oracle input.
+    Returns (aggregate rel-L2, worst per-token rel-L2, number of near-tie
+    tokens checked)."""
+    tokens = np.asarray(tokens, np.int64)
+    agree = (gpu_idx[tokens] == o_idx[tokens]).all(axis=1)
+    ref = np.zeros((tokens.size, L["x"].shape[1]))
+    ta = tokens[agree]
+    if ta.size:
+        ref[agree] = oracle.forward_with_routing(L["x"][ta], o_idx[ta], o_gate[ta], L["w1"], L["w3"], L["w2"])
+    yg = y_as_f64(y_gpu[tokens])
+    tied = np.nonzero(~agree)[0]
+    for j in tied:
+        t = int(tokens[j])
+        alts = oracle.routing_alternatives(o_logits[t], K, NEAR_TIE)
+        assert tuple(gpu_idx[t]) in {tuple(int(e) for e in i) for i, _ in alts}, \
+            "token %d: GPU routing %s is no near-tie alternative of the oracle's" % (t, gpu_idx[t])
+        ai = np.stack([i for i, _ in alts])
+        ag = np.stack([g for _, g in alts])
+        xs = np.repeat(L["x"][t:t + 1], len(alts), axis=0)
+        ys = oracle.forward_with_routing(xs, ai, ag, L["w1"], L["w3"], L["w2"])
+        errs = np.linalg.norm(ys - yg[j], axis=1)
+        ref[j] = ys[int(np.argmin(errs))]
+    per_tok = np.linalg.norm(yg - ref, axis=1) / np.maximum(np.linalg.norm(ref, axis=1), 1e-30)
+    return rel_l2(yg, ref), float(per_tok.max()), int(tied.size)

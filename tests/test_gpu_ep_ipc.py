@@ -7,7 +7,8 @@ No kernel of one rank waits on another rank's kernel: the ranks are ordered
 only by the host-side barriers (gloo all-reduce after each rank's stream has
 drained), so the two processes' kernels may run in any interleaving.  Each
 rank's y must equal, bit for bit, the single-process layer under that rank's
-routing, over two consecutive steps."""
+routing, over three consecutive steps, the last on a side stream that is not
+torch's current stream."""
 import os
 import socket
 
@@ -56,8 +57,16 @@ def rank_main(rank, world, port, Ts, dims):
         layer = ExpertParallelMoE(n, K, d, F, recv_rows=sum(Ts) * K)
         single = m.MoELayer(n, K, d, F, "bf16")
         try:
-            for step in range(2):
-                y, idx, gate = layer.forward(x, Wg, *wl)
+            side = torch.cuda.Stream()
+            for step in range(3):
+                if step < 2:
+                    y, idx, gate = layer.forward(x, Wg, *wl)
+                else:
+                    # a stream that is not torch's current one: the step's
+                    # barriers must still order this rank's peer stores
+                    side.wait_stream(torch.cuda.current_stream())
+                    y, idx, gate = layer.forward(x, Wg, *wl, stream=side)
+                    torch.cuda.current_stream().wait_stream(side)
                 layer._rank.layer.sync_status()
                 y_ref = single.forward_with_routing(x, idx, gate, *w)
                 single.sync_status()

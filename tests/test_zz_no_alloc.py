@@ -39,7 +39,12 @@ def _noalloc(T, n, K, idx_d):
 
 def test_noalloc_dispatch_matches_moe_dispatch_twice_in_a_row():
     torch = require_cuda()
-    cases = [(777, 256, 8), (300, 8, 2)]   # the second call is smaller: stale scratch remains
+    # Both calls have more than 4,096 pairs, so both take the three-kernel
+    # path that reads the scratch array.  The first sits exactly at the
+    # 65,536-pair limit (256 pair blocks x 256 experts: every word of the
+    # per-block counts); the second is smaller, with another n, and runs over
+    # what the first left behind.
+    cases = [(8192, 256, 8), (2100, 8, 2)]
     for T, n, K in cases:
         rng = np.random.default_rng(T + n)
         idx = np.stack([rng.permutation(n)[:K] for _ in range(T)]).astype(np.int32)
@@ -51,12 +56,17 @@ def test_noalloc_dispatch_matches_moe_dispatch_twice_in_a_row():
     torch.cuda.synchronize()
 
 
-def test_noalloc_dispatch_refuses_sizes_over_its_limit():
+@pytest.mark.parametrize("T,K", [(65537, 1), (32769, 2), (2 ** 61, 4)])
+def test_noalloc_dispatch_refuses_sizes_over_its_limit(T, K):
+    """One pair over the limit is refused, and so is a T whose product with K
+    would overflow 64 bits; nothing is launched."""
     import sparse_mixture_experts_24_b200 as m
     torch = require_cuda()
-    idx = torch.zeros((40000, 2), dtype=torch.int32, device="cuda")
-    buf = torch.zeros(80001, dtype=torch.int32, device="cuda")
+    rows = min(T, 65537)
+    idx = torch.zeros((rows, K), dtype=torch.int32, device="cuda")
+    buf = torch.zeros(rows * K + 1, dtype=torch.int32, device="cuda")
     with pytest.raises(m.MoEError) as ei:
-        m.moe_dispatch_noalloc(40000, 8, 2, idx, buf, buf, buf, buf)
+        m.moe_dispatch_noalloc(T, 8, K, idx, buf, buf, buf, buf)
     assert ei.value.status == m.MOE_ERR_INVALID_ARG
     assert "65536" in str(ei.value)
+    torch.cuda.synchronize()
