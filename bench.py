@@ -2,7 +2,7 @@
 """Benchmark of the sparse MoE layer forward (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
-                    [--experts bf16|e4m3|fp4|w4a4] [--ep W]
+                    [--experts bf16|e4m3|fp4|w4a16|w4a4] [--ep W]
 
 A step is one moe_forward over one batch: router, top-K, softmax, dispatch,
 gather, GEMM1 (w1/w3 + SwiGLU), GEMM2 (w2), combine.  The default workload is
@@ -30,7 +30,9 @@ sample of the same workload on this host's cores.
 expert weights (per-column scales, quantised once before the timed region)
 and per-row E4M3 activations; --experts fp4 times moe_forward_fp4: 4-bit
 (E2M1) expert weights with E4M3 scales per 16 rows and bf16 activations (bf16
-handle and workloads only); --experts w4a4 times moe_forward_w4a4: the same
+handle and workloads only); --experts w4a16 times moe_forward_w4a16: the same
+layer on weights packed once by moe_pack_weights_w4a16, which the GEMMs decode
+straight into tensor memory; --experts w4a4 times moe_forward_w4a4: the same
 4-bit weights with 4-bit activations on the block-scaled tensor cores (d and
 ffn multiples of 256).
 
@@ -75,6 +77,7 @@ def workload_desc(cfg, experts="bf16"):
     return "%s: T=%d, d=%d, ffn=%d, n=%d, K=%d, %s%s%s" % (
         cfg.name, cfg.T, cfg.d, cfg.ffn, cfg.n, cfg.K, cfg.dtype, ", skewed router" if cfg.skew else "",
         {"e4m3": ", E4M3 experts", "fp4": ", 4-bit (E2M1) experts",
+         "w4a16": ", 4-bit (E2M1) experts decoded into tensor memory",
          "w4a4": ", 4-bit (E2M1) experts and activations"}.get(experts, ""))
 
 
@@ -94,7 +97,7 @@ def algorithmic(cfg, counts, experts="bf16"):
     T, d, F, n, K = cfg.T, cfg.d, cfg.ffn, cfg.n, cfg.K
     R = T * K
     used = int((counts > 0).sum())
-    if experts == "fp4":
+    if experts in ("fp4", "w4a16"):
         # codes 0.5 B + block scale 1/16 B per weight; gather, H and O in bf16
         w13 = used * 2 * (d * F // 2 + d * F // 16 + 4)
         w2 = used * (F * d // 2 + F * d // 16 + 4)
@@ -139,7 +142,8 @@ def recorded_traffic(kernel, config):
     p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(p):
         return None
-    src_file = "gemm_w4a4.cu" if config.endswith("_w4a4") else "gemm_tc.cu"
+    src_file = {"_w4a4": "gemm_w4a4.cu", "_w4a16": "gemm_w4a16.cu", "_fp4": "gemm_fp4.cu"}.get(
+        config[config.rfind("_"):], "gemm_tc.cu")
     sha = source_sha(os.path.join(ROOT, "sparse_mixture_experts_24_b200", "csrc", src_file))
     with open(p) as f:
         for line in f:
@@ -250,9 +254,9 @@ def oracle_tokens_per_s(cfg, L, budget_s=12.0, experts="bf16"):
         def layer(xs):
             i, g, _ = oracle.router(xs, L["W_g"], cfg.K)
             oracle.forward_e4m3(xs, i, g, *q)
-    elif experts in ("fp4", "w4a4"):
+    elif experts in ("fp4", "w4a16", "w4a4"):
         q4 = [oracle.quantize_weights_fp4(L[w]) for w in ("w1", "w3", "w2")]
-        fwd = oracle.forward_fp4 if experts == "fp4" else oracle.forward_w4a4
+        fwd = oracle.forward_w4a4 if experts == "w4a4" else oracle.forward_fp4
 
         def layer(xs):
             i, g, _ = oracle.router(xs, L["W_g"], cfg.K)
@@ -458,7 +462,7 @@ def main():
     ap.add_argument("--config", default="skew_prefill", choices=sorted(mi.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--experts", default="bf16", choices=["bf16", "e4m3", "fp4", "w4a4"])
+    ap.add_argument("--experts", default="bf16", choices=["bf16", "e4m3", "fp4", "w4a16", "w4a4"])
     ap.add_argument("--ep", type=int, default=0,
                     help="expert parallelism with this many ranks, emulated on one GPU")
     args = ap.parse_args()
@@ -507,14 +511,18 @@ def main():
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if cfg.name == "tiny_fp32" else None
     e4m3 = args.experts == "e4m3"
     fp4 = args.experts == "fp4"
+    w4a16 = args.experts == "w4a16"
     w4a4 = args.experts == "w4a4"
-    if e4m3 or fp4 or w4a4:
+    if e4m3 or fp4 or w4a16 or w4a4:
         # quantised once, outside the timed region; the bf16 copies are freed
         quant = m.quantize_weights_e4m3 if e4m3 else m.quantize_weights_fp4
         if w4a4:
             # the gate/up pair pack of w1 and w3, then w2
             q = list(m.pack_weights_w4a4(*m.quantize_weights_fp4(w1), pair=m.quantize_weights_fp4(w3)))
             q += list(m.pack_weights_w4a4(*m.quantize_weights_fp4(w2)))
+        elif w4a16:
+            q = list(m.pack_weights_w4a16(*m.quantize_weights_fp4(w1), pair=m.quantize_weights_fp4(w3)))
+            q += list(m.pack_weights_w4a16(*m.quantize_weights_fp4(w2)))
         else:
             q = [t for w in (w1, w3, w2) for t in quant(w)]
         torch.cuda.synchronize(dev)
@@ -529,6 +537,8 @@ def main():
             m.moe_forward_e4m3(layer.h, T, xin, Wg, *q, yout, iout, wout, stream)
         elif fp4:
             m.moe_forward_fp4(layer.h, T, xin, Wg, *q, yout, iout, wout, stream)
+        elif w4a16:
+            m.moe_forward_w4a16(layer.h, T, xin, Wg, *q, yout, iout, wout, stream)
         elif w4a4:
             m.moe_forward_w4a4(layer.h, T, xin, Wg, *q, yout, iout, wout, stream)
         else:
@@ -668,7 +678,8 @@ def main():
         roof["peak_source"] = peak_src
         roof["algorithmic_per_launch"] = work[dom]["bytes"] if roof["bound"] == "hbm" else work[dom]["flops"]
         roof["launch_ms"] = dom_ms
-        roof["traffic"] = recorded_traffic(dom, cfg.name + {"e4m3": "_e4m3", "fp4": "_fp4", "w4a4": "_w4a4"}.get(
+        roof["traffic"] = recorded_traffic(dom, cfg.name + {"e4m3": "_e4m3", "fp4": "_fp4", "w4a16": "_w4a16",
+                                                           "w4a4": "_w4a4"}.get(
             args.experts, ""))
 
     # ---- CPU baseline (rank 0, N = 1 only) ----
@@ -678,6 +689,7 @@ def main():
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": "first %d of %d tokens x %d repetitions, full layer in fp64%s (%.1f s)"
                          % (s, cfg.T, reps, {"e4m3": ", E4M3 experts", "fp4": ", 4-bit experts",
+                                             "w4a16": ", 4-bit experts",
                                              "w4a4": ", 4-bit experts and activations"}.get(args.experts, ""),
                             el)}
 
@@ -687,7 +699,7 @@ def main():
             "metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "e4m3" if e4m3 else ("e2m1 weights, bf16" if fp4 else ("e2m1" if w4a4 else cfg.dtype)),
+            "dtype": "e4m3" if e4m3 else ("e2m1 weights, bf16" if (fp4 or w4a16) else ("e2m1" if w4a4 else cfg.dtype)),
             "data": "synthetic",
             "config": {"workload": workload_desc(cfg, args.experts), "global_batch_tokens": T * world,
                        "parallelism": "replicas%d" % world if world > 1 else "single",

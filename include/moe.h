@@ -344,6 +344,56 @@ MOE_API moe_status moe_pack_weights_w4a4(int n, int rows, int cols, const uint8_
                                          uint8_t *scale_chunks, moe_stream_t stream);
 
 /*
+ * 4-bit weights with bf16 activations, the fast form (the weights at 4 bits
+ * as Part 4 of "Mixture of Experts: Why Mixtral Only Wakes Up Two
+ * Specialists" loads them; the layout is this library's).  The weights of
+ * moe_quantize_weights_fp4 are repacked once so that the GEMMs can decode
+ * them straight into tensor memory.  A matrix [n][rows][cols] becomes
+ *   packed [n][cols/128][rows/64][4608] bytes: for 128 columns and one 64-row
+ *   step, 4,096 bytes of codes as [2][128][16] (half h = rows 32h .. 32h+31 of
+ *   the step; per column four 32-bit words of 8 rows each, the bits of each
+ *   word arranged for the decoder: rows 2i and 2i+1 of the word come out of it
+ *   as one bf16 pair after a rotation by 0, 4, 10 bits (i = 0, 1, 2) or by 6
+ *   and 14 bits (i = 3) and a mask), then the 4 E4M3 block scales of each
+ *   column ([128][4] bytes).
+ * A gate/up pair (w1 with pair_codes / pair_block_scales = w3's) becomes one
+ * matrix of 2*cols packed columns whose tile j holds columns 64j .. 64j+63 of
+ * w1 and then the same columns of w3: packed [n][cols/64][rows/64][4608].
+ * Arguments: codes / block_scales (and the pair's) as moe_quantize_weights_fp4
+ * writes them; rows a multiple of 64; cols a multiple of 128 (64 for a pair).
+ * Needs no handle; enqueued on `stream`; the caller owns every buffer.
+ *   Errors: MOE_ERR_INVALID_ARG (sizes, null / misaligned pointer, one of the
+ *   pair pointers null), MOE_ERR_UNSUPPORTED (not an sm_100 device),
+ *   MOE_ERR_CUDA.
+ */
+MOE_API moe_status moe_pack_weights_w4a16(int n, int rows, int cols, const uint8_t *codes,
+                                          const uint8_t *block_scales, const uint8_t *pair_codes,
+                                          const uint8_t *pair_block_scales, uint8_t *packed,
+                                          moe_stream_t stream);
+
+/*
+ * The layer of moe_forward_fp4 (4-bit weights, bf16 activations: the bf16 layer
+ * of the dequantised weights E2M1(code) * sb, the accumulators multiplied by
+ * the matrix scales) on the packed weights of moe_pack_weights_w4a16: the
+ * GEMMs decode the codes straight into tensor memory, where the tensor core
+ * reads them, so the 4-bit weights cost 0.56 bytes each from memory and no
+ * shared-memory round trip.  MOE_BF16 handles with d a multiple of 128.
+ * w13_packed: the gate/up pair pack of w1 and w3 (rows = d, cols = ffn);
+ * w2_packed: w2 packed alone (rows = ffn, cols = d); w*_matrix_scales from
+ * moe_quantize_weights_fp4; x, W_g, y, topk_idx, topk_w as for moe_forward.
+ * The GEMMs take tokens in blocks of 32 rows when the experts average at most
+ * 32 rows per call (T*K <= 32*n), else 128 (MOE_W4A16_ROWS=32 or 128 forces
+ * one; same results either way).
+ *   Errors: as moe_forward; MOE_ERR_UNSUPPORTED for an fp32 handle or d not a
+ *   multiple of 128.
+ */
+MOE_API moe_status moe_forward_w4a16(moe_handle *h, int64_t T, const void *x, const float *W_g,
+                                     const uint8_t *w13_packed, const float *w1_matrix_scales,
+                                     const float *w3_matrix_scales, const uint8_t *w2_packed,
+                                     const float *w2_matrix_scales, void *y, int32_t *topk_idx,
+                                     float *topk_w, moe_stream_t stream);
+
+/*
  * The layer with 4-bit weights and 4-bit activations (MOE_BF16 handles with d
  * and ffn multiples of 256): the router, dispatch and capacity of moe_forward;
  * every gathered x row and every hidden row is quantised like a weight matrix

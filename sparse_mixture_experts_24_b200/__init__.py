@@ -69,6 +69,8 @@ lib.moe_quantize_weights_fp4.argtypes = [_int, _int, _int, _vp, _int, _vp, _vp, 
 lib.moe_forward_fp4.argtypes = [_vp, _i64, _vp, _vp] + [_vp] * 9 + [_vp, _vp, _vp, _vp]
 lib.moe_pack_weights_w4a4.argtypes = [_int, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.moe_forward_w4a4.argtypes = [_vp, _i64, _vp, _vp] + [_vp] * 7 + [_vp, _vp, _vp, _vp]
+lib.moe_pack_weights_w4a16.argtypes = [_int, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.moe_forward_w4a16.argtypes = [_vp, _i64, _vp, _vp] + [_vp] * 5 + [_vp, _vp, _vp, _vp]
 lib.moe_ep_dispatch.argtypes = [_vp, _int, _int, _i64, _vp, _vp, _vp, _vp, _i64, _vp, _vp]
 lib.moe_ep_experts.argtypes = [_vp, _int, _int, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp]
 lib.moe_ep_combine.argtypes = [_vp, _int, _i64, _vp, _vp, _vp, _vp, _vp, _vp]
@@ -83,7 +85,7 @@ for _f in ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispatc
            "moe_router_stats", "moe_launch_count", "moe_selftest_timeout",
            "moe_forward_expert_choice", "moe_quantize_weights_e4m3", "moe_forward_e4m3",
            "moe_quantize_weights_fp4", "moe_forward_fp4", "moe_pack_weights_w4a4", "moe_forward_w4a4",
-           "moe_ep_dispatch", "moe_ep_experts", "moe_ep_combine", "moe_ep_buffer_alloc", "moe_ep_buffer_open",
+           "moe_pack_weights_w4a16", "moe_forward_w4a16", "moe_ep_dispatch", "moe_ep_experts", "moe_ep_combine", "moe_ep_buffer_alloc", "moe_ep_buffer_open",
            "moe_ep_buffer_close", "moe_set_gate_rounding"):
     getattr(lib, _f).restype = _int
 
@@ -93,7 +95,8 @@ EXPORTED = ("moe_create", "moe_reserve", "moe_forward", "moe_route", "moe_dispat
             "moe_dispatch_noalloc", "moe_set_capacity_factor", "moe_router_stats",
             "moe_launch_count", "moe_selftest_timeout", "moe_forward_expert_choice",
             "moe_quantize_weights_e4m3", "moe_forward_e4m3", "moe_quantize_weights_fp4", "moe_forward_fp4",
-            "moe_pack_weights_w4a4", "moe_forward_w4a4", "moe_ep_dispatch", "moe_ep_experts", "moe_ep_combine",
+            "moe_pack_weights_w4a4", "moe_forward_w4a4", "moe_pack_weights_w4a16", "moe_forward_w4a16",
+            "moe_ep_dispatch", "moe_ep_experts", "moe_ep_combine",
             "moe_ep_buffer_alloc", "moe_ep_buffer_open", "moe_ep_buffer_close", "moe_set_gate_rounding")
 
 TRACE_STAGES = ("router", "dispatch", "gather", "gemm1", "gemm2", "combine")
@@ -307,6 +310,37 @@ def pack_weights_w4a4(codes, block_scales, matrix_scales, pair=None, stream=None
     return packed, chunks, matrix_scales
 
 
+def moe_pack_weights_w4a16(n, rows, cols, codes, block_scales, pair_codes, pair_block_scales, packed,
+                           stream=None) -> None:
+    _check(lib.moe_pack_weights_w4a16(n, rows, cols, _ptr(codes), _ptr(block_scales), _ptr(pair_codes),
+                                      _ptr(pair_block_scales), _ptr(packed), _stream(stream)),
+           "moe_pack_weights_w4a16")
+
+
+def moe_forward_w4a16(h, T, x, W_g, w13_p, w1_t, w3_t, w2_p, w2_t, y, topk_idx, topk_w, stream=None) -> None:
+    _check(lib.moe_forward_w4a16(h, T, _ptr(x), _ptr(W_g), _ptr(w13_p), _ptr(w1_t), _ptr(w3_t), _ptr(w2_p),
+                                 _ptr(w2_t), _ptr(y), _ptr(topk_idx), _ptr(topk_w), _stream(stream)),
+           "moe_forward_w4a16")
+
+
+def pack_weights_w4a16(codes, block_scales, matrix_scales, pair=None, stream=None):
+    """(codes [n][rows][cols/2], block scales [n][rows/16][cols], matrix scales [n])
+    of quantize_weights_fp4 (torch CUDA tensors) -> (packed [n][cols/128][rows/64][4608],
+    matrix scales).  With pair = w3's triple (codes being w1's): the gate/up pair
+    pack [n][cols/64][rows/64][4608], returned as (packed, w1 matrix scales,
+    w3 matrix scales)."""
+    import torch
+    n, rows, half = codes.shape
+    cols = 2 * half
+    tiles = cols // 64 if pair is not None else cols // 128
+    packed = torch.empty((n, tiles, rows // 64, 4608), dtype=torch.uint8, device=codes.device)
+    pc, pb = (pair[0], pair[1]) if pair is not None else (None, None)
+    moe_pack_weights_w4a16(n, rows, cols, codes, block_scales, pc, pb, packed, stream)
+    if pair is not None:
+        return packed, matrix_scales, pair[2]
+    return packed, matrix_scales
+
+
 def _ptr_table(ptrs):
     """Host array of device addresses (tensors, ints) for the peer tables."""
     return (ctypes.c_void_p * len(ptrs))(*[_ptr(p) for p in ptrs])
@@ -460,6 +494,21 @@ class MoELayer:
         if topk_w is None:
             topk_w = torch.empty((T, self.K), dtype=torch.float32, device=x.device)
         moe_forward_w4a4(self.h, T, x, W_g, *w13, *w2, y, topk_idx, topk_w, stream)
+        return y, topk_idx, topk_w
+
+    def forward_w4a16(self, x, W_g, w13, w2, y=None, topk_idx=None, topk_w=None, stream=None):
+        """The layer with 4-bit weights decoded into tensor memory and bf16
+        activations; w13 is the gate/up pair pack (packed, w1 scales, w3 scales)
+        and w2 the (packed, matrix scales) pair, both from pack_weights_w4a16."""
+        import torch
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty_like(x)
+        if topk_idx is None:
+            topk_idx = torch.empty((T, self.K), dtype=torch.int32, device=x.device)
+        if topk_w is None:
+            topk_w = torch.empty((T, self.K), dtype=torch.float32, device=x.device)
+        moe_forward_w4a16(self.h, T, x, W_g, *w13, *w2, y, topk_idx, topk_w, stream)
         return y, topk_idx, topk_w
 
     def set_capacity_factor(self, factor: float) -> None:

@@ -75,8 +75,27 @@ struct TileInfo {
     int e, n_tile, row0, rows;
 };
 
+// Tile order.  Tile t -> (expert, column tile, row block).  Per expert, with
+// A_e = its row blocks x a_blk_bytes and B_e = its column tiles x b_tile_bytes:
+//   plain   (A_e fits in the band budget, or no bands): the row block runs
+//           fastest over the whole expert; A_e stays in L2 while every
+//           column tile streams past it once.
+//   m-bands the row blocks are cut into bands of band_m blocks (the last may
+//           be shorter), row block fastest within a band: a band's A rows
+//           stay in L2, B_e streams once per band.
+//   n-bands the column tiles are cut into bands of band_n tiles, column tile
+//           fastest within a row block: a band's weight tiles stay in L2, A_e
+//           streams once per band.
+// Bands are chosen per expert by the smaller DRAM estimate (A_e + bands x B_e
+// against B_e + bands x A_e), so experts of a few row blocks keep the plain
+// order and a very large one (a skewed router's favourite) gets bands.
+struct TileOrder {
+    int band_m, band_n;             // 0: no bands
+    int64_t a_blk_bytes, b_tile_bytes;
+};
+
 __device__ __forceinline__ TileInfo tile_info(int t, const int32_t* off, const int32_t* mblk, int n,
-                                              int n_tiles) {
+                                              int n_tiles, const TileOrder& ord) {
     int lo = 0, hi = n - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -88,8 +107,45 @@ __device__ __forceinline__ TileInfo tile_info(int t, const int32_t* off, const i
     const int e = lo;
     const int local = t - mblk[e] * n_tiles;
     const int mb_count = mblk[e + 1] - mblk[e];
-    const int n_tile = local / mb_count;
-    const int m_blk = local - n_tile * mb_count;
+    int mode = 0;  // 0 plain, 1 m-bands, 2 n-bands
+    if (ord.band_m > 0 && mb_count > ord.band_m) {
+        const int64_t A = static_cast<int64_t>(mb_count) * ord.a_blk_bytes;
+        const int64_t B = static_cast<int64_t>(n_tiles) * ord.b_tile_bytes;
+        const int64_t cm = A + static_cast<int64_t>((mb_count + ord.band_m - 1) / ord.band_m) * B;
+        const int64_t cn = ord.band_n > 0 ? B + static_cast<int64_t>((n_tiles + ord.band_n - 1) / ord.band_n) * A
+                                          : cm + 1;
+        mode = cn < cm ? 2 : 1;
+    }
+    int n_tile, m_blk;
+    if (mode == 2) {
+        const int band = ord.band_n;
+        const int full = n_tiles / band * band;   // column tiles in whole bands
+        if (local < full * mb_count) {
+            const int b = local / (band * mb_count);
+            const int r = local - b * band * mb_count;
+            m_blk = r / band;
+            n_tile = b * band + (r - m_blk * band);
+        } else {
+            const int rem = n_tiles - full;
+            const int r = local - full * mb_count;
+            m_blk = r / rem;
+            n_tile = full + (r - m_blk * rem);
+        }
+    } else {
+        const int band = mode == 1 ? ord.band_m : mb_count;
+        const int full = mb_count / band * band;  // row blocks in whole bands
+        if (local < full * n_tiles) {
+            const int b = local / (band * n_tiles);
+            const int r = local - b * band * n_tiles;
+            n_tile = r / band;
+            m_blk = b * band + (r - n_tile * band);
+        } else {
+            const int rem = mb_count - full;
+            const int r = local - full * n_tiles;
+            n_tile = r / rem;
+            m_blk = full + (r - n_tile * rem);
+        }
+    }
     TileInfo ti;
     ti.e = e;
     ti.n_tile = n_tile;
@@ -99,6 +155,18 @@ __device__ __forceinline__ TileInfo tile_info(int t, const int32_t* off, const i
 }
 
 __device__ __forceinline__ float silu_f(float a) { return a / (1.f + __expf(-a)); }
+
+// Order of the reduction blocks of a tile.  GEMM2 (kSwiGLU false) walks K
+// downwards on odd column tiles: the tiles of one expert's row block that fall
+// into consecutive persistent rounds then meet at the same end of K, where the
+// H rows the previous round read last are still in L2 (measured on the prefill
+// shapes: 1.16x the algorithmic DRAM bytes with one direction).  The direction
+// depends only on the column tile, so every output element is summed in one
+// fixed order however the rows are tiled.
+template <bool kSwiGLU>
+__device__ __forceinline__ int k_block_at_t(int kb, int k_blocks, int n_tile, int alternate) {
+    return (!kSwiGLU && alternate && (n_tile & 1)) ? k_blocks - 1 - kb : kb;
+}
 
 // kSwiGLU: GEMM1 (two B maps, 128 output columns per tile); else GEMM2.
 // kFp8: E4M3 operands with the scales of TcGemmArgs applied in the epilogue.
@@ -151,6 +219,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int stride = args.balanced ? balanced_ctas(total_tiles, static_cast<int>(gridDim.x))
                                      : static_cast<int>(gridDim.x);
     const int first = static_cast<int>(blockIdx.x) < stride ? static_cast<int>(blockIdx.x) : total_tiles;
+    TileOrder ord;
+    ord.band_m = args.band_m;
+    ord.band_n = args.band_n;
+    ord.a_blk_bytes = static_cast<int64_t>(kBM) * args.k_blocks * (kFp8 ? kBK8 : kBK * 2);
+    ord.b_tile_bytes = static_cast<int64_t>(kBN) * args.k_blocks * (kFp8 ? kBK8 : kBK * 2);
     int* status = args.status;
 
     if (warp == 0) {
@@ -162,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int s = 0; s < kStages; ++s) armed[s] = -1;
             bool ok = true;
             for (int t = first; t < total_tiles && ok; t += stride) {
-                const TileInfo ti = tile_info(t, tail->off, tail->mblk, n, args.n_tiles);
+                const TileInfo ti = tile_info(t, tail->off, tail->mblk, n, args.n_tiles, ord);
                 for (int kb = 0; kb < args.k_blocks; ++kb) {
                     if (!mbar_wait(smem_u32(&tail->empty[stage]), phase ^ 1u, status,
                                    kStatusTimeoutEmpty)) {
@@ -174,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     armed[stage] = static_cast<int>(phase);
                     const uint32_t a_dst = smem_u32(smem + stage * kStageBytes);
                     const uint32_t b_dst = a_dst + kABytes;
-                    const int k0 = kb * (kFp8 ? kBK8 : kBK);
+                    const int k0 = k_block_at_t<kSwiGLU>(kb, args.k_blocks, ti.n_tile, args.k_alternate) * (kFp8 ? kBK8 : kBK);
                     tma_load_2d(a_dst, &tm_a, fb, k0, ti.row0);
                     if (kFp8) {
                         if (kSwiGLU) {
@@ -278,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* stage = smem + kStages * kStageBytes + kTailBytes + (warp - 2) * kWarpStageBytes;
         int local = 0;
         for (int t = first; t < total_tiles; t += stride, ++local) {
-            const TileInfo ti = tile_info(t, tail->off, tail->mblk, n, args.n_tiles);
+            const TileInfo ti = tile_info(t, tail->off, tail->mblk, n, args.n_tiles, ord);
             const int buf = local & 1;
             const uint32_t bph = static_cast<uint32_t>(local >> 1) & 1u;
             if (!mbar_wait(smem_u32(&tail->accum_full[buf]), bph, status, kStatusTimeoutAccum)) break;

@@ -184,6 +184,12 @@ struct TcGemmArgs {
     const float* col_scale0;
     const float* col_scale1;
     int balanced;      // 1: spread the tiles evenly over the fewest CTAs (balanced_ctas)
+    // single-SM kernel, tile order (gemm_tc.cu): row blocks per m-band and
+    // column tiles per n-band (0: no bands), and whether GEMM2 walks K
+    // downwards on odd column tiles
+    int band_m;
+    int band_n;
+    int k_alternate;
 };
 
 cudaError_t launch_tc_gemm1(const CUtensorMap& tm_xp, const CUtensorMap& tm_w1,
@@ -276,6 +282,37 @@ cudaError_t launch_w4a4_gemm1(const CUtensorMap& tm_xq, const CUtensorMap& tm_w1
 cudaError_t launch_w4a4_gemm2(const CUtensorMap& tm_hq, const CUtensorMap& tm_w2, const W4a4GemmArgs& a, bool wide,
                               int tile_rows, int num_sms, cudaStream_t st);
 
+// 4-bit weights with bf16 activations, the weights decoded into tensor
+// memory (gemm_w4a16.cu).  Packed weights: per (expert, tile of 128 packed
+// columns, 64 reduction rows) a 4,608-byte block of codes ([2][128][16]
+// bytes, 8 rows per 32-bit word in the decoder's bit order) and block scales
+// ([128][4] E4M3 codes).  With codes_pair (w3 beside w1) tile j holds columns
+// 64j .. 64j+63 of w1 then the same columns of w3.  K % 64 == 0; N % 128 == 0
+// (N % 64 == 0 with a pair).
+cudaError_t launch_w4a16_pack(const uint8_t* codes, const uint8_t* bscale, const uint8_t* codes_pair,
+                              const uint8_t* bscale_pair, int n, int K, int N, uint8_t* packed, cudaStream_t st);
+struct W4a16GemmArgs {
+    const int32_t* offsets;
+    const int32_t* mblk_base;  // per-expert prefix of tile_rows-row blocks
+    int n;
+    int64_t R;
+    int k_blocks;          // reduction length / 64
+    int n_tiles;           // weight tiles per expert (F / 64 for GEMM1, d / 128 for GEMM2)
+    int out_cols;          // F (GEMM1) or d (GEMM2)
+    void* out;             // bf16 [R][out_cols]
+    int* status;
+    const uint8_t* wpack;  // packed weights [n][n_tiles][k_blocks][4608]
+    const float* mscale0;  // [n] matrix scales: w1 (GEMM1) / w2 (GEMM2)
+    const float* mscale1;  // [n] w3 (GEMM1)
+    int balanced;          // as TcGemmArgs::balanced
+};
+// Token rows per tile: 32 when the experts average at most 32 rows, else 128.
+int w4a16_tile_rows(int64_t R, int n);
+// tm_xp / tm_h: bf16 rows in 64 x tile_rows boxes, 128-byte swizzle.
+cudaError_t launch_w4a16_gemm1(const CUtensorMap& tm_xp, const W4a16GemmArgs& a, int tile_rows, int num_sms,
+                               cudaStream_t st);
+cudaError_t launch_w4a16_gemm2(const CUtensorMap& tm_h, const W4a16GemmArgs& a, int tile_rows, int num_sms,
+                               cudaStream_t st);
 // E4M3 quantisation (e4m3.cu).  Codes are those of v / scale with the quotient
 // rounded to fp32, then to E4M3 by round-to-nearest-even with saturation to
 // +-448; scale = max |v| / 448 over the group (1 for an all-zero group).

@@ -222,6 +222,8 @@ struct moe_handle {
     CUtensorMap tm_xq4, tm_hq4, tm_wp4[2];
     CUtensorMap tm_xq4s, tm_hq4s;  // the same codes in 32-row boxes
     const void* c_wp4[2] = {nullptr, nullptr};
+    // 4-bit weights decoded into tensor memory: Xp and H in 32-row boxes
+    CUtensorMap tm_xp32, tm_h32;
     // 4-bit experts: maps over the caller's codes and block scales
     CUtensorMap tm_f4[6];  // codes w1, scales w1, codes w3, scales w3, codes w2, scales w2
     const void* c_f4[6] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
@@ -405,6 +407,8 @@ moe_status grow(moe_handle* h, int64_t T, int64_t rows_min = 0) {
     if (h->dtype == MOE_BF16) {
         if (!encode_rows(&h->tm_xp, h->xp, h->d, static_cast<uint64_t>(R)) ||
             !encode_rows(&h->tm_h, h->h, h->F, static_cast<uint64_t>(R)) ||
+            !encode_rows(&h->tm_xp32, h->xp, h->d, static_cast<uint64_t>(R), 32) ||
+            !encode_rows(&h->tm_h32, h->h, h->F, static_cast<uint64_t>(R), 32) ||
             !encode_rows(&h->tm_parts, h->wg_parts, h->d, static_cast<uint64_t>(3 * npad),
                          static_cast<uint32_t>(npad)))
             return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the workspace");
@@ -491,6 +495,29 @@ int grid_balance() {
     return (env && strcmp(env, "0") == 0) ? 0 : 1;
 }
 
+// Tile order of the single-SM GEMMs (gemm_tc.cu): bands of row blocks and of
+// column tiles sized to MOE_GEMM_BAND_MB megabytes of A rows / weight columns
+// (unset or 0: no bands), MOE_GEMM_BAND_AXIS=m or n to allow only one axis,
+// and MOE_GEMM2_KALT=0 to walk K upwards on every GEMM2 column tile.
+void gemm_tile_order(moe::TcGemmArgs& a, int64_t a_row_bytes, int64_t b_col_bytes, int b_cols) {
+    a.k_alternate = 1;
+    if (const char* v = getenv("MOE_GEMM2_KALT")) a.k_alternate = atoi(v) != 0;
+    a.band_m = a.band_n = 0;
+    const char* env = getenv("MOE_GEMM_BAND_MB");
+    if (!env) return;
+    const int64_t mb = atoll(env);
+    if (mb <= 0) return;
+    const int64_t budget = mb << 20;
+    const char* axis = getenv("MOE_GEMM_BAND_AXIS");
+    const bool allow_m = !axis || strcmp(axis, "n") != 0;
+    const bool allow_n = !axis || strcmp(axis, "m") != 0;
+    const int64_t bm = budget / (static_cast<int64_t>(moe::kTcBM) * a_row_bytes);
+    const int64_t bn = budget / (static_cast<int64_t>(b_cols) * b_col_bytes);
+    a.band_m = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(bm, 1 << 20)));
+    a.band_n = allow_n ? static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(bn, 1 << 20))) : 0;
+    if (!allow_m) a.band_m = 1;  // always banded, and n-bands win whenever they are cheaper
+}
+
 // Most (token, slot) pairs one expert takes in a call of T tokens:
 // ceil(factor * T * K / n), or no limit when the factor is 0.
 int capacity_for(const moe_handle* h, int64_t T) {
@@ -535,7 +562,8 @@ moe_status run_gemms(moe_handle* h, int64_t T, int64_t R, const void* x, const v
         a1.out_cols = h->F;
         a1.out = h->h;
         a1.status = h->status;
-    a1.balanced = grid_balance();
+        a1.balanced = grid_balance();
+        gemm_tile_order(a1, static_cast<int64_t>(h->d) * 2, static_cast<int64_t>(h->d) * 2, 256);
         e = pair ? moe::launch_tc_gemm1_pair(h->tm_xp, h->tm_w1, h->tm_w3, a1, h->num_sms, st)
                  : moe::launch_tc_gemm1(h->tm_xp, h->tm_w1, h->tm_w3, a1, h->num_sms, st);
         if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
@@ -546,6 +574,7 @@ moe_status run_gemms(moe_handle* h, int64_t T, int64_t R, const void* x, const v
         a2.n_tiles = (h->d + 255) / 256;
         a2.out_cols = h->d;
         a2.out = h->o;
+        gemm_tile_order(a2, static_cast<int64_t>(h->F) * 2, static_cast<int64_t>(h->F) * 2, 256);
         e = pair ? moe::launch_tc_gemm2_pair(h->tm_h, h->tm_w2, a2, h->num_sms, st)
                  : moe::launch_tc_gemm2(h->tm_h, h->tm_w2, a2, h->num_sms, st);
         if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
@@ -638,6 +667,7 @@ moe_status run_experts_e4m3(moe_handle* h, int64_t T, const void* x, const int32
     a1.row_scale = h->xs;
     a1.col_scale0 = s1;
     a1.col_scale1 = s3;
+    gemm_tile_order(a1, h->d, h->d, 256);
     e = pair ? moe::launch_tc_gemm1_pair_e4m3(h->tm_x8, h->tm_q1, h->tm_q3, a1, h->num_sms, st)
              : moe::launch_tc_gemm1_e4m3(h->tm_x8, h->tm_q1, h->tm_q3, a1, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
@@ -653,6 +683,7 @@ moe_status run_experts_e4m3(moe_handle* h, int64_t T, const void* x, const int32
     a2.row_scale = h->hs;
     a2.col_scale0 = s2;
     a2.col_scale1 = nullptr;
+    gemm_tile_order(a2, h->F, h->F, 256);
     e = pair ? moe::launch_tc_gemm2_pair_e4m3(h->tm_h8, h->tm_q2, a2, h->num_sms, st)
              : moe::launch_tc_gemm2_e4m3(h->tm_h8, h->tm_q2, a2, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
@@ -809,6 +840,64 @@ moe_status run_experts_w4a4(moe_handle* h, int64_t T, const void* x, const float
     a2.b_chunks = wc[1];
     e = moe::launch_w4a4_gemm2(tile_rows == 32 ? h->tm_hq4s : h->tm_hq4, h->tm_wp4[1], a2, wide, tile_rows,
                                h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
+    h->launches += 1;
+    trace_mark(h, 4, st);
+    e = moe::launch_combine(h->o, true, h->db.token_row, topk_w, T, h->K, h->d, y, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+    h->launches += 1;
+    trace_mark(h, 5, st);
+    trace_finish_call(h);
+    return MOE_OK;
+}
+
+// 4-bit weights with bf16 activations, decoded into tensor memory: dispatch
+// (token blocks of 32 rows when the experts average at most 32 rows, else
+// 128), gather, GEMM1 over the gate/up pair pack, GEMM2, combine.
+moe_status run_experts_w4a16(moe_handle* h, int64_t T, const void* x, const float* topk_w,
+                             const uint8_t* const* wp, const float* const* ws, void* y, const int32_t* topk_idx,
+                             cudaStream_t st) {
+    const int64_t R = T * h->K;
+    int tile_rows = moe::w4a16_tile_rows(R, h->n);
+    if (const char* v = getenv("MOE_W4A16_ROWS")) {  // 32 or 128 forces the token block
+        if (atoi(v) == 32) tile_rows = 32;
+        if (atoi(v) == 128) tile_rows = 128;
+    }
+    cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n, tile_rows, h->db, st, capacity_for(h, T));
+    if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
+    h->launches += moe::dispatch_kernel_count(R);
+    trace_mark(h, 1, st);
+    e = moe::launch_gather(x, h->db.row_token, R, T, static_cast<int64_t>(h->d) * 2, h->xp, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+    h->launches += 1;
+    trace_mark(h, 2, st);
+    moe::W4a16GemmArgs a1{};
+    a1.offsets = h->db.offsets;
+    a1.mblk_base = h->db.mblk_base;
+    a1.n = h->n;
+    a1.R = R;
+    a1.k_blocks = h->d / 64;
+    a1.n_tiles = h->F / 64;
+    a1.out_cols = h->F;
+    a1.out = h->h;
+    a1.status = h->status;
+    a1.wpack = wp[0];
+    a1.mscale0 = ws[0];
+    a1.mscale1 = ws[1];
+    a1.balanced = grid_balance();
+    e = moe::launch_w4a16_gemm1(tile_rows == 32 ? h->tm_xp32 : h->tm_xp, a1, tile_rows, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
+    h->launches += 1;
+    trace_mark(h, 3, st);
+    moe::W4a16GemmArgs a2 = a1;
+    a2.k_blocks = h->F / 64;
+    a2.n_tiles = h->d / 128;
+    a2.out_cols = h->d;
+    a2.out = h->o;
+    a2.wpack = wp[1];
+    a2.mscale0 = ws[2];
+    a2.mscale1 = ws[2];
+    e = moe::launch_w4a16_gemm2(tile_rows == 32 ? h->tm_h32 : h->tm_h, a2, tile_rows, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
     h->launches += 1;
     trace_mark(h, 4, st);
@@ -1249,6 +1338,70 @@ moe_status moe_forward_w4a4(moe_handle* h, int64_t T, const void* x, const float
     return s == MOE_OK ? ok() : s;
 }
 
+moe_status moe_pack_weights_w4a16(int n, int rows, int cols, const uint8_t* codes, const uint8_t* block_scales,
+                                   const uint8_t* pair_codes, const uint8_t* pair_block_scales, uint8_t* packed,
+                                   moe_stream_t stream) {
+    if (n < 1 || n > 65535) return fail(MOE_ERR_INVALID_ARG, "n = %d outside [1, 65535]", n);
+    if (rows < 64 || rows % 64 != 0 || rows > 1048576)
+        return fail(MOE_ERR_INVALID_ARG, "rows = %d is not a multiple of 64 in [64, 1048576]", rows);
+    if (pair_codes) {
+        if (cols < 64 || cols % 64 != 0 || cols > 1048576)
+            return fail(MOE_ERR_INVALID_ARG, "cols = %d is not a multiple of 64 in [64, 1048576]", cols);
+    } else if (cols < 128 || cols % 128 != 0 || cols > 1048576) {
+        return fail(MOE_ERR_INVALID_ARG, "cols = %d is not a multiple of 128 in [128, 1048576]", cols);
+    }
+    if ((pair_codes == nullptr) != (pair_block_scales == nullptr))
+        return fail(MOE_ERR_INVALID_ARG, "pair_codes and pair_block_scales must both be given or both be null");
+    if (static_cast<int64_t>(pair_codes ? 2 * cols : cols) * (rows / 64) > 2147483647LL / 256)
+        return fail(MOE_ERR_INVALID_ARG, "rows * cols too large");
+    REQUIRE_PTR(codes);
+    REQUIRE_PTR(block_scales);
+    REQUIRE_PTR(packed);
+    int dev = 0, major = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (major != 10) return fail(MOE_ERR_UNSUPPORTED, "device %d is not sm_100", dev);
+    e = moe::launch_w4a16_pack(codes, block_scales, pair_codes, pair_block_scales, n, rows, cols, packed,
+                               reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "4-bit weight packing launch");
+    return ok();
+}
+
+moe_status moe_forward_w4a16(moe_handle* h, int64_t T, const void* x, const float* W_g, const uint8_t* w13_packed,
+                             const float* w1_matrix_scales, const float* w3_matrix_scales, const uint8_t* w2_packed,
+                             const float* w2_matrix_scales, void* y, int32_t* topk_idx, float* topk_w,
+                             moe_stream_t stream) {
+    moe_status s = check_common(h, T);
+    if (s != MOE_OK) return s;
+    if (h->dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "the 4-bit weight path needs a MOE_BF16 handle");
+    if (h->d % 128 != 0)
+        return fail(MOE_ERR_UNSUPPORTED, "the 4-bit weight path needs d a multiple of 128 (d = %d)", h->d);
+    if (T == 0) return ok();
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(W_g);
+    REQUIRE_PTR(w13_packed);
+    REQUIRE_PTR(w1_matrix_scales);
+    REQUIRE_PTR(w3_matrix_scales);
+    REQUIRE_PTR(w2_packed);
+    REQUIRE_PTR(w2_matrix_scales);
+    REQUIRE_PTR(y);
+    REQUIRE_PTR(topk_idx);
+    REQUIRE_PTR(topk_w);
+    s = prepare(h, T);
+    if (s != MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    moe::chain_begin();
+    trace_mark(h, -1, st);
+    s = run_router(h, T, x, W_g, topk_idx, topk_w, st);
+    if (s != MOE_OK) return s;
+    trace_mark(h, 0, st);
+    const uint8_t* wp[2] = {w13_packed, w2_packed};
+    const float* ws[3] = {w1_matrix_scales, w3_matrix_scales, w2_matrix_scales};
+    s = run_experts_w4a16(h, T, x, topk_w, wp, ws, y, topk_idx, st);
+    return s == MOE_OK ? ok() : s;
+}
+
 moe_status moe_ep_dispatch(moe_handle* h, int world, int rank, int64_t T, const void* x, const int32_t* topk_idx,
                            const int32_t* counts_all, void* const* recv_buffers, int64_t recv_rows,
                            int32_t* row_pos, moe_stream_t stream) {
@@ -1332,6 +1485,7 @@ moe_status moe_ep_experts(moe_handle* h, int world, int rank, const int32_t* cou
     a1.out = h->h;
     a1.status = h->status;
     a1.balanced = grid_balance();
+    gemm_tile_order(a1, static_cast<int64_t>(h->d) * 2, static_cast<int64_t>(h->d) * 2, 256);
     e = moe::launch_tc_gemm1(h->tm_erecv, h->tm_ew1, h->tm_ew3, a1, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
     moe::TcGemmArgs a2 = a1;
@@ -1339,6 +1493,7 @@ moe_status moe_ep_experts(moe_handle* h, int world, int rank, const int32_t* cou
     a2.n_tiles = (h->d + 255) / 256;
     a2.out_cols = h->d;
     a2.out = out;
+    gemm_tile_order(a2, static_cast<int64_t>(h->F) * 2, static_cast<int64_t>(h->F) * 2, 256);
     e = moe::launch_tc_gemm2(h->tm_h, h->tm_ew2, a2, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
     h->launches += 3;
