@@ -13,8 +13,12 @@
 // Design (one persistent CTA per SM, 192 threads):
 //   warp 0   one thread issues TMA loads into a kStages-deep ring of shared
 //            memory stages (A: 128 rows x 64 of Xp or H, K-major, 128-byte
-//            swizzle; B: 64 x 256 of the weights, N-major, as four 64-column
-//            boxes, 128-byte swizzle).  GEMM1's B is 128 columns of w1 next to
+//            swizzle; B: 64 x 256 of the weights, N-major, four 64-column
+//            chunks, 128-byte swizzle).  The bf16 weight maps are 4-D (64
+//            columns, K rows, 64-column chunk, expert) so that one copy brings
+//            several chunks: a stage is 2 copies (GEMM2) or 3 (GEMM1) instead
+//            of 5 -- the producer thread issuing those copies, not the tensor
+//            core, was what held the tensor pipe near 80% busy.  GEMM1's B is 128 columns of w1 next to
 //            the same 128 columns of w3, so ONE N=256 MMA produces both the
 //            gate and the up projection of a 128-column slice of H.
 //   warp 1   allocates 512 TMEM columns (two 256-column fp32 accumulators);
@@ -55,6 +59,7 @@ constexpr int kBBytes = 4 * kBChunkBytes;         // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;    // 48 KB
 constexpr int kTmemCols = 512;
 constexpr int kThreads = 192;
+constexpr int kGatherThreads = 320;  // + 4 warps gathering A rows from x (GEMM1, bf16)
 constexpr int kMaxN = 256;
 
 struct __align__(8) TcSmemTail {
@@ -75,27 +80,18 @@ struct TileInfo {
     int e, n_tile, row0, rows;
 };
 
-// Tile order.  Tile t -> (expert, column tile, row block).  Per expert, with
-// A_e = its row blocks x a_blk_bytes and B_e = its column tiles x b_tile_bytes:
-//   plain   (A_e fits in the band budget, or no bands): the row block runs
-//           fastest over the whole expert; A_e stays in L2 while every
-//           column tile streams past it once.
-//   m-bands the row blocks are cut into bands of band_m blocks (the last may
-//           be shorter), row block fastest within a band: a band's A rows
-//           stay in L2, B_e streams once per band.
-//   n-bands the column tiles are cut into bands of band_n tiles, column tile
-//           fastest within a row block: a band's weight tiles stay in L2, A_e
-//           streams once per band.
-// Bands are chosen per expert by the smaller DRAM estimate (A_e + bands x B_e
-// against B_e + bands x A_e), so experts of a few row blocks keep the plain
-// order and a very large one (a skewed router's favourite) gets bands.
-struct TileOrder {
-    int band_m, band_n;             // 0: no bands
-    int64_t a_blk_bytes, b_tile_bytes;
-};
-
+// Tile order.  Tile t -> (expert, column tile, row block).  An expert's row
+// blocks are cut into bands of `band` blocks (the last may be shorter); within
+// a band the row block runs fastest, then the column tile, so a band's A rows
+// stay in L2 while every weight column tile of the expert streams past them
+// once per band.  An expert of at most `band` blocks is one band: its A rows
+// stay in L2 for all its column tiles.  Bands matter when one expert takes
+// far more rows than L2 holds (a skewed router's favourite): unbanded, every
+// round of persistent tiles would stream all of that expert's A rows again
+// (measured on the skewed prefill: 11.9 GB of DRAM reads in GEMM1 against
+// 2.9 GB with bands of 32 MB of A rows).
 __device__ __forceinline__ TileInfo tile_info(int t, const int32_t* off, const int32_t* mblk, int n,
-                                              int n_tiles, const TileOrder& ord) {
+                                              int n_tiles, int band_limit) {
     int lo = 0, hi = n - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -107,44 +103,19 @@ __device__ __forceinline__ TileInfo tile_info(int t, const int32_t* off, const i
     const int e = lo;
     const int local = t - mblk[e] * n_tiles;
     const int mb_count = mblk[e + 1] - mblk[e];
-    int mode = 0;  // 0 plain, 1 m-bands, 2 n-bands
-    if (ord.band_m > 0 && mb_count > ord.band_m) {
-        const int64_t A = static_cast<int64_t>(mb_count) * ord.a_blk_bytes;
-        const int64_t B = static_cast<int64_t>(n_tiles) * ord.b_tile_bytes;
-        const int64_t cm = A + static_cast<int64_t>((mb_count + ord.band_m - 1) / ord.band_m) * B;
-        const int64_t cn = ord.band_n > 0 ? B + static_cast<int64_t>((n_tiles + ord.band_n - 1) / ord.band_n) * A
-                                          : cm + 1;
-        mode = cn < cm ? 2 : 1;
-    }
+    const int band = min(mb_count, band_limit);
+    const int full = mb_count / band * band;  // row blocks in whole bands
     int n_tile, m_blk;
-    if (mode == 2) {
-        const int band = ord.band_n;
-        const int full = n_tiles / band * band;   // column tiles in whole bands
-        if (local < full * mb_count) {
-            const int b = local / (band * mb_count);
-            const int r = local - b * band * mb_count;
-            m_blk = r / band;
-            n_tile = b * band + (r - m_blk * band);
-        } else {
-            const int rem = n_tiles - full;
-            const int r = local - full * mb_count;
-            m_blk = r / rem;
-            n_tile = full + (r - m_blk * rem);
-        }
+    if (local < full * n_tiles) {
+        const int b = local / (band * n_tiles);
+        const int r = local - b * band * n_tiles;
+        n_tile = r / band;
+        m_blk = b * band + (r - n_tile * band);
     } else {
-        const int band = mode == 1 ? ord.band_m : mb_count;
-        const int full = mb_count / band * band;  // row blocks in whole bands
-        if (local < full * n_tiles) {
-            const int b = local / (band * n_tiles);
-            const int r = local - b * band * n_tiles;
-            n_tile = r / band;
-            m_blk = b * band + (r - n_tile * band);
-        } else {
-            const int rem = mb_count - full;
-            const int r = local - full * n_tiles;
-            n_tile = r / rem;
-            m_blk = full + (r - n_tile * rem);
-        }
+        const int rem = mb_count - full;
+        const int r = local - full * n_tiles;
+        n_tile = r / rem;
+        m_blk = full + (r - n_tile * rem);
     }
     TileInfo ti;
     ti.e = e;
@@ -156,22 +127,28 @@ __device__ __forceinline__ TileInfo tile_info(int t, const int32_t* off, const i
 
 __device__ __forceinline__ float silu_f(float a) { return a / (1.f + __expf(-a)); }
 
-// Order of the reduction blocks of a tile.  GEMM2 (kSwiGLU false) walks K
-// downwards on odd column tiles: the tiles of one expert's row block that fall
-// into consecutive persistent rounds then meet at the same end of K, where the
-// H rows the previous round read last are still in L2 (measured on the prefill
-// shapes: 1.16x the algorithmic DRAM bytes with one direction).  The direction
-// depends only on the column tile, so every output element is summed in one
-// fixed order however the rows are tiled.
-template <bool kSwiGLU>
-__device__ __forceinline__ int k_block_at_t(int kb, int k_blocks, int n_tile, int alternate) {
-    return (!kSwiGLU && alternate && (n_tile & 1)) ? k_blocks - 1 - kb : kb;
-}
-
 // kSwiGLU: GEMM1 (two B maps, 128 output columns per tile); else GEMM2.
 // kFp8: E4M3 operands with the scales of TcGemmArgs applied in the epilogue.
-template <bool kSwiGLU, bool kFp8>
-__global__ void __launch_bounds__(kThreads, 1)
+// 16-byte copy global -> shared (zero-filled when src_bytes is 0), in the
+// thread's current cp.async group.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
+}
+
+// kGather (GEMM1, bf16 only): A is not read from Xp by TMA; warps 6-9 gather
+// the tile's rows straight from x (row r of the tile = token row_token[row0 +
+// r]) with 16-byte cp.async copies into the same 128-byte-swizzled layout,
+// so the gather kernel and the Xp round trip through HBM are gone.  Each
+// gather thread owns one 16-byte column chunk of 8 rows; it retires a stage
+// (waits for its copies, fences them for the tensor core's async proxy,
+// arrives on the stage's full barrier) two stages after issuing it.
+template <bool kSwiGLU, bool kFp8, bool kGather>
+__global__ void __launch_bounds__(kGather ? kGatherThreads : kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
                    const __grid_constant__ CUtensorMap tm_b1, const TcGemmArgs args) {
     extern __shared__ uint8_t smem_raw[];
@@ -184,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(smem_u32(&tail->full[s]), 1);
+            mbar_init(smem_u32(&tail->full[s]), kGather ? 5 : 1);  // TMA (+ the 4 gather warps)
             mbar_init(smem_u32(&tail->empty[s]), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -207,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // everything above overlaps the previous kernel; its outputs (segment
     // offsets, the A operand) are read only after this wait
     griddep_wait();
-    for (int i = threadIdx.x; i <= n; i += kThreads) {
+    for (int i = threadIdx.x; i <= n; i += static_cast<int>(blockDim.x)) {
         tail->off[i] = args.offsets[i];
         tail->mblk[i] = args.mblk_base[i];
     }
@@ -219,11 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int stride = args.balanced ? balanced_ctas(total_tiles, static_cast<int>(gridDim.x))
                                      : static_cast<int>(gridDim.x);
     const int first = static_cast<int>(blockIdx.x) < stride ? static_cast<int>(blockIdx.x) : total_tiles;
-    TileOrder ord;
-    ord.band_m = args.band_m;
-    ord.band_n = args.band_n;
-    ord.a_blk_bytes = static_cast<int64_t>(kBM) * args.k_blocks * (kFp8 ? kBK8 : kBK * 2);
-    ord.b_tile_bytes = static_cast<int64_t>(kBN) * args.k_blocks * (kFp8 ? kBK8 : kBK * 2);
+    const int band_limit = args.band_m > 0 ? args.band_m : 0x40000000;
     int* status = args.status;
 
     if (warp == 0) {
@@ -235,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int s = 0; s < kStages; ++s) armed[s] = -1;
             bool ok = true;
             for (int t = first; t < total_tiles && ok; t += stride) {
-                const TileInfo ti = tile_info(t, tail->off, tail->mblk, n, args.n_tiles, ord);
+                const TileInfo ti = tile_info(t, tail->off, tail->mblk, n, args.n_tiles, band_limit);
                 for (int kb = 0; kb < args.k_blocks; ++kb) {
                     if (!mbar_wait(smem_u32(&tail->empty[stage]), phase ^ 1u, status,
                                    kStatusTimeoutEmpty)) {
@@ -243,12 +216,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     const uint32_t fb = smem_u32(&tail->full[stage]);
-                    mbar_arrive_expect_tx(fb, kStageBytes);
+                    mbar_arrive_expect_tx(fb, kGather ? kBBytes : kStageBytes);
                     armed[stage] = static_cast<int>(phase);
                     const uint32_t a_dst = smem_u32(smem + stage * kStageBytes);
                     const uint32_t b_dst = a_dst + kABytes;
-                    const int k0 = k_block_at_t<kSwiGLU>(kb, args.k_blocks, ti.n_tile, args.k_alternate) * (kFp8 ? kBK8 : kBK);
-                    tma_load_2d(a_dst, &tm_a, fb, k0, ti.row0);
+                    const int k0 = kb * (kFp8 ? kBK8 : kBK);
+                    if (!kGather) tma_load_2d(a_dst, &tm_a, fb, k0, ti.row0);
                     if (kFp8) {
                         if (kSwiGLU) {
                             const int c0 = ti.n_tile * 128;
@@ -260,16 +233,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tma_load_3d(b_dst + kB8ChunkBytes, &tm_b0, fb, c0 + 128, k0, ti.e);
                         }
                     } else if (kSwiGLU) {
-                        const int c0 = ti.n_tile * 128;
-                        tma_load_3d(b_dst + 0 * kBChunkBytes, &tm_b0, fb, c0, k0, ti.e);
-                        tma_load_3d(b_dst + 1 * kBChunkBytes, &tm_b0, fb, c0 + 64, k0, ti.e);
-                        tma_load_3d(b_dst + 2 * kBChunkBytes, &tm_b1, fb, c0, k0, ti.e);
-                        tma_load_3d(b_dst + 3 * kBChunkBytes, &tm_b1, fb, c0 + 64, k0, ti.e);
+                        // the weight maps are 4-D (64 columns, K rows, 64-column chunk,
+                        // expert): one copy brings two whole 64-column chunks
+                        tma_load_4d(b_dst, &tm_b0, fb, 0, k0, ti.n_tile * 2, ti.e);
+                        tma_load_4d(b_dst + 2 * kBChunkBytes, &tm_b1, fb, 0, k0, ti.n_tile * 2, ti.e);
                     } else {
-                        const int c0 = ti.n_tile * 256;
-#pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            tma_load_3d(b_dst + c * kBChunkBytes, &tm_b0, fb, c0 + 64 * c, k0, ti.e);
+                        tma_load_4d(b_dst, &tm_b0, fb, 0, k0, ti.n_tile * 4, ti.e);  // four chunks
                     }
                     if (++stage == kStages) {
                         stage = 0;
@@ -345,13 +314,73 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_commit(smem_u32(&tail->done));
             mbar_wait(smem_u32(&tail->done), 0, status, kStatusTimeoutDrain);
         }
+    } else if (kGather && warp >= 6) {
+        // ---------------- A gather (warps 6..9) ----------------
+        const int gt = static_cast<int>(threadIdx.x) - kThreads;  // 0..127
+        const int c = gt & 7;                                      // 16-byte chunk of a 128-byte row slice
+        const int r0 = gt >> 3;                                    // rows r0, r0 + 16, ..., r0 + 112
+        const uint16_t* x = args.x;
+        int stage = 0;
+        uint32_t phase = 0;
+        int pend[2] = {0, 0};
+        int npend = 0;
+        bool ok = true;
+        for (int t = first; t < total_tiles && ok; t += stride) {
+            const TileInfo ti = tile_info(t, tail->off, tail->mblk, n, args.n_tiles, band_limit);
+            const uint16_t* src[8];
+            uint32_t bytes[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int r = r0 + 16 * i;
+                const int tok = r < ti.rows ? __ldg(args.row_token + ti.row0 + r) : -1;
+                const bool valid = tok >= 0 && tok < args.x_rows;
+                src[i] = x + (valid ? static_cast<int64_t>(tok) * args.x_cols : 0) + c * 8;
+                bytes[i] = valid ? 16u : 0u;
+            }
+            for (int kb = 0; kb < args.k_blocks; ++kb) {
+                uint32_t okw = 1;
+                if (lane == 0)
+                    okw = mbar_wait(smem_u32(&tail->empty[stage]), phase ^ 1u, status, kStatusTimeoutEmpty) ? 1u : 0u;
+                okw = __shfl_sync(0xffffffffu, okw, 0);
+                if (!okw) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t a_dst = smem_u32(smem + stage * kStageBytes);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = r0 + 16 * i;
+                    cp_async_16(a_dst + r * 128 + ((c ^ (r & 7)) << 4), src[i] + kb * kBK, bytes[i]);
+                }
+                cp_async_commit();
+                if (npend == 2) {
+                    // the stage issued two stages ago is complete: publish it
+                    cp_async_wait<2>();
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&tail->full[pend[0]]));
+                    pend[0] = pend[1];
+                    npend = 1;
+                }
+                pend[npend++] = stage;
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0)
+            for (int i = 0; i < npend; ++i) mbar_arrive(smem_u32(&tail->full[pend[i]]));
     } else {
         // ---------------- epilogue (warps 2..5) ----------------
         const int quad = warp & 3;  // TMEM lanes [32*quad, 32*quad+32)
         uint8_t* stage = smem + kStages * kStageBytes + kTailBytes + (warp - 2) * kWarpStageBytes;
         int local = 0;
         for (int t = first; t < total_tiles; t += stride, ++local) {
-            const TileInfo ti = tile_info(t, tail->off, tail->mblk, n, args.n_tiles, ord);
+            const TileInfo ti = tile_info(t, tail->off, tail->mblk, n, args.n_tiles, band_limit);
             const int buf = local & 1;
             const uint32_t bph = static_cast<uint32_t>(local >> 1) & 1u;
             if (!mbar_wait(smem_u32(&tail->accum_full[buf]), bph, status, kStatusTimeoutAccum)) break;
@@ -461,15 +490,20 @@ static int grid_for(const TcGemmArgs& a, int num_sms) {
     return static_cast<int>(g < 1 ? 1 : g);
 }
 
-template <bool kSwiGLU, bool kFp8>
+template <bool kSwiGLU, bool kFp8, bool kGather = false>
 static cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1,
                              const TcGemmArgs& a, int num_sms, cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<kSwiGLU, kFp8>,
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<kSwiGLU, kFp8, kGather>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    launch_k(tc_gemm_kernel<kSwiGLU, kFp8>, dim3(grid_for(a, num_sms)), dim3(kThreads), kSmemBytes, st, ta, tb0,
-             tb1, a);
+    launch_k(tc_gemm_kernel<kSwiGLU, kFp8, kGather>, dim3(grid_for(a, num_sms)),
+             dim3(kGather ? kGatherThreads : kThreads), kSmemBytes, st, ta, tb0, tb1, a);
     return cudaGetLastError();
+}
+
+cudaError_t launch_tc_gemm1_gather(const CUtensorMap& tm_w1, const CUtensorMap& tm_w3, const TcGemmArgs& a,
+                                   int num_sms, cudaStream_t st) {
+    return launch_tc<true, false, true>(tm_w1, tm_w1, tm_w3, a, num_sms, st);
 }
 
 cudaError_t launch_tc_gemm1(const CUtensorMap& tm_xp, const CUtensorMap& tm_w1,

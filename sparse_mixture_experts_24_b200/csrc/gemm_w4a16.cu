@@ -40,19 +40,25 @@
 // E2M1(code) * sb * 2^-8, and the epilogue multiplies the fp32 accumulators
 // by st * 2^8.
 //
-// Design (persistent, one CTA per SM, 14 warps):
-//   warp 12     TMA producer: per stage the weight block (cp.async.bulk) and
-//               the activation tile (kBN rows x 64, 128-byte swizzle).
+// Design (persistent, one CTA per SM, 15 warps):
+//   warp 12     weight producer: one cp.async.bulk of a 4,608-byte block per
+//               stage into a deep ring (DRAM latency under full load is about
+//               3 us; a shallow ring tied to the TMEM slots held the decode
+//               layer to 0.2 ms for 0.53 GB before any decoding was done).
+//   warp 13     activation producer: the kBN x 64 activation tile of each
+//               stage (TMA, 128-byte swizzle) into a short ring (L2 hits).
 //   warps 4-11  decoders, two per TMEM lane quarter (alternate stages): each
 //               thread is one packed column; it reads its 32 code bytes and 4
 //               scales, decodes 64 weights into 32 bf16x2 words and stores
 //               them to the stage's A slot in tensor memory (32 columns).
-//   warp 13     allocates TMEM; one thread issues tcgen05.mma (A from TMEM,
-//               B from shared memory, M = 128, N = kBN, K = 16).
+//   warp 14     allocates TMEM; one thread issues tcgen05.mma (A from TMEM,
+//               B from shared memory, M = 128, N = kBN, K = 16) and frees the
+//               A slot and the activation stage with tcgen05.commit.
 //   warps 0-3   epilogue: tcgen05.ld of the accumulator (thread = packed
 //               column, registers = tokens); GEMM1 exchanges the w3 half
 //               through shared memory and applies silu(a) * b; bf16 stores.
-// TMEM: two kBN-column accumulators, then one 32-column A slot per stage.
+// TMEM: two kBN-column accumulators, then one 32-column A slot per stage in
+// flight.
 // Every wait is bounded (common.cuh).
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -68,24 +74,47 @@ constexpr int kW16Cols = 128;              // packed columns per tile (MMA M)
 constexpr int kW16K = 64;                  // reduction rows per stage
 constexpr int kW16CodeBytes = 4096;        // 128 columns x 64 rows x 4 bits
 constexpr int kW16BlockBytes = kW16CodeBytes + 512;
-constexpr int kW16Threads = 448;
-constexpr int kProducerWarp = 12;
-constexpr int kMmaWarp = 13;
+constexpr int kDecGroups = 2;  // decoder groups of 4 warps, taking stages in turn
+constexpr int kW16Threads = (4 + 4 * kDecGroups + 3) * 32;
+constexpr int kWeightWarp = 4 + 4 * kDecGroups;   // producer of the weight ring
+constexpr int kActWarp = 5 + 4 * kDecGroups;      // producer of the activation ring
+constexpr int kMmaWarp = 6 + 4 * kDecGroups;
 constexpr uint32_t kPairMask = 0x81C081C0u;
+constexpr int kMaxRing = 8;
 
+// A stage is kBlocks 64-row reduction blocks, moved by ONE copy per ring:
+// the weight blocks of consecutive reduction steps are adjacent in the pack,
+// and the activation tile comes through a 3-D map (64 columns, rows, 64-column
+// chunk) whose box holds kBlocks chunks.  Small copies are what limit a TMA
+// pipeline (about 250 cycles each here, however small): one copy per 4.6 KB
+// held the decode layer to 2.6 TB/s before any decoding was done.
+// Three rings, each sized for what feeds it: weight blocks come from DRAM
+// (deep ring), activation tiles are re-read from L2 by every weight tile of an
+// expert (short ring), and the decoded weights sit in TMEM A slots, which need
+// only cover the MMA's lag behind the decoders.  TMEM: two kBN-column
+// accumulators, then the A slots (32 columns per block).
 template <int kBN>
 struct W16Cfg {
+    static constexpr int kBlocks = kBN == 32 ? 4 : 2;        // 64-row blocks per stage
     static constexpr int kAccCols = 2 * kBN;
-    static constexpr int kStages = (512 - kAccCols) / 32;
-    static constexpr int kBBytes = kBN * 128;  // kBN rows x 64 bf16
-    static constexpr int kStageBytes = (kBBytes + kW16BlockBytes + 1023) / 1024 * 1024;
-    static constexpr int kXbufBytes = kBN * 64 * 4;  // GEMM1: w3 half of the accumulator, fp32
+    static constexpr int kSlotCols = 32 * kBlocks;
+    static constexpr int kASlots = (512 - kAccCols) / kSlotCols;  // 3 (kBN 32) or 4 (kBN 128)
+    static constexpr int kActStages = 3;
+    static constexpr int kWStages = 8;
+    static constexpr int kBBytes = kBN * 128 * kBlocks;      // kBlocks chunks of kBN rows x 64 bf16
+    static constexpr int kWStageBytes = kW16BlockBytes * kBlocks;
+    static constexpr int kActBytes = kActStages * kBBytes;
+    static constexpr int kWBytes = kWStages * kWStageBytes;
+    static constexpr int kXbufBytes = kBN * 64 * 4;          // GEMM1: w3 half of the accumulator, fp32
 };
 
 struct __align__(8) W16Tail {
-    uint64_t full[14];
-    uint64_t empty[14];
-    uint64_t afull[14];
+    uint64_t wfull[kMaxRing];
+    uint64_t wempty[kMaxRing];
+    uint64_t xfull[kMaxRing];
+    uint64_t xempty[kMaxRing];
+    uint64_t afull[kMaxRing];
+    uint64_t aempty[kMaxRing];
     uint64_t accum_full[2];
     uint64_t accum_empty[2];
     uint64_t done;
@@ -97,9 +126,10 @@ constexpr int kW16TailBytes = (static_cast<int>(sizeof(W16Tail)) + 127) / 128 * 
 
 template <int kBN>
 constexpr int w16_smem_bytes() {
-    return W16Cfg<kBN>::kStages * W16Cfg<kBN>::kStageBytes + W16Cfg<kBN>::kXbufBytes + kW16TailBytes + 1024;
+    return W16Cfg<kBN>::kActBytes + W16Cfg<kBN>::kWBytes + W16Cfg<kBN>::kXbufBytes + kW16TailBytes + 1024;
 }
-static_assert(W16Cfg<32>::kStages == 14 && W16Cfg<128>::kStages == 8, "stage counts");
+static_assert(W16Cfg<32>::kWStages <= kMaxRing && W16Cfg<128>::kWStages <= kMaxRing, "ring sizes");
+static_assert(W16Cfg<32>::kASlots <= kMaxRing && W16Cfg<32>::kActStages <= kMaxRing, "ring sizes");
 static_assert(w16_smem_bytes<32>() <= 232448 && w16_smem_bytes<128>() <= 232448, "shared memory");
 
 struct W16Tile {
@@ -203,22 +233,30 @@ template <bool kSwiGLU, int kBN>
 __global__ void __launch_bounds__(kW16Threads, 1)
     w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const W4a16GemmArgs args) {
     using C = W16Cfg<kBN>;
-    constexpr int S = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    float* xbuf = reinterpret_cast<float*>(smem + S * C::kStageBytes);
-    W16Tail* tail = reinterpret_cast<W16Tail*>(smem + S * C::kStageBytes + C::kXbufBytes);
+    uint8_t* act_ring = smem;                         // 1 KB-aligned swizzled tiles
+    uint8_t* w_ring = smem + C::kActBytes;            // kBlocks weight blocks of 4,608 bytes per stage
+    float* xbuf = reinterpret_cast<float*>(w_ring + C::kWBytes);
+    W16Tail* tail = reinterpret_cast<W16Tail*>(w_ring + C::kWBytes + C::kXbufBytes);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int n = args.n;
     int* status = args.status;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(smem_u32(&tail->full[s]), 1);
-            mbar_init(smem_u32(&tail->empty[s]), 5);   // 4 decoder warps + the MMA commit
-            mbar_init(smem_u32(&tail->afull[s]), 4);   // 4 decoder warps
+        for (int s = 0; s < C::kWStages; ++s) {
+            mbar_init(smem_u32(&tail->wfull[s]), 1);
+            mbar_init(smem_u32(&tail->wempty[s]), 4);  // the 4 decoder warps of the stage's group
+        }
+        for (int s = 0; s < C::kActStages; ++s) {
+            mbar_init(smem_u32(&tail->xfull[s]), 1);
+            mbar_init(smem_u32(&tail->xempty[s]), 1);  // MMA commit
+        }
+        for (int s = 0; s < C::kASlots; ++s) {
+            mbar_init(smem_u32(&tail->afull[s]), 4);   // the 4 decoder warps
+            mbar_init(smem_u32(&tail->aempty[s]), 1);  // MMA commit
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&tail->accum_full[b]), 1);
@@ -228,7 +266,7 @@ __global__ void __launch_bounds__(kW16Threads, 1)
         fence_barrier_init();
         fence_proxy_async_smem();
     }
-    if (warp == kProducerWarp && lane == 0) tma_prefetch_desc(&tm_act);
+    if (warp == kActWarp && lane == 0) tma_prefetch_desc(&tm_act);
     if (warp == kMmaWarp) {
         tmem_alloc(smem_u32(&tail->tmem_base), 512);
         tmem_relinquish();
@@ -248,36 +286,44 @@ __global__ void __launch_bounds__(kW16Threads, 1)
     const int first = static_cast<int>(blockIdx.x) < stride ? static_cast<int>(blockIdx.x) : total_tiles;
     const int kb_n = args.k_blocks;
 
-    if (warp == kProducerWarp) {
+    if (warp == kWeightWarp || warp == kActWarp) {
+        // ---------------- producers: one ring each ----------------
         if (lane == 0) {
-            int armed[14];
-            for (int s = 0; s < S; ++s) armed[s] = -1;
+            const bool weights = warp == kWeightWarp;
+            const int ring = weights ? C::kWStages : C::kActStages;
+            uint64_t* full = weights ? tail->wfull : tail->xfull;
+            uint64_t* empty = weights ? tail->wempty : tail->xempty;
             uint32_t i = 0;
             bool ok = true;
             for (int t = first; t < total_tiles && ok; t += stride) {
                 const W16Tile ti = w16_tile(t, tail->off, tail->mblk, n, args.n_tiles, kBN);
                 const uint8_t* wsrc =
                     args.wpack + (static_cast<int64_t>(ti.e) * args.n_tiles + ti.j) * kb_n * kW16BlockBytes;
-                for (int kb = 0; kb < kb_n; ++kb, ++i) {
-                    const int slot = static_cast<int>(i % S);
-                    const uint32_t ph = (i / S) & 1u;
-                    if (!mbar_wait(smem_u32(&tail->empty[slot]), ph ^ 1u, status, kStatusTimeoutEmpty)) {
+                for (int kb = 0; kb < kb_n; kb += C::kBlocks, ++i) {
+                    const int slot = static_cast<int>(i % ring);
+                    const uint32_t ph = (i / ring) & 1u;
+                    if (!mbar_wait(smem_u32(&empty[slot]), ph ^ 1u, status, kStatusTimeoutEmpty)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t fb = smem_u32(&tail->full[slot]);
-                    mbar_arrive_expect_tx(fb, C::kBBytes + kW16BlockBytes);
-                    armed[slot] = static_cast<int>(ph);
-                    const uint32_t dst = smem_u32(smem + slot * C::kStageBytes);
-                    tma_load_2d(dst, &tm_act, fb, kb * kW16K, ti.row0);
-                    bulk_load(dst + C::kBBytes, wsrc + static_cast<int64_t>(kb) * kW16BlockBytes, kW16BlockBytes,
-                              fb);
+                    const uint32_t fb = smem_u32(&full[slot]);
+                    if (weights) {
+                        const uint32_t bytes = static_cast<uint32_t>(min(C::kBlocks, kb_n - kb)) * kW16BlockBytes;
+                        mbar_arrive_expect_tx(fb, bytes);
+                        bulk_load(smem_u32(w_ring + slot * C::kWStageBytes),
+                                  wsrc + static_cast<int64_t>(kb) * kW16BlockBytes, bytes, fb);
+                    } else {
+                        // the box always lands kBlocks chunks (zeros past K)
+                        mbar_arrive_expect_tx(fb, C::kBBytes);
+                        tma_load_3d(smem_u32(act_ring + slot * C::kBBytes), &tm_act, fb, 0, ti.row0, kb);
+                    }
                 }
             }
-            for (int s = 0; s < S; ++s)
-                if (armed[s] >= 0)
-                    mbar_wait(smem_u32(&tail->full[s]), static_cast<uint32_t>(armed[s]), status,
-                              kStatusTimeoutDrain);
+            // Drain: no copy may still be writing shared memory when the CTA exits.
+            // The last min(i, ring) stages were armed; wait for each one's phase.
+            const uint32_t armed = i < static_cast<uint32_t>(ring) ? i : static_cast<uint32_t>(ring);
+            for (uint32_t k = i - armed; k < i; ++k)
+                mbar_wait(smem_u32(&full[k % ring]), (k / ring) & 1u, status, kStatusTimeoutDrain);
         }
     } else if (warp == kMmaWarp) {
         if (lane == 0) {
@@ -294,24 +340,31 @@ __global__ void __launch_bounds__(kW16Threads, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
-                for (int kb = 0; kb < kb_n; ++kb, ++i) {
-                    const int slot = static_cast<int>(i % S);
-                    const uint32_t ph = (i / S) & 1u;
-                    if (!mbar_wait(smem_u32(&tail->afull[slot]), ph, status, kStatusTimeoutFull) ||
-                        !mbar_wait(smem_u32(&tail->full[slot]), ph, status, kStatusTimeoutFull)) {
+                for (int kb = 0; kb < kb_n; kb += C::kBlocks, ++i) {
+                    const int as = static_cast<int>(i % C::kASlots);
+                    const int xs = static_cast<int>(i % C::kActStages);
+                    if (!mbar_wait(smem_u32(&tail->afull[as]), (i / C::kASlots) & 1u, status, kStatusTimeoutFull) ||
+                        !mbar_wait(smem_u32(&tail->xfull[xs]), (i / C::kActStages) & 1u, status,
+                                   kStatusTimeoutFull)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t b_base = smem_u32(smem + slot * C::kStageBytes);
-                    const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(C::kAccCols + slot * 32);
+                    const int nblk = min(C::kBlocks, kb_n - kb);
+                    for (int b = 0; b < nblk; ++b) {
+                        const uint32_t b_base = smem_u32(act_ring + xs * C::kBBytes + b * kBN * 128);
+                        const uint32_t a_tmem =
+                            tmem_base + static_cast<uint32_t>(C::kAccCols + as * C::kSlotCols + b * 32);
 #pragma unroll
-                    for (int kk = 0; kk < kW16K / 16; ++kk) {
-                        // B: K-major, 128-byte swizzle; K by 16 = 32 bytes inside the swizzle row.
-                        const uint64_t bdesc = make_smem_desc(b_base + kk * 32, 16, 1024, 2);
-                        tc_mma_f16_tmem_a(d_tmem, a_tmem + kk * 8, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        for (int kk = 0; kk < kW16K / 16; ++kk) {
+                            // B: K-major, 128-byte swizzle; K by 16 = 32 bytes inside the swizzle row.
+                            const uint64_t bdesc = make_smem_desc(b_base + kk * 32, 16, 1024, 2);
+                            tc_mma_f16_tmem_a(d_tmem, a_tmem + kk * 8, bdesc, idesc,
+                                              (kb | b | kk) != 0 ? 1u : 0u);
+                        }
                     }
-                    tc_commit(smem_u32(&tail->empty[slot]));
+                    tc_commit(smem_u32(&tail->aempty[as]));
+                    tc_commit(smem_u32(&tail->xempty[xs]));
                 }
                 if (ok) tc_commit(smem_u32(&tail->accum_full[buf]));
             }
@@ -321,44 +374,49 @@ __global__ void __launch_bounds__(kW16Threads, 1)
     } else if (warp >= 4) {
         // ---------------- decoders ----------------
         const int q = warp & 3;
-        const uint32_t group = static_cast<uint32_t>(warp - 4) >> 2;
+        const uint32_t group = static_cast<uint32_t>(warp - 4) >> 2;  // stages i with i % kDecGroups == group
         const int p = q * 32 + lane;  // packed column = TMEM lane
         uint32_t i = 0;
         bool ok = true;
         for (int t = first; t < total_tiles && ok; t += stride) {
-            for (int kb = 0; kb < kb_n; ++kb, ++i) {
-                if ((i & 1u) != group) continue;
-                const int slot = static_cast<int>(i % S);
-                const uint32_t ph = (i / S) & 1u;
-                if (!mbar_wait(smem_u32(&tail->full[slot]), ph, status, kStatusTimeoutFull)) {
+            for (int kb = 0; kb < kb_n; kb += C::kBlocks, ++i) {
+                if (i % kDecGroups != group) continue;
+                const int ws = static_cast<int>(i % C::kWStages);
+                const int as = static_cast<int>(i % C::kASlots);
+                if (!mbar_wait(smem_u32(&tail->wfull[ws]), (i / C::kWStages) & 1u, status, kStatusTimeoutFull) ||
+                    !mbar_wait(smem_u32(&tail->aempty[as]), ((i / C::kASlots) & 1u) ^ 1u, status,
+                               kStatusTimeoutEmpty)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint8_t* blk = smem + slot * C::kStageBytes + C::kBBytes;
-                const uint4 u0 = *reinterpret_cast<const uint4*>(blk + p * 16);
-                const uint4 u1 = *reinterpret_cast<const uint4*>(blk + 2048 + p * 16);
-                const uint32_t sw = *reinterpret_cast<const uint32_t*>(blk + kW16CodeBytes + p * 4);
-                const uint32_t s0 = scale_pair(sw), s1 = scale_pair(sw >> 8), s2 = scale_pair(sw >> 16),
-                               s3 = scale_pair(sw >> 24);
-                uint32_t r[32];
-                decode_word(u0.x, s0, r + 0);
-                decode_word(u0.y, s0, r + 4);
-                decode_word(u0.z, s1, r + 8);
-                decode_word(u0.w, s1, r + 12);
-                decode_word(u1.x, s2, r + 16);
-                decode_word(u1.y, s2, r + 20);
-                decode_word(u1.z, s3, r + 24);
-                decode_word(u1.w, s3, r + 28);
-                tmem_st_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                       static_cast<uint32_t>(C::kAccCols + slot * 32),
-                                   r);
+                const int nblk = min(C::kBlocks, kb_n - kb);
+                for (int b = 0; b < nblk; ++b) {
+                    const uint8_t* blk = w_ring + ws * C::kWStageBytes + b * kW16BlockBytes;
+                    const uint4 u0 = *reinterpret_cast<const uint4*>(blk + p * 16);
+                    const uint4 u1 = *reinterpret_cast<const uint4*>(blk + 2048 + p * 16);
+                    const uint32_t sw = *reinterpret_cast<const uint32_t*>(blk + kW16CodeBytes + p * 4);
+                    const uint32_t s0 = scale_pair(sw), s1 = scale_pair(sw >> 8), s2 = scale_pair(sw >> 16),
+                                   s3 = scale_pair(sw >> 24);
+                    uint32_t r[32];
+                    decode_word(u0.x, s0, r + 0);
+                    decode_word(u0.y, s0, r + 4);
+                    decode_word(u0.z, s1, r + 8);
+                    decode_word(u0.w, s1, r + 12);
+                    decode_word(u1.x, s2, r + 16);
+                    decode_word(u1.y, s2, r + 20);
+                    decode_word(u1.z, s3, r + 24);
+                    decode_word(u1.w, s3, r + 28);
+                    tmem_st_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                           static_cast<uint32_t>(C::kAccCols + as * C::kSlotCols + b * 32),
+                                       r);
+                }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive(smem_u32(&tail->afull[slot]));
-                    mbar_arrive(smem_u32(&tail->empty[slot]));
+                    mbar_arrive(smem_u32(&tail->afull[as]));
+                    mbar_arrive(smem_u32(&tail->wempty[ws]));
                 }
             }
         }

@@ -184,12 +184,13 @@ struct TcGemmArgs {
     const float* col_scale0;
     const float* col_scale1;
     int balanced;      // 1: spread the tiles evenly over the fewest CTAs (balanced_ctas)
-    // single-SM kernel, tile order (gemm_tc.cu): row blocks per m-band and
-    // column tiles per n-band (0: no bands), and whether GEMM2 walks K
-    // downwards on odd column tiles
-    int band_m;
-    int band_n;
-    int k_alternate;
+    int band_m;        // single-SM kernel: row blocks per band of the tile order (0: no bands)
+    // launch_tc_gemm1_gather only: A rows gathered from x [x_rows][x_cols] bf16
+    // (tile row r = token row_token[row0 + r])
+    const uint16_t* x;
+    const int32_t* row_token;
+    int64_t x_rows;
+    int64_t x_cols;
 };
 
 cudaError_t launch_tc_gemm1(const CUtensorMap& tm_xp, const CUtensorMap& tm_w1,
@@ -197,6 +198,9 @@ cudaError_t launch_tc_gemm1(const CUtensorMap& tm_xp, const CUtensorMap& tm_w1,
                             cudaStream_t st);
 cudaError_t launch_tc_gemm2(const CUtensorMap& tm_h, const CUtensorMap& tm_w2, const TcGemmArgs& a,
                             int num_sms, cudaStream_t st);
+// GEMM1 with the A rows gathered from x by the kernel itself (no Xp).
+cudaError_t launch_tc_gemm1_gather(const CUtensorMap& tm_w1, const CUtensorMap& tm_w3, const TcGemmArgs& a,
+                                   int num_sms, cudaStream_t st);
 cudaError_t launch_tc_gemm1_e4m3(const CUtensorMap& tm_x8, const CUtensorMap& tm_q1,
                                  const CUtensorMap& tm_q3, const TcGemmArgs& a, int num_sms,
                                  cudaStream_t st);
@@ -308,7 +312,8 @@ struct W4a16GemmArgs {
 };
 // Token rows per tile: 32 when the experts average at most 32 rows, else 128.
 int w4a16_tile_rows(int64_t R, int n);
-// tm_xp / tm_h: bf16 rows in 64 x tile_rows boxes, 128-byte swizzle.
+// tm_xp / tm_h: bf16 rows as 3-D maps (64 columns, rows, 64-column chunk),
+// boxes of 64 x tile_rows x (4 chunks for 32 rows, 2 for 128), 128-byte swizzle.
 cudaError_t launch_w4a16_gemm1(const CUtensorMap& tm_xp, const W4a16GemmArgs& a, int tile_rows, int num_sms,
                                cudaStream_t st);
 cudaError_t launch_w4a16_gemm2(const CUtensorMap& tm_h, const W4a16GemmArgs& a, int tile_rows, int num_sms,

@@ -109,6 +109,38 @@ bool encode_weights(CUtensorMap* m, const void* base, uint64_t cols, uint64_t ro
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 rows [rows][cols] as a 3-D map (64 columns, rows, 64-column chunk)
+// read in boxes of 64 columns x box_rows rows x `chunks` chunks: one copy
+// lands `chunks` row tiles of box_rows x 64, back to back.
+bool encode_rows_chunked(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows,
+                         uint32_t chunks) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[3] = {64, rows, cols / 64};
+    cuuint64_t strides[2] = {cols * 2, 128};
+    cuuint32_t box[3] = {64, box_rows, chunks};
+    cuuint32_t es[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 weights [n][rows][cols] as a 4-D map (64 columns, rows, 64-column
+// chunk, expert) read in boxes of 64 columns x 64 rows x `chunks` chunks:
+// one copy lands `chunks` 64-column chunks of 8 KB each, back to back.
+bool encode_weights_wide(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t n,
+                         uint32_t chunks) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[4] = {64, rows, cols / 64, n};
+    cuuint64_t strides[3] = {cols * 2, 128, cols * rows * 2};
+    cuuint32_t box[4] = {64, 64, chunks, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // E4M3 codes, uint8: [rows][cols] (box_rows x 128) or weights [n][rows][cols]
 // (128 x 128 boxes of one expert); out-of-range boxes read zeros.
 bool encode_codes(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t n,
@@ -169,6 +201,7 @@ struct moe_handle {
     void* o = nullptr;
     int* status = nullptr;
     CUtensorMap tm_xp, tm_h, tm_w1, tm_w3, tm_w2;
+    CUtensorMap tm_w1x, tm_w3x, tm_w2x;  // the same weights as 4-D maps (single-SM GEMMs)
     const void* c_w1 = nullptr;
     const void* c_w3 = nullptr;
     const void* c_w2 = nullptr;
@@ -222,8 +255,9 @@ struct moe_handle {
     CUtensorMap tm_xq4, tm_hq4, tm_wp4[2];
     CUtensorMap tm_xq4s, tm_hq4s;  // the same codes in 32-row boxes
     const void* c_wp4[2] = {nullptr, nullptr};
-    // 4-bit weights decoded into tensor memory: Xp and H in 32-row boxes
-    CUtensorMap tm_xp32, tm_h32;
+    // 4-bit weights decoded into tensor memory: Xp and H as 3-D maps whose
+    // boxes hold 4 chunks of 32 rows ([0]) or 2 chunks of 128 rows ([1])
+    CUtensorMap tm_xpw[2], tm_hw[2];
     // 4-bit experts: maps over the caller's codes and block scales
     CUtensorMap tm_f4[6];  // codes w1, scales w1, codes w3, scales w3, codes w2, scales w2
     const void* c_f4[6] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
@@ -407,8 +441,10 @@ moe_status grow(moe_handle* h, int64_t T, int64_t rows_min = 0) {
     if (h->dtype == MOE_BF16) {
         if (!encode_rows(&h->tm_xp, h->xp, h->d, static_cast<uint64_t>(R)) ||
             !encode_rows(&h->tm_h, h->h, h->F, static_cast<uint64_t>(R)) ||
-            !encode_rows(&h->tm_xp32, h->xp, h->d, static_cast<uint64_t>(R), 32) ||
-            !encode_rows(&h->tm_h32, h->h, h->F, static_cast<uint64_t>(R), 32) ||
+            !encode_rows_chunked(&h->tm_xpw[0], h->xp, h->d, static_cast<uint64_t>(R), 32, 4) ||
+            !encode_rows_chunked(&h->tm_hw[0], h->h, h->F, static_cast<uint64_t>(R), 32, 4) ||
+            !encode_rows_chunked(&h->tm_xpw[1], h->xp, h->d, static_cast<uint64_t>(R), 128, 2) ||
+            !encode_rows_chunked(&h->tm_hw[1], h->h, h->F, static_cast<uint64_t>(R), 128, 2) ||
             !encode_rows(&h->tm_parts, h->wg_parts, h->d, static_cast<uint64_t>(3 * npad),
                          static_cast<uint32_t>(npad)))
             return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the workspace");
@@ -495,27 +531,20 @@ int grid_balance() {
     return (env && strcmp(env, "0") == 0) ? 0 : 1;
 }
 
-// Tile order of the single-SM GEMMs (gemm_tc.cu): bands of row blocks and of
-// column tiles sized to MOE_GEMM_BAND_MB megabytes of A rows / weight columns
-// (unset or 0: no bands), MOE_GEMM_BAND_AXIS=m or n to allow only one axis,
-// and MOE_GEMM2_KALT=0 to walk K upwards on every GEMM2 column tile.
-void gemm_tile_order(moe::TcGemmArgs& a, int64_t a_row_bytes, int64_t b_col_bytes, int b_cols) {
-    a.k_alternate = 1;
-    if (const char* v = getenv("MOE_GEMM2_KALT")) a.k_alternate = atoi(v) != 0;
-    a.band_m = a.band_n = 0;
-    const char* env = getenv("MOE_GEMM_BAND_MB");
-    if (!env) return;
-    const int64_t mb = atoll(env);
-    if (mb <= 0) return;
-    const int64_t budget = mb << 20;
-    const char* axis = getenv("MOE_GEMM_BAND_AXIS");
-    const bool allow_m = !axis || strcmp(axis, "n") != 0;
-    const bool allow_n = !axis || strcmp(axis, "m") != 0;
-    const int64_t bm = budget / (static_cast<int64_t>(moe::kTcBM) * a_row_bytes);
-    const int64_t bn = budget / (static_cast<int64_t>(b_cols) * b_col_bytes);
-    a.band_m = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(bm, 1 << 20)));
-    a.band_n = allow_n ? static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(bn, 1 << 20))) : 0;
-    if (!allow_m) a.band_m = 1;  // always banded, and n-bands win whenever they are cheaper
+// Tile order of the single-SM GEMMs (gemm_tc.cu): bands of as many 128-row
+// blocks of the A operand (rows of a_row_bytes) as fit in the band budget.
+// The budget is 32 MB (measured best on the skewed prefill, against 16 and
+// 64 MB); MOE_GEMM1_BAND_KB / MOE_GEMM2_BAND_KB override it in kilobytes
+// (0: no bands).
+void gemm_tile_order(moe::TcGemmArgs& a, int64_t a_row_bytes, bool gemm2) {
+    int64_t kb = 32 * 1024;
+    if (const char* v = getenv(gemm2 ? "MOE_GEMM2_BAND_KB" : "MOE_GEMM1_BAND_KB")) kb = atoll(v);
+    if (kb <= 0) {
+        a.band_m = 0;
+        return;
+    }
+    const int64_t b = (kb << 10) / (static_cast<int64_t>(moe::kTcBM) * a_row_bytes);
+    a.band_m = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(b, 1 << 20)));
 }
 
 // Most (token, slot) pairs one expert takes in a call of T tokens:
@@ -528,27 +557,49 @@ int capacity_for(const moe_handle* h, int64_t T) {
 
 // Gather the segment rows of x, then GEMM1 (w1/w3 + SwiGLU) and GEMM2 (w2)
 // over R rows laid out by the dispatch arrays already on the device.
+// bf16 GEMM1 on the single-SM tiles gathers its A rows from x itself (no
+// gather kernel, no Xp) when the experts average at most 256 rows: there the
+// GEMMs stream weights and the gather kernel's round trip through HBM is
+// what the fused gather saves (decode 0.435 -> 0.424 ms, many_expert 0.317 ->
+// 0.308 ms).  With more rows GEMM1 is bound by the tensor cores and the
+// cp.async gather, two stages behind the tensor core, slowed it (prefill
+// GEMM1 1.62 -> 1.99 ms), so the gather kernel stays.  MOE_GATHER=separate /
+// fused forces either.
+bool gather_in_gemm1(int64_t R, int n) {
+    const char* env = getenv("MOE_GATHER");
+    if (env && strcmp(env, "separate") == 0) return false;
+    if (env && strcmp(env, "fused") == 0) return true;
+    return R <= 256 * static_cast<int64_t>(n);
+}
+
 moe_status run_gemms(moe_handle* h, int64_t T, int64_t R, const void* x, const void* w1, const void* w3,
                      const void* w2, bool pair, cudaStream_t st) {
     const bool bf = h->dtype == MOE_BF16;
-    cudaError_t e = moe::launch_gather(x, h->db.row_token, R, T, static_cast<int64_t>(h->d) * h->esize(),
-                                       h->xp, h->num_sms, st);
-    if (e != cudaSuccess) return cuda_fail(e, "gather launch");
-    h->launches += 1;
+    const bool fused_gather = bf && !pair && gather_in_gemm1(R, h->n);
+    cudaError_t e;
+    if (!fused_gather) {
+        e = moe::launch_gather(x, h->db.row_token, R, T, static_cast<int64_t>(h->d) * h->esize(), h->xp,
+                               h->num_sms, st);
+        if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+        h->launches += 1;
+    }
     trace_mark(h, 2, st);
     if (bf) {
         if (w1 != h->c_w1) {
-            if (!encode_weights(&h->tm_w1, w1, h->F, h->d, h->n))
+            if (!encode_weights(&h->tm_w1, w1, h->F, h->d, h->n) ||
+                !encode_weights_wide(&h->tm_w1x, w1, h->F, h->d, h->n, 2))
                 return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for w1");
             h->c_w1 = w1;
         }
         if (w3 != h->c_w3) {
-            if (!encode_weights(&h->tm_w3, w3, h->F, h->d, h->n))
+            if (!encode_weights(&h->tm_w3, w3, h->F, h->d, h->n) ||
+                !encode_weights_wide(&h->tm_w3x, w3, h->F, h->d, h->n, 2))
                 return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for w3");
             h->c_w3 = w3;
         }
         if (w2 != h->c_w2) {
-            if (!encode_weights(&h->tm_w2, w2, h->d, h->F, h->n))
+            if (!encode_weights(&h->tm_w2, w2, h->d, h->F, h->n) ||
+                !encode_weights_wide(&h->tm_w2x, w2, h->d, h->F, h->n, 4))
                 return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for w2");
             h->c_w2 = w2;
         }
@@ -563,9 +614,17 @@ moe_status run_gemms(moe_handle* h, int64_t T, int64_t R, const void* x, const v
         a1.out = h->h;
         a1.status = h->status;
         a1.balanced = grid_balance();
-        gemm_tile_order(a1, static_cast<int64_t>(h->d) * 2, static_cast<int64_t>(h->d) * 2, 256);
-        e = pair ? moe::launch_tc_gemm1_pair(h->tm_xp, h->tm_w1, h->tm_w3, a1, h->num_sms, st)
-                 : moe::launch_tc_gemm1(h->tm_xp, h->tm_w1, h->tm_w3, a1, h->num_sms, st);
+        gemm_tile_order(a1, static_cast<int64_t>(h->d) * 2, false);
+        if (fused_gather) {
+            a1.x = static_cast<const uint16_t*>(x);
+            a1.row_token = h->db.row_token;
+            a1.x_rows = T;
+            a1.x_cols = h->d;
+            e = moe::launch_tc_gemm1_gather(h->tm_w1x, h->tm_w3x, a1, h->num_sms, st);
+        } else {
+            e = pair ? moe::launch_tc_gemm1_pair(h->tm_xp, h->tm_w1, h->tm_w3, a1, h->num_sms, st)
+                     : moe::launch_tc_gemm1(h->tm_xp, h->tm_w1x, h->tm_w3x, a1, h->num_sms, st);
+        }
         if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
         h->launches += 1;
         trace_mark(h, 3, st);
@@ -574,9 +633,9 @@ moe_status run_gemms(moe_handle* h, int64_t T, int64_t R, const void* x, const v
         a2.n_tiles = (h->d + 255) / 256;
         a2.out_cols = h->d;
         a2.out = h->o;
-        gemm_tile_order(a2, static_cast<int64_t>(h->F) * 2, static_cast<int64_t>(h->F) * 2, 256);
+        gemm_tile_order(a2, static_cast<int64_t>(h->F) * 2, true);
         e = pair ? moe::launch_tc_gemm2_pair(h->tm_h, h->tm_w2, a2, h->num_sms, st)
-                 : moe::launch_tc_gemm2(h->tm_h, h->tm_w2, a2, h->num_sms, st);
+                 : moe::launch_tc_gemm2(h->tm_h, h->tm_w2x, a2, h->num_sms, st);
         if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
         h->launches += 1;
         trace_mark(h, 4, st);
@@ -667,7 +726,7 @@ moe_status run_experts_e4m3(moe_handle* h, int64_t T, const void* x, const int32
     a1.row_scale = h->xs;
     a1.col_scale0 = s1;
     a1.col_scale1 = s3;
-    gemm_tile_order(a1, h->d, h->d, 256);
+    gemm_tile_order(a1, h->d, false);
     e = pair ? moe::launch_tc_gemm1_pair_e4m3(h->tm_x8, h->tm_q1, h->tm_q3, a1, h->num_sms, st)
              : moe::launch_tc_gemm1_e4m3(h->tm_x8, h->tm_q1, h->tm_q3, a1, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
@@ -683,7 +742,7 @@ moe_status run_experts_e4m3(moe_handle* h, int64_t T, const void* x, const int32
     a2.row_scale = h->hs;
     a2.col_scale0 = s2;
     a2.col_scale1 = nullptr;
-    gemm_tile_order(a2, h->F, h->F, 256);
+    gemm_tile_order(a2, h->F, true);
     e = pair ? moe::launch_tc_gemm2_pair_e4m3(h->tm_h8, h->tm_q2, a2, h->num_sms, st)
              : moe::launch_tc_gemm2_e4m3(h->tm_h8, h->tm_q2, a2, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
@@ -885,7 +944,7 @@ moe_status run_experts_w4a16(moe_handle* h, int64_t T, const void* x, const floa
     a1.mscale0 = ws[0];
     a1.mscale1 = ws[1];
     a1.balanced = grid_balance();
-    e = moe::launch_w4a16_gemm1(tile_rows == 32 ? h->tm_xp32 : h->tm_xp, a1, tile_rows, h->num_sms, st);
+    e = moe::launch_w4a16_gemm1(h->tm_xpw[tile_rows == 32 ? 0 : 1], a1, tile_rows, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
     h->launches += 1;
     trace_mark(h, 3, st);
@@ -897,7 +956,7 @@ moe_status run_experts_w4a16(moe_handle* h, int64_t T, const void* x, const floa
     a2.wpack = wp[1];
     a2.mscale0 = ws[2];
     a2.mscale1 = ws[2];
-    e = moe::launch_w4a16_gemm2(tile_rows == 32 ? h->tm_h32 : h->tm_h, a2, tile_rows, h->num_sms, st);
+    e = moe::launch_w4a16_gemm2(h->tm_hw[tile_rows == 32 ? 0 : 1], a2, tile_rows, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
     h->launches += 1;
     trace_mark(h, 4, st);
@@ -1466,7 +1525,8 @@ moe_status moe_ep_experts(moe_handle* h, int world, int rank, const int32_t* cou
     for (int m = 0; m < 3; ++m) {
         if (w[m] == h->c_ew[m] && nl == h->c_ew_nl) continue;
         const bool down = m == 2;
-        if (!encode_weights(tm[m], w[m], down ? h->d : h->F, down ? h->F : h->d, static_cast<uint64_t>(nl)))
+        if (!encode_weights_wide(tm[m], w[m], down ? h->d : h->F, down ? h->F : h->d, static_cast<uint64_t>(nl),
+                                 down ? 4 : 2))
             return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the local expert weights");
         h->c_ew[m] = w[m];
     }
@@ -1485,7 +1545,7 @@ moe_status moe_ep_experts(moe_handle* h, int world, int rank, const int32_t* cou
     a1.out = h->h;
     a1.status = h->status;
     a1.balanced = grid_balance();
-    gemm_tile_order(a1, static_cast<int64_t>(h->d) * 2, static_cast<int64_t>(h->d) * 2, 256);
+    gemm_tile_order(a1, static_cast<int64_t>(h->d) * 2, false);
     e = moe::launch_tc_gemm1(h->tm_erecv, h->tm_ew1, h->tm_ew3, a1, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
     moe::TcGemmArgs a2 = a1;
@@ -1493,7 +1553,7 @@ moe_status moe_ep_experts(moe_handle* h, int world, int rank, const int32_t* cou
     a2.n_tiles = (h->d + 255) / 256;
     a2.out_cols = h->d;
     a2.out = out;
-    gemm_tile_order(a2, static_cast<int64_t>(h->F) * 2, static_cast<int64_t>(h->F) * 2, 256);
+    gemm_tile_order(a2, static_cast<int64_t>(h->F) * 2, true);
     e = moe::launch_tc_gemm2(h->tm_h, h->tm_ew2, a2, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
     h->launches += 3;

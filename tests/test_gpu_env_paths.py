@@ -7,7 +7,13 @@ these variables once per process):
   MOE_ROUTER_TOPK=separate   tensor-core router writes logits, then the
                              standalone top-K kernel selects;
   MOE_GEMM_PATH=pair         CTA-pair (cta_group::2) expert GEMMs (bf16 and E4M3);
-  MOE_GRID_BALANCE=0         persistent GEMM tiles strided over the whole grid.
+  MOE_GRID_BALANCE=0         persistent GEMM tiles strided over the whole grid;
+  MOE_GATHER=separate/fused  the x rows gathered into Xp by their own kernel
+                             before GEMM1, or by GEMM1 itself (default: by
+                             GEMM1 when the experts average <= 256 rows);
+  MOE_GEMM1_BAND_KB=0 / 64, MOE_GEMM2_BAND_KB=0 / 64
+                             the expert GEMMs' tile order without bands, and
+                             with bands of a row block or two.
 """
 import os
 import subprocess
@@ -23,7 +29,9 @@ SLICE = "small and (bf16_ragged or bf16_k3_n16 or router_split2 or router_split4
 
 
 @pytest.mark.parametrize("env", [{"MOE_PDL": "0"}, {"MOE_ROUTER_TOPK": "separate"}, {"MOE_GEMM_PATH": "pair"},
-                                 {"MOE_GRID_BALANCE": "0"}],
+                                 {"MOE_GRID_BALANCE": "0"}, {"MOE_GATHER": "separate"}, {"MOE_GATHER": "fused"},
+                                 {"MOE_GEMM1_BAND_KB": "0", "MOE_GEMM2_BAND_KB": "0"},
+                                 {"MOE_GEMM1_BAND_KB": "64", "MOE_GEMM2_BAND_KB": "64"}],
                          ids=lambda e: ",".join("%s=%s" % kv for kv in e.items()))
 def test_parity_slice_under_env(env):
     full_env = dict(os.environ)
