@@ -75,7 +75,7 @@ constexpr int kW16K = 64;                  // reduction rows per stage
 constexpr int kW16CodeBytes = 4096;        // 128 columns x 64 rows x 4 bits
 constexpr int kW16BlockBytes = kW16CodeBytes + 512;
 constexpr int kDecGroups = 2;  // decoder groups of 4 warps, taking stages in turn
-constexpr int kW16Threads = (4 + 4 * kDecGroups + 3) * 32;
+
 constexpr int kWeightWarp = 4 + 4 * kDecGroups;   // producer of the weight ring
 constexpr int kActWarp = 5 + 4 * kDecGroups;      // producer of the activation ring
 constexpr int kMmaWarp = 6 + 4 * kDecGroups;
@@ -96,7 +96,15 @@ constexpr int kMaxRing = 8;
 template <int kBN>
 struct W16Cfg {
     static constexpr int kBlocks = kBN == 32 ? 4 : 2;        // 64-row blocks per stage
-    static constexpr int kAccCols = 2 * kBN;
+    // MMA issuers: a tcgen05.mma costs its issuing thread about 90 cycles at
+    // N = 32 whatever the operands, so at decode two warps issue alternate
+    // stages, each into its own accumulator, and the epilogue adds the two
+    // (measured: 1.45x the issue rate of one thread).  N = 128 MMAs do 4x
+    // the work per instruction, and TMEM has room for one issuer's pair of
+    // accumulators only.
+    static constexpr int kIssuers = kBN == 32 ? 2 : 1;
+    static constexpr int kThreads = (4 + 4 * kDecGroups + 2 + kIssuers) * 32;
+    static constexpr int kAccCols = 2 * kIssuers * kBN;  // [buffer][issuer] accumulators
     static constexpr int kSlotCols = 32 * kBlocks;
     static constexpr int kASlots = (512 - kAccCols) / kSlotCols;  // 3 (kBN 32) or 4 (kBN 128)
     static constexpr int kActStages = 3;
@@ -207,6 +215,22 @@ __device__ __forceinline__ void tc_mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tm
         : "memory");
 }
 
+// 32 accumulator columns from taddr, plus (when `second`) the same columns of
+// the second issuer's accumulator kBN columns further on, added in fp32.
+template <int kIssuers, int kBN>
+__device__ __forceinline__ void ld_acc(uint32_t taddr, uint32_t (&r)[32], bool second) {
+    tmem_ld_32x32b_x32(taddr, r);
+    if (kIssuers > 1 && second) {
+        uint32_t r2[32];
+        tmem_ld_32x32b_x32(taddr + kBN, r2);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) + __uint_as_float(r2[k]));
+    } else {
+        tmem_wait_ld();
+    }
+}
+
 // Named barrier 1 over the four epilogue warps (threads 0-127).
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
@@ -230,7 +254,7 @@ __device__ __forceinline__ float silu_w16(float a) { return a / (1.f + __expf(-a
 // kSwiGLU: GEMM1 over the gate/up pair pack (64 hidden columns per tile);
 // else GEMM2 (128 output columns per tile).  kBN: tokens per tile (MMA N).
 template <bool kSwiGLU, int kBN>
-__global__ void __launch_bounds__(kW16Threads, 1)
+__global__ void __launch_bounds__(W16Cfg<kBN>::kThreads, 1)
     w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const W4a16GemmArgs args) {
     using C = W16Cfg<kBN>;
     extern __shared__ uint8_t smem_raw[];
@@ -259,10 +283,10 @@ __global__ void __launch_bounds__(kW16Threads, 1)
             mbar_init(smem_u32(&tail->aempty[s]), 1);  // MMA commit
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(smem_u32(&tail->accum_full[b]), 1);
+            mbar_init(smem_u32(&tail->accum_full[b]), C::kIssuers);
             mbar_init(smem_u32(&tail->accum_empty[b]), 4);
         }
-        mbar_init(smem_u32(&tail->done), 1);
+        mbar_init(smem_u32(&tail->done), C::kIssuers);
         fence_barrier_init();
         fence_proxy_async_smem();
     }
@@ -272,7 +296,7 @@ __global__ void __launch_bounds__(kW16Threads, 1)
         tmem_relinquish();
     }
     griddep_wait();
-    for (int i = threadIdx.x; i <= n; i += kW16Threads) {
+    for (int i = threadIdx.x; i <= n; i += C::kThreads) {
         tail->off[i] = args.offsets[i];
         tail->mblk[i] = args.mblk_base[i];
     }
@@ -325,8 +349,10 @@ __global__ void __launch_bounds__(kW16Threads, 1)
             for (uint32_t k = i - armed; k < i; ++k)
                 mbar_wait(smem_u32(&full[k % ring]), (k / ring) & 1u, status, kStatusTimeoutDrain);
         }
-    } else if (warp == kMmaWarp) {
+    } else if (warp >= kMmaWarp && warp < kMmaWarp + C::kIssuers) {
         if (lane == 0) {
+            // issuer j takes the stages s of each tile with s % kIssuers == j
+            const int j = warp - kMmaWarp;
             constexpr uint32_t idesc = make_idesc_bf16(kW16Cols, kBN, 0, 0);
             uint32_t i = 0;
             int local = 0;
@@ -339,8 +365,10 @@ __global__ void __launch_bounds__(kW16Threads, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
-                for (int kb = 0; kb < kb_n; kb += C::kBlocks, ++i) {
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>((buf * C::kIssuers + j) * kBN);
+                int sl = 0;  // stage within the tile
+                for (int kb = 0; kb < kb_n; kb += C::kBlocks, ++i, ++sl) {
+                    if (sl % C::kIssuers != j) continue;
                     const int as = static_cast<int>(i % C::kASlots);
                     const int xs = static_cast<int>(i % C::kActStages);
                     if (!mbar_wait(smem_u32(&tail->afull[as]), (i / C::kASlots) & 1u, status, kStatusTimeoutFull) ||
@@ -360,7 +388,7 @@ __global__ void __launch_bounds__(kW16Threads, 1)
                             // B: K-major, 128-byte swizzle; K by 16 = 32 bytes inside the swizzle row.
                             const uint64_t bdesc = make_smem_desc(b_base + kk * 32, 16, 1024, 2);
                             tc_mma_f16_tmem_a(d_tmem, a_tmem + kk * 8, bdesc, idesc,
-                                              (kb | b | kk) != 0 ? 1u : 0u);
+                                              (sl != j || b != 0 || kk != 0) ? 1u : 0u);
                         }
                     }
                     tc_commit(smem_u32(&tail->aempty[as]));
@@ -424,6 +452,9 @@ __global__ void __launch_bounds__(kW16Threads, 1)
         // ---------------- epilogue (warps 0..3) ----------------
         const int q = warp;
         uint16_t* out = static_cast<uint16_t*>(args.out);
+        // the second issuer's accumulator holds a partial sum only if the tiles
+        // have more than one stage
+        const bool second = C::kIssuers > 1 && kb_n > C::kBlocks;
         int local = 0;
         for (int t = first; t < total_tiles; t += stride, ++local) {
             const W16Tile ti = w16_tile(t, tail->off, tail->mblk, n, args.n_tiles, kBN);
@@ -432,8 +463,8 @@ __global__ void __launch_bounds__(kW16Threads, 1)
             const bool got = epi_all(mbar_wait(smem_u32(&tail->accum_full[buf]), bph, status, kStatusTimeoutAccum));
             if (!got) break;  // all four warps together
             tc_fence_after();
-            const uint32_t tbase =
-                tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * kBN);
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>(buf * C::kIssuers * kBN);
             const int valid = ti.rows;
             if (kSwiGLU) {
                 const float sa = __ldg(args.mscale0 + ti.e) * 256.f;
@@ -442,8 +473,7 @@ __global__ void __launch_bounds__(kW16Threads, 1)
 #pragma unroll 1
                     for (int c0 = 0; c0 < kBN; c0 += 32) {
                         uint32_t b[32];
-                        tmem_ld_32x32b_x32(tbase + c0, b);
-                        tmem_wait_ld();
+                        ld_acc<C::kIssuers, kBN>(tbase + c0, b, second);
 #pragma unroll
                         for (int k = 0; k < 32; ++k)
                             xbuf[(c0 + k) * 64 + (q - 2) * 32 + lane] = __uint_as_float(b[k]) * sb;
@@ -455,8 +485,7 @@ __global__ void __launch_bounds__(kW16Threads, 1)
 #pragma unroll 1
                     for (int c0 = 0; c0 < kBN; c0 += 32) {
                         uint32_t a[32];
-                        tmem_ld_32x32b_x32(tbase + c0, a);
-                        tmem_wait_ld();
+                        ld_acc<C::kIssuers, kBN>(tbase + c0, a, second);
 #pragma unroll
                         for (int k = 0; k < 32; ++k) {
                             const float h = silu_w16(__uint_as_float(a[k]) * sa) * xbuf[(c0 + k) * 64 + q * 32 + lane];
@@ -476,8 +505,7 @@ __global__ void __launch_bounds__(kW16Threads, 1)
 #pragma unroll 1
                 for (int c0 = 0; c0 < kBN; c0 += 32) {
                     uint32_t a[32];
-                    tmem_ld_32x32b_x32(tbase + c0, a);
-                    tmem_wait_ld();
+                    ld_acc<C::kIssuers, kBN>(tbase + c0, a, second);
 #pragma unroll
                     for (int k = 0; k < 32; ++k)
                         if (c0 + k < valid)
@@ -572,7 +600,8 @@ cudaError_t launch_w16(const CUtensorMap& tm, const W4a16GemmArgs& a, int num_sm
     int64_t g = num_sms;
     if (max_tiles < g) g = max_tiles;
     if (g < 1) g = 1;
-    launch_k(w4a16_gemm_kernel<kSwiGLU, kBN>, dim3(static_cast<unsigned>(g)), dim3(kW16Threads), smem, st, tm, a);
+    launch_k(w4a16_gemm_kernel<kSwiGLU, kBN>, dim3(static_cast<unsigned>(g)), dim3(W16Cfg<kBN>::kThreads), smem, st, tm,
+             a);
     return cudaGetLastError();
 }
 
