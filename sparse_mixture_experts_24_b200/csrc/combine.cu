@@ -15,6 +15,11 @@
 
 namespace moe {
 
+// kChunk slots at a time: their row indices and gates are loaded first, then
+// all their O vectors, so that a thread has kChunk loads of O in flight (the
+// row lookups make each load depend on an earlier one); the products are
+// still added in slot order.
+template <int kChunk>
 __global__ void __launch_bounds__(256) combine_bf16_kernel(const uint4* __restrict__ O,
                                                            const int32_t* __restrict__ token_row,
                                                            const float* __restrict__ topk_w,
@@ -30,11 +35,22 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const uint4* __restri
         float acc[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-        for (int k = 0; k < K; ++k) {
-            const int32_t r = __ldg(token_row + t * K + k);
-            if (r < 0) continue;
-            const float g = __ldg(topk_w + t * K + k);
-            fma_bf16x8(acc, g, __ldg(O + static_cast<int64_t>(r) * vec_per_row + v));
+        for (int k0 = 0; k0 < K; k0 += kChunk) {
+            int32_t r[kChunk];
+            float g[kChunk];
+            uint4 o[kChunk];
+#pragma unroll
+            for (int j = 0; j < kChunk; ++j) {
+                const bool in = k0 + j < K;
+                r[j] = in ? __ldg(token_row + t * K + k0 + j) : -1;
+                g[j] = in ? __ldg(topk_w + t * K + k0 + j) : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < kChunk; ++j)
+                o[j] = r[j] >= 0 ? __ldg(O + static_cast<int64_t>(r[j]) * vec_per_row + v) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int j = 0; j < kChunk; ++j)
+                if (r[j] >= 0) fma_bf16x8(acc, g[j], o[j]);
         }
         y[i] = pack_bf16x8(acc);
     }
@@ -76,10 +92,17 @@ cudaError_t launch_combine(const void* O, bool bf16, const int32_t* token_row, c
     const int64_t cap = static_cast<int64_t>(num_sms) * 16;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    if (bf16)
-        launch_k(combine_bf16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, 
-            static_cast<const uint4*>(O), token_row, topk_w, T, K, d / 8, static_cast<uint4*>(y));
-    else
+    if (bf16) {
+        const dim3 grid(static_cast<unsigned>(blocks));
+        const uint4* o = static_cast<const uint4*>(O);
+        uint4* yv = static_cast<uint4*>(y);
+        if (K == 1)
+            launch_k(combine_bf16_kernel<1>, grid, dim3(256), 0, st, o, token_row, topk_w, T, K, d / 8, yv);
+        else if (K == 2)
+            launch_k(combine_bf16_kernel<2>, grid, dim3(256), 0, st, o, token_row, topk_w, T, K, d / 8, yv);
+        else
+            launch_k(combine_bf16_kernel<4>, grid, dim3(256), 0, st, o, token_row, topk_w, T, K, d / 8, yv);
+    } else
         launch_k(combine_f32_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, 
             static_cast<const float4*>(O), token_row, topk_w, T, K, d / 4, static_cast<float4*>(y));
     return cudaGetLastError();

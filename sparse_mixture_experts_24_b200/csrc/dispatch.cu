@@ -64,11 +64,12 @@ __global__ void __launch_bounds__(kPairsPerBlock) rank_kernel(const int32_t* __r
 }
 
 // Per-block counts are walked in chunks staged through shared memory, so
-// the loads of a chunk are all in flight together; each expert's column is
+// the loads of a chunk are all in flight together (16 per thread); each expert's column is
 // then scanned in place.  blockcounts ends up holding, for every block and
 // expert, the block's first rank inside the expert's segment (the segment's
 // offset is added by the scatter).
 constexpr int kScanSmemInts = 8192;
+constexpr int kScanUnroll = 16;
 
 __global__ void __launch_bounds__(256) scan_kernel(int32_t* __restrict__ blockcounts, int nblk,
                                                    int n, int capacity, int bm,
@@ -86,7 +87,19 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* __restrict__ blockco
         const int cnt = nb * n;
         int32_t* g = blockcounts + static_cast<int64_t>(b0) * n;
         __syncthreads();
-        for (int i = threadIdx.x; i < cnt; i += 256) s_chunk[i] = g[i];
+        for (int i0 = 0; i0 < cnt; i0 += 256 * kScanUnroll) {
+            int32_t v[kScanUnroll];  // all of a thread's loads in flight together
+#pragma unroll
+            for (int u = 0; u < kScanUnroll; ++u) {
+                const int i = i0 + u * 256 + static_cast<int>(threadIdx.x);
+                v[u] = i < cnt ? g[i] : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < kScanUnroll; ++u) {
+                const int i = i0 + u * 256 + static_cast<int>(threadIdx.x);
+                if (i < cnt) s_chunk[i] = v[u];
+            }
+        }
         __syncthreads();
         if (e < n) {
             for (int b = 0; b < nb; ++b) {

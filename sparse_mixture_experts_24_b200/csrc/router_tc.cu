@@ -15,9 +15,16 @@
 //
 // router_tc_kernel: one CTA per (128 tokens, slice of d): the d range is split
 // over gridDim.y CTAs so that small token counts still fill the GPU; warp 0
-// streams x (128 x 64) and the three W_g parts (Npad x 64 each) by TMA through
-// a multi-stage ring; warp 1 issues tcgen05.mma M=128, N=Npad, K=16 three
-// times per K step; warps 2-5 read the 128 x Npad fp32 accumulator from TMEM.
+// streams x (128 x 64) and the three W_g parts (Npad x 64 each, adjacent in
+// shared memory) by TMA through a multi-stage ring; warp 1 issues the
+// tcgen05.mma (M=128, K=16) of every K step; warps 2-5 read the fp32
+// accumulators from TMEM.  With Npad <= 128 each part has an accumulator of
+// its own, so that the three parts are one B operand of N = 3 Npad (one MMA
+// per K step for Npad <= 80; N = 2 Npad and N = Npad up to 128), and the
+// epilogue adds (hi + mid) + lo; wider W_g keeps one accumulator that the
+// three MMAs of a K step all add into.  A tcgen05.mma costs its issuing thread
+// about the same whatever its N, so fewer, wider MMAs finish the K steps
+// sooner when Npad is small.
 //   Logits variant: each CTA stages its partial logits in shared memory and
 //   writes them as whole rows to [split][T][n]; router_topk_kernel (router.cu)
 //   sums the splits in order and selects.
@@ -37,24 +44,46 @@
 
 namespace moe {
 
-// W_g [d][n] fp32 -> parts [3][npad][d] bf16 (rows n..npad-1 are zero).
+// W_g [d][n] fp32 -> parts [3][npad][d] bf16 (rows n..npad-1 are zero).  One
+// block per 32 rows of d and 32 experts: the tile is read along the experts
+// (W_g's contiguous dimension) into shared memory, four loads per thread in
+// flight together, and written along d, two values per 32-bit store (d is a
+// multiple of 64).
 __global__ void __launch_bounds__(256) wg_split_kernel(const float* __restrict__ Wg, int d, int n,
                                                        int npad, uint16_t* __restrict__ parts) {
     griddep_wait();
+    __shared__ float tile[32][33];
+    const int j0 = static_cast<int>(blockIdx.x) * 32, e0 = static_cast<int>(blockIdx.y) * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    float v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        v[u] = (e0 + tx < n) ? __ldg(Wg + static_cast<int64_t>(j0 + ty + 8 * u) * n + e0 + tx) : 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) tile[ty + 8 * u][tx] = v[u];
+    __syncthreads();
     const int64_t total = static_cast<int64_t>(npad) * d;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int e = static_cast<int>(i / d);
-        const int j = static_cast<int>(i - static_cast<int64_t>(e) * d);
-        const float w = (e < n) ? __ldg(Wg + static_cast<int64_t>(j) * n + e) : 0.f;
-        const __nv_bfloat16 hi = __float2bfloat16_rn(w);
-        const float r1 = w - __bfloat162float(hi);
-        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-        const float r2 = r1 - __bfloat162float(mid);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
-        parts[i] = __bfloat16_as_ushort(hi);
-        parts[total + i] = __bfloat16_as_ushort(mid);
-        parts[2 * total + i] = __bfloat16_as_ushort(lo);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int q = static_cast<int>(threadIdx.x) + 256 * u;
+        const int c = q >> 4, pr = q & 15;  // expert e0 + c, rows j0 + 2 pr, j0 + 2 pr + 1
+        if (e0 + c >= npad) continue;
+        const int64_t at = static_cast<int64_t>(e0 + c) * d + j0 + 2 * pr;
+        uint32_t packed[3] = {0u, 0u, 0u};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float w = tile[2 * pr + h][c];
+            const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+            const float r1 = w - __bfloat162float(hi);
+            const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+            const float r2 = r1 - __bfloat162float(mid);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+            packed[0] |= static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << (16 * h);
+            packed[1] |= static_cast<uint32_t>(__bfloat16_as_ushort(mid)) << (16 * h);
+            packed[2] |= static_cast<uint32_t>(__bfloat16_as_ushort(lo)) << (16 * h);
+        }
+#pragma unroll
+        for (int p = 0; p < 3; ++p) *reinterpret_cast<uint32_t*>(parts + p * total + at) = packed[p];
     }
     griddep_launch_dependents();
 }
@@ -80,9 +109,8 @@ __host__ __device__ inline int rt_stages(int npad) {
     return s > kRtMaxStages ? kRtMaxStages : s;
 }
 
-// Partial logits staged per CTA: 128 rows of npad rounded up to 32 (the
-// accumulator is read 32 columns at a time) plus one float (the odd pitch keeps
-// a warp's 32 rows in 32 different banks).
+// Partial logits staged per CTA: 128 rows of npad rounded up to 32 plus one
+// float (the odd pitch keeps a warp's 32 rows in 32 different banks).
 __host__ __device__ inline int rt_stage_pitch(int npad) { return (npad + 31) / 32 * 32 + 1; }
 __host__ __device__ inline int rt_ring_bytes(int npad) {
     const int ring = rt_stages(npad) * rt_stage_bytes(npad);
@@ -90,15 +118,21 @@ __host__ __device__ inline int rt_ring_bytes(int npad) {
     return ring > staged ? ring : staged;
 }
 
+// volatile keeps these loads after the cluster barrier that publishes the
+// partials; with no memory clobber, arithmetic may move around them, so that
+// several loads are issued before their first use.
 __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
     float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
     return v;
 }
 
+// Accumulator columns: one group of Npad per part (Npad <= 128), else one.
+__host__ __device__ inline int rt_groups(int npad) { return npad <= 128 ? 3 : 1; }
+
 __host__ inline int rt_tmem_cols(int npad) {
     int c = 32;
-    while (c < npad) c <<= 1;
+    while (c < rt_groups(npad) * npad) c <<= 1;
     return c;
 }
 
@@ -177,7 +211,13 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t idesc = make_idesc_bf16(kRtBM, npad, 0, 0);
+            // the three parts: one MMA of N = 3 Npad (Npad <= 80), N = 2 Npad
+            // plus N = Npad (Npad <= 128), or three of N = Npad into one
+            // accumulator
+            const int groups = rt_groups(npad);
+            const int n_first = groups == 1 ? npad : (npad <= 80 ? 3 * npad : 2 * npad);
+            const uint32_t idesc_first = make_idesc_bf16(kRtBM, n_first, 0, 0);
+            const uint32_t idesc_part = make_idesc_bf16(kRtBM, npad, 0, 0);
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -192,11 +232,15 @@ __global__ void __launch_bounds__(kRtThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < kRtBK / 16; ++kk) {
                     const uint64_t adesc = make_smem_desc(a_base + kk * 32, 16, 1024, 2);
-#pragma unroll
-                    for (int p = 0; p < 3; ++p) {
-                        const uint64_t bdesc =
-                            make_smem_desc(b_base + p * part_bytes + kk * 32, 16, 1024, 2);
-                        tc_mma_f16(tmem_base, adesc, bdesc, idesc, (kb | kk | p) != 0 ? 1u : 0u);
+                    const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+                    tc_mma_f16(tmem_base, adesc, make_smem_desc(b_base + kk * 32, 16, 1024, 2), idesc_first, acc);
+                    if (groups == 1) {
+                        for (int p = 1; p < 3; ++p)
+                            tc_mma_f16(tmem_base, adesc, make_smem_desc(b_base + p * part_bytes + kk * 32, 16, 1024, 2),
+                                       idesc_part, 1u);
+                    } else if (n_first == 2 * npad) {
+                        tc_mma_f16(tmem_base + static_cast<uint32_t>(2 * npad), adesc,
+                                   make_smem_desc(b_base + 2 * part_bytes + kk * 32, 16, 1024, 2), idesc_part, acc);
                     }
                 }
                 tc_commit(smem_u32(&tail->empty[stage]));
@@ -224,12 +268,23 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         have_acc = mbar_wait(smem_u32(&tail->accum_full), 0, status, kStatusTimeoutAccum);
         if (have_acc) {
             tc_fence_after();
-            for (int c = 0; c < npad; c += 32) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + c, v);
+            const int groups = rt_groups(npad);
+            const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+            for (int c = 0; c < npad; c += 16) {
+                float a[16];
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(lane_base + c, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int q = 0; q < 32; ++q) stage_rows[r * pitch + c + q] = __uint_as_float(v[q]);
+                for (int q = 0; q < 16; ++q) a[q] = __uint_as_float(v[q]);
+                for (int g = 1; g < groups; ++g) {  // (hi + mid) + lo
+                    tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(g * npad + c), v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) a[q] += __uint_as_float(v[q]);
+                }
+#pragma unroll
+                for (int q = 0; q < 16; ++q) stage_rows[r * pitch + c + q] = a[q];
             }
             tc_fence_before();
         }
@@ -254,26 +309,40 @@ __global__ void __launch_bounds__(kRtThreads, 1)
 #pragma unroll
         for (int sp = 0; sp < kRouterMaxSplits; ++sp)
             part_base[sp] = mapa_shared(smem_u32(stage_rows), static_cast<uint32_t>(sp < splits ? sp : 0));
-        for (int r = static_cast<int>(rank) * rows_per + warp; r < r_end; r += kRtThreads / 32) {
-            const int64_t t = static_cast<int64_t>(m0) + r;
-            if (t >= T) break;  // rows ascend: the rest of this warp's rows are past T too
-            float v[kNS];
+        // a warp takes kRows consecutive rows at a time: all their partials
+        // are loaded before any selection, so that the remote loads of the
+        // kRows rows are in flight together
+        constexpr int kRows = kNS <= 4 ? 4 : 2;
+        constexpr int kWarps = kRtThreads / 32;
+        for (int r0 = static_cast<int>(rank) * rows_per + warp * kRows; r0 < r_end; r0 += kWarps * kRows) {
+            float v[kRows][kNS];
 #pragma unroll
-            for (int i = 0; i < kNS; ++i) {
-                const int e = lane + 32 * i;
-                float part[kRouterMaxSplits];
+            for (int j = 0; j < kRows; ++j) {
+                const int r = r0 + j;
+                const bool row_ok = r < r_end && static_cast<int64_t>(m0) + r < T;
 #pragma unroll
-                for (int sp = 0; sp < kRouterMaxSplits; ++sp)
-                    part[sp] = (e < n && sp < splits)
-                                   ? ld_shared_cluster_f32(part_base[sp] + static_cast<uint32_t>(r * pitch + e) * 4u)
-                                   : 0.f;
-                float a = 0.f;
+                for (int i = 0; i < kNS; ++i) {
+                    const int e = lane + 32 * i;
+                    float part[kRouterMaxSplits];
 #pragma unroll
-                for (int sp = 0; sp < kRouterMaxSplits; ++sp)
-                    if (sp < splits) a += part[sp];
-                v[i] = (a != a) ? -INFINITY : a;  // NaN ranks lowest
+                    for (int sp = 0; sp < kRouterMaxSplits; ++sp)
+                        part[sp] = (row_ok && e < n && sp < splits)
+                                       ? ld_shared_cluster_f32(part_base[sp] +
+                                                               static_cast<uint32_t>(r * pitch + e) * 4u)
+                                       : 0.f;
+                    float a = 0.f;
+#pragma unroll
+                    for (int sp = 0; sp < kRouterMaxSplits; ++sp)
+                        if (sp < splits) a += part[sp];
+                    v[j][i] = (a != a) ? -INFINITY : a;  // NaN ranks lowest
+                }
             }
-            warp_topk_softmax<kNS>(v, n, K, lane, topk_idx + t * K, topk_w + t * K);
+#pragma unroll
+            for (int j = 0; j < kRows; ++j) {
+                const int r = r0 + j;
+                const int64_t t = static_cast<int64_t>(m0) + r;
+                if (r < r_end && t < T) warp_topk_softmax<kNS>(v[j], n, K, lane, topk_idx + t * K, topk_w + t * K);
+            }
         }
         cluster_sync();  // no CTA leaves while another reads its staged partial
     }
@@ -303,11 +372,10 @@ static int router_splits(int64_t T, int d, int num_sms) {
 }
 
 static void launch_wg_split(const float* Wg, uint16_t* parts, int d, int n, int num_sms, cudaStream_t st) {
+    (void)num_sms;
     const int npad = (n + 15) / 16 * 16;
-    const int64_t total = static_cast<int64_t>(npad) * d;
-    int64_t sb = (total + 255) / 256;
-    if (sb > static_cast<int64_t>(num_sms) * 8) sb = static_cast<int64_t>(num_sms) * 8;
-    launch_k(wg_split_kernel, dim3(static_cast<unsigned>(sb)), dim3(256), 0, st, Wg, d, n, npad, parts);
+    const dim3 grid(static_cast<unsigned>(d / 32), static_cast<unsigned>((npad + 31) / 32));
+    launch_k(wg_split_kernel, grid, dim3(256), 0, st, Wg, d, n, npad, parts);
 }
 
 cudaError_t launch_router_logits_tc(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const float* Wg,

@@ -9,19 +9,17 @@
 
 namespace moe {
 
-// Candidate key: larger key = larger logit, equal logits -> lower expert
-// index (the low word holds the inverted index).  The float is mapped to an
-// unsigned integer with the same order (sign bit set for non-negative values,
-// all bits inverted for negative ones); -0 is folded into +0 first so that
-// the two zeros tie like the comparison of their values.  0 = no candidate.
-__device__ __forceinline__ uint64_t topk_key(float v, int e) {
+// Order key of a logit: an unsigned integer with the same order as the
+// value (sign bit set for non-negative values, all bits inverted for negative
+// ones); -0 is folded into +0 first so that the two zeros tie like the
+// comparison of their values.  Every finite or infinite value maps above 0, so
+// 0 means "no candidate".
+__device__ __forceinline__ uint32_t topk_ord(float v) {
     const uint32_t b = __float_as_uint(v + 0.0f);
-    const uint32_t ord = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-    return (static_cast<uint64_t>(ord) << 32) | static_cast<uint64_t>(0xFFFFFFFFu - static_cast<uint32_t>(e));
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-__device__ __forceinline__ float topk_key_value(uint64_t key) {
-    const uint32_t ord = static_cast<uint32_t>(key >> 32);
+__device__ __forceinline__ float topk_ord_value(uint32_t ord) {
     return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord);
 }
 
@@ -37,20 +35,24 @@ __device__ __forceinline__ void warp_topk_softmax(const float (&v)[NS], int n, i
     int my_idx = 0;      // selection `lane` (K <= 32)
     float my_ex = 0.f;
     for (int k = 0; k < K; ++k) {
-        uint64_t best = 0;
+        // this lane's best untaken slot (slots ascend in expert index, so the
+        // strict '>' keeps the lower index on equal keys), then the warp's
+        // largest key and, among the lanes holding it, the lowest index
+        uint32_t best = 0;
+        int best_e = 0x7FFFFFFF;
 #pragma unroll
         for (int i = 0; i < NS; ++i) {
             const int e = lane + 32 * i;
-            const uint64_t key = (e < n && !((taken >> i) & 1u)) ? topk_key(v[i], e) : 0ull;
-            best = key > best ? key : best;
+            const uint32_t key = (e < n && !((taken >> i) & 1u)) ? topk_ord(v[i]) : 0u;
+            if (key > best) {
+                best = key;
+                best_e = e;
+            }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
-            best = other > best ? other : best;
-        }
-        const int bi = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(best));
-        const float bv = topk_key_value(best);
+        const uint32_t top = __reduce_max_sync(0xffffffffu, best);
+        const int bi = static_cast<int>(
+            __reduce_min_sync(0xffffffffu, best == top ? static_cast<uint32_t>(best_e) : 0x7FFFFFFFu));
+        const float bv = topk_ord_value(top);
         if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
         if (k == 0) m = bv;
         const float ex = expf(bv - m);

@@ -32,6 +32,13 @@ SMALL = [
     ("bf16_router_split2", 600, 1024, 128, 40, 3, "bf16"),
     ("bf16_router_split4", 1000, 2048, 128, 8, 2, "bf16"),
     ("bf16_router_K10", 600, 1024, 64, 32, 10, "bf16"),
+    # tensor-core router accumulators: one MMA of N = 3 Npad (Npad = 80), two
+    # (N = 2 Npad + Npad; Npad = 112 with padding rows, 128), three into one
+    # accumulator (Npad = 144)
+    ("bf16_router_n80", 600, 256, 64, 80, 2, "bf16"),
+    ("bf16_router_n100", 520, 512, 64, 100, 4, "bf16"),
+    ("bf16_router_n128", 600, 256, 128, 128, 2, "bf16"),
+    ("bf16_router_n130", 530, 256, 64, 130, 2, "bf16"),
     ("f32_tiny", 64, 128, 256, 8, 2, "f32"),
     ("f32_n40_k4", 200, 64, 128, 40, 4, "f32"),
     ("f32_n1", 33, 64, 64, 1, 1, "f32"),
