@@ -10,17 +10,21 @@
 // 4-bit weights ("Mixture of Experts: Why Mixtral Only Wakes Up Two
 // Specialists", Part 4).
 //
-// One persistent CTA per SM, 320 threads, tiles of 128 rows x kBN columns of
+// One persistent CTA per SM, 352 threads, tiles of 128 rows x kBN columns of
 // the packed B (kBN = 128: two accumulators, 6 stages of 36 KB; kBN = 256: one
 // accumulator, 4 stages of 54 KB -- the block scales take the rest of TMEM):
 //   warp 0     TMA producer: per stage a K step of 256 (128 bytes of codes per
-//              row): A 128 rows (128-byte swizzle), kBN / 128 blocks of 128
-//              K-major weight rows (GEMM1: the w1|w3 pair pack, 64 hidden
-//              columns per block; GEMM2: w2), and by plain bulk copies the
-//              matching 512-byte scale chunks (4 for A, 4 per B block).
-//   warp 1     allocates 512 TMEM columns; per 64-wide K step it copies the
-//              scale chunks into TMEM (tcgen05.cp 32x128b.warpx4) and issues
-//              tcgen05.mma kind::mxf4nvf4 block16 M=128 N=kBN.
+//              row): A 128 rows (128-byte swizzle), the kBN K-major weight rows
+//              in one copy (GEMM1: the w1|w3 pair pack, 64 hidden columns per
+//              128-row block; GEMM2: w2), and by plain bulk copies the matching
+//              512-byte scale chunks (4 for A, 4 per 128-row B block).
+//   warp 10    per stage, copies the scale chunks into that stage's TMEM
+//              columns (tcgen05.cp 32x128b.warpx4, 3 or 2 per 64-wide K step)
+//              and commits them to the stage's scales-ready barrier.
+//   warp 1     allocates 512 TMEM columns; once a stage's scales are in TMEM
+//              it issues tcgen05.mma kind::mxf4nvf4 block16 M=128 N=kBN.
+//              With the scale copies on a warp of their own, neither issuing
+//              thread carries all 16 of a stage's tensor-core instructions.
 //   warps 2-9  epilogue, two warps per TMEM lane quadrant splitting the
 //              columns: accumulator x row scale x matrix scale, SwiGLU (GEMM1)
 //              or a copy (GEMM2), bf16 rows.
@@ -39,7 +43,8 @@ constexpr int kSfbBlockBytes = 4 * 512; // the same for one 128-row block of B
 constexpr int kMaxN = 256;
 constexpr int kTmemCols = 512;
 constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, each taking half the columns
-constexpr int kThreads = (2 + kEpiWarps) * 32;
+constexpr int kCpWarp = 2 + kEpiWarps;  // the scale-factor copies
+constexpr int kThreads = (3 + kEpiWarps) * 32;
 
 // Tile width kBN (128 or 256 output columns of the packed B, i.e. 64 or 128
 // hidden columns of GEMM1's w1|w3 pairs) and tile height kTM (rows of A per
@@ -64,6 +69,8 @@ struct Cfg {
 struct __align__(8) SmemTail {
     uint64_t full[6];
     uint64_t empty[6];
+    uint64_t sf_ready[6];  // the stage's scale chunks are in TMEM
+    uint64_t cp_done;
     uint64_t accum_full[2];
     uint64_t accum_empty[2];
     uint64_t done;
@@ -130,12 +137,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(smem_u32(&tail->full[s]), 1);
             mbar_init(smem_u32(&tail->empty[s]), 1);
+            mbar_init(smem_u32(&tail->sf_ready[s]), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&tail->accum_full[b]), 1);
             mbar_init(smem_u32(&tail->accum_empty[b]), kEpiWarps);
         }
         mbar_init(smem_u32(&tail->done), 1);
+        mbar_init(smem_u32(&tail->cp_done), 1);
         fence_barrier_init();
         fence_proxy_async_smem();
     }
@@ -193,12 +202,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int64_t ck = static_cast<int64_t>(ks) * 4 * 512;
                     tma_load_2d(base, &tm_a, fb, kx, ti.row0);
                     bulk_load(sf_smem, sfa + ck, kSfaBytes, fb);
+                    // the map's box is kBN rows: the tile's B blocks in one copy
+                    tma_load_3d(base + C::kABytes, &tm_b, fb, kx, r0, ti.e);
 #pragma unroll
-                    for (int b = 0; b < C::kBlocks; ++b) {
-                        tma_load_3d(base + C::kABytes + b * kBBlockBytes, &tm_b, fb, kx, r0 + 128 * b, ti.e);
+                    for (int b = 0; b < C::kBlocks; ++b)
                         bulk_load(sf_smem + kSfaBytes + b * kSfbBlockBytes,
                                   sfb + static_cast<int64_t>(b) * kb64_total * 512 + ck, kSfbBlockBytes, fb);
-                    }
                     if (++stage == C::kStages) {
                         stage = 0;
                         phase ^= 1u;
@@ -227,24 +236,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
                 for (int ks = 0; ks < args.k_steps; ++ks) {
-                    if (!mbar_wait(smem_u32(&tail->full[stage]), phase, status, kStatusTimeoutFull)) {
+                    // the scale copies of this stage are complete (so are its TMA copies)
+                    if (!mbar_wait(smem_u32(&tail->sf_ready[stage]), phase, status, kStatusTimeoutFull)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t base = smem_u32(smem + stage * C::kStageBytes);
-                    const uint32_t sfa_smem = base + C::kABytes + C::kBlocks * kBBlockBytes;
-                    const uint32_t sfb_smem = sfa_smem + kSfaBytes;
                     const uint32_t sf_col = tmem_base + static_cast<uint32_t>(C::kSfBase + stage * C::kSfCols);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint32_t sfa_t = sf_col + 4 * kk;
                         const uint32_t sfb_t = sf_col + 16 + 4 * C::kBlocks * kk;
-                        tc_cp_32x128b_warpx4(sfa_t, make_smem_desc(sfa_smem + kk * 512, 0, 128, 0));
-#pragma unroll
-                        for (int b = 0; b < C::kBlocks; ++b)
-                            tc_cp_32x128b_warpx4(sfb_t + 4 * b,
-                                                 make_smem_desc(sfb_smem + b * kSfbBlockBytes + kk * 512, 0, 128, 0));
                         const uint64_t adesc = make_smem_desc(base + kk * 32, 16, 1024, 2);
                         const uint64_t bdesc = make_smem_desc(base + C::kABytes + kk * 32, 16, 1024, 2);
                         tc_mma_fp4_block16(d_tmem, adesc, bdesc, idesc, sfa_t, sfb_t, (ks | kk) != 0 ? 1u : 0u);
@@ -259,6 +262,46 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_commit(smem_u32(&tail->done));
             mbar_wait(smem_u32(&tail->done), 0, status, kStatusTimeoutDrain);
+        }
+    } else if (warp == kCpWarp) {
+        if (lane == 0) {
+            // ---------------- scale chunks -> TMEM ----------------
+            // A stage's TMEM scale columns are written again only after its
+            // next full barrier, which follows the empty barrier that the
+            // MMAs reading them committed to.
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int t = first; t < total_tiles; t += stride) {
+                bool ok = true;
+                for (int ks = 0; ks < args.k_steps; ++ks) {
+                    if (!mbar_wait(smem_u32(&tail->full[stage]), phase, status, kStatusTimeoutFull)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t base = smem_u32(smem + stage * C::kStageBytes);
+                    const uint32_t sfa_smem = base + C::kABytes + C::kBlocks * kBBlockBytes;
+                    const uint32_t sfb_smem = sfa_smem + kSfaBytes;
+                    const uint32_t sf_col = tmem_base + static_cast<uint32_t>(C::kSfBase + stage * C::kSfCols);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        tc_cp_32x128b_warpx4(sf_col + 4 * kk, make_smem_desc(sfa_smem + kk * 512, 0, 128, 0));
+#pragma unroll
+                        for (int b = 0; b < C::kBlocks; ++b)
+                            tc_cp_32x128b_warpx4(sf_col + 16 + 4 * C::kBlocks * kk + 4 * b,
+                                                 make_smem_desc(sfb_smem + b * kSfbBlockBytes + kk * 512, 0, 128, 0));
+                    }
+                    tc_commit(smem_u32(&tail->sf_ready[stage]));
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+            }
+            // every copy of this thread is complete before TMEM is freed
+            tc_commit(smem_u32(&tail->cp_done));
+            mbar_wait(smem_u32(&tail->cp_done), 0, status, kStatusTimeoutDrain);
         }
     } else {
         // ---------------- epilogue (warps 2..9) ----------------

@@ -255,6 +255,7 @@ struct moe_handle {
     CUtensorMap tm_xq4, tm_hq4, tm_wp4[2];
     CUtensorMap tm_xq4s, tm_hq4s;  // the same codes in 32-row boxes
     const void* c_wp4[2] = {nullptr, nullptr};
+    int c_wp4_rows[2] = {0, 0};  // box rows the cached maps were encoded with
     // 4-bit weights decoded into tensor memory: Xp and H as 3-D maps whose
     // boxes hold 4 chunks of 32 rows ([0]) or 2 chunks of 128 rows ([1])
     CUtensorMap tm_xpw[2], tm_hw[2];
@@ -852,15 +853,17 @@ moe_status run_experts_w4a4(moe_handle* h, int64_t T, const void* x, const float
     h->launches += 1;
     trace_mark(h, 2, st);
     // wp[0]: the gate/up pair pack (2 ffn rows of d codes), wp[1]: w2 (d rows of ffn)
+    const int bn = moe::w4a4_tile_cols(wide);
     for (int m = 0; m < 2; ++m) {
+        // boxes of a whole tile's rows: the kernel brings them in one copy
         const uint64_t K = m == 0 ? h->d : h->F, N = m == 0 ? 2 * static_cast<uint64_t>(h->F) : h->d;
-        if (wp[m] != h->c_wp4[m]) {
-            if (!encode_codes(&h->tm_wp4[m], wp[m], K / 2, N, h->n))
+        if (wp[m] != h->c_wp4[m] || h->c_wp4_rows[m] != bn) {
+            if (!encode_codes(&h->tm_wp4[m], wp[m], K / 2, N, h->n, static_cast<uint32_t>(bn)))
                 return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for packed 4-bit weights");
             h->c_wp4[m] = wp[m];
+            h->c_wp4_rows[m] = bn;
         }
     }
-    const int bn = moe::w4a4_tile_cols(wide);
     moe::W4a4GemmArgs a1{};
     a1.offsets = h->db.offsets;
     a1.mblk_base = h->db.mblk_base;
