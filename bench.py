@@ -91,7 +91,7 @@ def touched_experts(idx: np.ndarray, n: int) -> np.ndarray:
 
 def algorithmic(cfg, counts, experts="bf16"):
     """Bytes and FLOPs each stage must move / do, from the routing of the step.
-    E4M3 experts: one byte per weight plus its column's fp32 scale; the gemm1
+    E4M3 experts: one byte per weight plus its column's fp32 scale; the gemm2
     stage also holds the hidden-row quantisation (bf16 H read, codes written)."""
     es = 2 if cfg.dtype == "bf16" else 4
     T, d, F, n, K = cfg.T, cfg.d, cfg.ffn, cfg.n, cfg.K
@@ -104,17 +104,18 @@ def algorithmic(cfg, counts, experts="bf16"):
         gemm1_bytes = w13 + R * d * es + R * F * es
         gemm2_bytes = w2 + R * F * es + R * d * es
     elif experts == "w4a4":
-        # weights as fp4; A operands as 4-bit codes + scales; the gemm1 stage
+        # weights as fp4; A operands as 4-bit codes + scales; the gemm2 stage
         # also holds the hidden-row quantisation (bf16 H read, codes written)
         w13 = used * 2 * (d * F // 2 + d * F // 16 + 4)
         w2 = used * (F * d // 2 + F * d // 16 + 4)
-        gemm1_bytes = w13 + R * (d // 2 + d // 16 + 4) + R * F * es + (R * F * es + R * (F // 2 + F // 16 + 4))
-        gemm2_bytes = w2 + R * (F // 2 + F // 16 + 4) + R * d * es
+        hq = R * F * es + R * (F // 2 + F // 16 + 4)
+        gemm1_bytes = w13 + R * (d // 2 + d // 16 + 4) + R * F * es
+        gemm2_bytes = hq + w2 + R * (F // 2 + F // 16 + 4) + R * d * es
     elif experts == "e4m3":
         w13 = used * 2 * (d * F + F * 4)
         w2 = used * (F * d + d * 4)
-        gemm1_bytes = w13 + R * (d + 4) + R * F * 2 + (R * F * 2 + R * (F + 4))
-        gemm2_bytes = w2 + R * (F + 4) + R * d * es
+        gemm1_bytes = w13 + R * (d + 4) + R * F * 2
+        gemm2_bytes = (R * F * 2 + R * (F + 4)) + w2 + R * (F + 4) + R * d * es
     else:
         w13 = used * 2 * d * F * es
         w2 = used * F * d * es

@@ -525,8 +525,10 @@ MOE_API moe_status moe_sync_status(moe_handle *h, moe_stream_t stream);
  * Per-stage timing with CUDA events, for profiling.  After moe_trace_begin(h,
  * max_calls) each of the next max_calls moe_forward / moe_forward_with_routing
  * calls records events around its stages on its stream:
- *   stage 0 router, 1 dispatch (rank, scan, scatter), 2 gather, 3 GEMM1 (w1/w3
- *   + SwiGLU), 4 GEMM2 (w2), 5 combine
+ *   stage 0 router, 1 dispatch (rank, scan, scatter), 2 gather (or the x-row
+ *   quantisation of the 8- and 4-bit forms), 3 GEMM1 (w1/w3 + SwiGLU), 4 GEMM2
+ *   (w2; with the H-row quantisation first in the 8- and 4-bit-activation
+ *   forms), 5 combine
  * (stage 0 is 0 ms for moe_forward_with_routing).  moe_trace_end waits for the
  * recorded events, writes the summed milliseconds of each stage into
  * stage_ms[0 .. n_stages-1] (n_stages <= 6), the number of traced calls into

@@ -731,10 +731,10 @@ moe_status run_experts_e4m3(moe_handle* h, int64_t T, const void* x, const int32
     e = pair ? moe::launch_tc_gemm1_pair_e4m3(h->tm_x8, h->tm_q1, h->tm_q3, a1, h->num_sms, st)
              : moe::launch_tc_gemm1_e4m3(h->tm_x8, h->tm_q1, h->tm_q3, a1, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
+    trace_mark(h, 3, st);  // the GEMM1 stage is the GEMM1 kernel alone; the H rows go with GEMM2
     e = moe::launch_quantize_rows_e4m3(h->h, true, nullptr, R, R, used_rows, h->F, h->h8, h->hs, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "hidden-row quantisation launch");
     h->launches += 2;
-    trace_mark(h, 3, st);
     moe::TcGemmArgs a2 = a1;
     a2.k_blocks = (h->F + 127) / 128;
     a2.n_tiles = (h->d + 255) / 256;
@@ -884,11 +884,11 @@ moe_status run_experts_w4a4(moe_handle* h, int64_t T, const void* x, const float
     e = moe::launch_w4a4_gemm1(tile_rows == 32 ? h->tm_xq4s : h->tm_xq4, h->tm_wp4[0], a1, wide, tile_rows,
                                h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
+    trace_mark(h, 3, st);  // the GEMM1 stage is the GEMM1 kernel alone; the H rows go with GEMM2
     e = moe::launch_w4a4_rows(static_cast<const uint16_t*>(h->h), nullptr, R, R, h->F, h->db.offsets,
                               h->db.mblk_base, h->n, tile_rows, h->hq4, h->hc4, h->hr4, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "hidden-row quantisation launch");
     h->launches += 2;
-    trace_mark(h, 3, st);
     moe::W4a4GemmArgs a2 = a1;
     a2.k_steps = h->F / 256;
     a2.n_tiles = h->d / bn;
