@@ -19,6 +19,8 @@ CAP_CASES = [
     ("cap_loose_bf16", 300, 128, 128, 8, 2, "bf16", True, 8.0),
     ("cap_skew_f32", 200, 64, 128, 8, 2, "f32", True, 1.0),
     ("cap_many_bf16", 700, 128, 128, 64, 2, "bf16", False, 1.0),
+    # 6,000 pairs: the three-kernel dispatch with a capacity
+    ("cap_mid_bf16", 3000, 64, 64, 16, 2, "bf16", True, 1.0),
 ]
 
 

@@ -117,8 +117,9 @@ def test_route_entry_point_matches_forward_routing():
         layer.close()
 
 
+# up to 4,096 pairs: the one-block kernel; above: rank, scan, scatter
 @pytest.mark.parametrize("T,n,K", [(1, 1, 1), (5, 8, 2), (300, 8, 2), (1000, 16, 3), (777, 256, 8),
-                                   (64, 4, 4), (4096, 128, 2)])
+                                   (64, 4, 4), (4096, 128, 2), (9000, 8, 2), (40000, 64, 2)])
 def test_dispatch_matches_oracle_bit_exact(T, n, K):
     import sparse_mixture_experts_24_b200 as m
     torch = require_cuda()
