@@ -18,8 +18,10 @@
 // its 128 rows and the SwiGLU epilogue is unchanged.
 //
 // Roles (192 threads per CTA, one cluster of two CTAs per pair of SMs):
-//   warp 0   (both CTAs) TMA of this CTA's A rows and B columns into its own
-//            ring; completion is counted on the LEADER's full barrier
+//   warp 0   (both CTAs) TMA of this CTA's A rows and B columns (bf16: one
+//            copy of two 64-column chunks through a 4-D weight map) into its
+//            own ring, in the banded tile order of gemm_tc.cu; completion is
+//            counted on the LEADER's full barrier
 //            (cp.async.bulk.tensor ... cta_group::2, no multicast); the leader
 //            arms that barrier with the pair's byte count.
 //   warp 1   (both CTAs) allocate 512 TMEM columns as a pair; the leader's lane
@@ -74,8 +76,12 @@ struct PairTile {
     int e, n_tile, row0, rows;
 };
 
+// Tile order: tile t -> (expert, column tile, 256-row block), an expert's row
+// blocks cut into bands of `band` blocks with the row block fastest inside a
+// band (the order of gemm_tc.cu's tile_info), so that a band's A rows stay in
+// L2 while the expert's weight columns stream past them once per band.
 __device__ __forceinline__ PairTile pair_tile(int t, const int32_t* off, const int32_t* mblk, int n,
-                                              int n_tiles) {
+                                              int n_tiles, int band_limit) {
     int lo = 0, hi = n - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -87,8 +93,20 @@ __device__ __forceinline__ PairTile pair_tile(int t, const int32_t* off, const i
     const int e = lo;
     const int local = t - mblk[e] * n_tiles;
     const int mb_count = mblk[e + 1] - mblk[e];
-    const int n_tile = local / mb_count;
-    const int m_blk = local - n_tile * mb_count;
+    const int band = min(mb_count, band_limit);
+    const int full = mb_count / band * band;  // row blocks in whole bands
+    int n_tile, m_blk;
+    if (local < full * n_tiles) {
+        const int b = local / (band * n_tiles);
+        const int r = local - b * band * n_tiles;
+        n_tile = r / band;
+        m_blk = b * band + (r - n_tile * band);
+    } else {
+        const int rem = mb_count - full;
+        const int r = local - full * n_tiles;
+        n_tile = r / rem;
+        m_blk = full + (r - n_tile * rem);
+    }
     PairTile p;
     p.e = e;
     p.n_tile = n_tile;
@@ -148,6 +166,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const uint32_t tmem_base = tail->tmem_base;
     const int total_tiles = tail->mblk[n] * args.n_tiles;
     int* status = args.status;
+    // args.band_m counts 128-row blocks; a pair tile's row block is 256 rows
+    const int band_limit = args.band_m > 0 ? max(1, args.band_m / 2) : 0x40000000;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -158,7 +178,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             for (int s = 0; s < kPairStages; ++s) armed[s] = -1;
             bool ok = true;
             for (int t = cid; t < total_tiles && ok; t += ncl) {
-                const PairTile pt = pair_tile(t, tail->off, tail->mblk, n, args.n_tiles);
+                const PairTile pt = pair_tile(t, tail->off, tail->mblk, n, args.n_tiles, band_limit);
                 for (int kb = 0; kb < args.k_blocks; ++kb) {
                     if (!mbar_wait(smem_u32(&tail->empty[stage]), phase ^ 1u, status, kStatusTimeoutEmpty)) {
                         ok = false;
@@ -180,14 +200,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                         const int c0 = kSwiGLU ? pt.n_tile * 128 : pt.n_tile * kPairBN + 128 * static_cast<int>(rank);
                         tma_load_3d_pair(b_dst, src, full_leader, c0, k0, pt.e);
                     } else if (kSwiGLU) {
+                        // bf16 weight maps are 4-D (64 columns, K rows, 64-column
+                        // chunk, expert) with boxes of two chunks: this CTA's 128
+                        // columns in one copy
                         const CUtensorMap* src = rank == 0 ? &tm_b0 : &tm_b1;
-                        const int c0 = pt.n_tile * 128;
-                        tma_load_3d_pair(b_dst, src, full_leader, c0, k0, pt.e);
-                        tma_load_3d_pair(b_dst + kPairBChunk, src, full_leader, c0 + 64, k0, pt.e);
+                        tma_load_4d_pair(b_dst, src, full_leader, 0, k0, pt.n_tile * 2, pt.e);
                     } else {
-                        const int c0 = pt.n_tile * kPairBN + 128 * static_cast<int>(rank);
-                        tma_load_3d_pair(b_dst, &tm_b0, full_leader, c0, k0, pt.e);
-                        tma_load_3d_pair(b_dst + kPairBChunk, &tm_b0, full_leader, c0 + 64, k0, pt.e);
+                        tma_load_4d_pair(b_dst, &tm_b0, full_leader, 0, k0, pt.n_tile * 4 + 2 * static_cast<int>(rank),
+                                         pt.e);
                     }
                     if (++stage == kPairStages) {
                         stage = 0;
@@ -271,7 +291,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         const uint32_t accum_empty_leader1 = mapa_shared(smem_u32(&tail->accum_empty[1]), 0);
         int local = 0;
         for (int t = cid; t < total_tiles; t += ncl, ++local) {
-            const PairTile pt = pair_tile(t, tail->off, tail->mblk, n, args.n_tiles);
+            const PairTile pt = pair_tile(t, tail->off, tail->mblk, n, args.n_tiles, band_limit);
             const int buf = local & 1;
             const uint32_t bph = static_cast<uint32_t>(local >> 1) & 1u;
             if (!mbar_wait(smem_u32(&tail->accum_full[buf]), bph, status, kStatusTimeoutAccum)) break;

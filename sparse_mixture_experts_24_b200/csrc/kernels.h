@@ -334,7 +334,9 @@ cudaError_t launch_quantize_rows_e4m3(const void* src, bool bf16, const int32_t*
                                       float* scales, int num_sms, cudaStream_t st);
 
 // The same GEMMs on CTA pairs (cta_group::2, 256-row tiles): mblk_base must
-// count 256-row blocks.
+// count 256-row blocks; the weight maps are 4-D (64 columns, K rows, 64-column
+// chunk, expert) with boxes of two chunks; the tile order takes its bands
+// from a.band_m (counted in 128-row blocks).
 constexpr int kTcPairBM = 256;
 cudaError_t launch_tc_gemm1_pair(const CUtensorMap& tm_xp, const CUtensorMap& tm_w1,
                                  const CUtensorMap& tm_w3, const TcGemmArgs& a, int num_sms,

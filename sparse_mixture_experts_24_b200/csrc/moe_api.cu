@@ -202,6 +202,7 @@ struct moe_handle {
     int* status = nullptr;
     CUtensorMap tm_xp, tm_h, tm_w1, tm_w3, tm_w2;
     CUtensorMap tm_w1x, tm_w3x, tm_w2x;  // the same weights as 4-D maps (single-SM GEMMs)
+    CUtensorMap tm_w2p;                  // w2 as a 4-D map of two-chunk boxes (CTA-pair GEMM2)
     const void* c_w1 = nullptr;
     const void* c_w3 = nullptr;
     const void* c_w2 = nullptr;
@@ -600,7 +601,8 @@ moe_status run_gemms(moe_handle* h, int64_t T, int64_t R, const void* x, const v
         }
         if (w2 != h->c_w2) {
             if (!encode_weights(&h->tm_w2, w2, h->d, h->F, h->n) ||
-                !encode_weights_wide(&h->tm_w2x, w2, h->d, h->F, h->n, 4))
+                !encode_weights_wide(&h->tm_w2x, w2, h->d, h->F, h->n, 4) ||
+                !encode_weights_wide(&h->tm_w2p, w2, h->d, h->F, h->n, 2))
                 return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for w2");
             h->c_w2 = w2;
         }
@@ -623,7 +625,7 @@ moe_status run_gemms(moe_handle* h, int64_t T, int64_t R, const void* x, const v
             a1.x_cols = h->d;
             e = moe::launch_tc_gemm1_gather(h->tm_w1x, h->tm_w3x, a1, h->num_sms, st);
         } else {
-            e = pair ? moe::launch_tc_gemm1_pair(h->tm_xp, h->tm_w1, h->tm_w3, a1, h->num_sms, st)
+            e = pair ? moe::launch_tc_gemm1_pair(h->tm_xp, h->tm_w1x, h->tm_w3x, a1, h->num_sms, st)
                      : moe::launch_tc_gemm1(h->tm_xp, h->tm_w1x, h->tm_w3x, a1, h->num_sms, st);
         }
         if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
@@ -635,7 +637,7 @@ moe_status run_gemms(moe_handle* h, int64_t T, int64_t R, const void* x, const v
         a2.out_cols = h->d;
         a2.out = h->o;
         gemm_tile_order(a2, static_cast<int64_t>(h->F) * 2, true);
-        e = pair ? moe::launch_tc_gemm2_pair(h->tm_h, h->tm_w2, a2, h->num_sms, st)
+        e = pair ? moe::launch_tc_gemm2_pair(h->tm_h, h->tm_w2p, a2, h->num_sms, st)
                  : moe::launch_tc_gemm2(h->tm_h, h->tm_w2x, a2, h->num_sms, st);
         if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
         h->launches += 1;
