@@ -535,11 +535,12 @@ int grid_balance() {
 
 // Tile order of the single-SM GEMMs (gemm_tc.cu): bands of as many 128-row
 // blocks of the A operand (rows of a_row_bytes) as fit in the band budget.
-// The budget is 32 MB (measured best on the skewed prefill, against 16 and
-// 64 MB); MOE_GEMM1_BAND_KB / MOE_GEMM2_BAND_KB override it in kilobytes
-// (0: no bands).
+// The budget is 32 MB for GEMM1 (measured best on the skewed prefill, against
+// 16, 40, 48 and 64 MB) and 40 MB for GEMM2 (against 24 and 32 MB: GEMM2 3.08
+// against 3.13-3.19 ms there, 5.68 against 5.82 GB of DRAM traffic);
+// MOE_GEMM1_BAND_KB / MOE_GEMM2_BAND_KB override them in kilobytes (0: no bands).
 void gemm_tile_order(moe::TcGemmArgs& a, int64_t a_row_bytes, bool gemm2) {
-    int64_t kb = 32 * 1024;
+    int64_t kb = gemm2 ? 40 * 1024 : 32 * 1024;
     if (const char* v = getenv(gemm2 ? "MOE_GEMM2_BAND_KB" : "MOE_GEMM1_BAND_KB")) kb = atoll(v);
     if (kb <= 0) {
         a.band_m = 0;
