@@ -134,19 +134,25 @@ __device__ __forceinline__ float silu_f(float a) { return a / (1.f + __expf(-a))
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int kPending>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
+}
+// Arrive on the mbarrier once every cp.async this thread has issued so far has
+// landed; .noinc: the arrival counts toward the barrier's expected count.
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
 // kGather (GEMM1, bf16 only): A is not read from Xp by TMA; warps 6-9 gather
 // the tile's rows straight from x (row r of the tile = token row_token[row0 +
 // r]) with 16-byte cp.async copies into the same 128-byte-swizzled layout,
 // so the gather kernel and the Xp round trip through HBM are gone.  Each
-// gather thread owns one 16-byte column chunk of 8 rows; it retires a stage
-// (waits for its copies, fences them for the tensor core's async proxy,
-// arrives on the stage's full barrier) two stages after issuing it.
+// gather thread owns one 16-byte column chunk of 8 rows; after issuing a
+// stage's copies it makes their completion arrive on the stage's full barrier
+// (cp.async.mbarrier.arrive.noinc: 128 such arrivals plus the TMA producer's),
+// so the gather warps never wait for their own copies and run as far ahead as
+// the ring allows; the MMA thread fences the async proxy after each full wait.
 template <bool kSwiGLU, bool kFp8, bool kGather>
 __global__ void __launch_bounds__(kGather ? kGatherThreads : kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
@@ -161,7 +167,7 @@ __global__ void __launch_bounds__(kGather ? kGatherThreads : kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(smem_u32(&tail->full[s]), kGather ? 5 : 1);  // TMA (+ the 4 gather warps)
+            mbar_init(smem_u32(&tail->full[s]), kGather ? 129 : 1);  // TMA (+ the 128 gather threads)
             mbar_init(smem_u32(&tail->empty[s]), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -275,6 +281,7 @@ __global__ void __launch_bounds__(kGather ? kGatherThreads : kThreads, 1)
                         ok = false;
                         break;
                     }
+                    if (kGather) fence_proxy_async_smem();  // the gathered rows came by cp.async
                     tc_fence_after();
                     const uint32_t a_base = smem_u32(smem + stage * kStageBytes);
                     const uint32_t b_base = a_base + kABytes;
@@ -322,8 +329,6 @@ __global__ void __launch_bounds__(kGather ? kGatherThreads : kThreads, 1)
         const uint16_t* x = args.x;
         int stage = 0;
         uint32_t phase = 0;
-        int pend[2] = {0, 0};
-        int npend = 0;
         bool ok = true;
         for (int t = first; t < total_tiles && ok; t += stride) {
             const TileInfo ti = tile_info(t, tail->off, tail->mblk, n, args.n_tiles, band_limit);
@@ -352,28 +357,14 @@ __global__ void __launch_bounds__(kGather ? kGatherThreads : kThreads, 1)
                     const int r = r0 + 16 * i;
                     cp_async_16(a_dst + r * 128 + ((c ^ (r & 7)) << 4), src[i] + kb * kBK, bytes[i]);
                 }
-                cp_async_commit();
-                if (npend == 2) {
-                    // the stage issued two stages ago is complete: publish it
-                    cp_async_wait<2>();
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(&tail->full[pend[0]]));
-                    pend[0] = pend[1];
-                    npend = 1;
-                }
-                pend[npend++] = stage;
+                cp_async_mbar_arrive_noinc(smem_u32(&tail->full[stage]));
                 if (++stage == kStages) {
                     stage = 0;
                     phase ^= 1u;
                 }
             }
         }
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0)
-            for (int i = 0; i < npend; ++i) mbar_arrive(smem_u32(&tail->full[pend[i]]));
+        cp_async_wait<0>();  // no copy of this thread may still be landing when the CTA exits
     } else {
         // ---------------- epilogue (warps 2..5) ----------------
         const int quad = warp & 3;  // TMEM lanes [32*quad, 32*quad+32)
