@@ -17,10 +17,10 @@
 //            chunks, 128-byte swizzle).  The bf16 weight maps are 4-D (64
 //            columns, K rows, 64-column chunk, expert) so that one copy brings
 //            several chunks: a stage is 2 copies (GEMM2) or 3 (GEMM1) instead
-//            of 5 -- the producer thread issuing those copies, not the tensor
-//            core, was what held the tensor pipe near 80% busy.  GEMM1's B is 128 columns of w1 next to
-//            the same 128 columns of w3, so ONE N=256 MMA produces both the
-//            gate and the up projection of a 128-column slice of H.
+//            of 5 (fewer copies for the one producer thread to issue).  GEMM1's
+//            B is 128 columns of w1 next to the same 128 columns of w3, so ONE
+//            N=256 MMA produces both the gate and the up projection of a
+//            128-column slice of H.
 //   warp 1   allocates 512 TMEM columns (two 256-column fp32 accumulators);
 //            one thread issues tcgen05.mma (M=128, N=256, K=16) and commits
 //            to the stage's "empty" barrier and, per tile, to "accum full".
