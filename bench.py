@@ -143,13 +143,15 @@ def recorded_traffic(kernel, config):
     p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(p):
         return None
-    src_file = {"_w4a4": "gemm_w4a4.cu", "_w4a16": "gemm_w4a16.cu", "_fp4": "gemm_fp4.cu"}.get(
+    default_file = {"_w4a4": "gemm_w4a4.cu", "_w4a16": "gemm_w4a16.cu", "_fp4": "gemm_fp4.cu"}.get(
         config[config.rfind("_"):], "gemm_tc.cu")
-    sha = source_sha(os.path.join(ROOT, "sparse_mixture_experts_24_b200", "csrc", src_file))
     with open(p) as f:
         for line in f:
             parts = line.split()
             if len(parts) >= 5 and parts[0] == "traffic" and parts[1] == kernel and parts[2] == config:
+                # an optional file=<name> names the kernel's source (else by the config)
+                src_file = next((t[5:] for t in parts[5:] if t.startswith("file=")), default_file)
+                sha = source_sha(os.path.join(ROOT, "sparse_mixture_experts_24_b200", "csrc", src_file))
                 if parts[4] == "src_sha=" + sha:
                     return float(parts[3])
     return None

@@ -333,6 +333,15 @@ cudaError_t launch_quantize_rows_e4m3(const void* src, bool bf16, const int32_t*
                                       int64_t rows, const int32_t* row_limit, int cols, uint8_t* codes,
                                       float* scales, int num_sms, cudaStream_t st);
 
+// The same GEMMs with two 128-row blocks per single-SM tile (two MMAs share
+// each stage's B; gemm_tc3.cu): mblk_base counts 128-row blocks as for
+// launch_tc_gemm1/2, the weight maps are the same 4-D maps, and the tile order
+// takes its bands from a.band_m (counted in 128-row blocks).
+cudaError_t launch_tc_gemm1_dual(const CUtensorMap& tm_xp, const CUtensorMap& tm_w1, const CUtensorMap& tm_w3,
+                                 const TcGemmArgs& a, int num_sms, cudaStream_t st);
+cudaError_t launch_tc_gemm2_dual(const CUtensorMap& tm_h, const CUtensorMap& tm_w2, const TcGemmArgs& a, int num_sms,
+                                 cudaStream_t st);
+
 // The same GEMMs on CTA pairs (cta_group::2, 256-row tiles): mblk_base must
 // count 256-row blocks; the weight maps are 4-D (64 columns, K rows, 64-column
 // chunk, expert) with boxes of two chunks; the tile order takes its bands

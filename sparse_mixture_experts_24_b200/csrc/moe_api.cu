@@ -568,6 +568,30 @@ int capacity_for(const moe_handle* h, int64_t T) {
 // cp.async gather, two stages behind the tensor core, slowed it (prefill
 // GEMM1 1.62 -> 1.99 ms), so the gather kernel stays.  MOE_GATHER=separate /
 // fused forces either.
+// Two 128-row blocks per single-SM tile (gemm_tc3.cu): three 64 KB stages in
+// flight instead of four 48 KB ones cover half again as much copy latency per
+// tensor cycle, but the two accumulators fill TMEM, so each tile's epilogue
+// stalls the next tile's MMAs.  GEMM2 takes it when the experts average more
+// than 256 rows (pairs of blocks are mostly full) and its K is at least 4,096
+// (the epilogue is short against the tile): prefill GEMM2 0.76-0.82 -> 0.71-
+// 0.72 ms, skew_prefill 3.12-3.15 -> 2.68 ms (tensor pipe 78 -> 86% busy).
+// GEMM1, whose SwiGLU epilogue is longer and K shorter, measured slower with
+// it (prefill 1.48-1.60 -> 1.87-1.91 ms), so it keeps one block per tile.
+// MOE_GEMM_PATH=dual puts both GEMMs on it; MOE_GEMM2_TILE=single|dual forces
+// GEMM2's choice.
+bool use_dual_gemm() {
+    const char* env = getenv("MOE_GEMM_PATH");
+    return env && strcmp(env, "dual") == 0;
+}
+
+bool use_dual_gemm2(int64_t R, int n, int F) {
+    if (use_dual_gemm()) return true;
+    const char* env = getenv("MOE_GEMM2_TILE");
+    if (env && strcmp(env, "single") == 0) return false;
+    if (env && strcmp(env, "dual") == 0) return true;
+    return R > 256 * static_cast<int64_t>(n) && F >= 4096;
+}
+
 bool gather_in_gemm1(int64_t R, int n) {
     const char* env = getenv("MOE_GATHER");
     if (env && strcmp(env, "separate") == 0) return false;
@@ -579,6 +603,8 @@ moe_status run_gemms(moe_handle* h, int64_t T, int64_t R, const void* x, const v
                      const void* w2, bool pair, cudaStream_t st) {
     const bool bf = h->dtype == MOE_BF16;
     const bool fused_gather = bf && !pair && gather_in_gemm1(R, h->n);
+    const bool dual = bf && !pair && !fused_gather && use_dual_gemm();
+    const bool dual2 = bf && !pair && use_dual_gemm2(R, h->n, h->F);
     cudaError_t e;
     if (!fused_gather) {
         e = moe::launch_gather(x, h->db.row_token, R, T, static_cast<int64_t>(h->d) * h->esize(), h->xp,
@@ -625,9 +651,12 @@ moe_status run_gemms(moe_handle* h, int64_t T, int64_t R, const void* x, const v
             a1.x_rows = T;
             a1.x_cols = h->d;
             e = moe::launch_tc_gemm1_gather(h->tm_w1x, h->tm_w3x, a1, h->num_sms, st);
+        } else if (pair) {
+            e = moe::launch_tc_gemm1_pair(h->tm_xp, h->tm_w1x, h->tm_w3x, a1, h->num_sms, st);
+        } else if (dual) {
+            e = moe::launch_tc_gemm1_dual(h->tm_xp, h->tm_w1x, h->tm_w3x, a1, h->num_sms, st);
         } else {
-            e = pair ? moe::launch_tc_gemm1_pair(h->tm_xp, h->tm_w1x, h->tm_w3x, a1, h->num_sms, st)
-                     : moe::launch_tc_gemm1(h->tm_xp, h->tm_w1x, h->tm_w3x, a1, h->num_sms, st);
+            e = moe::launch_tc_gemm1(h->tm_xp, h->tm_w1x, h->tm_w3x, a1, h->num_sms, st);
         }
         if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
         h->launches += 1;
@@ -639,7 +668,8 @@ moe_status run_gemms(moe_handle* h, int64_t T, int64_t R, const void* x, const v
         a2.out = h->o;
         gemm_tile_order(a2, static_cast<int64_t>(h->F) * 2, true);
         e = pair ? moe::launch_tc_gemm2_pair(h->tm_h, h->tm_w2p, a2, h->num_sms, st)
-                 : moe::launch_tc_gemm2(h->tm_h, h->tm_w2x, a2, h->num_sms, st);
+                 : (dual2 ? moe::launch_tc_gemm2_dual(h->tm_h, h->tm_w2x, a2, h->num_sms, st)
+                          : moe::launch_tc_gemm2(h->tm_h, h->tm_w2x, a2, h->num_sms, st));
         if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
         h->launches += 1;
         trace_mark(h, 4, st);

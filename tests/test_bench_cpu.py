@@ -64,22 +64,29 @@ def test_traffic_record_is_used_only_for_the_profiled_source(tmp_path, monkeypat
     src.mkdir(parents=True)
     (src / "gemm_tc.cu").write_text("kernel source A")
     (src / "gemm_w4a4.cu").write_text("kernel source B")
+    (src / "gemm_tc3.cu").write_text("kernel source C")
     sha_a = bench.source_sha(str(src / "gemm_tc.cu"))
     sha_b = bench.source_sha(str(src / "gemm_w4a4.cu"))
+    sha_c = bench.source_sha(str(src / "gemm_tc3.cu"))
     prof = tmp_path / "profiles"
     prof.mkdir()
     (prof / "ncu_traffic.txt").write_text(
         "# comment\n"
         "traffic gemm1 decode 123 src_sha=%s\n"
         "traffic gemm1 decode_w4a4 456 src_sha=%s\n"
-        "traffic gemm1 prefill 789 src_sha=0000000000000000\n" % (sha_a, sha_b))
+        "traffic gemm1 prefill 789 src_sha=0000000000000000\n"
+        "traffic gemm2 prefill 321 src_sha=%s file=gemm_tc3.cu\n" % (sha_a, sha_b, sha_c))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.recorded_traffic("gemm1", "decode") == 123.0
     assert bench.recorded_traffic("gemm1", "decode_w4a4") == 456.0
     assert bench.recorded_traffic("gemm1", "prefill") is None          # taken on another source
     assert bench.recorded_traffic("gemm2", "decode") is None           # never recorded
+    assert bench.recorded_traffic("gemm2", "prefill") == 321.0         # the line's own source file
     (src / "gemm_tc.cu").write_text("kernel source A, changed")
     assert bench.recorded_traffic("gemm1", "decode") is None           # stale after a change
+    assert bench.recorded_traffic("gemm2", "prefill") == 321.0
+    (src / "gemm_tc3.cu").write_text("kernel source C, changed")
+    assert bench.recorded_traffic("gemm2", "prefill") is None
 
 
 def test_committed_traffic_records_parse():
@@ -87,4 +94,5 @@ def test_committed_traffic_records_parse():
     lines = [l.split() for l in open(path) if l.startswith("traffic ")]
     assert lines, "no traffic records"
     for parts in lines:
-        assert len(parts) == 5 and parts[4].startswith("src_sha=") and float(parts[3]) > 0
+        assert len(parts) in (5, 6) and parts[4].startswith("src_sha=") and float(parts[3]) > 0
+        assert len(parts) == 5 or parts[5].startswith("file=")

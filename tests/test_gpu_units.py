@@ -35,16 +35,23 @@ def read_ws(layer, name, rows, cols, torch_dtype):
     return t.view(torch.bfloat16) if torch_dtype == torch.bfloat16 else t
 
 
-@pytest.mark.parametrize("path", ["single", "single_fused_gather", "single_separate_gather", "single_banded", "pair"])
+@pytest.mark.parametrize("path", ["single", "single_fused_gather", "single_separate_gather", "single_banded", "pair",
+                                  "dual", "dual_banded"])
 @pytest.mark.parametrize("T,d,F,n,K", [(200, 128, 256, 4, 2), (333, 256, 384, 8, 2), (129, 320, 192, 3, 1),
                                        (700, 192, 320, 2, 1), (1500, 256, 512, 3, 2)])
 def test_gemm1_and_gemm2_rows(T, d, F, n, K, path, monkeypatch):
     """path: single-SM tiles (128 rows; the library's choice of gather), the
     same with GEMM1 gathering its x rows itself, or with the x rows gathered
     into Xp by their own kernel, the same with
-    bands of a row block or two in the tile order (64 KB of A rows), or CTA-pair tiles (256 rows,
-    cta_group::2)."""
-    monkeypatch.setenv("MOE_GEMM_PATH", "pair" if path == "pair" else "single")
+    bands of a row block or two in the tile order (64 KB of A rows), CTA-pair tiles (256 rows,
+    cta_group::2), or two row blocks per single-SM tile (x rows gathered into
+    Xp by their own kernel; with and without bands of a pair or two)."""
+    monkeypatch.setenv("MOE_GEMM_PATH", path.split("_")[0] if path.startswith(("pair", "dual")) else "single")
+    if path.startswith("dual"):
+        monkeypatch.setenv("MOE_GATHER", "separate")
+    if path == "dual_banded":
+        monkeypatch.setenv("MOE_GEMM1_BAND_KB", "128")
+        monkeypatch.setenv("MOE_GEMM2_BAND_KB", "128")
     if path == "single_separate_gather":
         monkeypatch.setenv("MOE_GATHER", "separate")
     if path == "single_fused_gather":
