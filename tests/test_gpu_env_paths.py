@@ -13,7 +13,10 @@ these variables once per process):
                              GEMM1 when the experts average <= 256 rows);
   MOE_GEMM1_BAND_KB=0 / 64, MOE_GEMM2_BAND_KB=0 / 64
                              the expert GEMMs' tile order without bands, and
-                             with bands of a row block or two.
+                             with bands of a row block or two;
+  MOE_GEMM2_TILE=dual        GEMM2 on two row blocks per tile for every batch
+                             (default: only when the experts average more than
+                             256 rows and ffn >= 4,096).
 """
 import os
 import subprocess
@@ -31,7 +34,8 @@ SLICE = "small and (bf16_ragged or bf16_k3_n16 or router_split2 or router_split4
 @pytest.mark.parametrize("env", [{"MOE_PDL": "0"}, {"MOE_ROUTER_TOPK": "separate"}, {"MOE_GEMM_PATH": "pair"},
                                  {"MOE_GRID_BALANCE": "0"}, {"MOE_GATHER": "separate"}, {"MOE_GATHER": "fused"},
                                  {"MOE_GEMM1_BAND_KB": "0", "MOE_GEMM2_BAND_KB": "0"},
-                                 {"MOE_GEMM1_BAND_KB": "64", "MOE_GEMM2_BAND_KB": "64"}],
+                                 {"MOE_GEMM1_BAND_KB": "64", "MOE_GEMM2_BAND_KB": "64"},
+                                 {"MOE_GEMM2_TILE": "dual"}],
                          ids=lambda e: ",".join("%s=%s" % kv for kv in e.items()))
 def test_parity_slice_under_env(env):
     full_env = dict(os.environ)
