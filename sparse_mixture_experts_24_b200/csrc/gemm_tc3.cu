@@ -21,7 +21,7 @@
 // the two 256-column accumulators fill the 512 TMEM columns, so the next
 // tile's MMAs wait while the epilogue reads the accumulators out.
 //
-// Roles (192 threads, one persistent CTA per SM):
+// Roles (one persistent CTA per SM; 320 threads for GEMM1, 192 for GEMM2):
 //   warp 0   TMA producer: per 64-deep K step, A rows of both row blocks (the
 //            second skipped when the segment ends inside the first) and the
 //            256 weight columns (4-D maps: GEMM1 two chunks of w1 and two of
@@ -30,9 +30,10 @@
 //            slice, tcgen05.mma M=128 N=256 for row block 0 into columns
 //            0-255 and for row block 1 into columns 256-511, both reading the
 //            same B descriptor.
-//   warps 2-5 epilogue, thread = accumulator row: the two row blocks in turn,
-//            as gemm_tc.cu (SwiGLU with direct 16-byte stores; GEMM2 through a
-//            per-warp staging block), then hand the accumulators back.
+//   warps 2.. epilogue, thread = accumulator row, as gemm_tc.cu: GEMM1's
+//            SwiGLU with direct 16-byte stores, warps 2-5 on row block 0 and 6-9
+//            on row block 1; GEMM2's copy through per-warp staging blocks, warps
+//            2-5 on both blocks in turn; then they hand the accumulators back.
 // Tiles are (expert, column tile, pair of row blocks) in gemm_tc.cu's banded
 // order over pairs.  Every wait is bounded (common.cuh).
 #include "common.cuh"
@@ -51,8 +52,16 @@ constexpr int kBChunkBytes = kBK * 64 * 2;         // 8 KB: 64 K-rows x 64 colum
 constexpr int kBBytes = 4 * kBChunkBytes;          // 32 KB
 constexpr int kStageBytes = 2 * kABytes + kBBytes; // 64 KB
 constexpr int kTmemCols = 512;
-constexpr int kThreads = 192;
 constexpr int kMaxN = 256;
+// GEMM1's SwiGLU epilogue has two warps per TMEM lane quadrant, one per row
+// block (it stores straight from registers); GEMM2's four warps take the two
+// blocks in turn through their shared-memory staging blocks.
+template <bool kSwiGLU>
+struct Epi {
+    static constexpr int kWarps = kSwiGLU ? 8 : 4;
+    static constexpr int kThreads = (2 + kWarps) * 32;
+    static constexpr int kStagingBytes = kSwiGLU ? 0 : 4 * kWarpStageBytes;
+};
 
 struct __align__(8) Tail {
     uint64_t full[kStages];
@@ -66,8 +75,11 @@ struct __align__(8) Tail {
 };
 
 constexpr int kTailBytes = (static_cast<int>(sizeof(Tail)) + 127) / 128 * 128;
-constexpr int kSmemBytes = kStages * kStageBytes + kTailBytes + 4 * kWarpStageBytes + 1024;
-static_assert(kSmemBytes <= 232448, "shared memory");
+template <bool kSwiGLU>
+constexpr int smem_bytes() {
+    return kStages * kStageBytes + kTailBytes + Epi<kSwiGLU>::kStagingBytes + 1024;
+}
+static_assert(smem_bytes<false>() <= 232448 && smem_bytes<true>() <= 232448, "shared memory");
 
 struct Tile {
     int e, n_tile, row0, rows;  // rows: up to 256 (two row blocks)
@@ -111,7 +123,11 @@ __device__ __forceinline__ Tile tile_of(int t, const int32_t* off, const int32_t
     return ti;
 }
 
-__device__ __forceinline__ float silu_d(float a) { return a / (1.f + __expf(-a)); }
+// silu(a) = a / (1 + e^-a) with the fast division: the accumulators wait for
+// this epilogue, so its cost is the MMA's (exact to a few fp32 ulps before the
+// bf16 rounding of H; for a below about -88, e^-a is infinite and the quotient
+// is zero, the limit of silu).
+__device__ __forceinline__ float silu_d(float a) { return __fdividef(a, 1.f + __expf(-a)); }
 
 // The epilogue of one 128-row block: this warp's 32 accumulator rows (TMEM
 // lanes from tbase), `valid` of them inside the segment, rows from row_base.
@@ -120,26 +136,33 @@ __device__ __forceinline__ void epilogue_block(uint32_t tbase, int valid, int64_
                                                const TcGemmArgs& args, uint8_t* stage, int lane) {
     uint16_t* out = static_cast<uint16_t*>(args.out);
     if (kSwiGLU) {
+        // the TMEM loads of chunk c + 1 are in flight while chunk c is computed
         const bool row_ok = lane < valid;
-#pragma unroll 1
+        uint32_t a[2][32], b[2][32];
+        tmem_ld_32x32b_x32(tbase, a[0]);
+        tmem_ld_32x32b_x32(tbase + 128, b[0]);
+        tmem_wait_ld();
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
-            uint32_t a[32], b[32];
-            tmem_ld_32x32b_x32(tbase + c * 32, a);
-            tmem_ld_32x32b_x32(tbase + 128 + c * 32, b);
-            tmem_wait_ld();
+            if (c + 1 < 4) {
+                tmem_ld_32x32b_x32(tbase + (c + 1) * 32, a[(c + 1) & 1]);
+                tmem_ld_32x32b_x32(tbase + 128 + (c + 1) * 32, b[(c + 1) & 1]);
+            }
             const int col = n_tile * 128 + c * 32;
             if (row_ok && col < args.out_cols) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const float h0 = silu_d(__uint_as_float(a[2 * j])) * __uint_as_float(b[2 * j]);
-                    const float h1 = silu_d(__uint_as_float(a[2 * j + 1])) * __uint_as_float(b[2 * j + 1]);
+                    const float h0 = silu_d(__uint_as_float(a[c & 1][2 * j])) * __uint_as_float(b[c & 1][2 * j]);
+                    const float h1 =
+                        silu_d(__uint_as_float(a[c & 1][2 * j + 1])) * __uint_as_float(b[c & 1][2 * j + 1]);
                     pk[j] = pack_bf16x2(h0, h1);
                 }
                 uint4* dst = reinterpret_cast<uint4*>(out + (row_base + lane) * args.out_cols + col);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
             }
+            if (c + 1 < 4) tmem_wait_ld();
         }
     } else {
 #pragma unroll 1
@@ -165,7 +188,7 @@ __device__ __forceinline__ void epilogue_block(uint32_t tbase, int valid, int64_
 using namespace dual;
 
 template <bool kSwiGLU>
-__global__ void __launch_bounds__(dual::kThreads, 1)
+__global__ void __launch_bounds__(dual::Epi<kSwiGLU>::kThreads, 1)
     tc_gemm_dual_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
                         const __grid_constant__ CUtensorMap tm_b1, const TcGemmArgs args) {
     extern __shared__ uint8_t smem_raw[];
@@ -182,7 +205,7 @@ __global__ void __launch_bounds__(dual::kThreads, 1)
             mbar_init(smem_u32(&tail->empty[s]), 1);
         }
         mbar_init(smem_u32(&tail->accum_full), 1);
-        mbar_init(smem_u32(&tail->accum_empty), 4);
+        mbar_init(smem_u32(&tail->accum_empty), Epi<kSwiGLU>::kWarps);
         mbar_init(smem_u32(&tail->done), 1);
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -197,7 +220,7 @@ __global__ void __launch_bounds__(dual::kThreads, 1)
         tmem_relinquish();
     }
     griddep_wait();  // segment offsets and the A operand come from earlier kernels
-    for (int i = threadIdx.x; i <= n; i += kThreads) tail->off[i] = args.offsets[i];
+    for (int i = threadIdx.x; i <= n; i += Epi<kSwiGLU>::kThreads) tail->off[i] = args.offsets[i];
     if (threadIdx.x == 0) {
         // pairs of row blocks per expert, from the dispatch's 128-row block prefix
         int acc = 0;
@@ -309,16 +332,19 @@ __global__ void __launch_bounds__(dual::kThreads, 1)
             mbar_wait(smem_u32(&tail->done), 0, status, kStatusTimeoutDrain);
         }
     } else {
-        // ---------------- epilogue (warps 2..5) ----------------
+        // ---------------- epilogue (warps 2..) ----------------
         const int quad = warp & 3;  // TMEM lanes [32*quad, 32*quad+32)
-        uint8_t* stage = smem + kStages * kStageBytes + kTailBytes + (warp - 2) * kWarpStageBytes;
+        uint8_t* stage = kSwiGLU ? nullptr : smem + kStages * kStageBytes + kTailBytes + (warp - 2) * kWarpStageBytes;
+        // GEMM1: warps 2-5 take row block 0, warps 6-9 row block 1; GEMM2: both in turn
+        const int blk_first = kSwiGLU ? (warp - 2) >> 2 : 0;
+        const int blk_last = kSwiGLU ? blk_first : 1;
         int local = 0;
         for (int t = first; t < total_tiles; t += stride, ++local) {
             const Tile ti = tile_of(t, tail->off, tail->pblk, n, args.n_tiles, band_limit);
             if (!mbar_wait(smem_u32(&tail->accum_full), static_cast<uint32_t>(local) & 1u, status, kStatusTimeoutAccum))
                 break;
             tc_fence_after();
-            for (int blk = 0; blk < 2; ++blk) {
+            for (int blk = blk_first; blk <= blk_last; ++blk) {
                 const int rows_b = ti.rows - blk * kBM;
                 if (rows_b <= 0) break;  // the pair's second block is past the segment
                 const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
@@ -345,15 +371,16 @@ __global__ void __launch_bounds__(dual::kThreads, 1)
 template <bool kSwiGLU>
 static cudaError_t launch_dual(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1,
                                const TcGemmArgs& a, int num_sms, cudaStream_t st) {
+    constexpr int kSmem = smem_bytes<kSwiGLU>();
     cudaError_t e = cudaFuncSetAttribute(tc_gemm_dual_kernel<kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
+                                         kSmem);
     if (e != cudaSuccess) return e;
     const int64_t max_tiles = ((a.R + 2 * kBM - 1) / (2 * kBM) + a.n) * static_cast<int64_t>(a.n_tiles);
     int64_t g = num_sms;
     if (max_tiles < g) g = max_tiles;
     if (g < 1) g = 1;
-    launch_k(tc_gemm_dual_kernel<kSwiGLU>, dim3(static_cast<unsigned>(g)), dim3(kThreads), kSmemBytes, st, ta, tb0,
-             tb1, a);
+    launch_k(tc_gemm_dual_kernel<kSwiGLU>, dim3(static_cast<unsigned>(g)), dim3(Epi<kSwiGLU>::kThreads), kSmem, st, ta,
+             tb0, tb1, a);
     return cudaGetLastError();
 }
 

@@ -571,25 +571,26 @@ int capacity_for(const moe_handle* h, int64_t T) {
 // Two 128-row blocks per single-SM tile (gemm_tc3.cu): three 64 KB stages in
 // flight instead of four 48 KB ones cover half again as much copy latency per
 // tensor cycle, but the two accumulators fill TMEM, so each tile's epilogue
-// stalls the next tile's MMAs.  GEMM2 takes it when the experts average more
-// than 256 rows (pairs of blocks are mostly full) and its K is at least 4,096
-// (the epilogue is short against the tile): prefill GEMM2 0.76-0.82 -> 0.71-
-// 0.72 ms, skew_prefill 3.12-3.15 -> 2.68 ms (tensor pipe 78 -> 86% busy).
-// GEMM1, whose SwiGLU epilogue is longer and K shorter, measured slower with
-// it (prefill 1.48-1.60 -> 1.87-1.91 ms), so it keeps one block per tile.
-// MOE_GEMM_PATH=dual puts both GEMMs on it; MOE_GEMM2_TILE=single|dual forces
-// GEMM2's choice.
+// stalls the next tile's MMAs.  Both GEMMs take it when the experts average
+// more than 256 rows (pairs of blocks are mostly full; below that GEMM1
+// gathers its own rows and the GEMMs stream weights) and the GEMM's K is at
+// least 4,096 (the epilogue is short against the tile).  Measured on the
+// skewed prefill: GEMM2 3.06-3.12 -> 2.92-2.95 ms, GEMM1 6.11-6.15 -> 5.89-5.95
+// ms (GEMM1 with eight epilogue warps and its TMEM loads pipelined; with four
+// it was slower, 6.9-7.0 ms); prefill GEMM2 0.81 -> 0.75-0.79 ms.
+// MOE_GEMM_PATH=dual puts both GEMMs on it for every batch;
+// MOE_GEMM1_TILE / MOE_GEMM2_TILE = single|dual force one GEMM's choice.
 bool use_dual_gemm() {
     const char* env = getenv("MOE_GEMM_PATH");
     return env && strcmp(env, "dual") == 0;
 }
 
-bool use_dual_gemm2(int64_t R, int n, int F) {
+bool use_dual_tile(bool gemm2, int64_t R, int n, int K) {
     if (use_dual_gemm()) return true;
-    const char* env = getenv("MOE_GEMM2_TILE");
+    const char* env = getenv(gemm2 ? "MOE_GEMM2_TILE" : "MOE_GEMM1_TILE");
     if (env && strcmp(env, "single") == 0) return false;
     if (env && strcmp(env, "dual") == 0) return true;
-    return R > 256 * static_cast<int64_t>(n) && F >= 4096;
+    return R > 256 * static_cast<int64_t>(n) && K >= 4096;
 }
 
 bool gather_in_gemm1(int64_t R, int n) {
@@ -603,8 +604,8 @@ moe_status run_gemms(moe_handle* h, int64_t T, int64_t R, const void* x, const v
                      const void* w2, bool pair, cudaStream_t st) {
     const bool bf = h->dtype == MOE_BF16;
     const bool fused_gather = bf && !pair && gather_in_gemm1(R, h->n);
-    const bool dual = bf && !pair && !fused_gather && use_dual_gemm();
-    const bool dual2 = bf && !pair && use_dual_gemm2(R, h->n, h->F);
+    const bool dual = bf && !pair && !fused_gather && use_dual_tile(false, R, h->n, h->d);
+    const bool dual2 = bf && !pair && use_dual_tile(true, R, h->n, h->F);
     cudaError_t e;
     if (!fused_gather) {
         e = moe::launch_gather(x, h->db.row_token, R, T, static_cast<int64_t>(h->d) * h->esize(), h->xp,
