@@ -35,7 +35,10 @@
 //            on row block 1; GEMM2's copy through per-warp staging blocks, warps
 //            2-5 on both blocks in turn; then they hand the accumulators back.
 // Tiles are (expert, column tile, pair of row blocks) in gemm_tc.cu's banded
-// order over pairs.  Every wait is bounded (common.cuh).
+// order over pairs.  E4M3 form (kFp8): a stage is 128 K-elements of one-byte
+// codes (A 128 x 128 bytes per row block; B two 128 x 128 boxes), four
+// kind::f8f6f4 MMAs (K = 32) per block, and gemm_tc.cu's E4M3 scaling in the
+// epilogue.  Every wait is bounded (common.cuh).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -45,7 +48,9 @@ namespace dual {
 
 constexpr int kBM = kTcBM;                         // rows per MMA (one row block)
 constexpr int kBN = 256;                           // MMA N
-constexpr int kBK = 64;                            // K per stage
+constexpr int kBK = 64;                            // K per stage (bf16)
+constexpr int kBK8 = 128;                          // K per stage of the E4M3 form (128 bytes too)
+constexpr int kB8ChunkBytes = kBK8 * 128;          // 16 KB: 128 K-rows x 128 one-byte columns
 constexpr int kStages = 3;
 constexpr int kABytes = kBM * kBK * 2;             // 16 KB per row block
 constexpr int kBChunkBytes = kBK * 64 * 2;         // 8 KB: 64 K-rows x 64 columns
@@ -131,10 +136,27 @@ __device__ __forceinline__ float silu_d(float a) { return __fdividef(a, 1.f + __
 
 // The epilogue of one 128-row block: this warp's 32 accumulator rows (TMEM
 // lanes from tbase), `valid` of them inside the segment, rows from row_base.
-template <bool kSwiGLU>
-__device__ __forceinline__ void epilogue_block(uint32_t tbase, int valid, int64_t row_base, int n_tile,
+// E4M3 (kFp8): the accumulators are multiplied by the row's activation scale
+// and the column's weight scale first, as gemm_tc.cu's E4M3 epilogues do.
+template <bool kFp8>
+__device__ __forceinline__ void dequant32(uint32_t (&a)[32], float rs, const float* col_scale) {
+    if (!kFp8) return;
+    const float4* sc = reinterpret_cast<const float4*>(col_scale);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const float4 u = __ldg(sc + q);
+        a[4 * q + 0] = __float_as_uint(__uint_as_float(a[4 * q + 0]) * rs * u.x);
+        a[4 * q + 1] = __float_as_uint(__uint_as_float(a[4 * q + 1]) * rs * u.y);
+        a[4 * q + 2] = __float_as_uint(__uint_as_float(a[4 * q + 2]) * rs * u.z);
+        a[4 * q + 3] = __float_as_uint(__uint_as_float(a[4 * q + 3]) * rs * u.w);
+    }
+}
+
+template <bool kSwiGLU, bool kFp8>
+__device__ __forceinline__ void epilogue_block(uint32_t tbase, int valid, int64_t row_base, int n_tile, int e,
                                                const TcGemmArgs& args, uint8_t* stage, int lane) {
     uint16_t* out = static_cast<uint16_t*>(args.out);
+    const float rs = (kFp8 && lane < valid) ? args.row_scale[row_base + lane] : 1.f;
     if (kSwiGLU) {
         // the TMEM loads of chunk c + 1 are in flight while chunk c is computed
         const bool row_ok = lane < valid;
@@ -150,6 +172,9 @@ __device__ __forceinline__ void epilogue_block(uint32_t tbase, int valid, int64_
             }
             const int col = n_tile * 128 + c * 32;
             if (row_ok && col < args.out_cols) {
+                const int64_t sc = static_cast<int64_t>(e) * args.out_cols + col;
+                dequant32<kFp8>(a[c & 1], rs, args.col_scale0 + (kFp8 ? sc : 0));
+                dequant32<kFp8>(b[c & 1], rs, args.col_scale1 + (kFp8 ? sc : 0));
                 uint32_t pk[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
@@ -174,6 +199,8 @@ __device__ __forceinline__ void epilogue_block(uint32_t tbase, int valid, int64_
                 uint32_t a[32];
                 tmem_ld_32x32b_x32(tbase + g * 64 + c * 32, a);
                 tmem_wait_ld();
+                if (kFp8 && col < args.out_cols)
+                    dequant32<kFp8>(a, rs, args.col_scale0 + static_cast<int64_t>(e) * args.out_cols + col + c * 32);
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
                     pk[c * 16 + j] = pack_bf16x2(__uint_as_float(a[2 * j]), __uint_as_float(a[2 * j + 1]));
@@ -187,7 +214,7 @@ __device__ __forceinline__ void epilogue_block(uint32_t tbase, int valid, int64_
 
 using namespace dual;
 
-template <bool kSwiGLU>
+template <bool kSwiGLU, bool kFp8>
 __global__ void __launch_bounds__(dual::Epi<kSwiGLU>::kThreads, 1)
     tc_gemm_dual_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
                         const __grid_constant__ CUtensorMap tm_b1, const TcGemmArgs args) {
@@ -263,10 +290,19 @@ __global__ void __launch_bounds__(dual::Epi<kSwiGLU>::kThreads, 1)
                     armed[stage] = static_cast<int>(phase);
                     const uint32_t a_dst = smem_u32(smem + stage * kStageBytes);
                     const uint32_t b_dst = a_dst + 2 * kABytes;
-                    const int k0 = kb * kBK;
+                    const int k0 = kb * (kFp8 ? kBK8 : kBK);
                     tma_load_2d(a_dst, &tm_a, fb, k0, ti.row0);
                     if (two) tma_load_2d(a_dst + kABytes, &tm_a, fb, k0, ti.row0 + kBM);
-                    if (kSwiGLU) {
+                    if (kFp8) {
+                        // E4M3 weights [K][cols] per expert: 128 x 128-byte boxes
+                        if (kSwiGLU) {
+                            tma_load_3d(b_dst, &tm_b0, fb, ti.n_tile * 128, k0, ti.e);
+                            tma_load_3d(b_dst + kB8ChunkBytes, &tm_b1, fb, ti.n_tile * 128, k0, ti.e);
+                        } else {
+                            tma_load_3d(b_dst, &tm_b0, fb, ti.n_tile * 256, k0, ti.e);
+                            tma_load_3d(b_dst + kB8ChunkBytes, &tm_b0, fb, ti.n_tile * 256 + 128, k0, ti.e);
+                        }
+                    } else if (kSwiGLU) {
                         tma_load_4d(b_dst, &tm_b0, fb, 0, k0, ti.n_tile * 2, ti.e);
                         tma_load_4d(b_dst + 2 * kBChunkBytes, &tm_b1, fb, 0, k0, ti.n_tile * 2, ti.e);
                     } else {
@@ -286,7 +322,7 @@ __global__ void __launch_bounds__(dual::Epi<kSwiGLU>::kThreads, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer ----------------
-            constexpr uint32_t idesc = make_idesc_bf16(kBM, kBN, 0, 1);
+            constexpr uint32_t idesc = kFp8 ? make_idesc_e4m3(kBM, kBN, 0, 1) : make_idesc_bf16(kBM, kBN, 0, 1);
             int stage = 0;
             uint32_t phase = 0;
             int local = 0;
@@ -309,16 +345,30 @@ __global__ void __launch_bounds__(dual::Epi<kSwiGLU>::kThreads, 1)
                     tc_fence_after();
                     const uint32_t a_base = smem_u32(smem + stage * kStageBytes);
                     const uint32_t b_base = a_base + 2 * kABytes;
+                    if (kFp8) {
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk) {
-                        // A: K-major, 128-byte swizzle, K by 16 = 32 bytes; B: N-major,
-                        // K by 16 = two 8-row groups (2 KB), 8 KB between chunks
-                        const uint64_t bdesc = make_smem_desc(b_base + kk * 2048, kBChunkBytes, 1024, 2);
-                        const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
-                        tc_mma_f16(tmem_base, make_smem_desc(a_base + kk * 32, 16, 1024, 2), bdesc, idesc, acc);
-                        if (two)
-                            tc_mma_f16(tmem_base + static_cast<uint32_t>(kBN),
-                                       make_smem_desc(a_base + kABytes + kk * 32, 16, 1024, 2), bdesc, idesc, acc);
+                        for (int kk = 0; kk < kBK8 / 32; ++kk) {
+                            // A: K-major, K by 32 one-byte codes = 32 bytes; B: N-major, two
+                            // 128-column chunks 16 KB apart, K by 32 = four 8-row groups
+                            const uint64_t bdesc = make_smem_desc(b_base + kk * 4096, kB8ChunkBytes, 1024, 2);
+                            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+                            tc_mma_f8(tmem_base, make_smem_desc(a_base + kk * 32, 16, 1024, 2), bdesc, idesc, acc);
+                            if (two)
+                                tc_mma_f8(tmem_base + static_cast<uint32_t>(kBN),
+                                          make_smem_desc(a_base + kABytes + kk * 32, 16, 1024, 2), bdesc, idesc, acc);
+                        }
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < kBK / 16; ++kk) {
+                            // A: K-major, 128-byte swizzle, K by 16 = 32 bytes; B: N-major,
+                            // K by 16 = two 8-row groups (2 KB), 8 KB between chunks
+                            const uint64_t bdesc = make_smem_desc(b_base + kk * 2048, kBChunkBytes, 1024, 2);
+                            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+                            tc_mma_f16(tmem_base, make_smem_desc(a_base + kk * 32, 16, 1024, 2), bdesc, idesc, acc);
+                            if (two)
+                                tc_mma_f16(tmem_base + static_cast<uint32_t>(kBN),
+                                           make_smem_desc(a_base + kABytes + kk * 32, 16, 1024, 2), bdesc, idesc, acc);
+                        }
                     }
                     tc_commit(smem_u32(&tail->empty[stage]));
                     if (++stage == kStages) {
@@ -351,7 +401,7 @@ __global__ void __launch_bounds__(dual::Epi<kSwiGLU>::kThreads, 1)
                                        static_cast<uint32_t>(blk * kBN);
                 const int valid = min(32, rows_b - quad * 32);
                 const int64_t row_base = static_cast<int64_t>(ti.row0) + blk * kBM + quad * 32;
-                epilogue_block<kSwiGLU>(tbase, valid, row_base, ti.n_tile, args, stage, lane);
+                epilogue_block<kSwiGLU, kFp8>(tbase, valid, row_base, ti.n_tile, ti.e, args, stage, lane);
             }
             tc_fence_before();
             __syncwarp();
@@ -368,30 +418,40 @@ __global__ void __launch_bounds__(dual::Epi<kSwiGLU>::kThreads, 1)
     }
 }
 
-template <bool kSwiGLU>
+template <bool kSwiGLU, bool kFp8>
 static cudaError_t launch_dual(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1,
                                const TcGemmArgs& a, int num_sms, cudaStream_t st) {
     constexpr int kSmem = smem_bytes<kSwiGLU>();
-    cudaError_t e = cudaFuncSetAttribute(tc_gemm_dual_kernel<kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmem);
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_dual_kernel<kSwiGLU, kFp8>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     const int64_t max_tiles = ((a.R + 2 * kBM - 1) / (2 * kBM) + a.n) * static_cast<int64_t>(a.n_tiles);
     int64_t g = num_sms;
     if (max_tiles < g) g = max_tiles;
     if (g < 1) g = 1;
-    launch_k(tc_gemm_dual_kernel<kSwiGLU>, dim3(static_cast<unsigned>(g)), dim3(Epi<kSwiGLU>::kThreads), kSmem, st, ta,
-             tb0, tb1, a);
+    launch_k(tc_gemm_dual_kernel<kSwiGLU, kFp8>, dim3(static_cast<unsigned>(g)), dim3(Epi<kSwiGLU>::kThreads), kSmem,
+             st, ta, tb0, tb1, a);
     return cudaGetLastError();
 }
 
 cudaError_t launch_tc_gemm1_dual(const CUtensorMap& tm_xp, const CUtensorMap& tm_w1, const CUtensorMap& tm_w3,
                                  const TcGemmArgs& a, int num_sms, cudaStream_t st) {
-    return launch_dual<true>(tm_xp, tm_w1, tm_w3, a, num_sms, st);
+    return launch_dual<true, false>(tm_xp, tm_w1, tm_w3, a, num_sms, st);
 }
 
 cudaError_t launch_tc_gemm2_dual(const CUtensorMap& tm_h, const CUtensorMap& tm_w2, const TcGemmArgs& a, int num_sms,
                                  cudaStream_t st) {
-    return launch_dual<false>(tm_h, tm_w2, tm_w2, a, num_sms, st);
+    return launch_dual<false, false>(tm_h, tm_w2, tm_w2, a, num_sms, st);
+}
+
+cudaError_t launch_tc_gemm1_dual_e4m3(const CUtensorMap& tm_x8, const CUtensorMap& tm_q1, const CUtensorMap& tm_q3,
+                                      const TcGemmArgs& a, int num_sms, cudaStream_t st) {
+    return launch_dual<true, true>(tm_x8, tm_q1, tm_q3, a, num_sms, st);
+}
+
+cudaError_t launch_tc_gemm2_dual_e4m3(const CUtensorMap& tm_h8, const CUtensorMap& tm_q2, const TcGemmArgs& a,
+                                      int num_sms, cudaStream_t st) {
+    return launch_dual<false, true>(tm_h8, tm_q2, tm_q2, a, num_sms, st);
 }
 
 }  // namespace moe

@@ -341,6 +341,11 @@ cudaError_t launch_tc_gemm1_dual(const CUtensorMap& tm_xp, const CUtensorMap& tm
                                  const TcGemmArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_tc_gemm2_dual(const CUtensorMap& tm_h, const CUtensorMap& tm_w2, const TcGemmArgs& a, int num_sms,
                                  cudaStream_t st);
+// The same on E4M3 operands (maps as launch_tc_gemm1_e4m3 / launch_tc_gemm2_e4m3).
+cudaError_t launch_tc_gemm1_dual_e4m3(const CUtensorMap& tm_x8, const CUtensorMap& tm_q1, const CUtensorMap& tm_q3,
+                                      const TcGemmArgs& a, int num_sms, cudaStream_t st);
+cudaError_t launch_tc_gemm2_dual_e4m3(const CUtensorMap& tm_h8, const CUtensorMap& tm_q2, const TcGemmArgs& a,
+                                      int num_sms, cudaStream_t st);
 
 // The same GEMMs on CTA pairs (cta_group::2, 256-row tiles): mblk_base must
 // count 256-row blocks; the weight maps are 4-D (64 columns, K rows, 64-column

@@ -585,12 +585,16 @@ bool use_dual_gemm() {
     return env && strcmp(env, "dual") == 0;
 }
 
-bool use_dual_tile(bool gemm2, int64_t R, int n, int K) {
+// E4M3 (fp8 = true) stays on the single-block kernel unless a variable asks:
+// its main loop per tile is half as long, so the two-block kernel's epilogue,
+// which does not overlap the next tile's MMAs, costs twice the share (prefill
+// 1.37 -> 1.44 ms, skewed prefill 5.37-5.48 -> 5.60-5.70 ms measured).
+bool use_dual_tile(bool gemm2, int64_t R, int n, int K, bool fp8 = false) {
     if (use_dual_gemm()) return true;
     const char* env = getenv(gemm2 ? "MOE_GEMM2_TILE" : "MOE_GEMM1_TILE");
     if (env && strcmp(env, "single") == 0) return false;
     if (env && strcmp(env, "dual") == 0) return true;
-    return R > 256 * static_cast<int64_t>(n) && K >= 4096;
+    return !fp8 && R > 256 * static_cast<int64_t>(n) && K >= 4096;
 }
 
 bool gather_in_gemm1(int64_t R, int n) {
@@ -762,8 +766,11 @@ moe_status run_experts_e4m3(moe_handle* h, int64_t T, const void* x, const int32
     a1.col_scale0 = s1;
     a1.col_scale1 = s3;
     gemm_tile_order(a1, h->d, false);
-    e = pair ? moe::launch_tc_gemm1_pair_e4m3(h->tm_x8, h->tm_q1, h->tm_q3, a1, h->num_sms, st)
-             : moe::launch_tc_gemm1_e4m3(h->tm_x8, h->tm_q1, h->tm_q3, a1, h->num_sms, st);
+    const bool dual = !pair && use_dual_tile(false, R, h->n, h->d, true);
+    const bool dual2 = !pair && use_dual_tile(true, R, h->n, h->F, true);
+    e = pair   ? moe::launch_tc_gemm1_pair_e4m3(h->tm_x8, h->tm_q1, h->tm_q3, a1, h->num_sms, st)
+        : dual ? moe::launch_tc_gemm1_dual_e4m3(h->tm_x8, h->tm_q1, h->tm_q3, a1, h->num_sms, st)
+               : moe::launch_tc_gemm1_e4m3(h->tm_x8, h->tm_q1, h->tm_q3, a1, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM1 launch");
     trace_mark(h, 3, st);  // the GEMM1 stage is the GEMM1 kernel alone; the H rows go with GEMM2
     e = moe::launch_quantize_rows_e4m3(h->h, true, nullptr, R, R, used_rows, h->F, h->h8, h->hs, h->num_sms, st);
@@ -778,8 +785,9 @@ moe_status run_experts_e4m3(moe_handle* h, int64_t T, const void* x, const int32
     a2.col_scale0 = s2;
     a2.col_scale1 = nullptr;
     gemm_tile_order(a2, h->F, true);
-    e = pair ? moe::launch_tc_gemm2_pair_e4m3(h->tm_h8, h->tm_q2, a2, h->num_sms, st)
-             : moe::launch_tc_gemm2_e4m3(h->tm_h8, h->tm_q2, a2, h->num_sms, st);
+    e = pair    ? moe::launch_tc_gemm2_pair_e4m3(h->tm_h8, h->tm_q2, a2, h->num_sms, st)
+        : dual2 ? moe::launch_tc_gemm2_dual_e4m3(h->tm_h8, h->tm_q2, a2, h->num_sms, st)
+                : moe::launch_tc_gemm2_e4m3(h->tm_h8, h->tm_q2, a2, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM2 launch");
     h->launches += 1;
     trace_mark(h, 4, st);

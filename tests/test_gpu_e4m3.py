@@ -13,8 +13,8 @@ import pytest
 
 import moe_inputs as mi
 import oracle
-from gpu_helpers import (TOL_Y, compare_routing, dev, host, read_workspace, rel_l2, require_cuda,
-                         stratified_sample, y_as_f64)
+from gpu_helpers import (PER_TOKEN_FACTOR, TOL_Y, block_covering_sample, blocks_covered, compare_routing, dev,
+                         host, read_workspace, rel_l2, require_cuda, stratified_sample, y_as_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -246,6 +246,46 @@ def test_e4m3_full_size_decode():
     y_ref = oracle.forward_e4m3(L["x"][pick], o_idx[pick], o_gate[pick], *q)
     err = rel_l2(y_as_f64(y)[pick], y_ref)
     assert err <= TOL_Y["bf16"], err
+
+
+@pytest.mark.parametrize("name", ["prefill", "skew_prefill"])
+def test_e4m3_full_size_prefill(name):
+    """The prefill workloads (Mixtral layer shapes, 4,096 and 16,384 tokens,
+    the second with most of them on one expert) with E4M3 experts, in the
+    benchmark's launch configuration: routing on every token; y on a token
+    sample with a row in every (expert, 128-row M-block) of both GEMMs, the
+    ragged end of every segment included, against the oracle's E4M3 layer,
+    in aggregate and per token."""
+    import sparse_mixture_experts_24_b200 as m
+    torch = require_cuda()
+    cfg = mi.CONFIGS[name]
+    L = mi.make_layer(cfg, seed=0)
+    q = oracle_codes(L)
+    layer = m.MoELayer(cfg.n, cfg.K, cfg.d, cfg.ffn, "bf16")
+    try:
+        qd = [dev(a) for a in q]
+        y, idx, w = layer.forward_e4m3(dev(L["x"]), dev(L["W_g"]), *qd)
+        layer.sync_status()
+        y, idx, w = host(y), host(idx), host(w)
+        del qd
+    finally:
+        layer.close()
+    torch.cuda.empty_cache()
+    o_idx, o_gate, o_logits = oracle.router(L["x"], L["W_g"], cfg.K)
+    compare_routing(idx, w, o_idx, o_gate, o_logits, L["x"], L["W_g"], cfg.K)
+    pick, nblk = block_covering_sample(o_idx, cfg.n, count=256)
+    assert blocks_covered(pick, o_idx, cfg.n) == nblk
+    pick = pick[(idx[pick] == o_idx[pick]).all(axis=1)]
+    assert blocks_covered(pick, o_idx, cfg.n) >= nblk - 2
+    y_ref = oracle.forward_e4m3(L["x"][pick], o_idx[pick], o_gate[pick], *q)
+    yg = y_as_f64(y)[pick]
+    assert np.isfinite(y_as_f64(y)).all()
+    err = rel_l2(yg, y_ref)
+    per_tok = np.linalg.norm(yg - y_ref, axis=1) / np.maximum(np.linalg.norm(y_ref, axis=1), 1e-30)
+    print("\n%s E4M3 y rel-L2 on %d tokens (%d M-blocks): %.3e, worst token %.3e"
+          % (name, pick.size, nblk, err, per_tok.max()))
+    assert err <= TOL_Y["bf16"], err
+    assert per_tok.max() <= PER_TOKEN_FACTOR * TOL_Y["bf16"], per_tok.max()
 
 
 def test_e4m3_many_rows_sampled():

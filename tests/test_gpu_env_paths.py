@@ -16,7 +16,9 @@ these variables once per process):
                              with bands of a row block or two;
   MOE_GEMM2_TILE=dual        GEMM2 on two row blocks per tile for every batch
                              (default: only when the experts average more than
-                             256 rows and ffn >= 4,096).
+                             256 rows and ffn >= 4,096);
+  MOE_GEMM_PATH=dual         both GEMMs on two row blocks per tile (E4M3 here;
+                             bf16 in the unit tests).
 """
 import os
 import subprocess
@@ -66,11 +68,13 @@ def test_low_precision_paths_without_pdl(test_file, selection, count):
     assert "%d passed" % count in r.stdout, tail
 
 
-def test_e4m3_layer_on_cta_pairs():
-    """The E4M3 layer with the CTA-pair (cta_group::2, kind::f8f6f4) GEMMs:
-    every layer case, the capacity case and the 20,000-token sampled case."""
+@pytest.mark.parametrize("path", ["pair", "dual"])
+def test_e4m3_layer_on_other_tiles(path):
+    """The E4M3 layer with the CTA-pair (cta_group::2, kind::f8f6f4) GEMMs, and
+    with the GEMMs on two row blocks per tile: every layer case, the capacity
+    case and the 20,000-token sampled case."""
     full_env = dict(os.environ)
-    full_env["MOE_GEMM_PATH"] = "pair"
+    full_env["MOE_GEMM_PATH"] = path
     cmd = [sys.executable, "-m", "pytest", os.path.join(ROOT, "tests", "test_gpu_e4m3.py"), "-m", "gpu", "-q", "-x",
            "-p", "no:cacheprovider", "-k", "layer_matches_oracle or capacity or many_rows or full_size"]
     r = subprocess.run(cmd, cwd=ROOT, env=full_env, capture_output=True, text=True, timeout=900)

@@ -12,8 +12,8 @@ import pytest
 
 import moe_inputs as mi
 import oracle
-from gpu_helpers import (TOL_Y, agreeing_tokens, compare_routing, dev, host, rel_l2, require_cuda,
-                         stratified_sample, y_as_f64)
+from gpu_helpers import (PER_TOKEN_FACTOR, TOL_Y, agreeing_tokens, block_covering_sample, blocks_covered,
+                         compare_routing, dev, host, rel_l2, require_cuda, stratified_sample, y_as_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -218,6 +218,44 @@ def test_w4a4_full_size_decode():
     pick = pick[(idx[pick] == o_idx[pick]).all(axis=1)]
     y_ref = oracle.forward_w4a4(L["x"][pick], o_idx[pick], o_gate[pick], *q)
     assert rel_l2(y_as_f64(y)[pick], y_ref) <= TOL_Y["bf16"]
+
+
+@pytest.mark.parametrize("name", ["prefill", "many_expert"])
+def test_w4a4_full_size(name):
+    """The prefill (Mixtral layer shapes, 4,096 tokens) and many-expert
+    (128 experts) workloads with 4-bit weights and activations: routing on
+    every token; y on a token sample with a row in every (expert, 128-row
+    M-block), the ragged end of every segment included, against the oracle's
+    4-bit layer, in aggregate and per token."""
+    import sparse_mixture_experts_24_b200 as m
+    torch = require_cuda()
+    cfg = mi.CONFIGS[name]
+    L = mi.make_layer(cfg, seed=0)
+    q, packed = prepared_weights(L)
+    layer = m.MoELayer(cfg.n, cfg.K, cfg.d, cfg.ffn, "bf16")
+    try:
+        y, idx, w = layer.forward_w4a4(dev(L["x"]), dev(L["W_g"]), *packed)
+        layer.sync_status()
+        torch.cuda.synchronize()
+        y, idx, w = host(y), host(idx), host(w)
+    finally:
+        layer.close()
+    del packed
+    torch.cuda.empty_cache()
+    o_idx, o_gate, o_logits = oracle.router(L["x"], L["W_g"], cfg.K)
+    compare_routing(idx, w, o_idx, o_gate, o_logits, L["x"], L["W_g"], cfg.K)
+    pick, nblk = block_covering_sample(o_idx, cfg.n, count=256)
+    pick = pick[(idx[pick] == o_idx[pick]).all(axis=1)]
+    assert blocks_covered(pick, o_idx, cfg.n) >= nblk - 2
+    y_ref = oracle.forward_w4a4(L["x"][pick], o_idx[pick], o_gate[pick], *q)
+    yg = y_as_f64(y)[pick]
+    assert np.isfinite(y_as_f64(y)).all()
+    err = rel_l2(yg, y_ref)
+    per_tok = np.linalg.norm(yg - y_ref, axis=1) / np.maximum(np.linalg.norm(y_ref, axis=1), 1e-30)
+    print("\n%s W4A4 y rel-L2 on %d tokens (%d M-blocks): %.3e, worst token %.3e"
+          % (name, pick.size, nblk, err, per_tok.max()))
+    assert err <= TOL_Y["bf16"], err
+    assert per_tok.max() <= PER_TOKEN_FACTOR * TOL_Y["bf16"], per_tok.max()
 
 
 def test_w4a4_many_rows_sampled():
