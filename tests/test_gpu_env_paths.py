@@ -72,7 +72,8 @@ def test_low_precision_paths_without_pdl(test_file, selection, count):
 def test_e4m3_layer_on_other_tiles(path):
     """The E4M3 layer with the CTA-pair (cta_group::2, kind::f8f6f4) GEMMs, and
     with the GEMMs on two row blocks per tile: every layer case, the capacity
-    case and the 20,000-token sampled case."""
+    case, the 20,000-token sampled case and the full-size decode, prefill and
+    skewed-prefill workloads."""
     full_env = dict(os.environ)
     full_env["MOE_GEMM_PATH"] = path
     cmd = [sys.executable, "-m", "pytest", os.path.join(ROOT, "tests", "test_gpu_e4m3.py"), "-m", "gpu", "-q", "-x",
@@ -80,4 +81,4 @@ def test_e4m3_layer_on_other_tiles(path):
     r = subprocess.run(cmd, cwd=ROOT, env=full_env, capture_output=True, text=True, timeout=900)
     tail = "\n".join((r.stdout + r.stderr).strip().splitlines()[-15:])
     assert r.returncode == 0, tail
-    assert "9 passed" in r.stdout, tail
+    assert "11 passed" in r.stdout, tail   # 6 layer cases, capacity, many rows, 3 full-size workloads
