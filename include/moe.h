@@ -46,10 +46,15 @@
  *     programmatic dependent launches).  The captured call reads x and the
  *     weights from the addresses it was given.
  *   - Environment switches, for measurement and tests (every setting is
- *     parity-tested against the same oracle and tolerances): MOE_PDL=0 (plain stream order) and
- *     MOE_ROUTER_TOPK=separate, read once per process; MOE_GEMM_PATH=pair
- *     (CTA-pair GEMMs), MOE_GRID_BALANCE=0, MOE_W4A4_TILE=128|256 and
- *     MOE_W4A4_ROWS=32|128, read per call.
+ *     parity-tested against the same oracle and tolerances): MOE_PDL=0 (plain
+ *     stream order) and MOE_ROUTER_TOPK=separate, read once per process;
+ *     read per call: MOE_GEMM_PATH=single|pair|dual (the bf16 and E4M3 expert
+ *     GEMMs on one-block, CTA-pair or two-block tiles for every batch),
+ *     MOE_GEMM1_TILE / MOE_GEMM2_TILE=single|dual (one GEMM's tile),
+ *     MOE_GATHER=separate|fused (x rows gathered by their own kernel or by
+ *     GEMM1), MOE_GEMM1_BAND_KB / MOE_GEMM2_BAND_KB (the tile order's band of
+ *     A rows; 0: no bands), MOE_GRID_BALANCE=0, MOE_W4A4_TILE=128|256,
+ *     MOE_W4A4_ROWS=32|128 and MOE_W4A16_ROWS=32|128.
  */
 #ifndef MOE_B200_MOE_H
 #define MOE_B200_MOE_H
