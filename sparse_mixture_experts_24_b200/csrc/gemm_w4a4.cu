@@ -10,9 +10,10 @@
 // 4-bit weights ("Mixture of Experts: Why Mixtral Only Wakes Up Two
 // Specialists", Part 4).
 //
-// One persistent CTA per SM, 352 threads, tiles of 128 rows x kBN columns of
-// the packed B (kBN = 128: two accumulators, 6 stages of 36 KB; kBN = 256: one
-// accumulator, 4 stages of 54 KB -- the block scales take the rest of TMEM):
+// One persistent CTA per SM, 352 threads, tiles of kTM rows x kBN columns of
+// the packed B (kBN = 128: two accumulators, 6 stages of 36 KB, or 8 of 24 KB
+// with 32-row tiles; kBN = 256: one accumulator, 4 stages of 54 KB, or 5 of 42
+// KB with 32-row tiles -- the block scales take the rest of TMEM):
 //   warp 0     TMA producer: per stage a K step of 256 (128 bytes of codes per
 //              row): A 128 rows (128-byte swizzle), the kBN K-major weight rows
 //              in one copy (GEMM1: the w1|w3 pair pack, 64 hidden columns per
@@ -41,6 +42,7 @@ constexpr int kBBlockBytes = 128 * 128; // 16 KB: one 128-row block of B
 constexpr int kSfaBytes = 4 * 512;      // 4 chunks (64-wide K steps) of A scales
 constexpr int kSfbBlockBytes = 4 * 512; // the same for one 128-row block of B
 constexpr int kMaxN = 256;
+constexpr int kMaxStages = 8;
 constexpr int kTmemCols = 512;
 constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, each taking half the columns
 constexpr int kCpWarp = 2 + kEpiWarps;  // the scale-factor copies
@@ -58,18 +60,19 @@ struct Cfg {
     static constexpr int kBlocks = kBN / 128;
     static constexpr int kABytes = kTM * 128;  // kTM rows of 128 bytes (a K step of 256)
     static constexpr int kStageBytes = kABytes + kBlocks * kBBlockBytes + kSfaBytes + kBlocks * kSfbBlockBytes;
-    static constexpr int kStages = kBN == 128 ? 6 : (kTM == 32 ? 5 : 4);
+    static constexpr int kStages = kBN == 128 ? (kTM == 32 ? 8 : 6) : (kTM == 32 ? 5 : 4);
     static constexpr int kAccBufs = kBN == 128 ? 2 : 1;
     static constexpr int kSfCols = 4 * (4 + 4 * kBlocks);  // per stage: 4 K steps x (A + B chunks)
     static constexpr int kSfBase = kAccBufs * kBN;
     static_assert(kStageBytes % 1024 == 0, "stages keep the 1 KB alignment of the swizzled tiles");
     static_assert(kSfBase + kStages * kSfCols <= kTmemCols, "TMEM budget");
+    static_assert(kStages <= kMaxStages, "barrier arrays");
 };
 
 struct __align__(8) SmemTail {
-    uint64_t full[6];
-    uint64_t empty[6];
-    uint64_t sf_ready[6];  // the stage's scale chunks are in TMEM
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
+    uint64_t sf_ready[kMaxStages];  // the stage's scale chunks are in TMEM
     uint64_t cp_done;
     uint64_t accum_full[2];
     uint64_t accum_empty[2];
@@ -177,8 +180,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // ---------------- TMA producer ----------------
             int stage = 0;
             uint32_t phase = 0;
-            int armed[6];
-            for (int s = 0; s < 6; ++s) armed[s] = -1;
+            int armed[kMaxStages];
+            for (int s = 0; s < kMaxStages; ++s) armed[s] = -1;
             bool ok = true;
             const int blocks_per_e = args.n_rows_b / 128;
             for (int t = first; t < total_tiles && ok; t += stride) {
@@ -426,8 +429,9 @@ template <bool kSwiGLU>
 static cudaError_t launch_w4_any(const CUtensorMap& ta, const CUtensorMap& tb, const W4a4GemmArgs& a, bool wide,
                                  int tile_rows, int num_sms, cudaStream_t st) {
     if (!wide) {
-        if (tile_rows != 128) return cudaErrorInvalidValue;
-        return launch_w4<kSwiGLU, 128, 128>(ta, tb, a, num_sms, st);
+        if (tile_rows == 32) return launch_w4<kSwiGLU, 128, 32>(ta, tb, a, num_sms, st);
+        if (tile_rows == 128) return launch_w4<kSwiGLU, 128, 128>(ta, tb, a, num_sms, st);
+        return cudaErrorInvalidValue;
     }
     if (tile_rows == 32) return launch_w4<kSwiGLU, 256, 32>(ta, tb, a, num_sms, st);
     if (tile_rows == 128) return launch_w4<kSwiGLU, 256, 128>(ta, tb, a, num_sms, st);

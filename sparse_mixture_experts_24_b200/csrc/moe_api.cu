@@ -880,10 +880,10 @@ moe_status run_experts_w4a4(moe_handle* h, int64_t T, const void* x, const float
         if (atoi(v) == 128) wide = false;
         if (atoi(v) == 256) wide = true;
     }
-    int tile_rows = (wide && R <= 32 * static_cast<int64_t>(h->n)) ? 32 : 128;
-    if (const char* v = getenv("MOE_W4A4_ROWS")) {  // 32 or 128 forces a height (32: 256-column tiles only)
+    int tile_rows = R <= 32 * static_cast<int64_t>(h->n) ? 32 : 128;
+    if (const char* v = getenv("MOE_W4A4_ROWS")) {  // 32 or 128 forces a height
         if (atoi(v) == 128) tile_rows = 128;
-        if (atoi(v) == 32 && wide) tile_rows = 32;
+        if (atoi(v) == 32) tile_rows = 32;
     }
     cudaError_t e = moe::launch_dispatch(topk_idx, T, h->K, h->n, tile_rows, h->db, st, capacity_for(h, T));
     if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");

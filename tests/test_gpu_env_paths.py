@@ -53,7 +53,7 @@ def test_parity_slice_under_env(env):
 @pytest.mark.parametrize("test_file,selection,count", [
     ("test_gpu_e4m3.py", "e4m3_ragged or e4m3_tails", 2),
     ("test_gpu_fp4.py", "fp4_ragged or fp4_tails", 2),
-    ("test_gpu_w4a4.py", "w4a4_small or w4a4_tails", 6),    # three tile shapes
+    ("test_gpu_w4a4.py", "w4a4_small or w4a4_tails", 8),    # four tile shapes
 ], ids=["e4m3", "fp4", "w4a4"])
 def test_low_precision_paths_without_pdl(test_file, selection, count):
     """The E4M3, 4-bit and 4-bit weight-and-activation layers with plain

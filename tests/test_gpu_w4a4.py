@@ -118,11 +118,11 @@ FWD_CASES = [
 ]
 
 
-@pytest.mark.parametrize("tile", ["128x128", "256x128", "256x32"])
+@pytest.mark.parametrize("tile", ["128x128", "128x32", "256x128", "256x32"])
 @pytest.mark.parametrize("case", FWD_CASES, ids=[c[0] for c in FWD_CASES])
 def test_w4a4_layer_matches_oracle(case, tile, monkeypatch):
     """Every tile shape on every case: 128 packed columns with two
-    accumulators, 256 with one, and 256 columns over 32-row tiles."""
+    accumulators and 256 with one, each over 128-row and 32-row tiles."""
     import sparse_mixture_experts_24_b200 as m
     torch = require_cuda()
     cols, rows = tile.split("x")
