@@ -414,8 +414,8 @@ MOE_API moe_status moe_forward_w4a16(moe_handle *h, int64_t T, const void *x, co
  * x, W_g, y, topk_idx, topk_w as for moe_forward.  The GEMMs use tiles of
  * 256 packed columns, over 32 rows when the experts average at most 32 rows
  * per call (T*K <= 32*n) and over 128 rows otherwise; MOE_W4A4_TILE=128
- * selects 128-column tiles with two accumulators (128 rows), MOE_W4A4_ROWS=32
- * or 128 forces the row tiles (same results either way).
+ * selects 128-column tiles with two accumulators (the same row rule),
+ * MOE_W4A4_ROWS=32 or 128 forces the row tiles (same results either way).
  * The first call grows the workspace by about T*K*(d + ffn)*0.6 bytes.
  *   Errors: as moe_forward; MOE_ERR_UNSUPPORTED for an fp32 handle or d, ffn
  *   not multiples of 256.
