@@ -96,3 +96,16 @@ def test_committed_traffic_records_parse():
     for parts in lines:
         assert len(parts) in (5, 6) and parts[4].startswith("src_sha=") and float(parts[3]) > 0
         assert len(parts) == 5 or parts[5].startswith("file=")
+
+
+def test_committed_traffic_records_name_the_current_sources():
+    """Every committed traffic record was taken on the kernel source as it is
+    now: a kernel edited since its ncu capture would report no traffic."""
+    path = os.path.join(bench.ROOT, "profiles", "ncu_traffic.txt")
+    stale = []
+    for line in open(path):
+        if line.startswith("traffic "):
+            parts = line.split()
+            if bench.recorded_traffic(parts[1], parts[2]) != float(parts[3]):
+                stale.append(line.strip())
+    assert not stale, stale
