@@ -10,7 +10,7 @@
 // 4-bit weights ("Mixture of Experts: Why Mixtral Only Wakes Up Two
 // Specialists", Part 4).
 //
-// One persistent CTA per SM, 352 threads, tiles of kTM rows x kBN columns of
+// One persistent CTA per SM, 384 threads, tiles of kTM rows x kBN columns of
 // the packed B (kBN = 128: two accumulators, 6 stages of 36 KB, or 8 of 24 KB
 // with 32-row tiles; kBN = 256: one accumulator, 4 stages of 54 KB, or 5 of 42
 // KB with 32-row tiles -- the block scales take the rest of TMEM):
@@ -19,9 +19,10 @@
 //              in one copy (GEMM1: the w1|w3 pair pack, 64 hidden columns per
 //              128-row block; GEMM2: w2), and by plain bulk copies the matching
 //              512-byte scale chunks (4 for A, 4 per 128-row B block).
-//   warp 10    per stage, copies the scale chunks into that stage's TMEM
-//              columns (tcgen05.cp 32x128b.warpx4, 3 or 2 per 64-wide K step)
-//              and commits them to the stage's scales-ready barrier.
+//   warps 10-11 per stage (warp 10 the even stages, 11 the odd ones), copy
+//              the scale chunks into that stage's TMEM columns (tcgen05.cp
+//              32x128b.warpx4, 3 or 2 per 64-wide K step) and commit them to
+//              the stage's scales-ready barrier.
 //   warp 1     allocates 512 TMEM columns; once a stage's scales are in TMEM
 //              it issues tcgen05.mma kind::mxf4nvf4 block16 M=128 N=kBN.
 //              With the scale copies on a warp of their own, neither issuing
@@ -45,8 +46,9 @@ constexpr int kMaxN = 256;
 constexpr int kMaxStages = 8;
 constexpr int kTmemCols = 512;
 constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, each taking half the columns
-constexpr int kCpWarp = 2 + kEpiWarps;  // the scale-factor copies
-constexpr int kThreads = (3 + kEpiWarps) * 32;
+constexpr int kCpWarp = 2 + kEpiWarps;  // the scale-factor copies: warps kCpWarp, kCpWarp + 1
+constexpr int kCpWarps = 2;             // each owns the stages s with s % 2 == its index
+constexpr int kThreads = (2 + kEpiWarps + kCpWarps) * 32;
 
 // Tile width kBN (128 or 256 output columns of the packed B, i.e. 64 or 128
 // hidden columns of GEMM1's w1|w3 pairs) and tile height kTM (rows of A per
@@ -73,7 +75,7 @@ struct __align__(8) SmemTail {
     uint64_t full[kMaxStages];
     uint64_t empty[kMaxStages];
     uint64_t sf_ready[kMaxStages];  // the stage's scale chunks are in TMEM
-    uint64_t cp_done;
+    uint64_t cp_done[kCpWarps];
     uint64_t accum_full[2];
     uint64_t accum_empty[2];
     uint64_t done;
@@ -147,7 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&tail->accum_empty[b]), kEpiWarps);
         }
         mbar_init(smem_u32(&tail->done), 1);
-        mbar_init(smem_u32(&tail->cp_done), 1);
+        for (int c = 0; c < kCpWarps; ++c) mbar_init(smem_u32(&tail->cp_done[c]), 1);
         fence_barrier_init();
         fence_proxy_async_smem();
     }
@@ -266,17 +268,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_commit(smem_u32(&tail->done));
             mbar_wait(smem_u32(&tail->done), 0, status, kStatusTimeoutDrain);
         }
-    } else if (warp == kCpWarp) {
+    } else if (warp >= kCpWarp) {
         if (lane == 0) {
             // ---------------- scale chunks -> TMEM ----------------
-            // A stage's TMEM scale columns are written again only after its
-            // next full barrier, which follows the empty barrier that the
-            // MMAs reading them committed to.
+            // Two warps, each owning the stages s with s % 2 == its index (one
+            // thread issuing every copy was busy 70% of the time at decode and
+            // 91% at prefill, and a stage is released only after its copies
+            // and MMAs).  A stage keeps its owner for every use, so each full
+            // barrier is waited on by one thread, phase after phase: a waiter
+            // that reached a later phase of a barrier still in its earlier one
+            // would see the earlier parity as complete.  A stage's TMEM scale
+            // columns are written again only after its next full barrier,
+            // which follows the empty barrier that the MMAs reading them
+            // committed to.
+            const int cw = warp - kCpWarp;
             int stage = 0;
             uint32_t phase = 0;
             for (int t = first; t < total_tiles; t += stride) {
                 bool ok = true;
                 for (int ks = 0; ks < args.k_steps; ++ks) {
+                    if (stage % kCpWarps != cw) {
+                        if (++stage == C::kStages) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                        continue;
+                    }
                     if (!mbar_wait(smem_u32(&tail->full[stage]), phase, status, kStatusTimeoutFull)) {
                         ok = false;
                         break;
@@ -303,8 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
             }
             // every copy of this thread is complete before TMEM is freed
-            tc_commit(smem_u32(&tail->cp_done));
-            mbar_wait(smem_u32(&tail->cp_done), 0, status, kStatusTimeoutDrain);
+            tc_commit(smem_u32(&tail->cp_done[cw]));
+            mbar_wait(smem_u32(&tail->cp_done[cw]), 0, status, kStatusTimeoutDrain);
         }
     } else {
         // ---------------- epilogue (warps 2..9) ----------------
