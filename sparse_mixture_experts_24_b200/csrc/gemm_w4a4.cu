@@ -25,8 +25,8 @@
 //              the stage's scales-ready barrier.
 //   warp 1     allocates 512 TMEM columns; once a stage's scales are in TMEM
 //              it issues tcgen05.mma kind::mxf4nvf4 block16 M=128 N=kBN.
-//              With the scale copies on a warp of their own, neither issuing
-//              thread carries all 16 of a stage's tensor-core instructions.
+//              With the scale copies on warps of their own, the MMA thread
+//              issues only the stage's 4 MMAs.
 //   warps 2-9  epilogue, two warps per TMEM lane quadrant splitting the
 //              columns: accumulator x row scale x matrix scale, SwiGLU (GEMM1)
 //              or a copy (GEMM2), bf16 rows.
